@@ -1,0 +1,85 @@
+"""The pins have teeth: each plausible mistake planted in a copy of the oracle
+(on the CPU, rebuilt with the same compiler flags) makes at least one pin fail."""
+import ctypes
+import os
+
+import pytest
+
+import oracle
+from tests import test_oracle_pins as pins
+
+MUTANTS = [
+    # (name, original text, planted mistake, pins expected to catch it)
+    ("no_renormalisation", "w[j] = w[j] / sum;", "w[j] = w[j];",
+     [pins.test_gate_weights_sum_to_one_and_order, pins.test_two_way_gate_is_logistic_of_gap]),
+    ("unstable_tie_order", "scores[order[j]] < scores[key]", "scores[order[j]] <= scores[key]",
+     [pins.test_topk_matches_library_sort_with_many_ties, pins.test_tie_break_duplicate_router_columns]),
+    ("ascending_sort", "scores[order[j]] < scores[key]", "scores[order[j]] > scores[key]",
+     [pins.test_worked_router_example]),
+    ("combine_drops_last_slot", "for (int64_t j = 0; j < K; ++j)\n        for (int64_t c = 0; c < D; ++c) y[c]",
+     "for (int64_t j = 0; j < K - 1; ++j)\n        for (int64_t c = 0; c < D; ++c) y[c]",
+     [pins.test_sparse_layer_equals_dense_masked_gate]),
+    ("gate_up_swapped", "hid[n] = orc_silu(g) * u;", "hid[n] = orc_silu(u) * g;",
+     [pins.test_one_expert_top1_is_dense_ffn]),
+    ("down_weight_transposed", "orc_get(W2e, dtype, c * H + n)", "orc_get(W2e, dtype, n * D + c)",
+     [pins.test_one_expert_top1_is_dense_ffn]),
+    ("router_weight_transposed", "orc_get(Wg, w_dtype, i * N + e)", "orc_get(Wg, w_dtype, e * D + i)",
+     [pins.test_router_scores_match_library_matmul]),
+    ("router_bias_dropped", "if (bg) s += (double)bg[e];", "(void)bg;",
+     [pins.test_router_scores_match_library_matmul]),
+    ("gelu_tanh_form", "0.5 * v * (1.0 + erf(v / sqrt(2.0)))",
+     "0.5 * v * (1.0 + tanh(sqrt(2.0 / 3.141592653589793) * (v + 0.044715 * v * v * v)))",
+     [pins.test_activation_closed_forms]),
+    ("expert_bias_dropped", "if (b1e) a += (double)b1e[n];", "(void)b1e;",
+     [pins.test_one_expert_top1_is_dense_ffn]),
+    ("sample_variance", "var /= (double)n;", "var /= (double)(n - 1);",
+     [pins.test_cv_squared_closed_forms]),
+    ("switch_f_over_T", "(counts[e] / (double)(T * K))", "(counts[e] / (double)T)",
+     [pins.test_aux_stats_uniform_and_empty, pins.test_aux_stats_invariants_and_library_checks]),
+    ("p_mean_not_normalised", "p_mean[e] += p[e] / z;", "p_mean[e] += p[e];",
+     [pins.test_aux_stats_invariants_and_library_checks]),
+    ("expert_params_one_matrix", "return 2 * D * H + (has_bias ? H + D : 0);", "return D * H + (has_bias ? H + D : 0);",
+     [pins.test_gpt2_moe_parameter_totals]),
+]
+
+
+def _call(pin, golden_dir):
+    import inspect
+    params = inspect.signature(pin).parameters
+    if "golden_dir" in params:
+        pin(golden_dir)
+        return
+    marks = getattr(pin, "pytestmark", [])
+    cases = [m for m in marks if m.name == "parametrize"]
+    if cases:
+        names = [n.strip() for n in cases[0].args[0].split(",")]
+        for vals in cases[0].args[1]:
+            vals = vals if isinstance(vals, tuple) else (vals,)
+            pin(**dict(zip(names, vals)))
+    else:
+        pin()
+
+
+@pytest.mark.parametrize("name,old,new,catchers", MUTANTS, ids=[m[0] for m in MUTANTS])
+def test_planted_mistake_is_caught(name, old, new, catchers, tmp_path, golden_dir, monkeypatch):
+    src = open(oracle._SRC).read()
+    assert src.count(old) == 1, f"mutation site for {name} not unique"
+    mutated = tmp_path / "moe_oracle_mutant.c"
+    mutated.write_text(src.replace(old, new))
+    so = oracle.compile_source(str(mutated), str(tmp_path / "liboracle_mutant.so"))
+    monkeypatch.setattr(oracle, "_lib", oracle.configure(ctypes.CDLL(so)))
+    caught = 0
+    for pin in catchers:
+        try:
+            _call(pin, golden_dir)
+        except AssertionError:
+            caught += 1
+    assert caught > 0, f"no pin caught the planted mistake {name}"
+
+
+def test_unmutated_copy_passes_the_same_pins(tmp_path, golden_dir, monkeypatch):
+    so = oracle.compile_source(oracle._SRC, str(tmp_path / "liboracle_copy.so"))
+    monkeypatch.setattr(oracle, "_lib", oracle.configure(ctypes.CDLL(so)))
+    for _, _, _, catchers in MUTANTS:
+        for pin in catchers:
+            _call(pin, golden_dir)

@@ -1,0 +1,357 @@
+"""Pins of the fp64 oracle against facts fixed outside the oracle itself.
+
+Each test checks the oracle against something the pages print, a closed form,
+an invariant, a library routine on a special case, or brute force on tiny
+inputs.  None of them re-types the oracle's own formula.
+"""
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+import torch.nn.functional as F
+
+import oracle
+
+pytestmark = pytest.mark.filterwarnings("ignore")
+
+
+def _golden(golden_dir, name):
+    with open(os.path.join(golden_dir, name)) as f:
+        return json.load(f)
+
+
+# --------------------------------------------------------------------------- routing
+def test_worked_router_example(golden_dir):
+    """The printed router example selects experts 4 and 2 (best first)."""
+    g = _golden(golden_dir, "router_worked_example.json")
+    sel = oracle.select_topk(np.array(g["scores"]), g["top_k"])[0]
+    assert sel.tolist() == g["selected_best_first"]
+
+
+def test_two_way_gate_is_logistic_of_gap(golden_dir):
+    """Closed form: with k = 2 the renormalised softmax is the logistic function of the score gap."""
+    g = _golden(golden_dir, "router_worked_example.json")
+    s = np.array(g["scores"])
+    sel = oracle.select_topk(s, 2)
+    w = oracle.gate_weights(s, sel)[0]
+    gap = s[4] - s[2]
+    assert w[0] == pytest.approx(1.0 / (1.0 + math.exp(-gap)), rel=1e-15)
+    assert w[1] == pytest.approx(1.0 / (1.0 + math.exp(gap)), rel=1e-14)
+
+
+def _lexsort_topk(row, K):
+    # numpy's stable lexicographic sort: primary key descending score, secondary ascending index
+    order = np.lexsort((np.arange(row.shape[0]), -row))
+    return order[:K]
+
+
+@pytest.mark.parametrize("N,K", [(8, 2), (6, 2), (32, 4), (256, 8), (5, 5), (7, 1)])
+def test_topk_matches_library_sort_with_many_ties(N, K):
+    """Selection equals a library stable sort (desc score, asc index) on tie-heavy scores."""
+    rng = np.random.default_rng(N * 100 + K)
+    scores = rng.integers(-3, 4, size=(200, N)).astype(np.float64)  # lots of exact ties
+    scores[:5] = 0.0  # all-equal rows: selection must be 0..K-1
+    sel = oracle.select_topk(scores, K)
+    for t in range(scores.shape[0]):
+        assert sel[t].tolist() == _lexsort_topk(scores[t], K).tolist()
+    for t in range(5):
+        assert sel[t].tolist() == list(range(K))
+
+
+def test_topk_brute_force_over_subsets():
+    """Brute force: the selected set is the K-subset with the largest score sum; among equal sums,
+    the lexicographically smallest index tuple (integer scores, so sums are exact)."""
+    rng = np.random.default_rng(7)
+    for N, K in [(6, 2), (6, 3), (5, 1), (7, 4)]:
+        for _ in range(60):
+            s = rng.integers(-2, 3, size=N).astype(np.float64)
+            best = None
+            for sub in itertools.combinations(range(N), K):  # lexicographic order
+                tot = sum(s[list(sub)])
+                if best is None or tot > best[0]:
+                    best = (tot, sub)
+            sel = oracle.select_topk(s, K)[0]
+            assert sorted(sel.tolist()) == list(best[1])
+            # best-first order within the set: non-increasing scores, ties by index
+            vals = s[sel]
+            assert all(vals[i] >= vals[i + 1] for i in range(K - 1))
+
+
+def test_tie_break_duplicate_router_columns():
+    """Duplicate W_g columns give bit-equal scores; the lower expert index wins."""
+    rng = np.random.default_rng(3)
+    D, N = 16, 8
+    Wg = rng.standard_normal((D, N)).astype(np.float32)
+    Wg[:, 5] = Wg[:, 2]
+    Wg[:, 6] = Wg[:, 2]
+    x = rng.standard_normal((50, D)).astype(np.float32)
+    s = oracle.router_scores(x.astype(np.float64), Wg, oracle.F32)
+    sel = oracle.select_topk(s, 3)
+    for t in range(50):
+        picked = [e for e in sel[t].tolist() if e in (2, 5, 6)]
+        assert picked == sorted(picked)
+        if 5 in picked:
+            assert 2 in picked
+        if 6 in picked:
+            assert 5 in picked and 2 in picked
+    # signed zeros compare equal: a tie, lower index first
+    assert oracle.select_topk(np.array([-0.0, 0.0, -1.0]), 1)[0].tolist() == [0]
+
+
+def test_router_scores_match_library_matmul():
+    """Router scores equal a library fp64 matmul (+ bias) on random inputs."""
+    rng = np.random.default_rng(11)
+    x = rng.standard_normal((20, 33)).astype(np.float32)
+    Wg = rng.standard_normal((33, 7)).astype(np.float32)
+    bg = rng.standard_normal(7).astype(np.float32)
+    s = oracle.router_scores(x.astype(np.float64), Wg, oracle.F32, bg)
+    ref = x.astype(np.float64) @ Wg.astype(np.float64) + bg.astype(np.float64)
+    np.testing.assert_allclose(s, ref, rtol=1e-13, atol=1e-13)
+
+
+def test_bf16_widening_is_exact():
+    """bf16 bit patterns widen to the same doubles torch produces."""
+    t = torch.randn(40, dtype=torch.float32).to(torch.bfloat16)
+    bits = t.view(torch.int16).numpy().view(np.uint16).reshape(1, -1)
+    got = oracle.load_rows(bits, oracle.BF16, [0])[0]
+    np.testing.assert_array_equal(got, t.to(torch.float64).numpy())
+
+
+# --------------------------------------------------------------------------- gate weights
+def test_gate_weights_sum_to_one_and_order():
+    rng = np.random.default_rng(5)
+    for N, K in [(8, 2), (32, 4), (256, 8), (6, 6)]:
+        s = rng.standard_normal((100, N)) * 3
+        sel = oracle.select_topk(s, K)
+        w = oracle.gate_weights(s, sel)
+        np.testing.assert_allclose(w.sum(1), 1.0, rtol=0, atol=1e-15)
+        assert np.all(w > 0)
+        assert np.all(np.diff(w, axis=1) <= 1e-17)  # best slot carries the largest weight
+
+
+def test_gate_weights_equal_masked_full_softmax():
+    """softmax(KeepTopK(H, k)) with -inf masking (library softmax) equals the oracle's weights."""
+    rng = np.random.default_rng(9)
+    N, K = 16, 4
+    s = rng.standard_normal((64, N)) * 2
+    sel = oracle.select_topk(s, K)
+    w = oracle.gate_weights(s, sel)
+    masked = torch.full((64, N), -math.inf, dtype=torch.float64)
+    st = torch.from_numpy(s)
+    for t in range(64):
+        masked[t, sel[t]] = st[t, sel[t]]
+    G = torch.softmax(masked, dim=1).numpy()
+    for t in range(64):
+        np.testing.assert_allclose(w[t], G[t, sel[t]], rtol=1e-14)
+        off = np.setdiff1d(np.arange(N), sel[t])
+        assert np.all(G[t, off] == 0.0)
+
+
+# --------------------------------------------------------------------------- activations
+def test_activation_closed_forms():
+    assert oracle.gelu(0.0) == 0.0
+    assert oracle.silu(0.0) == 0.0
+    assert oracle.gelu(1.0) == pytest.approx(0.8413447460685429, rel=1e-15)  # Phi(1)
+    for v in [0.3, 1.7, 4.0, 9.0]:
+        assert oracle.gelu(v) - oracle.gelu(-v) == pytest.approx(v, rel=1e-14)
+        assert oracle.silu(v) - oracle.silu(-v) == pytest.approx(v, rel=1e-14)
+    assert oracle.silu(2.0) == pytest.approx(2.0 / (1.0 + math.exp(-2.0)), rel=1e-15)
+
+
+# --------------------------------------------------------------------------- experts / layer
+def _rand_layer(rng, T, D, H, N, act, bias):
+    x = rng.standard_normal((T, D)).astype(np.float32)
+    Wg = (rng.standard_normal((D, N)) * 0.5).astype(np.float32)
+    rows = H if act == oracle.ACT_GELU else 2 * H
+    W1 = (rng.standard_normal((N, rows, D)) * 0.2).astype(np.float32)
+    W2 = (rng.standard_normal((N, D, H)) * 0.2).astype(np.float32)
+    b1 = (rng.standard_normal((N, H)) * 0.1).astype(np.float32) if bias else None
+    b2 = (rng.standard_normal((N, D)) * 0.1).astype(np.float32) if bias else None
+    return x, Wg, W1, W2, b1, b2
+
+
+def _torch_expert(x64, act, W1e, W2e, b1e, b2e, H):
+    W1t = torch.from_numpy(W1e.astype(np.float64))
+    W2t = torch.from_numpy(W2e.astype(np.float64))
+    if act == oracle.ACT_GELU:
+        b1t = None if b1e is None else torch.from_numpy(b1e.astype(np.float64))
+        b2t = None if b2e is None else torch.from_numpy(b2e.astype(np.float64))
+        h = F.gelu(F.linear(x64, W1t, b1t), approximate="none")
+        return F.linear(h, W2t, b2t)
+    gu = F.linear(x64, W1t)
+    return F.linear(F.silu(gu[:, :H]) * gu[:, H:], W2t)
+
+
+@pytest.mark.parametrize("act,bias", [(oracle.ACT_GELU, True), (oracle.ACT_GELU, False), (oracle.ACT_SWIGLU, False)])
+def test_one_expert_top1_is_dense_ffn(act, bias):
+    """A 1-expert top-1 layer equals the dense FFN (library fp64 linear + activation)."""
+    rng = np.random.default_rng(21 + act)
+    T, D, H = 24, 16, 40
+    x, Wg, W1, W2, b1, b2 = _rand_layer(rng, T, D, H, 1, act, bias)
+    out = oracle.moe_layer(x, Wg, W1, W2, K=1, act=act, dtype_tag=oracle.F32, b1=b1, b2=b2, threads=2)
+    assert np.all(out["w"] == 1.0)
+    assert np.all(out["sel"] == 0)
+    ref = _torch_expert(torch.from_numpy(x.astype(np.float64)), act, W1[0], W2[0],
+                        None if b1 is None else b1[0], None if b2 is None else b2[0], H).numpy()
+    np.testing.assert_allclose(out["y"], ref, rtol=1e-12, atol=1e-13)
+
+
+@pytest.mark.parametrize("act,N,K", [(oracle.ACT_GELU, 6, 2), (oracle.ACT_SWIGLU, 8, 3), (oracle.ACT_GELU, 4, 4)])
+def test_sparse_layer_equals_dense_masked_gate(act, N, K):
+    """Brute force: evaluate every expert, weight by the dense masked gate softmax(KeepTopK(H, k)),
+    sum over all experts; equals the sparse oracle within 1e-12 relative."""
+    rng = np.random.default_rng(31 + N + K)
+    T, D, H = 40, 12, 20
+    x, Wg, W1, W2, b1, b2 = _rand_layer(rng, T, D, H, N, act, act == oracle.ACT_GELU)
+    bg = (rng.standard_normal(N) * 0.3).astype(np.float32)
+    out = oracle.moe_layer(x, Wg, W1, W2, K=K, act=act, dtype_tag=oracle.F32, bg=bg, b1=b1, b2=b2, threads=3)
+    x64 = torch.from_numpy(x.astype(np.float64))
+    logits = x64 @ torch.from_numpy(Wg.astype(np.float64)) + torch.from_numpy(bg.astype(np.float64))
+    np.testing.assert_allclose(out["scores"], logits.numpy(), rtol=1e-13, atol=1e-13)
+    # KeepTopK by a library sort (torch.sort is stable when asked), then the masked softmax
+    order = torch.sort(-logits, dim=1, stable=True).indices[:, :K]
+    masked = torch.full_like(logits, -math.inf)
+    masked.scatter_(1, order, logits.gather(1, order))
+    G = torch.softmax(masked, dim=1)
+    y = torch.zeros(T, D, dtype=torch.float64)
+    for e in range(N):
+        Ee = _torch_expert(x64, act, W1[e], W2[e], None if b1 is None else b1[e], None if b2 is None else b2[e], H)
+        y += G[:, e:e + 1] * Ee
+    np.testing.assert_allclose(out["y"], y.numpy(), rtol=1e-12, atol=1e-13)
+    assert out["sel"].tolist() == order.numpy().tolist()
+
+
+def test_selection_on_given_scores_keeps_fp64_weights():
+    """With sel_scores the selection follows the given scores while weights use the fp64 scores."""
+    rng = np.random.default_rng(41)
+    T, D, H, N, K = 10, 8, 16, 6, 2
+    x, Wg, W1, W2, b1, b2 = _rand_layer(rng, T, D, H, N, oracle.ACT_GELU, False)
+    ref = oracle.moe_layer(x, Wg, W1, W2, K=K, act=oracle.ACT_GELU, dtype_tag=oracle.F32, threads=1)
+    forced = np.zeros((T, N), dtype=np.float32)
+    forced[:, 5] = 2.0
+    forced[:, 3] = 1.0
+    out = oracle.moe_layer(x, Wg, W1, W2, K=K, act=oracle.ACT_GELU, dtype_tag=oracle.F32, sel_scores=forced,
+                           threads=1)
+    assert np.all(out["sel"] == np.array([5, 3]))
+    np.testing.assert_array_equal(out["scores"], ref["scores"])
+    s = ref["scores"]
+    np.testing.assert_allclose(out["w"][:, 0], 1 / (1 + np.exp(s[:, 3] - s[:, 5])), rtol=1e-14)
+
+
+def test_layer_rows_threads_are_independent():
+    rng = np.random.default_rng(43)
+    x, Wg, W1, W2, b1, b2 = _rand_layer(rng, 37, 8, 16, 5, oracle.ACT_SWIGLU, False)
+    a = oracle.moe_layer(x, Wg, W1, W2, K=2, act=oracle.ACT_SWIGLU, dtype_tag=oracle.F32, threads=1)
+    b = oracle.moe_layer(x, Wg, W1, W2, K=2, act=oracle.ACT_SWIGLU, dtype_tag=oracle.F32, threads=5)
+    for k in ("scores", "sel", "w", "y"):
+        np.testing.assert_array_equal(a[k], b[k])
+
+
+# --------------------------------------------------------------------------- statistics
+def test_balance_loss_extremes(golden_dir):
+    g = _golden(golden_dir, "balance_loss_extremes.json")
+    N = 8
+    assert oracle.simple_balance_loss(np.full(N, 5.0)) == pytest.approx(g["uniform_value"], rel=1e-15)
+    onehot = np.zeros(N)
+    onehot[3] = 10
+    assert oracle.simple_balance_loss(onehot) == pytest.approx(N, rel=1e-15)  # top-1, all on one
+    two = np.zeros(N)
+    two[[0, 1]] = 10
+    # top-2 with distinct experts per token cannot put everything on one expert: the maximum is N/K
+    assert oracle.simple_balance_loss(two) == pytest.approx(N / 2, rel=1e-15)
+    assert oracle.simple_balance_loss(np.zeros(N)) == 0.0
+
+
+def test_cv_squared_closed_forms():
+    N = 8
+    assert oracle.cv_squared(np.full(N, 3.0)) == 0.0
+    onehot = np.zeros(N)
+    onehot[0] = 7.0
+    assert oracle.cv_squared(onehot) == pytest.approx(N - 1, rel=1e-14)
+    assert oracle.cv_squared(np.array([1.0, 2.0, 3.0, 4.0])) == pytest.approx(1.25 / 6.25, rel=1e-15)
+    assert oracle.cv_squared(np.zeros(N)) == 0.0
+
+
+def test_aux_stats_invariants_and_library_checks():
+    rng = np.random.default_rng(51)
+    T, N, K = 300, 16, 4
+    s = rng.standard_normal((T, N)) * 2
+    sel = oracle.select_topk(s, K)
+    w = oracle.gate_weights(s, sel)
+    st = oracle.aux_stats(s, sel, w, N)
+    np.testing.assert_array_equal(st["counts"], np.bincount(sel.ravel(), minlength=N).astype(np.float64))
+    assert st["importance"].sum() == pytest.approx(T, rel=1e-13)
+    assert st["p_mean"].sum() == pytest.approx(1.0, rel=1e-13)
+    np.testing.assert_allclose(st["p_mean"], torch.softmax(torch.from_numpy(s), 1).mean(0).numpy(), rtol=1e-13)
+    f = st["counts"] / (T * K)
+    assert st["switch"] == pytest.approx(N * float(np.dot(f, st["p_mean"])), rel=1e-13)
+    assert st["simple"] == pytest.approx(N * float(np.sum(f * f)), rel=1e-13)
+    assert st["cv2_importance"] == pytest.approx(float(np.var(st["importance"]) / np.mean(st["importance"]) ** 2),
+                                                 rel=1e-12)
+    assert st["cv2_load"] == pytest.approx(float(np.var(st["counts"]) / np.mean(st["counts"]) ** 2), rel=1e-12)
+
+
+def test_aux_stats_uniform_and_empty():
+    N, K = 8, 2
+    T = 4 * N
+    s = np.zeros((T, N))  # all-equal scores: P = 1/N exactly
+    sel = np.array([[(2 * t) % N, (2 * t + 1) % N] for t in range(T)], dtype=np.int32)  # uniform load
+    w = np.full((T, K), 0.5)
+    st = oracle.aux_stats(s, sel, w, N)
+    assert st["switch"] == pytest.approx(1.0, rel=1e-15)
+    assert st["simple"] == pytest.approx(1.0, rel=1e-15)
+    assert st["cv2_importance"] == 0.0 and st["cv2_load"] == 0.0
+    empty = oracle.aux_stats(np.zeros((0, N)), np.zeros((0, K), np.int32), np.zeros((0, K)), N)
+    assert empty["switch"] == 0.0 and empty["simple"] == 0.0
+    assert np.all(empty["counts"] == 0)
+
+
+def test_demo_scenario_balanced_vs_biased():
+    """The chapter's demo: 10 tokens, 8 experts, top-2; a router biased towards a few experts
+    concentrates the load and raises N * sum f^2."""
+    rng = np.random.default_rng(61)
+    T, D, H, N, K = 10, 16, 32, 8, 2
+    x, Wg, W1, W2, b1, b2 = _rand_layer(rng, T, D, H, N, oracle.ACT_GELU, False)
+    Wg = (rng.standard_normal((D, N)) * 0.02).astype(np.float32)
+    bal = oracle.moe_layer(x, Wg, W1, W2, K=K, act=oracle.ACT_GELU, dtype_tag=oracle.F32, threads=1)
+    bias = np.zeros(N, dtype=np.float32)
+    bias[[1, 6]] = 5.0
+    biased = oracle.moe_layer(x, Wg, W1, W2, K=K, act=oracle.ACT_GELU, dtype_tag=oracle.F32, bg=bias, threads=1)
+    sb = oracle.aux_stats(bal["scores"], bal["sel"], bal["w"], N)
+    sz = oracle.aux_stats(biased["scores"], biased["sel"], biased["w"], N)
+    assert sb["counts"].sum() == T * K and sz["counts"].sum() == T * K
+    assert sorted(np.nonzero(sz["counts"])[0].tolist()) == [1, 6]
+    assert sz["simple"] == pytest.approx(N / K)
+    assert sz["simple"] > sb["simple"] >= 1.0
+
+
+# --------------------------------------------------------------------------- accounting
+def test_expert_total_is_four_times_active(golden_dir):
+    g = _golden(golden_dir, "param_accounting.json")["ratio_case"]
+    D, H, N, K = 64, 256, g["n_experts"], g["top_k"]
+    router = D * N
+    tot = oracle.total_params(D, H, N, K)
+    act = oracle.active_params(D, H, N, K)
+    assert (tot - router) == g["expert_total_over_active"] * (act - router)
+    assert oracle.expert_params(D, H) == 2 * D * H
+
+
+def test_gpt2_moe_parameter_totals(golden_dir):
+    """GPT-2-small dims + 6 experts/top-2 reproduce the printed 446M total / 220M active."""
+    gg = _golden(golden_dir, "param_accounting.json")
+    d = gg["gpt2_small_dims"]
+    c = gg["gpt2_case"]
+    D, H, L, V, C = d["d_model"], d["d_hidden"], d["layers"], d["vocab"], d["context"]
+    ln = 2 * D
+    attn = D * 3 * D + 3 * D + D * D + D
+    non_moe_block = 2 * ln + attn
+    embed_and_head = V * D + C * D + ln + V * D
+    total = embed_and_head + L * (non_moe_block + oracle.total_params(D, H, c["n_experts"], c["top_k"], has_bias=True))
+    active = embed_and_head + L * (non_moe_block + oracle.active_params(D, H, c["n_experts"], c["top_k"],
+                                                                        has_bias=True))
+    assert round(total / 1e6) == c["total_millions_printed"]
+    assert round(active / 1e6) == c["active_millions_printed"]
