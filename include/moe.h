@@ -1,0 +1,220 @@
+/*
+ * moe.h -- C ABI of the sparsely-gated Mixture-of-Experts FFN layer for one
+ * NVIDIA B200 (sm_100a).  Library: sparse_mixture_experts_10_b200/libmoe.so.
+ *
+ * The layer computes, for every token row x of a batch (Shazeer et al. 2017,
+ * as explained in the qiita article "Outrageously Large Neural Networks",
+ * section "Sparsely-Gated MoE layer formula"):
+ *
+ *     y = sum_{i in TopK(x)} G(x)_i * E_i(x),   G(x) = softmax(KeepTopK(x W_g, k))
+ *
+ * with only the selected experts evaluated.  The argument names follow the
+ * Config of the page "MoE(Mixture of Experts)" (sharin-2a1.pages.dev/parts/moe),
+ * section (1): DModel, DHidden, NExperts, TopK.
+ *
+ * Conventions for every entry point
+ *  - Pointers named as device buffers are CUDA device memory owned by the
+ *    caller.  The library never allocates or frees memory, never keeps a
+ *    pointer after a call returns, and never synchronises the stream except in
+ *    moe_get_device_status().  Work is enqueued on `stream` (a cudaStream_t;
+ *    NULL = the legacy default stream) and runs asynchronously.
+ *  - Arrays are row-major and contiguous; leading dimensions are implied by
+ *    the shapes given.  "dtype" arrays hold fp32 (MOE_F32) or bf16 (MOE_BF16)
+ *    elements as selected by moe_config.dtype; biases are always fp32.
+ *  - bf16 layers need DModel and DHidden to be multiples of 8 (16-byte rows
+ *    for the tensor-memory-accelerator copies); fp32 layers need multiples of 4.
+ *  - Return value: MOE_OK (0) or a negative MOE_ERR_* code.  Argument errors
+ *    are found on the host before anything is enqueued.  Errors raised inside
+ *    kernels (a bounded wait that ran out, an index out of range) are sticky in
+ *    a device status word read by moe_get_device_status().
+ *  - Results are deterministic: the same inputs give bitwise-identical
+ *    outputs on the same GPU.
+ */
+#ifndef MOE_H
+#define MOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A CUDA stream (cudaStream_t / CUstream); declared opaquely so that this
+ * header does not need the CUDA headers. */
+typedef struct CUstream_st *moe_stream_t;
+
+/* Element types of x, the weight matrices and the hidden activations. */
+enum { MOE_F32 = 0, MOE_BF16 = 1 };
+
+/* Expert FFN kinds.
+ *  MOE_ACT_GELU   GPT-2 FFN ("Extending Raschka's GPT-2: an MoE trained from
+ *                 scratch on an RTX 3090", section on how MoE works):
+ *                 E(x) = W2 gelu(W1 x + b1) + b2, exact-erf GELU.
+ *  MOE_ACT_SWIGLU SwiGLU FFN with the packed gate_up weight (Transformers-v5
+ *                 MoE article, section 1 "Weight Loading Refactor": experts
+ *                 stacked on dim 0, gate then up concatenated on dim 1):
+ *                 E(x) = W_down (silu(W_gate x) * (W_up x)). No biases. */
+enum { MOE_ACT_GELU = 0, MOE_ACT_SWIGLU = 1 };
+
+/* Return codes. */
+enum {
+    MOE_OK = 0,
+    MOE_ERR_INVALID_ARG = -1,         /* null required pointer, bad size or shape */
+    MOE_ERR_WORKSPACE_TOO_SMALL = -2, /* ws_bytes < the size the query returned */
+    MOE_ERR_UNSUPPORTED = -3,         /* dtype / act / size combination not built */
+    MOE_ERR_CUDA = -4,                /* a CUDA runtime call or launch failed */
+    MOE_ERR_DEVICE_TIMEOUT = -5,      /* a kernel's bounded wait ran out (status word) */
+    MOE_ERR_DEVICE_BOUNDS = -6        /* a kernel found an index out of range (status word) */
+};
+
+/* Bits of the device status word (moe_get_device_status). */
+enum {
+    MOE_STATUS_TIMEOUT = 1,   /* a bounded wait gave up; the kernel returned early */
+    MOE_STATUS_BOUNDS = 2,    /* an expert index or row count was out of range */
+    MOE_STATUS_NAN_LOGIT = 4  /* a NaN router logit was ranked as -inf (not fatal) */
+};
+
+/* Layer shape ("MoE(Mixture of Experts)", section (1), Config). */
+typedef struct {
+    int32_t DModel;   /* D: token width */
+    int32_t DHidden;  /* H: expert hidden width */
+    int32_t NExperts; /* N: number of experts, 1..1024 */
+    int32_t TopK;     /* K: experts per token, 1..min(N, 32) */
+    int32_t act;      /* MOE_ACT_GELU or MOE_ACT_SWIGLU */
+    int32_t dtype;    /* MOE_F32 or MOE_BF16 */
+    int32_t has_bias; /* GELU only: expert biases b1, b2 are given */
+} moe_config;
+
+/* Layer parameters, all device memory.
+ *  W_g [D, N] dtype      router matrix, scores = x W_g (Shazeer gate x W_g)
+ *  b_g [N] fp32 or NULL  per-expert router bias added to the scores
+ *  W1  [N, H, D] dtype   GELU: first linear, out x in
+ *      [N, 2H, D] dtype  SwiGLU: packed gate_up (rows 0..H-1 gate, H..2H-1 up)
+ *  b1  [N, H] fp32       GELU with has_bias, else NULL
+ *  W2  [N, D, H] dtype   second linear / down projection, out x in
+ *  b2  [N, D] fp32       GELU with has_bias, else NULL */
+typedef struct {
+    const void *W_g;
+    const float *b_g;
+    const void *W1;
+    const float *b1;
+    const void *W2;
+    const float *b2;
+} moe_weights;
+
+/* Per-batch statistics, device memory (any pointer may be NULL to skip it).
+ *  counts[N]      tokens routed to each expert ("MoE(Mixture of Experts)",
+ *                 section (2), Stats.TokensPerExpert)
+ *  importance[N]  sum over tokens of the gate weight given to each expert
+ *                 (Shazeer article, load-balancing losses, Importance(X))
+ *  p_mean[N]      mean over tokens of the full N-way softmax of the scores
+ *  scalars[4]     [0] Switch-style N * sum_e f_e * P_e, f_e = counts/(T*K),
+ *                     P_e = p_mean ("Extending Raschka's GPT-2", auxiliary
+ *                     loss section)
+ *                 [1] N * sum_e f_e^2 ("MoE(Mixture of Experts)", section (3))
+ *                 [2] CV(importance)^2, [3] CV(counts)^2 (Shazeer article,
+ *                     load-balancing losses; population variance, hard counts
+ *                     for Load).  The loss weights are left to the caller.
+ * All entries are 0 when T == 0. */
+typedef struct {
+    int32_t *counts;
+    float *importance;
+    float *p_mean;
+    float *scalars;
+} moe_aux;
+
+/* Bytes of device workspace moe_route / moe_forward / moe_aux_stats need for T
+ * tokens (0 if the configuration is invalid).  The workspace must be 256-byte
+ * aligned.  Its contents need no initialisation and are scratch between calls. */
+size_t moe_workspace_size(const moe_config *cfg, int64_t T);
+
+/* Routing only ("MoE(Mixture of Experts)", section (2), Route; Shazeer article,
+ * gating, inference form without noise).
+ *  x [T, D] dtype (device).
+ *  logits [T, N] fp32 or NULL: scores x W_g + b_g, fp32 accumulation.
+ *  topk_idx [T, K] int32: selected experts, best first; equal scores go to the
+ *      lower expert index (stable descending sort); a NaN score ranks as -inf.
+ *  topk_w [T, K] fp32: softmax over the K selected scores, shifted by the best.
+ *  counts [N] int32 or NULL: tokens per expert.
+ * T == 0 is a no-op that zeroes counts. */
+int moe_route(const moe_config *cfg, const void *x, int64_t T, const moe_weights *w,
+              float *logits, int32_t *topk_idx, float *topk_w, int32_t *counts,
+              void *ws, size_t ws_bytes, moe_stream_t stream);
+
+/* The whole layer ("MoE(Mixture of Experts)", section (2), Forward; Shazeer
+ * article, layer formula): route, group the (token, slot) pairs by expert,
+ * evaluate each selected expert once per pair on the tensor cores, scale by the
+ * gate weight and sum the K contributions of a token in slot order 0..K-1.
+ *  x [T, D] dtype (device); y [T, D] in y_dtype (MOE_F32 or MOE_BF16).
+ *  aux: optional statistics (see moe_aux), or NULL.
+ * The routing results and intermediates stay in the workspace; their places
+ * are given by moe_workspace_layout().  T == 0 is a no-op (aux zeroed). */
+int moe_forward(const moe_config *cfg, const void *x, int64_t T, const moe_weights *w,
+                void *y, int32_t y_dtype, moe_aux *aux, void *ws, size_t ws_bytes,
+                moe_stream_t stream);
+
+/* moe_forward that also records CUDA events between its stages, for timing.
+ * stage_events: MOE_N_STAGES + 1 cudaEvent_t handles (created by the caller);
+ * event i is recorded on `stream` before stage i and event MOE_N_STAGES after
+ * the last.  Stages: 0 route, 1 scan, 2 permute, 3 expert up-projection,
+ * 4 expert down-projection, 5 combine, 6 statistics (empty without aux). */
+#define MOE_N_STAGES 7
+int moe_forward_timed(const moe_config *cfg, const void *x, int64_t T, const moe_weights *w,
+                      void *y, int32_t y_dtype, moe_aux *aux, void *ws, size_t ws_bytes,
+                      moe_stream_t stream, void *const *stage_events);
+
+/* Statistics from routing results (see moe_aux for the definitions).
+ *  logits [T, N] fp32, topk_idx [T, K] int32, topk_w [T, K] fp32 (device).
+ *  ws: workspace of at least moe_workspace_size(cfg, T) bytes. */
+int moe_aux_stats(const moe_config *cfg, int64_t T, const float *logits, const int32_t *topk_idx,
+                  const float *topk_w, moe_aux *out, void *ws, size_t ws_bytes,
+                  moe_stream_t stream);
+
+/* Where moe_forward leaves its intermediates inside the workspace (byte
+ * offsets from ws), for inspection in tests.  Rows of each expert's segment in
+ * the permuted buffers start at a multiple of row_align; rows past an expert's
+ * count up to the next multiple are padding.
+ *  logits [T, N] fp32, topk_idx [T, K] int32, topk_w [T, K] fp32
+ *  counts [N] int32, offsets [N+1] int32 (exclusive scan of counts)
+ *  row_offsets [N+1] int32 (padded segment starts)
+ *  perm_slot [rows_cap] int32: slot t*K+j held by each permuted row, -1 = padding
+ *  slot_row [T*K] int32: permuted row of each slot
+ *  x_perm [rows_cap, D] dtype, h [rows_cap, H] dtype, z [T*K, D] fp32 */
+typedef struct {
+    size_t total;
+    size_t logits, topk_idx, topk_w, counts, offsets, row_offsets, perm_slot, slot_row;
+    size_t x_perm, h, z;
+    int64_t rows_cap;
+    int32_t row_align;
+} moe_workspace_layout;
+int moe_get_workspace_layout(const moe_config *cfg, int64_t T, moe_workspace_layout *out);
+
+/* Parameter accounting ("MoE(Mixture of Experts)", section (1)): router D*N
+ * plus all N experts (total) or the K active ones; an expert holds 2*D*H
+ * weights (GELU, + H + D with biases) or 3*D*H (SwiGLU).  -1 if invalid. */
+int64_t moe_total_params(const moe_config *cfg);
+int64_t moe_active_params(const moe_config *cfg);
+
+/* Waits for all work on the current device, returns the sticky device status
+ * bits (MOE_STATUS_*) and clears them.  Negative MOE_ERR_CUDA if the device
+ * cannot be reached. */
+int moe_get_device_status(void);
+
+/* Number of kernels this library has launched in this process (all devices). */
+int64_t moe_launch_count(void);
+
+/* Static description of a return code. */
+const char *moe_error_string(int code);
+
+/* Self-test of the bounded wait used by every kernel that waits on a barrier:
+ * one thread waits on a shared-memory barrier that nothing completes, gives up
+ * after timeout_ns nanoseconds, sets MOE_STATUS_TIMEOUT and returns.  Used by
+ * tests to show that an expired wait leaves the context usable. */
+int moe_selftest_wait_timeout(int64_t timeout_ns, moe_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_H */

@@ -1,0 +1,226 @@
+"""Sparsely-gated Mixture-of-Experts FFN layer for one NVIDIA B200 (sm_100a).
+
+This package is a thin ctypes binding of ``libmoe.so``, whose C ABI is declared
+in ``include/moe.h``.  The functions here carry the same names and arguments as
+the C entry points and only marshal arguments: torch tensors become device
+pointers, streams become ``cudaStream_t`` handles.  Every step of the layer runs
+in the library's CUDA kernels; there is no Python or CPU fallback, and importing
+the package fails loudly when the library has not been built
+(``python -m sparse_mixture_experts_10_b200.build``).
+
+PyTorch is used only to hold device memory and to name streams.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libmoe.so")
+
+MOE_F32, MOE_BF16 = 0, 1
+MOE_ACT_GELU, MOE_ACT_SWIGLU = 0, 1
+MOE_N_STAGES = 7
+STAGE_NAMES = ("route", "scan", "permute", "up", "down", "combine", "stats")
+
+MOE_OK = 0
+MOE_ERR_INVALID_ARG = -1
+MOE_ERR_WORKSPACE_TOO_SMALL = -2
+MOE_ERR_UNSUPPORTED = -3
+MOE_ERR_CUDA = -4
+MOE_ERR_DEVICE_TIMEOUT = -5
+MOE_ERR_DEVICE_BOUNDS = -6
+MOE_STATUS_TIMEOUT, MOE_STATUS_BOUNDS, MOE_STATUS_NAN_LOGIT = 1, 2, 4
+
+EXPORTED = ("moe_workspace_size", "moe_route", "moe_forward", "moe_forward_timed", "moe_aux_stats",
+            "moe_get_workspace_layout", "moe_total_params", "moe_active_params", "moe_get_device_status",
+            "moe_launch_count", "moe_error_string", "moe_selftest_wait_timeout")
+
+
+class moe_config(ctypes.Structure):
+    _fields_ = [("DModel", ctypes.c_int32), ("DHidden", ctypes.c_int32), ("NExperts", ctypes.c_int32),
+                ("TopK", ctypes.c_int32), ("act", ctypes.c_int32), ("dtype", ctypes.c_int32),
+                ("has_bias", ctypes.c_int32)]
+
+
+class moe_weights(ctypes.Structure):
+    _fields_ = [("W_g", ctypes.c_void_p), ("b_g", ctypes.c_void_p), ("W1", ctypes.c_void_p),
+                ("b1", ctypes.c_void_p), ("W2", ctypes.c_void_p), ("b2", ctypes.c_void_p)]
+
+
+class moe_aux(ctypes.Structure):
+    _fields_ = [("counts", ctypes.c_void_p), ("importance", ctypes.c_void_p), ("p_mean", ctypes.c_void_p),
+                ("scalars", ctypes.c_void_p)]
+
+
+class moe_workspace_layout(ctypes.Structure):
+    _fields_ = [("total", ctypes.c_size_t), ("logits", ctypes.c_size_t), ("topk_idx", ctypes.c_size_t),
+                ("topk_w", ctypes.c_size_t), ("counts", ctypes.c_size_t), ("offsets", ctypes.c_size_t),
+                ("row_offsets", ctypes.c_size_t), ("perm_slot", ctypes.c_size_t), ("slot_row", ctypes.c_size_t),
+                ("x_perm", ctypes.c_size_t), ("h", ctypes.c_size_t), ("z", ctypes.c_size_t),
+                ("rows_cap", ctypes.c_int64), ("row_align", ctypes.c_int32)]
+
+
+class MoeError(RuntimeError):
+    def __init__(self, code: int, what: str = ""):
+        self.code = code
+        super().__init__(f"{what}: {error_string(code)} ({code})" if what else f"{error_string(code)} ({code})")
+
+
+_lib = None
+
+
+def load_library():
+    """Load libmoe.so and declare its signatures.  Raises if it has not been built."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with `python -m sparse_mixture_experts_10_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    vp, i32, i64, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
+    cfgp = ctypes.POINTER(moe_config)
+    wp = ctypes.POINTER(moe_weights)
+    auxp = ctypes.POINTER(moe_aux)
+    L.moe_workspace_size.restype = sz
+    L.moe_workspace_size.argtypes = [cfgp, i64]
+    L.moe_route.restype = ctypes.c_int
+    L.moe_route.argtypes = [cfgp, vp, i64, wp, vp, vp, vp, vp, vp, sz, vp]
+    L.moe_forward.restype = ctypes.c_int
+    L.moe_forward.argtypes = [cfgp, vp, i64, wp, vp, i32, auxp, vp, sz, vp]
+    L.moe_forward_timed.restype = ctypes.c_int
+    L.moe_forward_timed.argtypes = [cfgp, vp, i64, wp, vp, i32, auxp, vp, sz, vp, ctypes.POINTER(vp)]
+    L.moe_aux_stats.restype = ctypes.c_int
+    L.moe_aux_stats.argtypes = [cfgp, i64, vp, vp, vp, auxp, vp, sz, vp]
+    L.moe_get_workspace_layout.restype = ctypes.c_int
+    L.moe_get_workspace_layout.argtypes = [cfgp, i64, ctypes.POINTER(moe_workspace_layout)]
+    L.moe_total_params.restype = i64
+    L.moe_total_params.argtypes = [cfgp]
+    L.moe_active_params.restype = i64
+    L.moe_active_params.argtypes = [cfgp]
+    L.moe_get_device_status.restype = ctypes.c_int
+    L.moe_get_device_status.argtypes = []
+    L.moe_launch_count.restype = i64
+    L.moe_launch_count.argtypes = []
+    L.moe_error_string.restype = ctypes.c_char_p
+    L.moe_error_string.argtypes = [ctypes.c_int]
+    L.moe_selftest_wait_timeout.restype = ctypes.c_int
+    L.moe_selftest_wait_timeout.argtypes = [i64, vp]
+    _lib = L
+    return L
+
+
+# ------------------------------------------------------------------ marshalling helpers
+def _ptr(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(s):
+    if s is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(s, int):
+        return s
+    return s.cuda_stream
+
+
+def dtype_code(dt: torch.dtype) -> int:
+    if dt == torch.float32:
+        return MOE_F32
+    if dt == torch.bfloat16:
+        return MOE_BF16
+    raise ValueError(f"unsupported dtype {dt}")
+
+
+def make_config(DModel, DHidden, NExperts, TopK, act=MOE_ACT_GELU, dtype=MOE_BF16, has_bias=False) -> moe_config:
+    return moe_config(DModel, DHidden, NExperts, TopK, act, dtype, int(bool(has_bias)))
+
+
+def make_weights(W_g, W1, W2, b_g=None, b1=None, b2=None) -> moe_weights:
+    return moe_weights(_ptr(W_g), _ptr(b_g), _ptr(W1), _ptr(b1), _ptr(W2), _ptr(b2))
+
+
+def make_aux(counts=None, importance=None, p_mean=None, scalars=None) -> moe_aux:
+    return moe_aux(_ptr(counts), _ptr(importance), _ptr(p_mean), _ptr(scalars))
+
+
+def check(rc: int, what: str = "") -> int:
+    if rc != MOE_OK:
+        raise MoeError(rc, what)
+    return rc
+
+
+def error_string(code: int) -> str:
+    return load_library().moe_error_string(code).decode()
+
+
+# ------------------------------------------------------------------ the C entry points
+def moe_workspace_size(cfg: moe_config, T: int) -> int:
+    return load_library().moe_workspace_size(ctypes.byref(cfg), T)
+
+
+def moe_route(cfg, x, T, weights, logits, topk_idx, topk_w, counts, ws, ws_bytes, stream=None) -> int:
+    return load_library().moe_route(ctypes.byref(cfg), _ptr(x), T, ctypes.byref(weights), _ptr(logits),
+                                    _ptr(topk_idx), _ptr(topk_w), _ptr(counts), _ptr(ws), ws_bytes, _stream(stream))
+
+
+def moe_forward(cfg, x, T, weights, y, y_dtype, aux, ws, ws_bytes, stream=None) -> int:
+    return load_library().moe_forward(ctypes.byref(cfg), _ptr(x), T, ctypes.byref(weights), _ptr(y), y_dtype,
+                                      None if aux is None else ctypes.byref(aux), _ptr(ws), ws_bytes,
+                                      _stream(stream))
+
+
+def moe_forward_timed(cfg, x, T, weights, y, y_dtype, aux, ws, ws_bytes, stream, stage_events) -> int:
+    """stage_events: MOE_N_STAGES + 1 torch.cuda.Event(enable_timing=True) objects."""
+    arr = (ctypes.c_void_p * len(stage_events))(*[e.cuda_event for e in stage_events])
+    return load_library().moe_forward_timed(ctypes.byref(cfg), _ptr(x), T, ctypes.byref(weights), _ptr(y), y_dtype,
+                                            None if aux is None else ctypes.byref(aux), _ptr(ws), ws_bytes,
+                                            _stream(stream), arr)
+
+
+def moe_aux_stats(cfg, T, logits, topk_idx, topk_w, out, ws, ws_bytes, stream=None) -> int:
+    return load_library().moe_aux_stats(ctypes.byref(cfg), T, _ptr(logits), _ptr(topk_idx), _ptr(topk_w),
+                                        ctypes.byref(out), _ptr(ws), ws_bytes, _stream(stream))
+
+
+def moe_get_workspace_layout(cfg, T) -> moe_workspace_layout:
+    out = moe_workspace_layout()
+    check(load_library().moe_get_workspace_layout(ctypes.byref(cfg), T, ctypes.byref(out)), "layout")
+    return out
+
+
+def moe_total_params(cfg) -> int:
+    return load_library().moe_total_params(ctypes.byref(cfg))
+
+
+def moe_active_params(cfg) -> int:
+    return load_library().moe_active_params(ctypes.byref(cfg))
+
+
+def moe_get_device_status() -> int:
+    return load_library().moe_get_device_status()
+
+
+def moe_launch_count() -> int:
+    return load_library().moe_launch_count()
+
+
+def moe_error_string(code: int) -> str:
+    return error_string(code)
+
+
+def moe_selftest_wait_timeout(timeout_ns: int, stream=None) -> int:
+    return load_library().moe_selftest_wait_timeout(timeout_ns, _stream(stream))
+
+
+def alloc_workspace(cfg: moe_config, T: int, device="cuda") -> torch.Tensor:
+    """A device byte buffer of moe_workspace_size bytes (torch's allocator aligns blocks to 512 bytes)."""
+    n = moe_workspace_size(cfg, T)
+    if n == 0:
+        raise MoeError(MOE_ERR_INVALID_ARG, "workspace size")
+    return torch.empty(n, dtype=torch.uint8, device=device)

@@ -1,0 +1,598 @@
+// moe_api.cu -- host side of the C ABI declared in include/moe.h.
+//
+// Validates arguments on the host, carves the caller's workspace, encodes the
+// TMA tensor maps and enqueues the stages of the layer on the caller's stream:
+//   route    fused router (N <= 32) or router GEMM + top-k kernel
+//   scan     counting-sort scan over chunk histograms
+//   permute  stable scatter of token rows into expert segments
+//   up       grouped GEMM + GELU / SwiGLU epilogue  -> h
+//   down     grouped GEMM + gate-weight epilogue    -> z (one row per slot)
+//   combine  y[t] = sum_j z[t, j] in slot order
+//   stats    optional per-batch statistics
+// No call synchronises the stream or allocates memory (moe_get_device_status
+// excepted, which synchronises the device).
+#include "../../include/moe.h"
+#include "moe_common.cuh"
+#include "moe_gemm_simt.cuh"
+#include "moe_gemm_tc.cuh"
+#include "moe_route.cuh"
+
+#include <algorithm>
+#include <atomic>
+#include <mutex>
+
+using namespace moe;
+
+namespace {
+
+std::atomic<int64_t> g_launches{0};
+constexpr uint64_t kTimeoutNs = 1000000000ull;  // bounded waits give up after 1 s
+constexpr int kMaxDevices = 64;
+constexpr size_t kSmallRouterSmemMax = 200 * 1024;
+
+struct DeviceInfo {
+    int sms = 0;
+    bool attrs = false;
+};
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_mu;
+
+size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
+int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+struct Plan {
+    int64_t T;
+    int D, H, N, K, act, dtype, has_bias, es;
+    bool small_router;
+    int np;       // padded expert count of the fused router (8, 16, 32)
+    int vpl;      // values per lane of the top-k kernel
+    int n_chunks;
+    int aux_blocks;
+    int64_t rows_cap;
+    size_t logits, idx, w, counts, offsets, row_offsets, chunk_counts, chunk_base, perm_slot, slot_row, x_perm, h, z,
+        wgt, aux_p, aux_i, aux_c, total;
+};
+
+int make_plan(const moe_config *c, int64_t T, Plan *p) {
+    if (!c || !p) return MOE_ERR_INVALID_ARG;
+    const int64_t D = c->DModel, H = c->DHidden, N = c->NExperts, K = c->TopK;
+    if (D <= 0 || H <= 0 || N <= 0 || K <= 0 || T < 0) return MOE_ERR_INVALID_ARG;
+    if (N > 1024 || K > N || K > 32) return MOE_ERR_INVALID_ARG;
+    if (c->act != MOE_ACT_GELU && c->act != MOE_ACT_SWIGLU) return MOE_ERR_INVALID_ARG;
+    if (c->dtype != MOE_F32 && c->dtype != MOE_BF16) return MOE_ERR_INVALID_ARG;
+    if (c->has_bias && c->act != MOE_ACT_GELU) return MOE_ERR_UNSUPPORTED;
+    const int es = c->dtype == MOE_F32 ? 4 : 2;
+    const int vec = 16 / es;
+    if (D % vec || H % vec) return MOE_ERR_INVALID_ARG;
+    // index arithmetic inside kernels uses 32-bit rows and slot ids
+    if (T * K + N * (int64_t)kRowAlign >= (int64_t)1 << 31) return MOE_ERR_UNSUPPORTED;
+    if (N * 2 * H >= (int64_t)1 << 31 || N * D >= (int64_t)1 << 31) return MOE_ERR_UNSUPPORTED;
+
+    p->T = T;
+    p->D = (int)D; p->H = (int)H; p->N = (int)N; p->K = (int)K;
+    p->act = c->act; p->dtype = c->dtype; p->has_bias = c->has_bias ? 1 : 0; p->es = es;
+    p->np = N <= 8 ? 8 : N <= 16 ? 16 : 32;
+    p->small_router = N <= 32 && (size_t)p->np * D * es + 256 <= kSmallRouterSmemMax;
+    const int need = (int)cdiv(N, 32);
+    p->vpl = need <= 1 ? 1 : need <= 2 ? 2 : need <= 4 ? 4 : need <= 8 ? 8 : need <= 16 ? 16 : 32;
+    p->n_chunks = (int)cdiv(T, kChunk);
+    p->aux_blocks = (int)cdiv(T, kAuxTokens);
+    p->rows_cap = cdiv(T * K + N * (kRowAlign - 1), kRowAlign) * kRowAlign;
+
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        const size_t o = off;
+        off = align256(off + bytes);
+        return o;
+    };
+    p->logits = take((size_t)T * N * 4);
+    p->idx = take((size_t)T * K * 4);
+    p->w = take((size_t)T * K * 4);
+    p->counts = take((size_t)N * 4);
+    p->offsets = take((size_t)(N + 1) * 4);
+    p->row_offsets = take((size_t)(N + 1) * 4);
+    p->chunk_counts = take((size_t)p->n_chunks * N * 4);
+    p->chunk_base = take((size_t)p->n_chunks * N * 4);
+    p->perm_slot = take((size_t)p->rows_cap * 4);
+    p->slot_row = take((size_t)T * K * 4);
+    p->x_perm = take((size_t)p->rows_cap * D * es);
+    p->h = take((size_t)p->rows_cap * H * es);
+    p->z = take((size_t)T * K * D * 4);
+    p->wgt = take(p->small_router ? 0 : (size_t)N * D * es);
+    p->aux_p = take((size_t)p->aux_blocks * N * 4);
+    p->aux_i = take((size_t)p->aux_blocks * N * 4);
+    p->aux_c = take((size_t)p->aux_blocks * N * 4);
+    p->total = off;
+    return MOE_OK;
+}
+
+bool aligned16(const void *ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) == 0; }
+
+int device_info(DeviceInfo **out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MOE_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(g_mu);
+    DeviceInfo &d = g_dev[dev];
+    if (d.sms == 0) {
+        if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return MOE_ERR_CUDA;
+    }
+    if (!d.attrs) {
+        const int big = 227 * 1024;
+        cudaFuncSetAttribute(tc::grouped_gemm_tc_kernel<256, tc::EPI_GELU>, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
+        cudaFuncSetAttribute(tc::grouped_gemm_tc_kernel<256, tc::EPI_SWIGLU>, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
+        cudaFuncSetAttribute(tc::grouped_gemm_tc_kernel<256, tc::EPI_SCATTER>, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
+        cudaFuncSetAttribute(tc::grouped_gemm_tc_kernel<256, tc::EPI_LOGITS>, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
+        cudaFuncSetAttribute(router_small_kernel<float, 8>, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
+        cudaFuncSetAttribute(router_small_kernel<float, 16>, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
+        cudaFuncSetAttribute(router_small_kernel<float, 32>, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
+        cudaFuncSetAttribute(router_small_kernel<__nv_bfloat16, 8>, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
+        cudaFuncSetAttribute(router_small_kernel<__nv_bfloat16, 16>, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
+        cudaFuncSetAttribute(router_small_kernel<__nv_bfloat16, 32>, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
+        cudaFuncSetAttribute(aux_partial_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
+        if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
+        d.attrs = true;
+    }
+    *out = &d;
+    return MOE_OK;
+}
+
+int check_launch() {
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+#define MOE_TRY(expr)                  \
+    do {                               \
+        const int _rc = (expr);        \
+        if (_rc != MOE_OK) return _rc; \
+    } while (0)
+
+// --------------------------------------------------------------- TMA tensor maps
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(f);
+    });
+    return fn;
+}
+
+// 2-D bf16 matrix [rows, cols] row-major; box of box_rows x 64 columns, 128-byte swizzle.
+int make_map(CUtensorMap *m, const void *base, int64_t rows, int64_t cols, int box_rows) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return MOE_ERR_CUDA;
+    const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+    const cuuint32_t box[2] = {64u, (cuuint32_t)box_rows};
+    const cuuint32_t estr[2] = {1u, 1u};
+    const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
+                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? MOE_OK : MOE_ERR_CUDA;
+}
+
+template <int BN, int EPI>
+int launch_tc(const CUtensorMap &A, const CUtensorMap &B, const tc::Params &p, int64_t tiles_upper, int sms,
+              cudaStream_t s) {
+    const int grid = (int)std::min<int64_t>(std::max<int64_t>(tiles_upper, 1), sms);
+    const size_t smem = tc::Shape<BN>::smem_bytes(p.num_groups);
+    tc::grouped_gemm_tc_kernel<BN, EPI><<<grid, tc::kThreads, smem, s>>>(A, B, p);
+    return check_launch();
+}
+
+template <int EPI>
+int launch_simt(const simt::Params &p, int64_t rows, int n_blocks, cudaStream_t s) {
+    const dim3 grid((unsigned)cdiv(std::max<int64_t>(rows, 1), simt::TM), (unsigned)std::max(n_blocks, 1));
+    simt::grouped_gemm_simt_kernel<EPI><<<grid, 256, 0, s>>>(p);
+    return check_launch();
+}
+
+struct Bufs {
+    char *ws;
+    const Plan *p;
+    template <typename T>
+    T *at(size_t off) const { return reinterpret_cast<T *>(ws + off); }
+};
+
+// ---------------------------------------------------------------- stages
+// route: logits (always written to `logits`), top-k, chunk histograms.
+int stage_route(const Plan &P, const Bufs &b, const void *x, const moe_weights *w, float *logits, int *idx,
+                float *tw, const DeviceInfo &dev, cudaStream_t s) {
+    const int T = (int)P.T, D = P.D, N = P.N, K = P.K;
+    int *cc = b.at<int>(P.chunk_counts);
+    if (P.small_router) {
+        const size_t smem = (size_t)P.np * D * P.es + (size_t)P.np * 4;
+#define MOE_ROUTER(TIN, NP)                                                                                     \
+    router_small_kernel<TIN, NP><<<P.n_chunks, 256, smem, s>>>(static_cast<const TIN *>(x), T, D, N, K,        \
+                                                               static_cast<const TIN *>(w->W_g), w->b_g, logits, \
+                                                               idx, tw, cc)
+        if (P.dtype == MOE_F32) {
+            if (P.np == 8) MOE_ROUTER(float, 8);
+            else if (P.np == 16) MOE_ROUTER(float, 16);
+            else MOE_ROUTER(float, 32);
+        } else {
+            if (P.np == 8) MOE_ROUTER(__nv_bfloat16, 8);
+            else if (P.np == 16) MOE_ROUTER(__nv_bfloat16, 16);
+            else MOE_ROUTER(__nv_bfloat16, 32);
+        }
+#undef MOE_ROUTER
+        return check_launch();
+    }
+    // scores by GEMM: logits = x W_g + b_g
+    if (P.dtype == MOE_BF16) {
+        __nv_bfloat16 *wgt = b.at<__nv_bfloat16>(P.wgt);
+        transpose_kernel<__nv_bfloat16><<<dim3((unsigned)cdiv(N, 32), (unsigned)cdiv(D, 32)), dim3(32, 8), 0, s>>>(
+            static_cast<const __nv_bfloat16 *>(w->W_g), D, N, wgt);
+        MOE_TRY(check_launch());
+        CUtensorMap ma, mb;
+        MOE_TRY(make_map(&ma, x, T, D, tc::BM));
+        MOE_TRY(make_map(&mb, wgt, N, D, 256));
+        tc::Params p{};
+        p.num_groups = 1;
+        p.row_offsets = nullptr;
+        p.dense_rows = T;
+        p.n_tiles = (int)cdiv(N, 256);
+        p.num_k_blocks = (int)cdiv(D, tc::BK);
+        p.b_group_rows = 0;
+        p.n_valid = N;
+        p.out = logits;
+        p.ldo = N;
+        p.bias = w->b_g;
+        p.timeout_ns = kTimeoutNs;
+        MOE_TRY((launch_tc<256, tc::EPI_LOGITS>(ma, mb, p, cdiv(T, tc::BM) * p.n_tiles, dev.sms, s)));
+    } else {
+        float *wgt = b.at<float>(P.wgt);
+        transpose_kernel<float><<<dim3((unsigned)cdiv(N, 32), (unsigned)cdiv(D, 32)), dim3(32, 8), 0, s>>>(
+            static_cast<const float *>(w->W_g), D, N, wgt);
+        MOE_TRY(check_launch());
+        simt::Params p{};
+        p.A = static_cast<const float *>(x);
+        p.lda = D;
+        p.B = wgt;
+        p.ldb = D;
+        p.K = D;
+        p.num_groups = 1;
+        p.dense_rows = T;
+        p.b_group_rows = 0;
+        p.n_valid = N;
+        p.out = logits;
+        p.ldo = N;
+        p.bias = w->b_g;
+        MOE_TRY(launch_simt<simt::EPI_LOGITS>(p, T, (int)cdiv(N, simt::TN), s));
+    }
+    const size_t hs = (size_t)N * 4;
+#define MOE_TOPK(V) topk_kernel<V><<<P.n_chunks, 256, hs, s>>>(logits, T, N, K, idx, tw, cc)
+    switch (P.vpl) {
+        case 1: MOE_TOPK(1); break;
+        case 2: MOE_TOPK(2); break;
+        case 4: MOE_TOPK(4); break;
+        case 8: MOE_TOPK(8); break;
+        case 16: MOE_TOPK(16); break;
+        default: MOE_TOPK(32); break;
+    }
+#undef MOE_TOPK
+    return check_launch();
+}
+
+int stage_scan(const Plan &P, const Bufs &b, int *counts_out, cudaStream_t s) {
+    const size_t smem = (size_t)(2 * P.N + 1) * 4;
+    scan_kernel<<<1, 1024, smem, s>>>(b.at<int>(P.chunk_counts), P.n_chunks, P.N, P.T * P.K, b.at<int>(P.chunk_base),
+                                      b.at<int>(P.counts), b.at<int>(P.offsets), b.at<int>(P.row_offsets),
+                                      b.at<int>(P.perm_slot), counts_out);
+    return check_launch();
+}
+
+int stage_permute(const Plan &P, const Bufs &b, const void *x, cudaStream_t s) {
+    const size_t smem = (size_t)(P.N + kChunk * P.K) * 4;
+    if (P.dtype == MOE_F32)
+        permute_kernel<float><<<P.n_chunks, 256, smem, s>>>(static_cast<const float *>(x), (int)P.T, P.D, P.K, P.N,
+                                                           b.at<int>(P.idx), b.at<int>(P.chunk_base),
+                                                           b.at<int>(P.row_offsets), b.at<int>(P.perm_slot),
+                                                           b.at<int>(P.slot_row), b.at<float>(P.x_perm));
+    else
+        permute_kernel<__nv_bfloat16><<<P.n_chunks, 256, smem, s>>>(
+            static_cast<const __nv_bfloat16 *>(x), (int)P.T, P.D, P.K, P.N, b.at<int>(P.idx), b.at<int>(P.chunk_base),
+            b.at<int>(P.row_offsets), b.at<int>(P.perm_slot), b.at<int>(P.slot_row), b.at<__nv_bfloat16>(P.x_perm));
+    return check_launch();
+}
+
+int stage_up(const Plan &P, const Bufs &b, const moe_weights *w, const DeviceInfo &dev, cudaStream_t s) {
+    const int D = P.D, H = P.H, N = P.N;
+    const bool swiglu = P.act == MOE_ACT_SWIGLU;
+    if (P.dtype == MOE_BF16) {
+        CUtensorMap ma, mb;
+        MOE_TRY(make_map(&ma, b.ws + P.x_perm, P.rows_cap, D, tc::BM));
+        MOE_TRY(make_map(&mb, w->W1, (int64_t)N * (swiglu ? 2 * H : H), D, swiglu ? 128 : 256));
+        tc::Params p{};
+        p.num_groups = N;
+        p.row_offsets = b.at<int>(P.row_offsets);
+        p.n_tiles = (int)cdiv(H, swiglu ? 128 : 256);
+        p.num_k_blocks = (int)cdiv(D, tc::BK);
+        p.b_group_rows = swiglu ? 2 * H : H;
+        p.b_up_offset = H;
+        p.n_valid = H;
+        p.out = b.ws + P.h;
+        p.ldo = H;
+        p.bias = swiglu ? nullptr : w->b1;
+        p.timeout_ns = kTimeoutNs;
+        const int64_t upper = (P.rows_cap / tc::BM) * p.n_tiles;
+        if (swiglu) return launch_tc<256, tc::EPI_SWIGLU>(ma, mb, p, upper, dev.sms, s);
+        return launch_tc<256, tc::EPI_GELU>(ma, mb, p, upper, dev.sms, s);
+    }
+    simt::Params p{};
+    p.A = b.at<float>(P.x_perm);
+    p.lda = D;
+    p.B = static_cast<const float *>(w->W1);
+    p.ldb = D;
+    p.K = D;
+    p.num_groups = N;
+    p.row_offsets = b.at<int>(P.row_offsets);
+    p.b_group_rows = swiglu ? 2 * H : H;
+    p.b_up_offset = H;
+    p.n_valid = H;
+    p.out = b.at<float>(P.h);
+    p.ldo = H;
+    p.bias = swiglu ? nullptr : w->b1;
+    if (swiglu) return launch_simt<simt::EPI_SWIGLU>(p, P.rows_cap, (int)cdiv(H, simt::TN / 2), s);
+    return launch_simt<simt::EPI_GELU>(p, P.rows_cap, (int)cdiv(H, simt::TN), s);
+}
+
+int stage_down(const Plan &P, const Bufs &b, const moe_weights *w, const DeviceInfo &dev, cudaStream_t s) {
+    const int D = P.D, H = P.H, N = P.N;
+    const float *bias = P.act == MOE_ACT_SWIGLU ? nullptr : w->b2;
+    if (P.dtype == MOE_BF16) {
+        CUtensorMap ma, mb;
+        MOE_TRY(make_map(&ma, b.ws + P.h, P.rows_cap, H, tc::BM));
+        MOE_TRY(make_map(&mb, w->W2, (int64_t)N * D, H, 256));
+        tc::Params p{};
+        p.num_groups = N;
+        p.row_offsets = b.at<int>(P.row_offsets);
+        p.n_tiles = (int)cdiv(D, 256);
+        p.num_k_blocks = (int)cdiv(H, tc::BK);
+        p.b_group_rows = D;
+        p.n_valid = D;
+        p.out = b.ws + P.z;
+        p.ldo = D;
+        p.bias = bias;
+        p.perm_slot = b.at<int>(P.perm_slot);
+        p.gate_w = b.at<float>(P.w);
+        p.timeout_ns = kTimeoutNs;
+        return launch_tc<256, tc::EPI_SCATTER>(ma, mb, p, (P.rows_cap / tc::BM) * p.n_tiles, dev.sms, s);
+    }
+    simt::Params p{};
+    p.A = b.at<float>(P.h);
+    p.lda = H;
+    p.B = static_cast<const float *>(w->W2);
+    p.ldb = H;
+    p.K = H;
+    p.num_groups = N;
+    p.row_offsets = b.at<int>(P.row_offsets);
+    p.b_group_rows = D;
+    p.n_valid = D;
+    p.out = b.at<float>(P.z);
+    p.ldo = D;
+    p.bias = bias;
+    p.perm_slot = b.at<int>(P.perm_slot);
+    p.gate_w = b.at<float>(P.w);
+    return launch_simt<simt::EPI_SCATTER>(p, P.rows_cap, (int)cdiv(D, simt::TN), s);
+}
+
+int stage_combine(const Plan &P, const Bufs &b, void *y, int y_dtype, const DeviceInfo &dev, cudaStream_t s) {
+    const int64_t nq = P.T * (P.D / 4);
+    const int grid = (int)std::min<int64_t>(cdiv(nq, 256), (int64_t)dev.sms * 8);
+    if (y_dtype == MOE_F32)
+        combine_kernel<float><<<grid, 256, 0, s>>>(b.at<float>(P.z), P.T, P.D, P.K, static_cast<float *>(y));
+    else
+        combine_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(b.at<float>(P.z), P.T, P.D, P.K,
+                                                           static_cast<__nv_bfloat16 *>(y));
+    return check_launch();
+}
+
+int stage_aux(const Plan &P, const Bufs &b, const float *logits, const int *idx, const float *tw, moe_aux *aux,
+              cudaStream_t s) {
+    const int N = P.N;
+    aux_partial_kernel<<<P.aux_blocks, 256, (size_t)24 * N * 4, s>>>(
+        logits, idx, tw, (int)P.T, N, P.K, b.at<float>(P.aux_p), b.at<float>(P.aux_i), b.at<int>(P.aux_c));
+    MOE_TRY(check_launch());
+    aux_finalize_kernel<<<1, 1024, (size_t)3 * N * 8, s>>>(b.at<float>(P.aux_p), b.at<float>(P.aux_i),
+                                                           b.at<int>(P.aux_c), P.aux_blocks, (int)P.T, N, P.K,
+                                                           aux->counts, aux->importance, aux->p_mean, aux->scalars);
+    return check_launch();
+}
+
+int zero_aux(const Plan &P, moe_aux *aux, cudaStream_t s) {
+    if (!aux) return MOE_OK;
+    if (aux->counts && cudaMemsetAsync(aux->counts, 0, (size_t)P.N * 4, s) != cudaSuccess) return MOE_ERR_CUDA;
+    if (aux->importance && cudaMemsetAsync(aux->importance, 0, (size_t)P.N * 4, s) != cudaSuccess) return MOE_ERR_CUDA;
+    if (aux->p_mean && cudaMemsetAsync(aux->p_mean, 0, (size_t)P.N * 4, s) != cudaSuccess) return MOE_ERR_CUDA;
+    if (aux->scalars && cudaMemsetAsync(aux->scalars, 0, 16, s) != cudaSuccess) return MOE_ERR_CUDA;
+    return MOE_OK;
+}
+
+int check_weights(const Plan &P, const moe_weights *w, bool need_experts) {
+    if (!w || !w->W_g) return MOE_ERR_INVALID_ARG;
+    if (!need_experts) return MOE_OK;
+    if (!w->W1 || !w->W2) return MOE_ERR_INVALID_ARG;
+    if (P.has_bias && (!w->b1 || !w->b2)) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(w->W1) || !aligned16(w->W2)) return MOE_ERR_INVALID_ARG;
+    return MOE_OK;
+}
+
+int forward_impl(const moe_config *cfg, const void *x, int64_t T, const moe_weights *w, void *y, int32_t y_dtype,
+                 moe_aux *aux, void *ws, size_t ws_bytes, cudaStream_t s, void *const *ev) {
+    Plan P;
+    MOE_TRY(make_plan(cfg, T, &P));
+    MOE_TRY(check_weights(P, w, true));
+    if (y_dtype != MOE_F32 && y_dtype != MOE_BF16) return MOE_ERR_INVALID_ARG;
+    if (T > 0 && (!x || !y || !aligned16(x) || !aligned16(y))) return MOE_ERR_INVALID_ARG;
+    if (T > 0 && (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u))) return MOE_ERR_INVALID_ARG;
+    if (T > 0 && ws_bytes < P.total) return MOE_ERR_WORKSPACE_TOO_SMALL;
+    auto rec = [&](int i) -> int {
+        if (!ev) return MOE_OK;
+        return cudaEventRecord(static_cast<cudaEvent_t>(ev[i]), s) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+    };
+    if (T == 0) {
+        for (int i = 0; i <= MOE_N_STAGES; ++i) MOE_TRY(rec(i));
+        return zero_aux(P, aux, s);
+    }
+    DeviceInfo *dev = nullptr;
+    MOE_TRY(device_info(&dev));
+    Bufs b{static_cast<char *>(ws), &P};
+    float *logits = b.at<float>(P.logits);
+    int *idx = b.at<int>(P.idx);
+    float *tw = b.at<float>(P.w);
+    MOE_TRY(rec(0));
+    MOE_TRY(stage_route(P, b, x, w, logits, idx, tw, *dev, s));
+    MOE_TRY(rec(1));
+    MOE_TRY(stage_scan(P, b, nullptr, s));
+    MOE_TRY(rec(2));
+    MOE_TRY(stage_permute(P, b, x, s));
+    MOE_TRY(rec(3));
+    MOE_TRY(stage_up(P, b, w, *dev, s));
+    MOE_TRY(rec(4));
+    MOE_TRY(stage_down(P, b, w, *dev, s));
+    MOE_TRY(rec(5));
+    MOE_TRY(stage_combine(P, b, y, y_dtype, *dev, s));
+    MOE_TRY(rec(6));
+    if (aux) MOE_TRY(stage_aux(P, b, logits, idx, tw, aux, s));
+    MOE_TRY(rec(7));
+    return MOE_OK;
+}
+
+}  // namespace
+
+// ===================================================================== C ABI
+extern "C" {
+
+size_t moe_workspace_size(const moe_config *cfg, int64_t T) {
+    Plan P;
+    if (make_plan(cfg, T, &P) != MOE_OK) return 0;
+    return P.total;
+}
+
+int moe_get_workspace_layout(const moe_config *cfg, int64_t T, moe_workspace_layout *out) {
+    if (!out) return MOE_ERR_INVALID_ARG;
+    Plan P;
+    MOE_TRY(make_plan(cfg, T, &P));
+    out->total = P.total;
+    out->logits = P.logits;
+    out->topk_idx = P.idx;
+    out->topk_w = P.w;
+    out->counts = P.counts;
+    out->offsets = P.offsets;
+    out->row_offsets = P.row_offsets;
+    out->perm_slot = P.perm_slot;
+    out->slot_row = P.slot_row;
+    out->x_perm = P.x_perm;
+    out->h = P.h;
+    out->z = P.z;
+    out->rows_cap = P.rows_cap;
+    out->row_align = kRowAlign;
+    return MOE_OK;
+}
+
+int moe_route(const moe_config *cfg, const void *x, int64_t T, const moe_weights *w, float *logits, int32_t *topk_idx,
+              float *topk_w, int32_t *counts, void *ws, size_t ws_bytes, moe_stream_t stream) {
+    Plan P;
+    MOE_TRY(make_plan(cfg, T, &P));
+    MOE_TRY(check_weights(P, w, false));
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (T == 0) {
+        if (counts && cudaMemsetAsync(counts, 0, (size_t)P.N * 4, s) != cudaSuccess) return MOE_ERR_CUDA;
+        return MOE_OK;
+    }
+    if (!x || !aligned16(x) || !topk_idx || !topk_w) return MOE_ERR_INVALID_ARG;
+    if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u)) return MOE_ERR_INVALID_ARG;
+    if (ws_bytes < P.total) return MOE_ERR_WORKSPACE_TOO_SMALL;
+    DeviceInfo *dev = nullptr;
+    MOE_TRY(device_info(&dev));
+    Bufs b{static_cast<char *>(ws), &P};
+    float *lg = logits ? logits : b.at<float>(P.logits);
+    MOE_TRY(stage_route(P, b, x, w, lg, topk_idx, topk_w, *dev, s));
+    if (counts) MOE_TRY(stage_scan(P, b, counts, s));
+    return MOE_OK;
+}
+
+int moe_forward(const moe_config *cfg, const void *x, int64_t T, const moe_weights *w, void *y, int32_t y_dtype,
+                moe_aux *aux, void *ws, size_t ws_bytes, moe_stream_t stream) {
+    return forward_impl(cfg, x, T, w, y, y_dtype, aux, ws, ws_bytes, reinterpret_cast<cudaStream_t>(stream), nullptr);
+}
+
+int moe_forward_timed(const moe_config *cfg, const void *x, int64_t T, const moe_weights *w, void *y, int32_t y_dtype,
+                      moe_aux *aux, void *ws, size_t ws_bytes, moe_stream_t stream, void *const *stage_events) {
+    if (!stage_events) return MOE_ERR_INVALID_ARG;
+    return forward_impl(cfg, x, T, w, y, y_dtype, aux, ws, ws_bytes, reinterpret_cast<cudaStream_t>(stream),
+                        stage_events);
+}
+
+int moe_aux_stats(const moe_config *cfg, int64_t T, const float *logits, const int32_t *topk_idx, const float *topk_w,
+                  moe_aux *out, void *ws, size_t ws_bytes, moe_stream_t stream) {
+    Plan P;
+    MOE_TRY(make_plan(cfg, T, &P));
+    if (!out) return MOE_ERR_INVALID_ARG;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (T == 0) return zero_aux(P, out, s);
+    if (!logits || !topk_idx || !topk_w) return MOE_ERR_INVALID_ARG;
+    if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u)) return MOE_ERR_INVALID_ARG;
+    if (ws_bytes < P.total) return MOE_ERR_WORKSPACE_TOO_SMALL;
+    DeviceInfo *dev = nullptr;
+    MOE_TRY(device_info(&dev));
+    Bufs b{static_cast<char *>(ws), &P};
+    return stage_aux(P, b, logits, topk_idx, topk_w, out, s);
+}
+
+int64_t moe_total_params(const moe_config *c) {
+    Plan P;
+    if (make_plan(c, 0, &P) != MOE_OK) return -1;
+    const int64_t D = P.D, H = P.H, N = P.N;
+    const int64_t ex = P.act == MOE_ACT_SWIGLU ? 3 * D * H : 2 * D * H + (P.has_bias ? H + D : 0);
+    return D * N + N * ex;
+}
+
+int64_t moe_active_params(const moe_config *c) {
+    Plan P;
+    if (make_plan(c, 0, &P) != MOE_OK) return -1;
+    const int64_t D = P.D, H = P.H, N = P.N, K = P.K;
+    const int64_t ex = P.act == MOE_ACT_SWIGLU ? 3 * D * H : 2 * D * H + (P.has_bias ? H + D : 0);
+    return D * N + K * ex;
+}
+
+int moe_get_device_status(void) {
+    if (cudaDeviceSynchronize() != cudaSuccess) return MOE_ERR_CUDA;
+    int v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_status, sizeof v) != cudaSuccess) return MOE_ERR_CUDA;
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(g_status, &zero, sizeof zero) != cudaSuccess) return MOE_ERR_CUDA;
+    return v;
+}
+
+int64_t moe_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+const char *moe_error_string(int code) {
+    switch (code) {
+        case MOE_OK: return "ok";
+        case MOE_ERR_INVALID_ARG: return "invalid argument";
+        case MOE_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
+        case MOE_ERR_UNSUPPORTED: return "unsupported configuration";
+        case MOE_ERR_CUDA: return "CUDA runtime error";
+        case MOE_ERR_DEVICE_TIMEOUT: return "a kernel's bounded wait ran out";
+        case MOE_ERR_DEVICE_BOUNDS: return "a kernel found an index out of range";
+        default: return "unknown error";
+    }
+}
+
+int moe_selftest_wait_timeout(int64_t timeout_ns, moe_stream_t stream) {
+    if (timeout_ns <= 0 || timeout_ns > 10000000000ll) return MOE_ERR_INVALID_ARG;
+    wait_selftest_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>((uint64_t)timeout_ns);
+    return check_launch();
+}
+
+}  // extern "C"

@@ -1,0 +1,561 @@
+// moe_route.cuh -- routing, dispatch, combine and statistics kernels.
+//
+// Routing follows the page "MoE(Mixture of Experts)" (sharin-2a1.pages.dev/
+// parts/moe), section (2) Route: scores = x W_g, a stable descending sort of
+// the expert indices (equal scores: lower index first), the first TopK kept,
+// and a softmax over only those scores shifted by the best one.  This is
+// softmax(KeepTopK(x W_g, k)) of the Shazeer article (qiita), gating section,
+// in its noise-free inference form.
+//
+// Dispatch groups the (token, slot) pairs by expert with a stable counting
+// sort: per-chunk histograms (written by the router), a scan over chunks and
+// experts, then a scatter of token rows into expert-contiguous segments, each
+// starting on a multiple of kRowAlign rows so that every 128-row tensor-core
+// tile lies inside one expert.  This is the "sort and group by expert id" step
+// of the grouped_mm backend (Transformers-v5 MoE article, section 2).
+#pragma once
+
+#include "moe_common.cuh"
+
+namespace moe {
+
+constexpr int kChunk = 32;       // tokens per router / permute block (counting-sort chunk)
+constexpr int kRowAlign = 128;   // expert segment alignment in the permuted buffers
+constexpr int kAuxTokens = 64;   // tokens per statistics block
+
+__device__ __forceinline__ unsigned lanemask_lt() {
+    unsigned m;
+    asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+    return m;
+}
+
+// (taken, value, index) ordering of the top-k selection: an untaken entry beats
+// a taken one; then the larger value; then the lower expert index.  NaN never
+// reaches this comparison (it is ranked as -inf beforehand).
+__device__ __forceinline__ bool beats(float v, int e, bool t, float ov, int oe, bool ot) {
+    if (t != ot) return !t;
+    return v > ov || (v == ov && e < oe);
+}
+
+// Reduce-scatter of 32 per-lane partial sums: afterwards lane l holds, in a[0],
+// the warp-wide sum of entry l.  Each step halves the entries a lane keeps.
+template <int C>
+__device__ __forceinline__ void reduce_scatter_step(float (&a)[32], int lane) {
+    constexpr int H = C / 2;
+    const bool upper = (lane & H) != 0;
+#pragma unroll
+    for (int i = 0; i < H; ++i) {
+        const float send = upper ? a[i] : a[i + H];
+        const float keep = upper ? a[i + H] : a[i];
+        a[i] = keep + __shfl_xor_sync(0xffffffffu, send, H);
+    }
+}
+
+__device__ __forceinline__ void reduce_scatter32(float (&a)[32], int lane) {
+    reduce_scatter_step<32>(a, lane);
+    reduce_scatter_step<16>(a, lane);
+    reduce_scatter_step<8>(a, lane);
+    reduce_scatter_step<4>(a, lane);
+    reduce_scatter_step<2>(a, lane);
+}
+
+template <typename T>
+struct Vec16;  // 16 bytes of T widened to float
+template <>
+struct Vec16<float> {
+    static constexpr int n = 4;
+    __device__ __forceinline__ static void load(const float *p, float (&f)[8]) {
+        const float4 v = *reinterpret_cast<const float4 *>(p);
+        f[0] = v.x; f[1] = v.y; f[2] = v.z; f[3] = v.w;
+    }
+};
+template <>
+struct Vec16<__nv_bfloat16> {
+    static constexpr int n = 8;
+    __device__ __forceinline__ static void load(const __nv_bfloat16 *p, float (&f)[8]) {
+        const uint4 v = *reinterpret_cast<const uint4 *>(p);
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            f[2 * i] = __uint_as_float(w[i] << 16);
+            f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+        }
+    }
+};
+
+// Top-k over one segment of NP lanes, each holding one (score, expert) entry,
+// then the renormalised softmax.  Lane r of the segment (r < K) returns slot r.
+// Returns true for lanes that hold a slot.
+template <int NP>
+__device__ __forceinline__ bool segment_topk(float v, int e, bool taken, int K, int seg_lane, int lane,
+                                             int &slot_e, float &slot_w) {
+    float best0 = 0.f, my_v = -INFINITY;
+    int my_e = 0;
+    for (int r = 0; r < K; ++r) {
+        float cv = v;
+        int ce = e;
+        bool ct = taken;
+#pragma unroll
+        for (int o = NP / 2; o >= 1; o >>= 1) {
+            const float ov = __shfl_xor_sync(0xffffffffu, cv, o);
+            const int oe = __shfl_xor_sync(0xffffffffu, ce, o);
+            const bool ot = __shfl_xor_sync(0xffffffffu, (int)ct, o) != 0;
+            if (beats(ov, oe, ot, cv, ce, ct)) { cv = ov; ce = oe; ct = ot; }
+        }
+        if (e == ce) taken = true;
+        if (r == 0) best0 = cv;
+        if (seg_lane == r) { my_v = cv; my_e = ce; }
+    }
+    const float ex = seg_lane < K ? expf(my_v - best0) : 0.f;
+    float sum = 0.f;
+    const int seg_base = lane - seg_lane;
+    for (int m = 0; m < K; ++m) sum += __shfl_sync(0xffffffffu, ex, seg_base + m);  // slot order
+    slot_e = my_e;
+    slot_w = ex / sum;
+    return seg_lane < K;
+}
+
+// ---------------------------------------------------------------------------
+// Fused router for N <= 32 experts: scores, top-k, softmax, chunk histogram.
+// One block per chunk of kChunk tokens; W_g is staged transposed ([NP][D],
+// zero rows for experts N..NP-1) in shared memory; each warp handles 32/NP
+// tokens at a time, each lane a strided set of 16-byte slices of D; a
+// reduce-scatter leaves lane l with the score of (token l/NP, expert l%NP).
+// ---------------------------------------------------------------------------
+template <typename Tin, int NP>
+__global__ void __launch_bounds__(256) router_small_kernel(const Tin *__restrict__ x, int T, int D, int N, int K,
+                                                           const Tin *__restrict__ Wg, const float *__restrict__ bg,
+                                                           float *__restrict__ logits, int *__restrict__ topk_idx,
+                                                           float *__restrict__ topk_w, int *__restrict__ chunk_counts) {
+    constexpr int TPW = 32 / NP;
+    constexpr int VEC = Vec16<Tin>::n;
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    Tin *WgT = reinterpret_cast<Tin *>(smem_raw);
+    int *hist = reinterpret_cast<int *>(smem_raw + (size_t)NP * D * sizeof(Tin));
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    for (int i = tid; i < D * N; i += blockDim.x) {
+        const int d = i / N, e = i - d * N;
+        WgT[(size_t)e * D + d] = Wg[i];
+    }
+    for (int i = tid; i < (NP - N) * D; i += blockDim.x) WgT[(size_t)N * D + i] = Tin(0.f);
+    if (tid < NP) hist[tid] = 0;
+    __syncthreads();
+
+    const int t_begin = blockIdx.x * kChunk;
+    const int nvec = D / VEC;
+    const int seg_lane = lane % NP;
+    for (int g = warp * TPW; g < kChunk; g += 8 * TPW) {
+        const int t0 = t_begin + g;
+        float a[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) a[i] = 0.f;
+        for (int v = lane; v < nvec; v += 32) {
+            float xf[TPW][8];
+#pragma unroll
+            for (int tt = 0; tt < TPW; ++tt) {
+                if (t0 + tt < T) {
+                    Vec16<Tin>::load(x + (size_t)(t0 + tt) * D + (size_t)v * VEC, xf[tt]);
+                } else {
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) xf[tt][u] = 0.f;
+                }
+            }
+#pragma unroll
+            for (int e = 0; e < NP; ++e) {
+                float wf[8];
+                Vec16<Tin>::load(WgT + (size_t)e * D + (size_t)v * VEC, wf);
+#pragma unroll
+                for (int tt = 0; tt < TPW; ++tt)
+#pragma unroll
+                    for (int u = 0; u < VEC; ++u) a[tt * NP + e] = fmaf(xf[tt][u], wf[u], a[tt * NP + e]);
+            }
+        }
+        reduce_scatter32(a, lane);
+        const int e = seg_lane;
+        const int t = t0 + lane / NP;
+        const bool valid_e = e < N;
+        float s = a[0];
+        if (valid_e && bg) s += bg[e];
+        if (logits && t < T && valid_e) logits[(size_t)t * N + e] = s;
+        if (s != s) {
+            if (valid_e && t < T) set_status(kStatusNanLogit);
+            s = -INFINITY;
+        }
+        int slot_e;
+        float slot_w;
+        const bool has_slot = segment_topk<NP>(s, e, !valid_e, K, seg_lane, lane, slot_e, slot_w);
+        if (has_slot && t < T) {
+            topk_idx[(size_t)t * K + seg_lane] = slot_e;
+            topk_w[(size_t)t * K + seg_lane] = slot_w;
+            atomicAdd(&hist[slot_e], 1);
+        }
+    }
+    __syncthreads();
+    if (tid < N) chunk_counts[(size_t)blockIdx.x * N + tid] = hist[tid];
+}
+
+// ---------------------------------------------------------------------------
+// Top-k + softmax from precomputed fp32 scores [T, N] (N <= 32 * VPL), with the
+// chunk histogram.  One warp per token; lane l holds experts l, l+32, ...
+// ---------------------------------------------------------------------------
+template <int VPL>
+__global__ void __launch_bounds__(256) topk_kernel(const float *__restrict__ logits, int T, int N, int K,
+                                                   int *__restrict__ topk_idx, float *__restrict__ topk_w,
+                                                   int *__restrict__ chunk_counts) {
+    extern __shared__ int hist_s[];
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    for (int e = tid; e < N; e += blockDim.x) hist_s[e] = 0;
+    __syncthreads();
+    for (int tl = warp; tl < kChunk; tl += 8) {
+        const int t = blockIdx.x * kChunk + tl;
+        if (t >= T) break;
+        float v[VPL];
+        uint32_t taken = 0;
+#pragma unroll
+        for (int i = 0; i < VPL; ++i) {
+            const int e = lane + 32 * i;
+            if (e < N) {
+                v[i] = logits[(size_t)t * N + e];
+                if (v[i] != v[i]) {
+                    set_status(kStatusNanLogit);
+                    v[i] = -INFINITY;
+                }
+            } else {
+                v[i] = -INFINITY;
+                taken |= 1u << i;
+            }
+        }
+        float best0 = 0.f, my_v = -INFINITY;
+        int my_e = 0;
+        for (int r = 0; r < K; ++r) {
+            // best untaken entry of this lane (lower index first on ties)
+            float cv = -INFINITY;
+            int ce = 0x7fffffff;
+            bool ct = true;
+#pragma unroll
+            for (int i = 0; i < VPL; ++i) {
+                const bool ti = (taken >> i) & 1u;
+                if (beats(v[i], lane + 32 * i, ti, cv, ce, ct)) { cv = v[i]; ce = lane + 32 * i; ct = ti; }
+            }
+#pragma unroll
+            for (int o = 16; o >= 1; o >>= 1) {
+                const float ov = __shfl_xor_sync(0xffffffffu, cv, o);
+                const int oe = __shfl_xor_sync(0xffffffffu, ce, o);
+                const bool ot = __shfl_xor_sync(0xffffffffu, (int)ct, o) != 0;
+                if (beats(ov, oe, ot, cv, ce, ct)) { cv = ov; ce = oe; ct = ot; }
+            }
+            if ((ce & 31) == lane) taken |= 1u << (ce >> 5);
+            if (r == 0) best0 = cv;
+            if (lane == r) { my_v = cv; my_e = ce; }
+        }
+        const float ex = lane < K ? expf(my_v - best0) : 0.f;
+        float sum = 0.f;
+        for (int m = 0; m < K; ++m) sum += __shfl_sync(0xffffffffu, ex, m);
+        if (lane < K) {
+            topk_idx[(size_t)t * K + lane] = my_e;
+            topk_w[(size_t)t * K + lane] = ex / sum;
+            atomicAdd(&hist_s[my_e], 1);
+        }
+    }
+    __syncthreads();
+    for (int e = tid; e < N; e += blockDim.x) chunk_counts[(size_t)blockIdx.x * N + e] = hist_s[e];
+}
+
+// ---------------------------------------------------------------------------
+// Scan: per expert, the exclusive prefix of the chunk histograms (chunk_base);
+// the per-expert counts, their exclusive scan (offsets) and the padded segment
+// starts (row_offsets, multiples of kRowAlign); padding rows get slot -1.
+// One block of 1024 threads.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(1024) scan_kernel(const int *__restrict__ chunk_counts, int n_chunks, int N,
+                                                    int64_t expect_total, int *__restrict__ chunk_base,
+                                                    int *__restrict__ counts, int *__restrict__ offsets,
+                                                    int *__restrict__ row_offsets, int *__restrict__ perm_slot,
+                                                    int *__restrict__ counts_out) {
+    extern __shared__ int s_scan[];
+    int *s_cnt = s_scan;           // [N]
+    int *s_row = s_scan + N;       // [N + 1]
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    for (int e = warp; e < N; e += 32) {
+        int carry = 0;
+        for (int c0 = 0; c0 < n_chunks; c0 += 32) {
+            const int c = c0 + lane;
+            const int v = c < n_chunks ? chunk_counts[(size_t)c * N + e] : 0;
+            int incl = v;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int n = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += n;
+            }
+            if (c < n_chunks) chunk_base[(size_t)c * N + e] = carry + incl - v;
+            carry += __shfl_sync(0xffffffffu, incl, 31);
+        }
+        if (lane == 0) s_cnt[e] = carry;
+    }
+    __syncthreads();
+    if (warp == 0) {
+        int carry = 0, pcarry = 0;
+        for (int e0 = 0; e0 < N; e0 += 32) {
+            const int e = e0 + lane;
+            const int c = e < N ? s_cnt[e] : 0;
+            const int pc = (c + kRowAlign - 1) / kRowAlign * kRowAlign;
+            int ic = c, ip = pc;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int n1 = __shfl_up_sync(0xffffffffu, ic, o);
+                const int n2 = __shfl_up_sync(0xffffffffu, ip, o);
+                if (lane >= o) { ic += n1; ip += n2; }
+            }
+            if (e < N) {
+                counts[e] = c;
+                if (counts_out) counts_out[e] = c;
+                offsets[e] = carry + ic - c;
+                row_offsets[e] = pcarry + ip - pc;
+                s_row[e] = pcarry + ip - pc;
+            }
+            carry += __shfl_sync(0xffffffffu, ic, 31);
+            pcarry += __shfl_sync(0xffffffffu, ip, 31);
+        }
+        if (lane == 0) {
+            offsets[N] = carry;
+            row_offsets[N] = pcarry;
+            s_row[N] = pcarry;
+            if ((int64_t)carry != expect_total) set_status(kStatusBounds);
+        }
+    }
+    __syncthreads();
+    for (int e = warp; e < N; e += 32) {
+        const int start = s_row[e] + s_cnt[e], end = s_row[e + 1];
+        for (int r = start + lane; r < end; r += 32) perm_slot[r] = -1;
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Permute: stable rank of every (token, slot) entry of a chunk inside its
+// expert (ascending token, then slot), its permuted row, the two index maps,
+// and the copy of the token row into the expert-contiguous buffer.
+// ---------------------------------------------------------------------------
+template <typename Tin>
+__global__ void __launch_bounds__(256) permute_kernel(const Tin *__restrict__ x, int T, int D, int K, int N,
+                                                      const int *__restrict__ topk_idx,
+                                                      const int *__restrict__ chunk_base,
+                                                      const int *__restrict__ row_offsets, int *__restrict__ perm_slot,
+                                                      int *__restrict__ slot_row, Tin *__restrict__ x_perm) {
+    extern __shared__ int s_perm[];
+    int *s_run = s_perm;            // [N]
+    int *s_dest = s_perm + N;       // [kChunk * K]
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int c = blockIdx.x;
+    const int t_begin = c * kChunk;
+    const int t_end = min(T, t_begin + kChunk);
+    const int n_entries = (t_end - t_begin) * K;
+    const int64_t f0 = (int64_t)t_begin * K;
+    for (int e = tid; e < N; e += blockDim.x) s_run[e] = row_offsets[e] + chunk_base[(size_t)c * N + e];
+    __syncthreads();
+    if (warp == 0) {
+        for (int base = 0; base < n_entries; base += 32) {
+            const int f = base + lane;
+            int e = f < n_entries ? topk_idx[f0 + f] : -1;
+            if (f < n_entries && (e < 0 || e >= N)) {
+                set_status(kStatusBounds);
+                e = -1;
+            }
+            const unsigned peers = __match_any_sync(0xffffffffu, e);
+            const int rank = __popc(peers & lanemask_lt());
+            const int leader = __ffs(peers) - 1;
+            const int base_row = e >= 0 ? s_run[e] : 0;
+            __syncwarp();
+            if (e >= 0 && lane == leader) s_run[e] = base_row + __popc(peers);
+            __syncwarp();
+            if (f < n_entries) {
+                const int dest = e >= 0 ? base_row + rank : -1;
+                s_dest[f] = dest;
+                if (dest >= 0) {
+                    perm_slot[dest] = (int)(f0 + f);
+                    slot_row[f0 + f] = dest;
+                } else {
+                    slot_row[f0 + f] = -1;
+                }
+            }
+        }
+    }
+    __syncthreads();
+    constexpr int VEC = 16 / sizeof(Tin);
+    const int nvec = D / VEC;
+    for (int f = warp; f < n_entries; f += 8) {
+        const int dest = s_dest[f];
+        if (dest < 0) continue;
+        const int64_t t = (f0 + f) / K;
+        const uint4 *src = reinterpret_cast<const uint4 *>(x + t * D);
+        uint4 *dst = reinterpret_cast<uint4 *>(x_perm + (int64_t)dest * D);
+        for (int v = lane; v < nvec; v += 32) dst[v] = src[v];
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Combine: y[t] = z[t, 0] + z[t, 1] + ... + z[t, K-1], left to right (slot
+// order), no atomics ("MoE(Mixture of Experts)", section (2), Forward, which
+// adds the weighted expert outputs of a row in selection order).
+// ---------------------------------------------------------------------------
+template <typename Tout>
+__global__ void __launch_bounds__(256) combine_kernel(const float *__restrict__ z, int64_t T, int D, int K,
+                                                      Tout *__restrict__ y) {
+    const int64_t nq = T * (D / 4);
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < nq; i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t t = i / (D / 4);
+        const int d = (int)(i - t * (D / 4)) * 4;
+        const float *zt = z + (t * K) * D + d;
+        float4 acc = *reinterpret_cast<const float4 *>(zt);
+        for (int j = 1; j < K; ++j) {
+            const float4 v = *reinterpret_cast<const float4 *>(zt + (int64_t)j * D);
+            acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+        }
+        if constexpr (sizeof(Tout) == 4) {
+            *reinterpret_cast<float4 *>(y + t * D + d) = acc;
+        } else {
+            uint2 o;
+            o.x = pack_bf16x2(acc.x, acc.y);
+            o.y = pack_bf16x2(acc.z, acc.w);
+            *reinterpret_cast<uint2 *>(y + t * D + d) = o;
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Statistics, pass 1: per block of kAuxTokens tokens, the sums of the full
+// softmax of the scores, of the gate weights per expert, and the counts.
+// Each warp accumulates its tokens in order into its own shared row; the rows
+// are then added in warp order, so the result does not depend on scheduling.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) aux_partial_kernel(const float *__restrict__ logits,
+                                                          const int *__restrict__ topk_idx,
+                                                          const float *__restrict__ topk_w, int T, int N, int K,
+                                                          float *__restrict__ part_p, float *__restrict__ part_imp,
+                                                          int *__restrict__ part_cnt) {
+    extern __shared__ float s_aux[];
+    float *acc_p = s_aux;                                     // [8][N]
+    float *acc_i = s_aux + 8 * N;                             // [8][N]
+    int *acc_c = reinterpret_cast<int *>(s_aux + 16 * N);     // [8][N]
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    for (int i = tid; i < 8 * N; i += blockDim.x) { acc_p[i] = 0.f; acc_i[i] = 0.f; acc_c[i] = 0; }
+    __syncthreads();
+    const int t_begin = blockIdx.x * kAuxTokens;
+    const int t_end = min(T, t_begin + kAuxTokens);
+    for (int t = t_begin + warp; t < t_end; t += 8) {
+        const float *s = logits + (size_t)t * N;
+        float mx = -INFINITY;
+        for (int e = lane; e < N; e += 32) mx = fmaxf(mx, s[e]);
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        float zsum = 0.f;
+        for (int e = lane; e < N; e += 32) zsum += expf(s[e] - mx);
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) zsum += __shfl_xor_sync(0xffffffffu, zsum, o);
+        for (int e = lane; e < N; e += 32) acc_p[warp * N + e] += expf(s[e] - mx) / zsum;
+        if (lane == 0) {
+            for (int j = 0; j < K; ++j) {
+                const int e = topk_idx[(size_t)t * K + j];
+                if (e < 0 || e >= N) {
+                    set_status(kStatusBounds);
+                    continue;
+                }
+                acc_i[warp * N + e] += topk_w[(size_t)t * K + j];
+                acc_c[warp * N + e] += 1;
+            }
+        }
+        __syncwarp();
+    }
+    __syncthreads();
+    for (int e = tid; e < N; e += blockDim.x) {
+        float p = 0.f, im = 0.f;
+        int c = 0;
+        for (int w = 0; w < 8; ++w) { p += acc_p[w * N + e]; im += acc_i[w * N + e]; c += acc_c[w * N + e]; }
+        part_p[(size_t)blockIdx.x * N + e] = p;
+        part_imp[(size_t)blockIdx.x * N + e] = im;
+        part_cnt[(size_t)blockIdx.x * N + e] = c;
+    }
+}
+
+// Statistics, pass 2 (one block): sums over blocks in block order, then the
+// scalars in double precision:
+//   f_e = counts_e / (T K); switch = N sum f_e P_e; simple = N sum f_e^2;
+//   CV^2 = population variance / mean^2 (0 when the mean is 0).
+__global__ void __launch_bounds__(1024) aux_finalize_kernel(const float *__restrict__ part_p,
+                                                            const float *__restrict__ part_imp,
+                                                            const int *__restrict__ part_cnt, int nblk, int T,
+                                                            int N, int K, int *__restrict__ counts,
+                                                            float *__restrict__ importance,
+                                                            float *__restrict__ p_mean, float *__restrict__ scalars) {
+    extern __shared__ double s_fin[];
+    double *sp = s_fin, *si = s_fin + N, *sc = s_fin + 2 * N;
+    for (int e = threadIdx.x; e < N; e += blockDim.x) {
+        float p = 0.f, im = 0.f;
+        int c = 0;
+        for (int b = 0; b < nblk; ++b) {
+            p += part_p[(size_t)b * N + e];
+            im += part_imp[(size_t)b * N + e];
+            c += part_cnt[(size_t)b * N + e];
+        }
+        const float pm = T > 0 ? p / (float)T : 0.f;
+        if (counts) counts[e] = c;
+        if (importance) importance[e] = im;
+        if (p_mean) p_mean[e] = pm;
+        sp[e] = pm;
+        si[e] = im;
+        sc[e] = c;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0 && scalars) {
+        double sw = 0.0, ss = 0.0, mi = 0.0, mc = 0.0;
+        const double tk = (double)T * (double)K;
+        for (int e = 0; e < N; ++e) {
+            const double f = tk > 0 ? sc[e] / tk : 0.0;
+            sw += f * sp[e];
+            ss += f * f;
+            mi += si[e];
+            mc += sc[e];
+        }
+        mi /= N;
+        mc /= N;
+        double vi = 0.0, vc = 0.0;
+        for (int e = 0; e < N; ++e) {
+            vi += (si[e] - mi) * (si[e] - mi);
+            vc += (sc[e] - mc) * (sc[e] - mc);
+        }
+        vi /= N;
+        vc /= N;
+        scalars[0] = (float)(N * sw);
+        scalars[1] = (float)(N * ss);
+        scalars[2] = mi == 0.0 ? 0.f : (float)(vi / (mi * mi));
+        scalars[3] = mc == 0.0 ? 0.f : (float)(vc / (mc * mc));
+    }
+}
+
+// W_g [D, N] -> W_g^T [N, D] (the K-major operand layout of the router GEMM).
+template <typename Tin>
+__global__ void transpose_kernel(const Tin *__restrict__ src, int R, int C, Tin *__restrict__ dst) {
+    __shared__ Tin tile[32][33];
+    const int c0 = blockIdx.x * 32, r0 = blockIdx.y * 32;
+    for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+        const int r = r0 + i, c = c0 + threadIdx.x;
+        if (r < R && c < C) tile[i][threadIdx.x] = src[(size_t)r * C + c];
+    }
+    __syncthreads();
+    for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+        const int c = c0 + i, r = r0 + threadIdx.x;
+        if (r < R && c < C) dst[(size_t)c * R + r] = tile[threadIdx.x][i];
+    }
+}
+
+// Bounded-wait self-test: one thread waits on a barrier nothing completes.
+__global__ void wait_selftest_kernel(uint64_t timeout_ns) {
+    __shared__ uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        fence_mbar_init();
+        mbar_wait(&bar, 0, timeout_ns);
+    }
+}
+
+}  // namespace moe

@@ -1,0 +1,371 @@
+"""Parity of the CUDA path (through the C ABI) against the fp64 oracle.
+
+Routing: top-k indices and per-expert counts bit-exact against the oracle's
+top-k applied to the device's own fp32 logits; logits within 1e-4 of the
+fp64 scores (row-scaled).  Layer outputs: bf16 layers within max-abs 2e-2 and
+relative L2 1e-2 of fp64; fp32 layers within 1e-4 (relative).  Dispatch
+(histogram, scan, permutation) is integer work and is compared exactly.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import sparse_mixture_experts_10_b200 as moe
+from moe_inputs import ACT_GELU, ACT_SWIGLU, WORKLOADS, Workload, make_inputs
+from sparse_mixture_experts_10_b200 import build as moe_build
+from tests import parity_helpers as ph
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    moe_build.build()
+    moe.load_library()
+    assert moe.moe_get_device_status() == 0
+    yield
+    torch.cuda.empty_cache()
+
+
+class Layer:
+    """Config, weights and workspace of one workload on the device."""
+
+    def __init__(self, wl: Workload, inp):
+        self.wl, self.inp = wl, inp
+        self.cfg = moe.make_config(wl.D, wl.H, wl.N, wl.K, wl.act, moe.dtype_code(wl.dtype), wl.has_bias)
+        self.w = moe.make_weights(inp["W_g"], inp["W1"], inp["W2"], inp["b_g"], inp["b1"], inp["b2"])
+
+    def forward(self, x=None, y_dtype=torch.float32, with_aux=True):
+        x = self.inp["x"] if x is None else x
+        T, N = x.shape[0], self.wl.N
+        ws = moe.alloc_workspace(self.cfg, max(T, 1))
+        y = torch.full((T, self.wl.D), float("nan"), dtype=y_dtype, device="cuda")
+        aux = None
+        if with_aux:
+            aux = dict(counts=torch.full((N,), -1, dtype=torch.int32, device="cuda"),
+                       importance=torch.full((N,), -1.0, device="cuda"),
+                       p_mean=torch.full((N,), -1.0, device="cuda"),
+                       scalars=torch.full((4,), -1.0, device="cuda"))
+        caux = moe.make_aux(**aux) if aux else None
+        moe.check(moe.moe_forward(self.cfg, x, T, self.w, y, moe.dtype_code(y_dtype), caux, ws, ws.numel()),
+                  "moe_forward")
+        torch.cuda.synchronize()
+        assert moe.moe_get_device_status() == 0
+        return y, ws, aux
+
+    def views(self, ws, T):
+        """The routing results and dispatch maps moe_forward left in the workspace."""
+        L = moe.moe_get_workspace_layout(self.cfg, T)
+        N, K = self.wl.N, self.wl.K
+
+        def v(off, n, dt):
+            return ws[off:off + n * torch.tensor([], dtype=dt).element_size()].view(dt)
+
+        es_dt = self.wl.dtype
+        return dict(
+            logits=v(L.logits, T * N, torch.float32).view(T, N).cpu().numpy(),
+            idx=v(L.topk_idx, T * K, torch.int32).view(T, K).cpu().numpy(),
+            w=v(L.topk_w, T * K, torch.float32).view(T, K).cpu().numpy(),
+            counts=v(L.counts, N, torch.int32).cpu().numpy(),
+            offsets=v(L.offsets, N + 1, torch.int32).cpu().numpy(),
+            row_offsets=v(L.row_offsets, N + 1, torch.int32).cpu().numpy(),
+            perm_slot=v(L.perm_slot, L.rows_cap, torch.int32).cpu().numpy(),
+            slot_row=v(L.slot_row, T * K, torch.int32).cpu().numpy(),
+            x_perm=v(L.x_perm, L.rows_cap * self.wl.D, es_dt).view(L.rows_cap, self.wl.D),
+            rows_cap=L.rows_cap,
+        )
+
+
+def check_routing(V, ref_scores, K):
+    """Logits within tolerance, top-k bit-exact on the device's logits, counts exact."""
+    ph.assert_logits_close(V["logits"], ref_scores)
+    sel = oracle.select_topk(V["logits"].astype(np.float64), K)
+    np.testing.assert_array_equal(V["idx"], sel)
+    N = V["counts"].shape[0]
+    np.testing.assert_array_equal(V["counts"], np.bincount(sel.ravel(), minlength=N))
+
+
+def check_dispatch(V, x, K):
+    """The permutation is the stable counting sort of the (token, slot) pairs by expert."""
+    idx = V["idx"]
+    T = idx.shape[0]
+    N = V["counts"].shape[0]
+    counts = np.bincount(idx.ravel(), minlength=N)
+    np.testing.assert_array_equal(V["counts"], counts)
+    np.testing.assert_array_equal(V["offsets"], np.concatenate([[0], np.cumsum(counts)]))
+    padded = (counts + 127) // 128 * 128
+    np.testing.assert_array_equal(V["row_offsets"], np.concatenate([[0], np.cumsum(padded)]))
+    ro = V["row_offsets"]
+    flat = idx.ravel()
+    for e in range(N):
+        seg = V["perm_slot"][ro[e]:ro[e + 1]]
+        expect = np.nonzero(flat == e)[0]
+        np.testing.assert_array_equal(seg[:counts[e]], expect)
+        assert np.all(seg[counts[e]:] == -1)
+        np.testing.assert_array_equal(V["slot_row"][expect], np.arange(ro[e], ro[e] + counts[e]))
+    rows = V["slot_row"]
+    tok = np.arange(T * K) // K
+    xp = V["x_perm"][torch.from_numpy(rows.astype(np.int64)).cuda()]
+    assert torch.equal(xp, x[torch.from_numpy(tok).cuda()])
+
+
+def run_full(wl, inp, y_dtype=torch.float32):
+    layer = Layer(wl, inp)
+    T = inp["x"].shape[0]
+    y, ws, aux = layer.forward(y_dtype=y_dtype)
+    V = layer.views(ws, T)
+    ref = ph.oracle_full_layer(inp, wl, wl.K, gpu_logits=V["logits"])
+    check_routing(V, ref["scores"], wl.K)
+    ph.assert_weights_close(V["w"], ref["w"], ref["scores"])
+    check_dispatch(V, inp["x"], wl.K)
+    errs = ph.assert_y_close(y.float().cpu().numpy(), ref["y"], wl.dtype if y_dtype == torch.float32 else y_dtype)
+    return layer, y, ws, aux, V, ref, errs
+
+
+def check_aux(aux, V, N, K):
+    st = oracle.aux_stats(V["logits"].astype(np.float64), V["idx"], V["w"].astype(np.float64), N)
+    np.testing.assert_array_equal(aux["counts"].cpu().numpy(), st["counts"].astype(np.int32))
+    np.testing.assert_allclose(aux["importance"].cpu().numpy(), st["importance"], rtol=1e-5, atol=1e-5)
+    np.testing.assert_allclose(aux["p_mean"].cpu().numpy(), st["p_mean"], rtol=1e-5, atol=1e-7)
+    sc = aux["scalars"].cpu().numpy()
+    np.testing.assert_allclose(sc, [st["switch"], st["simple"], st["cv2_importance"], st["cv2_load"]],
+                               rtol=1e-4, atol=1e-6)
+
+
+# ----------------------------------------------------------------------------- tiny fp32
+def test_tiny_fp32_full_layer():
+    wl = WORKLOADS["tiny"]
+    inp = make_inputs(wl, "cuda")
+    layer, y, ws, aux, V, ref, errs = run_full(wl, inp)
+    check_aux(aux, V, wl.N, wl.K)
+
+
+def test_tiny_fp32_random_biases_and_router_bias():
+    wl = WORKLOADS["tiny"].with_(random_bias=True, zipf_s=0.5)
+    inp = make_inputs(wl, "cuda", T=300)
+    run_full(wl, inp)
+
+
+@pytest.mark.parametrize("T", [1, 2, 33, 127, 129])
+def test_tiny_fp32_small_and_ragged_batches(T):
+    wl = WORKLOADS["tiny"].with_(random_bias=True)
+    inp = make_inputs(wl, "cuda", T=T)
+    run_full(wl, inp)
+
+
+def test_topk_equals_n_and_top1():
+    for N, K in [(8, 8), (8, 1), (6, 6), (32, 3), (20, 5)]:
+        wl = WORKLOADS["tiny"].with_(N=N, K=K, random_bias=True)
+        inp = make_inputs(wl, "cuda", T=200)
+        run_full(wl, inp)
+
+
+def test_single_expert_top1():
+    wl = WORKLOADS["tiny"].with_(N=1, K=1, random_bias=True)
+    inp = make_inputs(wl, "cuda", T=100)
+    layer, y, ws, aux, V, ref, errs = run_full(wl, inp)
+    assert np.all(V["w"] == 1.0)
+
+
+def test_all_tokens_on_one_expert_and_empty_experts():
+    wl = WORKLOADS["tiny"].with_(random_bias=True)
+    inp = make_inputs(wl, "cuda", T=400)
+    inp["b_g"] = torch.zeros(wl.N, device="cuda")
+    inp["b_g"][5] = 100.0
+    inp["b_g"][2] = 50.0
+    layer, y, ws, aux, V, ref, errs = run_full(wl, inp)
+    assert np.all(V["idx"][:, 0] == 5) and np.all(V["idx"][:, 1] == 2)
+    assert V["counts"][5] == 400 and V["counts"].sum() == 800
+    check_aux(aux, V, wl.N, wl.K)
+
+
+def test_exact_ties_go_to_lower_index():
+    wl = WORKLOADS["tiny"].with_(random_bias=True)
+    inp = make_inputs(wl, "cuda", T=256)
+    Wg = inp["W_g"]
+    Wg[:, 6] = Wg[:, 1]
+    Wg[:, 3] = Wg[:, 1]
+    layer, y, ws, aux, V, ref, errs = run_full(wl, inp)
+    for t in range(256):
+        tied = [e for e in V["idx"][t].tolist() if e in (1, 3, 6)]
+        assert tied == sorted(tied)
+        if 3 in tied:
+            assert 1 in tied
+        if 6 in tied:
+            assert 1 in tied and 3 in tied
+
+
+def test_zero_tokens():
+    wl = WORKLOADS["tiny"]
+    inp = make_inputs(wl, "cuda", T=4)
+    layer = Layer(wl, inp)
+    ws = moe.alloc_workspace(layer.cfg, 1)
+    aux = dict(counts=torch.full((wl.N,), 7, dtype=torch.int32, device="cuda"),
+               importance=torch.ones(wl.N, device="cuda"), p_mean=torch.ones(wl.N, device="cuda"),
+               scalars=torch.ones(4, device="cuda"))
+    y = torch.empty(0, wl.D, device="cuda")
+    moe.check(moe.moe_forward(layer.cfg, inp["x"], 0, layer.w, y, moe.MOE_F32, moe.make_aux(**aux), ws, ws.numel()))
+    torch.cuda.synchronize()
+    for k in aux:
+        assert torch.all(aux[k] == 0), k
+    cnt = torch.full((wl.N,), 3, dtype=torch.int32, device="cuda")
+    moe.check(moe.moe_route(layer.cfg, inp["x"], 0, layer.w, None, None, None, cnt, ws, ws.numel()))
+    torch.cuda.synchronize()
+    assert torch.all(cnt == 0)
+
+
+# ----------------------------------------------------------------------------- bf16, tensor cores
+def test_gpt2_bf16_reduced_batch_full_layer():
+    wl = WORKLOADS["gpt2"]
+    inp = make_inputs(wl, "cuda", T=1000)
+    layer, y, ws, aux, V, ref, errs = run_full(wl, inp)
+    check_aux(aux, V, wl.N, wl.K)
+
+
+def test_gpt2_bf16_random_biases():
+    wl = WORKLOADS["gpt2"].with_(random_bias=True)
+    inp = make_inputs(wl, "cuda", T=777)
+    run_full(wl, inp)
+
+
+def test_bf16_ragged_dims_gelu_and_swiglu():
+    """D and H not multiples of the 64-wide K slice or of the 256/128-wide column tiles."""
+    for act in (ACT_GELU, ACT_SWIGLU):
+        wl = Workload("ragged", 9, 300, 200, 328, 5, 2, act, torch.bfloat16, act == ACT_GELU, 0.05,
+                      random_bias=True)
+        inp = make_inputs(wl, "cuda")
+        run_full(wl, inp)
+
+
+def test_bf16_output_dtype():
+    wl = WORKLOADS["gpt2"]
+    inp = make_inputs(wl, "cuda", T=300)
+    layer = Layer(wl, inp)
+    y32, ws, _ = layer.forward(y_dtype=torch.float32, with_aux=False)
+    y16, _, _ = layer.forward(y_dtype=torch.bfloat16, with_aux=False)
+    assert torch.equal(y16, y32.to(torch.bfloat16))
+
+
+def test_gpt2_full_size_sampled_rows():
+    wl = WORKLOADS["gpt2"]
+    inp = make_inputs(wl, "cuda")
+    layer = Layer(wl, inp)
+    y, ws, aux = layer.forward()
+    V = layer.views(ws, wl.T)
+    sel = oracle.select_topk(V["logits"].astype(np.float64), wl.K)
+    np.testing.assert_array_equal(V["idx"], sel)
+    check_dispatch(V, inp["x"], wl.K)
+    check_aux(aux, V, wl.N, wl.K)
+    rows = ph.sample_rows(wl.T, 48, V["idx"], wl.N, seed=2)
+    ref = ph.oracle_rows(inp, wl, wl.K, rows, V["logits"])
+    ph.assert_logits_close(V["logits"][rows], ref["scores"])
+    ph.assert_weights_close(V["w"][rows], ref["w"], ref["scores"])
+    ph.assert_y_close(y[torch.from_numpy(rows).cuda()].cpu().numpy(), ref["y"], wl.dtype)
+
+
+def _full_size_sampled(name, n_rows, seed):
+    wl = WORKLOADS[name]
+    inp = make_inputs(wl, "cuda")
+    layer = Layer(wl, inp)
+    y, ws, aux = layer.forward()
+    V = layer.views(ws, wl.T)
+    sel = oracle.select_topk(V["logits"].astype(np.float64), wl.K)
+    np.testing.assert_array_equal(V["idx"], sel)
+    np.testing.assert_array_equal(V["counts"], np.bincount(sel.ravel(), minlength=wl.N))
+    check_aux(aux, V, wl.N, wl.K)
+    rows = ph.sample_rows(wl.T, n_rows, V["idx"], wl.N, seed=seed, least_loaded=2)
+    ref = ph.oracle_rows(inp, wl, wl.K, rows, V["logits"])
+    ph.assert_logits_close(V["logits"][rows], ref["scores"])
+    ph.assert_weights_close(V["w"][rows], ref["w"], ref["scores"])
+    errs = ph.assert_y_close(y[torch.from_numpy(rows).cuda()].cpu().numpy(), ref["y"], wl.dtype)
+    del inp, layer, ws, y
+    torch.cuda.empty_cache()
+    return errs
+
+
+def test_mixtral_full_size_sampled_rows():
+    _full_size_sampled("mixtral", 24, 3)
+
+
+@pytest.mark.parametrize("name", ["deepseek", "deepseek_zipf"])
+def test_deepseek_full_size_sampled_rows(name):
+    _full_size_sampled(name, 12, 4)
+
+
+@pytest.mark.parametrize("name", ["decode1", "decode8", "decode64"])
+def test_decode_full_layer(name):
+    wl = WORKLOADS[name]
+    inp = make_inputs(wl, "cuda")
+    run_full(wl, inp)
+
+
+# ----------------------------------------------------------------------------- entry points, determinism
+def test_route_entry_point_matches_forward():
+    wl = WORKLOADS["gpt2"]
+    inp = make_inputs(wl, "cuda", T=500)
+    layer = Layer(wl, inp)
+    y, ws, aux = layer.forward()
+    V = layer.views(ws, 500)
+    logits = torch.empty(500, wl.N, device="cuda")
+    idx = torch.empty(500, wl.K, dtype=torch.int32, device="cuda")
+    w = torch.empty(500, wl.K, device="cuda")
+    cnt = torch.empty(wl.N, dtype=torch.int32, device="cuda")
+    ws2 = moe.alloc_workspace(layer.cfg, 500)
+    moe.check(moe.moe_route(layer.cfg, inp["x"], 500, layer.w, logits, idx, w, cnt, ws2, ws2.numel()))
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(logits.cpu().numpy(), V["logits"])
+    np.testing.assert_array_equal(idx.cpu().numpy(), V["idx"])
+    np.testing.assert_array_equal(w.cpu().numpy(), V["w"])
+    np.testing.assert_array_equal(cnt.cpu().numpy(), V["counts"])
+    out = dict(counts=torch.empty(wl.N, dtype=torch.int32, device="cuda"), importance=torch.empty(wl.N, device="cuda"),
+               p_mean=torch.empty(wl.N, device="cuda"), scalars=torch.empty(4, device="cuda"))
+    moe.check(moe.moe_aux_stats(layer.cfg, 500, logits, idx, w, moe.make_aux(**out), ws2, ws2.numel()))
+    torch.cuda.synchronize()
+    for k in out:
+        assert torch.equal(out[k], aux[k]), k
+
+
+def test_bitwise_deterministic_runs():
+    for name, T in [("gpt2", 2000), ("mixtral", 300)]:
+        wl = WORKLOADS[name]
+        inp = make_inputs(wl, "cuda", T=T)
+        layer = Layer(wl, inp)
+        y1, ws1, a1 = layer.forward()
+        y2, ws2, a2 = layer.forward()
+        assert torch.equal(y1, y2)
+        for k in a1:
+            assert torch.equal(a1[k], a2[k])
+        del inp, layer
+        torch.cuda.empty_cache()
+
+
+def test_nan_scores_rank_last_and_flag_status():
+    wl = WORKLOADS["tiny"]
+    inp = make_inputs(wl, "cuda", T=64)
+    inp["x"][7, 3] = float("nan")
+    layer = Layer(wl, inp)
+    ws = moe.alloc_workspace(layer.cfg, 64)
+    y = torch.empty(64, wl.D, device="cuda")
+    moe.check(moe.moe_forward(layer.cfg, inp["x"], 64, layer.w, y, moe.MOE_F32, None, ws, ws.numel()))
+    st = moe.moe_get_device_status()
+    assert st & moe.MOE_STATUS_NAN_LOGIT
+    V = layer.views(ws, 64)
+    assert V["idx"][7].tolist() == [0, 1]  # every score NaN -> all rank as -inf -> lowest indices
+    ok = np.ones(64, bool)
+    ok[7] = False
+    ref = ph.oracle_full_layer(inp | {"x": inp["x"][torch.from_numpy(ok).cuda()]}, wl, wl.K,
+                               gpu_logits=V["logits"][ok])
+    ph.assert_y_close(y[torch.from_numpy(ok).cuda()].cpu().numpy(), ref["y"], wl.dtype)
+    assert moe.moe_get_device_status() == 0
+
+
+def test_bounded_wait_expires_and_context_survives():
+    moe.check(moe.moe_selftest_wait_timeout(20_000_000))
+    st = moe.moe_get_device_status()
+    assert st & moe.MOE_STATUS_TIMEOUT
+    assert moe.moe_get_device_status() == 0
+    wl = WORKLOADS["tiny"]
+    run_full(wl, make_inputs(wl, "cuda", T=64))
