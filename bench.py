@@ -4,10 +4,13 @@
 
 A step is one pass of the whole layer (route, scan, permute, expert up- and
 down-projections, combine, statistics) over one batch of synthetic tokens
-already resident in device memory.  Each timed step is bracketed by CUDA
-events recorded on the launching stream by the library itself
-(moe_forward_timed); the L2 cache is flushed (a 512 MiB buffer is written)
-before every step, outside the events.  With N > 1 (torchrun) every rank runs
+already resident in device memory.  One layer call (moe_forward_timed, which
+records CUDA events between its stages on the launching stream) is captured
+as a CUDA graph and replayed once per step; each step's time is the span of
+those events.  The L2 cache is flushed (a 512 MiB buffer is written) before
+every step, outside the events.  `e2e` repeats the measurement through plain
+moe_forward calls with the input copied in from pinned host memory and the
+output and losses copied back, every step.  With N > 1 (torchrun) every rank runs
 its own batch on its own GPU (weak scaling, no collective on the data path);
 the reported time is the maximum over ranks.
 
@@ -44,6 +47,27 @@ GEMM_KERNEL_SRC = os.path.join(ROOT, "sparse_mixture_experts_10_b200", "csrc", "
 NCU_TRAFFIC = {
     # "gpt2/up": {"bytes": ..., "src_sha256": "..."},
 }
+
+
+def rank_seed(wl, rank: int) -> int:
+    """Each rank draws its own batch (weak scaling: the per-GPU work is fixed)."""
+    return wl.seed + 7919 * rank
+
+
+def max_over_ranks(value_ms: float, device, world: int) -> float:
+    """The job's time is the slowest rank's (all ranks take the same collective steps)."""
+    if world == 1:
+        return value_ms
+    import torch.distributed as dist
+
+    t = torch.tensor([value_ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(tokens_per_rank: int, world: int, steps: int, max_total_ms: float) -> float:
+    """Whole-job tokens/s: the tokens every rank processed over the slowest rank's time."""
+    return tokens_per_rank * world * steps / (max_total_ms / 1e3)
 
 
 def parse():
@@ -220,7 +244,7 @@ def main():
     moe.load_library()
 
     T = wl.T
-    inp = make_inputs(wl, dev, seed=wl.seed + 7919 * rank)
+    inp = make_inputs(wl, dev, seed=rank_seed(wl, rank))
     cfg = moe.make_config(wl.D, wl.H, wl.N, wl.K, wl.act, moe.dtype_code(wl.dtype), wl.has_bias)
     W = moe.make_weights(inp["W_g"], inp["W1"], inp["W2"], inp["b_g"], inp["b1"], inp["b2"])
     ws = moe.alloc_workspace(cfg, T)
@@ -233,9 +257,9 @@ def main():
     stream = torch.cuda.current_stream(dev)
     NS = moe.MOE_N_STAGES
 
-    def step(evs):
-        moe.check(moe.moe_forward_timed(cfg, inp["x"], T, W, y, moe.MOE_F32, aux, ws, ws.numel(), stream, evs),
-                  "forward")
+    def step(evs, strm=None):
+        moe.check(moe.moe_forward_timed(cfg, inp["x"], T, W, y, moe.MOE_F32, aux, ws, ws.numel(),
+                                        strm or torch.cuda.current_stream(dev), evs), "forward")
 
     warm = [torch.cuda.Event(enable_timing=True) for _ in range(NS + 1)]
     for _ in range(max(args.warmup, 3)):
@@ -247,34 +271,47 @@ def main():
         raise RuntimeError(f"device status {st} after warm-up")
     counts = aux_t["counts"].cpu().numpy()
 
-    events = [[torch.cuda.Event(enable_timing=True) for _ in range(NS + 1)] for _ in range(args.steps)]
+    # One layer call captured as a CUDA graph (its stage events included) and
+    # replayed once per step, so host-side enqueue cost stays out of the step.
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(NS + 1)]
+    for e in evs:
+        e.record()
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    l0 = moe.moe_launch_count()
+    with torch.cuda.graph(graph):
+        step(evs)
+    launches_per_step = moe.moe_launch_count() - l0
+    for _ in range(2):
+        flush.zero_()
+        graph.replay()
+    torch.cuda.synchronize()
+
     sampler = ClockSampler(local)
     sampler.start()
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    launches0 = moe.moe_launch_count()
+    rows = []
     for i in range(args.steps):
         flush.zero_()
-        step(events[i])
-    torch.cuda.synchronize()
-    launches = moe.moe_launch_count() - launches0
+        graph.replay()
+        torch.cuda.synchronize()
+        rows.append([evs[s_].elapsed_time(evs[s_ + 1]) for s_ in range(NS)])
+    launches = launches_per_step * args.steps
     if world > 1:
         dist.barrier()
     clocks = sampler.stop()
     st = moe.moe_get_device_status()
     if st != 0:
         raise RuntimeError(f"device status {st} after timed steps")
+    del graph
 
-    stage_ms = np.array([[events[i][s].elapsed_time(events[i][s + 1]) for s in range(NS)] for i in range(args.steps)])
+    stage_ms = np.array(rows)
     step_ms = stage_ms.sum(axis=1)
-    total_ms = float(step_ms.sum())
-    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    total_ms = float(t.item())
+    total_ms = max_over_ranks(float(step_ms.sum()), dev, world)
     ms_per_step = total_ms / args.steps
-    tokens_per_s = T * world * args.steps / (total_ms / 1e3)
+    tokens_per_s = job_throughput(T, world, args.steps, total_ms)
 
     # ---- end to end through host buffers: pinned x in, y and the statistics out, every step
     x_host = inp["x"].cpu().pin_memory()
@@ -293,11 +330,8 @@ def main():
         if i >= max(args.warmup, 3):
             e2e_ev[i - max(args.warmup, 3)][1].record(stream)
     torch.cuda.synchronize()
-    e2e_ms = sum(a.elapsed_time(b) for a, b in e2e_ev)
-    t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    e2e_tps = T * world * args.steps / (float(t.item()) / 1e3)
+    e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in e2e_ev), dev, world)
+    e2e_tps = job_throughput(T, world, args.steps, e2e_ms)
     es = x_host.element_size()
     h2d = T * wl.D * es
     d2h = T * wl.D * 4 + 16

@@ -29,6 +29,7 @@ std::atomic<int64_t> g_launches{0};
 constexpr uint64_t kTimeoutNs = 1000000000ull;  // bounded waits give up after 1 s
 constexpr int kMaxDevices = 64;
 constexpr size_t kSmallRouterSmemMax = 200 * 1024;
+constexpr int64_t kRowdotMaxT = 2048;  // below this the chunked router has too few blocks
 
 struct DeviceInfo {
     int sms = 0;
@@ -43,14 +44,15 @@ int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
 struct Plan {
     int64_t T;
     int D, H, N, K, act, dtype, has_bias, es;
-    bool small_router;
+    bool small_router;   // chunked fused router (W_g staged in shared memory)
+    bool rowdot_router;  // one block per token (few tokens, N <= 32)
     int np;       // padded expert count of the fused router (8, 16, 32)
     int vpl;      // values per lane of the top-k kernel
     int n_chunks;
     int aux_blocks;
     int64_t rows_cap;
-    size_t logits, idx, w, counts, offsets, row_offsets, chunk_counts, chunk_base, perm_slot, slot_row, x_perm, h, z,
-        wgt, aux_p, aux_i, aux_c, total;
+    size_t counters, logits, idx, w, counts, offsets, row_offsets, chunk_counts, chunk_base, perm_slot, slot_row,
+        x_perm, h, z, wgt, aux_p, aux_i, aux_c, total;
 };
 
 int make_plan(const moe_config *c, int64_t T, Plan *p) {
@@ -72,7 +74,9 @@ int make_plan(const moe_config *c, int64_t T, Plan *p) {
     p->D = (int)D; p->H = (int)H; p->N = (int)N; p->K = (int)K;
     p->act = c->act; p->dtype = c->dtype; p->has_bias = c->has_bias ? 1 : 0; p->es = es;
     p->np = N <= 8 ? 8 : N <= 16 ? 16 : 32;
-    p->small_router = N <= 32 && (size_t)p->np * D * es + 256 <= kSmallRouterSmemMax;
+    const bool fits = N <= 32 && (size_t)p->np * D * es + 256 <= kSmallRouterSmemMax;
+    p->rowdot_router = N <= 32 && (T < kRowdotMaxT || !fits);
+    p->small_router = fits && !p->rowdot_router;
     const int need = (int)cdiv(N, 32);
     p->vpl = need <= 1 ? 1 : need <= 2 ? 2 : need <= 4 ? 4 : need <= 8 ? 8 : need <= 16 ? 16 : 32;
     p->n_chunks = (int)cdiv(T, kChunk);
@@ -85,6 +89,7 @@ int make_plan(const moe_config *c, int64_t T, Plan *p) {
         off = align256(off + bytes);
         return o;
     };
+    p->counters = take(256);
     p->logits = take((size_t)T * N * 4);
     p->idx = take((size_t)T * K * 4);
     p->w = take((size_t)T * K * 4);
@@ -98,7 +103,7 @@ int make_plan(const moe_config *c, int64_t T, Plan *p) {
     p->x_perm = take((size_t)p->rows_cap * D * es);
     p->h = take((size_t)p->rows_cap * H * es);
     p->z = take((size_t)T * K * D * 4);
-    p->wgt = take(p->small_router ? 0 : (size_t)N * D * es);
+    p->wgt = take(N <= 32 ? 0 : (size_t)N * D * es);
     p->aux_p = take((size_t)p->aux_blocks * N * 4);
     p->aux_i = take((size_t)p->aux_blocks * N * 4);
     p->aux_c = take((size_t)p->aux_blocks * N * 4);
@@ -122,13 +127,16 @@ int device_info(DeviceInfo **out) {
         cudaFuncSetAttribute(tc::grouped_gemm_tc_kernel<256, tc::EPI_SWIGLU>, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
         cudaFuncSetAttribute(tc::grouped_gemm_tc_kernel<256, tc::EPI_SCATTER>, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
         cudaFuncSetAttribute(tc::grouped_gemm_tc_kernel<256, tc::EPI_LOGITS>, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
+        cudaFuncSetAttribute(tc::grouped_gemm_tc_kernel<128, tc::EPI_GELU>, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
+        cudaFuncSetAttribute(tc::grouped_gemm_tc_kernel<128, tc::EPI_SWIGLU>, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
+        cudaFuncSetAttribute(tc::grouped_gemm_tc_kernel<128, tc::EPI_SCATTER>, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
         cudaFuncSetAttribute(router_small_kernel<float, 8>, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
         cudaFuncSetAttribute(router_small_kernel<float, 16>, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
         cudaFuncSetAttribute(router_small_kernel<float, 32>, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
         cudaFuncSetAttribute(router_small_kernel<__nv_bfloat16, 8>, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
         cudaFuncSetAttribute(router_small_kernel<__nv_bfloat16, 16>, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
         cudaFuncSetAttribute(router_small_kernel<__nv_bfloat16, 32>, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
-        cudaFuncSetAttribute(aux_partial_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
+        cudaFuncSetAttribute(aux_partial_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 160 * 1024);
         if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
         d.attrs = true;
     }
@@ -208,6 +216,18 @@ int stage_route(const Plan &P, const Bufs &b, const void *x, const moe_weights *
                 float *tw, const DeviceInfo &dev, cudaStream_t s) {
     const int T = (int)P.T, D = P.D, N = P.N, K = P.K;
     int *cc = b.at<int>(P.chunk_counts);
+    if (P.rowdot_router) {
+        if (cudaMemsetAsync(cc, 0, (size_t)P.n_chunks * N * 4, s) != cudaSuccess) return MOE_ERR_CUDA;
+        if (P.dtype == MOE_F32)
+            router_rowdot_kernel<float><<<T, 1024, 0, s>>>(static_cast<const float *>(x), T, D, N, K,
+                                                           static_cast<const float *>(w->W_g), w->b_g, logits, idx,
+                                                           tw, cc);
+        else
+            router_rowdot_kernel<__nv_bfloat16><<<T, 1024, 0, s>>>(static_cast<const __nv_bfloat16 *>(x), T, D, N, K,
+                                                                   static_cast<const __nv_bfloat16 *>(w->W_g), w->b_g,
+                                                                   logits, idx, tw, cc);
+        return check_launch();
+    }
     if (P.small_router) {
         const size_t smem = (size_t)P.np * D * P.es + (size_t)P.np * 4;
 #define MOE_ROUTER(TIN, NP)                                                                                     \
@@ -283,10 +303,9 @@ int stage_route(const Plan &P, const Bufs &b, const void *x, const moe_weights *
 }
 
 int stage_scan(const Plan &P, const Bufs &b, int *counts_out, cudaStream_t s) {
-    const size_t smem = (size_t)(2 * P.N + 1) * 4;
-    scan_kernel<<<1, 1024, smem, s>>>(b.at<int>(P.chunk_counts), P.n_chunks, P.N, P.T * P.K, b.at<int>(P.chunk_base),
-                                      b.at<int>(P.counts), b.at<int>(P.offsets), b.at<int>(P.row_offsets),
-                                      b.at<int>(P.perm_slot), counts_out);
+    scan_kernel<<<(unsigned)cdiv(P.N, 32), 1024, 0, s>>>(
+        b.at<int>(P.chunk_counts), P.n_chunks, P.N, P.T * P.K, b.at<int>(P.chunk_base), b.at<int>(P.counts),
+        b.at<int>(P.offsets), b.at<int>(P.row_offsets), b.at<int>(P.perm_slot), counts_out, b.at<unsigned>(P.counters));
     return check_launch();
 }
 
@@ -304,17 +323,27 @@ int stage_permute(const Plan &P, const Bufs &b, const void *x, cudaStream_t s) {
     return check_launch();
 }
 
+// True when the grouped GEMM would have too few 256-wide tiles to fill the
+// GPU: the row tiles are estimated from the routed rows (at least T*K/128),
+// since the per-expert counts live on the device.
+bool narrow_tiles(const Plan &P, int64_t n_tiles_256, const DeviceInfo &dev) {
+    const int64_t m_tiles_min = std::max<int64_t>(1, cdiv(P.T * P.K, tc::BM));
+    return m_tiles_min * n_tiles_256 < 2 * (int64_t)dev.sms;
+}
+
 int stage_up(const Plan &P, const Bufs &b, const moe_weights *w, const DeviceInfo &dev, cudaStream_t s) {
     const int D = P.D, H = P.H, N = P.N;
     const bool swiglu = P.act == MOE_ACT_SWIGLU;
     if (P.dtype == MOE_BF16) {
+        const int bn = narrow_tiles(P, swiglu ? cdiv(H, 128) : cdiv(H, 256), dev) ? 128 : 256;
+        const int out_cols = swiglu ? bn / 2 : bn;  // h columns per tile
         CUtensorMap ma, mb;
         MOE_TRY(make_map(&ma, b.ws + P.x_perm, P.rows_cap, D, tc::BM));
-        MOE_TRY(make_map(&mb, w->W1, (int64_t)N * (swiglu ? 2 * H : H), D, swiglu ? 128 : 256));
+        MOE_TRY(make_map(&mb, w->W1, (int64_t)N * (swiglu ? 2 * H : H), D, swiglu ? bn / 2 : bn));
         tc::Params p{};
         p.num_groups = N;
         p.row_offsets = b.at<int>(P.row_offsets);
-        p.n_tiles = (int)cdiv(H, swiglu ? 128 : 256);
+        p.n_tiles = (int)cdiv(H, out_cols);
         p.num_k_blocks = (int)cdiv(D, tc::BK);
         p.b_group_rows = swiglu ? 2 * H : H;
         p.b_up_offset = H;
@@ -324,6 +353,10 @@ int stage_up(const Plan &P, const Bufs &b, const moe_weights *w, const DeviceInf
         p.bias = swiglu ? nullptr : w->b1;
         p.timeout_ns = kTimeoutNs;
         const int64_t upper = (P.rows_cap / tc::BM) * p.n_tiles;
+        if (bn == 128) {
+            if (swiglu) return launch_tc<128, tc::EPI_SWIGLU>(ma, mb, p, upper, dev.sms, s);
+            return launch_tc<128, tc::EPI_GELU>(ma, mb, p, upper, dev.sms, s);
+        }
         if (swiglu) return launch_tc<256, tc::EPI_SWIGLU>(ma, mb, p, upper, dev.sms, s);
         return launch_tc<256, tc::EPI_GELU>(ma, mb, p, upper, dev.sms, s);
     }
@@ -349,13 +382,14 @@ int stage_down(const Plan &P, const Bufs &b, const moe_weights *w, const DeviceI
     const int D = P.D, H = P.H, N = P.N;
     const float *bias = P.act == MOE_ACT_SWIGLU ? nullptr : w->b2;
     if (P.dtype == MOE_BF16) {
+        const int bn = narrow_tiles(P, cdiv(D, 256), dev) ? 128 : 256;
         CUtensorMap ma, mb;
         MOE_TRY(make_map(&ma, b.ws + P.h, P.rows_cap, H, tc::BM));
-        MOE_TRY(make_map(&mb, w->W2, (int64_t)N * D, H, 256));
+        MOE_TRY(make_map(&mb, w->W2, (int64_t)N * D, H, bn));
         tc::Params p{};
         p.num_groups = N;
         p.row_offsets = b.at<int>(P.row_offsets);
-        p.n_tiles = (int)cdiv(D, 256);
+        p.n_tiles = (int)cdiv(D, bn);
         p.num_k_blocks = (int)cdiv(H, tc::BK);
         p.b_group_rows = D;
         p.n_valid = D;
@@ -365,7 +399,9 @@ int stage_down(const Plan &P, const Bufs &b, const moe_weights *w, const DeviceI
         p.perm_slot = b.at<int>(P.perm_slot);
         p.gate_w = b.at<float>(P.w);
         p.timeout_ns = kTimeoutNs;
-        return launch_tc<256, tc::EPI_SCATTER>(ma, mb, p, (P.rows_cap / tc::BM) * p.n_tiles, dev.sms, s);
+        const int64_t upper = (P.rows_cap / tc::BM) * p.n_tiles;
+        if (bn == 128) return launch_tc<128, tc::EPI_SCATTER>(ma, mb, p, upper, dev.sms, s);
+        return launch_tc<256, tc::EPI_SCATTER>(ma, mb, p, upper, dev.sms, s);
     }
     simt::Params p{};
     p.A = b.at<float>(P.h);
@@ -399,13 +435,27 @@ int stage_combine(const Plan &P, const Bufs &b, void *y, int y_dtype, const Devi
 int stage_aux(const Plan &P, const Bufs &b, const float *logits, const int *idx, const float *tw, moe_aux *aux,
               cudaStream_t s) {
     const int N = P.N;
-    aux_partial_kernel<<<P.aux_blocks, 256, (size_t)24 * N * 4, s>>>(
-        logits, idx, tw, (int)P.T, N, P.K, b.at<float>(P.aux_p), b.at<float>(P.aux_i), b.at<int>(P.aux_c));
-    MOE_TRY(check_launch());
-    aux_finalize_kernel<<<1, 1024, (size_t)3 * N * 8, s>>>(b.at<float>(P.aux_p), b.at<float>(P.aux_i),
-                                                           b.at<int>(P.aux_c), P.aux_blocks, (int)P.T, N, P.K,
-                                                           aux->counts, aux->importance, aux->p_mean, aux->scalars);
+    AuxOut out{aux->counts, aux->importance, aux->p_mean, aux->scalars};
+    unsigned *counter = b.at<unsigned>(P.counters) + 1;
+    if (N <= 32) {
+        const unsigned grid = (unsigned)cdiv(P.T, 256);
+#define MOE_AUX(NP)                                                                                        \
+    aux_small_kernel<NP><<<grid, 256, 0, s>>>(logits, idx, tw, (int)P.T, N, P.K, b.at<float>(P.aux_p),     \
+                                              b.at<float>(P.aux_i), b.at<int>(P.aux_c), counter, out)
+        if (N <= 8) MOE_AUX(8);
+        else if (N <= 16) MOE_AUX(16);
+        else MOE_AUX(32);
+#undef MOE_AUX
+        return check_launch();
+    }
+    aux_partial_kernel<<<P.aux_blocks, 256, (size_t)24 * N * 4, s>>>(logits, idx, tw, (int)P.T, N, P.K,
+                                                                     b.at<float>(P.aux_p), b.at<float>(P.aux_i),
+                                                                     b.at<int>(P.aux_c), counter, out);
     return check_launch();
+}
+
+int zero_counters(const Plan &P, const Bufs &b, cudaStream_t s) {
+    return cudaMemsetAsync(b.ws + P.counters, 0, 256, s) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
 int zero_aux(const Plan &P, moe_aux *aux, cudaStream_t s) {
@@ -435,9 +485,18 @@ int forward_impl(const moe_config *cfg, const void *x, int64_t T, const moe_weig
     if (T > 0 && (!x || !y || !aligned16(x) || !aligned16(y))) return MOE_ERR_INVALID_ARG;
     if (T > 0 && (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u))) return MOE_ERR_INVALID_ARG;
     if (T > 0 && ws_bytes < P.total) return MOE_ERR_WORKSPACE_TOO_SMALL;
+    // Under stream capture the events become external event-record nodes, so
+    // that a replayed graph records them (and they can be timed).
+    unsigned rec_flags = cudaEventRecordDefault;
+    if (ev) {
+        cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+        if (cudaStreamIsCapturing(s, &cs) != cudaSuccess) return MOE_ERR_CUDA;
+        if (cs == cudaStreamCaptureStatusActive) rec_flags = cudaEventRecordExternal;
+    }
     auto rec = [&](int i) -> int {
         if (!ev) return MOE_OK;
-        return cudaEventRecord(static_cast<cudaEvent_t>(ev[i]), s) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+        return cudaEventRecordWithFlags(static_cast<cudaEvent_t>(ev[i]), s, rec_flags) == cudaSuccess ? MOE_OK
+                                                                                                      : MOE_ERR_CUDA;
     };
     if (T == 0) {
         for (int i = 0; i <= MOE_N_STAGES; ++i) MOE_TRY(rec(i));
@@ -450,6 +509,7 @@ int forward_impl(const moe_config *cfg, const void *x, int64_t T, const moe_weig
     int *idx = b.at<int>(P.idx);
     float *tw = b.at<float>(P.w);
     MOE_TRY(rec(0));
+    MOE_TRY(zero_counters(P, b, s));
     MOE_TRY(stage_route(P, b, x, w, logits, idx, tw, *dev, s));
     MOE_TRY(rec(1));
     MOE_TRY(stage_scan(P, b, nullptr, s));
@@ -516,6 +576,7 @@ int moe_route(const moe_config *cfg, const void *x, int64_t T, const moe_weights
     MOE_TRY(device_info(&dev));
     Bufs b{static_cast<char *>(ws), &P};
     float *lg = logits ? logits : b.at<float>(P.logits);
+    MOE_TRY(zero_counters(P, b, s));
     MOE_TRY(stage_route(P, b, x, w, lg, topk_idx, topk_w, *dev, s));
     if (counts) MOE_TRY(stage_scan(P, b, counts, s));
     return MOE_OK;
@@ -546,6 +607,7 @@ int moe_aux_stats(const moe_config *cfg, int64_t T, const float *logits, const i
     DeviceInfo *dev = nullptr;
     MOE_TRY(device_info(&dev));
     Bufs b{static_cast<char *>(ws), &P};
+    MOE_TRY(zero_counters(P, b, s));
     return stage_aux(P, b, logits, topk_idx, topk_w, out, s);
 }
 

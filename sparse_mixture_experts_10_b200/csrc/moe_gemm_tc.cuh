@@ -68,7 +68,7 @@ struct Params {
 
 template <int BN>
 struct Shape {
-    static constexpr int kStages = 4;
+    static constexpr int kStages = BN == 256 ? 4 : 6;   // 192 KB of ring either way
     static constexpr uint32_t kABytes = BM * BK * 2;
     static constexpr uint32_t kBBytes = BN * BK * 2;
     static constexpr uint32_t kTmemCols = 2 * BN;
@@ -106,7 +106,21 @@ __device__ __forceinline__ TileCoord decode_tile(int i, const int *s_rowoff, int
     return c;
 }
 
-__device__ __forceinline__ float gelu_erf(float v) { return 0.5f * v * (1.0f + erff(v * 0.70710678118654752f)); }
+// GELU(v) = v Phi(v) = 0.5 v (1 + erf(v / sqrt 2)), exact-erf form, with erfc
+// from Abramowitz & Stegun, Handbook of Mathematical Functions, formula 7.1.26
+// (absolute error of erf at most 1.5e-7, far below the bf16 rounding of h):
+//   erfc(z) ~ (a1 t + a2 t^2 + a3 t^3 + a4 t^4 + a5 t^5) exp(-z^2), t = 1 / (1 + p z), z >= 0.
+// For v < 0, 1 + erf(v / sqrt 2) = erfc(|v| / sqrt 2) is used directly (no cancellation).
+__device__ __forceinline__ float gelu_erf(float v) {
+    const float z = fabsf(v) * 0.70710678118654752f;
+    const float t = __fdividef(1.0f, fmaf(0.3275911f, z, 1.0f));
+    float poly = fmaf(t, 1.061405429f, -1.453152027f);
+    poly = fmaf(t, poly, 1.421413741f);
+    poly = fmaf(t, poly, -0.284496736f);
+    poly = fmaf(t, poly, 0.254829592f);
+    const float q = poly * t * __expf(-z * z);
+    return 0.5f * v * (v >= 0.f ? 2.0f - q : q);
+}
 __device__ __forceinline__ float silu_f(float g) { return g / (1.0f + __expf(-g)); }
 
 template <int BN, int EPI>
@@ -279,8 +293,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                         for (int v = 0; v < 4; ++v)
                             reinterpret_cast<uint4 *>(dst)[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
                     } else {
-                        for (int k = 0; k < 32 && n0 + k < p.n_valid; ++k)
-                            dst[k] = __ushort_as_bfloat16(static_cast<unsigned short>((pk[k >> 1] >> ((k & 1) * 16)) & 0xffffu));
+#pragma unroll
+                        for (int k = 0; k < 32; ++k)
+                            if (n0 + k < p.n_valid)
+                                dst[k] = __ushort_as_bfloat16(static_cast<unsigned short>((pk[k >> 1] >> ((k & 1) * 16)) & 0xffffu));
                     }
                 }
             } else {
@@ -301,12 +317,21 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (n0 >= p.n_valid) continue;
                     const bool full_chunk = n0 + 32 <= p.n_valid;
                     float v[32];
-                    const float *bias = p.bias ? p.bias + (int64_t)c.g * p.n_valid + n0 : nullptr;
 #pragma unroll
-                    for (int k = 0; k < 32; ++k) {
-                        float b = 0.f;
-                        if (bias && (full_chunk || n0 + k < p.n_valid)) b = __ldg(bias + k);
-                        v[k] = __uint_as_float(r[k]) + b;
+                    for (int k = 0; k < 32; ++k) v[k] = __uint_as_float(r[k]);
+                    if (p.bias) {
+                        const float *bias = p.bias + (int64_t)c.g * p.n_valid + n0;
+                        if (full_chunk) {
+#pragma unroll
+                            for (int u = 0; u < 8; ++u) {
+                                const float4 b4 = __ldg(reinterpret_cast<const float4 *>(bias) + u);
+                                v[4 * u] += b4.x; v[4 * u + 1] += b4.y; v[4 * u + 2] += b4.z; v[4 * u + 3] += b4.w;
+                            }
+                        } else {
+#pragma unroll
+                            for (int k = 0; k < 32; ++k)
+                                if (n0 + k < p.n_valid) v[k] += __ldg(bias + k);
+                        }
                     }
                     if (EPI == EPI_GELU) {
                         __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(p.out) + (int64_t)row * p.ldo + n0;
@@ -318,8 +343,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                             for (int u = 0; u < 4; ++u)
                                 reinterpret_cast<uint4 *>(dst)[u] = make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
                         } else {
-                            for (int k = 0; n0 + k < p.n_valid; ++k)
-                                dst[k] = __ushort_as_bfloat16(static_cast<unsigned short>((pk[k >> 1] >> ((k & 1) * 16)) & 0xffffu));
+#pragma unroll
+                            for (int k = 0; k < 32; ++k)
+                                if (n0 + k < p.n_valid)
+                                    dst[k] = __ushort_as_bfloat16(static_cast<unsigned short>((pk[k >> 1] >> ((k & 1) * 16)) & 0xffffu));
                         }
                     } else if (EPI == EPI_SCATTER) {
                         if (slot >= 0) {
@@ -330,13 +357,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                                     reinterpret_cast<float4 *>(dst)[u] =
                                         make_float4(gw * v[4 * u], gw * v[4 * u + 1], gw * v[4 * u + 2], gw * v[4 * u + 3]);
                             } else {
-                                for (int k = 0; n0 + k < p.n_valid; ++k) dst[k] = gw * v[k];
+#pragma unroll
+                                for (int k = 0; k < 32; ++k)
+                                    if (n0 + k < p.n_valid) dst[k] = gw * v[k];
                             }
                         }
                     } else {  // EPI_LOGITS
                         if (row < p.dense_rows) {
                             float *dst = static_cast<float *>(p.out) + (int64_t)row * p.ldo + n0;
-                            for (int k = 0; k < 32 && n0 + k < p.n_valid; ++k) dst[k] = v[k];
+#pragma unroll
+                            for (int k = 0; k < 32; ++k)
+                                if (n0 + k < p.n_valid) dst[k] = v[k];
                         }
                     }
                 }

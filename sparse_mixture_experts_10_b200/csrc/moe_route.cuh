@@ -64,22 +64,26 @@ struct Vec16;  // 16 bytes of T widened to float
 template <>
 struct Vec16<float> {
     static constexpr int n = 4;
+    __device__ __forceinline__ static void unpack(const uint4 v, float (&f)[8]) {
+        f[0] = __uint_as_float(v.x); f[1] = __uint_as_float(v.y); f[2] = __uint_as_float(v.z); f[3] = __uint_as_float(v.w);
+    }
     __device__ __forceinline__ static void load(const float *p, float (&f)[8]) {
-        const float4 v = *reinterpret_cast<const float4 *>(p);
-        f[0] = v.x; f[1] = v.y; f[2] = v.z; f[3] = v.w;
+        unpack(*reinterpret_cast<const uint4 *>(p), f);
     }
 };
 template <>
 struct Vec16<__nv_bfloat16> {
     static constexpr int n = 8;
-    __device__ __forceinline__ static void load(const __nv_bfloat16 *p, float (&f)[8]) {
-        const uint4 v = *reinterpret_cast<const uint4 *>(p);
+    __device__ __forceinline__ static void unpack(const uint4 v, float (&f)[8]) {
         const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             f[2 * i] = __uint_as_float(w[i] << 16);
             f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
         }
+    }
+    __device__ __forceinline__ static void load(const __nv_bfloat16 *p, float (&f)[8]) {
+        unpack(*reinterpret_cast<const uint4 *>(p), f);
     }
 };
 
@@ -129,16 +133,17 @@ __global__ void __launch_bounds__(256) router_small_kernel(const Tin *__restrict
                                                            float *__restrict__ topk_w, int *__restrict__ chunk_counts) {
     constexpr int TPW = 32 / NP;
     constexpr int VEC = Vec16<Tin>::n;
+    constexpr int U = 4;  // 16-byte vectors in flight per token and lane
     extern __shared__ __align__(16) unsigned char smem_raw[];
     Tin *WgT = reinterpret_cast<Tin *>(smem_raw);
     int *hist = reinterpret_cast<int *>(smem_raw + (size_t)NP * D * sizeof(Tin));
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    for (int i = tid; i < D * N; i += blockDim.x) {
-        const int d = i / N, e = i - d * N;
-        WgT[(size_t)e * D + d] = Wg[i];
+    // one router row d per thread: contiguous global reads, consecutive shared addresses per expert row
+    for (int d = tid; d < D; d += blockDim.x) {
+#pragma unroll
+        for (int e = 0; e < NP; ++e) WgT[(size_t)e * D + d] = e < N ? Wg[(size_t)d * N + e] : Tin(0.f);
     }
-    for (int i = tid; i < (NP - N) * D; i += blockDim.x) WgT[(size_t)N * D + i] = Tin(0.f);
     if (tid < NP) hist[tid] = 0;
     __syncthreads();
 
@@ -150,25 +155,33 @@ __global__ void __launch_bounds__(256) router_small_kernel(const Tin *__restrict
         float a[32];
 #pragma unroll
         for (int i = 0; i < 32; ++i) a[i] = 0.f;
-        for (int v = lane; v < nvec; v += 32) {
-            float xf[TPW][8];
+        for (int v0 = lane; v0 < nvec; v0 += 32 * U) {
+            uint4 xr[TPW][U];
 #pragma unroll
-            for (int tt = 0; tt < TPW; ++tt) {
-                if (t0 + tt < T) {
-                    Vec16<Tin>::load(x + (size_t)(t0 + tt) * D + (size_t)v * VEC, xf[tt]);
-                } else {
+            for (int tt = 0; tt < TPW; ++tt)
 #pragma unroll
-                    for (int u = 0; u < 8; ++u) xf[tt][u] = 0.f;
+                for (int u = 0; u < U; ++u) {
+                    const int v = v0 + 32 * u;
+                    xr[tt][u] = (t0 + tt < T && v < nvec)
+                                    ? __ldg(reinterpret_cast<const uint4 *>(x + (size_t)(t0 + tt) * D) + v)
+                                    : make_uint4(0u, 0u, 0u, 0u);
                 }
-            }
 #pragma unroll
-            for (int e = 0; e < NP; ++e) {
-                float wf[8];
-                Vec16<Tin>::load(WgT + (size_t)e * D + (size_t)v * VEC, wf);
+            for (int u = 0; u < U; ++u) {
+                const int v = v0 + 32 * u;
+                if (v >= nvec) break;
+                float xf[TPW][8];
 #pragma unroll
-                for (int tt = 0; tt < TPW; ++tt)
+                for (int tt = 0; tt < TPW; ++tt) Vec16<Tin>::unpack(xr[tt][u], xf[tt]);
 #pragma unroll
-                    for (int u = 0; u < VEC; ++u) a[tt * NP + e] = fmaf(xf[tt][u], wf[u], a[tt * NP + e]);
+                for (int e = 0; e < NP; ++e) {
+                    float wf[8];
+                    Vec16<Tin>::load(WgT + (size_t)e * D + (size_t)v * VEC, wf);
+#pragma unroll
+                    for (int tt = 0; tt < TPW; ++tt)
+#pragma unroll
+                        for (int q = 0; q < VEC; ++q) a[tt * NP + e] = fmaf(xf[tt][q], wf[q], a[tt * NP + e]);
+                }
             }
         }
         reduce_scatter32(a, lane);
@@ -193,6 +206,62 @@ __global__ void __launch_bounds__(256) router_small_kernel(const Tin *__restrict
     }
     __syncthreads();
     if (tid < N) chunk_counts[(size_t)blockIdx.x * N + tid] = hist[tid];
+}
+
+// ---------------------------------------------------------------------------
+// Router for few tokens (N <= 32): one block per token, lane = expert, each of
+// the 32 warps accumulates a strided share of the D rows of W_g (one coalesced
+// row read per step, no staging), the warps' partial sums are added in warp
+// order, then warp 0 selects the top k.  Chunk histograms are built with
+// integer atomics on a zeroed array (order-independent).
+// ---------------------------------------------------------------------------
+template <typename Tin>
+__global__ void __launch_bounds__(1024) router_rowdot_kernel(const Tin *__restrict__ x, int T, int D, int N, int K,
+                                                             const Tin *__restrict__ Wg, const float *__restrict__ bg,
+                                                             float *__restrict__ logits, int *__restrict__ topk_idx,
+                                                             float *__restrict__ topk_w, int *__restrict__ chunk_counts) {
+    __shared__ float part[32][33];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int t = blockIdx.x;
+    const Tin *xt = x + (size_t)t * D;
+    // warp w takes rows w, w+32, ...; eight rows' loads are issued before their FMAs
+    constexpr int R = 8;
+    float acc[R];
+#pragma unroll
+    for (int r = 0; r < R; ++r) acc[r] = 0.f;
+    const bool live = lane < N;
+    for (int d0 = warp; d0 < D; d0 += 32 * R) {
+        float xv[R], wv[R];
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+            const int d = d0 + 32 * r;
+            xv[r] = d < D ? to_f32(__ldg(xt + d)) : 0.f;
+            wv[r] = (d < D && live) ? to_f32(__ldg(Wg + (size_t)d * N + lane)) : 0.f;
+        }
+#pragma unroll
+        for (int r = 0; r < R; ++r) acc[r] = fmaf(xv[r], wv[r], acc[r]);
+    }
+    float tot = 0.f;
+#pragma unroll
+    for (int r = 0; r < R; ++r) tot += acc[r];
+    part[warp][lane] = tot;
+    __syncthreads();
+    if (warp != 0) return;
+    float s = 0.f;
+    for (int w = 0; w < 32; ++w) s += part[w][lane];
+    if (live && bg) s += bg[lane];
+    if (logits && live) logits[(size_t)t * N + lane] = s;
+    if (s != s) {
+        if (live) set_status(kStatusNanLogit);
+        s = -INFINITY;
+    }
+    int slot_e;
+    float slot_w;
+    if (segment_topk<32>(s, lane, !live, K, lane, lane, slot_e, slot_w)) {
+        topk_idx[(size_t)t * K + lane] = slot_e;
+        topk_w[(size_t)t * K + lane] = slot_w;
+        atomicAdd(&chunk_counts[(size_t)(t / kChunk) * N + slot_e], 1);
+    }
 }
 
 // ---------------------------------------------------------------------------
@@ -264,41 +333,62 @@ __global__ void __launch_bounds__(256) topk_kernel(const float *__restrict__ log
 
 // ---------------------------------------------------------------------------
 // Scan: per expert, the exclusive prefix of the chunk histograms (chunk_base);
-// the per-expert counts, their exclusive scan (offsets) and the padded segment
-// starts (row_offsets, multiples of kRowAlign); padding rows get slot -1.
-// One block of 1024 threads.
+// then, in the last block to finish, the per-expert counts, their exclusive
+// scan (offsets) and the padded segment starts (row_offsets, multiples of
+// kRowAlign); padding rows get slot -1.  Grid: ceil(N/32) blocks of 32 warps,
+// warp w of block b owns expert 32b + w; each lane loads 16 consecutive chunk
+// counts at once.  *counter must be 0 at launch.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(1024) scan_kernel(const int *__restrict__ chunk_counts, int n_chunks, int N,
                                                     int64_t expect_total, int *__restrict__ chunk_base,
                                                     int *__restrict__ counts, int *__restrict__ offsets,
                                                     int *__restrict__ row_offsets, int *__restrict__ perm_slot,
-                                                    int *__restrict__ counts_out) {
-    extern __shared__ int s_scan[];
-    int *s_cnt = s_scan;           // [N]
-    int *s_row = s_scan + N;       // [N + 1]
+                                                    int *__restrict__ counts_out, unsigned *__restrict__ counter) {
+    constexpr int CPL = 16;
+    __shared__ int s_cnt[1024];
+    __shared__ int s_row[1025];
+    __shared__ bool s_last;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    for (int e = warp; e < N; e += 32) {
+    const int e = blockIdx.x * 32 + warp;
+    if (e < N) {
         int carry = 0;
-        for (int c0 = 0; c0 < n_chunks; c0 += 32) {
-            const int c = c0 + lane;
-            const int v = c < n_chunks ? chunk_counts[(size_t)c * N + e] : 0;
-            int incl = v;
+        for (int c0 = 0; c0 < n_chunks; c0 += 32 * CPL) {
+            const int cb = c0 + lane * CPL;
+            int v[CPL];
+#pragma unroll
+            for (int i = 0; i < CPL; ++i) v[i] = cb + i < n_chunks ? chunk_counts[(size_t)(cb + i) * N + e] : 0;
+            int run = 0;
+#pragma unroll
+            for (int i = 0; i < CPL; ++i) run += v[i];
+            int incl = run;
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
                 const int n = __shfl_up_sync(0xffffffffu, incl, o);
                 if (lane >= o) incl += n;
             }
-            if (c < n_chunks) chunk_base[(size_t)c * N + e] = carry + incl - v;
+            int base = carry + incl - run;
+#pragma unroll
+            for (int i = 0; i < CPL; ++i) {
+                if (cb + i < n_chunks) chunk_base[(size_t)(cb + i) * N + e] = base;
+                base += v[i];
+            }
             carry += __shfl_sync(0xffffffffu, incl, 31);
         }
-        if (lane == 0) s_cnt[e] = carry;
+        if (lane == 0) counts[e] = carry;
     }
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) s_last = atomicAdd(counter, 1u) == gridDim.x - 1;
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
+    for (int i = tid; i < N; i += blockDim.x) s_cnt[i] = __ldcg(counts + i);
     __syncthreads();
     if (warp == 0) {
         int carry = 0, pcarry = 0;
         for (int e0 = 0; e0 < N; e0 += 32) {
-            const int e = e0 + lane;
-            const int c = e < N ? s_cnt[e] : 0;
+            const int ee = e0 + lane;
+            const int c = ee < N ? s_cnt[ee] : 0;
             const int pc = (c + kRowAlign - 1) / kRowAlign * kRowAlign;
             int ic = c, ip = pc;
 #pragma unroll
@@ -307,12 +397,11 @@ __global__ void __launch_bounds__(1024) scan_kernel(const int *__restrict__ chun
                 const int n2 = __shfl_up_sync(0xffffffffu, ip, o);
                 if (lane >= o) { ic += n1; ip += n2; }
             }
-            if (e < N) {
-                counts[e] = c;
-                if (counts_out) counts_out[e] = c;
-                offsets[e] = carry + ic - c;
-                row_offsets[e] = pcarry + ip - pc;
-                s_row[e] = pcarry + ip - pc;
+            if (ee < N) {
+                if (counts_out) counts_out[ee] = c;
+                offsets[ee] = carry + ic - c;
+                row_offsets[ee] = pcarry + ip - pc;
+                s_row[ee] = pcarry + ip - pc;
             }
             carry += __shfl_sync(0xffffffffu, ic, 31);
             pcarry += __shfl_sync(0xffffffffu, ip, 31);
@@ -325,8 +414,8 @@ __global__ void __launch_bounds__(1024) scan_kernel(const int *__restrict__ chun
         }
     }
     __syncthreads();
-    for (int e = warp; e < N; e += 32) {
-        const int start = s_row[e] + s_cnt[e], end = s_row[e + 1];
+    for (int ee = warp; ee < N; ee += 32) {
+        const int start = s_row[ee] + s_cnt[ee], end = s_row[ee + 1];
         for (int r = start + lane; r < end; r += 32) perm_slot[r] = -1;
     }
 }
@@ -381,6 +470,7 @@ __global__ void __launch_bounds__(256) permute_kernel(const Tin *__restrict__ x,
         }
     }
     __syncthreads();
+    // one row per warp at a time, four 16-byte vectors in flight per lane
     constexpr int VEC = 16 / sizeof(Tin);
     const int nvec = D / VEC;
     for (int f = warp; f < n_entries; f += 8) {
@@ -389,7 +479,15 @@ __global__ void __launch_bounds__(256) permute_kernel(const Tin *__restrict__ x,
         const int64_t t = (f0 + f) / K;
         const uint4 *src = reinterpret_cast<const uint4 *>(x + t * D);
         uint4 *dst = reinterpret_cast<uint4 *>(x_perm + (int64_t)dest * D);
-        for (int v = lane; v < nvec; v += 32) dst[v] = src[v];
+        for (int v0 = lane; v0 < nvec; v0 += 128) {
+            uint4 r[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+                if (v0 + 32 * u < nvec) r[u] = __ldg(src + v0 + 32 * u);
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+                if (v0 + 32 * u < nvec) dst[v0 + 32 * u] = r[u];
+        }
     }
 }
 
@@ -423,16 +521,174 @@ __global__ void __launch_bounds__(256) combine_kernel(const float *__restrict__ 
 }
 
 // ---------------------------------------------------------------------------
-// Statistics, pass 1: per block of kAuxTokens tokens, the sums of the full
-// softmax of the scores, of the gate weights per expert, and the counts.
-// Each warp accumulates its tokens in order into its own shared row; the rows
-// are then added in warp order, so the result does not depend on scheduling.
+// Statistics.  Each block reduces a fixed range of tokens to partial sums per
+// expert (full-softmax probabilities, gate weights, counts) in a fixed order;
+// the last block to finish adds the partials block by block, also in a fixed
+// order, and computes the scalars in double precision:
+//   f_e = counts_e / (T K); switch = N sum f_e P_e; simple = N sum f_e^2;
+//   CV^2 = population variance / mean^2 (0 when the mean is 0).
+// No float atomics anywhere, so the results do not depend on scheduling.
 // ---------------------------------------------------------------------------
+struct AuxOut {
+    int *counts;
+    float *importance;
+    float *p_mean;
+    float *scalars;
+};
+
+__device__ void aux_finalize_block(const float *__restrict__ part_p, const float *__restrict__ part_imp,
+                                   const int *__restrict__ part_cnt, int nblk, int T, int N, int K, AuxOut out) {
+    __shared__ float f_p[1024], f_i[1024];
+    __shared__ int f_c[1024];
+    __shared__ float q_p[1024], q_i[1024];
+    __shared__ int q_c[1024];
+    const int nt = blockDim.x, tid = threadIdx.x;
+    int Q = 1;
+    while (Q * 2 * N <= nt && Q * 2 <= 32) Q *= 2;   // threads per expert
+    for (int e0 = 0; e0 < N; e0 += nt / Q) {
+        const int e = e0 + tid / Q, q = tid % Q;
+        float p = 0.f, im = 0.f;
+        int c = 0;
+        if (tid / Q < nt / Q && e < N) {
+#pragma unroll 4
+            for (int bb = q; bb < nblk; bb += Q) {
+                p += __ldcg(part_p + (size_t)bb * N + e);
+                im += __ldcg(part_imp + (size_t)bb * N + e);
+                c += __ldcg(part_cnt + (size_t)bb * N + e);
+            }
+        }
+        q_p[tid] = p;
+        q_i[tid] = im;
+        q_c[tid] = c;
+        __syncthreads();
+        if (q == 0 && tid / Q < nt / Q && e < N) {
+            float sp = 0.f, si = 0.f;
+            int sc = 0;
+            for (int j = 0; j < Q; ++j) { sp += q_p[tid + j]; si += q_i[tid + j]; sc += q_c[tid + j]; }
+            f_p[e] = T > 0 ? sp / (float)T : 0.f;
+            f_i[e] = si;
+            f_c[e] = sc;
+        }
+        __syncthreads();
+    }
+    for (int e = tid; e < N; e += nt) {
+        if (out.counts) out.counts[e] = f_c[e];
+        if (out.importance) out.importance[e] = f_i[e];
+        if (out.p_mean) out.p_mean[e] = f_p[e];
+    }
+    if (tid == 0 && out.scalars) {
+        double sw = 0.0, ss = 0.0, mi = 0.0, mc = 0.0;
+        const double tk = (double)T * (double)K;
+        for (int e = 0; e < N; ++e) {
+            const double f = tk > 0 ? f_c[e] / tk : 0.0;
+            sw += f * f_p[e];
+            ss += f * f;
+            mi += f_i[e];
+            mc += f_c[e];
+        }
+        mi /= N;
+        mc /= N;
+        double vi = 0.0, vc = 0.0;
+        for (int e = 0; e < N; ++e) {
+            vi += (f_i[e] - mi) * (f_i[e] - mi);
+            vc += (f_c[e] - mc) * (f_c[e] - mc);
+        }
+        vi /= N;
+        vc /= N;
+        out.scalars[0] = (float)(N * sw);
+        out.scalars[1] = (float)(N * ss);
+        out.scalars[2] = mi == 0.0 ? 0.f : (float)(vi / (mi * mi));
+        out.scalars[3] = mc == 0.0 ? 0.f : (float)(vc / (mc * mc));
+    }
+}
+
+// Returns true in every thread of the block that finished last (*counter must
+// start at 0 for the launch).
+__device__ __forceinline__ bool last_block_done(unsigned *counter) {
+    __shared__ bool s_last;
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) s_last = atomicAdd(counter, 1u) == gridDim.x - 1;
+    __syncthreads();
+    if (s_last) __threadfence();
+    return s_last;
+}
+
+// N <= NP <= 32: one thread per token, 256 tokens per block.
+template <int NP>
+__global__ void __launch_bounds__(256) aux_small_kernel(const float *__restrict__ logits,
+                                                        const int *__restrict__ topk_idx,
+                                                        const float *__restrict__ topk_w, int T, int N, int K,
+                                                        float *__restrict__ part_p, float *__restrict__ part_imp,
+                                                        int *__restrict__ part_cnt, unsigned *__restrict__ counter,
+                                                        AuxOut out) {
+    __shared__ float w_p[8][NP], w_i[8][NP];
+    __shared__ int w_c[8][NP];
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int t = blockIdx.x * 256 + tid;
+    float p[NP], im[NP];
+    int c[NP];
+#pragma unroll
+    for (int e = 0; e < NP; ++e) { p[e] = 0.f; im[e] = 0.f; c[e] = 0; }
+    if (t < T) {
+        float s[NP];
+        float mx = -INFINITY;
+#pragma unroll
+        for (int e = 0; e < NP; ++e) {
+            s[e] = e < N ? logits[(size_t)t * N + e] : -INFINITY;
+            mx = fmaxf(mx, s[e]);
+        }
+        float z = 0.f;
+#pragma unroll
+        for (int e = 0; e < NP; ++e) {
+            s[e] = e < N ? expf(s[e] - mx) : 0.f;
+            z += s[e];
+        }
+#pragma unroll
+        for (int e = 0; e < NP; ++e) p[e] = s[e] / z;
+        for (int j = 0; j < K; ++j) {
+            const int ej = topk_idx[(size_t)t * K + j];
+            const float wj = topk_w[(size_t)t * K + j];
+            if (ej < 0 || ej >= N) set_status(kStatusBounds);
+#pragma unroll
+            for (int e = 0; e < NP; ++e)
+                if (e == ej) { im[e] += wj; c[e] += 1; }
+        }
+    }
+#pragma unroll
+    for (int e = 0; e < NP; ++e) {
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) {
+            p[e] += __shfl_xor_sync(0xffffffffu, p[e], o);
+            im[e] += __shfl_xor_sync(0xffffffffu, im[e], o);
+            c[e] += __shfl_xor_sync(0xffffffffu, c[e], o);
+        }
+    }
+    if (lane == 0) {
+#pragma unroll
+        for (int e = 0; e < NP; ++e) { w_p[warp][e] = p[e]; w_i[warp][e] = im[e]; w_c[warp][e] = c[e]; }
+    }
+    __syncthreads();
+    if (tid < N) {
+        float sp = 0.f, si = 0.f;
+        int sc = 0;
+        for (int w = 0; w < 8; ++w) { sp += w_p[w][tid]; si += w_i[w][tid]; sc += w_c[w][tid]; }
+        part_p[(size_t)blockIdx.x * N + tid] = sp;
+        part_imp[(size_t)blockIdx.x * N + tid] = si;
+        part_cnt[(size_t)blockIdx.x * N + tid] = sc;
+    }
+    if (last_block_done(counter)) aux_finalize_block(part_p, part_imp, part_cnt, gridDim.x, T, N, K, out);
+}
+
+// Any N: one warp per token (lane holds experts lane, lane+32, ...), kAuxTokens
+// tokens per block, warp-private shared rows accumulated in token order and
+// added in warp order.
 __global__ void __launch_bounds__(256) aux_partial_kernel(const float *__restrict__ logits,
                                                           const int *__restrict__ topk_idx,
                                                           const float *__restrict__ topk_w, int T, int N, int K,
                                                           float *__restrict__ part_p, float *__restrict__ part_imp,
-                                                          int *__restrict__ part_cnt) {
+                                                          int *__restrict__ part_cnt, unsigned *__restrict__ counter,
+                                                          AuxOut out) {
     extern __shared__ float s_aux[];
     float *acc_p = s_aux;                                     // [8][N]
     float *acc_i = s_aux + 8 * N;                             // [8][N]
@@ -475,61 +731,7 @@ __global__ void __launch_bounds__(256) aux_partial_kernel(const float *__restric
         part_imp[(size_t)blockIdx.x * N + e] = im;
         part_cnt[(size_t)blockIdx.x * N + e] = c;
     }
-}
-
-// Statistics, pass 2 (one block): sums over blocks in block order, then the
-// scalars in double precision:
-//   f_e = counts_e / (T K); switch = N sum f_e P_e; simple = N sum f_e^2;
-//   CV^2 = population variance / mean^2 (0 when the mean is 0).
-__global__ void __launch_bounds__(1024) aux_finalize_kernel(const float *__restrict__ part_p,
-                                                            const float *__restrict__ part_imp,
-                                                            const int *__restrict__ part_cnt, int nblk, int T,
-                                                            int N, int K, int *__restrict__ counts,
-                                                            float *__restrict__ importance,
-                                                            float *__restrict__ p_mean, float *__restrict__ scalars) {
-    extern __shared__ double s_fin[];
-    double *sp = s_fin, *si = s_fin + N, *sc = s_fin + 2 * N;
-    for (int e = threadIdx.x; e < N; e += blockDim.x) {
-        float p = 0.f, im = 0.f;
-        int c = 0;
-        for (int b = 0; b < nblk; ++b) {
-            p += part_p[(size_t)b * N + e];
-            im += part_imp[(size_t)b * N + e];
-            c += part_cnt[(size_t)b * N + e];
-        }
-        const float pm = T > 0 ? p / (float)T : 0.f;
-        if (counts) counts[e] = c;
-        if (importance) importance[e] = im;
-        if (p_mean) p_mean[e] = pm;
-        sp[e] = pm;
-        si[e] = im;
-        sc[e] = c;
-    }
-    __syncthreads();
-    if (threadIdx.x == 0 && scalars) {
-        double sw = 0.0, ss = 0.0, mi = 0.0, mc = 0.0;
-        const double tk = (double)T * (double)K;
-        for (int e = 0; e < N; ++e) {
-            const double f = tk > 0 ? sc[e] / tk : 0.0;
-            sw += f * sp[e];
-            ss += f * f;
-            mi += si[e];
-            mc += sc[e];
-        }
-        mi /= N;
-        mc /= N;
-        double vi = 0.0, vc = 0.0;
-        for (int e = 0; e < N; ++e) {
-            vi += (si[e] - mi) * (si[e] - mi);
-            vc += (sc[e] - mc) * (sc[e] - mc);
-        }
-        vi /= N;
-        vc /= N;
-        scalars[0] = (float)(N * sw);
-        scalars[1] = (float)(N * ss);
-        scalars[2] = mi == 0.0 ? 0.f : (float)(vi / (mi * mi));
-        scalars[3] = mc == 0.0 ? 0.f : (float)(vc / (mc * mc));
-    }
+    if (last_block_done(counter)) aux_finalize_block(part_p, part_imp, part_cnt, gridDim.x, T, N, K, out);
 }
 
 // W_g [D, N] -> W_g^T [N, D] (the K-major operand layout of the router GEMM).

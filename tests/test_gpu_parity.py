@@ -217,6 +217,25 @@ def test_zero_tokens():
     assert torch.all(cnt == 0)
 
 
+@pytest.mark.parametrize("N,K,T", [(8, 2, 2500), (16, 3, 2100), (32, 4, 2049), (6, 2, 2080)])
+def test_chunked_router_path(N, K, T):
+    """T >= 2048 with N <= 32 takes the chunked router (W_g staged in shared memory)."""
+    wl = WORKLOADS["tiny"].with_(N=N, K=K, random_bias=True, zipf_s=0.3)
+    inp = make_inputs(wl, "cuda", T=T)
+    run_full(wl, inp)
+
+
+@pytest.mark.parametrize("dtype,N,K", [(torch.float32, 40, 3), (torch.float32, 64, 6), (torch.bfloat16, 64, 4),
+                                       (torch.bfloat16, 300, 8)])
+def test_gemm_router_path(dtype, N, K):
+    """N > 32 takes the router GEMM (SIMT for fp32, tcgen05 dense tile for bf16) and the top-k kernel."""
+    wl = Workload("many_experts", 11, 700, 256, 128, N, K, ACT_SWIGLU if dtype == torch.bfloat16 else ACT_GELU,
+                  dtype, dtype == torch.float32, 0.05, zipf_s=0.5, random_bias=True)
+    inp = make_inputs(wl, "cuda")
+    layer, y, ws, aux, V, ref, errs = run_full(wl, inp)
+    check_aux(aux, V, wl.N, wl.K)
+
+
 # ----------------------------------------------------------------------------- bf16, tensor cores
 def test_gpt2_bf16_reduced_batch_full_layer():
     wl = WORKLOADS["gpt2"]
