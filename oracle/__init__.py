@@ -189,8 +189,9 @@ def router_scores(x_rows64, Wg, dtype_tag, bg=None) -> np.ndarray:
 
 
 # --- experts and combine ----------------------------------------------------------------------------
-def expert(x_row64, act, dtype_tag, W1e, W2e, b1e=None, b2e=None) -> np.ndarray:
-    """One expert's output for one fp64 token row. W1e: [H, D] (GELU) or [2H, D] (SwiGLU); W2e: [D, H]."""
+def expert(x_row64, act, dtype_tag, W1e, W2e, b1e=None, b2e=None, return_hidden=False):
+    """One expert's output for one fp64 token row. W1e: [H, D] (GELU) or [2H, D] (SwiGLU); W2e: [D, H].
+    With return_hidden, also the hidden activations [H] (after GELU, or silu(gate) * up)."""
     xr = _c(x_row64, np.float64)
     A = _mat(W1e, dtype_tag)
     B = _mat(W2e, dtype_tag)
@@ -203,7 +204,7 @@ def expert(x_row64, act, dtype_tag, W1e, W2e, b1e=None, b2e=None) -> np.ndarray:
                           dtype_tag, _p(hid), _p(out))
     else:
         L.orc_expert_swiglu(D, H, _p(xr), _p(A), _p(B), dtype_tag, _p(hid), _p(out))
-    return out
+    return (out, hid) if return_hidden else out
 
 
 def combine(w, E) -> np.ndarray:

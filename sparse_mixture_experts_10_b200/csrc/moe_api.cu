@@ -14,8 +14,10 @@
 #include "../../include/moe.h"
 #include "moe_common.cuh"
 #include "moe_gemm_simt.cuh"
+#include "moe_gemm_decode.cuh"
 #include "moe_gemm_tc.cuh"
 #include "moe_route.cuh"
+#include "moe_router_tc.cuh"
 
 #include <algorithm>
 #include <atomic>
@@ -30,6 +32,7 @@ constexpr uint64_t kTimeoutNs = 1000000000ull;  // bounded waits give up after 1
 constexpr int kMaxDevices = 64;
 constexpr size_t kSmallRouterSmemMax = 200 * 1024;
 constexpr int64_t kRowdotMaxT = 2048;  // below this the chunked router has too few blocks
+constexpr int64_t kDecodeMaxT = 64;    // up to this many tokens the expert GEMMs stream weights (decode path)
 
 struct DeviceInfo {
     int sms = 0;
@@ -51,8 +54,14 @@ struct Plan {
     int n_chunks;
     int aux_blocks;
     int64_t rows_cap;
-    size_t counters, logits, idx, w, counts, offsets, row_offsets, chunk_counts, chunk_base, perm_slot, slot_row,
-        x_perm, h, z, wgt, aux_p, aux_i, aux_c, total;
+    bool tc_router;    // bf16, N <= 256: router, top-k, statistics and scan in one tensor-core kernel
+    bool few_router;   // bf16, T <= 64, N <= 32: one block per token instead
+    int chunk_tokens;  // tokens per dispatch chunk (32; the tensor-core router's 128-token tile; 1 token)
+    int rnp, rkm;      // tensor-core router: padded expert count, top-k list length
+    bool decode;  // few tokens: weight-streaming expert GEMMs
+    int nt;       // decode: padded token tile (16, 32 or 64)
+    size_t counters, logits, idx, w, counts, offsets, row_offsets, live, chunk_counts, chunk_base, tile_p, tile_imp,
+        perm_slot, slot_row, x_perm, h, z, wgt, aux_p, aux_i, aux_c, total;
 };
 
 int make_plan(const moe_config *c, int64_t T, Plan *p) {
@@ -79,7 +88,14 @@ int make_plan(const moe_config *c, int64_t T, Plan *p) {
     p->small_router = fits && !p->rowdot_router;
     const int need = (int)cdiv(N, 32);
     p->vpl = need <= 1 ? 1 : need <= 2 ? 2 : need <= 4 ? 4 : need <= 8 ? 8 : need <= 16 ? 16 : 32;
-    p->n_chunks = (int)cdiv(T, kChunk);
+    p->decode = c->dtype == MOE_BF16 && T <= kDecodeMaxT;
+    p->nt = T <= 16 ? 16 : T <= 32 ? 32 : 64;
+    p->tc_router = c->dtype == MOE_BF16 && N <= 256;
+    p->few_router = p->tc_router && T <= kDecodeMaxT && N <= 32;
+    p->chunk_tokens = p->few_router ? 1 : p->tc_router ? rtc::BM : kChunk;
+    p->rnp = N <= 16 ? 16 : N <= 32 ? 32 : N <= 64 ? 64 : N <= 128 ? 128 : 256;
+    p->rkm = K <= 8 ? 8 : 32;
+    p->n_chunks = (int)cdiv(T, p->chunk_tokens);
     p->aux_blocks = (int)cdiv(T, kAuxTokens);
     p->rows_cap = cdiv(T * K + N * (kRowAlign - 1), kRowAlign) * kRowAlign;
 
@@ -96,14 +112,18 @@ int make_plan(const moe_config *c, int64_t T, Plan *p) {
     p->counts = take((size_t)N * 4);
     p->offsets = take((size_t)(N + 1) * 4);
     p->row_offsets = take((size_t)(N + 1) * 4);
-    p->chunk_counts = take((size_t)p->n_chunks * N * 4);
-    p->chunk_base = take((size_t)p->n_chunks * N * 4);
+    p->live = take((size_t)N * 4);
+    const int64_t max_chunks = std::max<int64_t>(p->n_chunks, 1);
+    p->chunk_counts = take((size_t)max_chunks * N * 4);
+    p->chunk_base = take((size_t)max_chunks * N * 4);
+    p->tile_p = take(p->tc_router ? (size_t)max_chunks * N * 4 : 0);
+    p->tile_imp = take(p->tc_router ? (size_t)max_chunks * N * 8 : 0);
     p->perm_slot = take((size_t)p->rows_cap * 4);
     p->slot_row = take((size_t)T * K * 4);
     p->x_perm = take((size_t)p->rows_cap * D * es);
     p->h = take((size_t)p->rows_cap * H * es);
     p->z = take((size_t)T * K * D * 4);
-    p->wgt = take(N <= 32 ? 0 : (size_t)N * D * es);
+    p->wgt = take((N <= 32 && !(p->tc_router && !p->few_router)) ? 0 : (size_t)N * D * es);
     p->aux_p = take((size_t)p->aux_blocks * N * 4);
     p->aux_i = take((size_t)p->aux_blocks * N * 4);
     p->aux_c = take((size_t)p->aux_blocks * N * 4);
@@ -112,6 +132,24 @@ int make_plan(const moe_config *c, int64_t T, Plan *p) {
 }
 
 bool aligned16(const void *ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) == 0; }
+
+#define MOE_TRY(expr)                  \
+    do {                               \
+        const int _rc = (expr);        \
+        if (_rc != MOE_OK) return _rc; \
+    } while (0)
+
+// Lets a kernel use as much dynamic shared memory as the per-block limit leaves
+// next to its static shared memory.
+template <typename K>
+int allow_smem(K *kernel) {
+    cudaFuncAttributes fa;
+    if (cudaFuncGetAttributes(&fa, kernel) != cudaSuccess) return MOE_ERR_CUDA;
+    const int limit = 227 * 1024 - (int)fa.sharedSizeBytes;
+    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, limit) == cudaSuccess
+               ? MOE_OK
+               : MOE_ERR_CUDA;
+}
 
 int device_info(DeviceInfo **out) {
     int dev = 0;
@@ -122,22 +160,41 @@ int device_info(DeviceInfo **out) {
         if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return MOE_ERR_CUDA;
     }
     if (!d.attrs) {
-        const int big = 227 * 1024;
-        cudaFuncSetAttribute(tc::grouped_gemm_tc_kernel<256, tc::EPI_GELU>, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
-        cudaFuncSetAttribute(tc::grouped_gemm_tc_kernel<256, tc::EPI_SWIGLU>, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
-        cudaFuncSetAttribute(tc::grouped_gemm_tc_kernel<256, tc::EPI_SCATTER>, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
-        cudaFuncSetAttribute(tc::grouped_gemm_tc_kernel<256, tc::EPI_LOGITS>, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
-        cudaFuncSetAttribute(tc::grouped_gemm_tc_kernel<128, tc::EPI_GELU>, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
-        cudaFuncSetAttribute(tc::grouped_gemm_tc_kernel<128, tc::EPI_SWIGLU>, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
-        cudaFuncSetAttribute(tc::grouped_gemm_tc_kernel<128, tc::EPI_SCATTER>, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
-        cudaFuncSetAttribute(router_small_kernel<float, 8>, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
-        cudaFuncSetAttribute(router_small_kernel<float, 16>, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
-        cudaFuncSetAttribute(router_small_kernel<float, 32>, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
-        cudaFuncSetAttribute(router_small_kernel<__nv_bfloat16, 8>, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
-        cudaFuncSetAttribute(router_small_kernel<__nv_bfloat16, 16>, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
-        cudaFuncSetAttribute(router_small_kernel<__nv_bfloat16, 32>, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
-        cudaFuncSetAttribute(aux_partial_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 160 * 1024);
-        if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
+        MOE_TRY(allow_smem(tc::grouped_gemm_tc_kernel<256, tc::EPI_GELU>));
+        MOE_TRY(allow_smem(tc::grouped_gemm_tc_kernel<256, tc::EPI_SWIGLU>));
+        MOE_TRY(allow_smem(tc::grouped_gemm_tc_kernel<256, tc::EPI_SCATTER>));
+        MOE_TRY(allow_smem(tc::grouped_gemm_tc_kernel<256, tc::EPI_LOGITS>));
+        MOE_TRY(allow_smem(tc::grouped_gemm_tc2_kernel<tc::EPI_GELU>));
+        MOE_TRY(allow_smem(tc::grouped_gemm_tc2_kernel<tc::EPI_SWIGLU>));
+        MOE_TRY(allow_smem(tc::grouped_gemm_tc2_kernel<tc::EPI_SCATTER>));
+        MOE_TRY(allow_smem(tc::grouped_gemm_tc2_kernel<tc::EPI_LOGITS>));
+        MOE_TRY(allow_smem(tc::grouped_gemm_tc_kernel<128, tc::EPI_GELU>));
+        MOE_TRY(allow_smem(tc::grouped_gemm_tc_kernel<128, tc::EPI_SWIGLU>));
+        MOE_TRY(allow_smem(tc::grouped_gemm_tc_kernel<128, tc::EPI_SCATTER>));
+        MOE_TRY(allow_smem(router_small_kernel<float, 8>));
+        MOE_TRY(allow_smem(router_small_kernel<float, 16>));
+        MOE_TRY(allow_smem(router_small_kernel<float, 32>));
+        MOE_TRY(allow_smem(router_small_kernel<__nv_bfloat16, 8>));
+        MOE_TRY(allow_smem(router_small_kernel<__nv_bfloat16, 16>));
+        MOE_TRY(allow_smem(router_small_kernel<__nv_bfloat16, 32>));
+        MOE_TRY(allow_smem(aux_partial_kernel));
+#define MOE_RTC_ATTR(NP)                                                                                     \
+    MOE_TRY(allow_smem(rtc::router_tc_kernel<NP, 8>)); \
+    MOE_TRY(allow_smem(rtc::router_tc_kernel<NP, 32>))
+        MOE_RTC_ATTR(16);
+        MOE_RTC_ATTR(32);
+        MOE_RTC_ATTR(64);
+        MOE_RTC_ATTR(128);
+        MOE_RTC_ATTR(256);
+#undef MOE_RTC_ATTR
+#define MOE_DEC_ATTR(NT)                                                                                          \
+    MOE_TRY(allow_smem(dec::decode_gemm_kernel<NT, dec::EPI_GELU>)); \
+    MOE_TRY(allow_smem(dec::decode_gemm_kernel<NT, dec::EPI_SWIGLU>)); \
+    MOE_TRY(allow_smem(dec::decode_gemm_kernel<NT, dec::EPI_SCATTER>))
+        MOE_DEC_ATTR(16);
+        MOE_DEC_ATTR(32);
+        MOE_DEC_ATTR(64);
+#undef MOE_DEC_ATTR
         d.attrs = true;
     }
     *out = &d;
@@ -149,11 +206,6 @@ int check_launch() {
     return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
-#define MOE_TRY(expr)                  \
-    do {                               \
-        const int _rc = (expr);        \
-        if (_rc != MOE_OK) return _rc; \
-    } while (0)
 
 // --------------------------------------------------------------- TMA tensor maps
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
@@ -196,6 +248,16 @@ int launch_tc(const CUtensorMap &A, const CUtensorMap &B, const tc::Params &p, i
     return check_launch();
 }
 
+// Pair (2-CTA cluster) version for 256-column tiles: 256-row units per cluster.
+template <int EPI>
+int launch_tc2(const CUtensorMap &A, const CUtensorMap &B, const tc::Params &p, int64_t units_upper, int sms,
+               cudaStream_t s) {
+    const int64_t clusters = std::min<int64_t>(std::max<int64_t>(units_upper, 1), sms / 2);
+    const size_t smem = tc::Shape2::smem_bytes(p.num_groups);
+    tc::grouped_gemm_tc2_kernel<EPI><<<(unsigned)(2 * clusters), tc::kThreads, smem, s>>>(A, B, p);
+    return check_launch();
+}
+
 template <int EPI>
 int launch_simt(const simt::Params &p, int64_t rows, int n_blocks, cudaStream_t s) {
     const dim3 grid((unsigned)cdiv(std::max<int64_t>(rows, 1), simt::TM), (unsigned)std::max(n_blocks, 1));
@@ -212,6 +274,74 @@ struct Bufs {
 
 // ---------------------------------------------------------------- stages
 // route: logits (always written to `logits`), top-k, chunk histograms.
+template <int NP, int KM>
+int launch_rtc(const CUtensorMap &mx, const CUtensorMap &mw, const rtc::Params &p, int grid, cudaStream_t s) {
+    rtc::router_tc_kernel<NP, KM><<<grid, rtc::kThreads, rtc::Shape<NP>::kSmem, s>>>(mx, mw, p);
+    return check_launch();
+}
+
+// Tensor-core router: scores, top-k, statistics partials and (in the last CTA)
+// the dispatch tables and the finished statistics.
+int stage_route_tc(const Plan &P, const Bufs &b, const void *x, const moe_weights *w, float *logits, int *idx,
+                   float *tw, int *counts_out, const moe_aux *aux, cudaStream_t s) {
+    const int T = (int)P.T, D = P.D, N = P.N;
+    rtc::Params p{};
+    p.T = T;
+    p.D = D;
+    p.N = N;
+    p.K = P.K;
+    p.np = P.rnp;
+    p.bg = w->b_g;
+    p.logits = logits;
+    p.topk_idx = idx;
+    p.topk_w = tw;
+    p.tile_counts = b.at<int>(P.chunk_counts);
+    p.tile_p = b.at<float>(P.tile_p);
+    p.tile_imp = b.at<unsigned long long>(P.tile_imp);
+    p.ticket = b.at<unsigned>(P.counters);
+    p.chunk_base = b.at<int>(P.chunk_base);
+    p.counts = b.at<int>(P.counts);
+    p.offsets = b.at<int>(P.offsets);
+    p.row_offsets = b.at<int>(P.row_offsets);
+    p.perm_slot = b.at<int>(P.perm_slot);
+    p.live = b.at<int>(P.live);
+    p.n_live = b.at<int>(P.counters) + 2;
+    p.counts_out = counts_out;
+    if (aux) {
+        p.aux_counts = aux->counts;
+        p.aux_importance = aux->importance;
+        p.aux_p_mean = aux->p_mean;
+        p.aux_scalars = aux->scalars;
+    }
+    p.timeout_ns = kTimeoutNs;
+    if (P.few_router) {
+        const __nv_bfloat16 *xb = static_cast<const __nv_bfloat16 *>(x);
+        const __nv_bfloat16 *wg = static_cast<const __nv_bfloat16 *>(w->W_g);
+        if (N <= 8) rtc::router_few_kernel<8><<<T, 256, 0, s>>>(xb, wg, p);
+        else if (N <= 16) rtc::router_few_kernel<16><<<T, 256, 0, s>>>(xb, wg, p);
+        else rtc::router_few_kernel<32><<<T, 256, 0, s>>>(xb, wg, p);
+        return check_launch();
+    }
+    __nv_bfloat16 *wgt = b.at<__nv_bfloat16>(P.wgt);
+    transpose_kernel<__nv_bfloat16><<<dim3((unsigned)cdiv(N, 32), (unsigned)cdiv(D, 32)), dim3(32, 8), 0, s>>>(
+        static_cast<const __nv_bfloat16 *>(w->W_g), D, N, wgt);
+    MOE_TRY(check_launch());
+    CUtensorMap mx, mw;
+    MOE_TRY(make_map(&mx, x, T, D, rtc::BM));
+    MOE_TRY(make_map(&mw, wgt, N, D, P.rnp));
+    const int grid = P.n_chunks;
+#define MOE_RTC(NP)                                                                        \
+    return P.rkm == 8 ? launch_rtc<NP, 8>(mx, mw, p, grid, s) : launch_rtc<NP, 32>(mx, mw, p, grid, s)
+    switch (P.rnp) {
+        case 16: MOE_RTC(16);
+        case 32: MOE_RTC(32);
+        case 64: MOE_RTC(64);
+        case 128: MOE_RTC(128);
+        default: MOE_RTC(256);
+    }
+#undef MOE_RTC
+}
+
 int stage_route(const Plan &P, const Bufs &b, const void *x, const moe_weights *w, float *logits, int *idx,
                 float *tw, const DeviceInfo &dev, cudaStream_t s) {
     const int T = (int)P.T, D = P.D, N = P.N, K = P.K;
@@ -254,7 +384,7 @@ int stage_route(const Plan &P, const Bufs &b, const void *x, const moe_weights *
         MOE_TRY(check_launch());
         CUtensorMap ma, mb;
         MOE_TRY(make_map(&ma, x, T, D, tc::BM));
-        MOE_TRY(make_map(&mb, wgt, N, D, 256));
+        MOE_TRY(make_map(&mb, wgt, N, D, 128));
         tc::Params p{};
         p.num_groups = 1;
         p.row_offsets = nullptr;
@@ -267,7 +397,7 @@ int stage_route(const Plan &P, const Bufs &b, const void *x, const moe_weights *
         p.ldo = N;
         p.bias = w->b_g;
         p.timeout_ns = kTimeoutNs;
-        MOE_TRY((launch_tc<256, tc::EPI_LOGITS>(ma, mb, p, cdiv(T, tc::BM) * p.n_tiles, dev.sms, s)));
+        MOE_TRY((launch_tc2<tc::EPI_LOGITS>(ma, mb, p, cdiv(T, 2 * tc::BM) * p.n_tiles, dev.sms, s)));
     } else {
         float *wgt = b.at<float>(P.wgt);
         transpose_kernel<float><<<dim3((unsigned)cdiv(N, 32), (unsigned)cdiv(D, 32)), dim3(32, 8), 0, s>>>(
@@ -305,22 +435,94 @@ int stage_route(const Plan &P, const Bufs &b, const void *x, const moe_weights *
 int stage_scan(const Plan &P, const Bufs &b, int *counts_out, cudaStream_t s) {
     scan_kernel<<<(unsigned)cdiv(P.N, 32), 1024, 0, s>>>(
         b.at<int>(P.chunk_counts), P.n_chunks, P.N, P.T * P.K, b.at<int>(P.chunk_base), b.at<int>(P.counts),
-        b.at<int>(P.offsets), b.at<int>(P.row_offsets), b.at<int>(P.perm_slot), counts_out, b.at<unsigned>(P.counters));
+        b.at<int>(P.offsets), b.at<int>(P.row_offsets), b.at<int>(P.perm_slot), counts_out, b.at<unsigned>(P.counters),
+        b.at<int>(P.live), b.at<int>(P.counters) + 2);
     return check_launch();
 }
 
-int stage_permute(const Plan &P, const Bufs &b, const void *x, cudaStream_t s) {
-    const size_t smem = (size_t)(P.N + kChunk * P.K) * 4;
+int stage_permute(const Plan &P, const Bufs &b, const void *x, const DeviceInfo &dev, cudaStream_t s) {
+    const size_t smem = (size_t)(P.N + P.chunk_tokens * P.K) * 4;
+    // enough blocks to keep every SM copying: split each chunk's rows over several blocks
+    const int split = (int)std::max<int64_t>(1, std::min<int64_t>(8, cdiv(2 * dev.sms, P.n_chunks)));
+    const dim3 grid((unsigned)P.n_chunks, (unsigned)split);
     if (P.dtype == MOE_F32)
-        permute_kernel<float><<<P.n_chunks, 256, smem, s>>>(static_cast<const float *>(x), (int)P.T, P.D, P.K, P.N,
-                                                           b.at<int>(P.idx), b.at<int>(P.chunk_base),
-                                                           b.at<int>(P.row_offsets), b.at<int>(P.perm_slot),
-                                                           b.at<int>(P.slot_row), b.at<float>(P.x_perm));
+        permute_kernel<float><<<grid, 256, smem, s>>>(static_cast<const float *>(x), (int)P.T, P.D, P.K, P.N,
+                                                     P.chunk_tokens, b.at<int>(P.idx), b.at<int>(P.chunk_base),
+                                                     b.at<int>(P.row_offsets), b.at<int>(P.perm_slot),
+                                                     b.at<int>(P.slot_row), b.at<float>(P.x_perm));
     else
-        permute_kernel<__nv_bfloat16><<<P.n_chunks, 256, smem, s>>>(
-            static_cast<const __nv_bfloat16 *>(x), (int)P.T, P.D, P.K, P.N, b.at<int>(P.idx), b.at<int>(P.chunk_base),
-            b.at<int>(P.row_offsets), b.at<int>(P.perm_slot), b.at<int>(P.slot_row), b.at<__nv_bfloat16>(P.x_perm));
+        permute_kernel<__nv_bfloat16><<<grid, 256, smem, s>>>(
+            static_cast<const __nv_bfloat16 *>(x), (int)P.T, P.D, P.K, P.N, P.chunk_tokens, b.at<int>(P.idx),
+            b.at<int>(P.chunk_base), b.at<int>(P.row_offsets), b.at<int>(P.perm_slot), b.at<int>(P.slot_row),
+            b.at<__nv_bfloat16>(P.x_perm));
     return check_launch();
+}
+
+// Expert GEMMs for few tokens (decode path): weight rows are the MMA's M
+// operand, each expert's token rows (at most T <= 64) its narrow N operand.
+template <int NT, int EPI>
+int launch_dec(const CUtensorMap &W, const CUtensorMap &X, const dec::Params &p, int64_t items_upper, int sms,
+               cudaStream_t s) {
+    const int grid = (int)std::min<int64_t>(std::max<int64_t>(items_upper, 1), sms);
+    dec::decode_gemm_kernel<NT, EPI><<<grid, dec::kThreads, dec::Shape<NT, EPI>::kSmem, s>>>(W, X, p);
+    return check_launch();
+}
+
+template <int EPI>
+int launch_dec_nt(int nt, const CUtensorMap &W, const CUtensorMap &X, const dec::Params &p, int64_t items_upper,
+                  int sms, cudaStream_t s) {
+    if (nt == 16) return launch_dec<16, EPI>(W, X, p, items_upper, sms, s);
+    if (nt == 32) return launch_dec<32, EPI>(W, X, p, items_upper, sms, s);
+    return launch_dec<64, EPI>(W, X, p, items_upper, sms, s);
+}
+
+int stage_up_decode(const Plan &P, const Bufs &b, const moe_weights *w, const DeviceInfo &dev, cudaStream_t s) {
+    const int D = P.D, H = P.H, N = P.N;
+    const bool swiglu = P.act == MOE_ACT_SWIGLU;
+    CUtensorMap mw, mx;
+    MOE_TRY(make_map(&mw, w->W1, (int64_t)N * (swiglu ? 2 * H : H), D, swiglu ? 64 : 128));
+    MOE_TRY(make_map(&mx, b.ws + P.x_perm, P.rows_cap, D, P.nt));
+    dec::Params p{};
+    p.row_offsets = b.at<int>(P.row_offsets);
+    p.counts = b.at<int>(P.counts);
+    p.live = b.at<int>(P.live);
+    p.n_live = b.at<int>(P.counters) + 2;
+    p.tiles_per_group = (int)cdiv(H, swiglu ? 64 : 128);
+    p.num_k_blocks = (int)cdiv(D, dec::BK);
+    p.w_group_rows = swiglu ? 2 * H : H;
+    p.w_up_offset = H;
+    p.n_valid = H;
+    p.out = b.ws + P.h;
+    p.ldo = H;
+    p.bias = swiglu ? nullptr : w->b1;
+    p.timeout_ns = kTimeoutNs;
+    const int64_t upper = std::min<int64_t>(N, P.T * P.K) * p.tiles_per_group;
+    if (swiglu) return launch_dec_nt<dec::EPI_SWIGLU>(P.nt, mw, mx, p, upper, dev.sms, s);
+    return launch_dec_nt<dec::EPI_GELU>(P.nt, mw, mx, p, upper, dev.sms, s);
+}
+
+int stage_down_decode(const Plan &P, const Bufs &b, const moe_weights *w, const DeviceInfo &dev, cudaStream_t s) {
+    const int D = P.D, H = P.H, N = P.N;
+    CUtensorMap mw, mx;
+    MOE_TRY(make_map(&mw, w->W2, (int64_t)N * D, H, 128));
+    MOE_TRY(make_map(&mx, b.ws + P.h, P.rows_cap, H, P.nt));
+    dec::Params p{};
+    p.row_offsets = b.at<int>(P.row_offsets);
+    p.counts = b.at<int>(P.counts);
+    p.live = b.at<int>(P.live);
+    p.n_live = b.at<int>(P.counters) + 2;
+    p.tiles_per_group = (int)cdiv(D, 128);
+    p.num_k_blocks = (int)cdiv(H, dec::BK);
+    p.w_group_rows = D;
+    p.n_valid = D;
+    p.out = b.ws + P.z;
+    p.ldo = D;
+    p.bias = P.act == MOE_ACT_SWIGLU ? nullptr : w->b2;
+    p.perm_slot = b.at<int>(P.perm_slot);
+    p.gate_w = b.at<float>(P.w);
+    p.timeout_ns = kTimeoutNs;
+    const int64_t upper = std::min<int64_t>(N, P.T * P.K) * p.tiles_per_group;
+    return launch_dec_nt<dec::EPI_SCATTER>(P.nt, mw, mx, p, upper, dev.sms, s);
 }
 
 // True when the grouped GEMM would have too few 256-wide tiles to fill the
@@ -328,10 +530,11 @@ int stage_permute(const Plan &P, const Bufs &b, const void *x, cudaStream_t s) {
 // since the per-expert counts live on the device.
 bool narrow_tiles(const Plan &P, int64_t n_tiles_256, const DeviceInfo &dev) {
     const int64_t m_tiles_min = std::max<int64_t>(1, cdiv(P.T * P.K, tc::BM));
-    return m_tiles_min * n_tiles_256 < 2 * (int64_t)dev.sms;
+    return m_tiles_min * n_tiles_256 < (int64_t)dev.sms;
 }
 
 int stage_up(const Plan &P, const Bufs &b, const moe_weights *w, const DeviceInfo &dev, cudaStream_t s) {
+    if (P.decode) return stage_up_decode(P, b, w, dev, s);
     const int D = P.D, H = P.H, N = P.N;
     const bool swiglu = P.act == MOE_ACT_SWIGLU;
     if (P.dtype == MOE_BF16) {
@@ -339,7 +542,7 @@ int stage_up(const Plan &P, const Bufs &b, const moe_weights *w, const DeviceInf
         const int out_cols = swiglu ? bn / 2 : bn;  // h columns per tile
         CUtensorMap ma, mb;
         MOE_TRY(make_map(&ma, b.ws + P.x_perm, P.rows_cap, D, tc::BM));
-        MOE_TRY(make_map(&mb, w->W1, (int64_t)N * (swiglu ? 2 * H : H), D, swiglu ? bn / 2 : bn));
+        MOE_TRY(make_map(&mb, w->W1, (int64_t)N * (swiglu ? 2 * H : H), D, bn == 256 ? 128 : (swiglu ? bn / 2 : bn)));
         tc::Params p{};
         p.num_groups = N;
         p.row_offsets = b.at<int>(P.row_offsets);
@@ -357,8 +560,9 @@ int stage_up(const Plan &P, const Bufs &b, const moe_weights *w, const DeviceInf
             if (swiglu) return launch_tc<128, tc::EPI_SWIGLU>(ma, mb, p, upper, dev.sms, s);
             return launch_tc<128, tc::EPI_GELU>(ma, mb, p, upper, dev.sms, s);
         }
-        if (swiglu) return launch_tc<256, tc::EPI_SWIGLU>(ma, mb, p, upper, dev.sms, s);
-        return launch_tc<256, tc::EPI_GELU>(ma, mb, p, upper, dev.sms, s);
+        const int64_t units = (P.rows_cap / (2 * tc::BM) + N) * p.n_tiles;
+        if (swiglu) return launch_tc2<tc::EPI_SWIGLU>(ma, mb, p, units, dev.sms, s);
+        return launch_tc2<tc::EPI_GELU>(ma, mb, p, units, dev.sms, s);
     }
     simt::Params p{};
     p.A = b.at<float>(P.x_perm);
@@ -379,13 +583,14 @@ int stage_up(const Plan &P, const Bufs &b, const moe_weights *w, const DeviceInf
 }
 
 int stage_down(const Plan &P, const Bufs &b, const moe_weights *w, const DeviceInfo &dev, cudaStream_t s) {
+    if (P.decode) return stage_down_decode(P, b, w, dev, s);
     const int D = P.D, H = P.H, N = P.N;
     const float *bias = P.act == MOE_ACT_SWIGLU ? nullptr : w->b2;
     if (P.dtype == MOE_BF16) {
         const int bn = narrow_tiles(P, cdiv(D, 256), dev) ? 128 : 256;
         CUtensorMap ma, mb;
         MOE_TRY(make_map(&ma, b.ws + P.h, P.rows_cap, H, tc::BM));
-        MOE_TRY(make_map(&mb, w->W2, (int64_t)N * D, H, bn));
+        MOE_TRY(make_map(&mb, w->W2, (int64_t)N * D, H, 128));
         tc::Params p{};
         p.num_groups = N;
         p.row_offsets = b.at<int>(P.row_offsets);
@@ -401,7 +606,7 @@ int stage_down(const Plan &P, const Bufs &b, const moe_weights *w, const DeviceI
         p.timeout_ns = kTimeoutNs;
         const int64_t upper = (P.rows_cap / tc::BM) * p.n_tiles;
         if (bn == 128) return launch_tc<128, tc::EPI_SCATTER>(ma, mb, p, upper, dev.sms, s);
-        return launch_tc<256, tc::EPI_SCATTER>(ma, mb, p, upper, dev.sms, s);
+        return launch_tc2<tc::EPI_SCATTER>(ma, mb, p, (P.rows_cap / (2 * tc::BM) + N) * p.n_tiles, dev.sms, s);
     }
     simt::Params p{};
     p.A = b.at<float>(P.h);
@@ -510,11 +715,16 @@ int forward_impl(const moe_config *cfg, const void *x, int64_t T, const moe_weig
     float *tw = b.at<float>(P.w);
     MOE_TRY(rec(0));
     MOE_TRY(zero_counters(P, b, s));
-    MOE_TRY(stage_route(P, b, x, w, logits, idx, tw, *dev, s));
-    MOE_TRY(rec(1));
-    MOE_TRY(stage_scan(P, b, nullptr, s));
+    if (P.tc_router) {
+        MOE_TRY(stage_route_tc(P, b, x, w, logits, idx, tw, nullptr, aux, s));
+        MOE_TRY(rec(1));
+    } else {
+        MOE_TRY(stage_route(P, b, x, w, logits, idx, tw, *dev, s));
+        MOE_TRY(rec(1));
+        MOE_TRY(stage_scan(P, b, nullptr, s));
+    }
     MOE_TRY(rec(2));
-    MOE_TRY(stage_permute(P, b, x, s));
+    MOE_TRY(stage_permute(P, b, x, *dev, s));
     MOE_TRY(rec(3));
     MOE_TRY(stage_up(P, b, w, *dev, s));
     MOE_TRY(rec(4));
@@ -522,7 +732,7 @@ int forward_impl(const moe_config *cfg, const void *x, int64_t T, const moe_weig
     MOE_TRY(rec(5));
     MOE_TRY(stage_combine(P, b, y, y_dtype, *dev, s));
     MOE_TRY(rec(6));
-    if (aux) MOE_TRY(stage_aux(P, b, logits, idx, tw, aux, s));
+    if (aux && !P.tc_router) MOE_TRY(stage_aux(P, b, logits, idx, tw, aux, s));
     MOE_TRY(rec(7));
     return MOE_OK;
 }
@@ -577,6 +787,7 @@ int moe_route(const moe_config *cfg, const void *x, int64_t T, const moe_weights
     Bufs b{static_cast<char *>(ws), &P};
     float *lg = logits ? logits : b.at<float>(P.logits);
     MOE_TRY(zero_counters(P, b, s));
+    if (P.tc_router) return stage_route_tc(P, b, x, w, lg, topk_idx, topk_w, counts, nullptr, s);
     MOE_TRY(stage_route(P, b, x, w, lg, topk_idx, topk_w, *dev, s));
     if (counts) MOE_TRY(stage_scan(P, b, counts, s));
     return MOE_OK;

@@ -1,7 +1,7 @@
 // moe_gemm_tc.cuh -- grouped GEMM on the sm_100a tensor cores (tcgen05 + TMEM).
 //
 // C[r, n] = sum_k A[r, k] * B[g * b_group_rows + n, k], bf16 x bf16 -> fp32,
-// for every 128-row tile r of an expert segment g of the permuted activations
+// for every row tile r of an expert segment g of the permuted activations
 // (or of a plain row-major matrix, "dense" mode with one group).  Both operands
 // are K-major; A rows are tokens, B rows are output features of expert g
 // (weights stored out x in).  This evaluates each selected expert only on the
@@ -10,15 +10,29 @@
 // multiplied by zero -- as one grouped GEMM, the grouped_mm backend idea of the
 // Transformers-v5 MoE article, section 2.
 //
-// Kernel structure (one persistent CTA per SM, 320 threads):
+// Two kernels share the epilogue:
+//
+// grouped_gemm_tc_kernel<BN, EPI>  one CTA per tile of 128 rows x BN columns,
+//   persistent, 576 threads:
 //   warp 0      TMA producer: 64-wide K slices of A (128 rows) and B (BN rows)
-//               into a kStages-deep shared-memory ring (128-byte swizzle).
+//               into a shared-memory ring (128-byte swizzle).
 //   warp 1      allocates 2*BN TMEM columns; one thread issues
-//               tcgen05.mma (128 x BN x 16) into one of two TMEM accumulators
-//               and commits ring slots / finished accumulators to mbarriers.
-//   warps 2..9  epilogue: tcgen05.ld of the accumulator (warp w reads TMEM
-//               lanes 32*(w%4)..+31, half of the columns each), fused
+//               tcgen05.mma.cta_group::1 (128 x BN x 16) into one of two TMEM
+//               accumulators and commits ring slots / accumulators to mbarriers.
+//   warps 2..17 epilogue: tcgen05.ld of the accumulator (warp w reads TMEM
+//               lanes 32*(w%4)..+31 and a quarter of the columns), fused
 //               activation / scaling, stores to global memory.
+//
+// grouped_gemm_tc2_kernel<EPI>  a cluster of two CTAs (one per SM of a pair)
+//   per tile of 256 rows x 256 columns: each CTA loads its own 128 rows of A
+//   and its own 128 rows of B (no multicast), the leader CTA issues
+//   tcgen05.mma.cta_group::2 (256 x 256 x 16), which reads both CTAs' shared
+//   memory and accumulates into both CTAs' TMEM; ring slots and finished
+//   accumulators are committed to the barriers of both CTAs; the epilogue of
+//   each CTA reads its own TMEM and releases the accumulator on the leader's
+//   barrier.  Per SM, a 64-wide K slice then moves 32 KB for 4 MFLOP (instead
+//   of 48 KB), and the ring holds 6 slices instead of 4.
+//
 // The two accumulators let the epilogue of tile i overlap the MMAs of tile
 // i+1.  Tiles are ordered expert by expert and, inside an expert, by column
 // tile then row tile, so concurrently running CTAs share the same weight
@@ -26,8 +40,8 @@
 //
 // Epilogues:
 //   EPI_GELU     h = bf16(gelu_erf(acc + b1[g, n]))           (GPT-2 expert, first linear)
-//   EPI_SWIGLU   B tile = 128 gate rows + 128 up rows (two TMA boxes of the
-//                packed gate_up weight); h = bf16(silu(gate) * up)
+//   EPI_SWIGLU   B tile = 128 gate rows + 128 up rows of the packed gate_up
+//                weight; h = bf16(silu(gate) * up)
 //   EPI_SCATTER  z[slot(r), n] = w[slot(r)] * (acc + b2[g, n]), fp32, rows
 //                with slot -1 (padding) skipped      (down projection)
 //   EPI_LOGITS   out[r, n] = acc + b_g[n], fp32, rows < dense_rows   (router)
@@ -44,7 +58,8 @@ namespace tc {
 
 constexpr int BM = 128;
 constexpr int BK = 64;
-constexpr int kEpiWarps = 8;
+constexpr int kEpiWarps = 16;                  // four per TMEM lane quadrant
+constexpr int kEpiGroups = kEpiWarps / 4;      // column groups of a tile
 constexpr int kThreads = 64 + 32 * kEpiWarps;
 
 enum { EPI_GELU = 0, EPI_SWIGLU = 1, EPI_SCATTER = 2, EPI_LOGITS = 3 };
@@ -79,10 +94,24 @@ struct Shape {
     }
 };
 
+// Pair kernel: per CTA, 128 rows of A and 128 rows of B per K slice.
+struct Shape2 {
+    static constexpr int kStages = 6;
+    static constexpr uint32_t kABytes = BM * BK * 2;
+    static constexpr uint32_t kBBytes = 128 * BK * 2;
+    static constexpr uint32_t kTmemCols = 512;
+    static constexpr size_t kBarrierBytes = (2 * kStages + 5) * 8 + 16;
+    // ring + slack + barriers + tmem slot; group table and 256-row unit table follow
+    static size_t smem_bytes(int groups) {
+        return 1024 + kStages * (size_t)(kABytes + kBBytes) + kBarrierBytes + 8 * (size_t)(groups + 1) + 16;
+    }
+};
+
 struct TileCoord {
     int g, row0, nt;
 };
 
+// Tile i of 128-row tiles: group, first row and column tile.
 __device__ __forceinline__ TileCoord decode_tile(int i, const int *s_rowoff, int G, int n_tiles, int dense_mtiles) {
     TileCoord c;
     if (s_rowoff == nullptr) {
@@ -106,23 +135,196 @@ __device__ __forceinline__ TileCoord decode_tile(int i, const int *s_rowoff, int
     return c;
 }
 
+// Tile i of 256-row unit tiles.  s_units[g] = number of 256-row units before
+// group g (a group of 128*m padded rows has ceil(m/2) units); row0 is the first
+// row of the unit, whose upper half may lie past the group's end.
+__device__ __forceinline__ TileCoord decode_unit_tile(int i, const int *s_rowoff, const int *s_units, int G,
+                                                      int n_tiles, int dense_units) {
+    TileCoord c;
+    if (s_rowoff == nullptr) {
+        c.g = 0;
+        c.nt = i / dense_units;
+        c.row0 = (i - c.nt * dense_units) * 2 * BM;
+        return c;
+    }
+    int lo = 0, hi = G - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (s_units[mid] * n_tiles <= i) lo = mid;
+        else hi = mid - 1;
+    }
+    const int u0 = s_units[lo];
+    const int un = s_units[lo + 1] - u0;
+    const int local = i - u0 * n_tiles;
+    c.g = lo;
+    c.nt = local / un;
+    c.row0 = s_rowoff[lo] + (local - c.nt * un) * 2 * BM;
+    return c;
+}
+
+// 1/x for x in [1, 2.32] without the special-function unit: quadratic seed
+// (relative error < 1.8e-2, fitted here by weighted least squares) and two
+// Newton steps r <- r (2 - x r) (error squares each step: < 1e-7).
+__device__ __forceinline__ float rcp_1_2(float x) {
+    float r = fmaf(fmaf(0.24989176f, x, -1.24085286f), x, 1.97339064f);
+    r = r * fmaf(-x, r, 2.0f);
+    r = r * fmaf(-x, r, 2.0f);
+    return r;
+}
+
+// 2^y for y in [-126, 0] without the special-function unit: y = n + f with n
+// integer (rounded by adding 1.5 * 2^23) and |f| <= 1/2; 2^f by a degree-6
+// polynomial fitted here (relative error < 2e-9); n goes into the exponent bits.
+__device__ __forceinline__ float exp2_fma(float y) {
+    y = fmaxf(y, -126.0f);
+    const float t = y + 12582912.0f;
+    const float f = y - (t - 12582912.0f);
+    float q = fmaf(1.53458105e-4f, f, 1.33999315e-3f);
+    q = fmaf(q, f, 9.61848897e-3f);
+    q = fmaf(q, f, 5.55032878e-2f);
+    q = fmaf(q, f, 0.240226469f);
+    q = fmaf(q, f, 0.693147206f);
+    q = fmaf(q, f, 1.0f);
+    return __int_as_float(__float_as_int(q) + ((__float_as_int(t) - 0x4B400000) << 23));
+}
+
 // GELU(v) = v Phi(v) = 0.5 v (1 + erf(v / sqrt 2)), exact-erf form, with erfc
 // from Abramowitz & Stegun, Handbook of Mathematical Functions, formula 7.1.26
-// (absolute error of erf at most 1.5e-7, far below the bf16 rounding of h):
+// (absolute error of erf at most 1.5e-7):
 //   erfc(z) ~ (a1 t + a2 t^2 + a3 t^3 + a4 t^4 + a5 t^5) exp(-z^2), t = 1 / (1 + p z), z >= 0.
-// For v < 0, 1 + erf(v / sqrt 2) = erfc(|v| / sqrt 2) is used directly (no cancellation).
+// For v < 0, 1 + erf(v / sqrt 2) = erfc(|v| / sqrt 2) is used directly (no
+// cancellation).  z is capped at 4, where erfc < 1.6e-8.  The reciprocal runs
+// on the FMA pipe (rcp_1_2); one special-function op (the exponential) per
+// value.  Absolute error of the whole function below 5e-7.
 __device__ __forceinline__ float gelu_erf(float v) {
-    const float z = fabsf(v) * 0.70710678118654752f;
-    const float t = __fdividef(1.0f, fmaf(0.3275911f, z, 1.0f));
+    const float z = fminf(fabsf(v) * 0.70710678118654752f, 4.0f);
+    const float t = rcp_1_2(fmaf(0.3275911f, z, 1.0f));
     float poly = fmaf(t, 1.061405429f, -1.453152027f);
     poly = fmaf(t, poly, 1.421413741f);
     poly = fmaf(t, poly, -0.284496736f);
     poly = fmaf(t, poly, 0.254829592f);
     const float q = poly * t * __expf(-z * z);
-    return 0.5f * v * (v >= 0.f ? 2.0f - q : q);
+    return (0.5f * v) * (v >= 0.f ? 2.0f - q : q);
 }
 __device__ __forceinline__ float silu_f(float g) { return g / (1.0f + __expf(-g)); }
 
+__device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+}
+
+__device__ __forceinline__ void store_bf16x16(__nv_bfloat16 *dst, const uint32_t (&pk)[8], int n0, int n_valid) {
+    if (n0 + 16 <= n_valid) {
+        reinterpret_cast<uint4 *>(dst)[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        reinterpret_cast<uint4 *>(dst)[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+    } else {
+#pragma unroll
+        for (int k = 0; k < 16; ++k)
+            if (n0 + k < n_valid)
+                dst[k] = __ushort_as_bfloat16(static_cast<unsigned short>((pk[k >> 1] >> ((k & 1) * 16)) & 0xffffu));
+    }
+}
+
+// Epilogue of one accumulator tile for the calling warp.  The warp reads TMEM
+// lanes 32*(warp%4).. (this thread: output row `row`) from `tbase`; column
+// group `grp` (of kEpiGroups) of the tile is its share, in 16-column chunks.
+// Rows at or beyond row_limit are not stored.  Every lane executes the TMEM
+// loads (they are warp-wide).
+template <int BN, int EPI>
+__device__ __forceinline__ void epilogue_tile(const Params &p, const TileCoord &c, int row, int row_limit,
+                                              uint32_t tbase, int grp) {
+    const bool row_ok = row < row_limit;
+    if (EPI == EPI_SWIGLU) {
+        constexpr int kOutCols = BN / 2;                  // h columns per tile
+        constexpr int kPerGroup = kOutCols / kEpiGroups;  // per epilogue warp
+        __nv_bfloat16 *out = static_cast<__nv_bfloat16 *>(p.out);
+#pragma unroll 1
+        for (int cc = 0; cc < kPerGroup; cc += 16) {
+            const int col = grp * kPerGroup + cc;
+            uint32_t rg[16], ru[16];
+            tmem_ld_32x32b_x16(tbase + col, rg);
+            tmem_ld_32x32b_x16(tbase + kOutCols + col, ru);
+            tmem_ld_wait();
+            if (!row_ok) continue;
+            const int n0 = c.nt * kOutCols + col;
+            uint32_t pk[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                const float h0 = silu_f(__uint_as_float(rg[2 * k])) * __uint_as_float(ru[2 * k]);
+                const float h1 = silu_f(__uint_as_float(rg[2 * k + 1])) * __uint_as_float(ru[2 * k + 1]);
+                pk[k] = pack_bf16x2(h0, h1);
+            }
+            store_bf16x16(out + (int64_t)row * p.ldo + n0, pk, n0, p.n_valid);
+        }
+        return;
+    }
+    constexpr int kPerGroup = BN / kEpiGroups;
+    int slot = -1;
+    float gw = 0.f;
+    if (EPI == EPI_SCATTER && row_ok) {
+        slot = p.perm_slot[row];
+        if (slot >= 0) gw = p.gate_w[slot];
+    }
+#pragma unroll 1
+    for (int cc = 0; cc < kPerGroup; cc += 16) {
+        const int col = grp * kPerGroup + cc;
+        uint32_t r[16];
+        tmem_ld_32x32b_x16(tbase + col, r);
+        tmem_ld_wait();
+        const int n0 = c.nt * BN + col;
+        if (n0 >= p.n_valid || !row_ok) continue;
+        if (EPI == EPI_SCATTER && slot < 0) continue;
+        const bool full_chunk = n0 + 16 <= p.n_valid;
+        float v[16];
+#pragma unroll
+        for (int k = 0; k < 16; ++k) v[k] = __uint_as_float(r[k]);
+        if (p.bias) {
+            const float *bias = p.bias + (int64_t)c.g * p.n_valid + n0;
+            if (full_chunk) {
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const float4 b4 = __ldg(reinterpret_cast<const float4 *>(bias) + u);
+                    v[4 * u] += b4.x; v[4 * u + 1] += b4.y; v[4 * u + 2] += b4.z; v[4 * u + 3] += b4.w;
+                }
+            } else {
+#pragma unroll
+                for (int k = 0; k < 16; ++k)
+                    if (n0 + k < p.n_valid) v[k] += __ldg(bias + k);
+            }
+        }
+        if (EPI == EPI_GELU) {
+            uint32_t pk[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) pk[k] = pack_bf16x2(gelu_erf(v[2 * k]), gelu_erf(v[2 * k + 1]));
+            store_bf16x16(static_cast<__nv_bfloat16 *>(p.out) + (int64_t)row * p.ldo + n0, pk, n0, p.n_valid);
+        } else if (EPI == EPI_SCATTER) {
+            float *dst = static_cast<float *>(p.out) + (int64_t)slot * p.ldo + n0;
+            if (full_chunk) {
+#pragma unroll
+                for (int u = 0; u < 4; ++u)
+                    reinterpret_cast<float4 *>(dst)[u] =
+                        make_float4(gw * v[4 * u], gw * v[4 * u + 1], gw * v[4 * u + 2], gw * v[4 * u + 3]);
+            } else {
+#pragma unroll
+                for (int k = 0; k < 16; ++k)
+                    if (n0 + k < p.n_valid) dst[k] = gw * v[k];
+            }
+        } else {  // EPI_LOGITS
+            float *dst = static_cast<float *>(p.out) + (int64_t)row * p.ldo + n0;
+#pragma unroll
+            for (int k = 0; k < 16; ++k)
+                if (n0 + k < p.n_valid) dst[k] = v[k];
+        }
+    }
+}
+
+// =====================================================================================
+// One CTA per 128-row tile.
+// =====================================================================================
 template <int BN, int EPI>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -256,122 +458,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ------------------------------------------------------------ epilogue
         const int ew = warp - 2;
         const int q = warp & 3;
-        const int half = ew >> 2;
+        const int grp = ew >> 2;
         const int r_in_tile = q * 32 + lane;
         int local = 0;
         for (int i = blockIdx.x; i < total; i += gridDim.x, ++local) {
             const int a = local & 1;
             const uint32_t aph = (local >> 1) & 1;
             const TileCoord c = decode_tile(i, rowoff, G, p.n_tiles, dense_mtiles);
-            if (!mbar_wait(&tfull[a], aph, p.timeout_ns)) break;
+            // warp-uniform decision: the TMEM loads below are warp-collective
+            if (!__all_sync(0xffffffffu, mbar_wait(&tfull[a], aph, p.timeout_ns))) break;
             tc_fence_after();
-            const int row = c.row0 + r_in_tile;
-            const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + a * BN;
-
-            if (EPI == EPI_SWIGLU) {
-                constexpr int kOutCols = BN / 2;             // h columns per tile
-                constexpr int kPerHalf = kOutCols / 2;       // per epilogue warp
-                __nv_bfloat16 *out = static_cast<__nv_bfloat16 *>(p.out);
-#pragma unroll 1
-                for (int cc = 0; cc < kPerHalf; cc += 32) {
-                    const int col = half * kPerHalf + cc;
-                    uint32_t rg[32], ru[32];
-                    tmem_ld_32x32b_x32(tbase + col, rg);
-                    tmem_ld_32x32b_x32(tbase + kOutCols + col, ru);
-                    tmem_ld_wait();
-                    const int n0 = c.nt * kOutCols + col;
-                    uint32_t pk[16];
-#pragma unroll
-                    for (int k = 0; k < 16; ++k) {
-                        const float h0 = silu_f(__uint_as_float(rg[2 * k])) * __uint_as_float(ru[2 * k]);
-                        const float h1 = silu_f(__uint_as_float(rg[2 * k + 1])) * __uint_as_float(ru[2 * k + 1]);
-                        pk[k] = pack_bf16x2(h0, h1);
-                    }
-                    __nv_bfloat16 *dst = out + (int64_t)row * p.ldo + n0;
-                    if (n0 + 32 <= p.n_valid) {
-#pragma unroll
-                        for (int v = 0; v < 4; ++v)
-                            reinterpret_cast<uint4 *>(dst)[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
-                    } else {
-#pragma unroll
-                        for (int k = 0; k < 32; ++k)
-                            if (n0 + k < p.n_valid)
-                                dst[k] = __ushort_as_bfloat16(static_cast<unsigned short>((pk[k >> 1] >> ((k & 1) * 16)) & 0xffffu));
-                    }
-                }
-            } else {
-                constexpr int kPerHalf = BN / 2;
-                int slot = -1;
-                float gw = 0.f;
-                if (EPI == EPI_SCATTER) {
-                    slot = p.perm_slot[row];
-                    if (slot >= 0) gw = p.gate_w[slot];
-                }
-#pragma unroll 1
-                for (int cc = 0; cc < kPerHalf; cc += 32) {
-                    const int col = half * kPerHalf + cc;
-                    uint32_t r[32];
-                    tmem_ld_32x32b_x32(tbase + col, r);
-                    tmem_ld_wait();
-                    const int n0 = c.nt * BN + col;
-                    if (n0 >= p.n_valid) continue;
-                    const bool full_chunk = n0 + 32 <= p.n_valid;
-                    float v[32];
-#pragma unroll
-                    for (int k = 0; k < 32; ++k) v[k] = __uint_as_float(r[k]);
-                    if (p.bias) {
-                        const float *bias = p.bias + (int64_t)c.g * p.n_valid + n0;
-                        if (full_chunk) {
-#pragma unroll
-                            for (int u = 0; u < 8; ++u) {
-                                const float4 b4 = __ldg(reinterpret_cast<const float4 *>(bias) + u);
-                                v[4 * u] += b4.x; v[4 * u + 1] += b4.y; v[4 * u + 2] += b4.z; v[4 * u + 3] += b4.w;
-                            }
-                        } else {
-#pragma unroll
-                            for (int k = 0; k < 32; ++k)
-                                if (n0 + k < p.n_valid) v[k] += __ldg(bias + k);
-                        }
-                    }
-                    if (EPI == EPI_GELU) {
-                        __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(p.out) + (int64_t)row * p.ldo + n0;
-                        uint32_t pk[16];
-#pragma unroll
-                        for (int k = 0; k < 16; ++k) pk[k] = pack_bf16x2(gelu_erf(v[2 * k]), gelu_erf(v[2 * k + 1]));
-                        if (full_chunk) {
-#pragma unroll
-                            for (int u = 0; u < 4; ++u)
-                                reinterpret_cast<uint4 *>(dst)[u] = make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
-                        } else {
-#pragma unroll
-                            for (int k = 0; k < 32; ++k)
-                                if (n0 + k < p.n_valid)
-                                    dst[k] = __ushort_as_bfloat16(static_cast<unsigned short>((pk[k >> 1] >> ((k & 1) * 16)) & 0xffffu));
-                        }
-                    } else if (EPI == EPI_SCATTER) {
-                        if (slot >= 0) {
-                            float *dst = static_cast<float *>(p.out) + (int64_t)slot * p.ldo + n0;
-                            if (full_chunk) {
-#pragma unroll
-                                for (int u = 0; u < 8; ++u)
-                                    reinterpret_cast<float4 *>(dst)[u] =
-                                        make_float4(gw * v[4 * u], gw * v[4 * u + 1], gw * v[4 * u + 2], gw * v[4 * u + 3]);
-                            } else {
-#pragma unroll
-                                for (int k = 0; k < 32; ++k)
-                                    if (n0 + k < p.n_valid) dst[k] = gw * v[k];
-                            }
-                        }
-                    } else {  // EPI_LOGITS
-                        if (row < p.dense_rows) {
-                            float *dst = static_cast<float *>(p.out) + (int64_t)row * p.ldo + n0;
-#pragma unroll
-                            for (int k = 0; k < 32; ++k)
-                                if (n0 + k < p.n_valid) dst[k] = v[k];
-                        }
-                    }
-                }
-            }
+            const int row_limit = rowoff ? s_rowoff[c.g + 1] : p.dense_rows;
+            epilogue_tile<BN, EPI>(p, c, c.row0 + r_in_tile, row_limit,
+                                   tmem_base + (static_cast<uint32_t>(q * 32) << 16) + a * BN, grp);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&tempty[a]);
@@ -382,6 +481,279 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem_base, S::kTmemCols);
+    }
+}
+
+// =====================================================================================
+// Two CTAs (one cluster) per 256-row x 256-column tile.
+// =====================================================================================
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ uint32_t cluster_id_x() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%clusterid.x;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ uint32_t nclusters_x() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%nclusterid.x;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ void cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// shared::cluster address of the variable at shared::cta address `local` in CTA `rank`
+__device__ __forceinline__ uint32_t mapa_shared(uint32_t local, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local), "r"(rank));
+    return r;
+}
+// Allocation shared by the CTA pair: one warp of each CTA executes it.
+__device__ __forceinline__ void tmem_alloc2(uint32_t *slot, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(slot)),
+                 "r"(ncols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc2(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void tc_mma2_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                             uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+// Arrive once on the barrier at the offset of `bar` in every CTA of cta_mask
+// when all tcgen05 operations issued so far by this thread have completed.
+__device__ __forceinline__ void tc_commit2_mc(uint64_t *bar, uint16_t cta_mask) {
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+            smem_u32(bar)),
+        "h"(cta_mask)
+        : "memory");
+}
+__device__ __forceinline__ void tc_commit2(uint64_t *bar) {
+    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+                 : "memory");
+}
+// TMA load into this CTA's shared memory; completion is counted on the barrier
+// at shared::cluster address `mbar_cluster` (the leader CTA's barrier).
+__device__ __forceinline__ void tma_load_2d_pair(const CUtensorMap *map, uint32_t mbar_cluster, void *smem_dst,
+                                                 int32_t c0, int32_t c1) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, "
+        "%4}], [%2];" ::"r"(smem_u32(smem_dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(mbar_cluster), "r"(c0), "r"(c1)
+        : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t bar_cluster) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+// Bounded wait with cluster-scope acquire (arrivals come from the peer CTA).
+__device__ __forceinline__ bool mbar_wait_cluster(uint64_t *bar, uint32_t parity, uint64_t timeout_ns) {
+    if (mbar_try_wait_cluster(bar, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    while (true) {
+#pragma unroll 1
+        for (int i = 0; i < 64; ++i)
+            if (mbar_try_wait_cluster(bar, parity)) return true;
+        if (globaltimer_ns() - t0 > timeout_ns) {
+            set_status(kStatusTimeout);
+            return false;
+        }
+    }
+}
+
+template <int EPI>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+    grouped_gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                            const Params p) {
+    using S = Shape2;
+    constexpr int BN = 256;
+    constexpr int kStages = S::kStages;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *sA = smem;
+    uint8_t *sB = smem + kStages * S::kABytes;
+    uint64_t *full = reinterpret_cast<uint64_t *>(sB + kStages * S::kBBytes);
+    uint64_t *empty = full + kStages;
+    uint64_t *tfull = empty + kStages;
+    uint64_t *tempty = tfull + 2;
+    uint64_t *drain = tempty + 2;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
+    int *s_rowoff = reinterpret_cast<int *>(tmem_slot + 4);
+    const int G = p.num_groups;
+    int *s_units = s_rowoff + (G + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();
+    const int cid = (int)cluster_id_x(), ncl = (int)nclusters_x();
+    if (p.row_offsets) {
+        for (int i = threadIdx.x; i <= G; i += blockDim.x) s_rowoff[i] = p.row_offsets[i];
+        __syncthreads();
+        if (warp == 0) {   // 256-row units before each group
+            int carry = 0;
+            for (int g0 = 0; g0 <= G; g0 += 32) {
+                const int g = g0 + lane;
+                const int u = g < G ? (s_rowoff[g + 1] - s_rowoff[g] + 2 * BM - 1) / (2 * BM) : 0;
+                int incl = u;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const int n = __shfl_up_sync(0xffffffffu, incl, o);
+                    if (lane >= o) incl += n;
+                }
+                if (g <= G) s_units[g] = carry + incl - u;
+                carry += __shfl_sync(0xffffffffu, incl, 31);
+            }
+        }
+    }
+    if (warp == 0 && lane == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(&tfull[a], 1);
+            mbar_init(&tempty[a], 2 * kEpiWarps);
+        }
+        mbar_init(drain, 1);
+        fence_mbar_init();
+        tma_prefetch_desc(&tmA);
+        tma_prefetch_desc(&tmB);
+    }
+    if (warp == 1) tmem_alloc2(tmem_slot, S::kTmemCols);
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync();   // both CTAs' barriers initialised and TMEM allocated before any cross-CTA traffic
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    const int *rowoff = p.row_offsets ? s_rowoff : nullptr;
+    const int dense_units = (p.dense_rows + 2 * BM - 1) / (2 * BM);
+    const int units = rowoff ? s_units[G] : dense_units;
+    const int total = units * p.n_tiles;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ TMA producer (both CTAs)
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            bool ok = true;
+            for (int i = cid; i < total && ok; i += ncl) {
+                const TileCoord c = decode_unit_tile(i, rowoff, s_units, G, p.n_tiles, dense_units);
+                const int arow = c.row0 + (int)rank * BM;
+                int brow;
+                if (EPI == EPI_SWIGLU)   // CTA 0: 128 gate rows, CTA 1: the matching 128 up rows
+                    brow = c.g * p.b_group_rows + c.nt * (BN / 2) + (rank ? p.b_up_offset : 0);
+                else
+                    brow = c.g * p.b_group_rows + c.nt * BN + (int)rank * (BN / 2);
+                for (int kb = 0; kb < p.num_k_blocks; ++kb) {
+                    if (!mbar_wait(&empty[stage], phase ^ 1, p.timeout_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * (S::kABytes + S::kBBytes));
+                    const uint32_t leader_full = mapa_shared(smem_u32(&full[stage]), 0);
+                    tma_load_2d_pair(&tmA, leader_full, sA + stage * S::kABytes, kb * BK, arow);
+                    tma_load_2d_pair(&tmB, leader_full, sB + stage * S::kBBytes, kb * BK, brow);
+                    if (++stage == kStages) {
+                        stage = 0;
+                        phase ^= 1;
+                    }
+                }
+            }
+            if (!ok) {
+                const uint64_t t0 = globaltimer_ns();
+                while (globaltimer_ns() - t0 < 1000000ull) {
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer (leader CTA only)
+        if (lane == 0 && rank == 0) {
+            constexpr uint32_t idesc = idesc_bf16_f32(2 * BM, BN);
+            int stage = 0;
+            uint32_t phase = 0;
+            int local = 0;
+            bool ok = true;
+            for (int i = cid; i < total && ok; i += ncl, ++local) {
+                const int a = local & 1;
+                const uint32_t aph = (local >> 1) & 1;
+                if (!mbar_wait_cluster(&tempty[a], aph ^ 1, p.timeout_ns)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + a * BN;
+                for (int kb = 0; kb < p.num_k_blocks; ++kb) {
+                    if (!mbar_wait(&full[stage], phase, p.timeout_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint64_t adesc = smem_desc_sw128(smem_u32(sA + stage * S::kABytes));
+                    const uint64_t bdesc = smem_desc_sw128(smem_u32(sB + stage * S::kBBytes));
+#pragma unroll
+                    for (int k = 0; k < BK / 16; ++k)
+                        tc_mma2_bf16(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, (kb | k) != 0 ? 1u : 0u);
+                    tc_commit2_mc(&empty[stage], 0x3);
+                    if (++stage == kStages) {
+                        stage = 0;
+                        phase ^= 1;
+                    }
+                }
+                if (ok) tc_commit2_mc(&tfull[a], 0x3);
+            }
+            if (!ok) {
+                tc_commit2(drain);
+                mbar_wait(drain, 0, p.timeout_ns);
+            }
+        }
+    } else {
+        // ------------------------------------------------------------ epilogue (both CTAs)
+        const int ew = warp - 2;
+        const int q = warp & 3;
+        const int grp = ew >> 2;
+        const int r_in_tile = q * 32 + lane;
+        int local = 0;
+        for (int i = cid; i < total; i += ncl, ++local) {
+            const int a = local & 1;
+            const uint32_t aph = (local >> 1) & 1;
+            const TileCoord c = decode_unit_tile(i, rowoff, s_units, G, p.n_tiles, dense_units);
+            // warp-uniform decision: the TMEM loads below are warp-collective
+            if (!__all_sync(0xffffffffu, mbar_wait(&tfull[a], aph, p.timeout_ns))) break;
+            tc_fence_after();
+            const int row_limit = rowoff ? s_rowoff[c.g + 1] : p.dense_rows;
+            epilogue_tile<BN, EPI>(p, c, c.row0 + (int)rank * BM + r_in_tile, row_limit,
+                                   tmem_base + (static_cast<uint32_t>(q * 32) << 16) + a * BN, grp);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_remote(mapa_shared(smem_u32(&tempty[a]), 0));
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync();   // the leader's last MMAs read this CTA's shared memory and TMEM
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc2(tmem_base, S::kTmemCols);
     }
 }
 

@@ -343,7 +343,8 @@ __global__ void __launch_bounds__(1024) scan_kernel(const int *__restrict__ chun
                                                     int64_t expect_total, int *__restrict__ chunk_base,
                                                     int *__restrict__ counts, int *__restrict__ offsets,
                                                     int *__restrict__ row_offsets, int *__restrict__ perm_slot,
-                                                    int *__restrict__ counts_out, unsigned *__restrict__ counter) {
+                                                    int *__restrict__ counts_out, unsigned *__restrict__ counter,
+                                                    int *__restrict__ live, int *__restrict__ n_live) {
     constexpr int CPL = 16;
     __shared__ int s_cnt[1024];
     __shared__ int s_row[1025];
@@ -412,6 +413,16 @@ __global__ void __launch_bounds__(1024) scan_kernel(const int *__restrict__ chun
             s_row[N] = pcarry;
             if ((int64_t)carry != expect_total) set_status(kStatusBounds);
         }
+        // ascending list of the experts that received tokens
+        int nl = 0;
+        for (int e0 = 0; e0 < N; e0 += 32) {
+            const int ee = e0 + lane;
+            const bool has = ee < N && s_cnt[ee] > 0;
+            const unsigned m = __ballot_sync(0xffffffffu, has);
+            if (has) live[nl + __popc(m & lanemask_lt())] = ee;
+            nl += __popc(m);
+        }
+        if (lane == 0) *n_live = nl;
     }
     __syncthreads();
     for (int ee = warp; ee < N; ee += 32) {
@@ -425,19 +436,23 @@ __global__ void __launch_bounds__(1024) scan_kernel(const int *__restrict__ chun
 // expert (ascending token, then slot), its permuted row, the two index maps,
 // and the copy of the token row into the expert-contiguous buffer.
 // ---------------------------------------------------------------------------
+// Grid: (chunks, split).  Every block of a chunk ranks the chunk's entries
+// (cheap, identical results); block (c, 0) writes the index maps and block
+// (c, s) copies the entries f with f % split == s.
 template <typename Tin>
 __global__ void __launch_bounds__(256) permute_kernel(const Tin *__restrict__ x, int T, int D, int K, int N,
-                                                      const int *__restrict__ topk_idx,
+                                                      int chunk_tokens, const int *__restrict__ topk_idx,
                                                       const int *__restrict__ chunk_base,
                                                       const int *__restrict__ row_offsets, int *__restrict__ perm_slot,
                                                       int *__restrict__ slot_row, Tin *__restrict__ x_perm) {
     extern __shared__ int s_perm[];
     int *s_run = s_perm;            // [N]
-    int *s_dest = s_perm + N;       // [kChunk * K]
+    int *s_dest = s_perm + N;       // [chunk_tokens * K]
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int c = blockIdx.x;
-    const int t_begin = c * kChunk;
-    const int t_end = min(T, t_begin + kChunk);
+    const bool writer = blockIdx.y == 0;
+    const int t_begin = c * chunk_tokens;
+    const int t_end = min(T, t_begin + chunk_tokens);
     const int n_entries = (t_end - t_begin) * K;
     const int64_t f0 = (int64_t)t_begin * K;
     for (int e = tid; e < N; e += blockDim.x) s_run[e] = row_offsets[e] + chunk_base[(size_t)c * N + e];
@@ -460,11 +475,9 @@ __global__ void __launch_bounds__(256) permute_kernel(const Tin *__restrict__ x,
             if (f < n_entries) {
                 const int dest = e >= 0 ? base_row + rank : -1;
                 s_dest[f] = dest;
-                if (dest >= 0) {
-                    perm_slot[dest] = (int)(f0 + f);
+                if (writer) {
+                    if (dest >= 0) perm_slot[dest] = (int)(f0 + f);
                     slot_row[f0 + f] = dest;
-                } else {
-                    slot_row[f0 + f] = -1;
                 }
             }
         }
@@ -473,7 +486,7 @@ __global__ void __launch_bounds__(256) permute_kernel(const Tin *__restrict__ x,
     // one row per warp at a time, four 16-byte vectors in flight per lane
     constexpr int VEC = 16 / sizeof(Tin);
     const int nvec = D / VEC;
-    for (int f = warp; f < n_entries; f += 8) {
+    for (int f = blockIdx.y + gridDim.y * warp; f < n_entries; f += 8 * gridDim.y) {
         const int dest = s_dest[f];
         if (dest < 0) continue;
         const int64_t t = (f0 + f) / K;
@@ -550,7 +563,7 @@ __device__ void aux_finalize_block(const float *__restrict__ part_p, const float
         float p = 0.f, im = 0.f;
         int c = 0;
         if (tid / Q < nt / Q && e < N) {
-#pragma unroll 4
+#pragma unroll 16
             for (int bb = q; bb < nblk; bb += Q) {
                 p += __ldcg(part_p + (size_t)bb * N + e);
                 im += __ldcg(part_imp + (size_t)bb * N + e);
@@ -579,22 +592,24 @@ __device__ void aux_finalize_block(const float *__restrict__ part_p, const float
     if (tid == 0 && out.scalars) {
         double sw = 0.0, ss = 0.0, mi = 0.0, mc = 0.0;
         const double tk = (double)T * (double)K;
+        const double inv_tk = tk > 0 ? 1.0 / tk : 0.0;
+        const double inv_n = 1.0 / N;
         for (int e = 0; e < N; ++e) {
-            const double f = tk > 0 ? f_c[e] / tk : 0.0;
+            const double f = f_c[e] * inv_tk;
             sw += f * f_p[e];
             ss += f * f;
             mi += f_i[e];
             mc += f_c[e];
         }
-        mi /= N;
-        mc /= N;
+        mi *= inv_n;
+        mc *= inv_n;
         double vi = 0.0, vc = 0.0;
         for (int e = 0; e < N; ++e) {
             vi += (f_i[e] - mi) * (f_i[e] - mi);
             vc += (f_c[e] - mc) * (f_c[e] - mc);
         }
-        vi /= N;
-        vc /= N;
+        vi *= inv_n;
+        vc *= inv_n;
         out.scalars[0] = (float)(N * sw);
         out.scalars[1] = (float)(N * ss);
         out.scalars[2] = mi == 0.0 ? 0.f : (float)(vi / (mi * mi));
@@ -644,8 +659,9 @@ __global__ void __launch_bounds__(256) aux_small_kernel(const float *__restrict_
             s[e] = e < N ? expf(s[e] - mx) : 0.f;
             z += s[e];
         }
+        const float inv_z = 1.0f / z;
 #pragma unroll
-        for (int e = 0; e < NP; ++e) p[e] = s[e] / z;
+        for (int e = 0; e < NP; ++e) p[e] = s[e] * inv_z;
         for (int j = 0; j < K; ++j) {
             const int ej = topk_idx[(size_t)t * K + j];
             const float wj = topk_w[(size_t)t * K + j];

@@ -1,0 +1,550 @@
+// moe_router_tc.cuh -- routers for bf16 layers with N <= 256 (tensor cores) and
+// for few tokens (N <= 32), each with top-k, statistics and the dispatch scan
+// in one launch.
+//
+// Routing follows "MoE(Mixture of Experts)", section (2), Route: scores x W_g
+// (+ b_g), the K best experts of a stable descending sort (equal scores keep
+// ascending expert index), and the softmax over only the kept scores shifted
+// by the best one -- softmax(KeepTopK(H, k)) of the Shazeer article (qiita),
+// gating section, inference form.  Statistics follow the Shazeer article's
+// load-balancing section and the Switch-style loss: per expert the mean of the
+// full N-way softmax, the importance (sum of gate weights) and the counts.
+//
+// router_tc_kernel   one CTA per tile of 128 tokens: tcgen05.mma computes the
+//   128 x N logits (fp32 accumulation of exact bf16 products, operands staged by
+//   TMA); each of 128 epilogue threads owns one token (one TMEM lane), keeps the
+//   K best (value, index) pairs in a static insertion network, computes the
+//   gate weights and its full-softmax probabilities; the tile's per-expert
+//   probability sums are reduced in a fixed order (lanes, then warps), its
+//   counts and gate-weight sums with shared-memory atomics on integers (gate
+//   weights in 2^-32 fixed point), which are exact and order-independent.
+// router_few_kernel  one block per token (T <= 64, N <= 32): every thread
+//   streams its rows of W_g with all loads in flight, warps reduce-scatter the
+//   partial scores, warp 0 selects the top k; the token's probabilities, gate
+//   weights and counts are its partials.
+// In both, the last block to finish (atomic ticket) turns the per-tile (or
+// per-token) partials into the dispatch tables -- per tile and expert the first
+// row of its tokens inside the expert's segment, per-expert counts and offsets,
+// segment starts padded to 128 rows, padding slots -1, the ascending list of
+// experts with tokens -- and the statistics, scalars in double precision.  No
+// float atomics anywhere: results do not depend on scheduling.
+#pragma once
+
+#include "moe_common.cuh"
+#include "moe_route.cuh"
+
+namespace moe {
+namespace rtc {
+
+constexpr int BM = 128;   // tokens per tile (= dispatch chunk)
+constexpr int BK = 64;
+constexpr int kThreads = 192;   // warp 0 TMA, warp 1 MMA, warps 2..5 one token per thread
+constexpr double kImpScale = 4294967296.0;   // gate weights summed in 2^-32 fixed point
+
+struct Params {
+    int T, D, N, K, np;                  // np: N rounded up to the MMA width
+    const float *bg;                     // [N] or nullptr
+    float *logits;                       // [T, N]
+    int *topk_idx;                       // [T, K]
+    float *topk_w;                       // [T, K]
+    int *tile_counts;                    // [tiles, N]
+    float *tile_p;                       // [tiles, N]
+    unsigned long long *tile_imp;        // [tiles, N] fixed point
+    unsigned *ticket;                    // zero at launch
+    // dispatch tables (written by the last block)
+    int *chunk_base;                     // [tiles, N] first row (relative to the expert's segment) of the tile's tokens
+    int *counts;                         // [N]
+    int *offsets;                        // [N+1]
+    int *row_offsets;                    // [N+1]
+    int *perm_slot;                      // padding rows -> -1
+    int *live;                           // [N]
+    int *n_live;
+    int *counts_out;                     // [N] or nullptr (moe_route)
+    // statistics (each may be nullptr)
+    int *aux_counts;
+    float *aux_importance, *aux_p_mean, *aux_scalars;
+    uint64_t timeout_ns;
+};
+
+// Scratch of the finalisation (shared memory, up to 256 experts, 256 threads).
+struct FinalScratch {
+    int cnt[256];
+    float pm[256];
+    float im[256];
+    int row[257];
+    int q_cnt[256];
+    float q_p[256];
+    unsigned long long q_i[256];
+};
+
+// Executed by every thread of the last block.  Per expert e, Q threads take
+// contiguous tile ranges; the range totals are combined in range order, so the
+// float sums have a fixed order; counts and fixed-point gate weights are exact.
+__device__ void finalize_tables(const Params &p, int ntiles, FinalScratch &f) {
+    const int N = p.N, nt = blockDim.x, tid = threadIdx.x;
+    const int warp = tid >> 5, lane = tid & 31;
+    int Q = nt / N;
+    Q = Q < 1 ? 1 : (Q > 32 ? 32 : Q);
+    const int epp = nt / Q;                       // experts per pass
+    const int R = (ntiles + Q - 1) / Q;           // tiles per thread
+    for (int e0 = 0; e0 < N; e0 += epp) {
+        const int e = e0 + tid / Q, q = tid % Q;
+        const bool act = tid < epp * Q && e < N;
+        const int c0 = q * R, c1 = min(ntiles, c0 + R);
+        int cnt = 0;
+        float ps = 0.f;
+        unsigned long long im = 0;
+        if (act) {
+#pragma unroll 8
+            for (int c = c0; c < c1; ++c) {
+                cnt += __ldcg(p.tile_counts + (int64_t)c * N + e);
+                ps += __ldcg(p.tile_p + (int64_t)c * N + e);
+                im += __ldcg(p.tile_imp + (int64_t)c * N + e);
+            }
+        }
+        f.q_cnt[tid] = cnt;
+        f.q_p[tid] = ps;
+        f.q_i[tid] = im;
+        __syncthreads();
+        int base = 0;
+        if (act) {
+            for (int j = 0; j < q; ++j) base += f.q_cnt[tid - q + j];   // tiles before this range
+            if (q == 0) {
+                int tc = 0;
+                float tp = 0.f;
+                unsigned long long ti = 0;
+                for (int j = 0; j < Q; ++j) { tc += f.q_cnt[tid + j]; tp += f.q_p[tid + j]; ti += f.q_i[tid + j]; }
+                f.cnt[e] = tc;
+                f.pm[e] = p.T > 0 ? tp / (float)p.T : 0.f;
+                f.im[e] = (float)((double)ti / kImpScale);
+            }
+            for (int c = c0; c < c1; ++c) {
+                p.chunk_base[(int64_t)c * N + e] = base;
+                base += __ldcg(p.tile_counts + (int64_t)c * N + e);
+            }
+        }
+        __syncthreads();
+    }
+    for (int e = tid; e < N; e += nt) {
+        p.counts[e] = f.cnt[e];
+        if (p.counts_out) p.counts_out[e] = f.cnt[e];
+        if (p.aux_counts) p.aux_counts[e] = f.cnt[e];
+        if (p.aux_p_mean) p.aux_p_mean[e] = f.pm[e];
+        if (p.aux_importance) p.aux_importance[e] = f.im[e];
+    }
+    if (warp == 0) {
+        int carry = 0, pcarry = 0, nl = 0;
+        for (int e0 = 0; e0 < N; e0 += 32) {
+            const int e = e0 + lane;
+            const int c = e < N ? f.cnt[e] : 0;
+            const int pc = (c + kRowAlign - 1) / kRowAlign * kRowAlign;
+            int ic = c, ip = pc;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int n1 = __shfl_up_sync(0xffffffffu, ic, o);
+                const int n2 = __shfl_up_sync(0xffffffffu, ip, o);
+                if (lane >= o) { ic += n1; ip += n2; }
+            }
+            if (e < N) {
+                p.offsets[e] = carry + ic - c;
+                p.row_offsets[e] = pcarry + ip - pc;
+                f.row[e] = pcarry + ip - pc;
+            }
+            const unsigned m = __ballot_sync(0xffffffffu, c > 0);
+            if (c > 0) p.live[nl + __popc(m & lanemask_lt())] = e;
+            nl += __popc(m);
+            carry += __shfl_sync(0xffffffffu, ic, 31);
+            pcarry += __shfl_sync(0xffffffffu, ip, 31);
+        }
+        if (lane == 0) {
+            p.offsets[N] = carry;
+            p.row_offsets[N] = pcarry;
+            f.row[N] = pcarry;
+            *p.n_live = nl;
+            if ((int64_t)carry != (int64_t)p.T * p.K) set_status(kStatusBounds);
+        }
+    } else if (warp == 1 && p.aux_scalars) {
+        // f_e = counts_e / (T K); switch = N sum f P; simple = N sum f^2;
+        // CV^2 = popvar / mean^2; lanes take experts lane, lane+32, ...; xor tree in double
+        const double tk = (double)p.T * (double)p.K;
+        const double inv_tk = tk > 0 ? 1.0 / tk : 0.0;
+        double sw = 0.0, ss = 0.0, si = 0.0, sc = 0.0;
+        for (int e = lane; e < N; e += 32) {
+            const double fe = f.cnt[e] * inv_tk;
+            sw += fe * f.pm[e];
+            ss += fe * fe;
+            si += f.im[e];
+            sc += f.cnt[e];
+        }
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) {
+            sw += __shfl_xor_sync(0xffffffffu, sw, o);
+            ss += __shfl_xor_sync(0xffffffffu, ss, o);
+            si += __shfl_xor_sync(0xffffffffu, si, o);
+            sc += __shfl_xor_sync(0xffffffffu, sc, o);
+        }
+        const double mi = si / N, mc = sc / N;
+        double vi = 0.0, vc = 0.0;
+        for (int e = lane; e < N; e += 32) {
+            vi += (f.im[e] - mi) * (f.im[e] - mi);
+            vc += (f.cnt[e] - mc) * (f.cnt[e] - mc);
+        }
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) {
+            vi += __shfl_xor_sync(0xffffffffu, vi, o);
+            vc += __shfl_xor_sync(0xffffffffu, vc, o);
+        }
+        vi /= N;
+        vc /= N;
+        if (lane == 0) {
+            p.aux_scalars[0] = (float)(N * sw);
+            p.aux_scalars[1] = (float)(N * ss);
+            p.aux_scalars[2] = mi == 0.0 ? 0.f : (float)(vi / (mi * mi));
+            p.aux_scalars[3] = mc == 0.0 ? 0.f : (float)(vc / (mc * mc));
+        }
+    }
+    __syncthreads();
+    for (int e = warp; e < N; e += nt / 32) {
+        const int start = f.row[e] + f.cnt[e], end = f.row[e + 1];
+        for (int rr = start + lane; rr < end; rr += 32) p.perm_slot[rr] = -1;
+    }
+}
+
+// True in every thread of the block that finished last.
+__device__ __forceinline__ bool last_block(unsigned *ticket, int *s_flag) {
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) *s_flag = atomicAdd(ticket, 1u) == gridDim.x - 1;
+    __syncthreads();
+    const bool last = *s_flag != 0;
+    if (last) __threadfence();
+    return last;
+}
+
+template <int NP>
+struct Shape {
+    static constexpr uint32_t kABytes = BM * BK * 2;
+    static constexpr uint32_t kBBytes = NP * BK * 2;
+    static constexpr uint32_t kStageBytes = kABytes + kBBytes;
+    static constexpr int kStages0 = (160 * 1024) / (int)kStageBytes;
+    static constexpr int kStages = kStages0 > 8 ? 8 : kStages0;
+    static constexpr uint32_t kTmemCols = NP <= 32 ? 32 : NP <= 64 ? 64 : NP <= 128 ? 128 : 256;
+    // ring + per-warp probability rows + tile counters + finalisation scratch + barriers
+    static constexpr size_t kSmem = 1024 + (size_t)kStages * kStageBytes + 4 * 256 * 4 + 256 * 4 + 256 * 8 +
+                                    sizeof(FinalScratch) + (2 * kStages + 2) * 8 + 64;
+};
+
+// Columns [c, c+32) (or [c, c+16)) of this thread's TMEM lane as floats.
+__device__ __forceinline__ void ld_cols32(uint32_t taddr, float (&v)[32]) {
+    uint32_t r[32];
+    tmem_ld_32x32b_x32(taddr, r);
+    tmem_ld_wait();
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+__device__ __forceinline__ void ld_cols16(uint32_t taddr, float (&v)[32]) {
+    uint32_t r[16];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+    tmem_ld_wait();
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+#pragma unroll
+    for (int i = 16; i < 32; ++i) v[i] = 0.f;
+}
+
+// The logit of expert e from its accumulator: bias added, NaN ranked as -inf (flagged).
+__device__ __forceinline__ float score(const float *bg, float acc, int e) {
+    float s = acc + (bg ? __ldg(bg + e) : 0.f);
+    if (s != s) {
+        set_status(kStatusNanLogit);
+        s = -INFINITY;
+    }
+    return s;
+}
+
+// Visit the N logits of this thread's token in ascending expert order, 32 (or
+// 16) TMEM columns at a time.  f(e, s) is called for e < N.
+template <int NP, typename F>
+__device__ __forceinline__ void for_each_logit(const Params &p, uint32_t tlane, F &&f) {
+#pragma unroll 1
+    for (int c = 0; c < NP; c += 32) {
+        float v[32];
+        if (NP - c >= 32) ld_cols32(tlane + c, v);
+        else ld_cols16(tlane + c, v);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+            const int e = c + i;
+            if (e < p.N && (NP - c >= 32 || i < 16)) f(e, score(p.bg, v[i], e));
+        }
+    }
+}
+
+// Keep (s, e) in the best-first list (tv, te) of length KM if it belongs there:
+// larger value first, equal values in ascending expert index.
+template <int KM>
+__device__ __forceinline__ void topk_insert(float (&tv)[KM], int (&te)[KM], float s, int e) {
+    if (!(s > tv[KM - 1] || (s == tv[KM - 1] && e < te[KM - 1]))) return;
+    float cv = s;
+    int ce = e;
+#pragma unroll
+    for (int j = 0; j < KM; ++j) {
+        const bool better = cv > tv[j] || (cv == tv[j] && ce < te[j]);
+        const float ov = tv[j];
+        const int oe = te[j];
+        tv[j] = better ? cv : ov;
+        te[j] = better ? ce : oe;
+        cv = better ? ov : cv;
+        ce = better ? oe : ce;
+    }
+}
+
+template <int NP, int KM>
+__global__ void __launch_bounds__(kThreads, 1)
+    router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
+                     const Params p) {
+    using S = Shape<NP>;
+    constexpr int kStages = S::kStages;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *sA = smem;
+    uint8_t *sB = smem + kStages * S::kABytes;
+    float *s_wp = reinterpret_cast<float *>(sB + kStages * S::kBBytes);                  // [4][256]
+    int *s_cnt = reinterpret_cast<int *>(s_wp + 4 * 256);                                 // [256]
+    unsigned long long *s_imp = reinterpret_cast<unsigned long long *>(s_cnt + 256);      // [256]
+    FinalScratch *fs = reinterpret_cast<FinalScratch *>(s_imp + 256);
+    uint64_t *full = reinterpret_cast<uint64_t *>(fs + 1);
+    uint64_t *empty = full + kStages;
+    uint64_t *tfull = empty + kStages;
+    uint64_t *drain = tfull + 1;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
+    int *s_flag = reinterpret_cast<int *>(tmem_slot + 2);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int tile = blockIdx.x;
+    const int nkb = (p.D + BK - 1) / BK;
+    for (int e = threadIdx.x; e < 256; e += blockDim.x) {
+        s_cnt[e] = 0;
+        s_imp[e] = 0ull;
+    }
+    if (warp == 0 && lane == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        mbar_init(tfull, 1);
+        mbar_init(drain, 1);
+        fence_mbar_init();
+        tma_prefetch_desc(&tmX);
+        tma_prefetch_desc(&tmW);
+    }
+    if (warp == 1) tmem_alloc(tmem_slot, S::kTmemCols);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            bool ok = true;
+            for (int kb = 0; kb < nkb; ++kb) {
+                if (!mbar_wait(&empty[stage], phase ^ 1, p.timeout_ns)) {
+                    ok = false;
+                    break;
+                }
+                mbar_arrive_expect_tx(&full[stage], S::kStageBytes);
+                tma_load_2d(&tmX, &full[stage], sA + stage * S::kABytes, kb * BK, tile * BM);
+                tma_load_2d(&tmW, &full[stage], sB + stage * S::kBBytes, kb * BK, 0);
+                if (++stage == kStages) {
+                    stage = 0;
+                    phase ^= 1;
+                }
+            }
+            if (!ok) {
+                const uint64_t t0 = globaltimer_ns();
+                while (globaltimer_ns() - t0 < 1000000ull) {
+                }
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            constexpr uint32_t idesc = idesc_bf16_f32(BM, NP);
+            int stage = 0;
+            uint32_t phase = 0;
+            bool ok = true;
+            for (int kb = 0; kb < nkb; ++kb) {
+                if (!mbar_wait(&full[stage], phase, p.timeout_ns)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint64_t adesc = smem_desc_sw128(smem_u32(sA + stage * S::kABytes));
+                const uint64_t bdesc = smem_desc_sw128(smem_u32(sB + stage * S::kBBytes));
+#pragma unroll
+                for (int k = 0; k < BK / 16; ++k)
+                    tc_mma_bf16(tmem_base, adesc + 2 * k, bdesc + 2 * k, idesc, (kb | k) != 0 ? 1u : 0u);
+                tc_commit(&empty[stage]);
+                if (++stage == kStages) {
+                    stage = 0;
+                    phase ^= 1;
+                }
+            }
+            if (ok) tc_commit(tfull);
+            else {
+                tc_commit(drain);
+                mbar_wait(drain, 0, p.timeout_ns);
+            }
+        }
+    } else {
+        // ------------------------------------------------------------ one token per thread
+        // warp w may only read TMEM lanes 32*(w%4)..+31, which fixes the rows it owns
+        const int ew = warp & 3;
+        const int r = ew * 32 + lane;            // row of the tile = TMEM lane
+        const int t = tile * BM + r;
+        const bool live_row = t < p.T;
+        const bool have = __all_sync(0xffffffffu, mbar_wait(tfull, 0, p.timeout_ns));   // warp-uniform
+        tc_fence_after();
+        if (have) {
+            const uint32_t tlane = tmem_base + (static_cast<uint32_t>(ew * 32) << 16);
+            // pass 1: logits out, top-K
+            float tv[KM];
+            int te[KM];
+#pragma unroll
+            for (int j = 0; j < KM; ++j) { tv[j] = -INFINITY; te[j] = 0x7fffffff; }
+            for_each_logit<NP>(p, tlane, [&](int e, float s) {
+                if (live_row) p.logits[(int64_t)t * p.N + e] = s;
+                topk_insert<KM>(tv, te, s, e);
+            });
+            // gate weights over the K kept scores, slot order
+            float ex[KM];
+            float sum = 0.f;
+#pragma unroll
+            for (int j = 0; j < KM; ++j) {
+                ex[j] = j < p.K ? expf(tv[j] - tv[0]) : 0.f;
+                sum += ex[j];
+            }
+            const float inv = 1.0f / sum;
+#pragma unroll
+            for (int j = 0; j < KM; ++j) {
+                if (j < p.K && live_row) {
+                    const float wj = ex[j] * inv;
+                    p.topk_idx[(int64_t)t * p.K + j] = te[j];
+                    p.topk_w[(int64_t)t * p.K + j] = wj;
+                    atomicAdd(&s_cnt[te[j]], 1);
+                    atomicAdd(&s_imp[te[j]], (unsigned long long)__double2ull_rn((double)wj * kImpScale));
+                }
+            }
+            // pass 2: normaliser of the full softmax (the maximum is the best kept score)
+            const float m = tv[0];
+            float z = 0.f;
+            for_each_logit<NP>(p, tlane, [&](int e, float s) { z += expf(s - m); });
+            const float inv_z = live_row ? 1.0f / z : 0.f;
+            // pass 3: per-expert probability sums over the tile: lanes (xor tree), then warps (below)
+            for_each_logit<NP>(p, tlane, [&](int e, float s) {
+                float pe = expf(s - m) * inv_z;
+#pragma unroll
+                for (int o = 16; o >= 1; o >>= 1) pe += __shfl_xor_sync(0xffffffffu, pe, o);
+                if (lane == 0) s_wp[ew * 256 + e] = pe;
+            });
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    for (int e = threadIdx.x; e < p.N; e += blockDim.x) {
+        float ps = 0.f;
+        for (int w = 0; w < 4; ++w) ps += s_wp[w * 256 + e];
+        p.tile_p[(int64_t)tile * p.N + e] = ps;
+        p.tile_imp[(int64_t)tile * p.N + e] = s_imp[e];
+        p.tile_counts[(int64_t)tile * p.N + e] = s_cnt[e];
+    }
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, S::kTmemCols);
+    }
+    if (last_block(p.ticket, s_flag)) finalize_tables(p, gridDim.x, *fs);
+}
+
+// ---------------------------------------------------------------------------
+// Few tokens (T <= 64), N <= 32: one block of 256 threads per token.  Thread i
+// accumulates rows i, i+256, ... of W_g (four rows' loads issued together), the
+// 8 warps' partial scores are reduce-scattered (lane e: expert e) and added in
+// warp order by warp 0, which then selects the top k.  The token's partials are
+// its full-softmax probabilities, gate weights and counts (one-token "tiles").
+// ---------------------------------------------------------------------------
+template <int NP>
+__global__ void __launch_bounds__(256) router_few_kernel(const __nv_bfloat16 *__restrict__ x,
+                                                          const __nv_bfloat16 *__restrict__ Wg, const Params p) {
+    __shared__ float part[8][32];
+    __shared__ FinalScratch fs;
+    __shared__ int s_flag;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int t = blockIdx.x, N = p.N, D = p.D;
+    float a[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) a[i] = 0.f;
+    const __nv_bfloat16 *xt = x + (int64_t)t * D;
+    for (int d0 = tid; d0 < D; d0 += 4 * 256) {
+        float xv[4], wv[4][NP];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int d = d0 + u * 256;
+            xv[u] = d < D ? __bfloat162float(xt[d]) : 0.f;
+#pragma unroll
+            for (int e = 0; e < NP; ++e) wv[u][e] = (d < D && e < N) ? __bfloat162float(Wg[(int64_t)d * N + e]) : 0.f;
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+#pragma unroll
+            for (int e = 0; e < NP; ++e) a[e] = fmaf(xv[u], wv[u][e], a[e]);
+    }
+    reduce_scatter32(a, lane);   // lane l: this warp's sum for expert l
+    part[warp][lane] = a[0];
+    __syncthreads();
+    if (warp == 0) {
+        float s = 0.f;
+        for (int w = 0; w < 8; ++w) s += part[w][lane];
+        const bool live = lane < N;
+        s = live ? score(p.bg, s, lane) : -INFINITY;
+        if (live) p.logits[(int64_t)t * N + lane] = s;
+        int slot_e;
+        float slot_w;
+        const bool has = segment_topk<32>(s, lane, !live, p.K, lane, lane, slot_e, slot_w);
+        if (has) {
+            p.topk_idx[(int64_t)t * p.K + lane] = slot_e;
+            p.topk_w[(int64_t)t * p.K + lane] = slot_w;
+        }
+        // full softmax of the token; its counts and gate weights per expert
+        float mx = s;
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        const float ex = live ? expf(s - mx) : 0.f;
+        float z = ex;
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+        int cnt = 0;
+        unsigned long long im = 0;
+        for (int j = 0; j < p.K; ++j) {
+            const int ej = __shfl_sync(0xffffffffu, slot_e, j);
+            const float wj = __shfl_sync(0xffffffffu, slot_w, j);
+            if (ej == lane) {
+                ++cnt;
+                im += __double2ull_rn((double)wj * kImpScale);
+            }
+        }
+        if (live) {
+            p.tile_p[(int64_t)t * N + lane] = ex / z;
+            p.tile_counts[(int64_t)t * N + lane] = cnt;
+            p.tile_imp[(int64_t)t * N + lane] = im;
+        }
+    }
+    if (last_block(p.ticket, &s_flag)) finalize_tables(p, gridDim.x, fs);
+}
+
+}  // namespace rtc
+}  // namespace moe

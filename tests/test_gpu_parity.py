@@ -259,6 +259,46 @@ def test_bf16_ragged_dims_gelu_and_swiglu():
         run_full(wl, inp)
 
 
+@pytest.mark.parametrize("act,T,seed", [(ACT_SWIGLU, 1500, 0), (ACT_GELU, 1300, 1), (ACT_SWIGLU, 1100, 2)])
+def test_bf16_pair_tiles_with_ragged_segments(act, T, seed):
+    """Enough rows for the 2-CTA (256-row) tiles; skewed routing leaves experts with odd numbers of
+    128-row tiles, so some pair tiles have their upper half past the expert's segment."""
+    wl = Workload("pairs", 12 + seed, T, 512, 1024, 8, 2, act, torch.bfloat16, act == ACT_GELU, 0.04,
+                  zipf_s=0.7, random_bias=True)
+    inp = make_inputs(wl, "cuda")
+    layer, y, ws, aux, V, ref, errs = run_full(wl, inp)
+    counts = V["counts"]
+    assert any(((c + 127) // 128) % 2 == 1 for c in counts if c > 0)
+
+
+@pytest.mark.parametrize("act", [ACT_GELU, ACT_SWIGLU])
+def test_hidden_activations_match_oracle(act):
+    """The up-projection epilogue (GELU with bias, or SwiGLU) element by element: every hidden value of
+    sampled permuted rows is within bf16 rounding of the oracle's fp64 hidden layer."""
+    wl = Workload("hidden", 20 + act, 1200, 256, 384, 4, 2, act, torch.bfloat16, act == ACT_GELU, 0.08,
+                  random_bias=True)
+    inp = make_inputs(wl, "cuda")
+    layer = Layer(wl, inp)
+    y, ws, aux = layer.forward()
+    V = layer.views(ws, wl.T)
+    L = moe.moe_get_workspace_layout(layer.cfg, wl.T)
+    h = ws[L.h:L.h + L.rows_cap * wl.H * 2].view(torch.bfloat16).view(L.rows_cap, wl.H).float().cpu().numpy()
+    rng = np.random.default_rng(5)
+    slots = rng.choice(wl.T * wl.K, size=40, replace=False)
+    xb = ph.host(inp["x"])
+    for f in slots:
+        t, j = divmod(int(f), wl.K)
+        e = int(V["idx"][t, j])
+        row = int(V["slot_row"][f])
+        xr = oracle.load_rows(xb, oracle.BF16, [t])[0]
+        b1 = None if inp["b1"] is None else ph.host(inp["b1"][e])
+        b2 = None if inp["b2"] is None else ph.host(inp["b2"][e])
+        _, hid = oracle.expert(xr, act, oracle.BF16, ph.host(inp["W1"][e]), ph.host(inp["W2"][e]), b1, b2,
+                               return_hidden=True)
+        # bf16 keeps 8 significant bits: half an ulp is 2^-9 of the value; plus fp32 accumulation noise
+        np.testing.assert_allclose(h[row], hid, rtol=2.0 ** -8, atol=1e-4)
+
+
 def test_bf16_output_dtype():
     wl = WORKLOADS["gpt2"]
     inp = make_inputs(wl, "cuda", T=300)
@@ -343,8 +383,11 @@ def test_route_entry_point_matches_forward():
                p_mean=torch.empty(wl.N, device="cuda"), scalars=torch.empty(4, device="cuda"))
     moe.check(moe.moe_aux_stats(layer.cfg, 500, logits, idx, w, moe.make_aux(**out), ws2, ws2.numel()))
     torch.cuda.synchronize()
-    for k in out:
-        assert torch.equal(out[k], aux[k]), k
+    # the layer computes its statistics inside the router kernel, moe_aux_stats in its own kernels:
+    # counts are equal, the float sums agree to rounding (different fixed summation orders)
+    assert torch.equal(out["counts"], aux["counts"])
+    for k in ("importance", "p_mean", "scalars"):
+        torch.testing.assert_close(out[k], aux[k], rtol=1e-5, atol=1e-6)
 
 
 def test_bitwise_deterministic_runs():
