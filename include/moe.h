@@ -171,6 +171,34 @@ int moe_aux_stats(const moe_config *cfg, int64_t T, const float *logits, const i
                   const float *topk_w, moe_aux *out, void *ws, size_t ws_bytes,
                   moe_stream_t stream);
 
+/* moe_aux_stats without a workspace argument.  The pages define no such
+ * call: it is a library convenience for callers that cannot allocate device
+ * memory or keep a workspace buffer at the point of the call, for instance C
+ * code that may not call cudaMalloc there (it can synchronise the whole
+ * device) or that has no device allocator of its own.  The results are those
+ * of moe_aux_stats for the same arguments (same kernels, same summation
+ * order).
+ *
+ * Scratch: a fixed array of MOE_NOALLOC_SCRATCH_BYTES inside the library, one
+ * per device, shared by every call on that device.  The call clears the part
+ * that must start at zero itself.  Calls whose work overlaps on the device
+ * (different streams, or host threads that do not order their streams) race
+ * on that array and give wrong statistics: serialise them.
+ *
+ * Limit: the call fits when 256 + 3 * round_up_256(ceil(T / 64) * NExperts * 4)
+ * <= MOE_NOALLOC_SCRATCH_BYTES, about T * NExperts <= 11 million; otherwise it
+ * returns MOE_ERR_WORKSPACE_TOO_SMALL before enqueueing anything.
+ *
+ * Set-up: the first call on each device (with that device current) looks up
+ * the array's device address, once.  Make that first call before capturing
+ * the stream into a CUDA graph.
+ *
+ * Arguments, layouts and other errors as moe_aux_stats. */
+#define MOE_NOALLOC_SCRATCH_BYTES (2u << 20)
+int moe_aux_stats_noalloc(const moe_config *cfg, int64_t T, const float *logits,
+                          const int32_t *topk_idx, const float *topk_w, moe_aux *out,
+                          moe_stream_t stream);
+
 /* Where moe_forward leaves its intermediates inside the workspace (byte
  * offsets from ws), for inspection in tests.  Rows of each expert's segment in
  * the permuted buffers start at a multiple of row_align; rows past an expert's

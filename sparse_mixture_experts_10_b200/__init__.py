@@ -33,8 +33,10 @@ MOE_ERR_CUDA = -4
 MOE_ERR_DEVICE_TIMEOUT = -5
 MOE_ERR_DEVICE_BOUNDS = -6
 MOE_STATUS_TIMEOUT, MOE_STATUS_BOUNDS, MOE_STATUS_NAN_LOGIT = 1, 2, 4
+MOE_NOALLOC_SCRATCH_BYTES = 2 << 20
 
 EXPORTED = ("moe_workspace_size", "moe_route", "moe_forward", "moe_forward_timed", "moe_aux_stats",
+            "moe_aux_stats_noalloc",
             "moe_get_workspace_layout", "moe_total_params", "moe_active_params", "moe_get_device_status",
             "moe_launch_count", "moe_error_string", "moe_selftest_wait_timeout")
 
@@ -94,6 +96,8 @@ def load_library():
     L.moe_forward_timed.argtypes = [cfgp, vp, i64, wp, vp, i32, auxp, vp, sz, vp, ctypes.POINTER(vp)]
     L.moe_aux_stats.restype = ctypes.c_int
     L.moe_aux_stats.argtypes = [cfgp, i64, vp, vp, vp, auxp, vp, sz, vp]
+    L.moe_aux_stats_noalloc.restype = ctypes.c_int
+    L.moe_aux_stats_noalloc.argtypes = [cfgp, i64, vp, vp, vp, auxp, vp]
     L.moe_get_workspace_layout.restype = ctypes.c_int
     L.moe_get_workspace_layout.argtypes = [cfgp, i64, ctypes.POINTER(moe_workspace_layout)]
     L.moe_total_params.restype = i64
@@ -192,6 +196,14 @@ def moe_forward_timed(cfg, x, T, weights, y, y_dtype, aux, ws, ws_bytes, stream,
 def moe_aux_stats(cfg, T, logits, topk_idx, topk_w, out, ws, ws_bytes, stream=None) -> int:
     return load_library().moe_aux_stats(ctypes.byref(cfg), T, _ptr(logits), _ptr(topk_idx), _ptr(topk_w),
                                         ctypes.byref(out), _ptr(ws), ws_bytes, _stream(stream))
+
+
+def moe_aux_stats_noalloc(cfg, T, logits, topk_idx, topk_w, out, stream=None) -> int:
+    """moe_aux_stats with its scratch in the library's fixed array instead of a
+    workspace; for callers that cannot allocate.  Calls that overlap on the
+    device race on that array."""
+    return load_library().moe_aux_stats_noalloc(ctypes.byref(cfg), T, _ptr(logits), _ptr(topk_idx), _ptr(topk_w),
+                                                ctypes.byref(out), _stream(stream))
 
 
 def moe_get_workspace_layout(cfg, T) -> moe_workspace_layout:

@@ -862,6 +862,67 @@ const char *moe_error_string(int code) {
     }
 }
 
+// ---------------------------------------------------------------- statistics without a workspace
+// moe_aux_stats_noalloc keeps its scratch in one fixed array inside the library
+// instead of a caller-provided workspace: a 256-byte block of counters that
+// must be zero when the kernels start (cleared on every call), then the three
+// per-block partial arrays of the statistics kernels.  Every call on a device
+// uses the same array, so two calls whose kernels overlap (other streams,
+// other host threads) corrupt each other's results.
+}  // extern "C"
+
+namespace {
+__device__ __align__(256) unsigned char g_noalloc_scratch[MOE_NOALLOC_SCRATCH_BYTES];
+
+constexpr int kNoallocMaxDevices = 64;
+std::mutex g_noalloc_mutex;
+void *g_noalloc_ptr[kNoallocMaxDevices];
+
+// Device address of g_noalloc_scratch on the current device, looked up once per
+// device (the first call on it) with that device current.
+int noalloc_scratch(char **out) {
+    int d = -1;
+    if (cudaGetDevice(&d) != cudaSuccess) return MOE_ERR_CUDA;
+    if (d < 0 || d >= kNoallocMaxDevices) return MOE_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    if (!g_noalloc_ptr[d]) {
+        void *ptr = nullptr;
+        if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || !ptr) return MOE_ERR_CUDA;
+        g_noalloc_ptr[d] = ptr;
+    }
+    *out = static_cast<char *>(g_noalloc_ptr[d]);
+    return MOE_OK;
+}
+}  // namespace
+
+extern "C" {
+
+int moe_aux_stats_noalloc(const moe_config *cfg, int64_t T, const float *logits, const int32_t *topk_idx,
+                          const float *topk_w, moe_aux *out, moe_stream_t stream) {
+    Plan P;
+    MOE_TRY(make_plan(cfg, T, &P));
+    if (!out) return MOE_ERR_INVALID_ARG;
+    if (T > 0 && (!logits || !topk_idx || !topk_w)) return MOE_ERR_INVALID_ARG;
+    // the same kernels as moe_aux_stats, with their scratch moved into the fixed array
+    const size_t part = align256((size_t)P.aux_blocks * P.N * 4);
+    if (256 + 3 * part > (size_t)MOE_NOALLOC_SCRATCH_BYTES) return MOE_ERR_WORKSPACE_TOO_SMALL;
+    char *scratch = nullptr;
+    MOE_TRY(noalloc_scratch(&scratch));
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (T == 0) return zero_aux(P, out, s);
+    DeviceInfo *dev = nullptr;
+    MOE_TRY(device_info(&dev));
+    Plan Q = P;
+    Q.counters = 0;
+    Q.aux_p = 256;
+    Q.aux_i = 256 + part;
+    Q.aux_c = 256 + 2 * part;
+    Q.total = 256 + 3 * part;
+    Bufs b{scratch, &Q};
+    MOE_TRY(zero_counters(Q, b, s));
+    return stage_aux(Q, b, logits, topk_idx, topk_w, out, s);
+}
+
 int moe_selftest_wait_timeout(int64_t timeout_ns, moe_stream_t stream) {
     if (timeout_ns <= 0 || timeout_ns > 10000000000ll) return MOE_ERR_INVALID_ARG;
     wait_selftest_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>((uint64_t)timeout_ns);
