@@ -6,8 +6,11 @@ A step is one pass of the whole layer (route, scan, permute, expert up- and
 down-projections, combine, statistics) over one batch of synthetic tokens
 already resident in device memory.  One layer call (moe_forward_timed, which
 records CUDA events between its stages on the launching stream) is captured
-as a CUDA graph and replayed once per step; each step's time is the span of
-those events.  The L2 cache is flushed (a 512 MiB buffer is written) before
+as a CUDA graph and replayed once per step, with events only around the
+dominant stage (its duration gives the roofline figure); each step's time is
+the span of two events recorded on the stream around the replay.  A separate
+pass of up to 20 steps with an event between every two stages gives the stage
+breakdown.  The L2 cache is flushed (a 512 MiB buffer is written) before
 every step, outside the events.  `e2e` repeats the measurement through plain
 moe_forward calls with the input copied in from pinned host memory and the
 output and losses copied back, every step.  With N > 1 (torchrun) every rank runs
@@ -271,17 +274,48 @@ def main():
         raise RuntimeError(f"device status {st} after warm-up")
     counts = aux_t["counts"].cpu().numpy()
 
-    # One layer call captured as a CUDA graph (its stage events included) and
-    # replayed once per step, so host-side enqueue cost stays out of the step.
-    evs = [torch.cuda.Event(enable_timing=True) for _ in range(NS + 1)]
-    for e in evs:
-        e.record()
+    def capture(stage_events):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            step(stage_events)
+        return g
+
+    def new_events(n):
+        out = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+        for e in out:
+            e.record()
+        return out
+
+    # Stage breakdown: one layer call with an event between every two stages,
+    # captured as a CUDA graph and replayed (each event node adds a few
+    # microseconds, so these steps are not the timed ones).
+    evs = new_events(NS + 1)
     torch.cuda.synchronize()
-    graph = torch.cuda.CUDAGraph()
     l0 = moe.moe_launch_count()
-    with torch.cuda.graph(graph):
-        step(evs)
+    graph = capture(evs)
     launches_per_step = moe.moe_launch_count() - l0
+    rows = []
+    n_break = min(args.steps, 20)
+    for i in range(2 + n_break):
+        flush.zero_()
+        graph.replay()
+        torch.cuda.synchronize()
+        if i >= 2:
+            rows.append([evs[s_].elapsed_time(evs[s_ + 1]) for s_ in range(NS)])
+    del graph
+    stage_ms = np.array(rows)
+    mean_stage = stage_ms.mean(axis=0)
+    names = moe.STAGE_NAMES
+    dom = int(np.argmax(mean_stage))
+
+    # Timed steps: the layer call as a graph with events only around the
+    # dominant stage (its duration for the roofline); the step time is taken
+    # by events recorded on the stream around each replay.
+    dom_ev = [None] * (NS + 1)
+    dom_ev[dom], dom_ev[dom + 1] = new_events(2)
+    step_ev = [tuple(new_events(2)) for _ in range(args.steps)]
+    torch.cuda.synchronize()
+    graph = capture(dom_ev)
     for _ in range(2):
         flush.zero_()
         graph.replay()
@@ -292,12 +326,15 @@ def main():
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    rows = []
+    step_ms, dom_ms = [], []
     for i in range(args.steps):
         flush.zero_()
+        step_ev[i][0].record(stream)
         graph.replay()
+        step_ev[i][1].record(stream)
         torch.cuda.synchronize()
-        rows.append([evs[s_].elapsed_time(evs[s_ + 1]) for s_ in range(NS)])
+        step_ms.append(step_ev[i][0].elapsed_time(step_ev[i][1]))
+        dom_ms.append(dom_ev[dom].elapsed_time(dom_ev[dom + 1]))
     launches = launches_per_step * args.steps
     if world > 1:
         dist.barrier()
@@ -307,11 +344,10 @@ def main():
         raise RuntimeError(f"device status {st} after timed steps")
     del graph
 
-    stage_ms = np.array(rows)
-    step_ms = stage_ms.sum(axis=1)
-    total_ms = max_over_ranks(float(step_ms.sum()), dev, world)
+    total_ms = max_over_ranks(float(sum(step_ms)), dev, world)
     ms_per_step = total_ms / args.steps
     tokens_per_s = job_throughput(T, world, args.steps, total_ms)
+    dom_mean_ms = float(np.mean(dom_ms))
 
     # ---- end to end through host buffers: pinned x in, y and the statistics out, every step
     x_host = inp["x"].cpu().pin_memory()
@@ -336,26 +372,24 @@ def main():
     h2d = T * wl.D * es
     d2h = T * wl.D * 4 + 16
 
-    # ---- roofline of the dominant kernel
+    # ---- roofline of the dominant kernel (its duration from the timed steps)
     wm = work_model(wl, T, counts)
     pk, pk_kind = peaks()
-    mean_stage = stage_ms.mean(axis=0)
-    names = moe.STAGE_NAMES
-    dom = int(np.argmax(mean_stage))
     decode = wl.name.startswith("decode")
     if names[dom] in ("up", "down") and not decode:
         fl = wm["up_flops"] if names[dom] == "up" else wm["down_flops"]
-        achieved = fl / (mean_stage[dom] * 1e-3) / 1e12
+        achieved = fl / (dom_mean_ms * 1e-3) / 1e12
         peak = float(pk["bf16_tflops"])
         roof = {"kernel": f"grouped_gemm_tc ({names[dom]})", "bound": "tensor", "achieved": achieved, "peak": peak,
                 "unit": "TFLOP/s", "frac": achieved / peak, "peak_kind": f"{pk_kind} bf16 burst"}
     else:
         byt = {"route": wm["route_bytes"], "permute": wm["permute_bytes"], "combine": wm["combine_bytes"],
                "up": wm["up_weight_bytes"], "down": wm["down_weight_bytes"]}.get(names[dom], 0)
-        achieved = byt / (mean_stage[dom] * 1e-3) / 1e9
+        achieved = byt / (dom_mean_ms * 1e-3) / 1e9
         peak = float(pk["hbm_gbs"])
         roof = {"kernel": names[dom], "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                 "frac": achieved / peak, "peak_kind": f"{pk_kind} copy"}
+    roof["ms"] = dom_mean_ms
     key = f"{wl.name}/{names[dom]}"
     tr = NCU_TRAFFIC.get(key)
     roof["traffic"] = tr["bytes"] if tr and tr["src_sha256"] == sha256(GEMM_KERNEL_SRC) else None
@@ -384,6 +418,7 @@ def main():
                        "parallelism": f"dp{world}", "l2": "flushed (512 MiB write) before every step"},
             "active_tflops": wm["flops"] * world * args.steps / (total_ms / 1e3) / 1e12,
             "roofline": roof, "stages": stages,
+            "stages_note": f"{n_break} separate steps with an event between every two stages",
             "e2e": {"value": e2e_tps, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "gpu_launches": launches, "clocks": clocks}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -157,8 +157,9 @@ int moe_forward(const moe_config *cfg, const void *x, int64_t T, const moe_weigh
 /* moe_forward that also records CUDA events between its stages, for timing.
  * stage_events: MOE_N_STAGES + 1 cudaEvent_t handles (created by the caller);
  * event i is recorded on `stream` before stage i and event MOE_N_STAGES after
- * the last.  Stages: 0 route, 1 scan, 2 permute, 3 expert up-projection,
- * 4 expert down-projection, 5 combine, 6 statistics (empty without aux). */
+ * the last; a NULL entry is not recorded.  Stages: 0 route, 1 scan, 2 permute,
+ * 3 expert up-projection, 4 expert down-projection, 5 combine, 6 statistics
+ * (empty without aux). */
 #define MOE_N_STAGES 7
 int moe_forward_timed(const moe_config *cfg, const void *x, int64_t T, const moe_weights *w,
                       void *y, int32_t y_dtype, moe_aux *aux, void *ws, size_t ws_bytes,

@@ -180,14 +180,15 @@ def moe_forward(cfg, x, T, weights, y, y_dtype, aux, ws, ws_bytes, stream=None) 
 
 
 def moe_forward_timed(cfg, x, T, weights, y, y_dtype, aux, ws, ws_bytes, stream, stage_events) -> int:
-    """stage_events: MOE_N_STAGES + 1 torch.cuda.Event(enable_timing=True) objects.
+    """stage_events: MOE_N_STAGES + 1 torch.cuda.Event(enable_timing=True)
+    objects or None (that boundary is not recorded).
 
     torch creates an event's CUDA handle on its first record; events never
     recorded are recorded once here so that a valid handle is passed."""
     for e in stage_events:
-        if not e.cuda_event:
+        if e is not None and not e.cuda_event:
             e.record(torch.cuda.current_stream())
-    arr = (ctypes.c_void_p * len(stage_events))(*[e.cuda_event for e in stage_events])
+    arr = (ctypes.c_void_p * len(stage_events))(*[None if e is None else e.cuda_event for e in stage_events])
     return load_library().moe_forward_timed(ctypes.byref(cfg), _ptr(x), T, ctypes.byref(weights), _ptr(y), y_dtype,
                                             None if aux is None else ctypes.byref(aux), _ptr(ws), ws_bytes,
                                             _stream(stream), arr)

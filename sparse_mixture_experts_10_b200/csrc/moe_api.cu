@@ -33,6 +33,7 @@ constexpr int kMaxDevices = 64;
 constexpr size_t kSmallRouterSmemMax = 200 * 1024;
 constexpr int64_t kRowdotMaxT = 2048;  // below this the chunked router has too few blocks
 constexpr int64_t kDecodeMaxT = 64;    // up to this many tokens the expert GEMMs stream weights (decode path)
+constexpr int kDecodeMaxGrid = 256;    // decode GEMMs: most persistent CTAs (stream-K buffers are sized for it)
 
 struct DeviceInfo {
     int sms = 0;
@@ -60,8 +61,15 @@ struct Plan {
     int rnp, rkm;      // tensor-core router: padded expert count, top-k list length
     bool decode;  // few tokens: weight-streaming expert GEMMs
     int nt;       // decode: padded token tile (16, 32 or 64)
+    int route_splits;  // few-token router: W_g slabs per token
+    int dec_cap;       // decode GEMMs: CTAs the stream-K partials and tickets are sized for
+    // Counters region (zeroed on every call), 32-bit words: [0] router ticket,
+    // [1] statistics ticket, [2] number of live experts, [64, 128) per-token
+    // tickets of the few-token router; from byte 512 the stream-K tile tickets
+    // of the decode up- and then down-projection (dec_cap each).
+    size_t counters_bytes;
     size_t counters, logits, idx, w, counts, offsets, row_offsets, live, chunk_counts, chunk_base, tile_p, tile_imp,
-        perm_slot, slot_row, x_perm, h, z, wgt, aux_p, aux_i, aux_c, total;
+        perm_slot, slot_row, x_perm, h, z, wgt, aux_p, aux_i, aux_c, route_part, dec_part, total;
 };
 
 int make_plan(const moe_config *c, int64_t T, Plan *p) {
@@ -105,7 +113,10 @@ int make_plan(const moe_config *c, int64_t T, Plan *p) {
         off = align256(off + bytes);
         return o;
     };
-    p->counters = take(256);
+    p->route_splits = p->few_router ? (int)std::min<int64_t>(rtc::kFewMaxSplits, std::max<int64_t>(1, cdiv(D, 256))) : 1;
+    p->dec_cap = p->decode ? kDecodeMaxGrid : 0;
+    p->counters_bytes = align256(512 + (size_t)2 * p->dec_cap * 4);
+    p->counters = take(p->counters_bytes);
     p->logits = take((size_t)T * N * 4);
     p->idx = take((size_t)T * K * 4);
     p->w = take((size_t)T * K * 4);
@@ -127,6 +138,8 @@ int make_plan(const moe_config *c, int64_t T, Plan *p) {
     p->aux_p = take((size_t)p->aux_blocks * N * 4);
     p->aux_i = take((size_t)p->aux_blocks * N * 4);
     p->aux_c = take((size_t)p->aux_blocks * N * 4);
+    p->route_part = take(p->few_router ? (size_t)T * p->route_splits * 32 * 4 : 0);
+    p->dec_part = take(p->decode ? (size_t)p->dec_cap * 2 * dec::BM * p->nt * 4 : 0);
     p->total = off;
     return MOE_OK;
 }
@@ -317,9 +330,10 @@ int stage_route_tc(const Plan &P, const Bufs &b, const void *x, const moe_weight
     if (P.few_router) {
         const __nv_bfloat16 *xb = static_cast<const __nv_bfloat16 *>(x);
         const __nv_bfloat16 *wg = static_cast<const __nv_bfloat16 *>(w->W_g);
-        if (N <= 8) rtc::router_few_kernel<8><<<T, 256, 0, s>>>(xb, wg, p);
-        else if (N <= 16) rtc::router_few_kernel<16><<<T, 256, 0, s>>>(xb, wg, p);
-        else rtc::router_few_kernel<32><<<T, 256, 0, s>>>(xb, wg, p);
+        const int S = P.route_splits;
+        const int rows = (int)cdiv(D, S);
+        rtc::router_few_kernel<<<dim3((unsigned)T, (unsigned)S), 256, 0, s>>>(
+            xb, wg, p, b.at<float>(P.route_part), b.at<unsigned>(P.counters) + 64, rows);
         return check_launch();
     }
     __nv_bfloat16 *wgt = b.at<__nv_bfloat16>(P.wgt);
@@ -463,7 +477,10 @@ int stage_permute(const Plan &P, const Bufs &b, const void *x, const DeviceInfo 
 template <int NT, int EPI>
 int launch_dec(const CUtensorMap &W, const CUtensorMap &X, const dec::Params &p, int64_t items_upper, int sms,
                cudaStream_t s) {
-    const int grid = (int)std::min<int64_t>(std::max<int64_t>(items_upper, 1), sms);
+    // stream-K spreads any number of tiles over every SM (up to the CTAs its
+    // partial buffer is sized for); whole tiles need no more CTAs than tiles
+    const int grid = p.split_cap > 0 ? std::min(sms, p.split_cap)
+                                     : (int)std::min<int64_t>(std::max<int64_t>(items_upper, 1), sms);
     dec::decode_gemm_kernel<NT, EPI><<<grid, dec::kThreads, dec::Shape<NT, EPI>::kSmem, s>>>(W, X, p);
     return check_launch();
 }
@@ -495,6 +512,9 @@ int stage_up_decode(const Plan &P, const Bufs &b, const moe_weights *w, const De
     p.out = b.ws + P.h;
     p.ldo = H;
     p.bias = swiglu ? nullptr : w->b1;
+    p.split_cap = P.dec_cap;
+    p.part = b.at<float>(P.dec_part);
+    p.tickets = b.at<unsigned>(P.counters) + 128;
     p.timeout_ns = kTimeoutNs;
     const int64_t upper = std::min<int64_t>(N, P.T * P.K) * p.tiles_per_group;
     if (swiglu) return launch_dec_nt<dec::EPI_SWIGLU>(P.nt, mw, mx, p, upper, dev.sms, s);
@@ -520,6 +540,9 @@ int stage_down_decode(const Plan &P, const Bufs &b, const moe_weights *w, const 
     p.bias = P.act == MOE_ACT_SWIGLU ? nullptr : w->b2;
     p.perm_slot = b.at<int>(P.perm_slot);
     p.gate_w = b.at<float>(P.w);
+    p.split_cap = P.dec_cap;
+    p.part = b.at<float>(P.dec_part);
+    p.tickets = b.at<unsigned>(P.counters) + 128 + P.dec_cap;
     p.timeout_ns = kTimeoutNs;
     const int64_t upper = std::min<int64_t>(N, P.T * P.K) * p.tiles_per_group;
     return launch_dec_nt<dec::EPI_SCATTER>(P.nt, mw, mx, p, upper, dev.sms, s);
@@ -660,7 +683,7 @@ int stage_aux(const Plan &P, const Bufs &b, const float *logits, const int *idx,
 }
 
 int zero_counters(const Plan &P, const Bufs &b, cudaStream_t s) {
-    return cudaMemsetAsync(b.ws + P.counters, 0, 256, s) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+    return cudaMemsetAsync(b.ws + P.counters, 0, P.counters_bytes, s) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
 int zero_aux(const Plan &P, moe_aux *aux, cudaStream_t s) {
@@ -699,7 +722,7 @@ int forward_impl(const moe_config *cfg, const void *x, int64_t T, const moe_weig
         if (cs == cudaStreamCaptureStatusActive) rec_flags = cudaEventRecordExternal;
     }
     auto rec = [&](int i) -> int {
-        if (!ev) return MOE_OK;
+        if (!ev || !ev[i]) return MOE_OK;
         return cudaEventRecordWithFlags(static_cast<cudaEvent_t>(ev[i]), s, rec_flags) == cudaSuccess ? MOE_OK
                                                                                                       : MOE_ERR_CUDA;
     };
@@ -914,6 +937,7 @@ int moe_aux_stats_noalloc(const moe_config *cfg, int64_t T, const float *logits,
     MOE_TRY(device_info(&dev));
     Plan Q = P;
     Q.counters = 0;
+    Q.counters_bytes = 256;
     Q.aux_p = 256;
     Q.aux_i = 256 + part;
     Q.aux_c = 256 + 2 * part;

@@ -10,8 +10,17 @@
 // so no tensor-core work is spent on padding rows of tokens, and every CTA
 // streams 128 whole weight rows per item.
 //
-// Items are (live expert, tile of 128 weight rows), expert-major, handed to
-// persistent CTAs round-robin; one CTA per SM, 192 threads:
+// The work is (live expert, tile of 128 weight rows) tiles, expert-major, each
+// of num_k_blocks 64-wide K blocks.  When whole tiles dealt round-robin would
+// leave the last wave less than 90% full (e.g. 180 tiles on 148 SMs) and
+// split_cap > 0, the tiles x K blocks units are cut into gridDim.x equal
+// contiguous ranges, one per persistent CTA (stream-K): every SM streams the
+// same number of weight bytes whatever the number of tiles.  A CTA's range is a sequence of pieces (a tile and a K
+// range); a tile cut between CTAs has its pieces' fp32 partials written to
+// the workspace, and the CTA that finishes its last piece (an atomic ticket per
+// tile) adds them in piece order and runs the epilogue, so the result does not
+// depend on which CTA finishes when.  Without split_cap the tiles go whole to
+// the CTAs round-robin.  One CTA per SM, 192 threads:
 //   warp 0      TMA producer: weight tile (16 KB per 64-wide K slice) and the
 //               expert's token tile into a kStages-deep ring.
 //   warp 1      TMEM allocation; one thread issues 128 x NT x 16 MMAs into one
@@ -52,7 +61,37 @@ struct Params {
     const float *bias;        // [N, n_valid] or nullptr
     const int *perm_slot;     // EPI_SCATTER
     const float *gate_w;      // EPI_SCATTER
+    // stream-K (split_cap == 0: whole tiles round-robin)
+    int split_cap;            // CTAs the partial buffer and the tickets are sized for (>= gridDim.x)
+    float *part;              // [split_cap][2][BM][NT] fp32: each CTA's first and last cut piece
+    unsigned *tickets;        // [split_cap] zero at launch, indexed by the CTA holding a tile's first piece
     uint64_t timeout_ns;
+};
+
+__device__ __forceinline__ unsigned ld_acquire_u32(const unsigned *ptr) {
+    unsigned v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(ptr) : "memory");
+    return v;
+}
+
+// One CTA's share of the tiles x K-block units and the pieces it is cut into.
+struct Work {
+    int64_t W;     // units in all
+    int G, nkb;    // CTAs, K blocks per tile
+    __device__ __forceinline__ int64_t begin(int c) const { return (int64_t)c * W / G; }
+    // CTA whose range holds unit u: the largest c with begin(c) <= u
+    __device__ __forceinline__ int cta_of(int64_t u) const { return (int)(((u + 1) * G - 1) / W); }
+};
+
+// Piece of a CTA's range starting at unit u (< end): its tile and K blocks.
+struct Piece {
+    int tile, k0, k1;
+    __device__ __forceinline__ Piece(int64_t u, int64_t end, int nkb) {
+        tile = (int)(u / nkb);
+        k0 = (int)(u - (int64_t)tile * nkb);
+        const int64_t rest = (int64_t)k0 + (end - u);
+        k1 = rest < nkb ? (int)rest : nkb;
+    }
 };
 
 template <int NT, int EPI>
@@ -66,7 +105,7 @@ struct Shape {
     static constexpr int kStages0 = (200 * 1024 - (int)kEpiBytes) / (int)kStageBytes;
     static constexpr int kStages = kStages0 > 8 ? 8 : kStages0;
     static constexpr uint32_t kTmemCols = 2 * NT < 32 ? 32 : 2 * NT;
-    static constexpr size_t kSmem = 1024 + (size_t)kStages * kStageBytes + kEpiBytes + (2 * kStages + 6) * 8 + 16;
+    static constexpr size_t kSmem = 1024 + (size_t)kStages * kStageBytes + kEpiBytes + (2 * kStages + 6) * 8 + 32;
 };
 
 __device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t *r) {
@@ -133,6 +172,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t *drain = tempty + 2;
     uint64_t *epib = drain + 1;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(epib + 1);
+    int *s_last = reinterpret_cast<int *>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (warp == 0 && lane == 0) {
@@ -155,16 +195,32 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
-    const int total = *p.n_live * p.tiles_per_group;
+    const int tiles = *p.n_live * p.tiles_per_group;
+    const int nkb = p.num_k_blocks;
+    const Work wk{(int64_t)tiles * nkb, (int)gridDim.x, nkb};
+    // stream-K when whole tiles round-robin would leave more than a tenth of
+    // the CTA-tile slots of the last wave empty; it needs at least 4 units per
+    // CTA, so that every CTA's range is non-empty and every piece of a cut
+    // tile exists
+    const int waves = (tiles + (int)gridDim.x - 1) / (int)gridDim.x;
+    const bool stream_k = p.split_cap >= (int)gridDim.x && wk.W >= 4 * (int64_t)gridDim.x &&
+                          10 * tiles < 9 * waves * (int)gridDim.x;
+    // stream-K: this CTA's unit range; otherwise whole tiles blockIdx.x, +gridDim.x, ...
+    const int64_t u_begin = stream_k ? wk.begin(blockIdx.x) : (int64_t)blockIdx.x * nkb;
+    const int64_t u_end = stream_k ? wk.begin(blockIdx.x + 1) : wk.W;
+    const int64_t u_step = (int64_t)gridDim.x * nkb;   // whole tiles: on to this CTA's next tile
 
     if (warp == 0) {
         if (lane == 0) {
             int stage = 0;
             uint32_t phase = 0;
             bool ok = true;
-            for (int i = blockIdx.x; i < total && ok; i += gridDim.x) {
-                const int g = p.live[i / p.tiles_per_group];
-                const int mt = i % p.tiles_per_group;
+            for (int64_t u = u_begin; u < u_end && ok;) {
+                const Piece pc(u, stream_k ? u_end : u + nkb, nkb);
+                u = stream_k ? u + (pc.k1 - pc.k0) : u + u_step;
+                const int tile = pc.tile, k0 = pc.k0, k1 = pc.k1;
+                const int g = p.live[tile / p.tiles_per_group];
+                const int mt = tile % p.tiles_per_group;
                 const int trow = p.row_offsets[g];
                 int wrow, wrow2 = 0;
                 if (EPI == EPI_SWIGLU) {
@@ -173,7 +229,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 } else {
                     wrow = g * p.w_group_rows + mt * BM;
                 }
-                for (int kb = 0; kb < p.num_k_blocks; ++kb) {
+                for (int kb = k0; kb < k1; ++kb) {
                     if (!mbar_wait(&empty[stage], phase ^ 1, p.timeout_ns)) {
                         ok = false;
                         break;
@@ -205,7 +261,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t phase = 0;
             int local = 0;
             bool ok = true;
-            for (int i = blockIdx.x; i < total && ok; i += gridDim.x, ++local) {
+            for (int64_t u = u_begin; u < u_end && ok; ++local) {
+                const Piece pc(u, stream_k ? u_end : u + nkb, nkb);
+                u = stream_k ? u + (pc.k1 - pc.k0) : u + u_step;
+                const int k0 = pc.k0, k1 = pc.k1;
                 const int a = local & 1;
                 const uint32_t aph = (local >> 1) & 1;
                 if (!mbar_wait(&tempty[a], aph ^ 1, p.timeout_ns)) {
@@ -214,7 +273,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + a * NT;
-                for (int kb = 0; kb < p.num_k_blocks; ++kb) {
+                for (int kb = k0; kb < k1; ++kb) {
                     if (!mbar_wait(&full[stage], phase, p.timeout_ns)) {
                         ok = false;
                         break;
@@ -224,7 +283,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const uint64_t bdesc = smem_desc_sw128(smem_u32(sB + stage * S::kBBytes));
 #pragma unroll
                     for (int k = 0; k < BK / 16; ++k)
-                        tc_mma_bf16(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, (kb | k) != 0 ? 1u : 0u);
+                        tc_mma_bf16(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, (kb != k0 || k != 0) ? 1u : 0u);
                     tc_commit(&empty[stage]);
                     if (++stage == kStages) {
                         stage = 0;
@@ -244,13 +303,52 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int et = threadIdx.x - 64;             // 0..127 inside the epilogue warps
         EpiBarrier eb{epib, 0u, p.timeout_ns};
         int local = 0;
-        for (int i = blockIdx.x; i < total; i += gridDim.x, ++local) {
+        for (int64_t u = u_begin; u < u_end; ++local) {
+            const int64_t u_piece = u;
+            const Piece pc(u, stream_k ? u_end : u + nkb, nkb);
+            u = stream_k ? u + (pc.k1 - pc.k0) : u + u_step;
+            const int tile = pc.tile;
             const int a = local & 1;
             const uint32_t aph = (local >> 1) & 1;
-            const int g = p.live[i / p.tiles_per_group];
-            const int mt = i % p.tiles_per_group;
+            const int g = p.live[tile / p.tiles_per_group];
+            const int mt = tile % p.tiles_per_group;
             const int cnt = p.counts[g];
             const int trow = p.row_offsets[g];
+            // A cut tile's pieces belong to CTAs c_first..c_last and are added as
+            // a right fold in piece order, p_first + (... + (p_last-1 + p_last)),
+            // whichever piece does it.  A piece is slot 0 of its CTA when the
+            // CTA's range starts inside the tile (its first piece), else slot 1.
+            const bool cut = pc.k1 - pc.k0 < nkb;
+            const int64_t ts = (int64_t)tile * nkb;
+            const int c_first = cut ? wk.cta_of(ts) : 0, c_last = cut ? wk.cta_of(ts + nkb - 1) : 0;
+            // While this piece's MMAs run: if it is the tile's first piece and
+            // every other piece is already published, it will be the one to add
+            // them up, so the others' sum is loaded now.
+            constexpr int NR = NT <= 32 ? NT : 4;   // (64 token columns: no room in registers)
+            float rest[NR];
+            bool have_rest = false;
+            if (NT <= 32 && cut && c_first == (int)blockIdx.x) {
+                if (et == 0) *s_last = ld_acquire_u32(p.tickets + c_first) == (unsigned)(c_last - c_first);
+                if (!eb.sync()) break;
+                have_rest = *s_last != 0;
+                if (have_rest) {
+                    for (int c = c_last; c > c_first; --c) {
+                        const float *src = p.part + ((int64_t)(c * 2 + (wk.begin(c) >= ts ? 0 : 1)) * BM + L) * NT;
+#pragma unroll
+                        for (int j = 0; j < NR; j += 4) {
+                            const float4 v = __ldcg(reinterpret_cast<const float4 *>(src + j));
+                            if (c == c_last) {
+                                rest[j] = v.x; rest[j + 1] = v.y; rest[j + 2] = v.z; rest[j + 3] = v.w;
+                            } else {
+                                rest[j] = v.x + rest[j]; rest[j + 1] = v.y + rest[j + 1];
+                                rest[j + 2] = v.z + rest[j + 2]; rest[j + 3] = v.w + rest[j + 3];
+                            }
+                        }
+                    }
+                }
+                // the flag is read by all before the next item's writer may change it
+                if (!eb.sync()) break;
+            }
             // warp-uniform decision: the TMEM loads below are warp-collective
             if (!__all_sync(0xffffffffu, mbar_wait(&tfull[a], aph, p.timeout_ns))) break;
             tc_fence_after();
@@ -259,6 +357,53 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&tempty[a]);   // accumulator is in registers now
+
+            if (have_rest) {
+#pragma unroll
+                for (int j = 0; j < NR; ++j) acc[j] = acc[j] + rest[j];
+            } else if (cut) {
+                // publish this piece's partial row and take the tile's ticket;
+                // the last piece to arrive adds all of the tile's pieces
+                const int my_slot = (u_piece == u_begin && u_begin >= ts) ? 0 : 1;
+                float *mine = p.part + ((int64_t)(blockIdx.x * 2 + my_slot) * BM + L) * NT;
+#pragma unroll
+                for (int j = 0; j < NT; j += 4)
+                    __stcg(reinterpret_cast<float4 *>(mine + j), make_float4(acc[j], acc[j + 1], acc[j + 2], acc[j + 3]));
+                // the barrier orders every epilogue thread's stores before the
+                // ticket thread's fence, whose release covers them; the last
+                // piece's ticket thread fences again before the barrier that
+                // releases the other threads to read
+                if (!eb.sync()) break;
+                if (et == 0) {
+                    __threadfence();
+                    const bool last = atomicAdd(p.tickets + c_first, 1u) == (unsigned)(c_last - c_first);
+                    if (last) __threadfence();
+                    *s_last = last;
+                }
+                if (!eb.sync()) break;
+                if (!*s_last) continue;
+                float sum[NT];
+                for (int c = c_last; c >= c_first; --c) {
+                    if (c == (int)blockIdx.x) {
+#pragma unroll
+                        for (int j = 0; j < NT; ++j) sum[j] = c == c_last ? acc[j] : acc[j] + sum[j];
+                    } else {
+                        const float *src = p.part + ((int64_t)(c * 2 + (wk.begin(c) >= ts ? 0 : 1)) * BM + L) * NT;
+#pragma unroll
+                        for (int j = 0; j < NT; j += 4) {
+                            const float4 v = __ldcg(reinterpret_cast<const float4 *>(src + j));
+                            if (c == c_last) {
+                                sum[j] = v.x; sum[j + 1] = v.y; sum[j + 2] = v.z; sum[j + 3] = v.w;
+                            } else {
+                                sum[j] = v.x + sum[j]; sum[j + 1] = v.y + sum[j + 1];
+                                sum[j + 2] = v.z + sum[j + 2]; sum[j + 3] = v.w + sum[j + 3];
+                            }
+                        }
+                    }
+                }
+#pragma unroll
+                for (int j = 0; j < NT; ++j) acc[j] = sum[j];
+            }
 
             if (EPI == EPI_SCATTER) {
                 const int d = mt * BM + L;

@@ -18,10 +18,10 @@
 //   probability sums are reduced in a fixed order (lanes, then warps), its
 //   counts and gate-weight sums with shared-memory atomics on integers (gate
 //   weights in 2^-32 fixed point), which are exact and order-independent.
-// router_few_kernel  one block per token (T <= 64, N <= 32): every thread
-//   streams its rows of W_g with all loads in flight, warps reduce-scatter the
-//   partial scores, warp 0 selects the top k; the token's probabilities, gate
-//   weights and counts are its partials.
+// router_few_kernel  few tokens (T <= 64, N <= 32): several blocks per token,
+//   each over a slab of W_g rows with lane = expert (coalesced row loads); the
+//   block completing a token adds the slabs in order and selects the top k;
+//   the token's probabilities, gate weights and counts are its partials.
 // In both, the last block to finish (atomic ticket) turns the per-tile (or
 // per-token) partials into the dispatch tables -- per tile and expert the first
 // row of its tokens inside the expert's segment, per-expert counts and offsets,
@@ -211,14 +211,19 @@ __device__ void finalize_tables(const Params &p, int ntiles, FinalScratch &f) {
 }
 
 // True in every thread of the block that finished last.
+// The barrier orders the block's stores before thread 0's fence (a release
+// that covers them); the last block's thread 0 fences again before the
+// barrier that lets its other threads read what the other blocks wrote.
 __device__ __forceinline__ bool last_block(unsigned *ticket, int *s_flag) {
-    __threadfence();
     __syncthreads();
-    if (threadIdx.x == 0) *s_flag = atomicAdd(ticket, 1u) == gridDim.x - 1;
+    if (threadIdx.x == 0) {
+        __threadfence();
+        const bool last = atomicAdd(ticket, 1u) == gridDim.x - 1;
+        if (last) __threadfence();
+        *s_flag = last;
+    }
     __syncthreads();
-    const bool last = *s_flag != 0;
-    if (last) __threadfence();
-    return last;
+    return *s_flag != 0;
 }
 
 template <int NP>
@@ -471,45 +476,63 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ---------------------------------------------------------------------------
-// Few tokens (T <= 64), N <= 32: one block of 256 threads per token.  Thread i
-// accumulates rows i, i+256, ... of W_g (four rows' loads issued together), the
-// 8 warps' partial scores are reduce-scattered (lane e: expert e) and added in
-// warp order by warp 0, which then selects the top k.  The token's partials are
-// its full-softmax probabilities, gate weights and counts (one-token "tiles").
+// Few tokens (T <= 64, N <= 32): grid (T, S).  Block (t, s) takes the rows
+// [s*rows, (s+1)*rows) of W_g; lane e of every warp owns expert e, so each
+// warp-wide load reads one contiguous W_g row, and warp w takes the slab's rows
+// w, w+8, ... with kFewUnroll rows in flight.  The block adds its warps' sums
+// in warp order and publishes the slab's scores; the block that completes a
+// token (an atomic ticket per token) adds the S slabs in slab order, selects
+// the top k and writes the token's partials (full-softmax probabilities, gate
+// weights, counts: one-token "tiles"); the last token's block builds the
+// tables.  Every sum has a fixed order, so results do not depend on scheduling.
 // ---------------------------------------------------------------------------
-template <int NP>
+constexpr int kFewUnroll = 16;
+constexpr int kFewMaxSplits = 16;
+
 __global__ void __launch_bounds__(256) router_few_kernel(const __nv_bfloat16 *__restrict__ x,
-                                                          const __nv_bfloat16 *__restrict__ Wg, const Params p) {
+                                                          const __nv_bfloat16 *__restrict__ Wg, const Params p,
+                                                          float *__restrict__ slab_scores,   // [T][S][32]
+                                                          unsigned *__restrict__ token_ticket, int rows) {
     __shared__ float part[8][32];
     __shared__ FinalScratch fs;
     __shared__ int s_flag;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int t = blockIdx.x, N = p.N, D = p.D;
-    float a[32];
-#pragma unroll
-    for (int i = 0; i < 32; ++i) a[i] = 0.f;
+    const int t = blockIdx.x, sl = blockIdx.y, S = gridDim.y, N = p.N, D = p.D;
+    const bool live = lane < N;
+    const int d_begin = sl * rows, d_end = min(D, d_begin + rows);
     const __nv_bfloat16 *xt = x + (int64_t)t * D;
-    for (int d0 = tid; d0 < D; d0 += 4 * 256) {
-        float xv[4], wv[4][NP];
+    float acc = 0.f;
+    for (int d0 = d_begin + warp; d0 < d_end; d0 += 8 * kFewUnroll) {
+        float wv[kFewUnroll], xv[kFewUnroll];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const int d = d0 + u * 256;
-            xv[u] = d < D ? __bfloat162float(xt[d]) : 0.f;
-#pragma unroll
-            for (int e = 0; e < NP; ++e) wv[u][e] = (d < D && e < N) ? __bfloat162float(Wg[(int64_t)d * N + e]) : 0.f;
+        for (int u = 0; u < kFewUnroll; ++u) {
+            const int d = d0 + 8 * u;
+            const bool in = d < d_end;
+            xv[u] = in ? __bfloat162float(xt[d]) : 0.f;
+            wv[u] = (in && live) ? __bfloat162float(Wg[(int64_t)d * N + lane]) : 0.f;
         }
 #pragma unroll
-        for (int u = 0; u < 4; ++u)
-#pragma unroll
-            for (int e = 0; e < NP; ++e) a[e] = fmaf(xv[u], wv[u][e], a[e]);
+        for (int u = 0; u < kFewUnroll; ++u) acc = fmaf(xv[u], wv[u], acc);
     }
-    reduce_scatter32(a, lane);   // lane l: this warp's sum for expert l
-    part[warp][lane] = a[0];
+    part[warp][lane] = acc;
     __syncthreads();
     if (warp == 0) {
+        float v = 0.f;
+        for (int w = 0; w < 8; ++w) v += part[w][lane];
+        slab_scores[((int64_t)t * S + sl) * 32 + lane] = v;
+    }
+    __syncthreads();
+    if (tid == 0) {
+        __threadfence();
+        const bool last = atomicAdd(token_ticket + t, 1u) == (unsigned)(S - 1);
+        if (last) __threadfence();
+        s_flag = last;
+    }
+    __syncthreads();
+    if (!s_flag) return;   // block-uniform: another slab completes this token
+    if (warp == 0) {
         float s = 0.f;
-        for (int w = 0; w < 8; ++w) s += part[w][lane];
-        const bool live = lane < N;
+        for (int j = 0; j < S; ++j) s += __ldcg(slab_scores + ((int64_t)t * S + j) * 32 + lane);
         s = live ? score(p.bg, s, lane) : -INFINITY;
         if (live) p.logits[(int64_t)t * N + lane] = s;
         int slot_e;

@@ -391,7 +391,7 @@ def test_route_entry_point_matches_forward():
 
 
 def test_bitwise_deterministic_runs():
-    for name, T in [("gpt2", 2000), ("mixtral", 300)]:
+    for name, T in [("gpt2", 2000), ("mixtral", 300), ("decode1", 1), ("decode8", 8)]:
         wl = WORKLOADS[name]
         inp = make_inputs(wl, "cuda", T=T)
         layer = Layer(wl, inp)
