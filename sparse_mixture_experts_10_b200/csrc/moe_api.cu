@@ -252,22 +252,39 @@ int make_map(CUtensorMap *m, const void *base, int64_t rows, int64_t cols, int b
     return r == CUDA_SUCCESS ? MOE_OK : MOE_ERR_CUDA;
 }
 
+// 2-D bf16 matrix [rows, cols] row-major as the destination of the epilogue's
+// bulk stores: boxes of 32 rows x 16 columns, no swizzle.
+int make_store_map(CUtensorMap *m, void *base, int64_t rows, int64_t cols) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return MOE_ERR_CUDA;
+    const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+    const cuuint32_t box[2] = {16u, 32u};
+    const cuuint32_t estr[2] = {1u, 1u};
+    const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, estr,
+                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? MOE_OK : MOE_ERR_CUDA;
+}
+
+// O: destination map of bf16 outputs (EPI_GELU, EPI_SWIGLU); other epilogues
+// store directly and get A in its place (unused).
 template <int BN, int EPI>
-int launch_tc(const CUtensorMap &A, const CUtensorMap &B, const tc::Params &p, int64_t tiles_upper, int sms,
-              cudaStream_t s) {
+int launch_tc(const CUtensorMap &A, const CUtensorMap &B, const CUtensorMap &O, const tc::Params &p,
+              int64_t tiles_upper, int sms, cudaStream_t s) {
     const int grid = (int)std::min<int64_t>(std::max<int64_t>(tiles_upper, 1), sms);
     const size_t smem = tc::Shape<BN>::smem_bytes(p.num_groups);
-    tc::grouped_gemm_tc_kernel<BN, EPI><<<grid, tc::kThreads, smem, s>>>(A, B, p);
+    tc::grouped_gemm_tc_kernel<BN, EPI><<<grid, tc::kThreads, smem, s>>>(A, B, O, p);
     return check_launch();
 }
 
 // Pair (2-CTA cluster) version for 256-column tiles: 256-row units per cluster.
 template <int EPI>
-int launch_tc2(const CUtensorMap &A, const CUtensorMap &B, const tc::Params &p, int64_t units_upper, int sms,
-               cudaStream_t s) {
+int launch_tc2(const CUtensorMap &A, const CUtensorMap &B, const CUtensorMap &O, const tc::Params &p,
+               int64_t units_upper, int sms, cudaStream_t s) {
     const int64_t clusters = std::min<int64_t>(std::max<int64_t>(units_upper, 1), sms / 2);
     const size_t smem = tc::Shape2::smem_bytes(p.num_groups);
-    tc::grouped_gemm_tc2_kernel<EPI><<<(unsigned)(2 * clusters), tc::kThreads, smem, s>>>(A, B, p);
+    tc::grouped_gemm_tc2_kernel<EPI><<<(unsigned)(2 * clusters), tc::kThreads, smem, s>>>(A, B, O, p);
     return check_launch();
 }
 
@@ -411,7 +428,7 @@ int stage_route(const Plan &P, const Bufs &b, const void *x, const moe_weights *
         p.ldo = N;
         p.bias = w->b_g;
         p.timeout_ns = kTimeoutNs;
-        MOE_TRY((launch_tc2<tc::EPI_LOGITS>(ma, mb, p, cdiv(T, 2 * tc::BM) * p.n_tiles, dev.sms, s)));
+        MOE_TRY((launch_tc2<tc::EPI_LOGITS>(ma, mb, ma, p, cdiv(T, 2 * tc::BM) * p.n_tiles, dev.sms, s)));
     } else {
         float *wgt = b.at<float>(P.wgt);
         transpose_kernel<float><<<dim3((unsigned)cdiv(N, 32), (unsigned)cdiv(D, 32)), dim3(32, 8), 0, s>>>(
@@ -578,14 +595,16 @@ int stage_up(const Plan &P, const Bufs &b, const moe_weights *w, const DeviceInf
         p.ldo = H;
         p.bias = swiglu ? nullptr : w->b1;
         p.timeout_ns = kTimeoutNs;
+        CUtensorMap mo;
+        MOE_TRY(make_store_map(&mo, b.ws + P.h, P.rows_cap, H));
         const int64_t upper = (P.rows_cap / tc::BM) * p.n_tiles;
         if (bn == 128) {
-            if (swiglu) return launch_tc<128, tc::EPI_SWIGLU>(ma, mb, p, upper, dev.sms, s);
-            return launch_tc<128, tc::EPI_GELU>(ma, mb, p, upper, dev.sms, s);
+            if (swiglu) return launch_tc<128, tc::EPI_SWIGLU>(ma, mb, mo, p, upper, dev.sms, s);
+            return launch_tc<128, tc::EPI_GELU>(ma, mb, mo, p, upper, dev.sms, s);
         }
         const int64_t units = (P.rows_cap / (2 * tc::BM) + N) * p.n_tiles;
-        if (swiglu) return launch_tc2<tc::EPI_SWIGLU>(ma, mb, p, units, dev.sms, s);
-        return launch_tc2<tc::EPI_GELU>(ma, mb, p, units, dev.sms, s);
+        if (swiglu) return launch_tc2<tc::EPI_SWIGLU>(ma, mb, mo, p, units, dev.sms, s);
+        return launch_tc2<tc::EPI_GELU>(ma, mb, mo, p, units, dev.sms, s);
     }
     simt::Params p{};
     p.A = b.at<float>(P.x_perm);
@@ -628,8 +647,8 @@ int stage_down(const Plan &P, const Bufs &b, const moe_weights *w, const DeviceI
         p.gate_w = b.at<float>(P.w);
         p.timeout_ns = kTimeoutNs;
         const int64_t upper = (P.rows_cap / tc::BM) * p.n_tiles;
-        if (bn == 128) return launch_tc<128, tc::EPI_SCATTER>(ma, mb, p, upper, dev.sms, s);
-        return launch_tc2<tc::EPI_SCATTER>(ma, mb, p, (P.rows_cap / (2 * tc::BM) + N) * p.n_tiles, dev.sms, s);
+        if (bn == 128) return launch_tc<128, tc::EPI_SCATTER>(ma, mb, ma, p, upper, dev.sms, s);
+        return launch_tc2<tc::EPI_SCATTER>(ma, mb, ma, p, (P.rows_cap / (2 * tc::BM) + N) * p.n_tiles, dev.sms, s);
     }
     simt::Params p{};
     p.A = b.at<float>(P.h);

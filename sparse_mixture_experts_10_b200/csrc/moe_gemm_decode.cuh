@@ -423,7 +423,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int f = mt * BM + L;
                 const float b = (p.bias && f < p.n_valid) ? __ldg(p.bias + (int64_t)g * p.n_valid + f) : 0.f;
 #pragma unroll
-                for (int j = 0; j < NT; ++j) o[j * 128 + L] = __float2bfloat16_rn(tc::gelu_erf(acc[j] + b));
+                for (int j = 0; j < NT; j += 2) {
+                    const uint32_t hv = tc::gelu_erf_bf16x2(acc[j] + b, acc[j + 1] + b);
+                    o[j * 128 + L] = __ushort_as_bfloat16(static_cast<unsigned short>(hv & 0xffffu));
+                    o[(j + 1) * 128 + L] = __ushort_as_bfloat16(static_cast<unsigned short>(hv >> 16));
+                }
                 if (!eb.sync()) break;
                 __nv_bfloat16 *h = static_cast<__nv_bfloat16 *>(p.out);
                 const int f0 = mt * BM;
@@ -452,10 +456,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!eb.sync()) break;
                 if (L < 64) {
 #pragma unroll
-                    for (int j = 0; j < NT; ++j) {
-                        const float gt = acc[j];
-                        const float hv = gt / (1.0f + __expf(-gt)) * up[j * 64 + L];
-                        o[j * 64 + L] = __float2bfloat16_rn(hv);
+                    for (int j = 0; j < NT; j += 2) {
+                        const uint32_t hv = tc::swiglu_bf16x2(acc[j], acc[j + 1], up[j * 64 + L], up[(j + 1) * 64 + L]);
+                        o[j * 64 + L] = __ushort_as_bfloat16(static_cast<unsigned short>(hv & 0xffffu));
+                        o[(j + 1) * 64 + L] = __ushort_as_bfloat16(static_cast<unsigned short>(hv >> 16));
                     }
                 }
                 if (!eb.sync()) break;

@@ -81,6 +81,11 @@ struct Params {
     uint64_t timeout_ns;
 };
 
+// bf16 output staging for the bulk tensor stores: 32 rows x 16 columns per
+// epilogue warp.
+constexpr uint32_t kOutStageWarpBytes = 32 * 16 * 2;
+constexpr uint32_t kOutStageBytes = kEpiWarps * kOutStageWarpBytes;
+
 template <int BN>
 struct Shape {
     static constexpr int kStages = BN == 256 ? 4 : 6;   // 192 KB of ring either way
@@ -88,9 +93,10 @@ struct Shape {
     static constexpr uint32_t kBBytes = BN * BK * 2;
     static constexpr uint32_t kTmemCols = 2 * BN;
     static constexpr size_t kBarrierBytes = (2 * kStages + 5) * 8 + 16;
-    // ring + alignment slack + barriers + tmem slot; the group table follows
+    // ring + alignment slack + output staging + barriers + tmem slot; the group table follows
     static size_t smem_bytes(int groups) {
-        return 1024 + kStages * (size_t)(kABytes + kBBytes) + kBarrierBytes + 4 * (size_t)(groups + 1) + 16;
+        return 1024 + kStages * (size_t)(kABytes + kBBytes) + kOutStageBytes + kBarrierBytes +
+               4 * (size_t)(groups + 1) + 16;
     }
 };
 
@@ -101,9 +107,10 @@ struct Shape2 {
     static constexpr uint32_t kBBytes = 128 * BK * 2;
     static constexpr uint32_t kTmemCols = 512;
     static constexpr size_t kBarrierBytes = (2 * kStages + 5) * 8 + 16;
-    // ring + slack + barriers + tmem slot; group table and 256-row unit table follow
+    // ring + slack + output staging + barriers + tmem slot; group table and 256-row unit table follow
     static size_t smem_bytes(int groups) {
-        return 1024 + kStages * (size_t)(kABytes + kBBytes) + kBarrierBytes + 8 * (size_t)(groups + 1) + 16;
+        return 1024 + kStages * (size_t)(kABytes + kBBytes) + kOutStageBytes + kBarrierBytes +
+               8 * (size_t)(groups + 1) + 16;
     }
 };
 
@@ -162,51 +169,52 @@ __device__ __forceinline__ TileCoord decode_unit_tile(int i, const int *s_rowoff
     return c;
 }
 
-// 1/x for x in [1, 2.32] without the special-function unit: quadratic seed
-// (relative error < 1.8e-2, fitted here by weighted least squares) and two
-// Newton steps r <- r (2 - x r) (error squares each step: < 1e-7).
-__device__ __forceinline__ float rcp_1_2(float x) {
-    float r = fmaf(fmaf(0.24989176f, x, -1.24085286f), x, 1.97339064f);
-    r = r * fmaf(-x, r, 2.0f);
-    r = r * fmaf(-x, r, 2.0f);
-    return r;
+// GELU(v) = v Phi(v), exact-erf form, on a pair of values.  With
+// Phi(-|v|) = erfc(|v| / sqrt 2) / 2 from Abramowitz & Stegun, Handbook of
+// Mathematical Functions, formula 7.1.26 (absolute error of erf at most
+// 1.5e-7):
+//   erfc(z) ~ (a1 t + a2 t^2 + a3 t^3 + a4 t^4 + a5 t^5) exp(-z^2),  t = 1 / (1 + p z),
+// and v Phi(v) = relu(v) - |v| Phi(-|v|) for either sign of v (no
+// cancellation for v < 0).  The factor -1/2 is folded into the coefficients,
+// p into p / sqrt 2; exp(-v^2 / 2) = 2^(-v^2 log2(e) / 2).  Per pair: eleven
+// f32x2 instructions, two reciprocals and two exponentials on the
+// special-function unit.  Returns the two results rounded to bf16.
+__device__ __forceinline__ uint32_t gelu_erf_bf16x2(float v0, float v1) {
+    constexpr float kP = 0.2316418882663604f;          // p / sqrt 2, p = 0.3275911
+    constexpr float kB1 = -0.127414796f, kB2 = 0.142248368f, kB3 = -0.7107068705f,
+                    kB4 = 0.7265760135f, kB5 = -0.5307027145f;   // -a_i / 2
+    constexpr float kL = 0.7213475204444817f;          // log2(e) / 2
+    const float a0 = fabsf(v0), a1 = fabsf(v1);
+    const uint64_t v = f2_pack(v0, v1), a = f2_pack(a0, a1);
+    float d0, d1;
+    f2_unpack(f2_fma(a, f2_splat(kP), f2_splat(1.0f)), d0, d1);
+    const uint64_t t = f2_pack(rcp_approx(d0), rcp_approx(d1));
+    uint64_t q = f2_fma(t, f2_splat(kB5), f2_splat(kB4));
+    q = f2_fma(t, q, f2_splat(kB3));
+    q = f2_fma(t, q, f2_splat(kB2));
+    q = f2_fma(t, q, f2_splat(kB1));
+    q = f2_mul(q, t);                                   // -erfc-series / 2 without the Gaussian
+    float g0, g1;
+    f2_unpack(f2_mul(f2_mul(v, f2_splat(-kL)), v), g0, g1);
+    const uint64_t nphi = f2_mul(q, f2_pack(ex2_approx(g0), ex2_approx(g1)));   // -Phi(-|v|)
+    const uint64_t out = f2_fma(f2_add(v, a), f2_splat(0.5f), f2_mul(a, nphi));
+    float o0, o1;
+    f2_unpack(out, o0, o1);
+    return pack_bf16x2(o0, o1);
 }
 
-// 2^y for y in [-126, 0] without the special-function unit: y = n + f with n
-// integer (rounded by adding 1.5 * 2^23) and |f| <= 1/2; 2^f by a degree-6
-// polynomial fitted here (relative error < 2e-9); n goes into the exponent bits.
-__device__ __forceinline__ float exp2_fma(float y) {
-    y = fmaxf(y, -126.0f);
-    const float t = y + 12582912.0f;
-    const float f = y - (t - 12582912.0f);
-    float q = fmaf(1.53458105e-4f, f, 1.33999315e-3f);
-    q = fmaf(q, f, 9.61848897e-3f);
-    q = fmaf(q, f, 5.55032878e-2f);
-    q = fmaf(q, f, 0.240226469f);
-    q = fmaf(q, f, 0.693147206f);
-    q = fmaf(q, f, 1.0f);
-    return __int_as_float(__float_as_int(q) + ((__float_as_int(t) - 0x4B400000) << 23));
+// SwiGLU on a pair: silu(g) u = g u / (1 + 2^(-g log2 e)), rounded to bf16.
+__device__ __forceinline__ uint32_t swiglu_bf16x2(float g0, float g1, float u0, float u1) {
+    constexpr float kLog2e = 1.4426950408889634f;
+    const uint64_t g = f2_pack(g0, g1);
+    float e0, e1;
+    f2_unpack(f2_mul(g, f2_splat(-kLog2e)), e0, e1);
+    float d0, d1;
+    f2_unpack(f2_add(f2_pack(ex2_approx(e0), ex2_approx(e1)), f2_splat(1.0f)), d0, d1);
+    float o0, o1;
+    f2_unpack(f2_mul(f2_mul(g, f2_pack(u0, u1)), f2_pack(rcp_approx(d0), rcp_approx(d1))), o0, o1);
+    return pack_bf16x2(o0, o1);
 }
-
-// GELU(v) = v Phi(v) = 0.5 v (1 + erf(v / sqrt 2)), exact-erf form, with erfc
-// from Abramowitz & Stegun, Handbook of Mathematical Functions, formula 7.1.26
-// (absolute error of erf at most 1.5e-7):
-//   erfc(z) ~ (a1 t + a2 t^2 + a3 t^3 + a4 t^4 + a5 t^5) exp(-z^2), t = 1 / (1 + p z), z >= 0.
-// For v < 0, 1 + erf(v / sqrt 2) = erfc(|v| / sqrt 2) is used directly (no
-// cancellation).  z is capped at 4, where erfc < 1.6e-8.  The reciprocal runs
-// on the FMA pipe (rcp_1_2); one special-function op (the exponential) per
-// value.  Absolute error of the whole function below 5e-7.
-__device__ __forceinline__ float gelu_erf(float v) {
-    const float z = fminf(fabsf(v) * 0.70710678118654752f, 4.0f);
-    const float t = rcp_1_2(fmaf(0.3275911f, z, 1.0f));
-    float poly = fmaf(t, 1.061405429f, -1.453152027f);
-    poly = fmaf(t, poly, 1.421413741f);
-    poly = fmaf(t, poly, -0.284496736f);
-    poly = fmaf(t, poly, 0.254829592f);
-    const float q = poly * t * __expf(-z * z);
-    return (0.5f * v) * (v >= 0.f ? 2.0f - q : q);
-}
-__device__ __forceinline__ float silu_f(float g) { return g / (1.0f + __expf(-g)); }
 
 __device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t (&r)[16]) {
     asm volatile(
@@ -215,6 +223,16 @@ __device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t (&r)
         : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
           "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
         : "r"(taddr));
+}
+
+// tcgen05.wait::ld that also names the registers of the load it completes, so
+// that their uses cannot be scheduled above it.
+__device__ __forceinline__ void tmem_ld_wait_regs(uint32_t (&r)[16]) {
+    asm volatile("tcgen05.wait::ld.sync.aligned;"
+                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+                   "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15])
+                 :
+                 : "memory");
 }
 
 __device__ __forceinline__ void store_bf16x16(__nv_bfloat16 *dst, const uint32_t (&pk)[8], int n0, int n_valid) {
@@ -234,9 +252,34 @@ __device__ __forceinline__ void store_bf16x16(__nv_bfloat16 *dst, const uint32_t
 // group `grp` (of kEpiGroups) of the tile is its share, in 16-column chunks.
 // Rows at or beyond row_limit are not stored.  Every lane executes the TMEM
 // loads (they are warp-wide).
+// Stores one warp's 32 rows x 16 bf16 columns (pk: this lane's row) at
+// (column n0, row row0): through the warp's shared staging tile and one bulk
+// tensor store when all 32 rows are valid (rows of a 128-row aligned segment),
+// else row by row.
+__device__ __forceinline__ void store_h_chunk(const CUtensorMap *tmO, uint8_t *stage, __nv_bfloat16 *out,
+                                              int64_t ldo, int row, bool row_ok, const uint32_t (&pk)[8], int n0,
+                                              int n_valid) {
+    const int lane = threadIdx.x & 31;
+    if (__all_sync(0xffffffffu, row_ok)) {
+        if (lane == 0) bulk_wait_read_all();   // the previous store has read the staging tile
+        __syncwarp();
+        uint4 *dst = reinterpret_cast<uint4 *>(stage + lane * 32);
+        dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+            tma_store_2d(tmO, stage, n0, row - lane);
+            bulk_commit();
+        }
+    } else if (row_ok) {
+        store_bf16x16(out + (int64_t)row * ldo + n0, pk, n0, n_valid);
+    }
+}
+
 template <int BN, int EPI>
 __device__ __forceinline__ void epilogue_tile(const Params &p, const TileCoord &c, int row, int row_limit,
-                                              uint32_t tbase, int grp) {
+                                              uint32_t tbase, int grp, const CUtensorMap *tmO, uint8_t *stage) {
     const bool row_ok = row < row_limit;
     if (EPI == EPI_SWIGLU) {
         constexpr int kOutCols = BN / 2;                  // h columns per tile
@@ -249,93 +292,101 @@ __device__ __forceinline__ void epilogue_tile(const Params &p, const TileCoord &
             tmem_ld_32x32b_x16(tbase + col, rg);
             tmem_ld_32x32b_x16(tbase + kOutCols + col, ru);
             tmem_ld_wait();
-            if (!row_ok) continue;
             const int n0 = c.nt * kOutCols + col;
+            if (!__any_sync(0xffffffffu, row_ok) || n0 >= p.n_valid) continue;   // warp-uniform
             uint32_t pk[8];
 #pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                const float h0 = silu_f(__uint_as_float(rg[2 * k])) * __uint_as_float(ru[2 * k]);
-                const float h1 = silu_f(__uint_as_float(rg[2 * k + 1])) * __uint_as_float(ru[2 * k + 1]);
-                pk[k] = pack_bf16x2(h0, h1);
-            }
-            store_bf16x16(out + (int64_t)row * p.ldo + n0, pk, n0, p.n_valid);
+            for (int k = 0; k < 8; ++k)
+                pk[k] = swiglu_bf16x2(__uint_as_float(rg[2 * k]), __uint_as_float(rg[2 * k + 1]),
+                                      __uint_as_float(ru[2 * k]), __uint_as_float(ru[2 * k + 1]));
+            store_h_chunk(tmO, stage, out, p.ldo, row, row_ok, pk, n0, p.n_valid);
         }
         return;
     }
     constexpr int kPerGroup = BN / kEpiGroups;
+    constexpr int kChunks = kPerGroup / 16;
     int slot = -1;
     float gw = 0.f;
     if (EPI == EPI_SCATTER && row_ok) {
         slot = p.perm_slot[row];
         if (slot >= 0) gw = p.gate_w[slot];
     }
-#pragma unroll 1
-    for (int cc = 0; cc < kPerGroup; cc += 16) {
-        const int col = grp * kPerGroup + cc;
-        uint32_t r[16];
-        tmem_ld_32x32b_x16(tbase + col, r);
-        tmem_ld_wait();
-        const int n0 = c.nt * BN + col;
-        if (n0 >= p.n_valid || !row_ok) continue;
-        if (EPI == EPI_SCATTER && slot < 0) continue;
-        const bool full_chunk = n0 + 16 <= p.n_valid;
-        float v[16];
+    const float *bias_row = p.bias ? p.bias + (int64_t)c.g * p.n_valid : nullptr;
+    // Chunks of 16 columns, software-pipelined: tcgen05.wait::ld waits for all
+    // of a thread's outstanding loads, so chunk i+1's TMEM load is issued right
+    // after chunk i's wait and runs while chunk i is computed; chunk i's bias
+    // loads go out before its wait.
+    uint32_t r[2][16];
+    tmem_ld_32x32b_x16(tbase + grp * kPerGroup, r[0]);
 #pragma unroll
-        for (int k = 0; k < 16; ++k) v[k] = __uint_as_float(r[k]);
-        if (p.bias) {
-            const float *bias = p.bias + (int64_t)c.g * p.n_valid + n0;
+    for (int ci = 0; ci < kChunks; ++ci) {
+        const int col = grp * kPerGroup + ci * 16;
+        const int n0 = c.nt * BN + col;
+        // GELU: the store below is warp-collective, so lanes of invalid rows come along
+        const bool active = (EPI == EPI_GELU ? __any_sync(0xffffffffu, row_ok) : row_ok) && n0 < p.n_valid &&
+                            !(EPI == EPI_SCATTER && slot < 0);
+        const bool full_chunk = n0 + 16 <= p.n_valid;
+        float bv[16];
+#pragma unroll
+        for (int k = 0; k < 16; ++k) bv[k] = 0.f;
+        if (bias_row && active) {
+            const float *bias = bias_row + n0;
             if (full_chunk) {
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
                     const float4 b4 = __ldg(reinterpret_cast<const float4 *>(bias) + u);
-                    v[4 * u] += b4.x; v[4 * u + 1] += b4.y; v[4 * u + 2] += b4.z; v[4 * u + 3] += b4.w;
+                    bv[4 * u] = b4.x; bv[4 * u + 1] = b4.y; bv[4 * u + 2] = b4.z; bv[4 * u + 3] = b4.w;
                 }
             } else {
 #pragma unroll
                 for (int k = 0; k < 16; ++k)
-                    if (n0 + k < p.n_valid) v[k] += __ldg(bias + k);
+                    if (n0 + k < p.n_valid) bv[k] = __ldg(bias + k);
             }
         }
-        if (EPI == EPI_GELU) {
-            uint32_t pk[8];
+        tmem_ld_wait_regs(r[ci & 1]);
+        if (ci + 1 < kChunks) tmem_ld_32x32b_x16(tbase + col + 16, r[(ci + 1) & 1]);
+        if (active) {
+            float v[16];
 #pragma unroll
-            for (int k = 0; k < 8; ++k) pk[k] = pack_bf16x2(gelu_erf(v[2 * k]), gelu_erf(v[2 * k + 1]));
-            store_bf16x16(static_cast<__nv_bfloat16 *>(p.out) + (int64_t)row * p.ldo + n0, pk, n0, p.n_valid);
-        } else if (EPI == EPI_SCATTER) {
-            float *dst = static_cast<float *>(p.out) + (int64_t)slot * p.ldo + n0;
-            if (full_chunk) {
+            for (int k = 0; k < 16; ++k) v[k] = __uint_as_float(r[ci & 1][k]) + bv[k];
+            if (EPI == EPI_GELU) {
+                uint32_t pk[8];
 #pragma unroll
-                for (int u = 0; u < 4; ++u)
-                    reinterpret_cast<float4 *>(dst)[u] =
-                        make_float4(gw * v[4 * u], gw * v[4 * u + 1], gw * v[4 * u + 2], gw * v[4 * u + 3]);
-            } else {
+                for (int k = 0; k < 8; ++k) pk[k] = gelu_erf_bf16x2(v[2 * k], v[2 * k + 1]);
+                store_h_chunk(tmO, stage, static_cast<__nv_bfloat16 *>(p.out), p.ldo, row, row_ok, pk, n0, p.n_valid);
+            } else if (EPI == EPI_SCATTER) {
+                float *dst = static_cast<float *>(p.out) + (int64_t)slot * p.ldo + n0;
+                if (full_chunk) {
+#pragma unroll
+                    for (int u = 0; u < 4; ++u)
+                        reinterpret_cast<float4 *>(dst)[u] =
+                            make_float4(gw * v[4 * u], gw * v[4 * u + 1], gw * v[4 * u + 2], gw * v[4 * u + 3]);
+                } else {
+#pragma unroll
+                    for (int k = 0; k < 16; ++k)
+                        if (n0 + k < p.n_valid) dst[k] = gw * v[k];
+                }
+            } else {  // EPI_LOGITS
+                float *dst = static_cast<float *>(p.out) + (int64_t)row * p.ldo + n0;
 #pragma unroll
                 for (int k = 0; k < 16; ++k)
-                    if (n0 + k < p.n_valid) dst[k] = gw * v[k];
+                    if (n0 + k < p.n_valid) dst[k] = v[k];
             }
-        } else {  // EPI_LOGITS
-            float *dst = static_cast<float *>(p.out) + (int64_t)row * p.ldo + n0;
-#pragma unroll
-            for (int k = 0; k < 16; ++k)
-                if (n0 + k < p.n_valid) dst[k] = v[k];
         }
     }
 }
-
-// =====================================================================================
-// One CTA per 128-row tile.
-// =====================================================================================
 template <int BN, int EPI>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                           const Params p) {
+                           const __grid_constant__ CUtensorMap tmO, const Params p) {
     using S = Shape<BN>;
     constexpr int kStages = S::kStages;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sA = smem;
     uint8_t *sB = smem + kStages * S::kABytes;
-    uint64_t *full = reinterpret_cast<uint64_t *>(sB + kStages * S::kBBytes);
+    uint8_t *sOut = sB + kStages * S::kBBytes;
+    uint64_t *full = reinterpret_cast<uint64_t *>(sOut + kOutStageBytes);
     uint64_t *empty = full + kStages;
     uint64_t *tfull = empty + kStages;
     uint64_t *tempty = tfull + 2;
@@ -470,11 +521,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_after();
             const int row_limit = rowoff ? s_rowoff[c.g + 1] : p.dense_rows;
             epilogue_tile<BN, EPI>(p, c, c.row0 + r_in_tile, row_limit,
-                                   tmem_base + (static_cast<uint32_t>(q * 32) << 16) + a * BN, grp);
+                                   tmem_base + (static_cast<uint32_t>(q * 32) << 16) + a * BN, grp, &tmO,
+                                   sOut + ew * kOutStageWarpBytes);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&tempty[a]);
         }
+        if (lane == 0) bulk_wait_all();   // this warp's bulk stores are complete before the CTA exits
     }
     tc_fence_before();
     __syncthreads();
@@ -585,7 +638,7 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint64_t *bar, uint32_t parity
 template <int EPI>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     grouped_gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                            const Params p) {
+                            const __grid_constant__ CUtensorMap tmO, const Params p) {
     using S = Shape2;
     constexpr int BN = 256;
     constexpr int kStages = S::kStages;
@@ -593,7 +646,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sA = smem;
     uint8_t *sB = smem + kStages * S::kABytes;
-    uint64_t *full = reinterpret_cast<uint64_t *>(sB + kStages * S::kBBytes);
+    uint8_t *sOut = sB + kStages * S::kBBytes;
+    uint64_t *full = reinterpret_cast<uint64_t *>(sOut + kOutStageBytes);
     uint64_t *empty = full + kStages;
     uint64_t *tfull = empty + kStages;
     uint64_t *tempty = tfull + 2;
@@ -742,11 +796,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             tc_fence_after();
             const int row_limit = rowoff ? s_rowoff[c.g + 1] : p.dense_rows;
             epilogue_tile<BN, EPI>(p, c, c.row0 + (int)rank * BM + r_in_tile, row_limit,
-                                   tmem_base + (static_cast<uint32_t>(q * 32) << 16) + a * BN, grp);
+                                   tmem_base + (static_cast<uint32_t>(q * 32) << 16) + a * BN, grp, &tmO,
+                                   sOut + ew * kOutStageWarpBytes);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive_remote(mapa_shared(smem_u32(&tempty[a]), 0));
         }
+        if (lane == 0) bulk_wait_all();   // this warp's bulk stores are complete before the CTA exits
     }
     tc_fence_before();
     __syncthreads();
