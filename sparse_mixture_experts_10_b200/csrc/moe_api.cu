@@ -57,6 +57,7 @@ struct Plan {
     int64_t rows_cap;
     bool tc_router;    // bf16, N <= 256: router, top-k, statistics and scan in one tensor-core kernel
     bool few_router;   // bf16, T <= 64, N <= 32: one block per token instead
+    bool simt_router;  // bf16, N <= 32, more tokens: SIMT router with W_g in shared memory
     int chunk_tokens;  // tokens per dispatch chunk (32; the tensor-core router's 128-token tile; 1 token)
     int rnp, rkm;      // tensor-core router: padded expert count, top-k list length
     bool decode;  // few tokens: weight-streaming expert GEMMs
@@ -100,7 +101,11 @@ int make_plan(const moe_config *c, int64_t T, Plan *p) {
     p->nt = T <= 16 ? 16 : T <= 32 ? 32 : 64;
     p->tc_router = c->dtype == MOE_BF16 && N <= 256;
     p->few_router = p->tc_router && T <= kDecodeMaxT && N <= 32;
-    p->chunk_tokens = p->few_router ? 1 : p->tc_router ? rtc::BM : kChunk;
+    const size_t simt_bytes = p->np == 8    ? rtc::SimtShape<8>::smem_bytes((int)D)
+                              : p->np == 16 ? rtc::SimtShape<16>::smem_bytes((int)D)
+                                            : rtc::SimtShape<32>::smem_bytes((int)D);
+    p->simt_router = p->tc_router && !p->few_router && N <= 32 && simt_bytes <= kSmallRouterSmemMax;
+    p->chunk_tokens = p->few_router ? 1 : p->simt_router ? rtc::kSimtChunk : p->tc_router ? rtc::BM : kChunk;
     p->rnp = N <= 16 ? 16 : N <= 32 ? 32 : N <= 64 ? 64 : N <= 128 ? 128 : 256;
     p->rkm = K <= 8 ? 8 : 32;
     p->n_chunks = (int)cdiv(T, p->chunk_tokens);
@@ -134,7 +139,7 @@ int make_plan(const moe_config *c, int64_t T, Plan *p) {
     p->x_perm = take((size_t)p->rows_cap * D * es);
     p->h = take((size_t)p->rows_cap * H * es);
     p->z = take((size_t)T * K * D * 4);
-    p->wgt = take((N <= 32 && !(p->tc_router && !p->few_router)) ? 0 : (size_t)N * D * es);
+    p->wgt = take((N <= 32 && !(p->tc_router && !p->few_router && !p->simt_router)) ? 0 : (size_t)N * D * es);
     p->aux_p = take((size_t)p->aux_blocks * N * 4);
     p->aux_i = take((size_t)p->aux_blocks * N * 4);
     p->aux_c = take((size_t)p->aux_blocks * N * 4);
@@ -191,6 +196,9 @@ int device_info(DeviceInfo **out) {
         MOE_TRY(allow_smem(router_small_kernel<__nv_bfloat16, 16>));
         MOE_TRY(allow_smem(router_small_kernel<__nv_bfloat16, 32>));
         MOE_TRY(allow_smem(aux_partial_kernel));
+        MOE_TRY(allow_smem(rtc::router_simt_kernel<8>));
+        MOE_TRY(allow_smem(rtc::router_simt_kernel<16>));
+        MOE_TRY(allow_smem(rtc::router_simt_kernel<32>));
 #define MOE_RTC_ATTR(NP)                                                                                     \
     MOE_TRY(allow_smem(rtc::router_tc_kernel<NP, 8>)); \
     MOE_TRY(allow_smem(rtc::router_tc_kernel<NP, 32>))
@@ -351,6 +359,17 @@ int stage_route_tc(const Plan &P, const Bufs &b, const void *x, const moe_weight
         const int rows = (int)cdiv(D, S);
         rtc::router_few_kernel<<<dim3((unsigned)T, (unsigned)S), 256, 0, s>>>(
             xb, wg, p, b.at<float>(P.route_part), b.at<unsigned>(P.counters) + 64, rows);
+        return check_launch();
+    }
+    if (P.simt_router) {
+        const __nv_bfloat16 *xb = static_cast<const __nv_bfloat16 *>(x);
+        const __nv_bfloat16 *wg = static_cast<const __nv_bfloat16 *>(w->W_g);
+        const unsigned grid = (unsigned)P.n_chunks;
+#define MOE_SIMT(NP) rtc::router_simt_kernel<NP><<<grid, 256, rtc::SimtShape<NP>::smem_bytes(D), s>>>(xb, wg, p)
+        if (P.np == 8) MOE_SIMT(8);
+        else if (P.np == 16) MOE_SIMT(16);
+        else MOE_SIMT(32);
+#undef MOE_SIMT
         return check_launch();
     }
     __nv_bfloat16 *wgt = b.at<__nv_bfloat16>(P.wgt);

@@ -118,9 +118,16 @@ __device__ void finalize_tables(const Params &p, int ntiles, FinalScratch &f) {
                 f.pm[e] = p.T > 0 ? tp / (float)p.T : 0.f;
                 f.im[e] = (float)((double)ti / kImpScale);
             }
-            for (int c = c0; c < c1; ++c) {
-                p.chunk_base[(int64_t)c * N + e] = base;
-                base += __ldcg(p.tile_counts + (int64_t)c * N + e);
+            // eight tiles' counts loaded together, then the running base written
+            for (int cb = c0; cb < c1; cb += 8) {
+                int v[8];
+#pragma unroll
+                for (int k = 0; k < 8; ++k) v[k] = cb + k < c1 ? __ldcg(p.tile_counts + (int64_t)(cb + k) * N + e) : 0;
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    if (cb + k < c1) p.chunk_base[(int64_t)(cb + k) * N + e] = base;
+                    base += v[k];
+                }
             }
         }
         __syncthreads();
@@ -471,6 +478,207 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem_base, S::kTmemCols);
+    }
+    if (last_block(p.ticket, s_flag)) finalize_tables(p, gridDim.x, *fs);
+}
+
+// ---------------------------------------------------------------------------
+// N <= 32 experts (bf16): SIMT router.  One block of 256 threads per chunk of
+// kSimtChunk tokens.  W_g is staged transposed ([NP][D], rows N..NP-1 zero) in
+// shared memory; each warp takes 32/NP tokens at a time, one segment of NP
+// lanes per token, each lane a strided set of 16-byte slices of its token's x
+// row (four in flight) against all NP experts; a reduce-scatter inside the
+// segment leaves lane l with the score of (token l/NP, expert l%NP).
+// Per token: logits, the top k (ties to the lower index), renormalised gate
+// weights and the full-softmax probabilities.  Each lane accumulates, for its
+// expert and in token order, probabilities, counts and 2^-32 fixed-point gate
+// weights; lanes of the same expert, then warps, are added in fixed order into
+// the chunk's partials, and the last block builds the tables.
+// ---------------------------------------------------------------------------
+constexpr int kSimtChunk = 32;
+
+// Reduce-scatter over a segment of NP lanes (aligned at a multiple of NP):
+// afterwards lane seg_lane holds, in a[0], the segment's sum of entry seg_lane.
+template <int NP>
+__device__ __forceinline__ void reduce_scatter_seg(float (&a)[NP], int seg_lane) {
+#pragma unroll
+    for (int C = NP; C >= 2; C /= 2) {
+        const int H = C / 2;
+        const bool upper = (seg_lane & H) != 0;
+#pragma unroll
+        for (int i = 0; i < H; ++i) {
+            const float send = upper ? a[i] : a[i + H];
+            const float keep = upper ? a[i + H] : a[i];
+            a[i] = keep + __shfl_xor_sync(0xffffffffu, send, H);
+        }
+    }
+}
+
+// Shared memory of the SIMT router: W_g transposed ([NP][D] bf16), per-warp
+// partials, finalisation scratch.
+template <int NP>
+struct SimtShape {
+    __host__ __device__ static constexpr size_t w_bytes(int D) { return ((size_t)NP * D * 2 + 15) / 16 * 16; }
+    static size_t smem_bytes(int D) { return w_bytes(D) + 256 * (4 + 4 + 8) + sizeof(FinalScratch) + 16; }
+};
+
+template <int NP>
+__global__ void __launch_bounds__(256, NP == 8 ? 2 : 1) router_simt_kernel(const __nv_bfloat16 *__restrict__ x,
+                                                                          const __nv_bfloat16 *__restrict__ Wg,
+                                                                          const Params p) {
+    constexpr int TPW = 32 / NP;
+    constexpr int kSimtU = 8;   // 16-byte slices of x in flight per lane
+    using WT = __nv_bfloat16;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    const int D = p.D, N = p.N, K = p.K, T = p.T;
+    WT *WgT = reinterpret_cast<WT *>(smem_raw);
+    float *s_p = reinterpret_cast<float *>(smem_raw + SimtShape<NP>::w_bytes(D));   // [8][32]
+    int *s_c = reinterpret_cast<int *>(s_p + 256);                                        // [8][32]
+    unsigned long long *s_i = reinterpret_cast<unsigned long long *>(s_c + 256);          // [8][32]
+    FinalScratch *fs = reinterpret_cast<FinalScratch *>(s_i + 256);
+    int *s_flag = reinterpret_cast<int *>(fs + 1);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+    // W_g [D][N] -> WgT [NP][D]: 16-byte reads of the flat matrix, eight in
+    // flight per thread, (d, e) advanced per element
+    for (int i = tid; i < (NP - N) * D; i += blockDim.x) WgT[(size_t)N * D + i] = WT(0.f);
+    const int total = D * N;
+    if ((reinterpret_cast<uintptr_t>(Wg) & 15) == 0) {
+        for (int i_base = tid * 8; i_base < total; i_base += blockDim.x * 8 * 8) {
+            uint4 v[8];
+#pragma unroll
+            for (int r = 0; r < 8; ++r) {
+                const int i0 = i_base + r * blockDim.x * 8;
+                if (i0 + 8 <= total) {
+                    v[r] = __ldg(reinterpret_cast<const uint4 *>(Wg + i0));
+                } else {
+                    __nv_bfloat16 t8[8];
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) t8[k] = i0 + k < total ? Wg[i0 + k] : __float2bfloat16(0.f);
+                    v[r] = *reinterpret_cast<const uint4 *>(t8);
+                }
+            }
+#pragma unroll
+            for (int r = 0; r < 8; ++r) {
+                const int i0 = i_base + r * blockDim.x * 8;
+                if (i0 >= total) break;
+                const __nv_bfloat16 *t8 = reinterpret_cast<const __nv_bfloat16 *>(&v[r]);
+                int d = i0 / N, e = i0 - d * N;
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    if (i0 + k < total) WgT[(size_t)e * D + d] = WT(t8[k]);
+                    if (++e == N) { e = 0; ++d; }
+                }
+            }
+        }
+    } else {
+        for (int i = tid; i < total; i += blockDim.x) {
+            const int d = i / N, e = i - d * N;
+            WgT[(size_t)e * D + d] = WT(Wg[i]);
+        }
+    }
+    __syncthreads();
+
+    const int t_begin = blockIdx.x * kSimtChunk;
+    const int nvec = D / 8;
+    const int seg_lane = lane % NP, seg_base = lane - seg_lane;
+    const int e = seg_lane;
+    const bool valid_e = e < N;
+    float acc_p = 0.f;
+    int acc_c = 0;
+    unsigned long long acc_i = 0ull;
+    for (int g = warp * TPW; g < kSimtChunk; g += 8 * TPW) {
+        const int t0 = t_begin + g;
+        const int t = t0 + lane / NP;
+        const uint4 *xrow = reinterpret_cast<const uint4 *>(x + (int64_t)t * D);
+        float a[NP];
+#pragma unroll
+        for (int i = 0; i < NP; ++i) a[i] = 0.f;
+        for (int v0 = seg_lane; v0 < nvec; v0 += NP * kSimtU) {
+            uint4 xr[kSimtU];
+#pragma unroll
+            for (int u = 0; u < kSimtU; ++u) {
+                const int v = v0 + NP * u;
+                xr[u] = (t < T && v < nvec) ? __ldg(xrow + v) : make_uint4(0u, 0u, 0u, 0u);
+            }
+#pragma unroll
+            for (int u = 0; u < kSimtU; ++u) {
+                const int v = v0 + NP * u;
+                if (v >= nvec) break;
+                {
+                    float xf[8];
+                    Vec16<__nv_bfloat16>::unpack(xr[u], xf);
+#pragma unroll
+                    for (int ee = 0; ee < NP; ++ee) {
+                        float wf[8];
+                        Vec16<__nv_bfloat16>::load(reinterpret_cast<const __nv_bfloat16 *>(WgT) + (size_t)ee * D +
+                                                       (size_t)v * 8,
+                                                   wf);
+#pragma unroll
+                        for (int q = 0; q < 8; ++q) a[ee] = fmaf(xf[q], wf[q], a[ee]);
+                    }
+                }
+            }
+        }
+        reduce_scatter_seg<NP>(a, seg_lane);
+        const bool tok = t < T;
+        float s = a[0];
+        if (valid_e && p.bg) s += p.bg[e];
+        if (tok && valid_e) p.logits[(int64_t)t * N + e] = s;
+        if (s != s) {
+            if (valid_e && tok) set_status(kStatusNanLogit);
+            s = -INFINITY;
+        }
+        int slot_e;
+        float slot_w;
+        const bool has = segment_topk<NP>(s, e, !valid_e, K, seg_lane, lane, slot_e, slot_w);
+        if (has && tok) {
+            p.topk_idx[(int64_t)t * K + seg_lane] = slot_e;
+            p.topk_w[(int64_t)t * K + seg_lane] = slot_w;
+        }
+        // the token's full softmax (segment of NP lanes); its counts and gate weights per expert
+        float mx = valid_e ? s : -INFINITY;
+#pragma unroll
+        for (int o = NP / 2; o >= 1; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        const float ex = valid_e ? expf(s - mx) : 0.f;
+        float z = ex;
+#pragma unroll
+        for (int o = NP / 2; o >= 1; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+        if (tok && valid_e) acc_p += ex / z;
+        for (int j = 0; j < K; ++j) {
+            const int ej = __shfl_sync(0xffffffffu, slot_e, seg_base + j);
+            const float wj = __shfl_sync(0xffffffffu, slot_w, seg_base + j);
+            if (tok && valid_e && ej == e) {
+                ++acc_c;
+                acc_i += __double2ull_rn((double)wj * kImpScale);
+            }
+        }
+    }
+    // lanes e, e+NP, ... hold the same expert: fixed xor tree, then warps in order
+#pragma unroll
+    for (int o = NP; o < 32; o <<= 1) {
+        acc_p += __shfl_xor_sync(0xffffffffu, acc_p, o);
+        acc_c += __shfl_xor_sync(0xffffffffu, acc_c, o);
+        acc_i += __shfl_xor_sync(0xffffffffu, acc_i, o);
+    }
+    if (lane < NP) {
+        s_p[warp * 32 + lane] = acc_p;
+        s_c[warp * 32 + lane] = acc_c;
+        s_i[warp * 32 + lane] = acc_i;
+    }
+    __syncthreads();
+    if (tid < N) {
+        float ps = 0.f;
+        int cs = 0;
+        unsigned long long is = 0ull;
+        for (int w = 0; w < 8; ++w) {
+            ps += s_p[w * 32 + tid];
+            cs += s_c[w * 32 + tid];
+            is += s_i[w * 32 + tid];
+        }
+        p.tile_p[(int64_t)blockIdx.x * N + tid] = ps;
+        p.tile_counts[(int64_t)blockIdx.x * N + tid] = cs;
+        p.tile_imp[(int64_t)blockIdx.x * N + tid] = is;
     }
     if (last_block(p.ticket, s_flag)) finalize_tables(p, gridDim.x, *fs);
 }
