@@ -67,9 +67,11 @@ struct Plan {
     // Counters region (zeroed on every call), 32-bit words: [0] router ticket,
     // [1] statistics ticket, [2] number of live experts, [64, 128) per-token
     // tickets of the few-token router; from byte 512 the stream-K tile tickets
-    // of the decode up- and then down-projection (dec_cap each).
+    // of the decode up- and then down-projection (dec_cap each); then the
+    // routers' per-expert probability and gate-weight sums (u64, N each).
     size_t counters_bytes;
-    size_t counters, logits, idx, w, counts, offsets, row_offsets, live, chunk_counts, chunk_base, tile_p, tile_imp,
+    size_t stat_sums;  // offset inside the counters region of the routers' fixed-point sums [2][N] (u64)
+    size_t counters, logits, idx, w, counts, offsets, row_offsets, live, chunk_counts, chunk_base,
         perm_slot, slot_row, x_perm, h, z, wgt, aux_p, aux_i, aux_c, route_part, dec_part, total;
 };
 
@@ -120,7 +122,8 @@ int make_plan(const moe_config *c, int64_t T, Plan *p) {
     };
     p->route_splits = p->few_router ? (int)std::min<int64_t>(rtc::kFewMaxSplits, std::max<int64_t>(1, cdiv(D, 256))) : 1;
     p->dec_cap = p->decode ? kDecodeMaxGrid : 0;
-    p->counters_bytes = align256(512 + (size_t)2 * p->dec_cap * 4);
+    p->stat_sums = (512 + (size_t)2 * p->dec_cap * 4 + 7) / 8 * 8;
+    p->counters_bytes = align256(p->stat_sums + (size_t)2 * N * 8);
     p->counters = take(p->counters_bytes);
     p->logits = take((size_t)T * N * 4);
     p->idx = take((size_t)T * K * 4);
@@ -132,8 +135,6 @@ int make_plan(const moe_config *c, int64_t T, Plan *p) {
     const int64_t max_chunks = std::max<int64_t>(p->n_chunks, 1);
     p->chunk_counts = take((size_t)max_chunks * N * 4);
     p->chunk_base = take((size_t)max_chunks * N * 4);
-    p->tile_p = take(p->tc_router ? (size_t)max_chunks * N * 4 : 0);
-    p->tile_imp = take(p->tc_router ? (size_t)max_chunks * N * 8 : 0);
     p->perm_slot = take((size_t)p->rows_cap * 4);
     p->slot_row = take((size_t)T * K * 4);
     p->x_perm = take((size_t)p->rows_cap * D * es);
@@ -334,8 +335,8 @@ int stage_route_tc(const Plan &P, const Bufs &b, const void *x, const moe_weight
     p.topk_idx = idx;
     p.topk_w = tw;
     p.tile_counts = b.at<int>(P.chunk_counts);
-    p.tile_p = b.at<float>(P.tile_p);
-    p.tile_imp = b.at<unsigned long long>(P.tile_imp);
+    p.sum_p = reinterpret_cast<unsigned long long *>(b.ws + P.counters + P.stat_sums);
+    p.sum_imp = p.sum_p + N;
     p.ticket = b.at<unsigned>(P.counters);
     p.chunk_base = b.at<int>(P.chunk_base);
     p.counts = b.at<int>(P.counts);

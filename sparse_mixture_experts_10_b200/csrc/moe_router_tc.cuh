@@ -48,8 +48,8 @@ struct Params {
     int *topk_idx;                       // [T, K]
     float *topk_w;                       // [T, K]
     int *tile_counts;                    // [tiles, N]
-    float *tile_p;                       // [tiles, N]
-    unsigned long long *tile_imp;        // [tiles, N] fixed point
+    unsigned long long *sum_p;           // [N] full-softmax probability sums, 2^-32 fixed point (zero at launch)
+    unsigned long long *sum_imp;         // [N] gate-weight sums, 2^-32 fixed point (zero at launch)
     unsigned *ticket;                    // zero at launch
     // dispatch tables (written by the last block)
     int *chunk_base;                     // [tiles, N] first row (relative to the expert's segment) of the tile's tokens
@@ -67,22 +67,41 @@ struct Params {
 };
 
 // Scratch of the finalisation (shared memory, up to 256 experts, 256 threads).
-struct FinalScratch {
+// 16-byte aligned size: barriers and 8-byte words are placed right after it.
+struct __align__(16) FinalScratch {
     int cnt[256];
     float pm[256];
     float im[256];
     int row[257];
     int q_cnt[256];
-    float q_p[256];
-    unsigned long long q_i[256];
 };
 
-// Executed by every thread of the last block.  Per expert e, Q threads take
-// contiguous tile ranges; the range totals are combined in range order, so the
-// float sums have a fixed order; counts and fixed-point gate weights are exact.
-__device__ void finalize_tables(const Params &p, int ntiles, FinalScratch &f) {
+// Executed by every thread of the last block.  The blocks have added their
+// probability and gate-weight sums into sum_p / sum_imp (integer sums, exact
+// and order-independent) and written their per-expert token counts per tile.
+// The [tiles, N] count matrix is loaded into cnt_smem (cap ints of the
+// kernel's shared memory, no longer used by then) in one coalesced pass when
+// it fits; per expert e, Q threads then take contiguous tile ranges for the
+// totals and the exclusive scan that gives each tile's first row.
+__device__ void finalize_tables(const Params &p, int ntiles, FinalScratch &f, int *cnt_smem, int cap) {
     const int N = p.N, nt = blockDim.x, tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
+    const bool in_smem = cnt_smem != nullptr && (int64_t)ntiles * N <= cap;
+    if (in_smem) {
+        const int total = ntiles * N;
+        for (int i0 = tid; i0 < total; i0 += 8 * nt) {
+            int v[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) v[k] = i0 + k * nt < total ? __ldcg(p.tile_counts + i0 + k * nt) : 0;
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+                if (i0 + k * nt < total) cnt_smem[i0 + k * nt] = v[k];
+        }
+        __syncthreads();
+    }
+    auto count_at = [&](int c, int e) -> int {
+        return in_smem ? cnt_smem[c * N + e] : __ldcg(p.tile_counts + (int64_t)c * N + e);
+    };
     int Q = nt / N;
     Q = Q < 1 ? 1 : (Q > 32 ? 32 : Q);
     const int epp = nt / Q;                       // experts per pass
@@ -92,37 +111,27 @@ __device__ void finalize_tables(const Params &p, int ntiles, FinalScratch &f) {
         const bool act = tid < epp * Q && e < N;
         const int c0 = q * R, c1 = min(ntiles, c0 + R);
         int cnt = 0;
-        float ps = 0.f;
-        unsigned long long im = 0;
         if (act) {
 #pragma unroll 8
-            for (int c = c0; c < c1; ++c) {
-                cnt += __ldcg(p.tile_counts + (int64_t)c * N + e);
-                ps += __ldcg(p.tile_p + (int64_t)c * N + e);
-                im += __ldcg(p.tile_imp + (int64_t)c * N + e);
-            }
+            for (int c = c0; c < c1; ++c) cnt += count_at(c, e);
         }
         f.q_cnt[tid] = cnt;
-        f.q_p[tid] = ps;
-        f.q_i[tid] = im;
         __syncthreads();
         int base = 0;
         if (act) {
             for (int j = 0; j < q; ++j) base += f.q_cnt[tid - q + j];   // tiles before this range
             if (q == 0) {
                 int tc = 0;
-                float tp = 0.f;
-                unsigned long long ti = 0;
-                for (int j = 0; j < Q; ++j) { tc += f.q_cnt[tid + j]; tp += f.q_p[tid + j]; ti += f.q_i[tid + j]; }
+                for (int j = 0; j < Q; ++j) tc += f.q_cnt[tid + j];
                 f.cnt[e] = tc;
-                f.pm[e] = p.T > 0 ? tp / (float)p.T : 0.f;
-                f.im[e] = (float)((double)ti / kImpScale);
+                f.pm[e] = p.T > 0 ? (float)((double)__ldcg(p.sum_p + e) / kImpScale / (double)p.T) : 0.f;
+                f.im[e] = (float)((double)__ldcg(p.sum_imp + e) / kImpScale);
             }
-            // eight tiles' counts loaded together, then the running base written
+            // eight tiles' counts read together, then the running base written
             for (int cb = c0; cb < c1; cb += 8) {
                 int v[8];
 #pragma unroll
-                for (int k = 0; k < 8; ++k) v[k] = cb + k < c1 ? __ldcg(p.tile_counts + (int64_t)(cb + k) * N + e) : 0;
+                for (int k = 0; k < 8; ++k) v[k] = cb + k < c1 ? count_at(cb + k, e) : 0;
 #pragma unroll
                 for (int k = 0; k < 8; ++k) {
                     if (cb + k < c1) p.chunk_base[(int64_t)(cb + k) * N + e] = base;
@@ -471,15 +480,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int e = threadIdx.x; e < p.N; e += blockDim.x) {
         float ps = 0.f;
         for (int w = 0; w < 4; ++w) ps += s_wp[w * 256 + e];
-        p.tile_p[(int64_t)tile * p.N + e] = ps;
-        p.tile_imp[(int64_t)tile * p.N + e] = s_imp[e];
+        atomicAdd(p.sum_p + e, __double2ull_rn((double)ps * kImpScale));
+        atomicAdd(p.sum_imp + e, s_imp[e]);
         p.tile_counts[(int64_t)tile * p.N + e] = s_cnt[e];
     }
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem_base, S::kTmemCols);
     }
-    if (last_block(p.ticket, s_flag)) finalize_tables(p, gridDim.x, *fs);
+    if (last_block(p.ticket, s_flag))
+        finalize_tables(p, gridDim.x, *fs, reinterpret_cast<int *>(smem),
+                        (int)(kStages * (S::kABytes + S::kBBytes) / 4));
 }
 
 // ---------------------------------------------------------------------------
@@ -676,11 +687,13 @@ __global__ void __launch_bounds__(256, NP == 8 ? 2 : 1) router_simt_kernel(const
             cs += s_c[w * 32 + tid];
             is += s_i[w * 32 + tid];
         }
-        p.tile_p[(int64_t)blockIdx.x * N + tid] = ps;
         p.tile_counts[(int64_t)blockIdx.x * N + tid] = cs;
-        p.tile_imp[(int64_t)blockIdx.x * N + tid] = is;
+        atomicAdd(p.sum_p + tid, __double2ull_rn((double)ps * kImpScale));
+        atomicAdd(p.sum_imp + tid, is);
     }
-    if (last_block(p.ticket, s_flag)) finalize_tables(p, gridDim.x, *fs);
+    if (last_block(p.ticket, s_flag))
+        finalize_tables(p, gridDim.x, *fs, reinterpret_cast<int *>(smem_raw),
+                        (int)(SimtShape<NP>::w_bytes(D) / 4));
 }
 
 // ---------------------------------------------------------------------------
@@ -696,6 +709,7 @@ __global__ void __launch_bounds__(256, NP == 8 ? 2 : 1) router_simt_kernel(const
 // ---------------------------------------------------------------------------
 constexpr int kFewUnroll = 16;
 constexpr int kFewMaxSplits = 16;
+constexpr int kFewMaxT = 64;   // tokens (tiles) the few-token router handles
 
 __global__ void __launch_bounds__(256) router_few_kernel(const __nv_bfloat16 *__restrict__ x,
                                                           const __nv_bfloat16 *__restrict__ Wg, const Params p,
@@ -703,6 +717,7 @@ __global__ void __launch_bounds__(256) router_few_kernel(const __nv_bfloat16 *__
                                                           unsigned *__restrict__ token_ticket, int rows) {
     __shared__ float part[8][32];
     __shared__ FinalScratch fs;
+    __shared__ int s_cnt[kFewMaxT * 32];   // the count matrix in the finalisation
     __shared__ int s_flag;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int t = blockIdx.x, sl = blockIdx.y, S = gridDim.y, N = p.N, D = p.D;
@@ -769,12 +784,12 @@ __global__ void __launch_bounds__(256) router_few_kernel(const __nv_bfloat16 *__
             }
         }
         if (live) {
-            p.tile_p[(int64_t)t * N + lane] = ex / z;
             p.tile_counts[(int64_t)t * N + lane] = cnt;
-            p.tile_imp[(int64_t)t * N + lane] = im;
+            atomicAdd(p.sum_p + lane, __double2ull_rn((double)(ex / z) * kImpScale));
+            if (im) atomicAdd(p.sum_imp + lane, im);
         }
     }
-    if (last_block(p.ticket, &s_flag)) finalize_tables(p, gridDim.x, fs);
+    if (last_block(p.ticket, &s_flag)) finalize_tables(p, gridDim.x, fs, s_cnt, kFewMaxT * 32);
 }
 
 }  // namespace rtc
