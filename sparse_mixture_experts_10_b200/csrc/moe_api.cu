@@ -37,6 +37,7 @@ constexpr int kDecodeMaxGrid = 256;    // decode GEMMs: most persistent CTAs (st
 
 struct DeviceInfo {
     int sms = 0;
+    int pair_clusters = 0;   // 2-CTA clusters of the pair GEMM that can be resident at once
     bool attrs = false;
 };
 DeviceInfo g_dev[kMaxDevices];
@@ -217,6 +218,18 @@ int device_info(DeviceInfo **out) {
         MOE_DEC_ATTR(32);
         MOE_DEC_ATTR(64);
 #undef MOE_DEC_ATTR
+        // Clusters need both CTAs in one GPC, so fewer than sms / 2 pairs may fit
+        // at once; the persistent pair GEMM is launched with no more than fit
+        // (at the largest shared-memory size it uses).
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)(2 * (d.sms / 2)));
+        cfg.blockDim = dim3(tc::kThreads);
+        cfg.dynamicSmemBytes = tc::Shape2::smem_bytes(1024);
+        int n = 0;
+        if (cudaOccupancyMaxActiveClusters(&n, (const void *)tc::grouped_gemm_tc2_kernel<tc::EPI_GELU>, &cfg) !=
+            cudaSuccess)
+            return MOE_ERR_CUDA;
+        d.pair_clusters = n > 0 ? std::min(n, d.sms / 2) : d.sms / 2;
         d.attrs = true;
     }
     *out = &d;
@@ -290,8 +303,8 @@ int launch_tc(const CUtensorMap &A, const CUtensorMap &B, const CUtensorMap &O, 
 // Pair (2-CTA cluster) version for 256-column tiles: 256-row units per cluster.
 template <int EPI>
 int launch_tc2(const CUtensorMap &A, const CUtensorMap &B, const CUtensorMap &O, const tc::Params &p,
-               int64_t units_upper, int sms, cudaStream_t s) {
-    const int64_t clusters = std::min<int64_t>(std::max<int64_t>(units_upper, 1), sms / 2);
+               int64_t units_upper, int pair_clusters, cudaStream_t s) {
+    const int64_t clusters = std::min<int64_t>(std::max<int64_t>(units_upper, 1), pair_clusters);
     const size_t smem = tc::Shape2::smem_bytes(p.num_groups);
     tc::grouped_gemm_tc2_kernel<EPI><<<(unsigned)(2 * clusters), tc::kThreads, smem, s>>>(A, B, O, p);
     return check_launch();
@@ -448,7 +461,7 @@ int stage_route(const Plan &P, const Bufs &b, const void *x, const moe_weights *
         p.ldo = N;
         p.bias = w->b_g;
         p.timeout_ns = kTimeoutNs;
-        MOE_TRY((launch_tc2<tc::EPI_LOGITS>(ma, mb, ma, p, cdiv(T, 2 * tc::BM) * p.n_tiles, dev.sms, s)));
+        MOE_TRY((launch_tc2<tc::EPI_LOGITS>(ma, mb, ma, p, cdiv(T, 2 * tc::BM) * p.n_tiles, dev.pair_clusters, s)));
     } else {
         float *wgt = b.at<float>(P.wgt);
         transpose_kernel<float><<<dim3((unsigned)cdiv(N, 32), (unsigned)cdiv(D, 32)), dim3(32, 8), 0, s>>>(
@@ -623,8 +636,8 @@ int stage_up(const Plan &P, const Bufs &b, const moe_weights *w, const DeviceInf
             return launch_tc<128, tc::EPI_GELU>(ma, mb, mo, p, upper, dev.sms, s);
         }
         const int64_t units = (P.rows_cap / (2 * tc::BM) + N) * p.n_tiles;
-        if (swiglu) return launch_tc2<tc::EPI_SWIGLU>(ma, mb, mo, p, units, dev.sms, s);
-        return launch_tc2<tc::EPI_GELU>(ma, mb, mo, p, units, dev.sms, s);
+        if (swiglu) return launch_tc2<tc::EPI_SWIGLU>(ma, mb, mo, p, units, dev.pair_clusters, s);
+        return launch_tc2<tc::EPI_GELU>(ma, mb, mo, p, units, dev.pair_clusters, s);
     }
     simt::Params p{};
     p.A = b.at<float>(P.x_perm);
@@ -668,7 +681,8 @@ int stage_down(const Plan &P, const Bufs &b, const moe_weights *w, const DeviceI
         p.timeout_ns = kTimeoutNs;
         const int64_t upper = (P.rows_cap / tc::BM) * p.n_tiles;
         if (bn == 128) return launch_tc<128, tc::EPI_SCATTER>(ma, mb, ma, p, upper, dev.sms, s);
-        return launch_tc2<tc::EPI_SCATTER>(ma, mb, ma, p, (P.rows_cap / (2 * tc::BM) + N) * p.n_tiles, dev.sms, s);
+        return launch_tc2<tc::EPI_SCATTER>(ma, mb, ma, p, (P.rows_cap / (2 * tc::BM) + N) * p.n_tiles,
+                                           dev.pair_clusters, s);
     }
     simt::Params p{};
     p.A = b.at<float>(P.h);
