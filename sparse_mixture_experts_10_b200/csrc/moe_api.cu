@@ -657,7 +657,15 @@ int stage_up(const Plan &P, const Bufs &b, const moe_weights *w, const DeviceInf
     return launch_simt<simt::EPI_GELU>(p, P.rows_cap, (int)cdiv(H, simt::TN), s);
 }
 
-int stage_down(const Plan &P, const Bufs &b, const moe_weights *w, const DeviceInfo &dev, cudaStream_t s) {
+// The combine folds into the down projection (fp32 reductions into y) for bf16
+// prefill layers with K <= 2 and an fp32 y: at most two additions per element
+// onto +0, so the result is the same in any order.
+bool combine_in_down(const Plan &P, int y_dtype) {
+    return P.dtype == MOE_BF16 && !P.decode && P.K <= 2 && y_dtype == MOE_F32;
+}
+
+int stage_down(const Plan &P, const Bufs &b, const moe_weights *w, void *y, int y_dtype, const DeviceInfo &dev,
+               cudaStream_t s) {
     if (P.decode) return stage_down_decode(P, b, w, dev, s);
     const int D = P.D, H = P.H, N = P.N;
     const float *bias = P.act == MOE_ACT_SWIGLU ? nullptr : w->b2;
@@ -679,6 +687,11 @@ int stage_down(const Plan &P, const Bufs &b, const moe_weights *w, const DeviceI
         p.perm_slot = b.at<int>(P.perm_slot);
         p.gate_w = b.at<float>(P.w);
         p.timeout_ns = kTimeoutNs;
+        if (combine_in_down(P, y_dtype)) {
+            if (cudaMemsetAsync(y, 0, (size_t)P.T * D * 4, s) != cudaSuccess) return MOE_ERR_CUDA;
+            p.out = y;
+            p.accum_k = P.K;
+        }
         const int64_t upper = (P.rows_cap / tc::BM) * p.n_tiles;
         if (bn == 128) return launch_tc<128, tc::EPI_SCATTER>(ma, mb, ma, p, upper, dev.sms, s);
         return launch_tc2<tc::EPI_SCATTER>(ma, mb, ma, p, (P.rows_cap / (2 * tc::BM) + N) * p.n_tiles,
@@ -804,9 +817,9 @@ int forward_impl(const moe_config *cfg, const void *x, int64_t T, const moe_weig
     MOE_TRY(rec(3));
     MOE_TRY(stage_up(P, b, w, *dev, s));
     MOE_TRY(rec(4));
-    MOE_TRY(stage_down(P, b, w, *dev, s));
+    MOE_TRY(stage_down(P, b, w, y, y_dtype, *dev, s));
     MOE_TRY(rec(5));
-    MOE_TRY(stage_combine(P, b, y, y_dtype, *dev, s));
+    if (!combine_in_down(P, y_dtype)) MOE_TRY(stage_combine(P, b, y, y_dtype, *dev, s));
     MOE_TRY(rec(6));
     if (aux && !P.tc_router) MOE_TRY(stage_aux(P, b, logits, idx, tw, aux, s));
     MOE_TRY(rec(7));

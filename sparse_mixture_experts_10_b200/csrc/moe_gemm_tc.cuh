@@ -78,8 +78,17 @@ struct Params {
     const float *bias;        // [G, n_valid] or nullptr
     const int *perm_slot;     // EPI_SCATTER: slot of each permuted row (-1 = padding)
     const float *gate_w;      // EPI_SCATTER: gate weight of each slot
+    // EPI_SCATTER with accum_k > 0: out is y [T, ldo] fp32 (zeroed before the
+    // launch) and each row's scaled result is added into row slot / accum_k with
+    // fp32 reductions; with accum_k <= 2 every element receives at most two
+    // additions onto +0, whose result does not depend on their order.
+    int accum_k;
     uint64_t timeout_ns;
 };
+
+__device__ __forceinline__ void red_add_v4(float *ptr, float a, float b, float c, float d) {
+    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(ptr), "f"(a), "f"(b), "f"(c), "f"(d) : "memory");
+}
 
 // bf16 output staging for the bulk tensor stores: 32 rows x 16 columns per
 // epilogue warp.
@@ -355,16 +364,30 @@ __device__ __forceinline__ void epilogue_tile(const Params &p, const TileCoord &
                 for (int k = 0; k < 8; ++k) pk[k] = gelu_erf_bf16x2(v[2 * k], v[2 * k + 1]);
                 store_h_chunk(tmO, stage, static_cast<__nv_bfloat16 *>(p.out), p.ldo, row, row_ok, pk, n0, p.n_valid);
             } else if (EPI == EPI_SCATTER) {
-                float *dst = static_cast<float *>(p.out) + (int64_t)slot * p.ldo + n0;
-                if (full_chunk) {
+                if (p.accum_k > 0) {
+                    float *dst = static_cast<float *>(p.out) + (int64_t)(slot / p.accum_k) * p.ldo + n0;
+                    if (full_chunk) {
 #pragma unroll
-                    for (int u = 0; u < 4; ++u)
-                        reinterpret_cast<float4 *>(dst)[u] =
-                            make_float4(gw * v[4 * u], gw * v[4 * u + 1], gw * v[4 * u + 2], gw * v[4 * u + 3]);
+                        for (int u = 0; u < 4; ++u)
+                            red_add_v4(dst + 4 * u, gw * v[4 * u], gw * v[4 * u + 1], gw * v[4 * u + 2],
+                                       gw * v[4 * u + 3]);
+                    } else {
+#pragma unroll
+                        for (int k = 0; k < 16; ++k)
+                            if (n0 + k < p.n_valid) atomicAdd(dst + k, gw * v[k]);
+                    }
                 } else {
+                    float *dst = static_cast<float *>(p.out) + (int64_t)slot * p.ldo + n0;
+                    if (full_chunk) {
 #pragma unroll
-                    for (int k = 0; k < 16; ++k)
-                        if (n0 + k < p.n_valid) dst[k] = gw * v[k];
+                        for (int u = 0; u < 4; ++u)
+                            reinterpret_cast<float4 *>(dst)[u] =
+                                make_float4(gw * v[4 * u], gw * v[4 * u + 1], gw * v[4 * u + 2], gw * v[4 * u + 3]);
+                    } else {
+#pragma unroll
+                        for (int k = 0; k < 16; ++k)
+                            if (n0 + k < p.n_valid) dst[k] = gw * v[k];
+                    }
                 }
             } else {  // EPI_LOGITS
                 float *dst = static_cast<float *>(p.out) + (int64_t)row * p.ldo + n0;
