@@ -241,6 +241,36 @@ int check_launch() {
     return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
+// Launch with programmatic stream serialisation: the kernel may be launched
+// while the previous kernel of the stream is still running; it calls
+// pdl_enter() before its first global access, which waits for that kernel's
+// completion.  Captured into a CUDA graph this is a programmatic edge.
+template <typename... KArgs, typename... Args>
+int launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, Args &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+// Zeroes `bytes` (a multiple of 16) at the 16-byte aligned p.
+int launch_zero(void *p, size_t bytes, int sms, cudaStream_t s) {
+    const int64_t n16 = (int64_t)(bytes / 16);
+    if (n16 == 0) return MOE_OK;
+    const int grid = (int)std::min<int64_t>(cdiv(n16, 256), (int64_t)sms * 8);
+    return launch_pdl(zero_kernel, dim3(grid), dim3(256), 0, s, static_cast<uint4 *>(p), n16);
+}
+
 
 // --------------------------------------------------------------- TMA tensor maps
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
@@ -296,8 +326,7 @@ int launch_tc(const CUtensorMap &A, const CUtensorMap &B, const CUtensorMap &O, 
               int64_t tiles_upper, int sms, cudaStream_t s) {
     const int grid = (int)std::min<int64_t>(std::max<int64_t>(tiles_upper, 1), sms);
     const size_t smem = tc::Shape<BN>::smem_bytes(p.num_groups);
-    tc::grouped_gemm_tc_kernel<BN, EPI><<<grid, tc::kThreads, smem, s>>>(A, B, O, p);
-    return check_launch();
+    return launch_pdl(tc::grouped_gemm_tc_kernel<BN, EPI>, dim3(grid), dim3(tc::kThreads), smem, s, A, B, O, p);
 }
 
 // Pair (2-CTA cluster) version for 256-column tiles: 256-row units per cluster.
@@ -306,8 +335,8 @@ int launch_tc2(const CUtensorMap &A, const CUtensorMap &B, const CUtensorMap &O,
                int64_t units_upper, int pair_clusters, cudaStream_t s) {
     const int64_t clusters = std::min<int64_t>(std::max<int64_t>(units_upper, 1), pair_clusters);
     const size_t smem = tc::Shape2::smem_bytes(p.num_groups);
-    tc::grouped_gemm_tc2_kernel<EPI><<<(unsigned)(2 * clusters), tc::kThreads, smem, s>>>(A, B, O, p);
-    return check_launch();
+    return launch_pdl(tc::grouped_gemm_tc2_kernel<EPI>, dim3((unsigned)(2 * clusters)), dim3(tc::kThreads), smem, s, A,
+                      B, O, p);
 }
 
 template <int EPI>
@@ -328,8 +357,8 @@ struct Bufs {
 // route: logits (always written to `logits`), top-k, chunk histograms.
 template <int NP, int KM>
 int launch_rtc(const CUtensorMap &mx, const CUtensorMap &mw, const rtc::Params &p, int grid, cudaStream_t s) {
-    rtc::router_tc_kernel<NP, KM><<<grid, rtc::kThreads, rtc::Shape<NP>::kSmem, s>>>(mx, mw, p);
-    return check_launch();
+    return launch_pdl(rtc::router_tc_kernel<NP, KM>, dim3(grid), dim3(rtc::kThreads), rtc::Shape<NP>::kSmem, s, mx, mw,
+                      p);
 }
 
 // Tensor-core router: scores, top-k, statistics partials and (in the last CTA)
@@ -371,25 +400,23 @@ int stage_route_tc(const Plan &P, const Bufs &b, const void *x, const moe_weight
         const __nv_bfloat16 *wg = static_cast<const __nv_bfloat16 *>(w->W_g);
         const int S = P.route_splits;
         const int rows = (int)cdiv(D, S);
-        rtc::router_few_kernel<<<dim3((unsigned)T, (unsigned)S), 256, 0, s>>>(
-            xb, wg, p, b.at<float>(P.route_part), b.at<unsigned>(P.counters) + 64, rows);
-        return check_launch();
+        return launch_pdl(rtc::router_few_kernel, dim3((unsigned)T, (unsigned)S), dim3(256), 0, s, xb, wg, p,
+                          b.at<float>(P.route_part), b.at<unsigned>(P.counters) + 64, rows);
     }
     if (P.simt_router) {
         const __nv_bfloat16 *xb = static_cast<const __nv_bfloat16 *>(x);
         const __nv_bfloat16 *wg = static_cast<const __nv_bfloat16 *>(w->W_g);
         const unsigned grid = (unsigned)P.n_chunks;
-#define MOE_SIMT(NP) rtc::router_simt_kernel<NP><<<grid, 256, rtc::SimtShape<NP>::smem_bytes(D), s>>>(xb, wg, p)
+#define MOE_SIMT(NP) \
+    return launch_pdl(rtc::router_simt_kernel<NP>, dim3(grid), dim3(256), rtc::SimtShape<NP>::smem_bytes(D), s, xb, wg, p)
         if (P.np == 8) MOE_SIMT(8);
-        else if (P.np == 16) MOE_SIMT(16);
-        else MOE_SIMT(32);
+        if (P.np == 16) MOE_SIMT(16);
+        MOE_SIMT(32);
 #undef MOE_SIMT
-        return check_launch();
     }
     __nv_bfloat16 *wgt = b.at<__nv_bfloat16>(P.wgt);
-    transpose_kernel<__nv_bfloat16><<<dim3((unsigned)cdiv(N, 32), (unsigned)cdiv(D, 32)), dim3(32, 8), 0, s>>>(
-        static_cast<const __nv_bfloat16 *>(w->W_g), D, N, wgt);
-    MOE_TRY(check_launch());
+    MOE_TRY(launch_pdl(transpose_kernel<__nv_bfloat16>, dim3((unsigned)cdiv(N, 32), (unsigned)cdiv(D, 32)), dim3(32, 8),
+                       0, s, static_cast<const __nv_bfloat16 *>(w->W_g), D, N, wgt));
     CUtensorMap mx, mw;
     MOE_TRY(make_map(&mx, x, T, D, rtc::BM));
     MOE_TRY(make_map(&mw, wgt, N, D, P.rnp));
@@ -510,16 +537,14 @@ int stage_permute(const Plan &P, const Bufs &b, const void *x, const DeviceInfo 
     const int split = (int)std::max<int64_t>(1, std::min<int64_t>(8, cdiv(2 * dev.sms, P.n_chunks)));
     const dim3 grid((unsigned)P.n_chunks, (unsigned)split);
     if (P.dtype == MOE_F32)
-        permute_kernel<float><<<grid, 256, smem, s>>>(static_cast<const float *>(x), (int)P.T, P.D, P.K, P.N,
-                                                     P.chunk_tokens, b.at<int>(P.idx), b.at<int>(P.chunk_base),
-                                                     b.at<int>(P.row_offsets), b.at<int>(P.perm_slot),
-                                                     b.at<int>(P.slot_row), b.at<float>(P.x_perm));
-    else
-        permute_kernel<__nv_bfloat16><<<grid, 256, smem, s>>>(
-            static_cast<const __nv_bfloat16 *>(x), (int)P.T, P.D, P.K, P.N, P.chunk_tokens, b.at<int>(P.idx),
-            b.at<int>(P.chunk_base), b.at<int>(P.row_offsets), b.at<int>(P.perm_slot), b.at<int>(P.slot_row),
-            b.at<__nv_bfloat16>(P.x_perm));
-    return check_launch();
+        return launch_pdl(permute_kernel<float>, grid, dim3(256), smem, s, static_cast<const float *>(x), (int)P.T, P.D,
+                          P.K, P.N, P.chunk_tokens, (const int *)b.at<int>(P.idx), (const int *)b.at<int>(P.chunk_base),
+                          (const int *)b.at<int>(P.row_offsets), b.at<int>(P.perm_slot), b.at<int>(P.slot_row),
+                          b.at<float>(P.x_perm));
+    return launch_pdl(permute_kernel<__nv_bfloat16>, grid, dim3(256), smem, s, static_cast<const __nv_bfloat16 *>(x),
+                      (int)P.T, P.D, P.K, P.N, P.chunk_tokens, (const int *)b.at<int>(P.idx),
+                      (const int *)b.at<int>(P.chunk_base), (const int *)b.at<int>(P.row_offsets),
+                      b.at<int>(P.perm_slot), b.at<int>(P.slot_row), b.at<__nv_bfloat16>(P.x_perm));
 }
 
 // Expert GEMMs for few tokens (decode path): weight rows are the MMA's M
@@ -531,8 +556,8 @@ int launch_dec(const CUtensorMap &W, const CUtensorMap &X, const dec::Params &p,
     // partial buffer is sized for); whole tiles need no more CTAs than tiles
     const int grid = p.split_cap > 0 ? std::min(sms, p.split_cap)
                                      : (int)std::min<int64_t>(std::max<int64_t>(items_upper, 1), sms);
-    dec::decode_gemm_kernel<NT, EPI><<<grid, dec::kThreads, dec::Shape<NT, EPI>::kSmem, s>>>(W, X, p);
-    return check_launch();
+    return launch_pdl(dec::decode_gemm_kernel<NT, EPI>, dim3(grid), dim3(dec::kThreads), dec::Shape<NT, EPI>::kSmem, s, W,
+                      X, p);
 }
 
 template <int EPI>
@@ -688,7 +713,7 @@ int stage_down(const Plan &P, const Bufs &b, const moe_weights *w, void *y, int 
         p.gate_w = b.at<float>(P.w);
         p.timeout_ns = kTimeoutNs;
         if (combine_in_down(P, y_dtype)) {
-            if (cudaMemsetAsync(y, 0, (size_t)P.T * D * 4, s) != cudaSuccess) return MOE_ERR_CUDA;
+            MOE_TRY(launch_zero(y, (size_t)P.T * D * 4, dev.sms, s));
             p.out = y;
             p.accum_k = P.K;
         }
@@ -719,11 +744,10 @@ int stage_combine(const Plan &P, const Bufs &b, void *y, int y_dtype, const Devi
     const int64_t nq = P.T * (P.D / 4);
     const int grid = (int)std::min<int64_t>(cdiv(nq, 256), (int64_t)dev.sms * 8);
     if (y_dtype == MOE_F32)
-        combine_kernel<float><<<grid, 256, 0, s>>>(b.at<float>(P.z), P.T, P.D, P.K, static_cast<float *>(y));
-    else
-        combine_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(b.at<float>(P.z), P.T, P.D, P.K,
-                                                           static_cast<__nv_bfloat16 *>(y));
-    return check_launch();
+        return launch_pdl(combine_kernel<float>, dim3(grid), dim3(256), 0, s, (const float *)b.at<float>(P.z), P.T, P.D,
+                          P.K, static_cast<float *>(y));
+    return launch_pdl(combine_kernel<__nv_bfloat16>, dim3(grid), dim3(256), 0, s, (const float *)b.at<float>(P.z), P.T,
+                      P.D, P.K, static_cast<__nv_bfloat16 *>(y));
 }
 
 int stage_aux(const Plan &P, const Bufs &b, const float *logits, const int *idx, const float *tw, moe_aux *aux,
@@ -749,7 +773,9 @@ int stage_aux(const Plan &P, const Bufs &b, const float *logits, const int *idx,
 }
 
 int zero_counters(const Plan &P, const Bufs &b, cudaStream_t s) {
-    return cudaMemsetAsync(b.ws + P.counters, 0, P.counters_bytes, s) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+    DeviceInfo *dev = nullptr;
+    MOE_TRY(device_info(&dev));
+    return launch_zero(b.ws + P.counters, P.counters_bytes, dev->sms, s);
 }
 
 int zero_aux(const Plan &P, moe_aux *aux, cudaStream_t s) {

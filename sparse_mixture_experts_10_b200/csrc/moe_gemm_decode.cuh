@@ -158,6 +158,7 @@ template <int NT, int EPI>
 __global__ void __launch_bounds__(kThreads, 1)
     decode_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
                        const Params p) {
+    pdl_enter();
     using S = Shape<NT, EPI>;
     constexpr int kStages = S::kStages;
     extern __shared__ __align__(1024) uint8_t smem_raw[];

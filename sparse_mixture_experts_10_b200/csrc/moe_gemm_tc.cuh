@@ -402,6 +402,7 @@ template <int BN, int EPI>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                            const __grid_constant__ CUtensorMap tmO, const Params p) {
+    pdl_enter();
     using S = Shape<BN>;
     constexpr int kStages = S::kStages;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -662,6 +663,7 @@ template <int EPI>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     grouped_gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                             const __grid_constant__ CUtensorMap tmO, const Params p) {
+    pdl_enter();
     using S = Shape2;
     constexpr int BN = 256;
     constexpr int kStages = S::kStages;

@@ -445,6 +445,7 @@ __global__ void __launch_bounds__(256) permute_kernel(const Tin *__restrict__ x,
                                                       const int *__restrict__ chunk_base,
                                                       const int *__restrict__ row_offsets, int *__restrict__ perm_slot,
                                                       int *__restrict__ slot_row, Tin *__restrict__ x_perm) {
+    pdl_enter();
     extern __shared__ int s_perm[];
     int *s_run = s_perm;            // [N]
     int *s_dest = s_perm + N;       // [chunk_tokens * K]
@@ -504,6 +505,14 @@ __global__ void __launch_bounds__(256) permute_kernel(const Tin *__restrict__ x,
     }
 }
 
+// Zero n16 16-byte words at p (a memset that takes part in programmatic
+// dependent launch).
+__global__ void __launch_bounds__(256) zero_kernel(uint4 *__restrict__ p, int64_t n16) {
+    pdl_enter();
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n16; i += (int64_t)gridDim.x * blockDim.x)
+        p[i] = make_uint4(0u, 0u, 0u, 0u);
+}
+
 // ---------------------------------------------------------------------------
 // Combine: y[t] = z[t, 0] + z[t, 1] + ... + z[t, K-1], left to right (slot
 // order), no atomics ("MoE(Mixture of Experts)", section (2), Forward, which
@@ -512,6 +521,7 @@ __global__ void __launch_bounds__(256) permute_kernel(const Tin *__restrict__ x,
 template <typename Tout>
 __global__ void __launch_bounds__(256) combine_kernel(const float *__restrict__ z, int64_t T, int D, int K,
                                                       Tout *__restrict__ y) {
+    pdl_enter();
     const int64_t nq = T * (D / 4);
     for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < nq; i += (int64_t)gridDim.x * blockDim.x) {
         const int64_t t = i / (D / 4);
@@ -753,6 +763,7 @@ __global__ void __launch_bounds__(256) aux_partial_kernel(const float *__restric
 // W_g [D, N] -> W_g^T [N, D] (the K-major operand layout of the router GEMM).
 template <typename Tin>
 __global__ void transpose_kernel(const Tin *__restrict__ src, int R, int C, Tin *__restrict__ dst) {
+    pdl_enter();
     __shared__ Tin tile[32][33];
     const int c0 = blockIdx.x * 32, r0 = blockIdx.y * 32;
     for (int i = threadIdx.y; i < 32; i += blockDim.y) {

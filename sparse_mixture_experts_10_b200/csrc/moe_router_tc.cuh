@@ -328,6 +328,7 @@ template <int NP, int KM>
 __global__ void __launch_bounds__(kThreads, 1)
     router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
                      const Params p) {
+    pdl_enter();
     using S = Shape<NP>;
     constexpr int kStages = S::kStages;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -537,6 +538,7 @@ template <int NP>
 __global__ void __launch_bounds__(256, NP == 8 ? 2 : 1) router_simt_kernel(const __nv_bfloat16 *__restrict__ x,
                                                                           const __nv_bfloat16 *__restrict__ Wg,
                                                                           const Params p) {
+    pdl_enter();
     constexpr int TPW = 32 / NP;
     constexpr int kSimtU = 8;   // 16-byte slices of x in flight per lane
     using WT = __nv_bfloat16;
@@ -715,6 +717,7 @@ __global__ void __launch_bounds__(256) router_few_kernel(const __nv_bfloat16 *__
                                                           const __nv_bfloat16 *__restrict__ Wg, const Params p,
                                                           float *__restrict__ slab_scores,   // [T][S][32]
                                                           unsigned *__restrict__ token_ticket, int rows) {
+    pdl_enter();
     __shared__ float part[8][32];
     __shared__ FinalScratch fs;
     __shared__ int s_cnt[kFewMaxT * 32];   // the count matrix in the finalisation
