@@ -48,7 +48,8 @@ GEMM_KERNEL_SRC = os.path.join(ROOT, "sparse_mixture_experts_10_b200", "csrc", "
 # (dram__bytes_read.sum + dram__bytes_write.sum); keyed by workload and stage,
 # valid only while the kernel source hash is unchanged (see profiles/).
 NCU_TRAFFIC = {
-    # "gpt2/up": {"bytes": ..., "src_sha256": "..."},
+    "gpt2/up": {"bytes": 110745856, "src_sha256": "d60a1633be6983872816c07aba378b5d5eec95e52cb4973be81ac710a7bfc60e"},
+    "gpt2/down": {"bytes": 183801856, "src_sha256": "d60a1633be6983872816c07aba378b5d5eec95e52cb4973be81ac710a7bfc60e"},
 }
 
 
