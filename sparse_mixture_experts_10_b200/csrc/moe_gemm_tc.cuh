@@ -286,9 +286,26 @@ __device__ __forceinline__ void store_h_chunk(const CUtensorMap *tmO, uint8_t *s
     }
 }
 
+// EPI_SCATTER: the row's slot and gate weight, loaded by the caller before it
+// waits for the accumulator (two dependent global loads off the critical path).
+struct RowGate {
+    int slot = -1;
+    float gw = 0.f;
+};
+template <int EPI>
+__device__ __forceinline__ RowGate load_row_gate(const Params &p, int row, int row_limit) {
+    RowGate r;
+    if (EPI == EPI_SCATTER && row < row_limit) {
+        r.slot = p.perm_slot[row];
+        if (r.slot >= 0) r.gw = p.gate_w[r.slot];
+    }
+    return r;
+}
+
 template <int BN, int EPI>
 __device__ __forceinline__ void epilogue_tile(const Params &p, const TileCoord &c, int row, int row_limit,
-                                              uint32_t tbase, int grp, const CUtensorMap *tmO, uint8_t *stage) {
+                                              uint32_t tbase, int grp, const CUtensorMap *tmO, uint8_t *stage,
+                                              const RowGate rg) {
     const bool row_ok = row < row_limit;
     if (EPI == EPI_SWIGLU) {
         constexpr int kOutCols = BN / 2;                  // h columns per tile
@@ -314,12 +331,8 @@ __device__ __forceinline__ void epilogue_tile(const Params &p, const TileCoord &
     }
     constexpr int kPerGroup = BN / kEpiGroups;
     constexpr int kChunks = kPerGroup / 16;
-    int slot = -1;
-    float gw = 0.f;
-    if (EPI == EPI_SCATTER && row_ok) {
-        slot = p.perm_slot[row];
-        if (slot >= 0) gw = p.gate_w[slot];
-    }
+    const int slot = rg.slot;
+    const float gw = rg.gw;
     const float *bias_row = p.bias ? p.bias + (int64_t)c.g * p.n_valid : nullptr;
     // Chunks of 16 columns, software-pipelined: tcgen05.wait::ld waits for all
     // of a thread's outstanding loads, so chunk i+1's TMEM load is issued right
@@ -540,13 +553,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int a = local & 1;
             const uint32_t aph = (local >> 1) & 1;
             const TileCoord c = decode_tile(i, rowoff, G, p.n_tiles, dense_mtiles);
+            const int row_limit = rowoff ? s_rowoff[c.g + 1] : p.dense_rows;
+            const RowGate rg = load_row_gate<EPI>(p, c.row0 + r_in_tile, row_limit);
             // warp-uniform decision: the TMEM loads below are warp-collective
             if (!__all_sync(0xffffffffu, mbar_wait(&tfull[a], aph, p.timeout_ns))) break;
             tc_fence_after();
-            const int row_limit = rowoff ? s_rowoff[c.g + 1] : p.dense_rows;
             epilogue_tile<BN, EPI>(p, c, c.row0 + r_in_tile, row_limit,
                                    tmem_base + (static_cast<uint32_t>(q * 32) << 16) + a * BN, grp, &tmO,
-                                   sOut + ew * kOutStageWarpBytes);
+                                   sOut + ew * kOutStageWarpBytes, rg);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&tempty[a]);
@@ -816,13 +830,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             const int a = local & 1;
             const uint32_t aph = (local >> 1) & 1;
             const TileCoord c = decode_unit_tile(i, rowoff, s_units, G, p.n_tiles, dense_units);
+            const int row_limit = rowoff ? s_rowoff[c.g + 1] : p.dense_rows;
+            const RowGate rg = load_row_gate<EPI>(p, c.row0 + (int)rank * BM + r_in_tile, row_limit);
             // warp-uniform decision: the TMEM loads below are warp-collective
             if (!__all_sync(0xffffffffu, mbar_wait(&tfull[a], aph, p.timeout_ns))) break;
             tc_fence_after();
-            const int row_limit = rowoff ? s_rowoff[c.g + 1] : p.dense_rows;
             epilogue_tile<BN, EPI>(p, c, c.row0 + (int)rank * BM + r_in_tile, row_limit,
                                    tmem_base + (static_cast<uint32_t>(q * 32) << 16) + a * BN, grp, &tmO,
-                                   sOut + ew * kOutStageWarpBytes);
+                                   sOut + ew * kOutStageWarpBytes, rg);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive_remote(mapa_shared(smem_u32(&tempty[a]), 0));
