@@ -140,7 +140,10 @@ int make_plan(const moe_config *c, int64_t T, Plan *p) {
     p->slot_row = take((size_t)T * K * 4);
     p->x_perm = take((size_t)p->rows_cap * D * es);
     p->h = take((size_t)p->rows_cap * H * es);
-    p->z = take((size_t)T * K * D * 4);
+    // z rows: slot order (T*K rows) for decode and fp32 layers; the permuted
+    // row order (rows_cap rows) for bf16 prefill layers, whose down projection
+    // writes it with bulk tensor stores
+    p->z = take((size_t)(p->dtype == MOE_BF16 && !p->decode ? p->rows_cap : T * K) * D * 4);
     p->wgt = take((N <= 32 && !(p->tc_router && !p->few_router && !p->simt_router)) ? 0 : (size_t)N * D * es);
     p->aux_p = take((size_t)p->aux_blocks * N * 4);
     p->aux_i = take((size_t)p->aux_blocks * N * 4);
@@ -314,6 +317,21 @@ int make_store_map(CUtensorMap *m, void *base, int64_t rows, int64_t cols) {
     const cuuint32_t box[2] = {16u, 32u};
     const cuuint32_t estr[2] = {1u, 1u};
     const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, estr,
+                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? MOE_OK : MOE_ERR_CUDA;
+}
+
+// 2-D fp32 matrix [rows, cols] row-major as the destination of the down
+// projection's bulk stores: boxes of 32 rows x 8 columns, no swizzle.
+int make_store_map_f32(CUtensorMap *m, void *base, int64_t rows, int64_t cols) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return MOE_ERR_CUDA;
+    const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)cols * 4};
+    const cuuint32_t box[2] = {8u, 32u};
+    const cuuint32_t estr[2] = {1u, 1u};
+    const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, base, dims, strides, box, estr,
                            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
                            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? MOE_OK : MOE_ERR_CUDA;
@@ -712,14 +730,18 @@ int stage_down(const Plan &P, const Bufs &b, const moe_weights *w, void *y, int 
         p.perm_slot = b.at<int>(P.perm_slot);
         p.gate_w = b.at<float>(P.w);
         p.timeout_ns = kTimeoutNs;
+        CUtensorMap mo = ma;   // unused unless z is written by rows
         if (combine_in_down(P, y_dtype)) {
             MOE_TRY(launch_zero(y, (size_t)P.T * D * 4, dev.sms, s));
             p.out = y;
             p.accum_k = P.K;
+        } else {
+            MOE_TRY(make_store_map_f32(&mo, b.ws + P.z, P.rows_cap, D));
+            p.scatter_rows = 1;
         }
         const int64_t upper = (P.rows_cap / tc::BM) * p.n_tiles;
-        if (bn == 128) return launch_tc<128, tc::EPI_SCATTER>(ma, mb, ma, p, upper, dev.sms, s);
-        return launch_tc2<tc::EPI_SCATTER>(ma, mb, ma, p, (P.rows_cap / (2 * tc::BM) + N) * p.n_tiles,
+        if (bn == 128) return launch_tc<128, tc::EPI_SCATTER>(ma, mb, mo, p, upper, dev.sms, s);
+        return launch_tc2<tc::EPI_SCATTER>(ma, mb, mo, p, (P.rows_cap / (2 * tc::BM) + N) * p.n_tiles,
                                            dev.pair_clusters, s);
     }
     simt::Params p{};
@@ -743,11 +765,13 @@ int stage_down(const Plan &P, const Bufs &b, const moe_weights *w, void *y, int 
 int stage_combine(const Plan &P, const Bufs &b, void *y, int y_dtype, const DeviceInfo &dev, cudaStream_t s) {
     const int64_t nq = P.T * (P.D / 4);
     const int grid = (int)std::min<int64_t>(cdiv(nq, 256), (int64_t)dev.sms * 8);
+    // bf16 prefill layers keep z in the permuted row order (see stage_down)
+    const int *slot_row = P.dtype == MOE_BF16 && !P.decode ? b.at<int>(P.slot_row) : nullptr;
     if (y_dtype == MOE_F32)
         return launch_pdl(combine_kernel<float>, dim3(grid), dim3(256), 0, s, (const float *)b.at<float>(P.z), P.T, P.D,
-                          P.K, static_cast<float *>(y));
+                          P.K, slot_row, static_cast<float *>(y));
     return launch_pdl(combine_kernel<__nv_bfloat16>, dim3(grid), dim3(256), 0, s, (const float *)b.at<float>(P.z), P.T,
-                      P.D, P.K, static_cast<__nv_bfloat16 *>(y));
+                      P.D, P.K, slot_row, static_cast<__nv_bfloat16 *>(y));
 }
 
 int stage_aux(const Plan &P, const Bufs &b, const float *logits, const int *idx, const float *tw, moe_aux *aux,

@@ -83,6 +83,10 @@ struct Params {
     // fp32 reductions; with accum_k <= 2 every element receives at most two
     // additions onto +0, whose result does not depend on their order.
     int accum_k;
+    // EPI_SCATTER with scatter_rows: out is z [rows, ldo] fp32 in the permuted
+    // row order (written by bulk tensor stores through tmO); otherwise z rows
+    // are indexed by slot.
+    int scatter_rows;
     uint64_t timeout_ns;
 };
 
@@ -302,6 +306,35 @@ __device__ __forceinline__ RowGate load_row_gate(const Params &p, int row, int r
     return r;
 }
 
+// Stores one warp's 32 rows x 16 fp32 columns (v: this lane's row) at (column
+// n0, row row0) as two 32 x 8 bulk tensor stores through the warp's shared
+// staging tile when all 32 rows are valid, else row by row.
+__device__ __forceinline__ void store_z_chunk(const CUtensorMap *tmO, uint8_t *stage, float *out, int64_t ldo, int row,
+                                              bool row_ok, const float (&v)[16], int n0, int n_valid) {
+    const int lane = threadIdx.x & 31;
+    if (__all_sync(0xffffffffu, row_ok)) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            if (lane == 0) bulk_wait_read_all();   // the previous store has read the staging tile
+            __syncwarp();
+            float4 *dst = reinterpret_cast<float4 *>(stage + lane * 32);
+            dst[0] = make_float4(v[8 * h], v[8 * h + 1], v[8 * h + 2], v[8 * h + 3]);
+            dst[1] = make_float4(v[8 * h + 4], v[8 * h + 5], v[8 * h + 6], v[8 * h + 7]);
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+                tma_store_2d(tmO, stage, n0 + 8 * h, row - lane);
+                bulk_commit();
+            }
+        }
+    } else if (row_ok) {
+        float *dst = out + (int64_t)row * ldo + n0;
+#pragma unroll
+        for (int k = 0; k < 16; ++k)
+            if (n0 + k < n_valid) dst[k] = v[k];
+    }
+}
+
 template <int BN, int EPI>
 __device__ __forceinline__ void epilogue_tile(const Params &p, const TileCoord &c, int row, int row_limit,
                                               uint32_t tbase, int grp, const CUtensorMap *tmO, uint8_t *stage,
@@ -344,9 +377,11 @@ __device__ __forceinline__ void epilogue_tile(const Params &p, const TileCoord &
     for (int ci = 0; ci < kChunks; ++ci) {
         const int col = grp * kPerGroup + ci * 16;
         const int n0 = c.nt * BN + col;
-        // GELU: the store below is warp-collective, so lanes of invalid rows come along
-        const bool active = (EPI == EPI_GELU ? __any_sync(0xffffffffu, row_ok) : row_ok) && n0 < p.n_valid &&
-                            !(EPI == EPI_SCATTER && slot < 0);
+        // bulk-stored outputs (GELU, row-ordered z): the store is warp-collective,
+        // so lanes of invalid rows come along
+        const bool warp_store = EPI == EPI_GELU || (EPI == EPI_SCATTER && p.scatter_rows);
+        const bool active = (warp_store ? __any_sync(0xffffffffu, row_ok) : row_ok) && n0 < p.n_valid &&
+                            !(EPI == EPI_SCATTER && !p.scatter_rows && slot < 0);
         const bool full_chunk = n0 + 16 <= p.n_valid;
         float bv[16];
 #pragma unroll
@@ -377,7 +412,12 @@ __device__ __forceinline__ void epilogue_tile(const Params &p, const TileCoord &
                 for (int k = 0; k < 8; ++k) pk[k] = gelu_erf_bf16x2(v[2 * k], v[2 * k + 1]);
                 store_h_chunk(tmO, stage, static_cast<__nv_bfloat16 *>(p.out), p.ldo, row, row_ok, pk, n0, p.n_valid);
             } else if (EPI == EPI_SCATTER) {
-                if (p.accum_k > 0) {
+                if (p.scatter_rows) {
+                    float sv[16];
+#pragma unroll
+                    for (int k = 0; k < 16; ++k) sv[k] = gw * v[k];
+                    store_z_chunk(tmO, stage, static_cast<float *>(p.out), p.ldo, row, row_ok, sv, n0, p.n_valid);
+                } else if (p.accum_k > 0) {
                     float *dst = static_cast<float *>(p.out) + (int64_t)(slot / p.accum_k) * p.ldo + n0;
                     if (full_chunk) {
 #pragma unroll

@@ -520,16 +520,20 @@ __global__ void __launch_bounds__(256) zero_kernel(uint4 *__restrict__ p, int64_
 // ---------------------------------------------------------------------------
 template <typename Tout>
 __global__ void __launch_bounds__(256) combine_kernel(const float *__restrict__ z, int64_t T, int D, int K,
-                                                      Tout *__restrict__ y) {
+                                                      const int *__restrict__ slot_row, Tout *__restrict__ y) {
     pdl_enter();
     const int64_t nq = T * (D / 4);
     for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < nq; i += (int64_t)gridDim.x * blockDim.x) {
         const int64_t t = i / (D / 4);
         const int d = (int)(i - t * (D / 4)) * 4;
-        const float *zt = z + (t * K) * D + d;
-        float4 acc = *reinterpret_cast<const float4 *>(zt);
+        // z row of slot (t, j): t*K + j, or its permuted row when slot_row is given
+        auto zrow = [&](int j) -> const float * {
+            const int64_t r = slot_row ? (int64_t)__ldg(slot_row + t * K + j) : t * K + j;
+            return z + r * D + d;
+        };
+        float4 acc = *reinterpret_cast<const float4 *>(zrow(0));
         for (int j = 1; j < K; ++j) {
-            const float4 v = *reinterpret_cast<const float4 *>(zt + (int64_t)j * D);
+            const float4 v = *reinterpret_cast<const float4 *>(zrow(j));
             acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
         }
         if constexpr (sizeof(Tout) == 4) {
