@@ -484,23 +484,27 @@ __global__ void __launch_bounds__(256) permute_kernel(const Tin *__restrict__ x,
         }
     }
     __syncthreads();
-    // one row per warp at a time, four 16-byte vectors in flight per lane
+    // one token per warp at a time: each 16-byte slice of its row is loaded
+    // once (four in flight per lane) and written to all K of its rows
     constexpr int VEC = 16 / sizeof(Tin);
     const int nvec = D / VEC;
-    for (int f = blockIdx.y + gridDim.y * warp; f < n_entries; f += 8 * gridDim.y) {
-        const int dest = s_dest[f];
-        if (dest < 0) continue;
-        const int64_t t = (f0 + f) / K;
-        const uint4 *src = reinterpret_cast<const uint4 *>(x + t * D);
-        uint4 *dst = reinterpret_cast<uint4 *>(x_perm + (int64_t)dest * D);
+    const int n_tok = t_end - t_begin;
+    for (int tt = blockIdx.y + gridDim.y * warp; tt < n_tok; tt += 8 * gridDim.y) {
+        const uint4 *src = reinterpret_cast<const uint4 *>(x + (int64_t)(t_begin + tt) * D);
+        const int *dest = s_dest + tt * K;
         for (int v0 = lane; v0 < nvec; v0 += 128) {
             uint4 r[4];
 #pragma unroll
             for (int u = 0; u < 4; ++u)
                 if (v0 + 32 * u < nvec) r[u] = __ldg(src + v0 + 32 * u);
+            for (int j = 0; j < K; ++j) {
+                const int d = dest[j];
+                if (d < 0) continue;
+                uint4 *dst = reinterpret_cast<uint4 *>(x_perm + (int64_t)d * D);
 #pragma unroll
-            for (int u = 0; u < 4; ++u)
-                if (v0 + 32 * u < nvec) dst[v0 + 32 * u] = r[u];
+                for (int u = 0; u < 4; ++u)
+                    if (v0 + 32 * u < nvec) dst[v0 + 32 * u] = r[u];
+            }
         }
     }
 }
