@@ -83,13 +83,17 @@ struct __align__(16) FinalScratch {
 // kernel's shared memory, no longer used by then) in one coalesced pass when
 // it fits; per expert e, Q threads then take contiguous tile ranges for the
 // totals and the exclusive scan that gives each tile's first row.
+// At most 256 threads work (the scratch arrays' size); larger blocks' other
+// threads only take part in the barriers.
 __device__ void finalize_tables(const Params &p, int ntiles, FinalScratch &f, int *cnt_smem, int cap) {
-    const int N = p.N, nt = blockDim.x, tid = threadIdx.x;
+    const int N = p.N, tid = threadIdx.x;
+    const int nt = blockDim.x < 256 ? (int)blockDim.x : 256;
+    const bool worker = tid < nt;
     const int warp = tid >> 5, lane = tid & 31;
     const bool in_smem = cnt_smem != nullptr && (int64_t)ntiles * N <= cap;
     if (in_smem) {
         const int total = ntiles * N;
-        for (int i0 = tid; i0 < total; i0 += 8 * nt) {
+        for (int i0 = tid; worker && i0 < total; i0 += 8 * nt) {
             int v[8];
 #pragma unroll
             for (int k = 0; k < 8; ++k) v[k] = i0 + k * nt < total ? __ldcg(p.tile_counts + i0 + k * nt) : 0;
@@ -108,14 +112,14 @@ __device__ void finalize_tables(const Params &p, int ntiles, FinalScratch &f, in
     const int R = (ntiles + Q - 1) / Q;           // tiles per thread
     for (int e0 = 0; e0 < N; e0 += epp) {
         const int e = e0 + tid / Q, q = tid % Q;
-        const bool act = tid < epp * Q && e < N;
+        const bool act = worker && tid < epp * Q && e < N;
         const int c0 = q * R, c1 = min(ntiles, c0 + R);
         int cnt = 0;
         if (act) {
 #pragma unroll 8
             for (int c = c0; c < c1; ++c) cnt += count_at(c, e);
         }
-        f.q_cnt[tid] = cnt;
+        if (worker) f.q_cnt[tid] = cnt;
         __syncthreads();
         int base = 0;
         if (act) {
@@ -220,7 +224,7 @@ __device__ void finalize_tables(const Params &p, int ntiles, FinalScratch &f, in
         }
     }
     __syncthreads();
-    for (int e = warp; e < N; e += nt / 32) {
+    for (int e = warp; worker && e < N; e += nt / 32) {
         const int start = f.row[e] + f.cnt[e], end = f.row[e + 1];
         for (int rr = start + lane; rr < end; rr += 32) p.perm_slot[rr] = -1;
     }
