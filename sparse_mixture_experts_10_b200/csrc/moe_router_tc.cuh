@@ -538,6 +538,17 @@ struct SimtShape {
     static size_t smem_bytes(int D) { return w_bytes(D) + 256 * (4 + 4 + 8) + sizeof(FinalScratch) + 16; }
 };
 
+// acc + x.lo * w.lo + x.hi * w.hi for two bf16 pairs, with sm_100's mixed
+// fp32 += bf16 x bf16 FMA: the products are exact and each step rounds as an
+// fp32 FMA of the widened values would, without widening them first.
+__device__ __forceinline__ float fma_bf16x2_acc(uint32_t x, uint32_t w, float acc) {
+    asm("{\n\t.reg .b16 xl, xh, wl, wh;\n\tmov.b32 {xl, xh}, %1;\n\tmov.b32 {wl, wh}, %2;\n\t"
+        "fma.rn.f32.bf16 %0, xl, wl, %0;\n\tfma.rn.f32.bf16 %0, xh, wh, %0;\n\t}"
+        : "+f"(acc)
+        : "r"(x), "r"(w));
+    return acc;
+}
+
 template <int NP>
 __global__ void __launch_bounds__(256, NP == 8 ? 2 : 1) router_simt_kernel(const __nv_bfloat16 *__restrict__ x,
                                                                           const __nv_bfloat16 *__restrict__ Wg,
@@ -623,16 +634,14 @@ __global__ void __launch_bounds__(256, NP == 8 ? 2 : 1) router_simt_kernel(const
                 const int v = v0 + NP * u;
                 if (v >= nvec) break;
                 {
-                    float xf[8];
-                    Vec16<__nv_bfloat16>::unpack(xr[u], xf);
+                    const uint32_t xw[4] = {xr[u].x, xr[u].y, xr[u].z, xr[u].w};
 #pragma unroll
                     for (int ee = 0; ee < NP; ++ee) {
-                        float wf[8];
-                        Vec16<__nv_bfloat16>::load(reinterpret_cast<const __nv_bfloat16 *>(WgT) + (size_t)ee * D +
-                                                       (size_t)v * 8,
-                                                   wf);
-#pragma unroll
-                        for (int q = 0; q < 8; ++q) a[ee] = fmaf(xf[q], wf[q], a[ee]);
+                        const uint4 w4 = *reinterpret_cast<const uint4 *>(WgT + (size_t)ee * D + (size_t)v * 8);
+                        a[ee] = fma_bf16x2_acc(xw[0], w4.x, a[ee]);
+                        a[ee] = fma_bf16x2_acc(xw[1], w4.y, a[ee]);
+                        a[ee] = fma_bf16x2_acc(xw[2], w4.z, a[ee]);
+                        a[ee] = fma_bf16x2_acc(xw[3], w4.w, a[ee]);
                     }
                 }
             }
