@@ -361,6 +361,37 @@ def test_decode_full_layer(name):
     run_full(wl, inp)
 
 
+@pytest.mark.parametrize("N,K,T", [(12, 3, 300), (32, 4, 300), (6, 2, 1), (20, 4, 40), (32, 8, 64), (33, 2, 50)])
+def test_bf16_router_paths(N, K, T):
+    """bf16 routers: the SIMT router with 16 and 32 padded experts (T > 64), the few-token
+    router at several sizes (T <= 64, N <= 32) and the tensor-core router below decode size."""
+    wl = Workload("routers", 20 + N, T, 256, 128, N, K, ACT_SWIGLU, torch.bfloat16, False, 0.05,
+                  zipf_s=0.4, random_bias=True)
+    inp = make_inputs(wl, "cuda")
+    layer, y, ws, aux, V, ref, errs = run_full(wl, inp)
+    check_aux(aux, V, wl.N, wl.K)
+
+
+@pytest.mark.parametrize("T", [1, 20, 50])
+def test_bf16_decode_gelu_with_bias(T):
+    """Decode path with the GELU expert and its biases; tile counts small enough for stream-K
+    (cut tiles summed in piece order) with 16, 32 and 64 token columns."""
+    wl = Workload("decode_gelu", 30, T, 1024, 1024, 6, 2, ACT_GELU, torch.bfloat16, True, 0.03,
+                  random_bias=True)
+    inp = make_inputs(wl, "cuda")
+    run_full(wl, inp)
+
+
+@pytest.mark.parametrize("K", [1, 3])
+def test_bf16_prefill_k1_and_k3(K):
+    """Top-1 (combine folded into the down projection) and top-3 (z in permuted row order,
+    combined by gathering each token's rows in slot order)."""
+    wl = Workload("prefill_k", 31 + K, 700, 512, 512, 6, K, ACT_SWIGLU, torch.bfloat16, False, 0.04,
+                  zipf_s=0.5, random_bias=True)
+    inp = make_inputs(wl, "cuda")
+    run_full(wl, inp)
+
+
 # ----------------------------------------------------------------------------- entry points, determinism
 def test_route_entry_point_matches_forward():
     wl = WORKLOADS["gpt2"]
