@@ -48,8 +48,8 @@ GEMM_KERNEL_SRC = os.path.join(ROOT, "sparse_mixture_experts_10_b200", "csrc", "
 # (dram__bytes_read.sum + dram__bytes_write.sum); keyed by workload and stage,
 # valid only while the kernel source hash is unchanged (see profiles/).
 NCU_TRAFFIC = {
-    "gpt2/up": {"bytes": 110745856, "src_sha256": "d60a1633be6983872816c07aba378b5d5eec95e52cb4973be81ac710a7bfc60e"},
-    "gpt2/down": {"bytes": 183801856, "src_sha256": "d60a1633be6983872816c07aba378b5d5eec95e52cb4973be81ac710a7bfc60e"},
+    "gpt2/up": {"bytes": 108708096, "src_sha256": "7c227d73ad4b51f9796bb92c7559833d64a345edf15e8706150dde12569545b6"},
+    "gpt2/down": {"bytes": 184628992, "src_sha256": "7c227d73ad4b51f9796bb92c7559833d64a345edf15e8706150dde12569545b6"},
 }
 
 
@@ -110,12 +110,15 @@ def work_model(wl, T, counts=None):
     router_flops = T * 2 * D * N
     live = int((counts > 0).sum()) if counts is not None else min(N, T * K)
     up_rows = 2 * H if wl.act == ACT_SWIGLU else H
+    # bf16 prefill with K <= 2 (y is fp32 here): the permute kernel clears y and
+    # the down projection adds into it, so there is no combine pass
+    fused_combine = b == 2 and T > 64 and K <= 2
     return dict(
         flops=router_flops + up_flops + down_flops,
         up_flops=up_flops, down_flops=down_flops, router_flops=router_flops,
         route_bytes=T * D * b + D * N * b + T * N * 4 + T * K * 8,
-        permute_bytes=T * D * b + T * K * D * b + T * K * 8,
-        combine_bytes=T * K * D * 4 + T * D * 4,
+        permute_bytes=T * D * b + T * K * D * b + T * K * 8 + (T * D * 4 if fused_combine else 0),
+        combine_bytes=0 if fused_combine else T * K * D * 4 + T * D * 4,
         up_weight_bytes=live * up_rows * D * b, down_weight_bytes=live * D * H * b,
         live_experts=live,
     )

@@ -381,8 +381,9 @@ int launch_rtc(const CUtensorMap &mx, const CUtensorMap &mw, const rtc::Params &
 
 // Tensor-core router: scores, top-k, statistics partials and (in the last CTA)
 // the dispatch tables and the finished statistics.
+// y_zero: the fp32 output to clear (SIMT router only; see stage_permute), else null.
 int stage_route_tc(const Plan &P, const Bufs &b, const void *x, const moe_weights *w, float *logits, int *idx,
-                   float *tw, int *counts_out, const moe_aux *aux, cudaStream_t s) {
+                   float *tw, int *counts_out, const moe_aux *aux, float *y_zero, cudaStream_t s) {
     const int T = (int)P.T, D = P.D, N = P.N;
     rtc::Params p{};
     p.T = T;
@@ -412,6 +413,7 @@ int stage_route_tc(const Plan &P, const Bufs &b, const void *x, const moe_weight
         p.aux_p_mean = aux->p_mean;
         p.aux_scalars = aux->scalars;
     }
+    p.y_zero = P.simt_router ? y_zero : nullptr;
     p.timeout_ns = kTimeoutNs;
     if (P.few_router) {
         const __nv_bfloat16 *xb = static_cast<const __nv_bfloat16 *>(x);
@@ -549,7 +551,10 @@ int stage_scan(const Plan &P, const Bufs &b, int *counts_out, cudaStream_t s) {
     return check_launch();
 }
 
-int stage_permute(const Plan &P, const Bufs &b, const void *x, const DeviceInfo &dev, cudaStream_t s) {
+// y_zero: the fp32 output to clear on the way (when the combine folds into the
+// down projection), else null.
+int stage_permute(const Plan &P, const Bufs &b, const void *x, float *y_zero, const DeviceInfo &dev,
+                  cudaStream_t s) {
     const size_t smem = (size_t)(P.N + P.chunk_tokens * P.K) * 4;
     // enough blocks to keep every SM copying: split each chunk's rows over several blocks
     const int split = (int)std::max<int64_t>(1, std::min<int64_t>(8, cdiv(2 * dev.sms, P.n_chunks)));
@@ -558,11 +563,11 @@ int stage_permute(const Plan &P, const Bufs &b, const void *x, const DeviceInfo 
         return launch_pdl(permute_kernel<float>, grid, dim3(256), smem, s, static_cast<const float *>(x), (int)P.T, P.D,
                           P.K, P.N, P.chunk_tokens, (const int *)b.at<int>(P.idx), (const int *)b.at<int>(P.chunk_base),
                           (const int *)b.at<int>(P.row_offsets), b.at<int>(P.perm_slot), b.at<int>(P.slot_row),
-                          b.at<float>(P.x_perm));
+                          b.at<float>(P.x_perm), y_zero);
     return launch_pdl(permute_kernel<__nv_bfloat16>, grid, dim3(256), smem, s, static_cast<const __nv_bfloat16 *>(x),
                       (int)P.T, P.D, P.K, P.N, P.chunk_tokens, (const int *)b.at<int>(P.idx),
                       (const int *)b.at<int>(P.chunk_base), (const int *)b.at<int>(P.row_offsets),
-                      b.at<int>(P.perm_slot), b.at<int>(P.slot_row), b.at<__nv_bfloat16>(P.x_perm));
+                      b.at<int>(P.perm_slot), b.at<int>(P.slot_row), b.at<__nv_bfloat16>(P.x_perm), y_zero);
 }
 
 // Expert GEMMs for few tokens (decode path): weight rows are the MMA's M
@@ -731,8 +736,7 @@ int stage_down(const Plan &P, const Bufs &b, const moe_weights *w, void *y, int 
         p.gate_w = b.at<float>(P.w);
         p.timeout_ns = kTimeoutNs;
         CUtensorMap mo = ma;   // unused unless z is written by rows
-        if (combine_in_down(P, y_dtype)) {
-            MOE_TRY(launch_zero(y, (size_t)P.T * D * 4, dev.sms, s));
+        if (combine_in_down(P, y_dtype)) {   // y was cleared by the router or the permute kernel
             p.out = y;
             p.accum_k = P.K;
         } else {
@@ -852,10 +856,13 @@ int forward_impl(const moe_config *cfg, const void *x, int64_t T, const moe_weig
     float *logits = b.at<float>(P.logits);
     int *idx = b.at<int>(P.idx);
     float *tw = b.at<float>(P.w);
+    // the down projection adds into y when the combine folds into it; y is then
+    // cleared on the way, by the SIMT router or else by the permute kernel
+    float *y_zero = combine_in_down(P, y_dtype) ? static_cast<float *>(y) : nullptr;
     MOE_TRY(rec(0));
     MOE_TRY(zero_counters(P, b, s));
     if (P.tc_router) {
-        MOE_TRY(stage_route_tc(P, b, x, w, logits, idx, tw, nullptr, aux, s));
+        MOE_TRY(stage_route_tc(P, b, x, w, logits, idx, tw, nullptr, aux, y_zero, s));
         MOE_TRY(rec(1));
     } else {
         MOE_TRY(stage_route(P, b, x, w, logits, idx, tw, *dev, s));
@@ -863,7 +870,7 @@ int forward_impl(const moe_config *cfg, const void *x, int64_t T, const moe_weig
         MOE_TRY(stage_scan(P, b, nullptr, s));
     }
     MOE_TRY(rec(2));
-    MOE_TRY(stage_permute(P, b, x, *dev, s));
+    MOE_TRY(stage_permute(P, b, x, P.simt_router ? nullptr : y_zero, *dev, s));
     MOE_TRY(rec(3));
     MOE_TRY(stage_up(P, b, w, *dev, s));
     MOE_TRY(rec(4));
@@ -926,7 +933,7 @@ int moe_route(const moe_config *cfg, const void *x, int64_t T, const moe_weights
     Bufs b{static_cast<char *>(ws), &P};
     float *lg = logits ? logits : b.at<float>(P.logits);
     MOE_TRY(zero_counters(P, b, s));
-    if (P.tc_router) return stage_route_tc(P, b, x, w, lg, topk_idx, topk_w, counts, nullptr, s);
+    if (P.tc_router) return stage_route_tc(P, b, x, w, lg, topk_idx, topk_w, counts, nullptr, nullptr, s);
     MOE_TRY(stage_route(P, b, x, w, lg, topk_idx, topk_w, *dev, s));
     if (counts) MOE_TRY(stage_scan(P, b, counts, s));
     return MOE_OK;

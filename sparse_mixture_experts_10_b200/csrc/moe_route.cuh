@@ -444,7 +444,8 @@ __global__ void __launch_bounds__(256) permute_kernel(const Tin *__restrict__ x,
                                                       int chunk_tokens, const int *__restrict__ topk_idx,
                                                       const int *__restrict__ chunk_base,
                                                       const int *__restrict__ row_offsets, int *__restrict__ perm_slot,
-                                                      int *__restrict__ slot_row, Tin *__restrict__ x_perm) {
+                                                      int *__restrict__ slot_row, Tin *__restrict__ x_perm,
+                                                      float *__restrict__ y_zero) {
     pdl_enter();
     extern __shared__ int s_perm[];
     int *s_run = s_perm;            // [N]
@@ -485,7 +486,9 @@ __global__ void __launch_bounds__(256) permute_kernel(const Tin *__restrict__ x,
     }
     __syncthreads();
     // one token per warp at a time: each 16-byte slice of its row is loaded
-    // once (four in flight per lane) and written to all K of its rows
+    // once (four in flight per lane) and written to all K of its rows; when
+    // y_zero is given the warp also clears the token's fp32 output row, which
+    // the down projection then accumulates into
     constexpr int VEC = 16 / sizeof(Tin);
     const int nvec = D / VEC;
     const int n_tok = t_end - t_begin;
@@ -505,6 +508,10 @@ __global__ void __launch_bounds__(256) permute_kernel(const Tin *__restrict__ x,
                 for (int u = 0; u < 4; ++u)
                     if (v0 + 32 * u < nvec) dst[v0 + 32 * u] = r[u];
             }
+        }
+        if (y_zero) {
+            uint4 *yr = reinterpret_cast<uint4 *>(y_zero + (int64_t)(t_begin + tt) * D);
+            for (int v = lane; v < D / 4; v += 32) yr[v] = make_uint4(0u, 0u, 0u, 0u);
         }
     }
 }

@@ -63,6 +63,9 @@ struct Params {
     // statistics (each may be nullptr)
     int *aux_counts;
     float *aux_importance, *aux_p_mean, *aux_scalars;
+    // SIMT router: the layer's fp32 output [T, D] to clear (each block its chunk's
+    // rows) for the down projection's reductions, or nullptr
+    float *y_zero;
     uint64_t timeout_ns;
 };
 
@@ -566,6 +569,16 @@ __global__ void __launch_bounds__(256, NP == 8 ? 2 : 1) router_simt_kernel(const
     FinalScratch *fs = reinterpret_cast<FinalScratch *>(s_i + 256);
     int *s_flag = reinterpret_cast<int *>(fs + 1);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+    // this chunk's output rows are cleared first: the stores drain while W_g is
+    // staged and the scores are computed (the router reads far below HBM speed)
+    if (p.y_zero) {
+        const int64_t t0 = (int64_t)blockIdx.x * kSimtChunk;
+        const int64_t t1 = t0 + kSimtChunk < T ? t0 + kSimtChunk : (int64_t)T;
+        const int64_t n16 = (t1 - t0) * (D / 4);
+        uint4 *yb = reinterpret_cast<uint4 *>(p.y_zero + t0 * D);
+        for (int64_t i = tid; i < n16; i += blockDim.x) yb[i] = make_uint4(0u, 0u, 0u, 0u);
+    }
 
     // W_g [D][N] -> WgT [NP][D]: 16-byte reads of the flat matrix, eight in
     // flight per thread, (d, e) advanced per element
