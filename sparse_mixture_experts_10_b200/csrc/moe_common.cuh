@@ -120,6 +120,19 @@ __device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, const void 
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 // Until this thread's bulk stores have finished reading shared memory.
 __device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// Ticket of the "last arrival does the work" pattern: adds 1 to *ticket with
+// gpu-scope acquire-release semantics and returns the previous count.  Called
+// by one thread after a block barrier: the release covers the block's earlier
+// writes (the barrier orders them before it), and in the last arrival the
+// acquire makes every earlier arrival's writes visible, to the other threads
+// of the block once a second barrier follows.  One atomic instead of a
+// sequentially consistent fence on each side of a relaxed one.
+__device__ __forceinline__ unsigned ticket_arrive(unsigned *ticket) {
+    unsigned old;
+    asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(old) : "l"(ticket) : "memory");
+    return old;
+}
+
 // Until this thread's bulk stores have completed.
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 // Makes this thread's shared-memory writes visible to the async proxy (TMA).

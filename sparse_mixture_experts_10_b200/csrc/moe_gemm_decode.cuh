@@ -371,16 +371,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int j = 0; j < NT; j += 4)
                     __stcg(reinterpret_cast<float4 *>(mine + j), make_float4(acc[j], acc[j + 1], acc[j + 2], acc[j + 3]));
                 // the barrier orders every epilogue thread's stores before the
-                // ticket thread's fence, whose release covers them; the last
-                // piece's ticket thread fences again before the barrier that
-                // releases the other threads to read
+                // ticket thread's acquire-release ticket, whose release covers
+                // them; in the last piece its acquire, followed by the barrier,
+                // lets the other threads read the earlier pieces
                 if (!eb.sync()) break;
-                if (et == 0) {
-                    __threadfence();
-                    const bool last = atomicAdd(p.tickets + c_first, 1u) == (unsigned)(c_last - c_first);
-                    if (last) __threadfence();
-                    *s_last = last;
-                }
+                if (et == 0) *s_last = ticket_arrive(p.tickets + c_first) == (unsigned)(c_last - c_first);
                 if (!eb.sync()) break;
                 if (!*s_last) continue;
                 float sum[NT];

@@ -234,17 +234,13 @@ __device__ void finalize_tables(const Params &p, int ntiles, FinalScratch &f, in
 }
 
 // True in every thread of the block that finished last.
-// The barrier orders the block's stores before thread 0's fence (a release
-// that covers them); the last block's thread 0 fences again before the
-// barrier that lets its other threads read what the other blocks wrote.
+// The barrier orders the block's stores before thread 0's acquire-release
+// ticket, whose release covers them; in the last block the acquire, followed
+// by the second barrier, lets its other threads read what the other blocks
+// wrote.
 __device__ __forceinline__ bool last_block(unsigned *ticket, int *s_flag) {
     __syncthreads();
-    if (threadIdx.x == 0) {
-        __threadfence();
-        const bool last = atomicAdd(ticket, 1u) == gridDim.x - 1;
-        if (last) __threadfence();
-        *s_flag = last;
-    }
+    if (threadIdx.x == 0) *s_flag = ticket_arrive(ticket) == gridDim.x - 1;
     __syncthreads();
     return *s_flag != 0;
 }
@@ -774,12 +770,7 @@ __global__ void __launch_bounds__(256) router_few_kernel(const __nv_bfloat16 *__
         slab_scores[((int64_t)t * S + sl) * 32 + lane] = v;
     }
     __syncthreads();
-    if (tid == 0) {
-        __threadfence();
-        const bool last = atomicAdd(token_ticket + t, 1u) == (unsigned)(S - 1);
-        if (last) __threadfence();
-        s_flag = last;
-    }
+    if (tid == 0) s_flag = ticket_arrive(token_ticket + t) == (unsigned)(S - 1);
     __syncthreads();
     if (!s_flag) return;   // block-uniform: another slab completes this token
     if (warp == 0) {
