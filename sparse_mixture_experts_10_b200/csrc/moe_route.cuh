@@ -457,12 +457,26 @@ __global__ void __launch_bounds__(256) permute_kernel(const Tin *__restrict__ x,
     const int t_end = min(T, t_begin + chunk_tokens);
     const int n_entries = (t_end - t_begin) * K;
     const int64_t f0 = (int64_t)t_begin * K;
+    const int n_tok = t_end - t_begin;
+    constexpr int VEC = 16 / sizeof(Tin);
+    const int nvec = D / VEC;
+    // loads that do not wait for the ranking go out first: warp 0's first 32
+    // entries and each warp's first token's first 128 slices
+    const int e_pre = warp == 0 && lane < n_entries ? topk_idx[f0 + lane] : -1;
+    const int tt_first = blockIdx.y + gridDim.y * warp;
+    uint4 pre[4];
+    if (tt_first < n_tok) {
+        const uint4 *src = reinterpret_cast<const uint4 *>(x + (int64_t)(t_begin + tt_first) * D);
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+            if (lane + 32 * u < nvec) pre[u] = __ldg(src + lane + 32 * u);
+    }
     for (int e = tid; e < N; e += blockDim.x) s_run[e] = row_offsets[e] + chunk_base[(size_t)c * N + e];
     __syncthreads();
     if (warp == 0) {
         for (int base = 0; base < n_entries; base += 32) {
             const int f = base + lane;
-            int e = f < n_entries ? topk_idx[f0 + f] : -1;
+            int e = f < n_entries ? (base == 0 ? e_pre : topk_idx[f0 + f]) : -1;
             if (f < n_entries && (e < 0 || e >= N)) {
                 set_status(kStatusBounds);
                 e = -1;
@@ -489,17 +503,15 @@ __global__ void __launch_bounds__(256) permute_kernel(const Tin *__restrict__ x,
     // once (four in flight per lane) and written to all K of its rows; when
     // y_zero is given the warp also clears the token's fp32 output row, which
     // the down projection then accumulates into
-    constexpr int VEC = 16 / sizeof(Tin);
-    const int nvec = D / VEC;
-    const int n_tok = t_end - t_begin;
-    for (int tt = blockIdx.y + gridDim.y * warp; tt < n_tok; tt += 8 * gridDim.y) {
+    for (int tt = tt_first; tt < n_tok; tt += 8 * gridDim.y) {
         const uint4 *src = reinterpret_cast<const uint4 *>(x + (int64_t)(t_begin + tt) * D);
         const int *dest = s_dest + tt * K;
         for (int v0 = lane; v0 < nvec; v0 += 128) {
             uint4 r[4];
+            const bool prefetched = tt == tt_first && v0 == lane;
 #pragma unroll
             for (int u = 0; u < 4; ++u)
-                if (v0 + 32 * u < nvec) r[u] = __ldg(src + v0 + 32 * u);
+                if (v0 + 32 * u < nvec) r[u] = prefetched ? pre[u] : __ldg(src + v0 + 32 * u);
             for (int j = 0; j < K; ++j) {
                 const int d = dest[j];
                 if (d < 0) continue;

@@ -566,16 +566,6 @@ __global__ void __launch_bounds__(256, NP == 8 ? 2 : 1) router_simt_kernel(const
     int *s_flag = reinterpret_cast<int *>(fs + 1);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
-    // this chunk's output rows are cleared first: the stores drain while W_g is
-    // staged and the scores are computed (the router reads far below HBM speed)
-    if (p.y_zero) {
-        const int64_t t0 = (int64_t)blockIdx.x * kSimtChunk;
-        const int64_t t1 = t0 + kSimtChunk < T ? t0 + kSimtChunk : (int64_t)T;
-        const int64_t n16 = (t1 - t0) * (D / 4);
-        uint4 *yb = reinterpret_cast<uint4 *>(p.y_zero + t0 * D);
-        for (int64_t i = tid; i < n16; i += blockDim.x) yb[i] = make_uint4(0u, 0u, 0u, 0u);
-    }
-
     // W_g [D][N] -> WgT [NP][D]: 16-byte reads of the flat matrix, eight in
     // flight per thread, (d, e) advanced per element
     for (int i = tid; i < (NP - N) * D; i += blockDim.x) WgT[(size_t)N * D + i] = WT(0.f);
@@ -715,9 +705,21 @@ __global__ void __launch_bounds__(256, NP == 8 ? 2 : 1) router_simt_kernel(const
         atomicAdd(p.sum_p + tid, __double2ull_rn((double)ps * kImpScale));
         atomicAdd(p.sum_imp + tid, is);
     }
-    if (last_block(p.ticket, s_flag))
+    const bool last = last_block(p.ticket, s_flag);
+    if (last)
         finalize_tables(p, gridDim.x, *fs, reinterpret_cast<int *>(smem_raw),
                         (int)(SimtShape<NP>::w_bytes(D) / 4));
+    // this chunk's output rows are cleared after the ticket, so that neither the
+    // ticket's release nor the tables wait for these stores: they drain while
+    // the last block builds the tables (the down projection, which adds into y,
+    // starts only after this kernel has completed)
+    if (p.y_zero) {
+        const int64_t t0 = (int64_t)blockIdx.x * kSimtChunk;
+        const int64_t t1 = t0 + kSimtChunk < T ? t0 + kSimtChunk : (int64_t)T;
+        const int64_t n16 = (t1 - t0) * (D / 4);
+        uint4 *yb = reinterpret_cast<uint4 *>(p.y_zero + t0 * D);
+        for (int64_t i = tid; i < n16; i += blockDim.x) yb[i] = make_uint4(0u, 0u, 0u, 0u);
+    }
 }
 
 // ---------------------------------------------------------------------------
