@@ -146,7 +146,12 @@ int moe_route(const moe_config *cfg, const void *x, int64_t T, const moe_weights
  * article, layer formula): route, group the (token, slot) pairs by expert,
  * evaluate each selected expert once per pair on the tensor cores, scale by the
  * gate weight and sum the K contributions of a token in slot order 0..K-1.
- *  x [T, D] dtype (device); y [T, D] in y_dtype (MOE_F32 or MOE_BF16).
+ *  x [T, D] dtype (device); y [T, D] in y_dtype (MOE_F32 or MOE_BF16), written
+ *      in full; it must not overlap x, the weights or the workspace.  For bf16
+ *      layers with T > 64, K <= 2 and an fp32 y, y is cleared before the expert
+ *      GEMMs and the down projection adds each token's K scaled rows into it;
+ *      with at most two terms on +0 this gives the same bits as the slot-order
+ *      sum.
  *  aux: optional statistics (see moe_aux), or NULL.
  * The routing results and intermediates stay in the workspace; their places
  * are given by moe_workspace_layout().  T == 0 is a no-op (aux zeroed). */
