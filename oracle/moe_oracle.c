@@ -26,7 +26,7 @@
  *        Loading Refactor" (packed gate_up_proj: experts on dim 0, gate then
  *        up on dim 1) and section 2 "Expert Backend".
  *
- * Readings where the pages are silent (each one is listed in the design doc):
+ * Readings where the pages are silent:
  *   - Load(X) of the Shazeer article is a smooth estimator that needs the
  *     training noise; it is not printed.  The oracle uses the hard per-expert
  *     count instead.  The smooth estimator itself is not implemented:
