@@ -226,9 +226,10 @@ def test_chunked_router_path(N, K, T):
 
 
 @pytest.mark.parametrize("dtype,N,K", [(torch.float32, 40, 3), (torch.float32, 64, 6), (torch.bfloat16, 64, 4),
-                                       (torch.bfloat16, 300, 8)])
+                                       (torch.bfloat16, 300, 8), (torch.bfloat16, 40, 2), (torch.bfloat16, 64, 1)])
 def test_gemm_router_path(dtype, N, K):
-    """N > 32 takes the router GEMM (SIMT for fp32, tcgen05 dense tile for bf16) and the top-k kernel."""
+    """N > 32 takes the router GEMM (SIMT for fp32, tcgen05 dense tile for bf16) and the top-k kernel.
+    bf16 with K <= 2: the combine folds into the down projection and the permute kernel clears y."""
     wl = Workload("many_experts", 11, 700, 256, 128, N, K, ACT_SWIGLU if dtype == torch.bfloat16 else ACT_GELU,
                   dtype, dtype == torch.float32, 0.05, zipf_s=0.5, random_bias=True)
     inp = make_inputs(wl, "cuda")
