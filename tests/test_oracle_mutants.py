@@ -40,6 +40,25 @@ MUTANTS = [
      [pins.test_aux_stats_invariants_and_library_checks]),
     ("expert_params_one_matrix", "return 2 * D * H + (has_bias ? H + D : 0);", "return D * H + (has_bias ? H + D : 0);",
      [pins.test_gpt2_moe_parameter_totals]),
+    ("softmax_shift_flipped", "w[j] = exp(scores[sel[j]] - smax);", "w[j] = exp(smax - scores[sel[j]]);",
+     [pins.test_gate_weights_sum_to_one_and_order, pins.test_two_way_gate_is_logistic_of_gap]),
+    ("down_bias_dropped", "if (b2e) a += (double)b2e[c];", "(void)b2e;",
+     [pins.test_one_expert_top1_is_dense_ffn]),
+    ("silu_sign_flipped", "return g / (1.0 + exp(-g));", "return g / (1.0 + exp(g));",
+     [pins.test_activation_closed_forms, pins.test_one_expert_top1_is_dense_ffn]),
+    ("combine_unweighted", "y[c] = y[c] + w[j] * E[j * D + c];", "y[c] = y[c] + E[j * D + c];",
+     [pins.test_sparse_layer_equals_dense_masked_gate]),
+    ("simple_loss_missing_N", "return (double)N * sum;", "return sum;",
+     [pins.test_balance_loss_extremes, pins.test_aux_stats_uniform_and_empty]),
+    ("switch_loss_missing_N", "scalars[0] = (double)N * fP;", "scalars[0] = fP;",
+     [pins.test_aux_stats_uniform_and_empty, pins.test_aux_stats_invariants_and_library_checks]),
+    ("cv2_mean_not_squared", "return var / (mean * mean);", "return var / mean;",
+     [pins.test_cv_squared_closed_forms]),
+    ("importance_counts_tokens", "importance[sel[t * K + j]] += w[t * K + j];", "importance[sel[t * K + j]] += 1.0;",
+     [pins.test_aux_stats_invariants_and_library_checks]),
+    ("p_mean_not_averaged", "for (int64_t e = 0; e < N; ++e) p_mean[e] /= (double)T;",
+     "for (int64_t e = 0; e < N; ++e) p_mean[e] /= 1.0;",
+     [pins.test_aux_stats_invariants_and_library_checks]),
 ]
 
 
