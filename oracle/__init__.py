@@ -74,9 +74,12 @@ def configure(L):
     L.orc_silu.argtypes = [dp]
     L.orc_load_row.argtypes = [i64, vp, i32, i64, vp]
     L.orc_router_scores.argtypes = [i64, i64, vp, vp, i32, vp, vp]
+    L.orc_expert_rank.restype = i64
+    L.orc_expert_rank.argtypes = [i64, vp, i64]
     L.orc_rank_experts.argtypes = [i64, vp, vp]
     L.orc_select_topk.argtypes = [i64, i64, vp, vp]
-    L.orc_gate_weights.argtypes = [i64, vp, vp, vp]
+    L.orc_softmax.argtypes = [i64, vp, vp]
+    L.orc_gate_weights.argtypes = [i64, i64, vp, vp, vp]
     L.orc_expert_gelu.argtypes = [i64, i64, vp, vp, vp, vp, vp, i32, vp, vp]
     L.orc_expert_swiglu.argtypes = [i64, i64, vp, vp, vp, i32, vp, vp]
     L.orc_combine.argtypes = [i64, i64, vp, vp, vp]
@@ -133,7 +136,7 @@ def silu(v: float) -> float:
 
 # --- routing ----------------------------------------------------------------------------------------
 def rank_experts(scores) -> np.ndarray:
-    """Stable descending order of one score row (equal scores: lower index first)."""
+    """The experts of one score row in rank order (descending score, equal scores: lower index first)."""
     s = _c(scores, np.float64)
     out = np.empty(s.shape[0], dtype=np.int32)
     lib().orc_rank_experts(s.shape[0], _p(s), _p(out))
@@ -152,14 +155,23 @@ def select_topk(scores, K: int) -> np.ndarray:
 
 
 def gate_weights(scores, sel) -> np.ndarray:
-    """Renormalised softmax over the selected scores of each row."""
+    """Slot weights G(x)[sel_j] of G = softmax(KeepTopK(scores)) with the kept set sel, per row."""
     s = np.atleast_2d(_c(scores, np.float64))
     sl = np.atleast_2d(_c(sel, np.int32))
     T, K = sl.shape
+    N = s.shape[1]
     out = np.empty((T, K), dtype=np.float64)
     L = lib()
     for t in range(T):
-        L.orc_gate_weights(K, _p(s[t]), _p(sl[t]), _p(out[t]))
+        L.orc_gate_weights(N, K, _p(s[t]), _p(sl[t]), _p(out[t]))
+    return out
+
+
+def softmax(v) -> np.ndarray:
+    """softmax of one vector (entries of -inf get probability 0)."""
+    a = _c(v, np.float64)
+    out = np.empty_like(a)
+    lib().orc_softmax(a.shape[0], _p(a), _p(out))
     return out
 
 

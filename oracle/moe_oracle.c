@@ -61,10 +61,10 @@ void orc_load_row(int64_t D, const void *x, int dtype, int64_t t, double *row) {
 }
 
 /* ------------------------------------------------------------------------
- * Router scores.  "MoE(Mixture of Experts)" section (2), Route: for each
- * expert e, s_e = sum_i x_i * router[i, e], i ascending; the Shazeer article's
- * gate is x W_g with W_g of shape [DModel, NExperts].  b_g (optional) is added
- * after the sum.
+ * Router scores.  Shazeer article, gating section: the gate's scores are
+ * H(x) = x W_g with W_g of shape [DModel, NExperts], i.e. the matrix-vector
+ * product s_e = sum_i x_i W_g[i, e] (summed here in ascending i).  b_g
+ * (optional) is added after the sum.
  * ---------------------------------------------------------------------- */
 void orc_router_scores(int64_t D, int64_t N, const double *x_row,
                        const void *Wg, int w_dtype, const float *bg,
@@ -78,47 +78,71 @@ void orc_router_scores(int64_t D, int64_t N, const double *x_row,
 }
 
 /* ------------------------------------------------------------------------
- * Expert order.  "MoE(Mixture of Experts)" section (2), Route: the expert
- * indices 0..N-1 are sorted by descending score with a STABLE sort, so equal
- * scores keep ascending expert index.  Insertion sort is stable: an element
- * moves left only past elements with a strictly smaller score.
+ * Ranking of the experts.  Shazeer article, gating section: KeepTopK(v, k)
+ * keeps the k largest entries of the score vector v.  Which of several equal
+ * scores count as "largest" is the reading that the lower expert index comes
+ * first (the chapter "MoE(Mixture of Experts)", section (2), gets the same
+ * order from a stable sort of the indices by descending score).  So the rank
+ * of expert e is the number of experts placed before it: those with a
+ * strictly larger score, and those with an equal score and a lower index.
+ * Ranks are a permutation of 0..N-1.
  * ---------------------------------------------------------------------- */
+int64_t orc_expert_rank(int64_t N, const double *scores, int64_t e) {
+    int64_t r = 0;
+    for (int64_t j = 0; j < N; ++j) {
+        if (scores[j] > scores[e]) r += 1;
+        else if (scores[j] == scores[e] && j < e) r += 1;
+    }
+    return r;
+}
+
+/* All experts by rank: order[rank(e)] = e. */
 void orc_rank_experts(int64_t N, const double *scores, int32_t *order) {
-    for (int64_t i = 0; i < N; ++i) order[i] = (int32_t)i;
-    for (int64_t i = 1; i < N; ++i) {
-        int32_t key = order[i];
-        int64_t j = i - 1;
-        while (j >= 0 && scores[order[j]] < scores[key]) {
-            order[j + 1] = order[j];
-            --j;
-        }
-        order[j + 1] = key;
+    for (int64_t e = 0; e < N; ++e) order[orc_expert_rank(N, scores, e)] = (int32_t)e;
+}
+
+/* The set KeepTopK keeps: the experts of rank below K, listed best first
+ * (slot j holds the expert of rank j). */
+void orc_select_topk(int64_t N, int64_t K, const double *scores, int32_t *sel) {
+    for (int64_t e = 0; e < N; ++e) {
+        int64_t r = orc_expert_rank(N, scores, e);
+        if (r < K) sel[r] = (int32_t)e;
     }
 }
 
-/* The selected experts are the first K of that order, best first. */
-void orc_select_topk(int64_t N, int64_t K, const double *scores, int32_t *sel) {
-    int32_t *order = (int32_t *)malloc(sizeof(int32_t) * (size_t)N);
-    orc_rank_experts(N, scores, order);
-    for (int64_t j = 0; j < K; ++j) sel[j] = order[j];
-    free(order);
+/* softmax(v)_i = exp(v_i) / sum_m exp(v_m) over n entries, an entry of -inf
+ * giving exp(-inf) = 0.  Evaluated as exp(v_i - M) / sum_m exp(v_m - M) with M
+ * the largest entry (the softmax does not change when every entry is
+ * shifted by the same amount). */
+void orc_softmax(int64_t n, const double *v, double *p) {
+    double M = -INFINITY;
+    for (int64_t i = 0; i < n; ++i)
+        if (v[i] > M) M = v[i];
+    double z = 0.0;
+    for (int64_t i = 0; i < n; ++i) {
+        p[i] = v[i] == -INFINITY ? 0.0 : exp(v[i] - M);
+        z += p[i];
+    }
+    for (int64_t i = 0; i < n; ++i) p[i] = p[i] / z;
 }
 
 /* ------------------------------------------------------------------------
- * Gate weights.  Shazeer article, gating: G(x) = softmax(KeepTopK(H(x), k)),
- * KeepTopK sets every unselected entry to -inf, so the softmax is taken over
- * the k kept scores only; "MoE(Mixture of Experts)" section (2) computes it
- * shifted by the best score: w_j = exp(s_{sel_j} - s_{sel_0}) / sum_m (...).
- * The inference form has no noise term.
+ * Gate weights.  Shazeer article, gating section, inference form (no noise
+ * term): G(x) = softmax(KeepTopK(H(x), k)) with H(x) = x W_g and
+ * KeepTopK(v, k)_e = v_e for a kept expert, -inf for every other one.  The
+ * kept set is given as sel (K experts, normally orc_select_topk of these same
+ * scores); G is dense over the N experts and zero outside the kept set.  The
+ * weight of slot j is G at expert sel_j.
  * ---------------------------------------------------------------------- */
-void orc_gate_weights(int64_t K, const double *scores, const int32_t *sel, double *w) {
-    double smax = scores[sel[0]];
-    double sum = 0.0;
-    for (int64_t j = 0; j < K; ++j) {
-        w[j] = exp(scores[sel[j]] - smax);
-        sum += w[j];
-    }
-    for (int64_t j = 0; j < K; ++j) w[j] = w[j] / sum;
+void orc_gate_weights(int64_t N, int64_t K, const double *scores, const int32_t *sel, double *w) {
+    double *v = (double *)malloc(sizeof(double) * (size_t)N);
+    double *G = (double *)malloc(sizeof(double) * (size_t)N);
+    for (int64_t e = 0; e < N; ++e) v[e] = -INFINITY;
+    for (int64_t j = 0; j < K; ++j) v[sel[j]] = scores[sel[j]];
+    orc_softmax(N, v, G);
+    for (int64_t j = 0; j < K; ++j) w[j] = G[sel[j]];
+    free(v);
+    free(G);
 }
 
 /* Exact-erf GELU: gelu(v) = v * Phi(v) = 0.5 v (1 + erf(v / sqrt 2)). */
@@ -252,7 +276,7 @@ void orc_moe_layer_rows(const orc_layer *L, int64_t t0, int64_t t1,
         } else {
             orc_select_topk(N, K, s, sel);
         }
-        orc_gate_weights(K, s, sel, w);
+        orc_gate_weights(N, K, s, sel, w);
         for (int64_t j = 0; j < K; ++j) orc_expert(L, sel[j], x_row, hid, E + j * D);
         orc_combine(K, D, w, E, y_out + t * D);
     }

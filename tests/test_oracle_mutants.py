@@ -10,12 +10,18 @@ from tests import test_oracle_pins as pins
 
 MUTANTS = [
     # (name, original text, planted mistake, pins expected to catch it)
-    ("no_renormalisation", "w[j] = w[j] / sum;", "w[j] = w[j];",
+    ("no_renormalisation", "for (int64_t i = 0; i < n; ++i) p[i] = p[i] / z;",
+     "for (int64_t i = 0; i < n; ++i) p[i] = p[i];",
      [pins.test_gate_weights_sum_to_one_and_order, pins.test_two_way_gate_is_logistic_of_gap]),
-    ("unstable_tie_order", "scores[order[j]] < scores[key]", "scores[order[j]] <= scores[key]",
+    ("ties_to_higher_index", "scores[j] == scores[e] && j < e", "scores[j] == scores[e] && j > e",
      [pins.test_topk_matches_library_sort_with_many_ties, pins.test_tie_break_duplicate_router_columns]),
-    ("ascending_sort", "scores[order[j]] < scores[key]", "scores[order[j]] > scores[key]",
+    ("ascending_rank", "if (scores[j] > scores[e]) r += 1;", "if (scores[j] < scores[e]) r += 1;",
      [pins.test_worked_router_example]),
+    ("ties_not_ranked", "else if (scores[j] == scores[e] && j < e) r += 1;", "else if (0) r += 1;",
+     [pins.test_topk_matches_library_sort_with_many_ties, pins.test_tie_break_duplicate_router_columns]),
+    ("softmax_over_all_experts", "for (int64_t e = 0; e < N; ++e) v[e] = -INFINITY;",
+     "for (int64_t e = 0; e < N; ++e) v[e] = scores[e];",
+     [pins.test_gate_weights_sum_to_one_and_order, pins.test_gate_weights_equal_masked_full_softmax]),
     ("combine_drops_last_slot", "for (int64_t j = 0; j < K; ++j)\n        for (int64_t c = 0; c < D; ++c) y[c]",
      "for (int64_t j = 0; j < K - 1; ++j)\n        for (int64_t c = 0; c < D; ++c) y[c]",
      [pins.test_sparse_layer_equals_dense_masked_gate]),
@@ -40,7 +46,8 @@ MUTANTS = [
      [pins.test_aux_stats_invariants_and_library_checks]),
     ("expert_params_one_matrix", "return 2 * D * H + (has_bias ? H + D : 0);", "return D * H + (has_bias ? H + D : 0);",
      [pins.test_gpt2_moe_parameter_totals]),
-    ("softmax_shift_flipped", "w[j] = exp(scores[sel[j]] - smax);", "w[j] = exp(smax - scores[sel[j]]);",
+    ("softmax_shift_flipped", "p[i] = v[i] == -INFINITY ? 0.0 : exp(v[i] - M);",
+     "p[i] = v[i] == -INFINITY ? 0.0 : exp(M - v[i]);",
      [pins.test_gate_weights_sum_to_one_and_order, pins.test_two_way_gate_is_logistic_of_gap]),
     ("down_bias_dropped", "if (b2e) a += (double)b2e[c];", "(void)b2e;",
      [pins.test_one_expert_top1_is_dense_ffn]),
