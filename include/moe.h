@@ -197,13 +197,52 @@ int moe_aux_stats(const moe_config *cfg, int64_t T, const float *logits, const i
  *
  * Set-up: the first call on each device (with that device current) looks up
  * the array's device address, once.  Make that first call before capturing
- * the stream into a CUDA graph.
+ * the stream into a CUDA graph.  The address is kept for the life of the
+ * process: after cudaDeviceReset (or anything else that destroys the device's
+ * primary context) the kept address is stale, so do not call this entry point
+ * again in that process.
  *
  * Arguments, layouts and other errors as moe_aux_stats. */
 #define MOE_NOALLOC_SCRATCH_BYTES (2u << 20)
 int moe_aux_stats_noalloc(const moe_config *cfg, int64_t T, const float *logits,
                           const int32_t *topk_idx, const float *topk_w, moe_aux *out,
                           moe_stream_t stream);
+
+/* Statistics under data parallelism ("MoE(Mixture of Experts)", section (3):
+ * f_e is the share of ALL routed tokens; Shazeer article, load-balancing
+ * losses: Importance(X) and Load(X) sum over the whole batch X).  When the
+ * tokens of one batch are split over ranks (each rank runs the layer on its
+ * own shard with replicated weights), the losses of the global batch come from
+ * each rank's partial sums added over the ranks, then finalised.
+ *
+ * moe_aux_partials writes one rank's partials as exact integers, so that the
+ * sum over ranks (an all-reduce of int64, e.g. NCCL ncclInt64 / ncclSum) is the
+ * same on every rank and in any order:
+ *   partials[0, N)    tokens routed to each expert
+ *   partials[N, 2N)   sum over the slots routed to e of round(w * 2^32)
+ *   partials[2N, 3N)  sum over tokens of round(softmax(scores)_e * 2^32), the
+ *                     full N-way softmax
+ *   partials[3N]      number of tokens T
+ * Arguments as moe_aux_stats (routing results in device memory; moe_forward
+ * leaves them in its workspace, see moe_get_workspace_layout); partials is
+ * MOE_AUX_PARTIALS_LEN(N) int64 of device memory, overwritten.  No workspace.
+ * T == 0 writes zeros. */
+#define MOE_AUX_PARTIALS_LEN(N) (3 * (int64_t)(N) + 1)
+int moe_aux_partials(const moe_config *cfg, int64_t T, const float *logits, const int32_t *topk_idx,
+                     const float *topk_w, int64_t *partials, moe_stream_t stream);
+
+/* The statistics of moe_aux (counts, importance, p_mean, the four scalars) from
+ * partials summed over ranks (device memory, read on `stream`); any output
+ * pointer may be NULL.  Every rank that finalises the same summed partials gets
+ * bitwise-identical statistics. */
+int moe_aux_finalize(const moe_config *cfg, const int64_t *partials, moe_aux *out, moe_stream_t stream);
+
+/* The same finalisation on the host, for host copies of the summed partials
+ * (for instance after an all-reduce over CPU processes); outputs are host
+ * arrays ([N], [N], [N], [4]), any of them NULL to skip.  Gives the same bits
+ * as moe_aux_finalize.  MOE_ERR_INVALID_ARG on a negative entry. */
+int moe_aux_finalize_host(const moe_config *cfg, const int64_t *partials, int32_t *counts, float *importance,
+                          float *p_mean, float *scalars);
 
 /* Where moe_forward leaves its intermediates inside the workspace (byte
  * offsets from ws), for inspection in tests.  Rows of each expert's segment in

@@ -36,7 +36,7 @@ MOE_STATUS_TIMEOUT, MOE_STATUS_BOUNDS, MOE_STATUS_NAN_LOGIT = 1, 2, 4
 MOE_NOALLOC_SCRATCH_BYTES = 2 << 20
 
 EXPORTED = ("moe_workspace_size", "moe_route", "moe_forward", "moe_forward_timed", "moe_aux_stats",
-            "moe_aux_stats_noalloc",
+            "moe_aux_stats_noalloc", "moe_aux_partials", "moe_aux_finalize", "moe_aux_finalize_host",
             "moe_get_workspace_layout", "moe_total_params", "moe_active_params", "moe_get_device_status",
             "moe_launch_count", "moe_error_string", "moe_selftest_wait_timeout")
 
@@ -98,6 +98,12 @@ def load_library():
     L.moe_aux_stats.argtypes = [cfgp, i64, vp, vp, vp, auxp, vp, sz, vp]
     L.moe_aux_stats_noalloc.restype = ctypes.c_int
     L.moe_aux_stats_noalloc.argtypes = [cfgp, i64, vp, vp, vp, auxp, vp]
+    L.moe_aux_partials.restype = ctypes.c_int
+    L.moe_aux_partials.argtypes = [cfgp, i64, vp, vp, vp, vp, vp]
+    L.moe_aux_finalize.restype = ctypes.c_int
+    L.moe_aux_finalize.argtypes = [cfgp, vp, auxp, vp]
+    L.moe_aux_finalize_host.restype = ctypes.c_int
+    L.moe_aux_finalize_host.argtypes = [cfgp, vp, vp, vp, vp, vp]
     L.moe_get_workspace_layout.restype = ctypes.c_int
     L.moe_get_workspace_layout.argtypes = [cfgp, i64, ctypes.POINTER(moe_workspace_layout)]
     L.moe_total_params.restype = i64
@@ -205,6 +211,26 @@ def moe_aux_stats_noalloc(cfg, T, logits, topk_idx, topk_w, out, stream=None) ->
     device race on that array."""
     return load_library().moe_aux_stats_noalloc(ctypes.byref(cfg), T, _ptr(logits), _ptr(topk_idx), _ptr(topk_w),
                                                 ctypes.byref(out), _stream(stream))
+
+
+def aux_partials_len(N: int) -> int:
+    return 3 * N + 1
+
+
+def moe_aux_partials(cfg, T, logits, topk_idx, topk_w, partials, stream=None) -> int:
+    """One rank's statistics as exact int64 partial sums (device tensor of 3N+1)."""
+    return load_library().moe_aux_partials(ctypes.byref(cfg), T, _ptr(logits), _ptr(topk_idx), _ptr(topk_w),
+                                           _ptr(partials), _stream(stream))
+
+
+def moe_aux_finalize(cfg, partials, out, stream=None) -> int:
+    return load_library().moe_aux_finalize(ctypes.byref(cfg), _ptr(partials), ctypes.byref(out), _stream(stream))
+
+
+def moe_aux_finalize_host(cfg, partials, counts=None, importance=None, p_mean=None, scalars=None) -> int:
+    """Host version: partials, counts, importance, p_mean, scalars are CPU tensors (int64, int32, fp32)."""
+    return load_library().moe_aux_finalize_host(ctypes.byref(cfg), _ptr(partials), _ptr(counts), _ptr(importance),
+                                                _ptr(p_mean), _ptr(scalars))
 
 
 def moe_get_workspace_layout(cfg, T) -> moe_workspace_layout:

@@ -201,6 +201,7 @@ int device_info(DeviceInfo **out) {
         MOE_TRY(allow_smem(router_small_kernel<__nv_bfloat16, 16>));
         MOE_TRY(allow_smem(router_small_kernel<__nv_bfloat16, 32>));
         MOE_TRY(allow_smem(aux_partial_kernel));
+        MOE_TRY(allow_smem(aux_partials_kernel));
         MOE_TRY(allow_smem(rtc::router_simt_kernel<8>));
         MOE_TRY(allow_smem(rtc::router_simt_kernel<16>));
         MOE_TRY(allow_smem(rtc::router_simt_kernel<32>));
@@ -966,6 +967,48 @@ int moe_aux_stats(const moe_config *cfg, int64_t T, const float *logits, const i
     Bufs b{static_cast<char *>(ws), &P};
     MOE_TRY(zero_counters(P, b, s));
     return stage_aux(P, b, logits, topk_idx, topk_w, out, s);
+}
+
+int moe_aux_partials(const moe_config *cfg, int64_t T, const float *logits, const int32_t *topk_idx,
+                     const float *topk_w, int64_t *partials, moe_stream_t stream) {
+    Plan P;
+    MOE_TRY(make_plan(cfg, T, &P));
+    if (!partials) return MOE_ERR_INVALID_ARG;
+    if (T > 0 && (!logits || !topk_idx || !topk_w)) return MOE_ERR_INVALID_ARG;
+    if (T > INT32_MAX) return MOE_ERR_UNSUPPORTED;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const size_t bytes = (size_t)(3 * P.N + 1) * 8;
+    if (cudaMemsetAsync(partials, 0, bytes, s) != cudaSuccess) return MOE_ERR_CUDA;
+    if (T == 0) return MOE_OK;
+    DeviceInfo *dev = nullptr;
+    MOE_TRY(device_info(&dev));
+    const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(cdiv(T, 8), (int64_t)dev->sms * 4));
+    aux_partials_kernel<<<grid, 256, (size_t)3 * P.N * 8, s>>>(logits, topk_idx, topk_w, (int)T, P.N, P.K,
+                                                                reinterpret_cast<unsigned long long *>(partials));
+    return check_launch();
+}
+
+int moe_aux_finalize(const moe_config *cfg, const int64_t *partials, moe_aux *out, moe_stream_t stream) {
+    Plan P;
+    MOE_TRY(make_plan(cfg, 0, &P));
+    if (!partials || !out) return MOE_ERR_INVALID_ARG;
+    AuxOut o{out->counts, out->importance, out->p_mean, out->scalars};
+    aux_finalize_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+        P.N, P.K, reinterpret_cast<const long long *>(partials), o);
+    return check_launch();
+}
+
+int moe_aux_finalize_host(const moe_config *cfg, const int64_t *partials, int32_t *counts, float *importance,
+                          float *p_mean, float *scalars) {
+    Plan P;
+    MOE_TRY(make_plan(cfg, 0, &P));
+    if (!partials) return MOE_ERR_INVALID_ARG;
+    if (partials[3 * P.N] < 0) return MOE_ERR_INVALID_ARG;
+    for (int e = 0; e < 3 * P.N; ++e)
+        if (partials[e] < 0) return MOE_ERR_INVALID_ARG;
+    aux_finalize_partials(P.N, P.K, reinterpret_cast<const long long *>(partials), counts, importance, p_mean,
+                          scalars);
+    return MOE_OK;
 }
 
 int64_t moe_total_params(const moe_config *c) {

@@ -92,6 +92,24 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint64
     }
 }
 
+// Producer bookkeeping of a ring of at most 32 slots: which slots have had
+// copies issued and the barrier phase of the last one.  When a bounded wait
+// has run out and the producer stops, drain() waits (again bounded) until
+// every slot's last issued copies have landed, so that the CTA never leaves
+// with a bulk copy still writing into its shared memory.  A copy that has
+// been consumed already completed its phase, so its wait returns at once.
+struct IssuedSlots {
+    uint32_t mask = 0, phase = 0;
+    __device__ __forceinline__ void note(int stage, uint32_t ph) {
+        mask |= 1u << stage;
+        phase = (phase & ~(1u << stage)) | ((ph & 1u) << stage);
+    }
+    __device__ __forceinline__ void drain(uint64_t *full, uint64_t timeout_ns) const {
+        for (int s = 0; s < 32; ++s)
+            if ((mask >> s) & 1u) mbar_wait(&full[s], (phase >> s) & 1u, timeout_ns);
+    }
+};
+
 // ---------------------------------------------------------------- TMA
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap *map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");

@@ -216,6 +216,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             int stage = 0;
             uint32_t phase = 0;
             bool ok = true;
+            IssuedSlots iss;
             for (int64_t u = u_begin; u < u_end && ok;) {
                 const Piece pc(u, stream_k ? u_end : u + nkb, nkb);
                 u = stream_k ? u + (pc.k1 - pc.k0) : u + u_step;
@@ -243,17 +244,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                         tma_load_2d(&tmW, &full[stage], sA + stage * S::kABytes, kb * BK, wrow);
                     }
                     tma_load_2d(&tmX, &full[stage], sB + stage * S::kBBytes, kb * BK, trow);
+                    iss.note(stage, phase);
                     if (++stage == kStages) {
                         stage = 0;
                         phase ^= 1;
                     }
                 }
             }
-            if (!ok) {
-                const uint64_t t0 = globaltimer_ns();
-                while (globaltimer_ns() - t0 < 1000000ull) {
-                }
-            }
+            if (!ok) iss.drain(full, p.timeout_ns);   // copies in flight land before the CTA leaves
         }
     } else if (warp == 1) {
         if (lane == 0) {

@@ -505,6 +505,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             int stage = 0;
             uint32_t phase = 0;
             bool ok = true;
+            IssuedSlots iss;
             for (int i = blockIdx.x; i < total && ok; i += gridDim.x) {
                 const TileCoord c = decode_tile(i, rowoff, G, p.n_tiles, dense_mtiles);
                 int brow, brow2 = 0;
@@ -527,18 +528,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                     } else {
                         tma_load_2d(&tmB, &full[stage], sB + stage * S::kBBytes, kb * BK, brow);
                     }
+                    iss.note(stage, phase);
                     if (++stage == kStages) {
                         stage = 0;
                         phase ^= 1;
                     }
                 }
             }
-            if (!ok) {
-                // let copies already in flight land before the CTA leaves
-                const uint64_t t0 = globaltimer_ns();
-                while (globaltimer_ns() - t0 < 1000000ull) {
-                }
-            }
+            if (!ok) iss.drain(full, p.timeout_ns);   // copies in flight land before the CTA leaves
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
@@ -789,6 +786,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             int stage = 0;
             uint32_t phase = 0;
             bool ok = true;
+            IssuedSlots iss;
             for (int i = cid; i < total && ok; i += ncl) {
                 const TileCoord c = decode_unit_tile(i, rowoff, s_units, G, p.n_tiles, dense_units);
                 const int arow = c.row0 + (int)rank * BM;
@@ -806,17 +804,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     const uint32_t leader_full = mapa_shared(smem_u32(&full[stage]), 0);
                     tma_load_2d_pair(&tmA, leader_full, sA + stage * S::kABytes, kb * BK, arow);
                     tma_load_2d_pair(&tmB, leader_full, sB + stage * S::kBBytes, kb * BK, brow);
+                    iss.note(stage, phase);
                     if (++stage == kStages) {
                         stage = 0;
                         phase ^= 1;
                     }
                 }
             }
-            if (!ok) {
-                const uint64_t t0 = globaltimer_ns();
-                while (globaltimer_ns() - t0 < 1000000ull) {
-                }
-            }
+            // both CTAs' copies complete on the leader's barriers: the leader waits
+            // (bounded) for every slot's last copies; the cluster barrier at the end
+            // keeps the other CTA resident until then
+            if (!ok && rank == 0) iss.drain(full, p.timeout_ns);
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer (leader CTA only)

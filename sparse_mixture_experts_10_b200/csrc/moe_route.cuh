@@ -787,6 +787,118 @@ __global__ void __launch_bounds__(256) aux_partial_kernel(const float *__restric
     if (last_block_done(counter)) aux_finalize_block(part_p, part_imp, part_cnt, gridDim.x, T, N, K, out);
 }
 
+// ---------------------------------------------------------------------------
+// Statistics as exact integer sums, for data parallelism.  Under token-sharded
+// data parallelism the layer's losses are defined over the global batch (the
+// Shazeer article's Importance(X) and Load(X) sum over the batch X; the chapter
+// "MoE(Mixture of Experts)", section (3), takes f_e over all routed tokens), so
+// each rank's partial sums are added across ranks and then finalised.  Here
+// every partial is an integer: per expert the routed slots, the gate weights
+// and the full-softmax probabilities, each term rounded to 2^-32 fixed point.
+// Integer additions give the same bits in any order -- inside the kernel (its
+// atomics), across ranks (an all-reduce of int64) -- so every rank finalises
+// the same numbers.
+//   part[0, N)    counts
+//   part[N, 2N)   sum of round(w * 2^32) over the slots routed to e
+//   part[2N, 3N)  sum over tokens of round(softmax(scores)_e * 2^32)
+//   part[3N]      tokens
+// ---------------------------------------------------------------------------
+constexpr double kFixScale = 4294967296.0;
+
+// part must be zero at launch.  One warp per token; per-block sums in shared
+// memory (integer atomics), then one global integer atomic per nonzero entry.
+__global__ void __launch_bounds__(256) aux_partials_kernel(const float *__restrict__ logits,
+                                                           const int *__restrict__ topk_idx,
+                                                           const float *__restrict__ topk_w, int T, int N, int K,
+                                                           unsigned long long *__restrict__ part) {
+    extern __shared__ unsigned long long s_fx[];   // [3N]
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    for (int i = tid; i < 3 * N; i += blockDim.x) s_fx[i] = 0ull;
+    __syncthreads();
+    for (int t = blockIdx.x * 8 + warp; t < T; t += gridDim.x * 8) {
+        const float *row = logits + (size_t)t * N;
+        float mx = -INFINITY;
+        for (int e = lane; e < N; e += 32) {
+            const float v = row[e];
+            mx = fmaxf(mx, v != v ? -INFINITY : v);
+        }
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        float z = 0.f;
+        for (int e = lane; e < N; e += 32) {
+            const float v = row[e];
+            z += (v != v || mx == -INFINITY) ? 0.f : expf(v - mx);
+        }
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+        for (int e = lane; e < N; e += 32) {
+            const float v = row[e];
+            const float pe = (v != v || mx == -INFINITY) ? 0.f : expf(v - mx) / z;
+            const unsigned long long q = __double2ull_rn((double)pe * kFixScale);
+            if (q) atomicAdd(&s_fx[2 * N + e], q);
+        }
+        for (int j = lane; j < K; j += 32) {
+            const int e = topk_idx[(size_t)t * K + j];
+            if (e < 0 || e >= N) {
+                set_status(kStatusBounds);
+                continue;
+            }
+            atomicAdd(&s_fx[e], 1ull);
+            atomicAdd(&s_fx[N + e], __double2ull_rn((double)topk_w[(size_t)t * K + j] * kFixScale));
+        }
+    }
+    __syncthreads();
+    for (int i = tid; i < 3 * N; i += blockDim.x)
+        if (s_fx[i]) atomicAdd(part + i, s_fx[i]);
+    if (blockIdx.x == 0 && tid == 0) atomicAdd(part + 3 * N, (unsigned long long)T);
+}
+
+// The statistics from summed partials (the layout above).  Shared by the device
+// kernel and the host entry point, so both give the same bits:
+//   counts_e, importance_e = fixed / 2^32, p_mean_e = fixed / 2^32 / T,
+//   f_e = counts_e / (T K); switch = N sum_e f_e P_e; simple = N sum_e f_e^2;
+//   CV^2 = population variance / mean^2 (0 when the mean is 0); sums over e in
+// ascending order, in double precision.  All zero when T = 0.
+__host__ __device__ inline void aux_finalize_partials(int N, int K, const long long *part, int *counts,
+                                                      float *importance, float *p_mean, float *scalars) {
+    const long long T = part[3 * N];
+    const double tk = (double)T * (double)K;
+    double sw = 0.0, ss = 0.0, si = 0.0, sc = 0.0;
+    for (int e = 0; e < N; ++e) {
+        const double c = (double)part[e];
+        const double im = (double)part[N + e] / kFixScale;
+        const double pm = T > 0 ? (double)part[2 * N + e] / kFixScale / (double)T : 0.0;
+        if (counts) counts[e] = (int)part[e];
+        if (importance) importance[e] = (float)im;
+        if (p_mean) p_mean[e] = (float)pm;
+        const double f = tk > 0 ? c / tk : 0.0;
+        sw += f * pm;
+        ss += f * f;
+        si += im;
+        sc += c;
+    }
+    const double mi = si / N, mc = sc / N;
+    double vi = 0.0, vc = 0.0;
+    for (int e = 0; e < N; ++e) {
+        const double im = (double)part[N + e] / kFixScale, c = (double)part[e];
+        vi += (im - mi) * (im - mi);
+        vc += (c - mc) * (c - mc);
+    }
+    vi /= N;
+    vc /= N;
+    if (scalars) {
+        scalars[0] = (float)(N * sw);
+        scalars[1] = (float)(N * ss);
+        scalars[2] = mi == 0.0 ? 0.f : (float)(vi / (mi * mi));
+        scalars[3] = mc == 0.0 ? 0.f : (float)(vc / (mc * mc));
+    }
+}
+
+__global__ void aux_finalize_kernel(int N, int K, const long long *__restrict__ part, AuxOut out) {
+    if (blockIdx.x == 0 && threadIdx.x == 0)
+        aux_finalize_partials(N, K, part, out.counts, out.importance, out.p_mean, out.scalars);
+}
+
 // W_g [D, N] -> W_g^T [N, D] (the K-major operand layout of the router GEMM).
 template <typename Tin>
 __global__ void transpose_kernel(const Tin *__restrict__ src, int R, int C, Tin *__restrict__ dst) {

@@ -378,6 +378,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             int stage = 0;
             uint32_t phase = 0;
             bool ok = true;
+            IssuedSlots iss;
             for (int kb = 0; kb < nkb; ++kb) {
                 if (!mbar_wait(&empty[stage], phase ^ 1, p.timeout_ns)) {
                     ok = false;
@@ -386,16 +387,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                 mbar_arrive_expect_tx(&full[stage], S::kStageBytes);
                 tma_load_2d(&tmX, &full[stage], sA + stage * S::kABytes, kb * BK, tile * BM);
                 tma_load_2d(&tmW, &full[stage], sB + stage * S::kBBytes, kb * BK, 0);
+                iss.note(stage, phase);
                 if (++stage == kStages) {
                     stage = 0;
                     phase ^= 1;
                 }
             }
-            if (!ok) {
-                const uint64_t t0 = globaltimer_ns();
-                while (globaltimer_ns() - t0 < 1000000ull) {
-                }
-            }
+            if (!ok) iss.drain(full, p.timeout_ns);   // copies in flight land before the CTA leaves
         }
     } else if (warp == 1) {
         if (lane == 0) {

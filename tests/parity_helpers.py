@@ -108,3 +108,28 @@ def sample_rows(T, n, gpu_idx, N, seed=0, least_loaded=2):
     for e in nonempty:
         rows |= set(np.nonzero((gpu_idx == e).any(axis=1))[0][:64].tolist())
     return np.array(sorted(rows), dtype=np.int64)
+
+
+def expert_end_rows(gpu_idx, N):
+    """For every expert with tokens, the first and the last token routed to it (the rows that
+    open and close its segment of the permuted buffers)."""
+    T, K = gpu_idx.shape
+    rows = set()
+    for e in range(N):
+        toks = np.nonzero((gpu_idx == e).any(axis=1))[0]
+        if toks.size:
+            rows |= {int(toks[0]), int(toks[-1])}
+    return np.array(sorted(rows), dtype=np.int64)
+
+
+def oracle_scores(inp, wl, rows, threads=None):
+    """fp64 router scores of the given token rows, computed on host threads."""
+    t = tag(wl.dtype)
+    rows = np.asarray(rows, dtype=np.int64)
+    xr = oracle.load_rows(host(inp["x"][torch.from_numpy(rows).to(inp["x"].device)]), t, range(len(rows)))
+    Wg, bg = host(inp["W_g"]), host(inp["b_g"])
+    nthr = threads or oracle.default_threads()
+    chunks = [c for c in np.array_split(np.arange(len(rows)), nthr) if c.size]
+    with ThreadPoolExecutor(len(chunks)) as ex:
+        parts = list(ex.map(lambda c: oracle.router_scores(xr[c], Wg, t, bg), chunks))
+    return np.concatenate(parts)

@@ -326,7 +326,7 @@ def test_gpt2_full_size_sampled_rows():
     ph.assert_y_close(y[torch.from_numpy(rows).cuda()].cpu().numpy(), ref["y"], wl.dtype)
 
 
-def _full_size_sampled(name, n_rows, seed):
+def _full_size_sampled(name, n_rows, seed, every_expert=False):
     wl = WORKLOADS[name]
     inp = make_inputs(wl, "cuda")
     layer = Layer(wl, inp)
@@ -337,6 +337,18 @@ def _full_size_sampled(name, n_rows, seed):
     np.testing.assert_array_equal(V["counts"], np.bincount(sel.ravel(), minlength=wl.N))
     check_aux(aux, V, wl.N, wl.K)
     rows = ph.sample_rows(wl.T, n_rows, V["idx"], wl.N, seed=seed, least_loaded=2)
+    if every_expert:
+        # the first and the last token routed to every live expert: their rows open and close
+        # the expert's segment, so every expert's first tile and ragged last tile are compared
+        ends = ph.expert_end_rows(V["idx"], wl.N)
+        rows = np.union1d(rows, ends)
+        live = np.nonzero(V["counts"] > 0)[0]
+        covered = np.unique(V["idx"][rows])
+        assert np.array_equal(covered, live), "a live expert has no compared output row"
+        assert len(live) > 0.9 * wl.N
+        # logits of a strided subset of 1024 rows against the oracle's fp64 scores
+        strided = np.arange(0, wl.T, max(1, wl.T // 1024))[:1024]
+        ph.assert_logits_close(V["logits"][strided], ph.oracle_scores(inp, wl, strided))
     ref = ph.oracle_rows(inp, wl, wl.K, rows, V["logits"])
     ph.assert_logits_close(V["logits"][rows], ref["scores"])
     ph.assert_weights_close(V["w"][rows], ref["w"], ref["scores"])
@@ -352,7 +364,7 @@ def test_mixtral_full_size_sampled_rows():
 
 @pytest.mark.parametrize("name", ["deepseek", "deepseek_zipf"])
 def test_deepseek_full_size_sampled_rows(name):
-    _full_size_sampled(name, 12, 4)
+    _full_size_sampled(name, 12, 4, every_expert=True)
 
 
 @pytest.mark.parametrize("name", ["decode1", "decode8", "decode64"])
@@ -391,6 +403,68 @@ def test_bf16_prefill_k1_and_k3(K):
                   zipf_s=0.5, random_bias=True)
     inp = make_inputs(wl, "cuda")
     run_full(wl, inp)
+
+
+# ----------------------------------------------------------------------------- data parallelism
+def _ws_view(ws, off, n, dt):
+    return ws[off:off + n * torch.tensor([], dtype=dt).element_size()].view(dt)
+
+
+@pytest.mark.parametrize("name,T0,T1", [("gpt2", 700, 333), ("tiny", 200, 77), ("many", 300, 129)])
+def test_data_parallel_statistics_from_two_shards(name, T0, T1):
+    """Token-sharded data parallelism emulated on one GPU: each shard's layer call leaves its
+    routing in its workspace, moe_aux_partials exports exact integer sums, their sum is
+    finalised, and the statistics equal the oracle's over the union batch.  The fixed-point
+    sums equal their definition exactly, and the device and host finalisations give the
+    same bits."""
+    if name == "many":
+        wl = Workload("many_dp", 40, T0 + T1, 256, 128, 64, 4, ACT_SWIGLU, torch.bfloat16, False, 0.05,
+                      zipf_s=0.5)
+    else:
+        wl = WORKLOADS[name]
+    inp = make_inputs(wl, "cuda", T=T0 + T1)
+    layer = Layer(wl, inp)
+    N, K = wl.N, wl.K
+    parts, routed = [], []
+    for a, b in ((0, T0), (T0, T0 + T1)):
+        T = b - a
+        x = inp["x"][a:b].contiguous()
+        y, ws, _ = layer.forward(x=x, with_aux=False)
+        L = moe.moe_get_workspace_layout(layer.cfg, T)
+        lg = _ws_view(ws, L.logits, T * N, torch.float32)
+        idx = _ws_view(ws, L.topk_idx, T * K, torch.int32)
+        w = _ws_view(ws, L.topk_w, T * K, torch.float32)
+        part = torch.full((moe.aux_partials_len(N),), -7, dtype=torch.int64, device="cuda")
+        moe.check(moe.moe_aux_partials(layer.cfg, T, lg, idx, w, part), "partials")
+        torch.cuda.synchronize()
+        assert moe.moe_get_device_status() == 0
+        parts.append(part)
+        routed.append((lg.view(T, N).cpu().numpy(), idx.view(T, K).cpu().numpy(), w.view(T, K).cpu().numpy()))
+    lg = np.concatenate([r[0] for r in routed])
+    sel = np.concatenate([r[1] for r in routed])
+    w = np.concatenate([r[2] for r in routed])
+    total = parts[0] + parts[1]          # the all-reduce of two ranks
+    p = total.cpu().numpy()
+    fixed = np.rint(w.astype(np.float64) * 4294967296.0).astype(np.int64)
+    np.testing.assert_array_equal(p[:N], np.bincount(sel.ravel(), minlength=N))
+    np.testing.assert_array_equal(p[N:2 * N], np.array([fixed[sel == e].sum() for e in range(N)]))
+    assert p[3 * N] == T0 + T1
+    out = dict(counts=torch.full((N,), -1, dtype=torch.int32, device="cuda"),
+               importance=torch.full((N,), -1.0, device="cuda"), p_mean=torch.full((N,), -1.0, device="cuda"),
+               scalars=torch.full((4,), -1.0, device="cuda"))
+    moe.check(moe.moe_aux_finalize(layer.cfg, total, moe.make_aux(**out)), "finalize")
+    torch.cuda.synchronize()
+    host = dict(counts=torch.empty(N, dtype=torch.int32), importance=torch.empty(N), p_mean=torch.empty(N),
+                scalars=torch.empty(4))
+    moe.check(moe.moe_aux_finalize_host(layer.cfg, total.cpu(), **host), "finalize host")
+    for k in out:
+        assert torch.equal(out[k].cpu(), host[k]), k
+    st = oracle.aux_stats(lg.astype(np.float64), sel, w.astype(np.float64), N)
+    np.testing.assert_array_equal(out["counts"].cpu().numpy(), st["counts"].astype(np.int32))
+    np.testing.assert_allclose(out["importance"].cpu().numpy(), st["importance"], rtol=1e-6, atol=1e-6)
+    np.testing.assert_allclose(out["p_mean"].cpu().numpy(), st["p_mean"], rtol=1e-5, atol=1e-7)
+    np.testing.assert_allclose(out["scalars"].cpu().numpy(),
+                               [st["switch"], st["simple"], st["cv2_importance"], st["cv2_load"]], rtol=1e-4, atol=1e-6)
 
 
 # ----------------------------------------------------------------------------- entry points, determinism
