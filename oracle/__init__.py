@@ -62,7 +62,8 @@ class _Layer(ctypes.Structure):
                 ("act", ctypes.c_int32), ("dtype", ctypes.c_int32),
                 ("x", ctypes.c_void_p), ("Wg", ctypes.c_void_p), ("bg", ctypes.c_void_p),
                 ("W1", ctypes.c_void_p), ("b1", ctypes.c_void_p),
-                ("W2", ctypes.c_void_p), ("b2", ctypes.c_void_p)]
+                ("W2", ctypes.c_void_p), ("b2", ctypes.c_void_p), ("bsel", ctypes.c_void_p),
+                ("S1", ctypes.c_void_p), ("sb1", ctypes.c_void_p), ("S2", ctypes.c_void_p), ("sb2", ctypes.c_void_p)]
 
 
 def configure(L):
@@ -83,6 +84,7 @@ def configure(L):
     L.orc_expert_gelu.argtypes = [i64, i64, vp, vp, vp, vp, vp, i32, vp, vp]
     L.orc_expert_swiglu.argtypes = [i64, i64, vp, vp, vp, i32, vp, vp]
     L.orc_combine.argtypes = [i64, i64, vp, vp, vp]
+    L.orc_add_shared.argtypes = [i64, vp, vp]
     L.orc_moe_layer_rows.argtypes = [ctypes.POINTER(_Layer), i64, i64, vp, vp, vp, vp, vp]
     L.orc_cv_squared.restype = dp
     L.orc_cv_squared.argtypes = [i64, vp]
@@ -229,13 +231,24 @@ def combine(w, E) -> np.ndarray:
     return y
 
 
+def add_shared(y, s) -> np.ndarray:
+    """y + s (the shared expert's output added after the routed sum), one token."""
+    yv = np.array(_c(y, np.float64))
+    sv = _c(s, np.float64)
+    lib().orc_add_shared(yv.shape[0], _p(sv), _p(yv))
+    return yv
+
+
 def moe_layer(x, Wg, W1, W2, *, K, act, dtype_tag, bg=None, b1=None, b2=None, sel_scores=None,
-              threads=None, rows=None):
+              threads=None, rows=None, bsel=None, S1=None, S2=None, sb1=None, sb2=None):
     """The whole layer on host arrays, in fp64.
 
     x [T, D]; Wg [D, N]; W1 [N, H, D] (GELU) or [N, 2H, D] (SwiGLU); W2 [N, D, H].
+    bsel [N] float32 (optional): selection-only bias (changes the kept set, not the weights).
+    S1 [H or 2H, D], S2 [D, H], sb1 [H], sb2 [D] (optional): the shared expert.
     sel_scores [T, N] float32 (optional): make the expert selection on these scores
-    (the device's fp32 logits) while the gate weights use the fp64 scores.
+    (the device's fp32 logits, plus any selection bias in fp32) while the gate
+    weights use the fp64 scores.
     rows: optional (t0, t1) range; other rows of the outputs are left as zeros.
     Returns dict(scores [T,N], sel [T,K], w [T,K], y [T,D]) in fp64 / int32.
     """
@@ -248,7 +261,10 @@ def moe_layer(x, Wg, W1, W2, *, K, act, dtype_tag, bg=None, b1=None, b2=None, se
     W1m = _mat(W1, dtype_tag)
     bgm, b1m, b2m = _c(bg, np.float32), _c(b1, np.float32), _c(b2, np.float32)
     ss = _c(sel_scores, np.float32)
-    lay = _Layer(D, H, N, K, act, dtype_tag, _p(xm), _p(Wgm), _p(bgm), _p(W1m), _p(b1m), _p(W2m), _p(b2m))
+    bselm, S1m, S2m = _c(bsel, np.float32), _mat(S1, dtype_tag), _mat(S2, dtype_tag)
+    sb1m, sb2m = _c(sb1, np.float32), _c(sb2, np.float32)
+    lay = _Layer(D, H, N, K, act, dtype_tag, _p(xm), _p(Wgm), _p(bgm), _p(W1m), _p(b1m), _p(W2m), _p(b2m),
+                 _p(bselm), _p(S1m), _p(sb1m), _p(S2m), _p(sb2m))
     scores = np.zeros((T, N), dtype=np.float64)
     sel = np.zeros((T, K), dtype=np.int32)
     w = np.zeros((T, K), dtype=np.float64)

@@ -224,6 +224,11 @@ typedef struct {
     const float *b1;  /* [N, H] or NULL (GELU only) */
     const void *W2;   /* [N, D, H] */
     const float *b2;  /* [N, D] or NULL (GELU only) */
+    const float *bsel; /* [N] or NULL: selection-only bias (see orc_moe_layer_rows) */
+    const void *S1;   /* shared expert or NULL: GELU [H, D] ; SwiGLU [2H, D] */
+    const float *sb1; /* [H] or NULL (GELU only) */
+    const void *S2;   /* shared expert [D, H] */
+    const float *sb2; /* [D] or NULL (GELU only) */
 } orc_layer;
 
 /* Byte size of one element of the layer's dtype. */
@@ -245,13 +250,39 @@ void orc_expert(const orc_layer *L, int64_t e, const double *x_row, double *hid,
 }
 
 /* ------------------------------------------------------------------------
+ * Shared expert.  "MoE(Mixture of Experts)", design notes (merits and
+ * examples): the fine-grained MoE of DeepSeek-V3 adds to the many small routed
+ * experts a shared part that every token passes through.  Read here as one
+ * FFN of the same form and sizes as a routed expert (GELU or SwiGLU), not
+ * gated: its output is added with weight 1 after the routed experts' sum.
+ * ---------------------------------------------------------------------- */
+void orc_shared_expert(const orc_layer *L, const double *x_row, double *hid, double *out) {
+    if (L->act == ORC_ACT_GELU)
+        orc_expert_gelu(L->D, L->H, x_row, L->S1, L->sb1, L->S2, L->sb2, L->dtype, hid, out);
+    else
+        orc_expert_swiglu(L->D, L->H, x_row, L->S1, L->S2, L->dtype, hid, out);
+}
+
+/* y = y + s, element by element. */
+void orc_add_shared(int64_t D, const double *s, double *y) {
+    for (int64_t c = 0; c < D; ++c) y[c] = y[c] + s[c];
+}
+
+/* ------------------------------------------------------------------------
  * The whole layer for tokens t0..t1-1 ("MoE(Mixture of Experts)" section (2),
  * Forward: route each row, evaluate only the selected experts, mix in order).
+ *   bsel (optional, in the layer): a per-expert bias that changes which
+ *       experts are kept and nothing else -- the auxiliary-loss-free load
+ *       balancing of DeepSeek-V3 named in the chapter's design notes (a bias
+ *       adjusted during training).  Read here as: KeepTopK is taken on
+ *       s_e + bsel_e, and the gate weights are softmax(KeepTopK) of the raw
+ *       scores s over that kept set; the statistics use the raw scores.
+ *   S1/S2 (optional): the shared expert, added after the routed sum.
  *   scores_out [T, N]: fp64 router scores.
  *   sel_scores [T, N] (optional): if given, the expert selection is made on
- *       these scores instead of the fp64 ones (used to apply the oracle's sort
- *       to the device's fp32 logits); the gate weights always use the fp64
- *       scores.
+ *       these scores instead of the fp64 s + bsel (used to apply the oracle's
+ *       ranking to the device's fp32 logits, with any selection bias already
+ *       added in fp32); the gate weights always use the fp64 scores.
  *   sel_out [T, K], w_out [T, K], y_out [T, D].
  * Rows outside [t0, t1) are not touched, so disjoint ranges may run on
  * separate threads.
@@ -264,6 +295,7 @@ void orc_moe_layer_rows(const orc_layer *L, int64_t t0, int64_t t1,
     double *hid = (double *)malloc(sizeof(double) * (size_t)H);
     double *E = (double *)malloc(sizeof(double) * (size_t)(K * D));
     double *tmp = (double *)malloc(sizeof(double) * (size_t)N);
+    double *sh = (double *)malloc(sizeof(double) * (size_t)D);
     for (int64_t t = t0; t < t1; ++t) {
         double *s = scores_out + t * N;
         int32_t *sel = sel_out + t * K;
@@ -272,18 +304,23 @@ void orc_moe_layer_rows(const orc_layer *L, int64_t t0, int64_t t1,
         orc_router_scores(D, N, x_row, L->Wg, L->dtype, L->bg, s);
         if (sel_scores) {
             for (int64_t e = 0; e < N; ++e) tmp[e] = (double)sel_scores[t * N + e];
-            orc_select_topk(N, K, tmp, sel);
         } else {
-            orc_select_topk(N, K, s, sel);
+            for (int64_t e = 0; e < N; ++e) tmp[e] = s[e] + (L->bsel ? (double)L->bsel[e] : 0.0);
         }
+        orc_select_topk(N, K, tmp, sel);
         orc_gate_weights(N, K, s, sel, w);
         for (int64_t j = 0; j < K; ++j) orc_expert(L, sel[j], x_row, hid, E + j * D);
         orc_combine(K, D, w, E, y_out + t * D);
+        if (L->S1) {
+            orc_shared_expert(L, x_row, hid, sh);
+            orc_add_shared(D, sh, y_out + t * D);
+        }
     }
     free(x_row);
     free(hid);
     free(E);
     free(tmp);
+    free(sh);
 }
 
 /* ------------------------------------------------------------------------

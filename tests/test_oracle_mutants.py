@@ -63,6 +63,17 @@ MUTANTS = [
      [pins.test_cv_squared_closed_forms]),
     ("importance_counts_tokens", "importance[sel[t * K + j]] += w[t * K + j];", "importance[sel[t * K + j]] += 1.0;",
      [pins.test_aux_stats_invariants_and_library_checks]),
+    ("shared_expert_dropped", "            orc_add_shared(D, sh, y_out + t * D);", "            (void)sh;",
+     [pins.test_one_expert_with_shared_expert_is_two_dense_ffns,
+      pins.test_shared_expert_alone_when_routed_experts_are_zero]),
+    ("shared_expert_replaces_routed", "for (int64_t c = 0; c < D; ++c) y[c] = y[c] + s[c];",
+     "for (int64_t c = 0; c < D; ++c) y[c] = s[c];",
+     [pins.test_one_expert_with_shared_expert_is_two_dense_ffns]),
+    ("selection_bias_ignored", "tmp[e] = s[e] + (L->bsel ? (double)L->bsel[e] : 0.0);", "tmp[e] = s[e];",
+     [pins.test_selection_bias_changes_the_kept_set_not_the_weights]),
+    ("selection_bias_in_weights", "        orc_gate_weights(N, K, s, sel, w);\n        for (int64_t j = 0; j < K; ++j) orc_expert",
+     "        orc_gate_weights(N, K, tmp, sel, w);\n        for (int64_t j = 0; j < K; ++j) orc_expert",
+     [pins.test_selection_bias_changes_the_kept_set_not_the_weights]),
     ("p_mean_not_averaged", "for (int64_t e = 0; e < N; ++e) p_mean[e] /= (double)T;",
      "for (int64_t e = 0; e < N; ++e) p_mean[e] /= 1.0;",
      [pins.test_aux_stats_invariants_and_library_checks]),

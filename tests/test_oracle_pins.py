@@ -251,6 +251,70 @@ def test_layer_rows_threads_are_independent():
         np.testing.assert_array_equal(a[k], b[k])
 
 
+# --------------------------------------------------------------------------- shared expert, selection bias
+@pytest.mark.parametrize("act,bias", [(oracle.ACT_GELU, True), (oracle.ACT_SWIGLU, False)])
+def test_one_expert_with_shared_expert_is_two_dense_ffns(act, bias):
+    """A 1-expert top-1 layer with a shared expert equals the sum of two dense FFNs
+    (library fp64 linear + activation)."""
+    rng = np.random.default_rng(51 + act)
+    T, D, H = 20, 16, 24
+    x, Wg, W1, W2, b1, b2 = _rand_layer(rng, T, D, H, 1, act, bias)
+    _, _, S1, S2, sb1, sb2 = _rand_layer(rng, 1, D, H, 1, act, bias)
+    out = oracle.moe_layer(x, Wg, W1, W2, K=1, act=act, dtype_tag=oracle.F32, b1=b1, b2=b2, threads=2,
+                           S1=S1[0], S2=S2[0], sb1=None if sb1 is None else sb1[0],
+                           sb2=None if sb2 is None else sb2[0])
+    x64 = torch.from_numpy(x.astype(np.float64))
+    ref = _torch_expert(x64, act, W1[0], W2[0], None if b1 is None else b1[0], None if b2 is None else b2[0], H)
+    ref = ref + _torch_expert(x64, act, S1[0], S2[0], None if sb1 is None else sb1[0],
+                              None if sb2 is None else sb2[0], H)
+    np.testing.assert_allclose(out["y"], ref.numpy(), rtol=1e-12, atol=1e-13)
+
+
+def test_shared_expert_alone_when_routed_experts_are_zero():
+    """Routed experts with all-zero weights contribute nothing: y is the shared FFN alone."""
+    rng = np.random.default_rng(57)
+    T, D, H, N = 12, 8, 16, 4
+    x, Wg, W1, W2, b1, b2 = _rand_layer(rng, T, D, H, N, oracle.ACT_SWIGLU, False)
+    _, _, S1, S2, _, _ = _rand_layer(rng, 1, D, H, 1, oracle.ACT_SWIGLU, False)
+    out = oracle.moe_layer(x, Wg, np.zeros_like(W1), np.zeros_like(W2), K=2, act=oracle.ACT_SWIGLU,
+                           dtype_tag=oracle.F32, S1=S1[0], S2=S2[0], threads=1)
+    ref = _torch_expert(torch.from_numpy(x.astype(np.float64)), oracle.ACT_SWIGLU, S1[0], S2[0], None, None, H)
+    np.testing.assert_allclose(out["y"], ref.numpy(), rtol=1e-12, atol=1e-14)
+
+
+def test_zero_selection_bias_is_the_plain_layer():
+    rng = np.random.default_rng(61)
+    x, Wg, W1, W2, b1, b2 = _rand_layer(rng, 30, 8, 16, 6, oracle.ACT_GELU, True)
+    a = oracle.moe_layer(x, Wg, W1, W2, K=2, act=oracle.ACT_GELU, dtype_tag=oracle.F32, b1=b1, b2=b2, threads=1)
+    b = oracle.moe_layer(x, Wg, W1, W2, K=2, act=oracle.ACT_GELU, dtype_tag=oracle.F32, b1=b1, b2=b2, threads=1,
+                         bsel=np.zeros(6, np.float32))
+    for k in ("scores", "sel", "w", "y"):
+        np.testing.assert_array_equal(a[k], b[k])
+
+
+def test_selection_bias_changes_the_kept_set_not_the_weights():
+    """A selection bias picks the kept set by s + b; the weights are the masked softmax of the raw
+    scores over that set (library masked softmax), and the scores themselves are unchanged."""
+    rng = np.random.default_rng(63)
+    T, D, H, N, K = 40, 8, 16, 6, 3
+    x, Wg, W1, W2, b1, b2 = _rand_layer(rng, T, D, H, N, oracle.ACT_SWIGLU, False)
+    bsel = np.array([0.0, 3.0, -1.0, 0.5, 9.0, -9.0], np.float32)
+    out = oracle.moe_layer(x, Wg, W1, W2, K=K, act=oracle.ACT_SWIGLU, dtype_tag=oracle.F32, bsel=bsel, threads=2)
+    logits = torch.from_numpy(x.astype(np.float64)) @ torch.from_numpy(Wg.astype(np.float64))
+    np.testing.assert_allclose(out["scores"], logits.numpy(), rtol=1e-13, atol=1e-13)
+    biased = logits + torch.from_numpy(bsel.astype(np.float64))
+    order = torch.sort(-biased, dim=1, stable=True).indices[:, :K]
+    assert out["sel"].tolist() == order.numpy().tolist()
+    assert np.all(out["sel"][:, 0] == 4)             # the +9 bias always wins the first slot
+    assert not np.any(out["sel"] == 5)               # the -9 bias never gets in
+    masked = torch.full_like(logits, -math.inf)
+    masked.scatter_(1, order, logits.gather(1, order))   # raw scores on the kept set
+    G = torch.softmax(masked, dim=1)
+    np.testing.assert_allclose(out["w"], G.gather(1, order).numpy(), rtol=1e-13, atol=1e-15)
+    # the weight of the forced expert follows its raw score, not its bias
+    assert np.any(out["w"][:, 0] < 0.5)
+
+
 # --------------------------------------------------------------------------- statistics
 def test_balance_loss_extremes(golden_dir):
     g = _golden(golden_dir, "balance_loss_extremes.json")
