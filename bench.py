@@ -463,8 +463,9 @@ def main():
 
     T = wl.T
     inp = make_inputs(wl, dev, seed=rank_seed(wl, rank))
-    cfg = moe.make_config(wl.D, wl.H, wl.N, wl.K, wl.act, moe.dtype_code(wl.dtype), wl.has_bias)
-    W = moe.make_weights(inp["W_g"], inp["W1"], inp["W2"], inp["b_g"], inp["b1"], inp["b2"])
+    cfg = moe.make_config(wl.D, wl.H, wl.N, wl.K, wl.act, moe.dtype_code(wl.dtype), wl.has_bias, wl.n_shared)
+    W = moe.make_weights(inp["W_g"], inp["W1"], inp["W2"], inp["b_g"], inp["b1"], inp["b2"], inp["b_sel"],
+                         inp["S1"], inp["sb1"], inp["S2"], inp["sb2"])
     ws = moe.alloc_workspace(cfg, T)
     y = torch.empty(T, wl.D, dtype=torch.float32, device=dev)
 

@@ -84,6 +84,12 @@ typedef struct {
     int32_t act;      /* MOE_ACT_GELU or MOE_ACT_SWIGLU */
     int32_t dtype;    /* MOE_F32 or MOE_BF16 */
     int32_t has_bias; /* GELU only: expert biases b1, b2 are given */
+    int32_t n_shared; /* 0 or 1: a shared expert every token passes through
+                         ("MoE(Mixture of Experts)", design notes: DeepSeek-V3's
+                         fine-grained experts plus a shared part).  It has the
+                         routed experts' form and sizes (GELU with the same
+                         has_bias, or SwiGLU) and is added with weight 1 after
+                         the routed experts' slot-order sum. */
 } moe_config;
 
 /* Layer parameters, all device memory.
@@ -93,7 +99,20 @@ typedef struct {
  *      [N, 2H, D] dtype  SwiGLU: packed gate_up (rows 0..H-1 gate, H..2H-1 up)
  *  b1  [N, H] fp32       GELU with has_bias, else NULL
  *  W2  [N, D, H] dtype   second linear / down projection, out x in
- *  b2  [N, D] fp32       GELU with has_bias, else NULL */
+ *  b2  [N, D] fp32       GELU with has_bias, else NULL
+ *  b_sel [N] fp32 or NULL  selection-only bias: added (in fp32) to the scores
+ *                        for choosing the K experts and for nothing else; the
+ *                        gate weights stay the softmax over the kept experts'
+ *                        raw scores and the statistics use the raw scores.
+ *                        This is the auxiliary-loss-free load balancing of
+ *                        DeepSeek-V3 named in "MoE(Mixture of Experts)",
+ *                        design notes (the bias itself is adjusted in
+ *                        training; here it is an input).
+ *  S1  [H, D] / [2H, D] dtype  shared expert's first linear or packed gate_up
+ *  sb1 [H] fp32          shared expert bias (GELU with has_bias), else NULL
+ *  S2  [D, H] dtype      shared expert's second linear
+ *  sb2 [D] fp32          shared expert bias (GELU with has_bias), else NULL
+ *  S1, S2 are required when n_shared == 1 and ignored otherwise. */
 typedef struct {
     const void *W_g;
     const float *b_g;
@@ -101,6 +120,11 @@ typedef struct {
     const float *b1;
     const void *W2;
     const float *b2;
+    const float *b_sel;
+    const void *S1;
+    const float *sb1;
+    const void *S2;
+    const float *sb2;
 } moe_weights;
 
 /* Per-batch statistics, device memory (any pointer may be NULL to skip it).
@@ -153,6 +177,9 @@ int moe_route(const moe_config *cfg, const void *x, int64_t T, const moe_weights
  *      with at most two terms on +0 this gives the same bits as the slot-order
  *      sum.
  *  aux: optional statistics (see moe_aux), or NULL.
+ * With a shared expert (n_shared == 1) its output is added after the routed
+ * sum, y[t] = sum_j w_j E_j(x_t) + S(x_t), and the down projection never adds
+ * into y directly.
  * The routing results and intermediates stay in the workspace; their places
  * are given by moe_workspace_layout().  T == 0 is a no-op (aux zeroed). */
 int moe_forward(const moe_config *cfg, const void *x, int64_t T, const moe_weights *w,
@@ -264,8 +291,9 @@ typedef struct {
 int moe_get_workspace_layout(const moe_config *cfg, int64_t T, moe_workspace_layout *out);
 
 /* Parameter accounting ("MoE(Mixture of Experts)", section (1)): router D*N
- * plus all N experts (total) or the K active ones; an expert holds 2*D*H
- * weights (GELU, + H + D with biases) or 3*D*H (SwiGLU).  -1 if invalid. */
+ * plus all N experts (total) or the K active ones, plus the shared expert
+ * (n_shared) in both; an expert holds 2*D*H weights (GELU, + H + D with
+ * biases) or 3*D*H (SwiGLU).  -1 if invalid. */
 int64_t moe_total_params(const moe_config *cfg);
 int64_t moe_active_params(const moe_config *cfg);
 

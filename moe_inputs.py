@@ -12,7 +12,14 @@ Recipe (same for every workload):
     ``random_bias`` is set (then N(0, 0.02));
   * bf16 tensors are drawn in fp32 and rounded to bf16 (round to nearest even);
   * the skewed workloads add a per-expert router bias b_g[e] = -s ln(e + 1)
-    (Zipf-like, s = 1), so expert 0 is the most loaded.
+    (Zipf-like, s = 1), so expert 0 is the most loaded;
+  * a shared expert (when the workload has one) is drawn last, after all of
+    the above: S1 (H or 2H rows) then S2, N(0, w_std), then its biases like
+    the experts' (GELU with biases);
+  * a selection-only bias (when the workload has one) is b_sel[e] =
+    sel_s ln(e + 1): with sel_s = s it cancels the Zipf skew for the choice of
+    experts (the balanced state DeepSeek-V3's bias adjustment aims at) while
+    the gate weights keep the skewed scores.
 
 Layouts: x [T, D]; W_g [D, N]; W1 [N, H, D] or W_gu [N, 2H, D] (gate rows first,
 then up rows); W2 / W_down [N, D, H]; b_g [N], b1 [N, H], b2 [N, D] in fp32.
@@ -42,6 +49,8 @@ class Workload:
     w_std: float
     zipf_s: float = 0.0   # router bias strength; 0 = no router bias
     random_bias: bool = False
+    n_shared: int = 0     # 1: a shared expert every token passes through
+    sel_s: float = 0.0    # selection-only bias strength; 0 = none
 
     @property
     def seed(self) -> int:
@@ -63,6 +72,9 @@ WORKLOADS = {
     # same, Zipf-skewed router
     "deepseek_zipf": Workload("deepseek_zipf", 4, 16384, 7168, 2048, 256, 8, ACT_SWIGLU, torch.bfloat16,
                               False, 0.006, 1.0),
+    # DeepSeek-V3 shape with its shared expert and a selection-only bias that cancels the Zipf skew
+    "deepseek_shared": Workload("deepseek_shared", 6, 16384, 7168, 2048, 256, 8, ACT_SWIGLU, torch.bfloat16,
+                                False, 0.006, 1.0, n_shared=1, sel_s=1.0),
     # gpt-oss-20b decode shape (T = 1, 8 or 64)
     "decode1": Workload("decode1", 5, 1, 2880, 2880, 32, 4, ACT_SWIGLU, torch.bfloat16, False, 0.02),
     "decode8": Workload("decode8", 5, 8, 2880, 2880, 32, 4, ACT_SWIGLU, torch.bfloat16, False, 0.02),
@@ -110,6 +122,19 @@ def make_inputs(wl: Workload, device="cpu", T: int | None = None, seed: int | No
                                   device=device)
     else:
         out["b_g"] = None
+    out["S1"] = out["S2"] = out["sb1"] = out["sb2"] = None
+    if wl.n_shared:
+        out["S1"] = _randn((rows1, D), g, device, wl.w_std).to(wl.dtype)
+        out["S2"] = _randn((D, H), g, device, wl.w_std).to(wl.dtype)
+        if wl.has_bias:
+            if wl.random_bias:
+                out["sb1"] = _randn((H,), g, device, 0.02)
+                out["sb2"] = _randn((D,), g, device, 0.02)
+            else:
+                out["sb1"] = torch.zeros((H,), dtype=torch.float32, device=device)
+                out["sb2"] = torch.zeros((D,), dtype=torch.float32, device=device)
+    out["b_sel"] = (torch.tensor([wl.sel_s * math.log(e + 1) for e in range(N)], dtype=torch.float32, device=device)
+                    if wl.sel_s else None)
     return out
 
 

@@ -44,12 +44,14 @@ EXPORTED = ("moe_workspace_size", "moe_route", "moe_forward", "moe_forward_timed
 class moe_config(ctypes.Structure):
     _fields_ = [("DModel", ctypes.c_int32), ("DHidden", ctypes.c_int32), ("NExperts", ctypes.c_int32),
                 ("TopK", ctypes.c_int32), ("act", ctypes.c_int32), ("dtype", ctypes.c_int32),
-                ("has_bias", ctypes.c_int32)]
+                ("has_bias", ctypes.c_int32), ("n_shared", ctypes.c_int32)]
 
 
 class moe_weights(ctypes.Structure):
     _fields_ = [("W_g", ctypes.c_void_p), ("b_g", ctypes.c_void_p), ("W1", ctypes.c_void_p),
-                ("b1", ctypes.c_void_p), ("W2", ctypes.c_void_p), ("b2", ctypes.c_void_p)]
+                ("b1", ctypes.c_void_p), ("W2", ctypes.c_void_p), ("b2", ctypes.c_void_p),
+                ("b_sel", ctypes.c_void_p), ("S1", ctypes.c_void_p), ("sb1", ctypes.c_void_p),
+                ("S2", ctypes.c_void_p), ("sb2", ctypes.c_void_p)]
 
 
 class moe_aux(ctypes.Structure):
@@ -147,12 +149,15 @@ def dtype_code(dt: torch.dtype) -> int:
     raise ValueError(f"unsupported dtype {dt}")
 
 
-def make_config(DModel, DHidden, NExperts, TopK, act=MOE_ACT_GELU, dtype=MOE_BF16, has_bias=False) -> moe_config:
-    return moe_config(DModel, DHidden, NExperts, TopK, act, dtype, int(bool(has_bias)))
+def make_config(DModel, DHidden, NExperts, TopK, act=MOE_ACT_GELU, dtype=MOE_BF16, has_bias=False,
+                n_shared=0) -> moe_config:
+    return moe_config(DModel, DHidden, NExperts, TopK, act, dtype, int(bool(has_bias)), int(n_shared))
 
 
-def make_weights(W_g, W1, W2, b_g=None, b1=None, b2=None) -> moe_weights:
-    return moe_weights(_ptr(W_g), _ptr(b_g), _ptr(W1), _ptr(b1), _ptr(W2), _ptr(b2))
+def make_weights(W_g, W1, W2, b_g=None, b1=None, b2=None, b_sel=None, S1=None, sb1=None, S2=None,
+                 sb2=None) -> moe_weights:
+    return moe_weights(_ptr(W_g), _ptr(b_g), _ptr(W1), _ptr(b1), _ptr(W2), _ptr(b2), _ptr(b_sel), _ptr(S1),
+                       _ptr(sb1), _ptr(S2), _ptr(sb2))
 
 
 def make_aux(counts=None, importance=None, p_mean=None, scalars=None) -> moe_aux:

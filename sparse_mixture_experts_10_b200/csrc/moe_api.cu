@@ -65,15 +65,18 @@ struct Plan {
     int nt;       // decode: padded token tile (16, 32 or 64)
     int route_splits;  // few-token router: W_g slabs per token
     int dec_cap;       // decode GEMMs: CTAs the stream-K partials and tickets are sized for
+    int n_shared;      // 1: a shared expert (dense FFN over every token) is added after the routed sum
     // Counters region (zeroed on every call), 32-bit words: [0] router ticket,
     // [1] statistics ticket, [2] number of live experts, [64, 128) per-token
     // tickets of the few-token router; from byte 512 the stream-K tile tickets
-    // of the decode up- and then down-projection (dec_cap each); then the
-    // routers' per-expert probability and gate-weight sums (u64, N each).
+    // of the decode up- and down-projections and of the shared expert's two
+    // decode GEMMs (dec_cap each); then the routers' per-expert probability and
+    // gate-weight sums (u64, N each).
     size_t counters_bytes;
     size_t stat_sums;  // offset inside the counters region of the routers' fixed-point sums [2][N] (u64)
     size_t counters, logits, idx, w, counts, offsets, row_offsets, live, chunk_counts, chunk_base,
-        perm_slot, slot_row, x_perm, h, z, wgt, aux_p, aux_i, aux_c, route_part, dec_part, total;
+        perm_slot, slot_row, x_perm, h, z, wgt, aux_p, aux_i, aux_c, route_part, dec_part, shared_tbl, h_s, s_out,
+        total;
 };
 
 int make_plan(const moe_config *c, int64_t T, Plan *p) {
@@ -84,6 +87,7 @@ int make_plan(const moe_config *c, int64_t T, Plan *p) {
     if (c->act != MOE_ACT_GELU && c->act != MOE_ACT_SWIGLU) return MOE_ERR_INVALID_ARG;
     if (c->dtype != MOE_F32 && c->dtype != MOE_BF16) return MOE_ERR_INVALID_ARG;
     if (c->has_bias && c->act != MOE_ACT_GELU) return MOE_ERR_UNSUPPORTED;
+    if (c->n_shared != 0 && c->n_shared != 1) return MOE_ERR_INVALID_ARG;
     const int es = c->dtype == MOE_F32 ? 4 : 2;
     const int vec = 16 / es;
     if (D % vec || H % vec) return MOE_ERR_INVALID_ARG;
@@ -94,6 +98,7 @@ int make_plan(const moe_config *c, int64_t T, Plan *p) {
     p->T = T;
     p->D = (int)D; p->H = (int)H; p->N = (int)N; p->K = (int)K;
     p->act = c->act; p->dtype = c->dtype; p->has_bias = c->has_bias ? 1 : 0; p->es = es;
+    p->n_shared = c->n_shared;
     p->np = N <= 8 ? 8 : N <= 16 ? 16 : 32;
     const bool fits = N <= 32 && (size_t)p->np * D * es + 256 <= kSmallRouterSmemMax;
     p->rowdot_router = N <= 32 && (T < kRowdotMaxT || !fits);
@@ -123,7 +128,7 @@ int make_plan(const moe_config *c, int64_t T, Plan *p) {
     };
     p->route_splits = p->few_router ? (int)std::min<int64_t>(rtc::kFewMaxSplits, std::max<int64_t>(1, cdiv(D, 256))) : 1;
     p->dec_cap = p->decode ? kDecodeMaxGrid : 0;
-    p->stat_sums = (512 + (size_t)2 * p->dec_cap * 4 + 7) / 8 * 8;
+    p->stat_sums = (512 + (size_t)4 * p->dec_cap * 4 + 7) / 8 * 8;
     p->counters_bytes = align256(p->stat_sums + (size_t)2 * N * 8);
     p->counters = take(p->counters_bytes);
     p->logits = take((size_t)T * N * 4);
@@ -150,6 +155,11 @@ int make_plan(const moe_config *c, int64_t T, Plan *p) {
     p->aux_c = take((size_t)p->aux_blocks * N * 4);
     p->route_part = take(p->few_router ? (size_t)T * p->route_splits * 32 * 4 : 0);
     p->dec_part = take(p->decode ? (size_t)p->dec_cap * 2 * dec::BM * p->nt * 4 : 0);
+    // shared expert: its one-group dispatch table for the decode GEMMs (live = {0},
+    // one live group, count T, first row 0), its hidden rows and its fp32 output
+    p->shared_tbl = take(16);
+    p->h_s = take(p->n_shared ? (size_t)std::max<int64_t>(T, 1) * H * es : 0);
+    p->s_out = take(p->n_shared ? (size_t)T * D * 4 : 0);
     p->total = off;
     return MOE_OK;
 }
@@ -267,12 +277,13 @@ int launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cud
     return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
-// Zeroes `bytes` (a multiple of 16) at the 16-byte aligned p.
-int launch_zero(void *p, size_t bytes, int sms, cudaStream_t s) {
+// Zeroes `bytes` (a multiple of 16) at the 16-byte aligned p; with tbl, also
+// writes the shared expert's one-group table {0, 1, T, 0} there.
+int launch_zero(void *p, size_t bytes, int sms, cudaStream_t s, int *tbl = nullptr, int tbl_T = 0) {
     const int64_t n16 = (int64_t)(bytes / 16);
-    if (n16 == 0) return MOE_OK;
-    const int grid = (int)std::min<int64_t>(cdiv(n16, 256), (int64_t)sms * 8);
-    return launch_pdl(zero_kernel, dim3(grid), dim3(256), 0, s, static_cast<uint4 *>(p), n16);
+    if (n16 == 0 && !tbl) return MOE_OK;
+    const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(cdiv(n16, 256), (int64_t)sms * 8));
+    return launch_pdl(zero_kernel, dim3(grid), dim3(256), 0, s, static_cast<uint4 *>(p), n16, tbl, tbl_T);
 }
 
 
@@ -393,6 +404,7 @@ int stage_route_tc(const Plan &P, const Bufs &b, const void *x, const moe_weight
     p.K = P.K;
     p.np = P.rnp;
     p.bg = w->b_g;
+    p.bsel = w->b_sel;
     p.logits = logits;
     p.topk_idx = idx;
     p.topk_w = tw;
@@ -462,20 +474,20 @@ int stage_route(const Plan &P, const Bufs &b, const void *x, const moe_weights *
         if (cudaMemsetAsync(cc, 0, (size_t)P.n_chunks * N * 4, s) != cudaSuccess) return MOE_ERR_CUDA;
         if (P.dtype == MOE_F32)
             router_rowdot_kernel<float><<<T, 1024, 0, s>>>(static_cast<const float *>(x), T, D, N, K,
-                                                           static_cast<const float *>(w->W_g), w->b_g, logits, idx,
-                                                           tw, cc);
+                                                           static_cast<const float *>(w->W_g), w->b_g, w->b_sel,
+                                                           logits, idx, tw, cc);
         else
             router_rowdot_kernel<__nv_bfloat16><<<T, 1024, 0, s>>>(static_cast<const __nv_bfloat16 *>(x), T, D, N, K,
                                                                    static_cast<const __nv_bfloat16 *>(w->W_g), w->b_g,
-                                                                   logits, idx, tw, cc);
+                                                                   w->b_sel, logits, idx, tw, cc);
         return check_launch();
     }
     if (P.small_router) {
         const size_t smem = (size_t)P.np * D * P.es + (size_t)P.np * 4;
 #define MOE_ROUTER(TIN, NP)                                                                                     \
     router_small_kernel<TIN, NP><<<P.n_chunks, 256, smem, s>>>(static_cast<const TIN *>(x), T, D, N, K,        \
-                                                               static_cast<const TIN *>(w->W_g), w->b_g, logits, \
-                                                               idx, tw, cc)
+                                                               static_cast<const TIN *>(w->W_g), w->b_g, w->b_sel, \
+                                                               logits, idx, tw, cc)
         if (P.dtype == MOE_F32) {
             if (P.np == 8) MOE_ROUTER(float, 8);
             else if (P.np == 16) MOE_ROUTER(float, 16);
@@ -531,7 +543,7 @@ int stage_route(const Plan &P, const Bufs &b, const void *x, const moe_weights *
         MOE_TRY(launch_simt<simt::EPI_LOGITS>(p, T, (int)cdiv(N, simt::TN), s));
     }
     const size_t hs = (size_t)N * 4;
-#define MOE_TOPK(V) topk_kernel<V><<<P.n_chunks, 256, hs, s>>>(logits, T, N, K, idx, tw, cc)
+#define MOE_TOPK(V) topk_kernel<V><<<P.n_chunks, 256, hs, s>>>(logits, T, N, K, w->b_sel, idx, tw, cc)
     switch (P.vpl) {
         case 1: MOE_TOPK(1); break;
         case 2: MOE_TOPK(2); break;
@@ -710,7 +722,7 @@ int stage_up(const Plan &P, const Bufs &b, const moe_weights *w, const DeviceInf
 // prefill layers with K <= 2 and an fp32 y: at most two additions per element
 // onto +0, so the result is the same in any order.
 bool combine_in_down(const Plan &P, int y_dtype) {
-    return P.dtype == MOE_BF16 && !P.decode && P.K <= 2 && y_dtype == MOE_F32;
+    return P.dtype == MOE_BF16 && !P.decode && P.K <= 2 && y_dtype == MOE_F32 && !P.n_shared;
 }
 
 int stage_down(const Plan &P, const Bufs &b, const moe_weights *w, void *y, int y_dtype, const DeviceInfo &dev,
@@ -767,16 +779,172 @@ int stage_down(const Plan &P, const Bufs &b, const moe_weights *w, void *y, int 
     return launch_simt<simt::EPI_SCATTER>(p, P.rows_cap, (int)cdiv(D, simt::TN), s);
 }
 
+// ---------------------------------------------------------------- shared expert
+// A dense FFN over every token: the grouped GEMMs in dense mode (one group,
+// the token rows of x as the A operand, no dispatch) for prefill, the
+// weight-streaming GEMMs with a one-group table for few tokens.  Its fp32
+// output s_out is added by the combine after the routed sum.
+int stage_shared_up(const Plan &P, const Bufs &b, const void *x, const moe_weights *w, const DeviceInfo &dev,
+                    cudaStream_t s) {
+    const int D = P.D, H = P.H;
+    const bool swiglu = P.act == MOE_ACT_SWIGLU;
+    const int rows1 = swiglu ? 2 * H : H;
+    const float *bias = swiglu ? nullptr : w->sb1;
+    if (P.dtype == MOE_F32) {
+        simt::Params p{};
+        p.A = static_cast<const float *>(x);
+        p.lda = D;
+        p.B = static_cast<const float *>(w->S1);
+        p.ldb = D;
+        p.K = D;
+        p.num_groups = 1;
+        p.row_offsets = nullptr;
+        p.dense_rows = (int)P.T;
+        p.b_group_rows = rows1;
+        p.b_up_offset = H;
+        p.n_valid = H;
+        p.out = b.at<float>(P.h_s);
+        p.ldo = H;
+        p.bias = bias;
+        if (swiglu) return launch_simt<simt::EPI_SWIGLU>(p, P.T, (int)cdiv(H, simt::TN / 2), s);
+        return launch_simt<simt::EPI_GELU>(p, P.T, (int)cdiv(H, simt::TN), s);
+    }
+    if (P.decode) {
+        CUtensorMap mw, mx;
+        MOE_TRY(make_map(&mw, w->S1, rows1, D, swiglu ? 64 : 128));
+        MOE_TRY(make_map(&mx, x, P.T, D, P.nt));
+        dec::Params p{};
+        int *tbl = b.at<int>(P.shared_tbl);
+        p.live = tbl;
+        p.n_live = tbl + 1;
+        p.counts = tbl + 2;
+        p.row_offsets = tbl + 3;
+        p.tiles_per_group = (int)cdiv(H, swiglu ? 64 : 128);
+        p.num_k_blocks = (int)cdiv(D, dec::BK);
+        p.w_group_rows = rows1;
+        p.w_up_offset = H;
+        p.n_valid = H;
+        p.out = b.ws + P.h_s;
+        p.ldo = H;
+        p.bias = bias;
+        p.split_cap = P.dec_cap;
+        p.part = b.at<float>(P.dec_part);
+        p.tickets = b.at<unsigned>(P.counters) + 128 + 2 * P.dec_cap;
+        p.timeout_ns = kTimeoutNs;
+        if (swiglu) return launch_dec_nt<dec::EPI_SWIGLU>(P.nt, mw, mx, p, p.tiles_per_group, dev.sms, s);
+        return launch_dec_nt<dec::EPI_GELU>(P.nt, mw, mx, p, p.tiles_per_group, dev.sms, s);
+    }
+    const int bn = narrow_tiles(P, swiglu ? cdiv(H, 128) : cdiv(H, 256), dev) ? 128 : 256;
+    const int out_cols = swiglu ? bn / 2 : bn;
+    CUtensorMap ma, mb, mo;
+    MOE_TRY(make_map(&ma, x, P.T, D, tc::BM));
+    MOE_TRY(make_map(&mb, w->S1, rows1, D, bn == 256 ? 128 : (swiglu ? bn / 2 : bn)));
+    MOE_TRY(make_store_map(&mo, b.ws + P.h_s, P.T, H));
+    tc::Params p{};
+    p.num_groups = 1;
+    p.row_offsets = nullptr;
+    p.dense_rows = (int)P.T;
+    p.n_tiles = (int)cdiv(H, out_cols);
+    p.num_k_blocks = (int)cdiv(D, tc::BK);
+    p.b_group_rows = rows1;
+    p.b_up_offset = H;
+    p.n_valid = H;
+    p.out = b.ws + P.h_s;
+    p.ldo = H;
+    p.bias = bias;
+    p.timeout_ns = kTimeoutNs;
+    if (bn == 128) {
+        const int64_t upper = cdiv(P.T, tc::BM) * p.n_tiles;
+        if (swiglu) return launch_tc<128, tc::EPI_SWIGLU>(ma, mb, mo, p, upper, dev.sms, s);
+        return launch_tc<128, tc::EPI_GELU>(ma, mb, mo, p, upper, dev.sms, s);
+    }
+    const int64_t units = cdiv(P.T, 2 * tc::BM) * p.n_tiles;
+    if (swiglu) return launch_tc2<tc::EPI_SWIGLU>(ma, mb, mo, p, units, dev.pair_clusters, s);
+    return launch_tc2<tc::EPI_GELU>(ma, mb, mo, p, units, dev.pair_clusters, s);
+}
+
+int stage_shared_down(const Plan &P, const Bufs &b, const moe_weights *w, const DeviceInfo &dev, cudaStream_t s) {
+    const int D = P.D, H = P.H;
+    const float *bias = P.act == MOE_ACT_SWIGLU ? nullptr : w->sb2;
+    if (P.dtype == MOE_F32) {
+        simt::Params p{};
+        p.A = b.at<float>(P.h_s);
+        p.lda = H;
+        p.B = static_cast<const float *>(w->S2);
+        p.ldb = H;
+        p.K = H;
+        p.num_groups = 1;
+        p.row_offsets = nullptr;
+        p.dense_rows = (int)P.T;
+        p.b_group_rows = D;
+        p.n_valid = D;
+        p.out = b.at<float>(P.s_out);
+        p.ldo = D;
+        p.bias = bias;
+        p.perm_slot = nullptr;   // row r is token r, weight 1
+        p.gate_w = nullptr;
+        return launch_simt<simt::EPI_SCATTER>(p, P.T, (int)cdiv(D, simt::TN), s);
+    }
+    if (P.decode) {
+        CUtensorMap mw, mx;
+        MOE_TRY(make_map(&mw, w->S2, D, H, 128));
+        MOE_TRY(make_map(&mx, b.ws + P.h_s, P.T, H, P.nt));
+        dec::Params p{};
+        int *tbl = b.at<int>(P.shared_tbl);
+        p.live = tbl;
+        p.n_live = tbl + 1;
+        p.counts = tbl + 2;
+        p.row_offsets = tbl + 3;
+        p.tiles_per_group = (int)cdiv(D, 128);
+        p.num_k_blocks = (int)cdiv(H, dec::BK);
+        p.w_group_rows = D;
+        p.n_valid = D;
+        p.out = b.ws + P.s_out;
+        p.ldo = D;
+        p.bias = bias;
+        p.perm_slot = nullptr;   // row j is token j, weight 1
+        p.gate_w = nullptr;
+        p.split_cap = P.dec_cap;
+        p.part = b.at<float>(P.dec_part);
+        p.tickets = b.at<unsigned>(P.counters) + 128 + 3 * P.dec_cap;
+        p.timeout_ns = kTimeoutNs;
+        return launch_dec_nt<dec::EPI_SCATTER>(P.nt, mw, mx, p, p.tiles_per_group, dev.sms, s);
+    }
+    const int bn = narrow_tiles(P, cdiv(D, 256), dev) ? 128 : 256;
+    CUtensorMap ma, mb, mo;
+    MOE_TRY(make_map(&ma, b.ws + P.h_s, P.T, H, tc::BM));
+    MOE_TRY(make_map(&mb, w->S2, D, H, 128));
+    MOE_TRY(make_store_map_f32(&mo, b.ws + P.s_out, P.T, D));
+    tc::Params p{};
+    p.num_groups = 1;
+    p.row_offsets = nullptr;
+    p.dense_rows = (int)P.T;
+    p.n_tiles = (int)cdiv(D, bn);
+    p.num_k_blocks = (int)cdiv(H, tc::BK);
+    p.b_group_rows = D;
+    p.n_valid = D;
+    p.out = b.ws + P.s_out;
+    p.ldo = D;
+    p.bias = bias;
+    p.perm_slot = nullptr;   // dense rows: row r is token r, weight 1
+    p.gate_w = nullptr;
+    p.scatter_rows = 1;
+    p.timeout_ns = kTimeoutNs;
+    if (bn == 128) return launch_tc<128, tc::EPI_SCATTER>(ma, mb, mo, p, cdiv(P.T, tc::BM) * p.n_tiles, dev.sms, s);
+    return launch_tc2<tc::EPI_SCATTER>(ma, mb, mo, p, cdiv(P.T, 2 * tc::BM) * p.n_tiles, dev.pair_clusters, s);
+}
+
 int stage_combine(const Plan &P, const Bufs &b, void *y, int y_dtype, const DeviceInfo &dev, cudaStream_t s) {
     const int64_t nq = P.T * (P.D / 4);
     const int grid = (int)std::min<int64_t>(cdiv(nq, 256), (int64_t)dev.sms * 8);
     // bf16 prefill layers keep z in the permuted row order (see stage_down)
     const int *slot_row = P.dtype == MOE_BF16 && !P.decode ? b.at<int>(P.slot_row) : nullptr;
+    const float *shared = P.n_shared ? b.at<float>(P.s_out) : nullptr;
     if (y_dtype == MOE_F32)
         return launch_pdl(combine_kernel<float>, dim3(grid), dim3(256), 0, s, (const float *)b.at<float>(P.z), P.T, P.D,
-                          P.K, slot_row, static_cast<float *>(y));
+                          P.K, slot_row, shared, static_cast<float *>(y));
     return launch_pdl(combine_kernel<__nv_bfloat16>, dim3(grid), dim3(256), 0, s, (const float *)b.at<float>(P.z), P.T,
-                      P.D, P.K, slot_row, static_cast<__nv_bfloat16 *>(y));
+                      P.D, P.K, slot_row, shared, static_cast<__nv_bfloat16 *>(y));
 }
 
 int stage_aux(const Plan &P, const Bufs &b, const float *logits, const int *idx, const float *tw, moe_aux *aux,
@@ -804,7 +972,8 @@ int stage_aux(const Plan &P, const Bufs &b, const float *logits, const int *idx,
 int zero_counters(const Plan &P, const Bufs &b, cudaStream_t s) {
     DeviceInfo *dev = nullptr;
     MOE_TRY(device_info(&dev));
-    return launch_zero(b.ws + P.counters, P.counters_bytes, dev->sms, s);
+    return launch_zero(b.ws + P.counters, P.counters_bytes, dev->sms, s,
+                       P.n_shared ? b.at<int>(P.shared_tbl) : nullptr, (int)P.T);
 }
 
 int zero_aux(const Plan &P, moe_aux *aux, cudaStream_t s) {
@@ -822,6 +991,10 @@ int check_weights(const Plan &P, const moe_weights *w, bool need_experts) {
     if (!w->W1 || !w->W2) return MOE_ERR_INVALID_ARG;
     if (P.has_bias && (!w->b1 || !w->b2)) return MOE_ERR_INVALID_ARG;
     if (!aligned16(w->W1) || !aligned16(w->W2)) return MOE_ERR_INVALID_ARG;
+    if (P.n_shared) {
+        if (!w->S1 || !w->S2 || !aligned16(w->S1) || !aligned16(w->S2)) return MOE_ERR_INVALID_ARG;
+        if (P.has_bias && (!w->sb1 || !w->sb2)) return MOE_ERR_INVALID_ARG;
+    }
     return MOE_OK;
 }
 
@@ -874,8 +1047,10 @@ int forward_impl(const moe_config *cfg, const void *x, int64_t T, const moe_weig
     MOE_TRY(stage_permute(P, b, x, P.simt_router ? nullptr : y_zero, *dev, s));
     MOE_TRY(rec(3));
     MOE_TRY(stage_up(P, b, w, *dev, s));
+    if (P.n_shared) MOE_TRY(stage_shared_up(P, b, x, w, *dev, s));
     MOE_TRY(rec(4));
     MOE_TRY(stage_down(P, b, w, y, y_dtype, *dev, s));
+    if (P.n_shared) MOE_TRY(stage_shared_down(P, b, w, *dev, s));
     MOE_TRY(rec(5));
     if (!combine_in_down(P, y_dtype)) MOE_TRY(stage_combine(P, b, y, y_dtype, *dev, s));
     MOE_TRY(rec(6));
@@ -1016,7 +1191,7 @@ int64_t moe_total_params(const moe_config *c) {
     if (make_plan(c, 0, &P) != MOE_OK) return -1;
     const int64_t D = P.D, H = P.H, N = P.N;
     const int64_t ex = P.act == MOE_ACT_SWIGLU ? 3 * D * H : 2 * D * H + (P.has_bias ? H + D : 0);
-    return D * N + N * ex;
+    return D * N + (N + P.n_shared) * ex;
 }
 
 int64_t moe_active_params(const moe_config *c) {
@@ -1024,7 +1199,7 @@ int64_t moe_active_params(const moe_config *c) {
     if (make_plan(c, 0, &P) != MOE_OK) return -1;
     const int64_t D = P.D, H = P.H, N = P.N, K = P.K;
     const int64_t ex = P.act == MOE_ACT_SWIGLU ? 3 * D * H : 2 * D * H + (P.has_bias ? H + D : 0);
-    return D * N + K * ex;
+    return D * N + (K + P.n_shared) * ex;
 }
 
 int moe_get_device_status(void) {
@@ -1102,6 +1277,7 @@ int moe_aux_stats_noalloc(const moe_config *cfg, int64_t T, const float *logits,
     DeviceInfo *dev = nullptr;
     MOE_TRY(device_info(&dev));
     Plan Q = P;
+    Q.n_shared = 0;   // nothing outside the fixed array is written
     Q.counters = 0;
     Q.counters_bytes = 256;
     Q.aux_p = 256;

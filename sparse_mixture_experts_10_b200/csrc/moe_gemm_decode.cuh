@@ -59,7 +59,7 @@ struct Params {
     void *out;                // h [rows, H] (token rows) or z [T*K, D] (slot rows)
     int64_t ldo;
     const float *bias;        // [N, n_valid] or nullptr
-    const int *perm_slot;     // EPI_SCATTER
+    const int *perm_slot;     // EPI_SCATTER (nullptr: row j is token j, weight 1)
     const float *gate_w;      // EPI_SCATTER
     // stream-K (split_cap == 0: whole tiles round-robin)
     int split_cap;            // CTAs the partial buffer and the tickets are sized for (>= gridDim.x)
@@ -406,9 +406,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                     float *z = static_cast<float *>(p.out);
 #pragma unroll
                     for (int j = 0; j < NT; ++j) {
-                        if (j < cnt) {
-                            const int slot = p.perm_slot[trow + j];
-                            z[(int64_t)slot * p.ldo + d] = p.gate_w[slot] * (acc[j] + b);
+                        if (j < cnt) {   // no perm_slot (shared expert): row j is token j, weight 1
+                            const int slot = p.perm_slot ? p.perm_slot[trow + j] : trow + j;
+                            const float gw = p.perm_slot ? p.gate_w[slot] : 1.f;
+                            z[(int64_t)slot * p.ldo + d] = gw * (acc[j] + b);
                         }
                     }
                 }

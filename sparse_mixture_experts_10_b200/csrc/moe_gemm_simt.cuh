@@ -119,9 +119,9 @@ __global__ void __launch_bounds__(256) grouped_gemm_simt_kernel(const Params p) 
         float v = Cs[m][n] + (p.bias ? p.bias[(int64_t)g * p.n_valid + f] : 0.f);
         if (EPI == EPI_GELU) {
             p.out[(int64_t)r * p.ldo + f] = gelu_erf(v);
-        } else if (EPI == EPI_SCATTER) {
-            const int slot = p.perm_slot[r];
-            if (slot >= 0) p.out[(int64_t)slot * p.ldo + f] = p.gate_w[slot] * v;
+        } else if (EPI == EPI_SCATTER) {   // no perm_slot (dense rows, shared expert): row r is token r, weight 1
+            const int slot = p.perm_slot ? p.perm_slot[r] : r;
+            if (slot >= 0) p.out[(int64_t)slot * p.ldo + f] = (p.perm_slot ? p.gate_w[slot] : 1.f) * v;
         } else {
             p.out[(int64_t)r * p.ldo + f] = v;
         }

@@ -76,7 +76,7 @@ struct Params {
     void *out;                // output base
     int64_t ldo;              // output row stride (elements)
     const float *bias;        // [G, n_valid] or nullptr
-    const int *perm_slot;     // EPI_SCATTER: slot of each permuted row (-1 = padding)
+    const int *perm_slot;     // EPI_SCATTER: slot of each permuted row (-1 = padding); nullptr: row = slot, weight 1
     const float *gate_w;      // EPI_SCATTER: gate weight of each slot
     // EPI_SCATTER with accum_k > 0: out is y [T, ldo] fp32 (zeroed before the
     // launch) and each row's scaled result is added into row slot / accum_k with
@@ -300,8 +300,13 @@ template <int EPI>
 __device__ __forceinline__ RowGate load_row_gate(const Params &p, int row, int row_limit) {
     RowGate r;
     if (EPI == EPI_SCATTER && row < row_limit) {
-        r.slot = p.perm_slot[row];
-        if (r.slot >= 0) r.gw = p.gate_w[r.slot];
+        if (p.perm_slot) {
+            r.slot = p.perm_slot[row];
+            if (r.slot >= 0) r.gw = p.gate_w[r.slot];
+        } else {   // dense rows (shared expert): row r is token r, weight 1
+            r.slot = row;
+            r.gw = 1.f;
+        }
     }
     return r;
 }

@@ -87,36 +87,50 @@ struct Vec16<__nv_bfloat16> {
     }
 };
 
-// Top-k over one segment of NP lanes, each holding one (score, expert) entry,
-// then the renormalised softmax.  Lane r of the segment (r < K) returns slot r.
-// Returns true for lanes that hold a slot.
+// Top-k over one segment of NP lanes, each holding one expert: its selection
+// value v (the score, plus a selection-only bias when one is given) and its raw
+// score.  The K best by (v, lower index on ties) are kept; the gate weights
+// are the softmax over the kept experts' raw scores, shifted by the largest of
+// them -- softmax(KeepTopK(.)) of the Shazeer article's gating section with the
+// kept set chosen on v.  Without a selection bias v == raw and the shift is
+// slot 0's score.  Lane r of the segment (r < K) returns slot r.  Returns true
+// for lanes that hold a slot.
 template <int NP>
-__device__ __forceinline__ bool segment_topk(float v, int e, bool taken, int K, int seg_lane, int lane,
+__device__ __forceinline__ bool segment_topk(float v, float raw, int e, bool taken, int K, int seg_lane, int lane,
                                              int &slot_e, float &slot_w) {
-    float best0 = 0.f, my_v = -INFINITY;
+    float my_raw = -INFINITY;
     int my_e = 0;
     for (int r = 0; r < K; ++r) {
-        float cv = v;
+        float cv = v, cr = raw;
         int ce = e;
         bool ct = taken;
 #pragma unroll
         for (int o = NP / 2; o >= 1; o >>= 1) {
             const float ov = __shfl_xor_sync(0xffffffffu, cv, o);
+            const float orw = __shfl_xor_sync(0xffffffffu, cr, o);
             const int oe = __shfl_xor_sync(0xffffffffu, ce, o);
             const bool ot = __shfl_xor_sync(0xffffffffu, (int)ct, o) != 0;
-            if (beats(ov, oe, ot, cv, ce, ct)) { cv = ov; ce = oe; ct = ot; }
+            if (beats(ov, oe, ot, cv, ce, ct)) { cv = ov; cr = orw; ce = oe; ct = ot; }
         }
         if (e == ce) taken = true;
-        if (r == 0) best0 = cv;
-        if (seg_lane == r) { my_v = cv; my_e = ce; }
+        if (seg_lane == r) { my_raw = cr; my_e = ce; }
     }
-    const float ex = seg_lane < K ? expf(my_v - best0) : 0.f;
+    float m = seg_lane < K ? my_raw : -INFINITY;
+#pragma unroll
+    for (int o = NP / 2; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    const float ex = seg_lane < K ? expf(my_raw - m) : 0.f;
     float sum = 0.f;
     const int seg_base = lane - seg_lane;
-    for (int m = 0; m < K; ++m) sum += __shfl_sync(0xffffffffu, ex, seg_base + m);  // slot order
+    for (int q = 0; q < K; ++q) sum += __shfl_sync(0xffffffffu, ex, seg_base + q);  // slot order
     slot_e = my_e;
     slot_w = ex / sum;
     return seg_lane < K;
+}
+
+// The selection value of a score: score + selection-only bias (fp32), or the
+// score itself.
+__device__ __forceinline__ float sel_value(const float *bsel, float s, int e, bool valid) {
+    return (bsel && valid) ? s + __ldg(bsel + e) : s;
 }
 
 // ---------------------------------------------------------------------------
@@ -129,6 +143,7 @@ __device__ __forceinline__ bool segment_topk(float v, int e, bool taken, int K, 
 template <typename Tin, int NP>
 __global__ void __launch_bounds__(256) router_small_kernel(const Tin *__restrict__ x, int T, int D, int N, int K,
                                                            const Tin *__restrict__ Wg, const float *__restrict__ bg,
+                                                           const float *__restrict__ bsel,
                                                            float *__restrict__ logits, int *__restrict__ topk_idx,
                                                            float *__restrict__ topk_w, int *__restrict__ chunk_counts) {
     constexpr int TPW = 32 / NP;
@@ -197,7 +212,8 @@ __global__ void __launch_bounds__(256) router_small_kernel(const Tin *__restrict
         }
         int slot_e;
         float slot_w;
-        const bool has_slot = segment_topk<NP>(s, e, !valid_e, K, seg_lane, lane, slot_e, slot_w);
+        const bool has_slot =
+            segment_topk<NP>(sel_value(bsel, s, e, valid_e), s, e, !valid_e, K, seg_lane, lane, slot_e, slot_w);
         if (has_slot && t < T) {
             topk_idx[(size_t)t * K + seg_lane] = slot_e;
             topk_w[(size_t)t * K + seg_lane] = slot_w;
@@ -218,6 +234,7 @@ __global__ void __launch_bounds__(256) router_small_kernel(const Tin *__restrict
 template <typename Tin>
 __global__ void __launch_bounds__(1024) router_rowdot_kernel(const Tin *__restrict__ x, int T, int D, int N, int K,
                                                              const Tin *__restrict__ Wg, const float *__restrict__ bg,
+                                                             const float *__restrict__ bsel,
                                                              float *__restrict__ logits, int *__restrict__ topk_idx,
                                                              float *__restrict__ topk_w, int *__restrict__ chunk_counts) {
     __shared__ float part[32][33];
@@ -257,7 +274,7 @@ __global__ void __launch_bounds__(1024) router_rowdot_kernel(const Tin *__restri
     }
     int slot_e;
     float slot_w;
-    if (segment_topk<32>(s, lane, !live, K, lane, lane, slot_e, slot_w)) {
+    if (segment_topk<32>(sel_value(bsel, s, lane, live), s, lane, !live, K, lane, lane, slot_e, slot_w)) {
         topk_idx[(size_t)t * K + lane] = slot_e;
         topk_w[(size_t)t * K + lane] = slot_w;
         atomicAdd(&chunk_counts[(size_t)(t / kChunk) * N + slot_e], 1);
@@ -270,6 +287,7 @@ __global__ void __launch_bounds__(1024) router_rowdot_kernel(const Tin *__restri
 // ---------------------------------------------------------------------------
 template <int VPL>
 __global__ void __launch_bounds__(256) topk_kernel(const float *__restrict__ logits, int T, int N, int K,
+                                                   const float *__restrict__ bsel,
                                                    int *__restrict__ topk_idx, float *__restrict__ topk_w,
                                                    int *__restrict__ chunk_counts) {
     extern __shared__ int hist_s[];
@@ -279,46 +297,51 @@ __global__ void __launch_bounds__(256) topk_kernel(const float *__restrict__ log
     for (int tl = warp; tl < kChunk; tl += 8) {
         const int t = blockIdx.x * kChunk + tl;
         if (t >= T) break;
-        float v[VPL];
+        float v[VPL], raw[VPL];   // selection values (score + selection bias) and raw scores
         uint32_t taken = 0;
 #pragma unroll
         for (int i = 0; i < VPL; ++i) {
             const int e = lane + 32 * i;
             if (e < N) {
-                v[i] = logits[(size_t)t * N + e];
-                if (v[i] != v[i]) {
+                raw[i] = logits[(size_t)t * N + e];
+                if (raw[i] != raw[i]) {
                     set_status(kStatusNanLogit);
-                    v[i] = -INFINITY;
+                    raw[i] = -INFINITY;
                 }
+                v[i] = sel_value(bsel, raw[i], e, true);
             } else {
-                v[i] = -INFINITY;
+                v[i] = raw[i] = -INFINITY;
                 taken |= 1u << i;
             }
         }
-        float best0 = 0.f, my_v = -INFINITY;
+        float my_raw = -INFINITY;
         int my_e = 0;
         for (int r = 0; r < K; ++r) {
             // best untaken entry of this lane (lower index first on ties)
-            float cv = -INFINITY;
+            float cv = -INFINITY, cr = -INFINITY;
             int ce = 0x7fffffff;
             bool ct = true;
 #pragma unroll
             for (int i = 0; i < VPL; ++i) {
                 const bool ti = (taken >> i) & 1u;
-                if (beats(v[i], lane + 32 * i, ti, cv, ce, ct)) { cv = v[i]; ce = lane + 32 * i; ct = ti; }
+                if (beats(v[i], lane + 32 * i, ti, cv, ce, ct)) { cv = v[i]; cr = raw[i]; ce = lane + 32 * i; ct = ti; }
             }
 #pragma unroll
             for (int o = 16; o >= 1; o >>= 1) {
                 const float ov = __shfl_xor_sync(0xffffffffu, cv, o);
+                const float orw = __shfl_xor_sync(0xffffffffu, cr, o);
                 const int oe = __shfl_xor_sync(0xffffffffu, ce, o);
                 const bool ot = __shfl_xor_sync(0xffffffffu, (int)ct, o) != 0;
-                if (beats(ov, oe, ot, cv, ce, ct)) { cv = ov; ce = oe; ct = ot; }
+                if (beats(ov, oe, ot, cv, ce, ct)) { cv = ov; cr = orw; ce = oe; ct = ot; }
             }
             if ((ce & 31) == lane) taken |= 1u << (ce >> 5);
-            if (r == 0) best0 = cv;
-            if (lane == r) { my_v = cv; my_e = ce; }
+            if (lane == r) { my_raw = cr; my_e = ce; }
         }
-        const float ex = lane < K ? expf(my_v - best0) : 0.f;
+        // shift by the largest kept raw score (slot 0's without a selection bias)
+        float best0 = lane < K ? my_raw : -INFINITY;
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) best0 = fmaxf(best0, __shfl_xor_sync(0xffffffffu, best0, o));
+        const float ex = lane < K ? expf(my_raw - best0) : 0.f;
         float sum = 0.f;
         for (int m = 0; m < K; ++m) sum += __shfl_sync(0xffffffffu, ex, m);
         if (lane < K) {
@@ -529,21 +552,31 @@ __global__ void __launch_bounds__(256) permute_kernel(const Tin *__restrict__ x,
 }
 
 // Zero n16 16-byte words at p (a memset that takes part in programmatic
-// dependent launch).
-__global__ void __launch_bounds__(256) zero_kernel(uint4 *__restrict__ p, int64_t n16) {
+// dependent launch); with tbl, also write the shared expert's one-group
+// dispatch table there: live = {0}, one live group, count T, first row 0.
+__global__ void __launch_bounds__(256) zero_kernel(uint4 *__restrict__ p, int64_t n16, int *__restrict__ tbl,
+                                                   int tbl_T) {
     pdl_enter();
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n16; i += (int64_t)gridDim.x * blockDim.x)
         p[i] = make_uint4(0u, 0u, 0u, 0u);
+    if (tbl && blockIdx.x == 0 && threadIdx.x == 0) {
+        tbl[0] = 0;
+        tbl[1] = 1;
+        tbl[2] = tbl_T;
+        tbl[3] = 0;
+    }
 }
 
 // ---------------------------------------------------------------------------
 // Combine: y[t] = z[t, 0] + z[t, 1] + ... + z[t, K-1], left to right (slot
 // order), no atomics ("MoE(Mixture of Experts)", section (2), Forward, which
-// adds the weighted expert outputs of a row in selection order).
+// adds the weighted expert outputs of a row in selection order); then, with a
+// shared expert, + s[t] (its output, added after the routed sum).
 // ---------------------------------------------------------------------------
 template <typename Tout>
 __global__ void __launch_bounds__(256) combine_kernel(const float *__restrict__ z, int64_t T, int D, int K,
-                                                      const int *__restrict__ slot_row, Tout *__restrict__ y) {
+                                                      const int *__restrict__ slot_row,
+                                                      const float *__restrict__ shared, Tout *__restrict__ y) {
     pdl_enter();
     const int64_t nq = T * (D / 4);
     for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < nq; i += (int64_t)gridDim.x * blockDim.x) {
@@ -557,6 +590,10 @@ __global__ void __launch_bounds__(256) combine_kernel(const float *__restrict__ 
         float4 acc = *reinterpret_cast<const float4 *>(zrow(0));
         for (int j = 1; j < K; ++j) {
             const float4 v = *reinterpret_cast<const float4 *>(zrow(j));
+            acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+        }
+        if (shared) {
+            const float4 v = *reinterpret_cast<const float4 *>(shared + t * D + d);
             acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
         }
         if constexpr (sizeof(Tout) == 4) {

@@ -44,6 +44,7 @@ constexpr double kImpScale = 4294967296.0;   // gate weights summed in 2^-32 fix
 struct Params {
     int T, D, N, K, np;                  // np: N rounded up to the MMA width
     const float *bg;                     // [N] or nullptr
+    const float *bsel;                   // [N] or nullptr: selection-only bias (changes the kept set only)
     float *logits;                       // [T, N]
     int *topk_idx;                       // [T, K]
     float *topk_w;                       // [T, K]
@@ -308,21 +309,24 @@ __device__ __forceinline__ void for_each_logit(const Params &p, uint32_t tlane, 
     }
 }
 
-// Keep (s, e) in the best-first list (tv, te) of length KM if it belongs there:
-// larger value first, equal values in ascending expert index.
+// Keep (v, e) with its raw score r in the best-first list (tv, te, tr) of length
+// KM if it belongs there: larger selection value first, equal values in
+// ascending expert index.
 template <int KM>
-__device__ __forceinline__ void topk_insert(float (&tv)[KM], int (&te)[KM], float s, int e) {
+__device__ __forceinline__ void topk_insert(float (&tv)[KM], int (&te)[KM], float (&tr)[KM], float s, int e, float r) {
     if (!(s > tv[KM - 1] || (s == tv[KM - 1] && e < te[KM - 1]))) return;
-    float cv = s;
+    float cv = s, cr = r;
     int ce = e;
 #pragma unroll
     for (int j = 0; j < KM; ++j) {
         const bool better = cv > tv[j] || (cv == tv[j] && ce < te[j]);
-        const float ov = tv[j];
+        const float ov = tv[j], orw = tr[j];
         const int oe = te[j];
         tv[j] = better ? cv : ov;
+        tr[j] = better ? cr : orw;
         te[j] = better ? ce : oe;
         cv = better ? ov : cv;
+        cr = better ? orw : cr;
         ce = better ? oe : ce;
     }
 }
@@ -435,21 +439,28 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         if (have) {
             const uint32_t tlane = tmem_base + (static_cast<uint32_t>(ew * 32) << 16);
-            // pass 1: logits out, top-K
-            float tv[KM];
+            // pass 1: logits out, top-K on the selection values, the largest raw score
+            float tv[KM], tr[KM];
             int te[KM];
 #pragma unroll
-            for (int j = 0; j < KM; ++j) { tv[j] = -INFINITY; te[j] = 0x7fffffff; }
+            for (int j = 0; j < KM; ++j) { tv[j] = tr[j] = -INFINITY; te[j] = 0x7fffffff; }
+            float smax = -INFINITY;
             for_each_logit<NP>(p, tlane, [&](int e, float s) {
                 if (live_row) p.logits[(int64_t)t * p.N + e] = s;
-                topk_insert<KM>(tv, te, s, e);
+                topk_insert<KM>(tv, te, tr, p.bsel ? s + __ldg(p.bsel + e) : s, e, s);
+                smax = fmaxf(smax, s);
             });
-            // gate weights over the K kept scores, slot order
+            // gate weights: softmax over the K kept raw scores, shifted by their largest
+            // (slot 0's without a selection bias), slot order
+            float kmax = -INFINITY;
+#pragma unroll
+            for (int j = 0; j < KM; ++j)
+                if (j < p.K) kmax = fmaxf(kmax, tr[j]);
             float ex[KM];
             float sum = 0.f;
 #pragma unroll
             for (int j = 0; j < KM; ++j) {
-                ex[j] = j < p.K ? expf(tv[j] - tv[0]) : 0.f;
+                ex[j] = j < p.K ? expf(tr[j] - kmax) : 0.f;
                 sum += ex[j];
             }
             const float inv = 1.0f / sum;
@@ -463,8 +474,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     atomicAdd(&s_imp[te[j]], (unsigned long long)__double2ull_rn((double)wj * kImpScale));
                 }
             }
-            // pass 2: normaliser of the full softmax (the maximum is the best kept score)
-            const float m = tv[0];
+            // pass 2: normaliser of the full softmax of the raw scores
+            const float m = smax;
             float z = 0.f;
             for_each_logit<NP>(p, tlane, [&](int e, float s) { z += expf(s - m); });
             const float inv_z = live_row ? 1.0f / z : 0.f;
@@ -654,7 +665,8 @@ __global__ void __launch_bounds__(256, NP == 8 ? 2 : 1) router_simt_kernel(const
         }
         int slot_e;
         float slot_w;
-        const bool has = segment_topk<NP>(s, e, !valid_e, K, seg_lane, lane, slot_e, slot_w);
+        const bool has = segment_topk<NP>(sel_value(p.bsel, s, e, valid_e), s, e, !valid_e, K, seg_lane, lane, slot_e,
+                                          slot_w);
         if (has && tok) {
             p.topk_idx[(int64_t)t * K + seg_lane] = slot_e;
             p.topk_w[(int64_t)t * K + seg_lane] = slot_w;
@@ -780,7 +792,8 @@ __global__ void __launch_bounds__(256) router_few_kernel(const __nv_bfloat16 *__
         if (live) p.logits[(int64_t)t * N + lane] = s;
         int slot_e;
         float slot_w;
-        const bool has = segment_topk<32>(s, lane, !live, p.K, lane, lane, slot_e, slot_w);
+        const bool has = segment_topk<32>(sel_value(p.bsel, s, lane, live), s, lane, !live, p.K, lane, lane, slot_e,
+                                          slot_w);
         if (has) {
             p.topk_idx[(int64_t)t * p.K + lane] = slot_e;
             p.topk_w[(int64_t)t * p.K + lane] = slot_w;

@@ -57,12 +57,24 @@ def assert_y_close(y_gpu: np.ndarray, y_ref: np.ndarray, dtype: torch.dtype):
     return max_abs, rel_l2
 
 
+def selection_scores(logits, inp):
+    """What the device ranks: its fp32 logits, plus the selection-only bias added in fp32."""
+    lg = np.asarray(logits, dtype=np.float32)
+    b = inp.get("b_sel")
+    return lg if b is None else (lg + host(b).astype(np.float32)).astype(np.float32)
+
+
+def shared_kwargs(inp):
+    return dict(S1=host(inp.get("S1")), S2=host(inp.get("S2")), sb1=host(inp.get("sb1")), sb2=host(inp.get("sb2")))
+
+
 def oracle_full_layer(inp, wl, K, gpu_logits=None, threads=None):
     """The whole layer on every token (small workloads)."""
     t = tag(wl.dtype)
+    sel = None if gpu_logits is None else selection_scores(gpu_logits, inp)
     return oracle.moe_layer(host(inp["x"]), host(inp["W_g"]), host(inp["W1"]), host(inp["W2"]), K=K, act=wl.act,
                             dtype_tag=t, bg=host(inp["b_g"]), b1=host(inp["b1"]), b2=host(inp["b2"]),
-                            sel_scores=gpu_logits, threads=threads)
+                            sel_scores=sel, threads=threads, bsel=host(inp.get("b_sel")), **shared_kwargs(inp))
 
 
 def oracle_rows(inp, wl, K, rows, gpu_logits, threads=None):
@@ -73,7 +85,7 @@ def oracle_rows(inp, wl, K, rows, gpu_logits, threads=None):
     rows = np.asarray(rows, dtype=np.int64)
     xr = oracle.load_rows(host(inp["x"][rows]), t, range(len(rows)))
     scores = oracle.router_scores(xr, host(inp["W_g"]), t, host(inp["b_g"]))
-    sel = oracle.select_topk(gpu_logits[rows].astype(np.float64), K)
+    sel = oracle.select_topk(selection_scores(gpu_logits[rows], inp).astype(np.float64), K)
     w = oracle.gate_weights(scores, sel)
     D = wl.D
     E = np.zeros((len(rows), K, D), dtype=np.float64)
@@ -95,6 +107,14 @@ def oracle_rows(inp, wl, K, rows, gpu_logits, threads=None):
 
             list(ex.map(run, pairs))
     y = np.stack([oracle.combine(w[i], E[i]) for i in range(len(rows))]) if len(rows) else np.zeros((0, D))
+    if inp.get("S1") is not None:
+        sk = shared_kwargs(inp)
+
+        def shared(i):
+            return oracle.add_shared(y[i], oracle.expert(xr[i], wl.act, t, sk["S1"], sk["S2"], sk["sb1"], sk["sb2"]))
+
+        with ThreadPoolExecutor(nthr) as ex:
+            y = np.stack(list(ex.map(shared, range(len(rows))))) if len(rows) else y
     return dict(scores=scores, sel=sel, w=w, y=y)
 
 

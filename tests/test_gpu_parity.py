@@ -35,8 +35,10 @@ class Layer:
 
     def __init__(self, wl: Workload, inp):
         self.wl, self.inp = wl, inp
-        self.cfg = moe.make_config(wl.D, wl.H, wl.N, wl.K, wl.act, moe.dtype_code(wl.dtype), wl.has_bias)
-        self.w = moe.make_weights(inp["W_g"], inp["W1"], inp["W2"], inp["b_g"], inp["b1"], inp["b2"])
+        self.cfg = moe.make_config(wl.D, wl.H, wl.N, wl.K, wl.act, moe.dtype_code(wl.dtype), wl.has_bias,
+                                   wl.n_shared)
+        self.w = moe.make_weights(inp["W_g"], inp["W1"], inp["W2"], inp["b_g"], inp["b1"], inp["b2"],
+                                  inp.get("b_sel"), inp.get("S1"), inp.get("sb1"), inp.get("S2"), inp.get("sb2"))
 
     def forward(self, x=None, y_dtype=torch.float32, with_aux=True):
         x = self.inp["x"] if x is None else x
@@ -79,10 +81,11 @@ class Layer:
         )
 
 
-def check_routing(V, ref_scores, K):
-    """Logits within tolerance, top-k bit-exact on the device's logits, counts exact."""
+def check_routing(V, ref_scores, K, inp):
+    """Logits within tolerance, top-k bit-exact on the device's logits (plus any selection bias,
+    added in fp32 as the device does), counts exact."""
     ph.assert_logits_close(V["logits"], ref_scores)
-    sel = oracle.select_topk(V["logits"].astype(np.float64), K)
+    sel = oracle.select_topk(ph.selection_scores(V["logits"], inp).astype(np.float64), K)
     np.testing.assert_array_equal(V["idx"], sel)
     N = V["counts"].shape[0]
     np.testing.assert_array_equal(V["counts"], np.bincount(sel.ravel(), minlength=N))
@@ -118,7 +121,7 @@ def run_full(wl, inp, y_dtype=torch.float32):
     y, ws, aux = layer.forward(y_dtype=y_dtype)
     V = layer.views(ws, T)
     ref = ph.oracle_full_layer(inp, wl, wl.K, gpu_logits=V["logits"])
-    check_routing(V, ref["scores"], wl.K)
+    check_routing(V, ref["scores"], wl.K, inp)
     ph.assert_weights_close(V["w"], ref["w"], ref["scores"])
     check_dispatch(V, inp["x"], wl.K)
     errs = ph.assert_y_close(y.float().cpu().numpy(), ref["y"], wl.dtype if y_dtype == torch.float32 else y_dtype)
@@ -315,7 +318,7 @@ def test_gpt2_full_size_sampled_rows():
     layer = Layer(wl, inp)
     y, ws, aux = layer.forward()
     V = layer.views(ws, wl.T)
-    sel = oracle.select_topk(V["logits"].astype(np.float64), wl.K)
+    sel = oracle.select_topk(ph.selection_scores(V["logits"], inp).astype(np.float64), wl.K)
     np.testing.assert_array_equal(V["idx"], sel)
     check_dispatch(V, inp["x"], wl.K)
     check_aux(aux, V, wl.N, wl.K)
@@ -332,7 +335,7 @@ def _full_size_sampled(name, n_rows, seed, every_expert=False):
     layer = Layer(wl, inp)
     y, ws, aux = layer.forward()
     V = layer.views(ws, wl.T)
-    sel = oracle.select_topk(V["logits"].astype(np.float64), wl.K)
+    sel = oracle.select_topk(ph.selection_scores(V["logits"], inp).astype(np.float64), wl.K)
     np.testing.assert_array_equal(V["idx"], sel)
     np.testing.assert_array_equal(V["counts"], np.bincount(sel.ravel(), minlength=wl.N))
     check_aux(aux, V, wl.N, wl.K)
@@ -362,7 +365,7 @@ def test_mixtral_full_size_sampled_rows():
     _full_size_sampled("mixtral", 24, 3)
 
 
-@pytest.mark.parametrize("name", ["deepseek", "deepseek_zipf"])
+@pytest.mark.parametrize("name", ["deepseek", "deepseek_zipf", "deepseek_shared"])
 def test_deepseek_full_size_sampled_rows(name):
     _full_size_sampled(name, 12, 4, every_expert=True)
 
@@ -403,6 +406,57 @@ def test_bf16_prefill_k1_and_k3(K):
                   zipf_s=0.5, random_bias=True)
     inp = make_inputs(wl, "cuda")
     run_full(wl, inp)
+
+
+# ----------------------------------------------------------------------------- shared expert, selection bias
+SHARED_CASES = [
+    # (name, workload, T): every router and GEMM family with a shared expert and a selection bias
+    ("fp32_gelu_bias", Workload("sh_f32", 50, 300, 64, 256, 8, 2, ACT_GELU, torch.float32, True, 0.05,
+                                zipf_s=0.6, random_bias=True, n_shared=1, sel_s=0.6), None),
+    ("fp32_swiglu_n40", Workload("sh_f32b", 51, 200, 64, 128, 40, 3, ACT_SWIGLU, torch.float32, False, 0.05,
+                                 zipf_s=0.4, n_shared=1, sel_s=0.8), None),
+    ("bf16_gelu_simt_router_k2", Workload("sh_gelu", 52, 1100, 256, 512, 6, 2, ACT_GELU, torch.bfloat16, True,
+                                          0.04, zipf_s=0.7, random_bias=True, n_shared=1, sel_s=0.7), None),
+    ("bf16_swiglu_tc_router", Workload("sh_tc", 53, 900, 256, 256, 64, 4, ACT_SWIGLU, torch.bfloat16, False,
+                                       0.05, zipf_s=0.5, n_shared=1, sel_s=0.5), None),
+    ("bf16_pairs_ragged", Workload("sh_pairs", 54, 1500, 512, 1024, 8, 2, ACT_SWIGLU, torch.bfloat16, False, 0.04,
+                                   zipf_s=0.7, n_shared=1, sel_s=0.35), None),
+    ("decode1", WORKLOADS["decode1"].with_(n_shared=1, sel_s=0.5, zipf_s=0.5), None),
+    ("decode8", WORKLOADS["decode8"].with_(n_shared=1, sel_s=0.5, zipf_s=0.5), None),
+    ("decode_gelu_t50", Workload("sh_dec", 55, 50, 1024, 1024, 6, 2, ACT_GELU, torch.bfloat16, True, 0.03,
+                                 random_bias=True, n_shared=1, sel_s=0.4, zipf_s=0.4), None),
+    ("few_router_n32", Workload("sh_few", 56, 40, 256, 128, 32, 8, ACT_SWIGLU, torch.bfloat16, False, 0.05,
+                                zipf_s=0.4, n_shared=1, sel_s=0.9), None),
+]
+
+
+@pytest.mark.parametrize("name,wl,_", SHARED_CASES, ids=[c[0] for c in SHARED_CASES])
+def test_shared_expert_and_selection_bias(name, wl, _):
+    """DeepSeek-V3's shared expert and selection-only bias: the kept set follows the device's
+    logits plus the bias (in fp32), the gate weights and statistics the raw scores, and the
+    shared FFN is added after the routed sum; every router and GEMM family."""
+    inp = make_inputs(wl, "cuda")
+    layer, y, ws, aux, V, ref, errs = run_full(wl, inp)
+    check_aux(aux, V, wl.N, wl.K)
+    if wl.dtype == torch.bfloat16:
+        y16, _, _ = layer.forward(y_dtype=torch.bfloat16, with_aux=False)
+        assert torch.equal(y16, y.to(torch.bfloat16))
+
+
+def test_selection_bias_balances_a_skewed_router():
+    """With the selection bias equal and opposite to the Zipf router bias, the choice of experts
+    is as balanced as without either bias, while the weights keep the skew."""
+    base = Workload("bal", 57, 4000, 256, 128, 16, 2, ACT_SWIGLU, torch.bfloat16, False, 0.05)
+    counts = {}
+    for tag, wl in (("plain", base), ("skewed", base.with_(zipf_s=1.0)), ("balanced", base.with_(zipf_s=1.0,
+                                                                                                  sel_s=1.0))):
+        inp = make_inputs(wl, "cuda")
+        layer = Layer(wl, inp)
+        y, ws, aux = layer.forward()
+        counts[tag] = aux["counts"].cpu().numpy()
+    cv = {k: v.std() / v.mean() for k, v in counts.items()}
+    assert cv["skewed"] > 3 * cv["plain"]
+    assert cv["balanced"] < 1.5 * cv["plain"]
 
 
 # ----------------------------------------------------------------------------- data parallelism
