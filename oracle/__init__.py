@@ -85,7 +85,10 @@ def configure(L):
     L.orc_expert_swiglu.argtypes = [i64, i64, vp, vp, vp, i32, vp, vp]
     L.orc_combine.argtypes = [i64, i64, vp, vp, vp]
     L.orc_add_shared.argtypes = [i64, vp, vp]
-    L.orc_moe_layer_rows.argtypes = [ctypes.POINTER(_Layer), i64, i64, vp, vp, vp, vp, vp]
+    L.orc_moe_layer_rows.argtypes = [ctypes.POINTER(_Layer), i64, i64, vp, vp, vp, vp, vp, vp]
+    L.orc_capacity.restype = i64
+    L.orc_capacity.argtypes = [dp, i64, i64, i64]
+    L.orc_capacity_keep.argtypes = [i64, i64, i64, vp, i64, vp]
     L.orc_cv_squared.restype = dp
     L.orc_cv_squared.argtypes = [i64, vp]
     L.orc_simple_balance_loss.restype = dp
@@ -239,8 +242,22 @@ def add_shared(y, s) -> np.ndarray:
     return yv
 
 
+def capacity(cf: float, T: int, K: int, N: int) -> int:
+    """Per-expert capacity ceil(cf T K / N); no limit (a huge number) for cf <= 0."""
+    return lib().orc_capacity(float(cf), T, K, N)
+
+
+def capacity_keep(sel, N: int, C: int) -> np.ndarray:
+    """Drop decisions [T, K] (1 kept, 0 dropped): rows served in order, C per expert."""
+    sl = np.ascontiguousarray(np.atleast_2d(sel), dtype=np.int32)
+    T, K = sl.shape
+    keep = np.zeros((T, K), dtype=np.uint8)
+    lib().orc_capacity_keep(T, N, K, _p(sl), int(C), _p(keep))
+    return keep
+
+
 def moe_layer(x, Wg, W1, W2, *, K, act, dtype_tag, bg=None, b1=None, b2=None, sel_scores=None,
-              threads=None, rows=None, bsel=None, S1=None, S2=None, sb1=None, sb2=None):
+              threads=None, rows=None, bsel=None, S1=None, S2=None, sb1=None, sb2=None, keep=None):
     """The whole layer on host arrays, in fp64.
 
     x [T, D]; Wg [D, N]; W1 [N, H, D] (GELU) or [N, 2H, D] (SwiGLU); W2 [N, D, H].
@@ -249,6 +266,7 @@ def moe_layer(x, Wg, W1, W2, *, K, act, dtype_tag, bg=None, b1=None, b2=None, se
     sel_scores [T, N] float32 (optional): make the expert selection on these scores
     (the device's fp32 logits, plus any selection bias in fp32) while the gate
     weights use the fp64 scores.
+    keep [T, K] uint8 (optional): capacity decisions (capacity_keep); dropped slots add nothing.
     rows: optional (t0, t1) range; other rows of the outputs are left as zeros.
     Returns dict(scores [T,N], sel [T,K], w [T,K], y [T,D]) in fp64 / int32.
     """
@@ -261,6 +279,7 @@ def moe_layer(x, Wg, W1, W2, *, K, act, dtype_tag, bg=None, b1=None, b2=None, se
     W1m = _mat(W1, dtype_tag)
     bgm, b1m, b2m = _c(bg, np.float32), _c(b1, np.float32), _c(b2, np.float32)
     ss = _c(sel_scores, np.float32)
+    kp = _c(keep, np.uint8)
     bselm, S1m, S2m = _c(bsel, np.float32), _mat(S1, dtype_tag), _mat(S2, dtype_tag)
     sb1m, sb2m = _c(sb1, np.float32), _c(sb2, np.float32)
     lay = _Layer(D, H, N, K, act, dtype_tag, _p(xm), _p(Wgm), _p(bgm), _p(W1m), _p(b1m), _p(W2m), _p(b2m),
@@ -278,7 +297,7 @@ def moe_layer(x, Wg, W1, W2, *, K, act, dtype_tag, bg=None, b1=None, b2=None, se
     ranges = [(a, min(a + step, t1)) for a in range(t0, t1, step)]
 
     def run(r):
-        L.orc_moe_layer_rows(ctypes.byref(lay), r[0], r[1], _p(ss), _p(scores), _p(sel), _p(w), _p(y))
+        L.orc_moe_layer_rows(ctypes.byref(lay), r[0], r[1], _p(ss), _p(kp), _p(scores), _p(sel), _p(w), _p(y))
 
     if nthr == 1 or len(ranges) == 1:
         for r in ranges:
@@ -287,6 +306,20 @@ def moe_layer(x, Wg, W1, W2, *, K, act, dtype_tag, bg=None, b1=None, b2=None, se
         with ThreadPoolExecutor(nthr) as ex:
             list(ex.map(run, ranges))
     return dict(scores=scores, sel=sel, w=w, y=y)
+
+
+def moe_layer_capacity(x, Wg, W1, W2, *, K, act, dtype_tag, cf, sel_scores=None, **kw):
+    """The layer with a per-expert capacity (drop): route every token, decide which
+    assignments fit (rows in order, C = capacity(cf, T, K, N) each), then evaluate."""
+    routed = moe_layer(x, Wg, np.zeros_like(W1), np.zeros_like(W2), K=K, act=act, dtype_tag=dtype_tag,
+                       sel_scores=sel_scores, **{k: v for k, v in kw.items() if k in ("bg", "bsel", "threads")})
+    T = routed["sel"].shape[0]
+    N = _mat(Wg, dtype_tag).shape[1]
+    C = capacity(cf, T, K, N)
+    keep = capacity_keep(routed["sel"], N, C)
+    out = moe_layer(x, Wg, W1, W2, K=K, act=act, dtype_tag=dtype_tag, sel_scores=sel_scores, keep=keep, **kw)
+    out["keep"], out["capacity"] = keep, C
+    return out
 
 
 # --- statistics ---------------------------------------------------------------------------------------

@@ -250,6 +250,39 @@ void orc_expert(const orc_layer *L, int64_t e, const double *x_row, double *hid,
 }
 
 /* ------------------------------------------------------------------------
+ * Capacity.  "MoE(Mixture of Experts)", design notes (capacity factor): real
+ * layers give each expert an upper limit on the tokens it accepts; what
+ * overflows is dropped or passed to the next candidate.  Readings: the limit
+ * is C = ceil(cf * T * K / N) (the expected number of assignments per expert
+ * times the capacity factor cf; computed in double); cf <= 0 means no limit.
+ * ---------------------------------------------------------------------- */
+int64_t orc_capacity(double cf, int64_t T, int64_t K, int64_t N) {
+    if (cf <= 0.0) return INT64_MAX;
+    return (int64_t)ceil(cf * (double)T * (double)K / (double)N);
+}
+
+/* Drop: the rows are served in order (the chapter's Forward visits rows
+ * r = 0, 1, ...) and each of a row's K assignments is accepted when its expert
+ * has accepted fewer than C so far; keep[t*K + j] = 1 for an accepted
+ * assignment, 0 for a dropped one.  A dropped assignment contributes nothing
+ * to y (the kept weights are not renormalised). */
+void orc_capacity_keep(int64_t T, int64_t N, int64_t K, const int32_t *sel, int64_t C, uint8_t *keep) {
+    int64_t *load = (int64_t *)calloc((size_t)N, sizeof(int64_t));
+    for (int64_t t = 0; t < T; ++t) {
+        for (int64_t j = 0; j < K; ++j) {
+            const int32_t e = sel[t * K + j];
+            if (load[e] < C) {
+                load[e] += 1;
+                keep[t * K + j] = 1;
+            } else {
+                keep[t * K + j] = 0;
+            }
+        }
+    }
+    free(load);
+}
+
+/* ------------------------------------------------------------------------
  * Shared expert.  "MoE(Mixture of Experts)", design notes (merits and
  * examples): the fine-grained MoE of DeepSeek-V3 adds to the many small routed
  * experts a shared part that every token passes through.  Read here as one
@@ -278,6 +311,8 @@ void orc_add_shared(int64_t D, const double *s, double *y) {
  *       s_e + bsel_e, and the gate weights are softmax(KeepTopK) of the raw
  *       scores s over that kept set; the statistics use the raw scores.
  *   S1/S2 (optional): the shared expert, added after the routed sum.
+ *   keep [T, K] (optional): capacity decisions (orc_capacity_keep); a slot
+ *       with keep 0 is not evaluated and adds nothing.
  *   scores_out [T, N]: fp64 router scores.
  *   sel_scores [T, N] (optional): if given, the expert selection is made on
  *       these scores instead of the fp64 s + bsel (used to apply the oracle's
@@ -288,7 +323,7 @@ void orc_add_shared(int64_t D, const double *s, double *y) {
  * separate threads.
  * ---------------------------------------------------------------------- */
 void orc_moe_layer_rows(const orc_layer *L, int64_t t0, int64_t t1,
-                        const float *sel_scores, double *scores_out,
+                        const float *sel_scores, const uint8_t *keep, double *scores_out,
                         int32_t *sel_out, double *w_out, double *y_out) {
     int64_t D = L->D, H = L->H, N = L->N, K = L->K;
     double *x_row = (double *)malloc(sizeof(double) * (size_t)D);
@@ -309,7 +344,13 @@ void orc_moe_layer_rows(const orc_layer *L, int64_t t0, int64_t t1,
         }
         orc_select_topk(N, K, tmp, sel);
         orc_gate_weights(N, K, s, sel, w);
-        for (int64_t j = 0; j < K; ++j) orc_expert(L, sel[j], x_row, hid, E + j * D);
+        for (int64_t j = 0; j < K; ++j) {
+            if (keep && !keep[t * K + j]) {
+                for (int64_t c = 0; c < D; ++c) E[j * D + c] = 0.0;   /* dropped: no contribution */
+                continue;
+            }
+            orc_expert(L, sel[j], x_row, hid, E + j * D);
+        }
         orc_combine(K, D, w, E, y_out + t * D);
         if (L->S1) {
             orc_shared_expert(L, x_row, hid, sh);

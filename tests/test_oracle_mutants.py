@@ -71,9 +71,16 @@ MUTANTS = [
      [pins.test_one_expert_with_shared_expert_is_two_dense_ffns]),
     ("selection_bias_ignored", "tmp[e] = s[e] + (L->bsel ? (double)L->bsel[e] : 0.0);", "tmp[e] = s[e];",
      [pins.test_selection_bias_changes_the_kept_set_not_the_weights]),
-    ("selection_bias_in_weights", "        orc_gate_weights(N, K, s, sel, w);\n        for (int64_t j = 0; j < K; ++j) orc_expert",
-     "        orc_gate_weights(N, K, tmp, sel, w);\n        for (int64_t j = 0; j < K; ++j) orc_expert",
+    ("selection_bias_in_weights", "        orc_gate_weights(N, K, s, sel, w);\n        for (int64_t j = 0; j < K; ++j) {",
+     "        orc_gate_weights(N, K, tmp, sel, w);\n        for (int64_t j = 0; j < K; ++j) {",
      [pins.test_selection_bias_changes_the_kept_set_not_the_weights]),
+    ("capacity_floor", "return (int64_t)ceil(cf * (double)T * (double)K / (double)N);",
+     "return (int64_t)floor(cf * (double)T * (double)K / (double)N);",
+     [pins.test_capacity_closed_forms]),
+    ("capacity_off_by_one", "if (load[e] < C) {", "if (load[e] <= C) {",
+     [pins.test_capacity_keeps_the_first_C_of_each_expert_in_row_order]),
+    ("dropped_slot_still_added", "            if (keep && !keep[t * K + j]) {", "            if (0) {",
+     [pins.test_capacity_layer_is_the_masked_dense_gate]),
     ("p_mean_not_averaged", "for (int64_t e = 0; e < N; ++e) p_mean[e] /= (double)T;",
      "for (int64_t e = 0; e < N; ++e) p_mean[e] /= 1.0;",
      [pins.test_aux_stats_invariants_and_library_checks]),

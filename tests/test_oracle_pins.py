@@ -315,6 +315,77 @@ def test_selection_bias_changes_the_kept_set_not_the_weights():
     assert np.any(out["w"][:, 0] < 0.5)
 
 
+# --------------------------------------------------------------------------- capacity (drop)
+def test_capacity_closed_forms():
+    """C = ceil(cf T K / N): the expected assignments per expert times the capacity factor."""
+    assert oracle.capacity(1.25, 16384, 8, 256) == 640        # 512 per expert x 1.25
+    assert oracle.capacity(1.0, 8192, 2, 6) == 2731          # 2730.67 rounded up
+    assert oracle.capacity(2.0, 10, 2, 8) == 5
+    assert oracle.capacity(0.5, 7, 1, 7) == 1                # 0.5 rounded up
+    assert oracle.capacity(0.0, 100, 2, 4) >= 2 ** 62        # no limit
+
+
+def test_capacity_keeps_the_first_C_of_each_expert_in_row_order():
+    """Brute force with a library routine: for each expert, the first C of its assignments in
+    row-major (row, slot) order are kept (numpy flatnonzero), the others dropped."""
+    rng = np.random.default_rng(71)
+    T, N, K = 300, 8, 3
+    sel = np.stack([rng.permutation(N)[:K] for _ in range(T)]).astype(np.int32)
+    sel[:40, 0] = 2                                            # a burst on expert 2
+    for C in (1, 7, 50, 113, 1000):
+        keep = oracle.capacity_keep(sel, N, C)
+        ref = np.zeros(T * K, dtype=np.uint8)
+        flat = sel.ravel()
+        for e in range(N):
+            ref[np.flatnonzero(flat == e)[:C]] = 1
+        np.testing.assert_array_equal(keep.ravel(), ref)
+        counts = np.bincount(flat, minlength=N)
+        np.testing.assert_array_equal(np.bincount(flat, weights=keep.ravel(), minlength=N), np.minimum(counts, C))
+
+
+def test_capacity_layer_is_the_masked_dense_gate():
+    """Brute force: every expert evaluated, weighted by the dense gate softmax(KeepTopK) times the
+    keep mask of the capacity decision, summed; equals the capacity layer (library routines)."""
+    rng = np.random.default_rng(73)
+    T, D, H, N, K = 60, 10, 16, 5, 2
+    x, Wg, W1, W2, b1, b2 = _rand_layer(rng, T, D, H, N, oracle.ACT_SWIGLU, False)
+    bg = np.array([1.5, 0.5, 0.0, -0.5, -1.0], np.float32)   # skewed: expert 0 overflows
+    out = oracle.moe_layer_capacity(x, Wg, W1, W2, K=K, act=oracle.ACT_SWIGLU, dtype_tag=oracle.F32, cf=0.8,
+                                    bg=bg, threads=2)
+    C = out["capacity"]
+    assert C == math.ceil(0.8 * T * K / N)
+    x64 = torch.from_numpy(x.astype(np.float64))
+    logits = x64 @ torch.from_numpy(Wg.astype(np.float64)) + torch.from_numpy(bg.astype(np.float64))
+    order = torch.sort(-logits, dim=1, stable=True).indices[:, :K]
+    masked = torch.full_like(logits, -math.inf)
+    masked.scatter_(1, order, logits.gather(1, order))
+    G = torch.softmax(masked, dim=1)
+    keep = np.zeros((T, N))
+    flat = order.numpy().ravel()
+    for e in range(N):
+        idx = np.flatnonzero(flat == e)[:C]
+        keep[idx // K, e] = 1.0
+    assert keep.sum() < T * K                                  # something was dropped
+    y = torch.zeros(T, D, dtype=torch.float64)
+    for e in range(N):
+        Ee = _torch_expert(x64, oracle.ACT_SWIGLU, W1[e], W2[e], None, None, H)
+        y += (G[:, e:e + 1] * torch.from_numpy(keep[:, e:e + 1])) * Ee
+    np.testing.assert_allclose(out["y"], y.numpy(), rtol=1e-12, atol=1e-13)
+    # the kept gate weights are the unrenormalised ones of the plain layer
+    plain = oracle.moe_layer(x, Wg, W1, W2, K=K, act=oracle.ACT_SWIGLU, dtype_tag=oracle.F32, bg=bg, threads=2)
+    np.testing.assert_array_equal(out["w"], plain["w"])
+
+
+def test_large_capacity_is_the_plain_layer():
+    rng = np.random.default_rng(79)
+    x, Wg, W1, W2, b1, b2 = _rand_layer(rng, 40, 8, 16, 4, oracle.ACT_GELU, True)
+    a = oracle.moe_layer(x, Wg, W1, W2, K=2, act=oracle.ACT_GELU, dtype_tag=oracle.F32, b1=b1, b2=b2, threads=1)
+    b = oracle.moe_layer_capacity(x, Wg, W1, W2, K=2, act=oracle.ACT_GELU, dtype_tag=oracle.F32, cf=4.0, b1=b1,
+                                  b2=b2, threads=1)
+    assert b["keep"].all()
+    np.testing.assert_array_equal(a["y"], b["y"])
+
+
 # --------------------------------------------------------------------------- statistics
 def test_balance_loss_extremes(golden_dir):
     g = _golden(golden_dir, "balance_loss_extremes.json")
