@@ -90,6 +90,17 @@ typedef struct {
                          routed experts' form and sizes (GELU with the same
                          has_bias, or SwiGLU) and is added with weight 1 after
                          the routed experts' slot-order sum. */
+    float capacity_factor; /* > 0: each expert accepts at most
+                         C = ceil(capacity_factor * T * K / N) assignments
+                         (computed in double) per call; 0: no limit.
+                         "MoE(Mixture of Experts)", design notes (capacity
+                         factor: overflow is dropped or sent to the next
+                         candidate).  Here overflow is dropped: rows are served
+                         in token order, an assignment is accepted while its
+                         expert holds fewer than C, and a dropped assignment
+                         adds nothing to y (the kept gate weights are not
+                         renormalised).  The statistics (moe_aux) describe the
+                         router's choice before the limit. */
 } moe_config;
 
 /* Layer parameters, all device memory.

@@ -51,6 +51,7 @@ class Workload:
     random_bias: bool = False
     n_shared: int = 0     # 1: a shared expert every token passes through
     sel_s: float = 0.0    # selection-only bias strength; 0 = none
+    capacity_factor: float = 0.0   # per-expert capacity ceil(cf T K / N); 0 = no limit
 
     @property
     def seed(self) -> int:

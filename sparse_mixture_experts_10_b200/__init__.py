@@ -44,7 +44,7 @@ EXPORTED = ("moe_workspace_size", "moe_route", "moe_forward", "moe_forward_timed
 class moe_config(ctypes.Structure):
     _fields_ = [("DModel", ctypes.c_int32), ("DHidden", ctypes.c_int32), ("NExperts", ctypes.c_int32),
                 ("TopK", ctypes.c_int32), ("act", ctypes.c_int32), ("dtype", ctypes.c_int32),
-                ("has_bias", ctypes.c_int32), ("n_shared", ctypes.c_int32)]
+                ("has_bias", ctypes.c_int32), ("n_shared", ctypes.c_int32), ("capacity_factor", ctypes.c_float)]
 
 
 class moe_weights(ctypes.Structure):
@@ -150,8 +150,9 @@ def dtype_code(dt: torch.dtype) -> int:
 
 
 def make_config(DModel, DHidden, NExperts, TopK, act=MOE_ACT_GELU, dtype=MOE_BF16, has_bias=False,
-                n_shared=0) -> moe_config:
-    return moe_config(DModel, DHidden, NExperts, TopK, act, dtype, int(bool(has_bias)), int(n_shared))
+                n_shared=0, capacity_factor=0.0) -> moe_config:
+    return moe_config(DModel, DHidden, NExperts, TopK, act, dtype, int(bool(has_bias)), int(n_shared),
+                      float(capacity_factor))
 
 
 def make_weights(W_g, W1, W2, b_g=None, b1=None, b2=None, b_sel=None, S1=None, sb1=None, S2=None,

@@ -20,6 +20,7 @@
 #include "moe_router_tc.cuh"
 
 #include <algorithm>
+#include <cmath>
 #include <atomic>
 #include <mutex>
 
@@ -66,6 +67,7 @@ struct Plan {
     int route_splits;  // few-token router: W_g slabs per token
     int dec_cap;       // decode GEMMs: CTAs the stream-K partials and tickets are sized for
     int n_shared;      // 1: a shared expert (dense FFN over every token) is added after the routed sum
+    int capacity;      // assignments each expert accepts (rows served in order; the rest are dropped)
     // Counters region (zeroed on every call), 32-bit words: [0] router ticket,
     // [1] statistics ticket, [2] number of live experts, [64, 128) per-token
     // tickets of the few-token router; from byte 512 the stream-K tile tickets
@@ -88,6 +90,7 @@ int make_plan(const moe_config *c, int64_t T, Plan *p) {
     if (c->dtype != MOE_F32 && c->dtype != MOE_BF16) return MOE_ERR_INVALID_ARG;
     if (c->has_bias && c->act != MOE_ACT_GELU) return MOE_ERR_UNSUPPORTED;
     if (c->n_shared != 0 && c->n_shared != 1) return MOE_ERR_INVALID_ARG;
+    if (!(c->capacity_factor >= 0.0f) || c->capacity_factor > 1.0e6f) return MOE_ERR_INVALID_ARG;   // NaN too
     const int es = c->dtype == MOE_F32 ? 4 : 2;
     const int vec = 16 / es;
     if (D % vec || H % vec) return MOE_ERR_INVALID_ARG;
@@ -99,6 +102,13 @@ int make_plan(const moe_config *c, int64_t T, Plan *p) {
     p->D = (int)D; p->H = (int)H; p->N = (int)N; p->K = (int)K;
     p->act = c->act; p->dtype = c->dtype; p->has_bias = c->has_bias ? 1 : 0; p->es = es;
     p->n_shared = c->n_shared;
+    // C = ceil(cf T K / N) in double; no limit without a capacity factor
+    if (c->capacity_factor > 0.0f) {
+        const double cap = std::ceil((double)c->capacity_factor * (double)T * (double)K / (double)N);
+        p->capacity = cap >= (double)INT32_MAX ? INT32_MAX : (int)cap;
+    } else {
+        p->capacity = INT32_MAX;
+    }
     p->np = N <= 8 ? 8 : N <= 16 ? 16 : 32;
     const bool fits = N <= 32 && (size_t)p->np * D * es + 256 <= kSmallRouterSmemMax;
     p->rowdot_router = N <= 32 && (T < kRowdotMaxT || !fits);
@@ -420,6 +430,7 @@ int stage_route_tc(const Plan &P, const Bufs &b, const void *x, const moe_weight
     p.live = b.at<int>(P.live);
     p.n_live = b.at<int>(P.counters) + 2;
     p.counts_out = counts_out;
+    p.capacity = P.capacity;
     if (aux) {
         p.aux_counts = aux->counts;
         p.aux_importance = aux->importance;
@@ -558,7 +569,7 @@ int stage_route(const Plan &P, const Bufs &b, const void *x, const moe_weights *
 
 int stage_scan(const Plan &P, const Bufs &b, int *counts_out, cudaStream_t s) {
     scan_kernel<<<(unsigned)cdiv(P.N, 32), 1024, 0, s>>>(
-        b.at<int>(P.chunk_counts), P.n_chunks, P.N, P.T * P.K, b.at<int>(P.chunk_base), b.at<int>(P.counts),
+        b.at<int>(P.chunk_counts), P.n_chunks, P.N, P.T * P.K, P.capacity, b.at<int>(P.chunk_base), b.at<int>(P.counts),
         b.at<int>(P.offsets), b.at<int>(P.row_offsets), b.at<int>(P.perm_slot), counts_out, b.at<unsigned>(P.counters),
         b.at<int>(P.live), b.at<int>(P.counters) + 2);
     return check_launch();
@@ -568,17 +579,18 @@ int stage_scan(const Plan &P, const Bufs &b, int *counts_out, cudaStream_t s) {
 // down projection), else null.
 int stage_permute(const Plan &P, const Bufs &b, const void *x, float *y_zero, const DeviceInfo &dev,
                   cudaStream_t s) {
-    const size_t smem = (size_t)(P.N + P.chunk_tokens * P.K) * 4;
+    const size_t smem = (size_t)(2 * P.N + P.chunk_tokens * P.K) * 4;
     // enough blocks to keep every SM copying: split each chunk's rows over several blocks
     const int split = (int)std::max<int64_t>(1, std::min<int64_t>(8, cdiv(2 * dev.sms, P.n_chunks)));
     const dim3 grid((unsigned)P.n_chunks, (unsigned)split);
     if (P.dtype == MOE_F32)
         return launch_pdl(permute_kernel<float>, grid, dim3(256), smem, s, static_cast<const float *>(x), (int)P.T, P.D,
-                          P.K, P.N, P.chunk_tokens, (const int *)b.at<int>(P.idx), (const int *)b.at<int>(P.chunk_base),
+                          P.K, P.N, P.chunk_tokens, P.capacity, (const int *)b.at<int>(P.idx),
+                          (const int *)b.at<int>(P.chunk_base),
                           (const int *)b.at<int>(P.row_offsets), b.at<int>(P.perm_slot), b.at<int>(P.slot_row),
                           b.at<float>(P.x_perm), y_zero);
     return launch_pdl(permute_kernel<__nv_bfloat16>, grid, dim3(256), smem, s, static_cast<const __nv_bfloat16 *>(x),
-                      (int)P.T, P.D, P.K, P.N, P.chunk_tokens, (const int *)b.at<int>(P.idx),
+                      (int)P.T, P.D, P.K, P.N, P.chunk_tokens, P.capacity, (const int *)b.at<int>(P.idx),
                       (const int *)b.at<int>(P.chunk_base), (const int *)b.at<int>(P.row_offsets),
                       b.at<int>(P.perm_slot), b.at<int>(P.slot_row), b.at<__nv_bfloat16>(P.x_perm), y_zero);
 }
@@ -937,14 +949,16 @@ int stage_shared_down(const Plan &P, const Bufs &b, const moe_weights *w, const 
 int stage_combine(const Plan &P, const Bufs &b, void *y, int y_dtype, const DeviceInfo &dev, cudaStream_t s) {
     const int64_t nq = P.T * (P.D / 4);
     const int grid = (int)std::min<int64_t>(cdiv(nq, 256), (int64_t)dev.sms * 8);
-    // bf16 prefill layers keep z in the permuted row order (see stage_down)
-    const int *slot_row = P.dtype == MOE_BF16 && !P.decode ? b.at<int>(P.slot_row) : nullptr;
+    // bf16 prefill layers keep z in the permuted row order (see stage_down); every
+    // layer marks the slots the capacity limit dropped with slot_row -1
+    const int *slot_row = b.at<int>(P.slot_row);
+    const int z_by_row = P.dtype == MOE_BF16 && !P.decode ? 1 : 0;
     const float *shared = P.n_shared ? b.at<float>(P.s_out) : nullptr;
     if (y_dtype == MOE_F32)
         return launch_pdl(combine_kernel<float>, dim3(grid), dim3(256), 0, s, (const float *)b.at<float>(P.z), P.T, P.D,
-                          P.K, slot_row, shared, static_cast<float *>(y));
+                          P.K, slot_row, z_by_row, shared, static_cast<float *>(y));
     return launch_pdl(combine_kernel<__nv_bfloat16>, dim3(grid), dim3(256), 0, s, (const float *)b.at<float>(P.z), P.T,
-                      P.D, P.K, slot_row, shared, static_cast<__nv_bfloat16 *>(y));
+                      P.D, P.K, slot_row, z_by_row, shared, static_cast<__nv_bfloat16 *>(y));
 }
 
 int stage_aux(const Plan &P, const Bufs &b, const float *logits, const int *idx, const float *tw, moe_aux *aux,

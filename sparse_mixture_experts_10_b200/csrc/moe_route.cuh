@@ -363,7 +363,7 @@ __global__ void __launch_bounds__(256) topk_kernel(const float *__restrict__ log
 // counts at once.  *counter must be 0 at launch.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(1024) scan_kernel(const int *__restrict__ chunk_counts, int n_chunks, int N,
-                                                    int64_t expect_total, int *__restrict__ chunk_base,
+                                                    int64_t expect_total, int capacity, int *__restrict__ chunk_base,
                                                     int *__restrict__ counts, int *__restrict__ offsets,
                                                     int *__restrict__ row_offsets, int *__restrict__ perm_slot,
                                                     int *__restrict__ counts_out, unsigned *__restrict__ counter,
@@ -372,6 +372,7 @@ __global__ void __launch_bounds__(1024) scan_kernel(const int *__restrict__ chun
     __shared__ int s_cnt[1024];
     __shared__ int s_row[1025];
     __shared__ bool s_last;
+    __shared__ int s_routed;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int e = blockIdx.x * 32 + warp;
     if (e < N) {
@@ -402,11 +403,23 @@ __global__ void __launch_bounds__(1024) scan_kernel(const int *__restrict__ chun
     }
     __threadfence();
     __syncthreads();
-    if (tid == 0) s_last = atomicAdd(counter, 1u) == gridDim.x - 1;
+    if (tid == 0) {
+        s_last = atomicAdd(counter, 1u) == gridDim.x - 1;
+        s_routed = 0;
+    }
     __syncthreads();
     if (!s_last) return;
     __threadfence();
-    for (int i = tid; i < N; i += blockDim.x) s_cnt[i] = __ldcg(counts + i);
+    int routed = 0;
+    for (int i = tid; i < N; i += blockDim.x) {
+        const int c = __ldcg(counts + i);
+        if (counts_out) counts_out[i] = c;          // the router's choice
+        routed += c;
+        s_cnt[i] = min(c, capacity);                // rows each expert accepts
+        counts[i] = s_cnt[i];
+    }
+    routed = __reduce_add_sync(0xffffffffu, routed);
+    if (lane == 0 && routed) atomicAdd(&s_routed, routed);
     __syncthreads();
     if (warp == 0) {
         int carry = 0, pcarry = 0;
@@ -422,7 +435,6 @@ __global__ void __launch_bounds__(1024) scan_kernel(const int *__restrict__ chun
                 if (lane >= o) { ic += n1; ip += n2; }
             }
             if (ee < N) {
-                if (counts_out) counts_out[ee] = c;
                 offsets[ee] = carry + ic - c;
                 row_offsets[ee] = pcarry + ip - pc;
                 s_row[ee] = pcarry + ip - pc;
@@ -434,7 +446,7 @@ __global__ void __launch_bounds__(1024) scan_kernel(const int *__restrict__ chun
             offsets[N] = carry;
             row_offsets[N] = pcarry;
             s_row[N] = pcarry;
-            if ((int64_t)carry != expect_total) set_status(kStatusBounds);
+            if ((int64_t)s_routed != expect_total) set_status(kStatusBounds);
         }
         // ascending list of the experts that received tokens
         int nl = 0;
@@ -464,15 +476,16 @@ __global__ void __launch_bounds__(1024) scan_kernel(const int *__restrict__ chun
 // (c, s) copies the entries f with f % split == s.
 template <typename Tin>
 __global__ void __launch_bounds__(256) permute_kernel(const Tin *__restrict__ x, int T, int D, int K, int N,
-                                                      int chunk_tokens, const int *__restrict__ topk_idx,
+                                                      int chunk_tokens, int capacity, const int *__restrict__ topk_idx,
                                                       const int *__restrict__ chunk_base,
                                                       const int *__restrict__ row_offsets, int *__restrict__ perm_slot,
                                                       int *__restrict__ slot_row, Tin *__restrict__ x_perm,
                                                       float *__restrict__ y_zero) {
     pdl_enter();
     extern __shared__ int s_perm[];
-    int *s_run = s_perm;            // [N]
-    int *s_dest = s_perm + N;       // [chunk_tokens * K]
+    int *s_run = s_perm;            // [N] next position inside each expert's assignments
+    int *s_row0 = s_perm + N;       // [N] first row of each expert's segment
+    int *s_dest = s_perm + 2 * N;   // [chunk_tokens * K]
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int c = blockIdx.x;
     const bool writer = blockIdx.y == 0;
@@ -494,7 +507,10 @@ __global__ void __launch_bounds__(256) permute_kernel(const Tin *__restrict__ x,
         for (int u = 0; u < 4; ++u)
             if (lane + 32 * u < nvec) pre[u] = __ldg(src + lane + 32 * u);
     }
-    for (int e = tid; e < N; e += blockDim.x) s_run[e] = row_offsets[e] + chunk_base[(size_t)c * N + e];
+    for (int e = tid; e < N; e += blockDim.x) {
+        s_run[e] = chunk_base[(size_t)c * N + e];
+        s_row0[e] = row_offsets[e];
+    }
     __syncthreads();
     if (warp == 0) {
         for (int base = 0; base < n_entries; base += 32) {
@@ -512,7 +528,9 @@ __global__ void __launch_bounds__(256) permute_kernel(const Tin *__restrict__ x,
             if (e >= 0 && lane == leader) s_run[e] = base_row + __popc(peers);
             __syncwarp();
             if (f < n_entries) {
-                const int dest = e >= 0 ? base_row + rank : -1;
+                // the assignment's position among its expert's: accepted below the capacity
+                const int pos = base_row + rank;
+                const int dest = (e >= 0 && pos < capacity) ? s_row0[e] + pos : -1;
                 s_dest[f] = dest;
                 if (writer) {
                     if (dest >= 0) perm_slot[dest] = (int)(f0 + f);
@@ -573,24 +591,32 @@ __global__ void __launch_bounds__(256) zero_kernel(uint4 *__restrict__ p, int64_
 // adds the weighted expert outputs of a row in selection order); then, with a
 // shared expert, + s[t] (its output, added after the routed sum).
 // ---------------------------------------------------------------------------
+// slot_row: the permuted row of each slot, -1 for a slot dropped by the
+// capacity limit (it adds nothing); z_by_row: z rows are permuted rows (bf16
+// prefill) rather than slots.
 template <typename Tout>
 __global__ void __launch_bounds__(256) combine_kernel(const float *__restrict__ z, int64_t T, int D, int K,
-                                                      const int *__restrict__ slot_row,
+                                                      const int *__restrict__ slot_row, int z_by_row,
                                                       const float *__restrict__ shared, Tout *__restrict__ y) {
     pdl_enter();
     const int64_t nq = T * (D / 4);
     for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < nq; i += (int64_t)gridDim.x * blockDim.x) {
         const int64_t t = i / (D / 4);
         const int d = (int)(i - t * (D / 4)) * 4;
-        // z row of slot (t, j): t*K + j, or its permuted row when slot_row is given
-        auto zrow = [&](int j) -> const float * {
-            const int64_t r = slot_row ? (int64_t)__ldg(slot_row + t * K + j) : t * K + j;
-            return z + r * D + d;
-        };
-        float4 acc = *reinterpret_cast<const float4 *>(zrow(0));
-        for (int j = 1; j < K; ++j) {
-            const float4 v = *reinterpret_cast<const float4 *>(zrow(j));
-            acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+        // z row of slot (t, j): its permuted row or t*K + j; -1 when the slot was dropped
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        bool first = true;
+        for (int j = 0; j < K; ++j) {
+            const int rr = __ldg(slot_row + t * K + j);
+            if (rr < 0) continue;
+            const int64_t r = z_by_row ? (int64_t)rr : t * K + j;
+            const float4 v = *reinterpret_cast<const float4 *>(z + r * D + d);
+            if (first) {
+                acc = v;
+                first = false;
+            } else {
+                acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+            }
         }
         if (shared) {
             const float4 v = *reinterpret_cast<const float4 *>(shared + t * D + d);

@@ -61,6 +61,7 @@ struct Params {
     int *live;                           // [N]
     int *n_live;
     int *counts_out;                     // [N] or nullptr (moe_route)
+    int capacity;                        // rows each expert accepts (assignments beyond are dropped)
     // statistics (each may be nullptr)
     int *aux_counts;
     float *aux_importance, *aux_p_mean, *aux_scalars;
@@ -149,8 +150,10 @@ __device__ void finalize_tables(const Params &p, int ntiles, FinalScratch &f, in
         }
         __syncthreads();
     }
+    // the dispatch tables hold each expert's accepted rows, min(count, capacity);
+    // the statistics and moe_route's counts the router's own choice
     for (int e = tid; e < N; e += nt) {
-        p.counts[e] = f.cnt[e];
+        p.counts[e] = min(f.cnt[e], p.capacity);
         if (p.counts_out) p.counts_out[e] = f.cnt[e];
         if (p.aux_counts) p.aux_counts[e] = f.cnt[e];
         if (p.aux_p_mean) p.aux_p_mean[e] = f.pm[e];
@@ -158,9 +161,11 @@ __device__ void finalize_tables(const Params &p, int ntiles, FinalScratch &f, in
     }
     if (warp == 0) {
         int carry = 0, pcarry = 0, nl = 0;
+        int routed = 0;
         for (int e0 = 0; e0 < N; e0 += 32) {
             const int e = e0 + lane;
-            const int c = e < N ? f.cnt[e] : 0;
+            routed += e < N ? f.cnt[e] : 0;
+            const int c = e < N ? min(f.cnt[e], p.capacity) : 0;
             const int pc = (c + kRowAlign - 1) / kRowAlign * kRowAlign;
             int ic = c, ip = pc;
 #pragma unroll
@@ -185,7 +190,10 @@ __device__ void finalize_tables(const Params &p, int ntiles, FinalScratch &f, in
             p.row_offsets[N] = pcarry;
             f.row[N] = pcarry;
             *p.n_live = nl;
-            if ((int64_t)carry != (int64_t)p.T * p.K) set_status(kStatusBounds);
+        }
+        routed = __reduce_add_sync(0xffffffffu, routed);
+        if (lane == 0) {
+            if ((int64_t)routed != (int64_t)p.T * p.K) set_status(kStatusBounds);
         }
     } else if (warp == 1 && p.aux_scalars) {
         // f_e = counts_e / (T K); switch = N sum f P; simple = N sum f^2;
@@ -229,7 +237,7 @@ __device__ void finalize_tables(const Params &p, int ntiles, FinalScratch &f, in
     }
     __syncthreads();
     for (int e = warp; worker && e < N; e += nt / 32) {
-        const int start = f.row[e] + f.cnt[e], end = f.row[e + 1];
+        const int start = f.row[e] + min(f.cnt[e], p.capacity), end = f.row[e + 1];
         for (int rr = start + lane; rr < end; rr += 32) p.perm_slot[rr] = -1;
     }
 }

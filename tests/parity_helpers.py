@@ -68,13 +68,21 @@ def shared_kwargs(inp):
     return dict(S1=host(inp.get("S1")), S2=host(inp.get("S2")), sb1=host(inp.get("sb1")), sb2=host(inp.get("sb2")))
 
 
+def capacity_factor(wl) -> float:
+    """The capacity factor as the library receives it (an fp32 field), widened to double."""
+    return float(np.float32(wl.capacity_factor))
+
+
 def oracle_full_layer(inp, wl, K, gpu_logits=None, threads=None):
-    """The whole layer on every token (small workloads)."""
+    """The whole layer on every token (small workloads); with the workload's capacity when it has one."""
     t = tag(wl.dtype)
     sel = None if gpu_logits is None else selection_scores(gpu_logits, inp)
-    return oracle.moe_layer(host(inp["x"]), host(inp["W_g"]), host(inp["W1"]), host(inp["W2"]), K=K, act=wl.act,
-                            dtype_tag=t, bg=host(inp["b_g"]), b1=host(inp["b1"]), b2=host(inp["b2"]),
-                            sel_scores=sel, threads=threads, bsel=host(inp.get("b_sel")), **shared_kwargs(inp))
+    args = (host(inp["x"]), host(inp["W_g"]), host(inp["W1"]), host(inp["W2"]))
+    kw = dict(K=K, act=wl.act, dtype_tag=t, bg=host(inp["b_g"]), b1=host(inp["b1"]), b2=host(inp["b2"]),
+              sel_scores=sel, threads=threads, bsel=host(inp.get("b_sel")), **shared_kwargs(inp))
+    if wl.capacity_factor > 0:
+        return oracle.moe_layer_capacity(*args, cf=capacity_factor(wl), **kw)
+    return oracle.moe_layer(*args, **kw)
 
 
 def oracle_rows(inp, wl, K, rows, gpu_logits, threads=None):

@@ -35,7 +35,7 @@ def test_every_declared_function_is_exported(lib):
 
 
 def test_struct_sizes_match_header_layout():
-    assert ctypes.sizeof(moe.moe_config) == 8 * 4
+    assert ctypes.sizeof(moe.moe_config) == 9 * 4
     assert ctypes.sizeof(moe.moe_weights) == 11 * 8
     assert ctypes.sizeof(moe.moe_aux) == 4 * 8
     assert ctypes.sizeof(moe.moe_workspace_layout) == 12 * 8 + 8 + 8

@@ -36,7 +36,7 @@ class Layer:
     def __init__(self, wl: Workload, inp):
         self.wl, self.inp = wl, inp
         self.cfg = moe.make_config(wl.D, wl.H, wl.N, wl.K, wl.act, moe.dtype_code(wl.dtype), wl.has_bias,
-                                   wl.n_shared)
+                                   wl.n_shared, wl.capacity_factor)
         self.w = moe.make_weights(inp["W_g"], inp["W1"], inp["W2"], inp["b_g"], inp["b1"], inp["b2"],
                                   inp.get("b_sel"), inp.get("S1"), inp.get("sb1"), inp.get("S2"), inp.get("sb2"))
 
@@ -91,26 +91,31 @@ def check_routing(V, ref_scores, K, inp):
     np.testing.assert_array_equal(V["counts"], np.bincount(sel.ravel(), minlength=N))
 
 
-def check_dispatch(V, x, K):
-    """The permutation is the stable counting sort of the (token, slot) pairs by expert."""
+def check_dispatch(V, x, K, C=None):
+    """The permutation is the stable counting sort of the (token, slot) pairs by expert; with a
+    capacity C each expert's segment holds its first C pairs (the oracle's drop decision) and
+    the dropped pairs have no row."""
     idx = V["idx"]
     T = idx.shape[0]
     N = V["counts"].shape[0]
-    counts = np.bincount(idx.ravel(), minlength=N)
+    flat = idx.ravel()
+    keep = np.ones(T * K, dtype=bool) if C is None else oracle.capacity_keep(idx, N, C).ravel().astype(bool)
+    counts = np.bincount(flat[keep], minlength=N)
     np.testing.assert_array_equal(V["counts"], counts)
     np.testing.assert_array_equal(V["offsets"], np.concatenate([[0], np.cumsum(counts)]))
     padded = (counts + 127) // 128 * 128
     np.testing.assert_array_equal(V["row_offsets"], np.concatenate([[0], np.cumsum(padded)]))
     ro = V["row_offsets"]
-    flat = idx.ravel()
     for e in range(N):
         seg = V["perm_slot"][ro[e]:ro[e + 1]]
-        expect = np.nonzero(flat == e)[0]
+        expect = np.nonzero((flat == e) & keep)[0]
         np.testing.assert_array_equal(seg[:counts[e]], expect)
         assert np.all(seg[counts[e]:] == -1)
         np.testing.assert_array_equal(V["slot_row"][expect], np.arange(ro[e], ro[e] + counts[e]))
-    rows = V["slot_row"]
-    tok = np.arange(T * K) // K
+    assert np.all(V["slot_row"][~keep] == -1)
+    kept = np.nonzero(keep)[0]
+    rows = V["slot_row"][kept]
+    tok = kept // K
     xp = V["x_perm"][torch.from_numpy(rows.astype(np.int64)).cuda()]
     assert torch.equal(xp, x[torch.from_numpy(tok).cuda()])
 
@@ -123,7 +128,7 @@ def run_full(wl, inp, y_dtype=torch.float32):
     ref = ph.oracle_full_layer(inp, wl, wl.K, gpu_logits=V["logits"])
     check_routing(V, ref["scores"], wl.K, inp)
     ph.assert_weights_close(V["w"], ref["w"], ref["scores"])
-    check_dispatch(V, inp["x"], wl.K)
+    check_dispatch(V, inp["x"], wl.K, ref.get("capacity"))
     errs = ph.assert_y_close(y.float().cpu().numpy(), ref["y"], wl.dtype if y_dtype == torch.float32 else y_dtype)
     return layer, y, ws, aux, V, ref, errs
 
@@ -457,6 +462,42 @@ def test_selection_bias_balances_a_skewed_router():
     cv = {k: v.std() / v.mean() for k, v in counts.items()}
     assert cv["skewed"] > 3 * cv["plain"]
     assert cv["balanced"] < 1.5 * cv["plain"]
+
+
+# ----------------------------------------------------------------------------- capacity (drop)
+CAPACITY_CASES = [
+    ("fp32_small_router", Workload("cap_f32", 60, 300, 64, 256, 8, 2, ACT_GELU, torch.float32, True, 0.05,
+                                   zipf_s=1.0, random_bias=True, capacity_factor=1.0)),
+    ("fp32_chunked_router", Workload("cap_f32c", 61, 2300, 64, 128, 16, 3, ACT_GELU, torch.float32, False, 0.05,
+                                     zipf_s=0.8, capacity_factor=1.25)),
+    ("bf16_simt_router_fused_k2", Workload("cap_k2", 62, 1500, 256, 512, 6, 2, ACT_GELU, torch.bfloat16, True, 0.04,
+                                           zipf_s=1.0, random_bias=True, capacity_factor=1.0)),
+    ("bf16_tc_router_k4", Workload("cap_tc", 63, 1200, 256, 256, 64, 4, ACT_SWIGLU, torch.bfloat16, False, 0.05,
+                                   zipf_s=1.0, capacity_factor=0.75)),
+    ("bf16_pairs_shared", Workload("cap_sh", 64, 1500, 512, 1024, 8, 2, ACT_SWIGLU, torch.bfloat16, False, 0.04,
+                                   zipf_s=0.9, n_shared=1, capacity_factor=1.0)),
+    ("decode8", WORKLOADS["decode8"].with_(zipf_s=2.0, capacity_factor=1.0)),
+    ("decode64_bias", WORKLOADS["decode64"].with_(zipf_s=1.0, sel_s=0.5, capacity_factor=0.5)),
+    ("huge_capacity", Workload("cap_big", 65, 700, 256, 256, 8, 2, ACT_SWIGLU, torch.bfloat16, False, 0.05,
+                               zipf_s=0.5, capacity_factor=8.0)),
+]
+
+
+@pytest.mark.parametrize("name,wl", CAPACITY_CASES, ids=[c[0] for c in CAPACITY_CASES])
+def test_capacity_drop(name, wl):
+    """Per-expert capacity with drop: each expert's segment holds its first C assignments in token
+    order (bit-exact against the oracle's decision on the device's routing), the dropped slots add
+    nothing, and the statistics still describe the router's own choice."""
+    inp = make_inputs(wl, "cuda")
+    layer, y, ws, aux, V, ref, errs = run_full(wl, inp)
+    check_aux(aux, V, wl.N, wl.K)
+    C = ref["capacity"]
+    assert C == int(np.ceil(ph.capacity_factor(wl) * wl.T * wl.K / wl.N))
+    dropped = int((ref["keep"] == 0).sum())
+    if name == "huge_capacity":
+        assert dropped == 0
+    else:
+        assert dropped > 0, "the case should overflow some expert"
 
 
 # ----------------------------------------------------------------------------- data parallelism
