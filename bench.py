@@ -107,7 +107,25 @@ def parse(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle sample")
     ap.add_argument("--ref-seconds", type=float, default=150.0,
                     help="target CPU time of the whole --impl reference run (all steps)")
+    ap.add_argument("--tokens", type=int, default=0,
+                    help="reduced case for profiling: override the workload's token count")
+    ap.add_argument("--experts", type=int, default=0,
+                    help="reduced case for profiling: override the number of experts (tokens per expert kept "
+                         "when --tokens is scaled with it)")
     return ap.parse_args(argv)
+
+
+def workload_from_args(args):
+    """The named workload, or its reduced profiling case (--tokens / --experts)."""
+    wl = WORKLOADS[args.workload]
+    kw = {}
+    if args.tokens:
+        kw["T"] = args.tokens
+    if args.experts:
+        kw["N"] = args.experts
+    if kw:
+        wl = wl.with_(name=f"{wl.name}[" + ",".join(f"{k}={v}" for k, v in kw.items()) + "]", **kw)
+    return wl
 
 
 def peaks():
@@ -437,7 +455,7 @@ def e2e_pipelined(moe, cfg, W, ws, wl, T, x_host, steps, warm, flush, dev, aux_b
 
 def main():
     args = parse()
-    wl = WORKLOADS[args.workload]
+    wl = workload_from_args(args)
     if args.impl == "reference":
         run_reference(args, wl)
         return

@@ -13,6 +13,7 @@
 // excepted, which synchronises the device).
 #include "../../include/moe.h"
 #include "moe_common.cuh"
+#include "moe_decode_fused.cuh"
 #include "moe_gemm_simt.cuh"
 #include "moe_gemm_decode.cuh"
 #include "moe_gemm_tc.cuh"
@@ -68,17 +69,21 @@ struct Plan {
     int dec_cap;       // decode GEMMs: CTAs the stream-K partials and tickets are sized for
     int n_shared;      // 1: a shared expert (dense FFN over every token) is added after the routed sum
     int capacity;      // assignments each expert accepts (rows served in order; the rest are dropped)
+    bool fused_decode; // few tokens, N <= 32, no shared expert: the whole layer in one cooperative kernel
+    int slab_rows, n_slabs;   // fused decode: W_g rows per routing slab, slabs
     // Counters region (zeroed on every call), 32-bit words: [0] router ticket,
     // [1] statistics ticket, [2] number of live experts, [64, 128) per-token
     // tickets of the few-token router; from byte 512 the stream-K tile tickets
     // of the decode up- and down-projections and of the shared expert's two
-    // decode GEMMs (dec_cap each); then the routers' per-expert probability and
-    // gate-weight sums (u64, N each).
+    // decode GEMMs (dec_cap each); then the fused decode kernel's combine
+    // tickets (one per 128 output features); then the routers' per-expert
+    // probability and gate-weight sums (u64, N each).  Word 4 counts the fused
+    // decode kernel's grid barrier arrivals.
     size_t counters_bytes;
     size_t stat_sums;  // offset inside the counters region of the routers' fixed-point sums [2][N] (u64)
     size_t counters, logits, idx, w, counts, offsets, row_offsets, live, chunk_counts, chunk_base,
         perm_slot, slot_row, x_perm, h, z, wgt, aux_p, aux_i, aux_c, route_part, dec_part, shared_tbl, h_s, s_out,
-        total;
+        fd_slab, fd_tokp, total;
 };
 
 int make_plan(const moe_config *c, int64_t T, Plan *p) {
@@ -138,7 +143,7 @@ int make_plan(const moe_config *c, int64_t T, Plan *p) {
     };
     p->route_splits = p->few_router ? (int)std::min<int64_t>(rtc::kFewMaxSplits, std::max<int64_t>(1, cdiv(D, 256))) : 1;
     p->dec_cap = p->decode ? kDecodeMaxGrid : 0;
-    p->stat_sums = (512 + (size_t)4 * p->dec_cap * 4 + 7) / 8 * 8;
+    p->stat_sums = (512 + (size_t)4 * p->dec_cap * 4 + (p->decode ? (size_t)cdiv(D, 128) * 4 : 0) + 7) / 8 * 8;
     p->counters_bytes = align256(p->stat_sums + (size_t)2 * N * 8);
     p->counters = take(p->counters_bytes);
     p->logits = take((size_t)T * N * 4);
@@ -168,6 +173,13 @@ int make_plan(const moe_config *c, int64_t T, Plan *p) {
     // shared expert: its one-group dispatch table for the decode GEMMs (live = {0},
     // one live group, count T, first row 0), its hidden rows and its fp32 output
     p->shared_tbl = take(16);
+    // fused decode: routing slabs of W_g rows (a multiple of 8 rows each, at most
+    // 32 slabs) and each token's full softmax
+    p->fused_decode = p->decode && N <= dfu::kMaxN && !p->n_shared && T <= dfu::kMaxT;
+    p->slab_rows = (int)(cdiv(cdiv(D, dfu::kMaxSlabs), 8) * 8);
+    p->n_slabs = (int)cdiv(D, p->slab_rows);
+    p->fd_slab = take(p->fused_decode ? (size_t)p->n_slabs * T * 32 * 4 : 0);
+    p->fd_tokp = take(p->fused_decode ? (size_t)T * 32 * 4 : 0);
     p->h_s = take(p->n_shared ? (size_t)std::max<int64_t>(T, 1) * H * es : 0);
     p->s_out = take(p->n_shared ? (size_t)T * D * 4 : 0);
     p->total = off;
@@ -222,6 +234,13 @@ int device_info(DeviceInfo **out) {
         MOE_TRY(allow_smem(router_small_kernel<__nv_bfloat16, 32>));
         MOE_TRY(allow_smem(aux_partial_kernel));
         MOE_TRY(allow_smem(aux_partials_kernel));
+#define MOE_FUSED_ATTR(NT)                                                  \
+    MOE_TRY(allow_smem(dfu::decode_layer_kernel<NT, dec::EPI_SWIGLU>)); \
+    MOE_TRY(allow_smem(dfu::decode_layer_kernel<NT, dec::EPI_GELU>))
+        MOE_FUSED_ATTR(16);
+        MOE_FUSED_ATTR(32);
+        MOE_FUSED_ATTR(64);
+#undef MOE_FUSED_ATTR
         MOE_TRY(allow_smem(rtc::router_simt_kernel<8>));
         MOE_TRY(allow_smem(rtc::router_simt_kernel<16>));
         MOE_TRY(allow_smem(rtc::router_simt_kernel<32>));
@@ -999,6 +1018,101 @@ int zero_aux(const Plan &P, moe_aux *aux, cudaStream_t s) {
     return MOE_OK;
 }
 
+// ---------------------------------------------------------------- fused decode
+template <int NT, int EPI>
+int launch_fused(const CUtensorMap &mw1, const CUtensorMap &mxp, const CUtensorMap &mw2, const CUtensorMap &mh,
+                 const dfu::Params &p, int grid, cudaStream_t s) {
+    using S = dfu::Shape<NT, EPI>;
+    // routing scratch (R1, R3) lives in the ring before the expert phases use it
+    const size_t scratch = std::max<size_t>(((size_t)p.T * p.slab_rows + (size_t)p.slab_rows * 32 +
+                                             (size_t)(dfu::kThreads / 32) * p.T * 32) * 4,
+                                            (size_t)2 * dfu::kMaxSlots * 4);
+    if (scratch > S::kRingBytes) return MOE_ERR_UNSUPPORTED;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(dfu::kThreads);
+    cfg.dynamicSmemBytes = S::kSmem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;   // every CTA resident: the grid barriers need it
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, dfu::decode_layer_kernel<NT, EPI>, mw1, mxp, mw2, mh, p);
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+template <int EPI>
+int launch_fused_nt(int nt, const CUtensorMap &mw1, const CUtensorMap &mxp, const CUtensorMap &mw2,
+                    const CUtensorMap &mh, const dfu::Params &p, int grid, cudaStream_t s) {
+    if (nt == 16) return launch_fused<16, EPI>(mw1, mxp, mw2, mh, p, grid, s);
+    if (nt == 32) return launch_fused<32, EPI>(mw1, mxp, mw2, mh, p, grid, s);
+    return launch_fused<64, EPI>(mw1, mxp, mw2, mh, p, grid, s);
+}
+
+// The whole layer for few tokens in one cooperative kernel (moe_decode_fused.cuh).
+int stage_decode_fused(const Plan &P, const Bufs &b, const void *x, const moe_weights *w, void *y, int y_dtype,
+                       moe_aux *aux, const DeviceInfo &dev, cudaStream_t s) {
+    const int D = P.D, H = P.H, N = P.N;
+    const bool swiglu = P.act == MOE_ACT_SWIGLU;
+    const int grid = dev.sms;
+    CUtensorMap mw1, mxp, mw2, mh;
+    MOE_TRY(make_map(&mw1, w->W1, (int64_t)N * (swiglu ? 2 * H : H), D, swiglu ? 64 : 128));
+    MOE_TRY(make_map(&mxp, b.ws + P.x_perm, P.rows_cap, D, P.nt));
+    MOE_TRY(make_map(&mw2, w->W2, (int64_t)N * D, H, 128));
+    MOE_TRY(make_map(&mh, b.ws + P.h, P.rows_cap, H, P.nt));
+    dfu::Params p{};
+    p.T = (int)P.T;
+    p.D = D;
+    p.H = H;
+    p.N = N;
+    p.K = P.K;
+    p.capacity = P.capacity;
+    p.slab_rows = P.slab_rows;
+    p.n_slabs = P.n_slabs;
+    p.x = static_cast<const __nv_bfloat16 *>(x);
+    p.Wg = static_cast<const __nv_bfloat16 *>(w->W_g);
+    p.bg = w->b_g;
+    p.bsel = w->b_sel;
+    p.b1 = swiglu ? nullptr : w->b1;
+    p.b2 = swiglu ? nullptr : w->b2;
+    p.logits = b.at<float>(P.logits);
+    p.topk_idx = b.at<int>(P.idx);
+    p.topk_w = b.at<float>(P.w);
+    p.counts = b.at<int>(P.counts);
+    p.offsets = b.at<int>(P.offsets);
+    p.row_offsets = b.at<int>(P.row_offsets);
+    p.perm_slot = b.at<int>(P.perm_slot);
+    p.slot_row = b.at<int>(P.slot_row);
+    p.live = b.at<int>(P.live);
+    p.n_live = b.at<int>(P.counters) + 2;
+    p.x_perm = b.at<__nv_bfloat16>(P.x_perm);
+    p.h = b.at<__nv_bfloat16>(P.h);
+    p.z = b.at<float>(P.z);
+    p.slab = b.at<float>(P.fd_slab);
+    p.tok_p = b.at<float>(P.fd_tokp);
+    unsigned *ctr = b.at<unsigned>(P.counters);
+    p.bar = ctr + 4;
+    p.tk_up = ctr + 128;
+    p.tk_down = ctr + 128 + P.dec_cap;
+    p.tk_comb = ctr + 128 + 4 * P.dec_cap;
+    p.part = b.at<float>(P.dec_part);
+    p.split_cap = P.dec_cap;
+    p.y = y;
+    p.y_bf16 = y_dtype == MOE_BF16 ? 1 : 0;
+    if (aux) {
+        p.aux_counts = aux->counts;
+        p.aux_importance = aux->importance;
+        p.aux_p_mean = aux->p_mean;
+        p.aux_scalars = aux->scalars;
+    }
+    p.timeout_ns = kTimeoutNs;
+    if (swiglu) return launch_fused_nt<dec::EPI_SWIGLU>(P.nt, mw1, mxp, mw2, mh, p, grid, s);
+    return launch_fused_nt<dec::EPI_GELU>(P.nt, mw1, mxp, mw2, mh, p, grid, s);
+}
+
 int check_weights(const Plan &P, const moe_weights *w, bool need_experts) {
     if (!w || !w->W_g) return MOE_ERR_INVALID_ARG;
     if (!need_experts) return MOE_OK;
@@ -1049,6 +1163,15 @@ int forward_impl(const moe_config *cfg, const void *x, int64_t T, const moe_weig
     float *y_zero = combine_in_down(P, y_dtype) ? static_cast<float *>(y) : nullptr;
     MOE_TRY(rec(0));
     MOE_TRY(zero_counters(P, b, s));
+    // few tokens: the whole layer in one cooperative kernel when the device can
+    // hold one CTA per token and W_g allows the routing's 16-byte loads
+    if (P.fused_decode && dev->sms >= (int)P.T && dev->sms >= P.n_slabs && dev->sms <= P.dec_cap &&
+        aligned16(w->W_g)) {
+        for (int i = 1; i <= 3; ++i) MOE_TRY(rec(i));
+        MOE_TRY(stage_decode_fused(P, b, x, w, y, y_dtype, aux, *dev, s));
+        for (int i = 4; i <= MOE_N_STAGES; ++i) MOE_TRY(rec(i));
+        return MOE_OK;
+    }
     if (P.tc_router) {
         MOE_TRY(stage_route_tc(P, b, x, w, logits, idx, tw, nullptr, aux, y_zero, s));
         MOE_TRY(rec(1));

@@ -127,3 +127,13 @@ def test_reference_arm_line(capsys):
     assert line["ms_per_step"] > 0 and line["ms_per_layer_extrapolated"] > 0
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["value"] == line["value"]
     assert line["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def test_reduced_profiling_case_keeps_the_shape_per_expert():
+    args = bench.parse(["--workload", "deepseek", "--tokens", "2048", "--experts", "32"])
+    wl = bench.workload_from_args(args)
+    full = WORKLOADS["deepseek"]
+    assert (wl.T, wl.N, wl.D, wl.H, wl.K) == (2048, 32, full.D, full.H, full.K)
+    assert wl.T * wl.K // wl.N == full.T * full.K // full.N      # 512 assignments per expert either way
+    assert wl.name.startswith("deepseek[")
+    assert bench.workload_from_args(bench.parse([])) == WORKLOADS["deepseek"]

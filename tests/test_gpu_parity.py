@@ -382,6 +382,29 @@ def test_decode_full_layer(name):
     run_full(wl, inp)
 
 
+@pytest.mark.parametrize("name,wl", [
+    ("gpt-oss T=1", WORKLOADS["decode1"]),
+    ("gpt-oss T=8 skewed, bias, capacity", WORKLOADS["decode8"].with_(zipf_s=1.5, sel_s=0.5, capacity_factor=1.0)),
+    ("gpt-oss T=64", WORKLOADS["decode64"]),
+    ("GELU + biases, N=6, T=37", Workload("fused_gelu", 70, 37, 1024, 1024, 6, 2, ACT_GELU, torch.bfloat16, True, 0.03,
+                                         random_bias=True, zipf_s=0.3)),
+    ("ragged D/H, T=5", Workload("fused_rag", 71, 5, 1000, 712, 12, 3, ACT_SWIGLU, torch.bfloat16, False, 0.04,
+                                 zipf_s=0.5)),
+], ids=lambda v: v if isinstance(v, str) else "")
+def test_decode_layer_is_one_kernel(name, wl):
+    """Few tokens: routing, dispatch, both expert GEMMs and the combine run as one cooperative
+    kernel after the counter clear (two launches per layer call), with the same results as the
+    oracle (routing bit-exact, y within the bf16 tolerance, statistics)."""
+    inp = make_inputs(wl, "cuda")
+    layer = Layer(wl, inp)
+    layer.forward(with_aux=False)            # the device's attributes are set up once
+    n0 = moe.moe_launch_count()
+    layer.forward(with_aux=False)
+    assert moe.moe_launch_count() - n0 == 2
+    run_layer, y, ws, aux, V, ref, errs = run_full(wl, inp)
+    check_aux(aux, V, wl.N, wl.K)
+
+
 @pytest.mark.parametrize("N,K,T", [(12, 3, 300), (32, 4, 300), (6, 2, 1), (20, 4, 40), (32, 8, 64), (33, 2, 50)])
 def test_bf16_router_paths(N, K, T):
     """bf16 routers: the SIMT router with 16 and 32 padded experts (T > 64), the few-token
