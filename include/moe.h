@@ -282,6 +282,54 @@ int moe_aux_finalize(const moe_config *cfg, const int64_t *partials, moe_aux *ou
 int moe_aux_finalize_host(const moe_config *cfg, const int64_t *partials, int32_t *counts, float *importance,
                           float *p_mean, float *scalars);
 
+/* Expert parallelism ("MoE(Mixture of Experts)", design notes: spread the
+ * experts over GPUs and an all-to-all sends each token to the GPU of its
+ * experts, every layer; Transformers-v5 MoE article, expert parallelism: the
+ * experts split on dim 0).  With R ranks, rank r holds experts
+ * [r * N/R, (r+1) * N/R) (N a multiple of R) and W_g in full.  A layer call is
+ *   1. moe_ep_dispatch on every rank: route its T tokens, group the (token,
+ *      slot) pairs by the rank holding their expert (stable: (token, slot)
+ *      order inside a rank) and pack them;
+ *   2. an all-to-all of send_counts, then of send_x / send_expert / send_w
+ *      (the caller's collective, e.g. NCCL);
+ *   3. moe_ep_experts on every rank, on the rows it received;
+ *   4. the reverse all-to-all of z (same splits, reversed);
+ *   5. moe_ep_combine on every rank: each token's K rows in slot order.
+ * The result is the layer's y.  Shared experts and capacity limits are not
+ * supported on this path (MOE_ERR_UNSUPPORTED).
+ *
+ * moe_ep_dispatch: cfg is the whole layer's (N experts); x [T, D]; w holds
+ * W_g (+ b_g, b_sel); outputs, device memory:
+ *   send_x [T*K, D] dtype     the pairs' token rows, rank after rank
+ *   send_expert [T*K] int32   each pair's expert index on its rank (0..N/R-1)
+ *   send_w [T*K] fp32         each pair's gate weight
+ *   send_counts [R] int32     pairs for each rank (send_x rows rank r holds
+ *                             start at the exclusive sum of the earlier counts)
+ *   send_pos [T*K] int32      the send_x row of slot t*K + j (for the combine)
+ *   aux                       statistics of this rank's routing, or NULL
+ * ws: moe_ep_workspace_size(cfg, n_ranks, T) bytes. */
+size_t moe_ep_workspace_size(const moe_config *cfg, int32_t n_ranks, int64_t T);
+int moe_ep_dispatch(const moe_config *cfg, int32_t n_ranks, const void *x, int64_t T, const moe_weights *w,
+                    void *send_x, int32_t *send_expert, float *send_w, int32_t *send_counts, int32_t *send_pos,
+                    moe_aux *aux, void *ws, size_t ws_bytes, moe_stream_t stream);
+
+/* moe_ep_experts: the local experts on M received rows.  cfg_local: NExperts =
+ * the rank's N/R experts, TopK = 1, otherwise the layer's.  recv_x [M, D],
+ * recv_expert [M] (local indices), recv_w [M] gate weights; w_local: W1, W2
+ * (b1, b2) of the local experts (W_g unused).  z_out [M, D] fp32: row i =
+ * recv_w[i] * E_{recv_expert[i]}(recv_x[i]).  ws:
+ * moe_ep_experts_workspace_size(cfg_local, M) bytes. */
+size_t moe_ep_experts_workspace_size(const moe_config *cfg_local, int64_t M);
+int moe_ep_experts(const moe_config *cfg_local, const void *recv_x, int64_t M, const int32_t *recv_expert,
+                   const float *recv_w, const moe_weights *w_local, float *z_out, void *ws, size_t ws_bytes,
+                   moe_stream_t stream);
+
+/* moe_ep_combine: y[t] = z_back[send_pos[t*K]] + ... + z_back[send_pos[t*K+K-1]],
+ * left to right; z_back [T*K, D] fp32 are the returned rows in send order; y
+ * [T, D] in y_dtype. */
+int moe_ep_combine(const moe_config *cfg, const float *z_back, int64_t T, const int32_t *send_pos, void *y,
+                   int32_t y_dtype, moe_stream_t stream);
+
 /* Where moe_forward leaves its intermediates inside the workspace (byte
  * offsets from ws), for inspection in tests.  Rows of each expert's segment in
  * the permuted buffers start at a multiple of row_align; rows past an expert's

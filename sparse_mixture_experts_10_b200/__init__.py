@@ -37,6 +37,8 @@ MOE_NOALLOC_SCRATCH_BYTES = 2 << 20
 
 EXPORTED = ("moe_workspace_size", "moe_route", "moe_forward", "moe_forward_timed", "moe_aux_stats",
             "moe_aux_stats_noalloc", "moe_aux_partials", "moe_aux_finalize", "moe_aux_finalize_host",
+            "moe_ep_workspace_size", "moe_ep_dispatch", "moe_ep_experts_workspace_size", "moe_ep_experts",
+            "moe_ep_combine",
             "moe_get_workspace_layout", "moe_total_params", "moe_active_params", "moe_get_device_status",
             "moe_launch_count", "moe_error_string", "moe_selftest_wait_timeout")
 
@@ -106,6 +108,16 @@ def load_library():
     L.moe_aux_finalize.argtypes = [cfgp, vp, auxp, vp]
     L.moe_aux_finalize_host.restype = ctypes.c_int
     L.moe_aux_finalize_host.argtypes = [cfgp, vp, vp, vp, vp, vp]
+    L.moe_ep_workspace_size.restype = sz
+    L.moe_ep_workspace_size.argtypes = [cfgp, i32, i64]
+    L.moe_ep_dispatch.restype = ctypes.c_int
+    L.moe_ep_dispatch.argtypes = [cfgp, i32, vp, i64, wp, vp, vp, vp, vp, vp, auxp, vp, sz, vp]
+    L.moe_ep_experts_workspace_size.restype = sz
+    L.moe_ep_experts_workspace_size.argtypes = [cfgp, i64]
+    L.moe_ep_experts.restype = ctypes.c_int
+    L.moe_ep_experts.argtypes = [cfgp, vp, i64, vp, vp, wp, vp, vp, sz, vp]
+    L.moe_ep_combine.restype = ctypes.c_int
+    L.moe_ep_combine.argtypes = [cfgp, vp, i64, vp, vp, i32, vp]
     L.moe_get_workspace_layout.restype = ctypes.c_int
     L.moe_get_workspace_layout.argtypes = [cfgp, i64, ctypes.POINTER(moe_workspace_layout)]
     L.moe_total_params.restype = i64
@@ -237,6 +249,33 @@ def moe_aux_finalize_host(cfg, partials, counts=None, importance=None, p_mean=No
     """Host version: partials, counts, importance, p_mean, scalars are CPU tensors (int64, int32, fp32)."""
     return load_library().moe_aux_finalize_host(ctypes.byref(cfg), _ptr(partials), _ptr(counts), _ptr(importance),
                                                 _ptr(p_mean), _ptr(scalars))
+
+
+def moe_ep_workspace_size(cfg, n_ranks, T) -> int:
+    return load_library().moe_ep_workspace_size(ctypes.byref(cfg), n_ranks, T)
+
+
+def moe_ep_dispatch(cfg, n_ranks, x, T, weights, send_x, send_expert, send_w, send_counts, send_pos, aux, ws,
+                    ws_bytes, stream=None) -> int:
+    return load_library().moe_ep_dispatch(ctypes.byref(cfg), n_ranks, _ptr(x), T, ctypes.byref(weights), _ptr(send_x),
+                                          _ptr(send_expert), _ptr(send_w), _ptr(send_counts), _ptr(send_pos),
+                                          None if aux is None else ctypes.byref(aux), _ptr(ws), ws_bytes,
+                                          _stream(stream))
+
+
+def moe_ep_experts_workspace_size(cfg_local, M) -> int:
+    return load_library().moe_ep_experts_workspace_size(ctypes.byref(cfg_local), M)
+
+
+def moe_ep_experts(cfg_local, recv_x, M, recv_expert, recv_w, weights_local, z_out, ws, ws_bytes, stream=None) -> int:
+    return load_library().moe_ep_experts(ctypes.byref(cfg_local), _ptr(recv_x), M, _ptr(recv_expert), _ptr(recv_w),
+                                         ctypes.byref(weights_local), _ptr(z_out), _ptr(ws), ws_bytes,
+                                         _stream(stream))
+
+
+def moe_ep_combine(cfg, z_back, T, send_pos, y, y_dtype, stream=None) -> int:
+    return load_library().moe_ep_combine(ctypes.byref(cfg), _ptr(z_back), T, _ptr(send_pos), _ptr(y), y_dtype,
+                                         _stream(stream))
 
 
 def moe_get_workspace_layout(cfg, T) -> moe_workspace_layout:

@@ -70,6 +70,7 @@ struct Plan {
     int n_shared;      // 1: a shared expert (dense FFN over every token) is added after the routed sum
     int capacity;      // assignments each expert accepts (rows served in order; the rest are dropped)
     bool fused_decode; // few tokens, N <= 32, no shared expert: the whole layer in one cooperative kernel
+    bool given_routing;
     int slab_rows, n_slabs;   // fused decode: W_g rows per routing slab, slabs
     // Counters region (zeroed on every call), 32-bit words: [0] router ticket,
     // [1] statistics ticket, [2] number of live experts, [64, 128) per-token
@@ -86,7 +87,10 @@ struct Plan {
         fd_slab, fd_tokp, total;
 };
 
-int make_plan(const moe_config *c, int64_t T, Plan *p) {
+// given_routing: the (token, slot) -> expert assignments and weights are inputs
+// (expert parallelism's received rows), so no router runs and the dispatch
+// tables come from chunk histograms of the given indices.
+int make_plan(const moe_config *c, int64_t T, Plan *p, bool given_routing = false) {
     if (!c || !p) return MOE_ERR_INVALID_ARG;
     const int64_t D = c->DModel, H = c->DHidden, N = c->NExperts, K = c->TopK;
     if (D <= 0 || H <= 0 || N <= 0 || K <= 0 || T < 0) return MOE_ERR_INVALID_ARG;
@@ -128,6 +132,8 @@ int make_plan(const moe_config *c, int64_t T, Plan *p) {
                               : p->np == 16 ? rtc::SimtShape<16>::smem_bytes((int)D)
                                             : rtc::SimtShape<32>::smem_bytes((int)D);
     p->simt_router = p->tc_router && !p->few_router && N <= 32 && simt_bytes <= kSmallRouterSmemMax;
+    p->given_routing = given_routing;
+    if (given_routing) p->tc_router = p->few_router = p->simt_router = p->rowdot_router = p->small_router = false;
     p->chunk_tokens = p->few_router ? 1 : p->simt_router ? rtc::kSimtChunk : p->tc_router ? rtc::BM : kChunk;
     p->rnp = N <= 16 ? 16 : N <= 32 ? 32 : N <= 64 ? 64 : N <= 128 ? 128 : 256;
     p->rkm = K <= 8 ? 8 : 32;
@@ -175,7 +181,7 @@ int make_plan(const moe_config *c, int64_t T, Plan *p) {
     p->shared_tbl = take(16);
     // fused decode: routing slabs of W_g rows (a multiple of 8 rows each, at most
     // 32 slabs) and each token's full softmax
-    p->fused_decode = p->decode && N <= dfu::kMaxN && !p->n_shared && T <= dfu::kMaxT;
+    p->fused_decode = p->decode && N <= dfu::kMaxN && !p->n_shared && T <= dfu::kMaxT && !given_routing;
     p->slab_rows = (int)(cdiv(cdiv(D, dfu::kMaxSlabs), 8) * 8);
     p->n_slabs = (int)cdiv(D, p->slab_rows);
     p->fd_slab = take(p->fused_decode ? (size_t)p->n_slabs * T * 32 * 4 : 0);
@@ -1114,7 +1120,7 @@ int stage_decode_fused(const Plan &P, const Bufs &b, const void *x, const moe_we
 }
 
 int check_weights(const Plan &P, const moe_weights *w, bool need_experts) {
-    if (!w || !w->W_g) return MOE_ERR_INVALID_ARG;
+    if (!w || (!w->W_g && !P.given_routing)) return MOE_ERR_INVALID_ARG;   // given routing needs no router
     if (!need_experts) return MOE_OK;
     if (!w->W1 || !w->W2) return MOE_ERR_INVALID_ARG;
     if (P.has_bias && (!w->b1 || !w->b2)) return MOE_ERR_INVALID_ARG;
@@ -1127,9 +1133,10 @@ int check_weights(const Plan &P, const moe_weights *w, bool need_experts) {
 }
 
 int forward_impl(const moe_config *cfg, const void *x, int64_t T, const moe_weights *w, void *y, int32_t y_dtype,
-                 moe_aux *aux, void *ws, size_t ws_bytes, cudaStream_t s, void *const *ev) {
+                 moe_aux *aux, void *ws, size_t ws_bytes, cudaStream_t s, void *const *ev,
+                 const int *given_idx = nullptr, const float *given_w = nullptr) {
     Plan P;
-    MOE_TRY(make_plan(cfg, T, &P));
+    MOE_TRY(make_plan(cfg, T, &P, given_idx != nullptr));
     MOE_TRY(check_weights(P, w, true));
     if (y_dtype != MOE_F32 && y_dtype != MOE_BF16) return MOE_ERR_INVALID_ARG;
     if (T > 0 && (!x || !y || !aligned16(x) || !aligned16(y))) return MOE_ERR_INVALID_ARG;
@@ -1172,7 +1179,17 @@ int forward_impl(const moe_config *cfg, const void *x, int64_t T, const moe_weig
         for (int i = 4; i <= MOE_N_STAGES; ++i) MOE_TRY(rec(i));
         return MOE_OK;
     }
-    if (P.tc_router) {
+    if (P.given_routing) {
+        // the assignments are inputs: into the workspace, then chunk histograms and the scan
+        if (cudaMemcpyAsync(idx, given_idx, (size_t)P.T * P.K * 4, cudaMemcpyDeviceToDevice, s) != cudaSuccess ||
+            cudaMemcpyAsync(tw, given_w, (size_t)P.T * P.K * 4, cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+            return MOE_ERR_CUDA;
+        hist_kernel<<<P.n_chunks, 256, (size_t)P.N * 4, s>>>(idx, P.T * P.K, P.chunk_tokens * P.K, P.N, 1,
+                                                              b.at<int>(P.chunk_counts));
+        MOE_TRY(check_launch());
+        MOE_TRY(rec(1));
+        MOE_TRY(stage_scan(P, b, nullptr, s));
+    } else if (P.tc_router) {
         MOE_TRY(stage_route_tc(P, b, x, w, logits, idx, tw, nullptr, aux, y_zero, s));
         MOE_TRY(rec(1));
     } else {
@@ -1191,7 +1208,7 @@ int forward_impl(const moe_config *cfg, const void *x, int64_t T, const moe_weig
     MOE_TRY(rec(5));
     if (!combine_in_down(P, y_dtype)) MOE_TRY(stage_combine(P, b, y, y_dtype, *dev, s));
     MOE_TRY(rec(6));
-    if (aux && !P.tc_router) MOE_TRY(stage_aux(P, b, logits, idx, tw, aux, s));
+    if (aux && !P.tc_router && !P.given_routing) MOE_TRY(stage_aux(P, b, logits, idx, tw, aux, s));
     MOE_TRY(rec(7));
     return MOE_OK;
 }
@@ -1321,6 +1338,133 @@ int moe_aux_finalize_host(const moe_config *cfg, const int64_t *partials, int32_
     aux_finalize_partials(P.N, P.K, reinterpret_cast<const long long *>(partials), counts, importance, p_mean,
                           scalars);
     return MOE_OK;
+}
+
+// ---------------------------------------------------------------- expert parallelism
+namespace {
+struct EpPlan {
+    Plan P;          // the routing of this rank's tokens
+    int R, epr, n_chunks;
+    size_t cc, cb, offsets, rowoff, live, perm, total;
+};
+
+int make_ep_plan(const moe_config *cfg, int32_t n_ranks, int64_t T, EpPlan *e) {
+    MOE_TRY(make_plan(cfg, T, &e->P));
+    const int N = e->P.N;
+    if (n_ranks < 1 || n_ranks > N || N % n_ranks) return MOE_ERR_INVALID_ARG;
+    if (e->P.n_shared || cfg->capacity_factor > 0.0f) return MOE_ERR_UNSUPPORTED;
+    e->R = n_ranks;
+    e->epr = N / n_ranks;
+    e->n_chunks = (int)std::max<int64_t>(1, cdiv(T, kChunk));
+    size_t off = align256(e->P.total);
+    auto take = [&](size_t bytes) {
+        const size_t o = off;
+        off = align256(off + bytes);
+        return o;
+    };
+    e->cc = take((size_t)e->n_chunks * n_ranks * 4);
+    e->cb = take((size_t)e->n_chunks * n_ranks * 4);
+    e->offsets = take((size_t)(n_ranks + 1) * 4);
+    e->rowoff = take((size_t)(n_ranks + 1) * 4);
+    e->live = take((size_t)n_ranks * 4);
+    e->perm = take((size_t)(cdiv(T * e->P.K + (int64_t)n_ranks * (kRowAlign - 1), kRowAlign) * kRowAlign) * 4);
+    e->total = off;
+    return MOE_OK;
+}
+}  // namespace
+
+size_t moe_ep_workspace_size(const moe_config *cfg, int32_t n_ranks, int64_t T) {
+    EpPlan e;
+    if (make_ep_plan(cfg, n_ranks, T, &e) != MOE_OK) return 0;
+    return e.total;
+}
+
+int moe_ep_dispatch(const moe_config *cfg, int32_t n_ranks, const void *x, int64_t T, const moe_weights *w,
+                    void *send_x, int32_t *send_expert, float *send_w, int32_t *send_counts, int32_t *send_pos,
+                    moe_aux *aux, void *ws, size_t ws_bytes, moe_stream_t stream) {
+    EpPlan e;
+    MOE_TRY(make_ep_plan(cfg, n_ranks, T, &e));
+    const Plan &P = e.P;
+    MOE_TRY(check_weights(P, w, false));
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (!send_counts) return MOE_ERR_INVALID_ARG;
+    if (T == 0) {
+        if (cudaMemsetAsync(send_counts, 0, (size_t)n_ranks * 4, s) != cudaSuccess) return MOE_ERR_CUDA;
+        return zero_aux(P, aux, s);
+    }
+    if (!x || !aligned16(x) || !send_x || !aligned16(send_x) || !send_expert || !send_w || !send_pos)
+        return MOE_ERR_INVALID_ARG;
+    if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u)) return MOE_ERR_INVALID_ARG;
+    if (ws_bytes < e.total) return MOE_ERR_WORKSPACE_TOO_SMALL;
+    DeviceInfo *dev = nullptr;
+    MOE_TRY(device_info(&dev));
+    Bufs b{static_cast<char *>(ws), &P};
+    float *logits = b.at<float>(P.logits);
+    int *idx = b.at<int>(P.idx);
+    float *tw = b.at<float>(P.w);
+    MOE_TRY(zero_counters(P, b, s));
+    if (P.tc_router) {
+        MOE_TRY(stage_route_tc(P, b, x, w, logits, idx, tw, nullptr, aux, nullptr, s));
+    } else {
+        MOE_TRY(stage_route(P, b, x, w, logits, idx, tw, *dev, s));
+        if (aux) MOE_TRY(stage_aux(P, b, logits, idx, tw, aux, s));
+    }
+    // group the (token, slot) pairs by the rank holding their expert: chunk
+    // histograms, the scan (send counts and offsets), the packing
+    const int R = e.R;
+    int *cc = b.at<int>(e.cc), *cb = b.at<int>(e.cb), *offs = b.at<int>(e.offsets);
+    unsigned *ctr = b.at<unsigned>(P.counters);
+    hist_kernel<<<e.n_chunks, 256, (size_t)R * 4, s>>>(idx, T * P.K, kChunk * P.K, R, e.epr, cc);
+    MOE_TRY(check_launch());
+    scan_kernel<<<(unsigned)cdiv(R, 32), 1024, 0, s>>>(cc, e.n_chunks, R, T * P.K, INT32_MAX, cb, send_counts, offs,
+                                                       b.at<int>(e.rowoff), b.at<int>(e.perm), nullptr, ctr + 5,
+                                                       b.at<int>(e.live), reinterpret_cast<int *>(ctr) + 6);
+    MOE_TRY(check_launch());
+    const size_t smem = (size_t)(R + kChunk * P.K) * 4;
+    if (P.dtype == MOE_F32)
+        ep_pack_kernel<float><<<e.n_chunks, 256, smem, s>>>(static_cast<const float *>(x), (int)T, P.D, P.K, R, e.epr,
+                                                             kChunk, idx, tw, cb, offs, static_cast<float *>(send_x),
+                                                             send_expert, send_w, send_pos);
+    else
+        ep_pack_kernel<__nv_bfloat16><<<e.n_chunks, 256, smem, s>>>(
+            static_cast<const __nv_bfloat16 *>(x), (int)T, P.D, P.K, R, e.epr, kChunk, idx, tw, cb, offs,
+            static_cast<__nv_bfloat16 *>(send_x), send_expert, send_w, send_pos);
+    return check_launch();
+}
+
+size_t moe_ep_experts_workspace_size(const moe_config *cfg_local, int64_t M) {
+    Plan P;
+    if (make_plan(cfg_local, M, &P, true) != MOE_OK || P.K != 1) return 0;
+    return P.total;
+}
+
+int moe_ep_experts(const moe_config *cfg_local, const void *recv_x, int64_t M, const int32_t *recv_expert,
+                   const float *recv_w, const moe_weights *w_local, float *z_out, void *ws, size_t ws_bytes,
+                   moe_stream_t stream) {
+    if (!cfg_local || cfg_local->TopK != 1 || cfg_local->n_shared || cfg_local->capacity_factor > 0.0f)
+        return MOE_ERR_INVALID_ARG;
+    if (M > 0 && (!recv_expert || !recv_w)) return MOE_ERR_INVALID_ARG;
+    return forward_impl(cfg_local, recv_x, M, w_local, z_out, MOE_F32, nullptr, ws, ws_bytes,
+                        reinterpret_cast<cudaStream_t>(stream), nullptr, recv_expert, recv_w);
+}
+
+int moe_ep_combine(const moe_config *cfg, const float *z_back, int64_t T, const int32_t *send_pos, void *y,
+                   int32_t y_dtype, moe_stream_t stream) {
+    Plan P;
+    MOE_TRY(make_plan(cfg, T, &P));
+    if (y_dtype != MOE_F32 && y_dtype != MOE_BF16) return MOE_ERR_INVALID_ARG;
+    if (T == 0) return MOE_OK;
+    if (!z_back || !send_pos || !y || !aligned16(z_back) || !aligned16(y)) return MOE_ERR_INVALID_ARG;
+    DeviceInfo *dev = nullptr;
+    MOE_TRY(device_info(&dev));
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const int64_t nq = T * (P.D / 4);
+    const int grid = (int)std::min<int64_t>(cdiv(nq, 256), (int64_t)dev->sms * 8);
+    if (y_dtype == MOE_F32)
+        return launch_pdl(combine_kernel<float>, dim3(grid), dim3(256), 0, s, z_back, T, P.D, P.K, (const int *)send_pos,
+                          1, (const float *)nullptr, static_cast<float *>(y));
+    return launch_pdl(combine_kernel<__nv_bfloat16>, dim3(grid), dim3(256), 0, s, z_back, T, P.D, P.K,
+                      (const int *)send_pos, 1, (const float *)nullptr, static_cast<__nv_bfloat16 *>(y));
 }
 
 int64_t moe_total_params(const moe_config *c) {

@@ -355,6 +355,96 @@ __global__ void __launch_bounds__(256) topk_kernel(const float *__restrict__ log
 }
 
 // ---------------------------------------------------------------------------
+// Chunk histograms of given assignments: chunk c holds entries
+// [c * per_chunk, (c + 1) * per_chunk) of idx; bucket = idx / div (div = 1:
+// experts; div = experts per rank: destination ranks).  Integer shared-memory
+// atomics, so the counts do not depend on scheduling.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) hist_kernel(const int *__restrict__ idx, int64_t n_entries, int per_chunk,
+                                                   int n_buckets, int div, int *__restrict__ chunk_counts) {
+    extern __shared__ int s_hist[];
+    for (int b = threadIdx.x; b < n_buckets; b += blockDim.x) s_hist[b] = 0;
+    __syncthreads();
+    const int64_t f0 = (int64_t)blockIdx.x * per_chunk;
+    const int64_t f1 = min(n_entries, f0 + per_chunk);
+    for (int64_t f = f0 + threadIdx.x; f < f1; f += blockDim.x) {
+        const int e = idx[f];
+        const int b = e / div;
+        if (e < 0 || b >= n_buckets) {
+            set_status(kStatusBounds);
+            continue;
+        }
+        atomicAdd(&s_hist[b], 1);
+    }
+    __syncthreads();
+    for (int b = threadIdx.x; b < n_buckets; b += blockDim.x) chunk_counts[(size_t)blockIdx.x * n_buckets + b] = s_hist[b];
+}
+
+// ---------------------------------------------------------------------------
+// Expert-parallel dispatch: the (token, slot) pairs of a chunk, grouped by the
+// rank that holds their expert (bucket = expert / experts_per_rank) in stable
+// (token, slot) order, packed without padding at
+// offsets[r] + chunk_base[c, r] + rank inside the chunk.  Writes the token row,
+// the expert's index on its rank and the gate weight of every pair, and the
+// pair's position in the send buffer (send_pos, read by the combine).
+// ---------------------------------------------------------------------------
+template <typename Tin>
+__global__ void __launch_bounds__(256) ep_pack_kernel(const Tin *__restrict__ x, int T, int D, int K, int R, int epr,
+                                                      int chunk_tokens, const int *__restrict__ topk_idx,
+                                                      const float *__restrict__ topk_w,
+                                                      const int *__restrict__ chunk_base,
+                                                      const int *__restrict__ offsets, Tin *__restrict__ send_x,
+                                                      int *__restrict__ send_expert, float *__restrict__ send_w,
+                                                      int *__restrict__ send_pos) {
+    extern __shared__ int s_ep[];
+    int *s_run = s_ep;          // [R]
+    int *s_dest = s_ep + R;     // [chunk_tokens * K]
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int c = blockIdx.x;
+    const int t_begin = c * chunk_tokens, t_end = min(T, t_begin + chunk_tokens);
+    const int n_entries = (t_end - t_begin) * K;
+    const int64_t f0 = (int64_t)t_begin * K;
+    for (int r = tid; r < R; r += blockDim.x) s_run[r] = offsets[r] + chunk_base[(size_t)c * R + r];
+    __syncthreads();
+    if (warp == 0) {
+        for (int base = 0; base < n_entries; base += 32) {
+            const int f = base + lane;
+            const int e = f < n_entries ? topk_idx[f0 + f] : -1;
+            int r = e >= 0 ? e / epr : -1;
+            if (f < n_entries && (e < 0 || r >= R)) {
+                set_status(kStatusBounds);
+                r = -1;
+            }
+            const unsigned peers = __match_any_sync(0xffffffffu, r);
+            const int rank = __popc(peers & lanemask_lt());
+            const int base_pos = r >= 0 ? s_run[r] : 0;
+            __syncwarp();
+            if (r >= 0 && lane == __ffs(peers) - 1) s_run[r] = base_pos + __popc(peers);
+            __syncwarp();
+            if (f < n_entries) {
+                const int dest = r >= 0 ? base_pos + rank : -1;
+                s_dest[f] = dest;
+                send_pos[f0 + f] = dest;
+                if (dest >= 0) {
+                    send_expert[dest] = e - r * epr;
+                    send_w[dest] = topk_w[f0 + f];
+                }
+            }
+        }
+    }
+    __syncthreads();
+    constexpr int VEC = 16 / sizeof(Tin);
+    const int nvec = D / VEC;
+    for (int f = warp; f < n_entries; f += blockDim.x / 32) {
+        const int dest = s_dest[f];
+        if (dest < 0) continue;
+        const uint4 *src = reinterpret_cast<const uint4 *>(x + (int64_t)(t_begin + f / K) * D);
+        uint4 *dst = reinterpret_cast<uint4 *>(send_x + (int64_t)dest * D);
+        for (int v = lane; v < nvec; v += 32) dst[v] = __ldg(src + v);
+    }
+}
+
+// ---------------------------------------------------------------------------
 // Scan: per expert, the exclusive prefix of the chunk histograms (chunk_base);
 // then, in the last block to finish, the per-expert counts, their exclusive
 // scan (offsets) and the padded segment starts (row_offsets, multiples of

@@ -523,6 +523,90 @@ def test_capacity_drop(name, wl):
         assert dropped > 0, "the case should overflow some expert"
 
 
+# ----------------------------------------------------------------------------- expert parallelism
+EP_CASES = [
+    ("gelu_bias_2_ranks", Workload("ep_a", 80, 700, 256, 512, 8, 2, ACT_GELU, torch.bfloat16, True, 0.04,
+                                   zipf_s=0.5, random_bias=True), 2),
+    ("swiglu_64_experts_4_ranks", Workload("ep_b", 81, 600, 256, 256, 64, 4, ACT_SWIGLU, torch.bfloat16, False, 0.05,
+                                           zipf_s=0.5, sel_s=0.3), 4),
+    ("few_tokens_4_ranks", Workload("ep_c", 82, 24, 512, 512, 16, 4, ACT_SWIGLU, torch.bfloat16, False, 0.04,
+                                    zipf_s=0.6), 4),
+    ("fp32_2_ranks", Workload("ep_d", 83, 300, 64, 256, 8, 2, ACT_GELU, torch.float32, True, 0.05,
+                              random_bias=True), 2),
+    ("one_rank", Workload("ep_e", 84, 500, 256, 256, 8, 2, ACT_SWIGLU, torch.bfloat16, False, 0.05), 1),
+]
+
+
+@pytest.mark.parametrize("name,wl,R", EP_CASES, ids=[c[0] for c in EP_CASES])
+def test_expert_parallel_virtual_ranks(name, wl, R):
+    """Expert parallelism emulated on one GPU: R virtual ranks each route and pack their own
+    tokens (moe_ep_dispatch), the all-to-alls are buffer copies, each rank's N/R experts run on
+    the rows it received (moe_ep_experts), the outputs go back and each rank combines
+    (moe_ep_combine).  Every rank's routing is bit-exact and its y equals the oracle's whole
+    layer on its tokens with all N experts."""
+    T, N, K, D = wl.T, wl.N, wl.K, wl.D
+    epr = N // R
+    big = make_inputs(wl, "cuda", T=T * R)
+    cfg = moe.make_config(wl.D, wl.H, N, K, wl.act, moe.dtype_code(wl.dtype), wl.has_bias)
+    w_router = moe.make_weights(big["W_g"], big["W1"], big["W2"], big["b_g"], big["b1"], big["b2"], big.get("b_sel"))
+    L = moe.moe_get_workspace_layout(cfg, T)
+    sent = []
+    for r in range(R):
+        x_r = big["x"][r * T:(r + 1) * T].contiguous()
+        ws = torch.empty(moe.moe_ep_workspace_size(cfg, R, T), dtype=torch.uint8, device="cuda")
+        send_x = torch.empty(T * K, D, dtype=wl.dtype, device="cuda")
+        send_e = torch.full((T * K,), -1, dtype=torch.int32, device="cuda")
+        send_w = torch.empty(T * K, device="cuda")
+        cnt = torch.empty(R, dtype=torch.int32, device="cuda")
+        pos = torch.empty(T * K, dtype=torch.int32, device="cuda")
+        moe.check(moe.moe_ep_dispatch(cfg, R, x_r, T, w_router, send_x, send_e, send_w, cnt, pos, None, ws,
+                                      ws.numel()), "dispatch")
+        torch.cuda.synchronize()
+        assert moe.moe_get_device_status() == 0
+        lg = _ws_view(ws, L.logits, T * N, torch.float32).view(T, N).cpu().numpy()
+        idx = _ws_view(ws, L.topk_idx, T * K, torch.int32).view(T, K).cpu().numpy()
+        sent.append(dict(x=x_r, send_x=send_x, send_e=send_e, send_w=send_w, cnt=cnt.cpu().tolist(), pos=pos,
+                         logits=lg, idx=idx))
+        # the packing: rank-major, (token, slot) order inside a rank, nothing lost
+        flat = idx.ravel()
+        dest = flat // epr
+        order = np.lexsort((np.arange(T * K), dest))
+        np.testing.assert_array_equal(pos.cpu().numpy()[order], np.arange(T * K))
+        np.testing.assert_array_equal(send_e.cpu().numpy()[pos.cpu().numpy()], flat - dest * epr)
+        np.testing.assert_array_equal(np.bincount(dest, minlength=R), sent[-1]["cnt"])
+    # the all-to-all, emulated: rank q receives every rank's block for q, source rank after source rank
+    offs = [np.concatenate([[0], np.cumsum(s_["cnt"])]) for s_ in sent]
+    z_parts = [[None] * R for _ in range(R)]
+    for q in range(R):
+        rx = torch.cat([s_["send_x"][offs[r][q]:offs[r][q + 1]] for r, s_ in enumerate(sent)])
+        re = torch.cat([s_["send_e"][offs[r][q]:offs[r][q + 1]] for r, s_ in enumerate(sent)])
+        rw = torch.cat([s_["send_w"][offs[r][q]:offs[r][q + 1]] for r, s_ in enumerate(sent)])
+        M = rx.shape[0]
+        cfg_l = moe.make_config(wl.D, wl.H, epr, 1, wl.act, moe.dtype_code(wl.dtype), wl.has_bias)
+        sl = slice(q * epr, (q + 1) * epr)
+        w_l = moe.make_weights(None, big["W1"][sl], big["W2"][sl], None,
+                               None if big["b1"] is None else big["b1"][sl],
+                               None if big["b2"] is None else big["b2"][sl])
+        z = torch.full((max(M, 1), D), float("nan"), device="cuda")
+        wsl = torch.empty(max(moe.moe_ep_experts_workspace_size(cfg_l, M), 1), dtype=torch.uint8, device="cuda")
+        moe.check(moe.moe_ep_experts(cfg_l, rx, M, re, rw, w_l, z, wsl, wsl.numel()), "experts")
+        torch.cuda.synchronize()
+        assert moe.moe_get_device_status() == 0
+        rstart = np.concatenate([[0], np.cumsum([s_["cnt"][q] for s_ in sent])])
+        for r in range(R):
+            z_parts[r][q] = z[rstart[r]:rstart[r + 1]]
+    for r, s_ in enumerate(sent):
+        z_back = torch.cat(z_parts[r]).contiguous()
+        y = torch.full((T, D), float("nan"), device="cuda")
+        moe.check(moe.moe_ep_combine(cfg, z_back, T, s_["pos"], y, moe.MOE_F32), "combine")
+        torch.cuda.synchronize()
+        inp_r = dict(big, x=s_["x"])
+        ref = ph.oracle_full_layer(inp_r, wl, K, gpu_logits=s_["logits"])
+        ph.assert_logits_close(s_["logits"], ref["scores"])
+        np.testing.assert_array_equal(s_["idx"], ref["sel"])
+        ph.assert_y_close(y.cpu().numpy(), ref["y"], wl.dtype)
+
+
 # ----------------------------------------------------------------------------- data parallelism
 def _ws_view(ws, off, n, dt):
     return ws[off:off + n * torch.tensor([], dtype=dt).element_size()].view(dt)

@@ -134,3 +134,48 @@ def test_two_cpu_ranks_global_statistics():
     np.testing.assert_allclose(out0["p_mean"], st["p_mean"], rtol=1e-6, atol=1e-8)
     np.testing.assert_allclose(out0["scalars"], [st["switch"], st["simple"], st["cv2_importance"], st["cv2_load"]],
                                rtol=1e-5, atol=1e-7)
+
+
+def _ep_worker(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        from sparse_mixture_experts_10_b200 import ep
+
+        # rank r sends counts[r][d] rows to rank d; a row holds (source rank, destination, index)
+        counts = [[3, 2, 0], [1, 4, 2], [0, 1, 5]][rank][:world]
+        rows = torch.tensor([[rank, d, i] for d, c in enumerate(counts) for i in range(c)], dtype=torch.float32)
+        recv, recv_counts = ep.exchange(rows, torch.tensor(counts, dtype=torch.int32))
+        # what a rank's experts do to a row (any function of the row alone)
+        out = recv * 10.0 + 1.0
+        back = ep.exchange_back(out, recv_counts, torch.tensor(counts, dtype=torch.int32))
+        q.put((rank, recv.tolist(), recv_counts.tolist(), back.tolist(), rows.tolist()))
+    except Exception as exc:
+        q.put((rank, repr(exc), None, None, None))
+        raise
+    finally:
+        dist.destroy_process_group()
+
+
+def test_expert_parallel_exchange_round_trip():
+    """The expert-parallel all-to-alls on CPU ranks (gloo, world size 3): every rank receives the
+    rows destined to it, source rank after source rank in the order they were packed, and the
+    reverse exchange returns each processed row to its place on its source rank."""
+    world = 3
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_ep_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = sorted((q.get(timeout=120) for _ in range(world)), key=lambda r: r[0])
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    all_counts = [[3, 2, 0], [1, 4, 2], [0, 1, 5]]
+    for rank, recv, recv_counts, back, rows in res:
+        assert isinstance(recv, list), recv
+        expect = [[src, rank, i] for src in range(world) for i in range(all_counts[src][rank])]
+        assert recv == expect
+        assert recv_counts == [all_counts[src][rank] for src in range(world)]
+        assert back == [[v * 10.0 + 1.0 for v in row] for row in rows]
