@@ -86,6 +86,11 @@ def configure(L):
     L.orc_combine.argtypes = [i64, i64, vp, vp, vp]
     L.orc_add_shared.argtypes = [i64, vp, vp]
     L.orc_moe_layer_rows.argtypes = [ctypes.POINTER(_Layer), i64, i64, vp, vp, vp, vp, vp, vp]
+    L.orc_gelu_grad.restype = dp
+    L.orc_gelu_grad.argtypes = [dp]
+    L.orc_silu_grad.restype = dp
+    L.orc_silu_grad.argtypes = [dp]
+    L.orc_moe_layer_backward.argtypes = [ctypes.POINTER(_Layer), i64, vp, vp, dp, dp, vp, vp, vp, vp, vp, vp, vp]
     L.orc_capacity.restype = i64
     L.orc_capacity.argtypes = [dp, i64, i64, i64]
     L.orc_capacity_keep.argtypes = [i64, i64, i64, vp, i64, vp]
@@ -319,6 +324,31 @@ def moe_layer_capacity(x, Wg, W1, W2, *, K, act, dtype_tag, cf, sel_scores=None,
     keep = capacity_keep(routed["sel"], N, C)
     out = moe_layer(x, Wg, W1, W2, K=K, act=act, dtype_tag=dtype_tag, sel_scores=sel_scores, keep=keep, **kw)
     out["keep"], out["capacity"] = keep, C
+    return out
+
+
+def moe_layer_backward(x, Wg, W1, W2, dy, *, K, act, dtype_tag, bg=None, b1=None, b2=None, bsel=None,
+                       sel_scores=None, alpha_switch=0.0, alpha_importance=0.0):
+    """Gradients of sum(y * dy) + alpha_switch * switch_loss + alpha_importance * cv2_importance
+    with respect to x, W_g, b_g, W1, b1, W2, b2 (fp64, single thread).  Returns a dict."""
+    xm = _mat(x, dtype_tag)
+    T, D = xm.shape
+    Wgm = _mat(Wg, dtype_tag)
+    N = Wgm.shape[1]
+    W1m, W2m = _mat(W1, dtype_tag), _mat(W2, dtype_tag)
+    H = W2m.shape[2]
+    bgm, b1m, b2m, bselm = _c(bg, np.float32), _c(b1, np.float32), _c(b2, np.float32), _c(bsel, np.float32)
+    ss = _c(sel_scores, np.float32)
+    dyv = _c(dy, np.float64)
+    lay = _Layer(D, H, N, K, act, dtype_tag, _p(xm), _p(Wgm), _p(bgm), _p(W1m), _p(b1m), _p(W2m), _p(b2m),
+                 _p(bselm), None, None, None, None)
+    out = dict(dx=np.empty((T, D)), dWg=np.empty((D, N)), dbg=np.empty(N), dW1=np.empty(W1m.shape),
+               dW2=np.empty(W2m.shape))
+    out["db1"] = np.empty((N, H)) if act == ACT_GELU else None
+    out["db2"] = np.empty((N, D)) if act == ACT_GELU else None
+    lib().orc_moe_layer_backward(ctypes.byref(lay), T, _p(ss), _p(dyv), float(alpha_switch), float(alpha_importance),
+                                 _p(out["dx"]), _p(out["dWg"]), _p(out["dbg"]), _p(out["dW1"]), _p(out["db1"]),
+                                 _p(out["dW2"]), _p(out["db2"]))
     return out
 
 

@@ -444,6 +444,174 @@ void orc_aux_stats(int64_t T, int64_t N, int64_t K, const double *scores,
 }
 
 /* ------------------------------------------------------------------------
+ * Backward pass.  "Extending Raschka's GPT-2 ...", section on making the
+ * router trainable: the router learns through the gate weights it produces
+ * (the softmax over the kept scores) and through the auxiliary loss; the
+ * experts learn through the outputs they are weighted into.  Everything below
+ * is the chain rule applied to the forward definitions above, in fp64:
+ *   y = sum_j w_j o_j,  o_j = E_{sel_j}(x),  w = softmax over the kept scores
+ *   dL/dw_j = <dy, o_j>,  dL/do_j = w_j dy
+ *   softmax over the kept set: ds_kept_j = w_j (dw_j - sum_m w_m dw_m), 0 for
+ *   the others; scores s = x W_g + b_g: dW_g += x ds, db_g += ds, dx += W_g ds
+ * plus, with weights alpha_switch and alpha_importance, the gradients of the
+ * Switch-style loss N sum_e f_e P_e (f_e counts, constant almost everywhere;
+ * P_e the mean full softmax) and of CV(importance)^2 (importance = sum of the
+ * gate weights per expert).  The count-based terms (N sum f^2, CV(load)^2)
+ * are piecewise constant and carry no gradient.
+ * ---------------------------------------------------------------------- */
+
+/* GELU'(v) = Phi(v) + v phi(v) for the exact-erf GELU. */
+double orc_gelu_grad(double v) {
+    return 0.5 * (1.0 + erf(v / sqrt(2.0))) + v * exp(-0.5 * v * v) / sqrt(2.0 * 3.14159265358979323846);
+}
+
+/* silu'(g) = s (1 + g (1 - s)) with s = 1 / (1 + exp(-g)). */
+double orc_silu_grad(double g) {
+    double sg = 1.0 / (1.0 + exp(-g));
+    return sg * (1.0 + g * (1.0 - sg));
+}
+
+/* One expert's backward for one token row: upstream gradient go [D] of its
+ * output; accumulates into dW1e ([H, D] or [2H, D]), db1e [H], dW2e [D, H],
+ * db2e [D] (bias pointers NULL for SwiGLU) and adds the input gradient to
+ * dx_row [D].  pre [2H], hid [H], dh [H] are scratch. */
+void orc_expert_backward(const orc_layer *L, int64_t e, const double *x_row, const double *go, double *dx_row,
+                         double *dW1e, double *db1e, double *dW2e, double *db2e, double *pre, double *hid,
+                         double *dh) {
+    int64_t D = L->D, H = L->H, es = orc_elem(L);
+    int swiglu = L->act == ORC_ACT_SWIGLU;
+    const char *W1e = (const char *)L->W1 + e * (swiglu ? 2 : 1) * H * D * es;
+    const char *W2e = (const char *)L->W2 + e * D * H * es;
+    /* forward of the expert again: pre-activations and hidden values */
+    for (int64_t n = 0; n < (swiglu ? 2 * H : H); ++n) {
+        double a = 0.0;
+        for (int64_t i = 0; i < D; ++i) a += orc_get(W1e, L->dtype, n * D + i) * x_row[i];
+        if (!swiglu && L->b1) a += (double)L->b1[e * H + n];
+        pre[n] = a;
+    }
+    for (int64_t n = 0; n < H; ++n) hid[n] = swiglu ? orc_silu(pre[n]) * pre[H + n] : orc_gelu(pre[n]);
+    /* second linear: dW2 += go hid^T, db2 += go, dh = W2^T go */
+    for (int64_t c = 0; c < D; ++c) {
+        for (int64_t n = 0; n < H; ++n) dW2e[c * H + n] += go[c] * hid[n];
+        if (db2e) db2e[c] += go[c];
+    }
+    for (int64_t n = 0; n < H; ++n) {
+        double a = 0.0;
+        for (int64_t c = 0; c < D; ++c) a += orc_get(W2e, L->dtype, c * H + n) * go[c];
+        dh[n] = a;
+    }
+    /* activation, then first linear: dW1 += da x^T, db1 += da, dx += W1^T da */
+    for (int64_t n = 0; n < H; ++n) {
+        if (swiglu) {
+            double dg = dh[n] * pre[H + n] * orc_silu_grad(pre[n]);
+            double du = dh[n] * orc_silu(pre[n]);
+            for (int64_t i = 0; i < D; ++i) {
+                dW1e[n * D + i] += dg * x_row[i];
+                dW1e[(H + n) * D + i] += du * x_row[i];
+                dx_row[i] += orc_get(W1e, L->dtype, n * D + i) * dg + orc_get(W1e, L->dtype, (H + n) * D + i) * du;
+            }
+        } else {
+            double da = dh[n] * orc_gelu_grad(pre[n]);
+            if (db1e) db1e[n] += da;
+            for (int64_t i = 0; i < D; ++i) {
+                dW1e[n * D + i] += da * x_row[i];
+                dx_row[i] += orc_get(W1e, L->dtype, n * D + i) * da;
+            }
+        }
+    }
+}
+
+/* The layer's backward for T tokens (single thread; the kept sets are chosen
+ * as in the forward: on sel_scores when given, else on the fp64 scores plus
+ * bsel).  dy [T, D]; outputs (zeroed here): dx [T, D], dWg [D, N], dbg [N],
+ * dW1 like W1, db1 [N, H] (GELU, else may be NULL), dW2 [N, D, H], db2
+ * [N, D] (GELU, else may be NULL). */
+void orc_moe_layer_backward(const orc_layer *L, int64_t T, const float *sel_scores, const double *dy,
+                            double alpha_switch, double alpha_importance, double *dx, double *dWg, double *dbg,
+                            double *dW1, double *db1, double *dW2, double *db2) {
+    int64_t D = L->D, H = L->H, N = L->N, K = L->K;
+    int swiglu = L->act == ORC_ACT_SWIGLU;
+    int64_t rows1 = swiglu ? 2 * H : H;
+    for (int64_t i = 0; i < T * D; ++i) dx[i] = 0.0;
+    for (int64_t i = 0; i < D * N; ++i) dWg[i] = 0.0;
+    for (int64_t e = 0; e < N; ++e) dbg[e] = 0.0;
+    for (int64_t i = 0; i < N * rows1 * D; ++i) dW1[i] = 0.0;
+    for (int64_t i = 0; i < N * D * H; ++i) dW2[i] = 0.0;
+    if (db1) for (int64_t i = 0; i < N * H; ++i) db1[i] = 0.0;
+    if (db2) for (int64_t i = 0; i < N * D; ++i) db2[i] = 0.0;
+    if (T == 0) return;
+    double *scores = (double *)malloc(sizeof(double) * (size_t)(T * N));
+    int32_t *sel = (int32_t *)malloc(sizeof(int32_t) * (size_t)(T * K));
+    double *w = (double *)malloc(sizeof(double) * (size_t)(T * K));
+    double *y = (double *)malloc(sizeof(double) * (size_t)(T * D));
+    orc_moe_layer_rows(L, 0, T, sel_scores, NULL, scores, sel, w, y);
+    /* batch quantities of the auxiliary losses: f_e and the importance */
+    double *f = (double *)calloc((size_t)N, sizeof(double));
+    double *imp = (double *)calloc((size_t)N, sizeof(double));
+    for (int64_t t = 0; t < T; ++t)
+        for (int64_t j = 0; j < K; ++j) {
+            f[sel[t * K + j]] += 1.0 / (double)(T * K);
+            imp[sel[t * K + j]] += w[t * K + j];
+        }
+    /* dCV^2/dimp_e = 2 (imp_e - m) / (N m^2) - 2 var / (N m^3), population variance */
+    double m = 0.0, var = 0.0;
+    for (int64_t e = 0; e < N; ++e) m += imp[e];
+    m /= (double)N;
+    for (int64_t e = 0; e < N; ++e) var += (imp[e] - m) * (imp[e] - m);
+    var /= (double)N;
+    double *dimp = (double *)calloc((size_t)N, sizeof(double));
+    if (m != 0.0)
+        for (int64_t e = 0; e < N; ++e)
+            dimp[e] = 2.0 * (imp[e] - m) / ((double)N * m * m) - 2.0 * var / ((double)N * m * m * m);
+    double *x_row = (double *)malloc(sizeof(double) * (size_t)D);
+    double *o = (double *)malloc(sizeof(double) * (size_t)D);
+    double *go = (double *)malloc(sizeof(double) * (size_t)D);
+    double *pre = (double *)malloc(sizeof(double) * (size_t)(2 * H));
+    double *hid = (double *)malloc(sizeof(double) * (size_t)H);
+    double *dh = (double *)malloc(sizeof(double) * (size_t)H);
+    double *dw = (double *)malloc(sizeof(double) * (size_t)K);
+    double *ds = (double *)malloc(sizeof(double) * (size_t)N);
+    double *p = (double *)malloc(sizeof(double) * (size_t)N);
+    int64_t es = orc_elem(L);
+    for (int64_t t = 0; t < T; ++t) {
+        orc_load_row(D, L->x, L->dtype, t, x_row);
+        double *dxr = dx + t * D;
+        const double *dyr = dy + t * D;
+        for (int64_t j = 0; j < K; ++j) {
+            int32_t e = sel[t * K + j];
+            orc_expert(L, e, x_row, hid, o);
+            double a = 0.0;
+            for (int64_t c = 0; c < D; ++c) a += dyr[c] * o[c];
+            dw[j] = a + alpha_importance * dimp[e];
+            for (int64_t c = 0; c < D; ++c) go[c] = w[t * K + j] * dyr[c];
+            orc_expert_backward(L, e, x_row, go, dxr, dW1 + e * rows1 * D, db1 ? db1 + e * H : NULL,
+                                dW2 + e * D * H, db2 ? db2 + e * D : NULL, pre, hid, dh);
+        }
+        /* the softmax over the kept scores, then the Switch-style loss on the full softmax */
+        for (int64_t e = 0; e < N; ++e) ds[e] = 0.0;
+        double wdw = 0.0;
+        for (int64_t j = 0; j < K; ++j) wdw += w[t * K + j] * dw[j];
+        for (int64_t j = 0; j < K; ++j) ds[sel[t * K + j]] += w[t * K + j] * (dw[j] - wdw);
+        if (alpha_switch != 0.0) {
+            orc_softmax(N, scores + t * N, p);
+            double fp = 0.0;
+            for (int64_t e = 0; e < N; ++e) fp += f[e] * p[e];
+            for (int64_t e = 0; e < N; ++e) ds[e] += alpha_switch * ((double)N / (double)T) * p[e] * (f[e] - fp);
+        }
+        for (int64_t e = 0; e < N; ++e) {
+            dbg[e] += ds[e];
+            for (int64_t i = 0; i < D; ++i) {
+                dWg[i * N + e] += x_row[i] * ds[e];
+                dxr[i] += orc_get(L->Wg, L->dtype, i * N + e) * ds[e];
+            }
+        }
+    }
+    (void)es;
+    free(scores); free(sel); free(w); free(y); free(f); free(imp); free(dimp);
+    free(x_row); free(o); free(go); free(pre); free(hid); free(dh); free(dw); free(ds); free(p);
+}
+
+/* ------------------------------------------------------------------------
  * Parameter accounting.  "MoE(Mixture of Experts)" section (1): the router
  * holds DModel*NExperts weights and each GELU expert 2*DModel*DHidden; the
  * total counts all NExperts experts, the active count only TopK of them.

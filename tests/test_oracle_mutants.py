@@ -81,6 +81,20 @@ MUTANTS = [
      [pins.test_capacity_keeps_the_first_C_of_each_expert_in_row_order]),
     ("dropped_slot_still_added", "            if (keep && !keep[t * K + j]) {", "            if (0) {",
      [pins.test_capacity_layer_is_the_masked_dense_gate]),
+    ("gelu_grad_missing_density", "+ v * exp(-0.5 * v * v) / sqrt(2.0 * 3.14159265358979323846);", ";",
+     [pins.test_activation_derivatives_closed_forms, pins.test_backward_one_expert_top1_is_dense_ffn_autograd]),
+    ("swiglu_grad_gate_up_swapped", "double dg = dh[n] * pre[H + n] * orc_silu_grad(pre[n]);",
+     "double dg = dh[n] * pre[n] * orc_silu_grad(pre[H + n]);",
+     [pins.test_backward_one_expert_top1_is_dense_ffn_autograd]),
+    ("expert_grad_unscaled", "for (int64_t c = 0; c < D; ++c) go[c] = w[t * K + j] * dyr[c];",
+     "for (int64_t c = 0; c < D; ++c) go[c] = dyr[c];",
+     [pins.test_backward_matches_central_differences]),
+    ("softmax_grad_not_centred", "ds[sel[t * K + j]] += w[t * K + j] * (dw[j] - wdw);",
+     "ds[sel[t * K + j]] += w[t * K + j] * dw[j];",
+     [pins.test_backward_matches_central_differences]),
+    ("switch_grad_sign", "ds[e] += alpha_switch * ((double)N / (double)T) * p[e] * (f[e] - fp);",
+     "ds[e] -= alpha_switch * ((double)N / (double)T) * p[e] * (f[e] - fp);",
+     [pins.test_backward_matches_central_differences]),
     ("p_mean_not_averaged", "for (int64_t e = 0; e < N; ++e) p_mean[e] /= (double)T;",
      "for (int64_t e = 0; e < N; ++e) p_mean[e] /= 1.0;",
      [pins.test_aux_stats_invariants_and_library_checks]),

@@ -386,6 +386,96 @@ def test_large_capacity_is_the_plain_layer():
     np.testing.assert_array_equal(a["y"], b["y"])
 
 
+# --------------------------------------------------------------------------- backward
+def _objective(x, Wg, W1, W2, bg, b1, b2, bsel, dy, K, act, a_s, a_i):
+    """sum(y * dy) + a_s * switch + a_i * cv2_importance, from the pinned forward and statistics."""
+    out = oracle.moe_layer(x, Wg, W1, W2, K=K, act=act, dtype_tag=oracle.F32, bg=bg, b1=b1, b2=b2, bsel=bsel,
+                           threads=1)
+    st = oracle.aux_stats(out["scores"], out["sel"], out["w"], Wg.shape[1])
+    return float((out["y"] * dy).sum() + a_s * st["switch"] + a_i * st["cv2_importance"]), out["sel"]
+
+
+@pytest.mark.parametrize("act", [oracle.ACT_GELU, oracle.ACT_SWIGLU])
+def test_backward_matches_central_differences(act):
+    """Every gradient of the backward against central differences of the pinned forward (and
+    statistics) on a tiny layer with router and selection biases and both trainable auxiliary
+    losses.  The step is the difference of the two fp32-rounded perturbed values, so rounding of
+    the stored parameter does not enter; entries whose perturbation changes the kept set are
+    skipped."""
+    rng = np.random.default_rng(91 + act)
+    T, D, H, N, K = 7, 6, 5, 4, 2
+    x, Wg, W1, W2, b1, b2 = _rand_layer(rng, T, D, H, N, act, act == oracle.ACT_GELU)
+    bg = (rng.standard_normal(N) * 0.3).astype(np.float32)
+    bsel = (rng.standard_normal(N) * 0.2).astype(np.float32)
+    dy = rng.standard_normal((T, D))
+    a_s, a_i = 0.7, 1.3
+    g = oracle.moe_layer_backward(x, Wg, W1, W2, dy, K=K, act=act, dtype_tag=oracle.F32, bg=bg, b1=b1, b2=b2,
+                                  bsel=bsel, alpha_switch=a_s, alpha_importance=a_i)
+    params = dict(x=x, Wg=Wg, bg=bg, W1=W1, W2=W2)
+    if act == oracle.ACT_GELU:
+        params.update(b1=b1, b2=b2)
+    names = dict(x="dx", Wg="dWg", bg="dbg", W1="dW1", W2="dW2", b1="db1", b2="db2")
+    _, sel0 = _objective(x, Wg, W1, W2, bg, b1, b2, bsel, dy, K, act, a_s, a_i)
+    checked = 0
+    for name, arr in params.items():
+        for flat in rng.choice(arr.size, size=min(8, arr.size), replace=False):
+            idx = np.unravel_index(flat, arr.shape)
+            base = arr[idx]
+            vals = {}
+            for sgn in (1, -1):
+                arr[idx] = np.float32(base + sgn * 1e-3)
+                kw = dict(params)
+                Jv, sel = _objective(kw["x"], kw["Wg"], kw["W1"], kw["W2"], kw["bg"], kw.get("b1", b1),
+                                     kw.get("b2", b2), bsel, dy, K, act, a_s, a_i)
+                vals[sgn] = (Jv, float(arr[idx]), np.array_equal(sel, sel0))
+            arr[idx] = base
+            if not (vals[1][2] and vals[-1][2]):
+                continue
+            fd = (vals[1][0] - vals[-1][0]) / (vals[1][1] - vals[-1][1])
+            an = g[names[name]][idx]
+            assert an == pytest.approx(fd, rel=2e-5, abs=2e-7), (name, idx)
+            checked += 1
+    assert checked >= 30
+
+
+@pytest.mark.parametrize("act,bias", [(oracle.ACT_GELU, True), (oracle.ACT_SWIGLU, False)])
+def test_backward_one_expert_top1_is_dense_ffn_autograd(act, bias):
+    """A 1-expert top-1 layer's backward is the dense FFN's (library autograd in fp64); the router
+    gets no gradient (its only gate weight is the constant 1)."""
+    rng = np.random.default_rng(95 + act)
+    T, D, H = 9, 8, 12
+    x, Wg, W1, W2, b1, b2 = _rand_layer(rng, T, D, H, 1, act, bias)
+    dy = rng.standard_normal((T, D))
+    g = oracle.moe_layer_backward(x, Wg, W1, W2, dy, K=1, act=act, dtype_tag=oracle.F32, b1=b1, b2=b2)
+    xt = torch.from_numpy(x.astype(np.float64)).requires_grad_()
+    W1t = torch.from_numpy(W1[0].astype(np.float64)).requires_grad_()
+    W2t = torch.from_numpy(W2[0].astype(np.float64)).requires_grad_()
+    b1t = torch.from_numpy(b1[0].astype(np.float64)).requires_grad_() if bias else None
+    b2t = torch.from_numpy(b2[0].astype(np.float64)).requires_grad_() if bias else None
+    if act == oracle.ACT_GELU:
+        y = F.linear(F.gelu(F.linear(xt, W1t, b1t), approximate="none"), W2t, b2t)
+    else:
+        gu = F.linear(xt, W1t)
+        y = F.linear(F.silu(gu[:, :H]) * gu[:, H:], W2t)
+    (y * torch.from_numpy(dy)).sum().backward()
+    np.testing.assert_allclose(g["dx"], xt.grad.numpy(), rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(g["dW1"][0], W1t.grad.numpy(), rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(g["dW2"][0], W2t.grad.numpy(), rtol=1e-12, atol=1e-13)
+    if bias:
+        np.testing.assert_allclose(g["db1"][0], b1t.grad.numpy(), rtol=1e-12, atol=1e-13)
+        np.testing.assert_allclose(g["db2"][0], b2t.grad.numpy(), rtol=1e-12, atol=1e-13)
+    assert np.all(g["dWg"] == 0) and np.all(g["dbg"] == 0)
+
+
+def test_activation_derivatives_closed_forms():
+    """GELU'(0) = 1/2, GELU'(v) + GELU'(-v) = 1 (odd part of GELU is v/2); SiLU'(0) = 1/2."""
+    assert oracle.lib().orc_gelu_grad(0.0) == pytest.approx(0.5, rel=1e-15)
+    assert oracle.lib().orc_silu_grad(0.0) == pytest.approx(0.5, rel=1e-15)
+    for v in (0.3, 1.1, 2.7):
+        assert oracle.lib().orc_gelu_grad(v) + oracle.lib().orc_gelu_grad(-v) == pytest.approx(1.0, rel=1e-14)
+        assert oracle.lib().orc_silu_grad(v) + oracle.lib().orc_silu_grad(-v) == pytest.approx(1.0, rel=1e-14)
+
+
 # --------------------------------------------------------------------------- statistics
 def test_balance_loss_extremes(golden_dir):
     g = _golden(golden_dir, "balance_loss_extremes.json")
