@@ -330,6 +330,33 @@ int moe_ep_experts(const moe_config *cfg_local, const void *recv_x, int64_t M, c
 int moe_ep_combine(const moe_config *cfg, const float *z_back, int64_t T, const int32_t *send_pos, void *y,
                    int32_t y_dtype, moe_stream_t stream);
 
+/* Backward pass ("Extending Raschka's GPT-2: an MoE trained from scratch on an
+ * RTX 3090", section on making the router trainable: the router learns
+ * through the gate weights it produces and through the auxiliary loss).
+ * The gradients of  sum(y * dy) + alpha_switch * switch + alpha_importance *
+ * cv2_importance  (the moe_aux scalars [0] and [2]; the count-based scalars
+ * [1] and [3] are piecewise constant and have no gradient) with respect to
+ * x and every parameter, for the routing the forward chooses on the same
+ * inputs (recomputed here; no forward state is kept).  All device memory,
+ * fp32, overwritten:
+ *   dx [T, D]; dW_g [D, N]; db_g [N] (or NULL); dW1 like W1; db1 [N, H] and
+ *   db2 [N, D] (GELU with has_bias, else NULL); dW2 [N, D, H].
+ * dy [T, D] fp32.  Shared experts and capacity limits are not supported
+ * (MOE_ERR_UNSUPPORTED).  ws: moe_backward_workspace_size(cfg, T) bytes. */
+typedef struct {
+    float *dx;
+    float *dW_g;
+    float *db_g;
+    float *dW1;
+    float *db1;
+    float *dW2;
+    float *db2;
+} moe_grads;
+size_t moe_backward_workspace_size(const moe_config *cfg, int64_t T);
+int moe_backward(const moe_config *cfg, const void *x, int64_t T, const moe_weights *w, const float *dy,
+                 float alpha_switch, float alpha_importance, moe_grads *grads, void *ws, size_t ws_bytes,
+                 moe_stream_t stream);
+
 /* Where moe_forward leaves its intermediates inside the workspace (byte
  * offsets from ws), for inspection in tests.  Rows of each expert's segment in
  * the permuted buffers start at a multiple of row_align; rows past an expert's

@@ -38,7 +38,7 @@ MOE_NOALLOC_SCRATCH_BYTES = 2 << 20
 EXPORTED = ("moe_workspace_size", "moe_route", "moe_forward", "moe_forward_timed", "moe_aux_stats",
             "moe_aux_stats_noalloc", "moe_aux_partials", "moe_aux_finalize", "moe_aux_finalize_host",
             "moe_ep_workspace_size", "moe_ep_dispatch", "moe_ep_experts_workspace_size", "moe_ep_experts",
-            "moe_ep_combine",
+            "moe_ep_combine", "moe_backward_workspace_size", "moe_backward",
             "moe_get_workspace_layout", "moe_total_params", "moe_active_params", "moe_get_device_status",
             "moe_launch_count", "moe_error_string", "moe_selftest_wait_timeout")
 
@@ -59,6 +59,11 @@ class moe_weights(ctypes.Structure):
 class moe_aux(ctypes.Structure):
     _fields_ = [("counts", ctypes.c_void_p), ("importance", ctypes.c_void_p), ("p_mean", ctypes.c_void_p),
                 ("scalars", ctypes.c_void_p)]
+
+
+class moe_grads(ctypes.Structure):
+    _fields_ = [("dx", ctypes.c_void_p), ("dW_g", ctypes.c_void_p), ("db_g", ctypes.c_void_p),
+                ("dW1", ctypes.c_void_p), ("db1", ctypes.c_void_p), ("dW2", ctypes.c_void_p), ("db2", ctypes.c_void_p)]
 
 
 class moe_workspace_layout(ctypes.Structure):
@@ -118,6 +123,11 @@ def load_library():
     L.moe_ep_experts.argtypes = [cfgp, vp, i64, vp, vp, wp, vp, vp, sz, vp]
     L.moe_ep_combine.restype = ctypes.c_int
     L.moe_ep_combine.argtypes = [cfgp, vp, i64, vp, vp, i32, vp]
+    L.moe_backward_workspace_size.restype = sz
+    L.moe_backward_workspace_size.argtypes = [cfgp, i64]
+    L.moe_backward.restype = ctypes.c_int
+    L.moe_backward.argtypes = [cfgp, vp, i64, wp, vp, ctypes.c_float, ctypes.c_float, ctypes.POINTER(moe_grads), vp,
+                               sz, vp]
     L.moe_get_workspace_layout.restype = ctypes.c_int
     L.moe_get_workspace_layout.argtypes = [cfgp, i64, ctypes.POINTER(moe_workspace_layout)]
     L.moe_total_params.restype = i64
@@ -276,6 +286,20 @@ def moe_ep_experts(cfg_local, recv_x, M, recv_expert, recv_w, weights_local, z_o
 def moe_ep_combine(cfg, z_back, T, send_pos, y, y_dtype, stream=None) -> int:
     return load_library().moe_ep_combine(ctypes.byref(cfg), _ptr(z_back), T, _ptr(send_pos), _ptr(y), y_dtype,
                                          _stream(stream))
+
+
+def make_grads(dx, dW_g, dW1, dW2, db_g=None, db1=None, db2=None) -> moe_grads:
+    return moe_grads(_ptr(dx), _ptr(dW_g), _ptr(db_g), _ptr(dW1), _ptr(db1), _ptr(dW2), _ptr(db2))
+
+
+def moe_backward_workspace_size(cfg, T) -> int:
+    return load_library().moe_backward_workspace_size(ctypes.byref(cfg), T)
+
+
+def moe_backward(cfg, x, T, weights, dy, alpha_switch, alpha_importance, grads, ws, ws_bytes, stream=None) -> int:
+    return load_library().moe_backward(ctypes.byref(cfg), _ptr(x), T, ctypes.byref(weights), _ptr(dy),
+                                       float(alpha_switch), float(alpha_importance), ctypes.byref(grads), _ptr(ws),
+                                       ws_bytes, _stream(stream))
 
 
 def moe_get_workspace_layout(cfg, T) -> moe_workspace_layout:

@@ -12,6 +12,7 @@
 // No call synchronises the stream or allocates memory (moe_get_device_status
 // excepted, which synchronises the device).
 #include "../../include/moe.h"
+#include "moe_backward.cuh"
 #include "moe_common.cuh"
 #include "moe_decode_fused.cuh"
 #include "moe_gemm_simt.cuh"
@@ -1465,6 +1466,211 @@ int moe_ep_combine(const moe_config *cfg, const float *z_back, int64_t T, const 
                           1, (const float *)nullptr, static_cast<float *>(y));
     return launch_pdl(combine_kernel<__nv_bfloat16>, dim3(grid), dim3(256), 0, s, z_back, T, P.D, P.K,
                       (const int *)send_pos, 1, (const float *)nullptr, static_cast<__nv_bfloat16 *>(y));
+}
+
+// ---------------------------------------------------------------- backward
+}  // extern "C"
+
+namespace {
+struct BwdPlan {
+    Plan P;
+    int rows1;
+    size_t g, pre, dhr, h, dA, gw, dxp, dw, ds, dxr, part, f, dimp, total;
+};
+
+int make_bwd_plan(const moe_config *cfg, int64_t T, BwdPlan *b) {
+    MOE_TRY(make_plan(cfg, T, &b->P));
+    const Plan &P = b->P;
+    if (P.n_shared || cfg->capacity_factor > 0.0f) return MOE_ERR_UNSUPPORTED;
+    b->rows1 = P.act == MOE_ACT_SWIGLU ? 2 * P.H : P.H;
+    size_t off = align256(P.total);
+    auto take = [&](size_t bytes) {
+        const size_t o = off;
+        off = align256(off + bytes);
+        return o;
+    };
+    const size_t R = (size_t)P.rows_cap;
+    b->g = take(R * P.D * 4);
+    b->pre = take(R * b->rows1 * 4);
+    b->dhr = take(R * P.H * 4);
+    b->h = take(R * P.H * 4);
+    b->dA = take(R * b->rows1 * 4);
+    b->gw = take(R * P.D * 4);
+    b->dxp = take(R * P.D * 4);
+    b->dw = take(R * 4);
+    b->ds = take((size_t)T * P.N * 4);
+    b->dxr = take((size_t)T * P.D * 4);
+    b->part = take((size_t)(3 * P.N + 1) * 8);
+    b->f = take((size_t)P.N * 4);
+    b->dimp = take((size_t)P.N * 4);
+    b->total = off;
+    return MOE_OK;
+}
+
+template <typename TA, typename TB>
+int launch_gemm_strided(const bwd::GemmParams<TA, TB> &p, int64_t m_extent, cudaStream_t s) {
+    if (m_extent <= 0 || p.N <= 0) return MOE_OK;
+    const dim3 grid((unsigned)cdiv(m_extent, bwd::TM), (unsigned)cdiv(p.N, bwd::TN),
+                    (unsigned)(p.mode == bwd::KGRP ? p.groups : 1));
+    bwd::gemm_strided_kernel<TA, TB><<<grid, 256, 0, s>>>(p);
+    return check_launch();
+}
+
+// The backward GEMMs for one element type of x and the weights (float or bf16).
+template <typename DT>
+int backward_gemms(const BwdPlan &B, const Bufs &b, const void *x, const moe_weights *w, moe_grads *gr, int phase,
+                   cudaStream_t s) {
+    const Plan &P = B.P;
+    const int D = P.D, H = P.H, N = P.N, R1 = B.rows1;
+    const DT *xp = b.at<DT>(P.x_perm);
+    const DT *W1 = static_cast<const DT *>(w->W1);
+    const DT *W2 = static_cast<const DT *>(w->W2);
+    const DT *Wg = static_cast<const DT *>(w->W_g);
+    const int *ro = b.at<int>(P.row_offsets), *cn = b.at<int>(P.counts);
+    if (phase == 0) {
+        // pre = W1 x (per permuted row), dhr = W2^T dy
+        bwd::GemmParams<DT, DT> g1{};
+        g1.A = xp; g1.a_sm = D; g1.a_sk = 1;
+        g1.B = W1; g1.b_sn = D; g1.b_sk = 1; g1.b_group = (int64_t)R1 * D;
+        g1.C = b.at<float>(B.pre); g1.c_sm = R1; g1.c_sn = 1;
+        g1.N = R1; g1.K = D; g1.row_offsets = ro; g1.counts = cn; g1.groups = N; g1.mode = bwd::ROWS;
+        MOE_TRY(launch_gemm_strided(g1, P.rows_cap, s));
+        bwd::GemmParams<float, DT> g2{};
+        g2.A = b.at<float>(B.g); g2.a_sm = D; g2.a_sk = 1;
+        g2.B = W2; g2.b_sn = 1; g2.b_sk = H; g2.b_group = (int64_t)D * H;
+        g2.C = b.at<float>(B.dhr); g2.c_sm = H; g2.c_sn = 1;
+        g2.N = H; g2.K = D; g2.row_offsets = ro; g2.counts = cn; g2.groups = N; g2.mode = bwd::ROWS;
+        return launch_gemm_strided(g2, P.rows_cap, s);
+    }
+    // dx_perm = W1^T da; dxr = W_g ds; dW2 = sum w dy h^T; dW1 = sum da x^T; dW_g = sum x ds^T
+    bwd::GemmParams<float, DT> g3{};
+    g3.A = b.at<float>(B.dA); g3.a_sm = R1; g3.a_sk = 1;
+    g3.B = W1; g3.b_sn = 1; g3.b_sk = D; g3.b_group = (int64_t)R1 * D;
+    g3.C = b.at<float>(B.dxp); g3.c_sm = D; g3.c_sn = 1;
+    g3.N = D; g3.K = R1; g3.row_offsets = ro; g3.counts = cn; g3.groups = N; g3.mode = bwd::ROWS;
+    MOE_TRY(launch_gemm_strided(g3, P.rows_cap, s));
+    bwd::GemmParams<float, DT> g6{};
+    g6.A = b.at<float>(B.ds); g6.a_sm = N; g6.a_sk = 1;
+    g6.B = Wg; g6.b_sn = N; g6.b_sk = 1;
+    g6.C = b.at<float>(B.dxr); g6.c_sm = D; g6.c_sn = 1;
+    g6.M = (int)P.T; g6.N = D; g6.K = N; g6.mode = bwd::DENSE;
+    MOE_TRY(launch_gemm_strided(g6, P.T, s));
+    bwd::GemmParams<float, float> g4{};
+    g4.A = b.at<float>(B.gw); g4.a_sm = 1; g4.a_sk = D;
+    g4.B = b.at<float>(B.h); g4.b_sn = 1; g4.b_sk = H;
+    g4.C = gr->dW2; g4.c_sm = H; g4.c_sn = 1; g4.c_group = (int64_t)D * H;
+    g4.M = D; g4.N = H; g4.row_offsets = ro; g4.counts = cn; g4.groups = N; g4.mode = bwd::KGRP;
+    MOE_TRY(launch_gemm_strided(g4, D, s));
+    bwd::GemmParams<float, DT> g5{};
+    g5.A = b.at<float>(B.dA); g5.a_sm = 1; g5.a_sk = R1;
+    g5.B = xp; g5.b_sn = 1; g5.b_sk = D;
+    g5.C = gr->dW1; g5.c_sm = D; g5.c_sn = 1; g5.c_group = (int64_t)R1 * D;
+    g5.M = R1; g5.N = D; g5.row_offsets = ro; g5.counts = cn; g5.groups = N; g5.mode = bwd::KGRP;
+    MOE_TRY(launch_gemm_strided(g5, R1, s));
+    bwd::GemmParams<DT, float> g7{};
+    g7.A = static_cast<const DT *>(x); g7.a_sm = 1; g7.a_sk = D;
+    g7.B = b.at<float>(B.ds); g7.b_sn = 1; g7.b_sk = N;
+    g7.C = gr->dW_g; g7.c_sm = N; g7.c_sn = 1;
+    g7.M = D; g7.N = N; g7.K = (int)P.T; g7.mode = bwd::DENSE;
+    return launch_gemm_strided(g7, D, s);
+}
+}  // namespace
+
+extern "C" {
+
+size_t moe_backward_workspace_size(const moe_config *cfg, int64_t T) {
+    BwdPlan B;
+    if (make_bwd_plan(cfg, T, &B) != MOE_OK) return 0;
+    return B.total;
+}
+
+int moe_backward(const moe_config *cfg, const void *x, int64_t T, const moe_weights *w, const float *dy,
+                 float alpha_switch, float alpha_importance, moe_grads *gr, void *ws, size_t ws_bytes,
+                 moe_stream_t stream) {
+    BwdPlan B;
+    MOE_TRY(make_bwd_plan(cfg, T, &B));
+    const Plan &P = B.P;
+    MOE_TRY(check_weights(P, w, true));
+    if (!gr || !gr->dx || !gr->dW_g || !gr->dW1 || !gr->dW2) return MOE_ERR_INVALID_ARG;
+    if (P.has_bias && (!gr->db1 || !gr->db2)) return MOE_ERR_INVALID_ARG;
+    if (!(alpha_switch == alpha_switch) || !(alpha_importance == alpha_importance)) return MOE_ERR_INVALID_ARG;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const int D = P.D, H = P.H, N = P.N, K = P.K, R1 = B.rows1;
+    if (T == 0) {
+        const size_t zs[] = {(size_t)D * N * 4, (size_t)N * R1 * D * 4, (size_t)N * D * H * 4};
+        void *zp[] = {gr->dW_g, gr->dW1, gr->dW2};
+        for (int i = 0; i < 3; ++i)
+            if (cudaMemsetAsync(zp[i], 0, zs[i], s) != cudaSuccess) return MOE_ERR_CUDA;
+        if (gr->db_g && cudaMemsetAsync(gr->db_g, 0, (size_t)N * 4, s) != cudaSuccess) return MOE_ERR_CUDA;
+        if (P.has_bias && (cudaMemsetAsync(gr->db1, 0, (size_t)N * H * 4, s) != cudaSuccess ||
+                           cudaMemsetAsync(gr->db2, 0, (size_t)N * D * 4, s) != cudaSuccess))
+            return MOE_ERR_CUDA;
+        return MOE_OK;
+    }
+    if (!x || !aligned16(x) || !dy || !aligned16(dy) || !aligned16(gr->dx)) return MOE_ERR_INVALID_ARG;
+    if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u)) return MOE_ERR_INVALID_ARG;
+    if (ws_bytes < B.total) return MOE_ERR_WORKSPACE_TOO_SMALL;
+    DeviceInfo *dev = nullptr;
+    MOE_TRY(device_info(&dev));
+    Bufs b{static_cast<char *>(ws), &P};
+    float *logits = b.at<float>(P.logits);
+    int *idx = b.at<int>(P.idx);
+    float *tw = b.at<float>(P.w);
+    // the forward's routing and dispatch
+    MOE_TRY(zero_counters(P, b, s));
+    if (P.tc_router) {
+        MOE_TRY(stage_route_tc(P, b, x, w, logits, idx, tw, nullptr, nullptr, nullptr, s));
+    } else {
+        MOE_TRY(stage_route(P, b, x, w, logits, idx, tw, *dev, s));
+        MOE_TRY(stage_scan(P, b, nullptr, s));
+    }
+    MOE_TRY(stage_permute(P, b, x, nullptr, *dev, s));
+    const int grid_ew = (int)std::min<int64_t>(cdiv(P.rows_cap * (D / 4), 256), (int64_t)dev->sms * 8);
+    bwd::gather_rows_kernel<<<grid_ew, 256, 0, s>>>(dy, P.rows_cap, D, K, b.at<int>(P.perm_slot), b.at<float>(B.g));
+    MOE_TRY(check_launch());
+    if (P.dtype == MOE_F32) MOE_TRY(backward_gemms<float>(B, b, x, w, gr, 0, s));
+    else MOE_TRY(backward_gemms<__nv_bfloat16>(B, b, x, w, gr, 0, s));
+    const bool swiglu = P.act == MOE_ACT_SWIGLU;
+    bwd::act_backward_kernel<<<(unsigned)cdiv(P.rows_cap * 32, 256), 256, 0, s>>>(
+        b.at<float>(B.pre), b.at<float>(B.dhr), b.at<float>(B.g), P.rows_cap, D, H, swiglu ? 1 : 0,
+        b.at<int>(P.perm_slot), idx, tw, swiglu ? nullptr : w->b1, swiglu ? nullptr : w->b2, b.at<float>(B.h),
+        b.at<float>(B.dA), b.at<float>(B.gw), b.at<float>(B.dw));
+    MOE_TRY(check_launch());
+    // the auxiliary losses' batch quantities, then the router scores' gradient
+    unsigned long long *part = b.at<unsigned long long>(B.part);
+    if (cudaMemsetAsync(part, 0, (size_t)(3 * N + 1) * 8, s) != cudaSuccess) return MOE_ERR_CUDA;
+    aux_partials_kernel<<<(int)std::max<int64_t>(1, std::min<int64_t>(cdiv(T, 8), (int64_t)dev->sms * 4)), 256,
+                          (size_t)3 * N * 8, s>>>(logits, idx, tw, (int)T, N, K, part);
+    MOE_TRY(check_launch());
+    bwd::aux_grad_prep_kernel<<<1, 32, 0, s>>>(N, K, reinterpret_cast<const long long *>(part), b.at<float>(B.f),
+                                               b.at<float>(B.dimp));
+    MOE_TRY(check_launch());
+    bwd::router_backward_kernel<<<(unsigned)cdiv(T * 32, 256), 256, 0, s>>>(
+        logits, idx, tw, b.at<int>(P.slot_row), b.at<float>(B.dw), b.at<float>(B.f), b.at<float>(B.dimp), (int)T, N,
+        K, alpha_switch, alpha_importance, b.at<float>(B.ds));
+    MOE_TRY(check_launch());
+    if (P.dtype == MOE_F32) MOE_TRY(backward_gemms<float>(B, b, x, w, gr, 1, s));
+    else MOE_TRY(backward_gemms<__nv_bfloat16>(B, b, x, w, gr, 1, s));
+    // dx[t] = sum_j dx_perm[row of (t, j)] in slot order + W_g ds[t]
+    const int grid_c = (int)std::min<int64_t>(cdiv(T * (D / 4), 256), (int64_t)dev->sms * 8);
+    combine_kernel<float><<<grid_c, 256, 0, s>>>(b.at<float>(B.dxp), T, D, K, b.at<int>(P.slot_row), 1,
+                                                 b.at<float>(B.dxr), gr->dx);
+    MOE_TRY(check_launch());
+    // bias gradients: column sums over each expert's rows (row order), over the tokens for b_g
+    if (P.has_bias) {
+        bwd::column_sums_kernel<<<dim3((unsigned)cdiv(D, 256), (unsigned)N), 256, 0, s>>>(
+            b.at<float>(B.gw), D, D, b.at<int>(P.row_offsets), b.at<int>(P.counts), 0, gr->db2);
+        MOE_TRY(check_launch());
+        bwd::column_sums_kernel<<<dim3((unsigned)cdiv(H, 256), (unsigned)N), 256, 0, s>>>(
+            b.at<float>(B.dA), R1, H, b.at<int>(P.row_offsets), b.at<int>(P.counts), 0, gr->db1);
+        MOE_TRY(check_launch());
+    }
+    if (gr->db_g) {
+        bwd::column_sums_kernel<<<dim3((unsigned)cdiv(N, 256), 1), 256, 0, s>>>(b.at<float>(B.ds), N, N, nullptr,
+                                                                                 nullptr, T, gr->db_g);
+        MOE_TRY(check_launch());
+    }
+    return MOE_OK;
 }
 
 int64_t moe_total_params(const moe_config *c) {
