@@ -1059,6 +1059,21 @@ int launch_fused_nt(int nt, const CUtensorMap &mw1, const CUtensorMap &mxp, cons
     return launch_fused<64, EPI>(mw1, mxp, mw2, mh, p, grid, s);
 }
 
+// Whether the fused kernel's routing scratch fits its ring for this layer.
+template <int EPI>
+bool fused_fits_nt(int nt, size_t scratch) {
+    if (nt == 16) return scratch <= dfu::Shape<16, EPI>::kRingBytes;
+    if (nt == 32) return scratch <= dfu::Shape<32, EPI>::kRingBytes;
+    return scratch <= dfu::Shape<64, EPI>::kRingBytes;
+}
+bool fused_fits(const Plan &P) {
+    const size_t scratch = std::max<size_t>(((size_t)P.T * P.slab_rows + (size_t)P.slab_rows * 32 +
+                                             (size_t)(dfu::kThreads / 32) * P.T * 32) * 4,
+                                            (size_t)2 * dfu::kMaxSlots * 4);
+    return P.act == MOE_ACT_SWIGLU ? fused_fits_nt<dec::EPI_SWIGLU>(P.nt, scratch)
+                                   : fused_fits_nt<dec::EPI_GELU>(P.nt, scratch);
+}
+
 // The whole layer for few tokens in one cooperative kernel (moe_decode_fused.cuh).
 int stage_decode_fused(const Plan &P, const Bufs &b, const void *x, const moe_weights *w, void *y, int y_dtype,
                        moe_aux *aux, const DeviceInfo &dev, cudaStream_t s) {
@@ -1174,7 +1189,7 @@ int forward_impl(const moe_config *cfg, const void *x, int64_t T, const moe_weig
     // few tokens: the whole layer in one cooperative kernel when the device can
     // hold one CTA per token and W_g allows the routing's 16-byte loads
     if (P.fused_decode && dev->sms >= (int)P.T && dev->sms >= P.n_slabs && dev->sms <= P.dec_cap &&
-        aligned16(w->W_g)) {
+        aligned16(w->W_g) && fused_fits(P)) {
         for (int i = 1; i <= 3; ++i) MOE_TRY(rec(i));
         MOE_TRY(stage_decode_fused(P, b, x, w, y, y_dtype, aux, *dev, s));
         for (int i = 4; i <= MOE_N_STAGES; ++i) MOE_TRY(rec(i));
@@ -1626,14 +1641,16 @@ int moe_backward(const moe_config *cfg, const void *x, int64_t T, const moe_weig
     }
     MOE_TRY(stage_permute(P, b, x, nullptr, *dev, s));
     const int grid_ew = (int)std::min<int64_t>(cdiv(P.rows_cap * (D / 4), 256), (int64_t)dev->sms * 8);
-    bwd::gather_rows_kernel<<<grid_ew, 256, 0, s>>>(dy, P.rows_cap, D, K, b.at<int>(P.perm_slot), b.at<float>(B.g));
+    const int *row_end = b.at<int>(P.row_offsets) + N;   // rows past it are outside every segment
+    bwd::gather_rows_kernel<<<grid_ew, 256, 0, s>>>(dy, P.rows_cap, D, K, b.at<int>(P.perm_slot), row_end,
+                                                    b.at<float>(B.g));
     MOE_TRY(check_launch());
     if (P.dtype == MOE_F32) MOE_TRY(backward_gemms<float>(B, b, x, w, gr, 0, s));
     else MOE_TRY(backward_gemms<__nv_bfloat16>(B, b, x, w, gr, 0, s));
     const bool swiglu = P.act == MOE_ACT_SWIGLU;
     bwd::act_backward_kernel<<<(unsigned)cdiv(P.rows_cap * 32, 256), 256, 0, s>>>(
         b.at<float>(B.pre), b.at<float>(B.dhr), b.at<float>(B.g), P.rows_cap, D, H, swiglu ? 1 : 0,
-        b.at<int>(P.perm_slot), idx, tw, swiglu ? nullptr : w->b1, swiglu ? nullptr : w->b2, b.at<float>(B.h),
+        b.at<int>(P.perm_slot), row_end, idx, tw, swiglu ? nullptr : w->b1, swiglu ? nullptr : w->b2, b.at<float>(B.h),
         b.at<float>(B.dA), b.at<float>(B.gw), b.at<float>(B.dw));
     MOE_TRY(check_launch());
     // the auxiliary losses' batch quantities, then the router scores' gradient

@@ -139,14 +139,18 @@ __global__ void __launch_bounds__(256) gemm_strided_kernel(const GemmParams<TA, 
 }
 
 // The upstream gradient per permuted row: g[r] = dy[token of r] (fp32), 0 on
-// padding rows.  Grid-stride over rows_cap * D / 4 float4s.
+// padding rows and on the rows past the last segment (*row_end = the end of
+// the last expert's segment; perm_slot holds nothing there).  Grid-stride over
+// rows_cap * D / 4 float4s.
 __global__ void __launch_bounds__(256) gather_rows_kernel(const float *__restrict__ dy, int64_t rows_cap, int D, int K,
-                                                          const int *__restrict__ perm_slot, float *__restrict__ g) {
+                                                          const int *__restrict__ perm_slot,
+                                                          const int *__restrict__ row_end, float *__restrict__ g) {
     const int64_t nq = rows_cap * (D / 4);
+    const int64_t rend = *row_end;
     for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < nq; i += (int64_t)gridDim.x * blockDim.x) {
         const int64_t r = i / (D / 4);
         const int d = (int)(i - r * (D / 4)) * 4;
-        const int slot = perm_slot[r];
+        const int slot = r < rend ? perm_slot[r] : -1;
         float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
         if (slot >= 0) v = *reinterpret_cast<const float4 *>(dy + (int64_t)(slot / K) * D + d);
         *reinterpret_cast<float4 *>(g + r * D + d) = v;
@@ -162,10 +166,11 @@ __device__ __forceinline__ float sigmoid_f(float v) { return 1.0f / (1.0f + expf
 // Per permuted row (one warp per row): the activation and its backward.
 //   pre [rows, rows1] (W1 x, without b1), dhr [rows, H] (W2^T dy), g [rows, D] (dy rows)
 //   -> h [rows, H] fp32, dA [rows, rows1], gw [rows, D] = w g, dw [rows] = <dhr, h> + <g, b2>
-// Padding rows get zeros everywhere.
+// Padding rows (and the rows past the last segment, *row_end on) get zeros everywhere.
 __global__ void __launch_bounds__(256) act_backward_kernel(const float *__restrict__ pre, const float *__restrict__ dhr,
                                                            const float *__restrict__ g, int64_t rows_cap, int D, int H,
                                                            int swiglu, const int *__restrict__ perm_slot,
+                                                           const int *__restrict__ row_end,
                                                            const int *__restrict__ topk_idx,
                                                            const float *__restrict__ topk_w,
                                                            const float *__restrict__ b1, const float *__restrict__ b2,
@@ -175,7 +180,7 @@ __global__ void __launch_bounds__(256) act_backward_kernel(const float *__restri
     const int64_t r = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
     if (r >= rows_cap) return;
     const int rows1 = swiglu ? 2 * H : H;
-    const int slot = perm_slot[r];
+    const int slot = r < (int64_t)*row_end ? perm_slot[r] : -1;
     const float *pr = pre + r * rows1;
     const float *dr = dhr + r * H;
     float *hr = h + r * H, *ar = dA + r * rows1, *gwr = gw + r * D;
