@@ -103,6 +103,8 @@ def parse(argv=None):
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--mode", default="forward", choices=["forward", "backward"],
+                    help="backward: time the layer's backward pass (moe_backward) instead")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle sample")
     ap.add_argument("--ref-seconds", type=float, default=150.0,
@@ -453,11 +455,87 @@ def e2e_pipelined(moe, cfg, W, ws, wl, T, x_host, steps, warm, flush, dev, aux_b
     return ms, ok
 
 
+def backward_flops(wl, T):
+    """FLOPs of the backward: the minimal chain rule (twice the forward's expert and router
+    contractions) and the recomputed pre-activations on top."""
+    c_up = 4 if wl.act == ACT_SWIGLU else 2
+    minimal = 2 * (T * wl.K * (c_up + 2) * wl.D * wl.H + 2 * T * wl.D * wl.N)
+    return minimal, minimal + T * wl.K * c_up * wl.D * wl.H
+
+
+def run_backward(args, wl):
+    """Time moe_backward (graph-captured, L2 flushed before every step) on one GPU."""
+    import sparse_mixture_experts_10_b200 as moe
+    from sparse_mixture_experts_10_b200 import build as moe_build
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    moe_build.build()
+    moe.load_library()
+    T = wl.T
+    inp = make_inputs(wl, dev, seed=wl.seed)
+    cfg = moe.make_config(wl.D, wl.H, wl.N, wl.K, wl.act, moe.dtype_code(wl.dtype), wl.has_bias)
+    W = moe.make_weights(inp["W_g"], inp["W1"], inp["W2"], inp["b_g"], inp["b1"], inp["b2"], inp["b_sel"])
+    rows1 = 2 * wl.H if wl.act == ACT_SWIGLU else wl.H
+    dy = torch.randn(T, wl.D, device=dev, generator=torch.Generator(device=dev).manual_seed(5))
+    g = dict(dx=torch.empty(T, wl.D, device=dev), dW_g=torch.empty(wl.D, wl.N, device=dev),
+             db_g=torch.empty(wl.N, device=dev), dW1=torch.empty(wl.N, rows1, wl.D, device=dev),
+             dW2=torch.empty(wl.N, wl.D, wl.H, device=dev))
+    if wl.has_bias:
+        g["db1"] = torch.empty(wl.N, wl.H, device=dev)
+        g["db2"] = torch.empty(wl.N, wl.D, device=dev)
+    grads = moe.make_grads(**g)
+    ws = torch.empty(moe.moe_backward_workspace_size(cfg, T), dtype=torch.uint8, device=dev)
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+
+    def step():
+        moe.check(moe.moe_backward(cfg, inp["x"], T, W, dy, 0.01, 0.01, grads, ws, ws.numel()), "backward")
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        step()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    sampler = ClockSampler(0)
+    sampler.start()
+    for a, b in ev:
+        flush.zero_()
+        a.record()
+        graph.replay()
+        b.record()
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    st = moe.moe_get_device_status()
+    if st != 0:
+        raise RuntimeError(f"device status {st}")
+    ms = float(np.mean([a.elapsed_time(b) for a, b in ev]))
+    minimal, with_recompute = backward_flops(wl, T)
+    pk, pk_kind = peaks()
+    # the contractions run on the CUDA cores in fp32: 148 SMs x 128 FMA lanes x 2 FLOP x the clock
+    fp32_peak = 148 * 128 * 2 * float(pk.get("sm_max_mhz", 1965.0)) * 1e6 / 1e12
+    line = {"metric": METRIC + " (backward pass)", "value": T / (ms * 1e-3), "unit": "tokens/s", "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "dtype": "bf16" if wl.dtype == torch.bfloat16 else "f32", "data": "synthetic",
+            "config": config_dict(wl, T, 1) | {"mode": "backward"},
+            "tflops_minimal": minimal / (ms * 1e-3) / 1e12, "tflops_with_recompute": with_recompute / (ms * 1e-3) / 1e12,
+            "roofline": {"bound": "alu", "unit": "TFLOP/s", "achieved": with_recompute / (ms * 1e-3) / 1e12,
+                         "peak": fp32_peak, "peak_kind": "fp32 FMA: 148 SMs x 128 lanes x 2 x max SM clock",
+                         "frac": with_recompute / (ms * 1e-3) / 1e12 / fp32_peak,
+                         "frac_of_bf16_tensor": with_recompute / (ms * 1e-3) / 1e12 / float(pk["bf16_tflops"])},
+            "clocks": clocks}
+    print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse()
     wl = workload_from_args(args)
     if args.impl == "reference":
         run_reference(args, wl)
+        return
+    if args.mode == "backward":
+        run_backward(args, wl)
         return
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
