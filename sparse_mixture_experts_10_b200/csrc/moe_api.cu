@@ -734,9 +734,19 @@ int stage_up(const Plan &P, const Bufs &b, const moe_weights *w, const DeviceInf
             if (swiglu) return launch_tc<128, tc::EPI_SWIGLU>(ma, mb, mo, p, upper, dev.sms, s);
             return launch_tc<128, tc::EPI_GELU>(ma, mb, mo, p, upper, dev.sms, s);
         }
+        // 256-row pair tiles for each expert's pairs of 128-row blocks, then
+        // 128-row tiles on one CTA for the experts' odd last blocks
         const int64_t units = (P.rows_cap / (2 * tc::BM) + N) * p.n_tiles;
-        if (swiglu) return launch_tc2<tc::EPI_SWIGLU>(ma, mb, mo, p, units, dev.pair_clusters, s);
-        return launch_tc2<tc::EPI_GELU>(ma, mb, mo, p, units, dev.pair_clusters, s);
+        p.tail_mode = 1;
+        if (swiglu) MOE_TRY(launch_tc2<tc::EPI_SWIGLU>(ma, mb, mo, p, units, dev.pair_clusters, s));
+        else MOE_TRY(launch_tc2<tc::EPI_GELU>(ma, mb, mo, p, units, dev.pair_clusters, s));
+        tc::Params pt = p;
+        pt.tail_mode = 2;
+        pt.n_tiles = (int)cdiv(H, swiglu ? 64 : 128);
+        CUtensorMap mbt = mb;
+        if (swiglu) MOE_TRY(make_map(&mbt, w->W1, (int64_t)N * 2 * H, D, 64));
+        if (swiglu) return launch_tc<128, tc::EPI_SWIGLU>(ma, mbt, mo, pt, (int64_t)N * pt.n_tiles, dev.sms, s);
+        return launch_tc<128, tc::EPI_GELU>(ma, mbt, mo, pt, (int64_t)N * pt.n_tiles, dev.sms, s);
     }
     simt::Params p{};
     p.A = b.at<float>(P.x_perm);
@@ -796,8 +806,14 @@ int stage_down(const Plan &P, const Bufs &b, const moe_weights *w, void *y, int 
         }
         const int64_t upper = (P.rows_cap / tc::BM) * p.n_tiles;
         if (bn == 128) return launch_tc<128, tc::EPI_SCATTER>(ma, mb, mo, p, upper, dev.sms, s);
-        return launch_tc2<tc::EPI_SCATTER>(ma, mb, mo, p, (P.rows_cap / (2 * tc::BM) + N) * p.n_tiles,
-                                           dev.pair_clusters, s);
+        // pair tiles, then the odd last blocks on one CTA (as in the up projection)
+        p.tail_mode = 1;
+        MOE_TRY(launch_tc2<tc::EPI_SCATTER>(ma, mb, mo, p, (P.rows_cap / (2 * tc::BM) + N) * p.n_tiles,
+                                            dev.pair_clusters, s));
+        tc::Params pt = p;
+        pt.tail_mode = 2;
+        pt.n_tiles = (int)cdiv(D, 128);
+        return launch_tc<128, tc::EPI_SCATTER>(ma, mb, mo, pt, (int64_t)N * pt.n_tiles, dev.sms, s);
     }
     simt::Params p{};
     p.A = b.at<float>(P.h);

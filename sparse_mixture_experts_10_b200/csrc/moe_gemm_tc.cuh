@@ -87,6 +87,12 @@ struct Params {
     // row order (written by bulk tensor stores through tmO); otherwise z rows
     // are indexed by slot.
     int scatter_rows;
+    // Row tiles of a group whose padded segment holds an odd number of 128-row
+    // blocks: the pair kernel's last 256-row unit would be half past the
+    // segment.  tail_mode 1 (pair kernel): leave each such group's last block
+    // out; tail_mode 2 (1-CTA kernel): compute only those blocks, one 128-row
+    // tile per group.  0: every row tile.
+    int tail_mode;
     uint64_t timeout_ns;
 };
 
@@ -106,10 +112,11 @@ struct Shape {
     static constexpr uint32_t kBBytes = BN * BK * 2;
     static constexpr uint32_t kTmemCols = 2 * BN;
     static constexpr size_t kBarrierBytes = (2 * kStages + 5) * 8 + 16;
-    // ring + alignment slack + output staging + barriers + tmem slot; the group table follows
+    // ring + alignment slack + output staging + barriers + tmem slot; the group
+    // table and the tail-tile table follow
     static size_t smem_bytes(int groups) {
         return 1024 + kStages * (size_t)(kABytes + kBBytes) + kOutStageBytes + kBarrierBytes +
-               4 * (size_t)(groups + 1) + 16;
+               8 * (size_t)(groups + 1) + 16;
     }
 };
 
@@ -152,6 +159,24 @@ __device__ __forceinline__ TileCoord decode_tile(int i, const int *s_rowoff, int
     c.g = lo;
     c.nt = local / mtn;
     c.row0 = (mt0 + local - c.nt * mtn) * BM;
+    return c;
+}
+
+// Tile i of the tail tiles (tail_mode 2): s_tcum[g] = number of groups before
+// g whose segment has an odd number of 128-row blocks; each such group has one
+// tile per column tile, its last 128 rows.
+__device__ __forceinline__ TileCoord decode_tail_tile(int i, const int *s_rowoff, const int *s_tcum, int G,
+                                                      int n_tiles) {
+    int lo = 0, hi = G - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (s_tcum[mid] * n_tiles <= i) lo = mid;
+        else hi = mid - 1;
+    }
+    TileCoord c;
+    c.g = lo;
+    c.nt = i - s_tcum[lo] * n_tiles;
+    c.row0 = s_rowoff[lo + 1] - BM;
     return c;
 }
 
@@ -478,8 +503,28 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int G = p.num_groups;
-    if (p.row_offsets)
+    int *s_tcum = s_rowoff + (G + 1);
+    if (p.row_offsets) {
         for (int i = threadIdx.x; i <= G; i += blockDim.x) s_rowoff[i] = p.row_offsets[i];
+        if (p.tail_mode == 2) {
+            __syncthreads();
+            if (warp == 0) {   // groups before each one whose segment has an odd number of blocks
+                int carry = 0;
+                for (int g0 = 0; g0 <= G; g0 += 32) {
+                    const int g = g0 + lane;
+                    const int u = g < G ? ((s_rowoff[g + 1] - s_rowoff[g]) / BM) & 1 : 0;
+                    int incl = u;
+#pragma unroll
+                    for (int o = 1; o < 32; o <<= 1) {
+                        const int n = __shfl_up_sync(0xffffffffu, incl, o);
+                        if (lane >= o) incl += n;
+                    }
+                    if (g <= G) s_tcum[g] = carry + incl - u;
+                    carry += __shfl_sync(0xffffffffu, incl, 31);
+                }
+            }
+        }
+    }
     if (warp == 0 && lane == 0) {
         for (int s = 0; s < kStages; ++s) {
             mbar_init(&full[s], 1);
@@ -502,7 +547,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int *rowoff = p.row_offsets ? s_rowoff : nullptr;
     const int dense_mtiles = (p.dense_rows + BM - 1) / BM;
     const int m_tiles = rowoff ? s_rowoff[G] / BM : dense_mtiles;
-    const int total = m_tiles * p.n_tiles;
+    const bool tails = rowoff && p.tail_mode == 2;
+    const int total = tails ? s_tcum[G] * p.n_tiles : m_tiles * p.n_tiles;
+    auto tile_of = [&](int i) {
+        return tails ? decode_tail_tile(i, s_rowoff, s_tcum, G, p.n_tiles)
+                     : decode_tile(i, rowoff, G, p.n_tiles, dense_mtiles);
+    };
 
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
@@ -512,7 +562,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             bool ok = true;
             IssuedSlots iss;
             for (int i = blockIdx.x; i < total && ok; i += gridDim.x) {
-                const TileCoord c = decode_tile(i, rowoff, G, p.n_tiles, dense_mtiles);
+                const TileCoord c = tile_of(i);
                 int brow, brow2 = 0;
                 if (EPI == EPI_SWIGLU) {
                     brow = c.g * p.b_group_rows + c.nt * (BN / 2);
@@ -594,7 +644,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = blockIdx.x; i < total; i += gridDim.x, ++local) {
             const int a = local & 1;
             const uint32_t aph = (local >> 1) & 1;
-            const TileCoord c = decode_tile(i, rowoff, G, p.n_tiles, dense_mtiles);
+            const TileCoord c = tile_of(i);
             const int row_limit = rowoff ? s_rowoff[c.g + 1] : p.dense_rows;
             const RowGate rg = load_row_gate<EPI>(p, c.row0 + r_in_tile, row_limit);
             // warp-uniform decision: the TMEM loads below are warp-collective
@@ -748,7 +798,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             int carry = 0;
             for (int g0 = 0; g0 <= G; g0 += 32) {
                 const int g = g0 + lane;
-                const int u = g < G ? (s_rowoff[g + 1] - s_rowoff[g] + 2 * BM - 1) / (2 * BM) : 0;
+                const int blocks = g < G ? (s_rowoff[g + 1] - s_rowoff[g]) / BM : 0;
+                const int u = p.tail_mode == 1 ? blocks / 2 : (blocks + 1) / 2;   // tail_mode 1: odd tails left out
                 int incl = u;
 #pragma unroll
                 for (int o = 1; o < 32; o <<= 1) {
