@@ -79,8 +79,9 @@ struct Plan {
     // of the decode up- and down-projections and of the shared expert's two
     // decode GEMMs (dec_cap each); then the fused decode kernel's combine
     // tickets (one per 128 output features); then the routers' per-expert
-    // probability and gate-weight sums (u64, N each).  Word 4 counts the fused
-    // decode kernel's grid barrier arrivals.
+    // probability and gate-weight sums (u64, N each).  Words 4, 8 and 9 count
+    // the fused decode kernel's grid barrier arrivals, word 7 the cooperative
+    // SIMT router's.
     size_t counters_bytes;
     size_t stat_sums;  // offset inside the counters region of the routers' fixed-point sums [2][N] (u64)
     size_t counters, logits, idx, w, counts, offsets, row_offsets, live, chunk_counts, chunk_base,
@@ -150,7 +151,7 @@ int make_plan(const moe_config *c, int64_t T, Plan *p, bool given_routing = fals
     };
     p->route_splits = p->few_router ? (int)std::min<int64_t>(rtc::kFewMaxSplits, std::max<int64_t>(1, cdiv(D, 256))) : 1;
     p->dec_cap = p->decode ? kDecodeMaxGrid : 0;
-    p->stat_sums = (512 + (size_t)4 * p->dec_cap * 4 + (p->decode ? (size_t)cdiv(D, 128) * 4 : 0) + 7) / 8 * 8;
+    p->stat_sums = (512 + (size_t)4 * p->dec_cap * 4 + 7) / 8 * 8;
     p->counters_bytes = align256(p->stat_sums + (size_t)2 * N * 8);
     p->counters = take(p->counters_bytes);
     p->logits = take((size_t)T * N * 4);
@@ -248,9 +249,12 @@ int device_info(DeviceInfo **out) {
         MOE_FUSED_ATTR(32);
         MOE_FUSED_ATTR(64);
 #undef MOE_FUSED_ATTR
-        MOE_TRY(allow_smem(rtc::router_simt_kernel<8>));
-        MOE_TRY(allow_smem(rtc::router_simt_kernel<16>));
-        MOE_TRY(allow_smem(rtc::router_simt_kernel<32>));
+        MOE_TRY(allow_smem(rtc::router_simt_kernel<8, false>));
+        MOE_TRY(allow_smem(rtc::router_simt_kernel<16, false>));
+        MOE_TRY(allow_smem(rtc::router_simt_kernel<32, false>));
+        MOE_TRY(allow_smem(rtc::router_simt_kernel<8, true>));
+        MOE_TRY(allow_smem(rtc::router_simt_kernel<16, true>));
+        MOE_TRY(allow_smem(rtc::router_simt_kernel<32, true>));
 #define MOE_RTC_ATTR(NP)                                                                                     \
     MOE_TRY(allow_smem(rtc::router_tc_kernel<NP, 8>)); \
     MOE_TRY(allow_smem(rtc::router_tc_kernel<NP, 32>))
@@ -478,7 +482,8 @@ int stage_route_tc(const Plan &P, const Bufs &b, const void *x, const moe_weight
         const __nv_bfloat16 *wg = static_cast<const __nv_bfloat16 *>(w->W_g);
         const unsigned grid = (unsigned)P.n_chunks;
 #define MOE_SIMT(NP) \
-    return launch_pdl(rtc::router_simt_kernel<NP>, dim3(grid), dim3(256), rtc::SimtShape<NP>::smem_bytes(D), s, xb, wg, p)
+    return launch_pdl(rtc::router_simt_kernel<NP, false>, dim3(grid), dim3(256), rtc::SimtShape<NP>::smem_bytes(D), s, xb, \
+                      wg, p)
         if (P.np == 8) MOE_SIMT(8);
         if (P.np == 16) MOE_SIMT(16);
         MOE_SIMT(32);
@@ -501,6 +506,83 @@ int stage_route_tc(const Plan &P, const Bufs &b, const void *x, const moe_weight
         default: MOE_RTC(256);
     }
 #undef MOE_RTC
+}
+
+// The SIMT router with the dispatch in the same cooperative launch (every chunk's
+// block resident at once): routing, the y clear, a grid barrier, then each
+// block scatters its own chunk.  Sets *done = false, launching nothing, when
+// the blocks would not all be resident; the caller then runs the router and
+// the permute kernel instead.
+template <int NP>
+int launch_simt_dispatch(const Plan &P, const rtc::Params &p, const __nv_bfloat16 *xb, const __nv_bfloat16 *wg,
+                         const DeviceInfo &dev, cudaStream_t s, bool *done) {
+    const size_t smem = rtc::SimtShape<NP>::smem_bytes(P.D);
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, rtc::router_simt_kernel<NP, true>, 256, smem) !=
+        cudaSuccess)
+        return MOE_ERR_CUDA;
+    if ((int64_t)per_sm * dev.sms < P.n_chunks) {
+        *done = false;
+        return MOE_OK;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)P.n_chunks);
+    cfg.blockDim = dim3(256);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, rtc::router_simt_kernel<NP, true>, xb, wg, p);
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+    *done = true;
+    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+int stage_route_simt_dispatch(const Plan &P, const Bufs &b, const void *x, const moe_weights *w, moe_aux *aux,
+                              float *y_zero, const DeviceInfo &dev, cudaStream_t s, bool *done) {
+    rtc::Params p{};
+    p.T = (int)P.T;
+    p.D = P.D;
+    p.N = P.N;
+    p.K = P.K;
+    p.np = P.rnp;
+    p.bg = w->b_g;
+    p.bsel = w->b_sel;
+    p.logits = b.at<float>(P.logits);
+    p.topk_idx = b.at<int>(P.idx);
+    p.topk_w = b.at<float>(P.w);
+    p.tile_counts = b.at<int>(P.chunk_counts);
+    p.sum_p = reinterpret_cast<unsigned long long *>(b.ws + P.counters + P.stat_sums);
+    p.sum_imp = p.sum_p + P.N;
+    p.ticket = b.at<unsigned>(P.counters);
+    p.chunk_base = b.at<int>(P.chunk_base);
+    p.counts = b.at<int>(P.counts);
+    p.offsets = b.at<int>(P.offsets);
+    p.row_offsets = b.at<int>(P.row_offsets);
+    p.perm_slot = b.at<int>(P.perm_slot);
+    p.live = b.at<int>(P.live);
+    p.n_live = b.at<int>(P.counters) + 2;
+    p.capacity = P.capacity;
+    if (aux) {
+        p.aux_counts = aux->counts;
+        p.aux_importance = aux->importance;
+        p.aux_p_mean = aux->p_mean;
+        p.aux_scalars = aux->scalars;
+    }
+    p.y_zero = y_zero;
+    p.x_perm = b.at<__nv_bfloat16>(P.x_perm);
+    p.slot_row = b.at<int>(P.slot_row);
+    p.grid_bar = b.at<unsigned>(P.counters) + 7;
+    p.timeout_ns = kTimeoutNs;
+    const __nv_bfloat16 *xb = static_cast<const __nv_bfloat16 *>(x);
+    const __nv_bfloat16 *wg = static_cast<const __nv_bfloat16 *>(w->W_g);
+    if (P.np == 8) return launch_simt_dispatch<8>(P, p, xb, wg, dev, s, done);
+    if (P.np == 16) return launch_simt_dispatch<16>(P, p, xb, wg, dev, s, done);
+    return launch_simt_dispatch<32>(P, p, xb, wg, dev, s, done);
 }
 
 int stage_route(const Plan &P, const Bufs &b, const void *x, const moe_weights *w, float *logits, int *idx,
@@ -1083,9 +1165,13 @@ bool fused_fits_nt(int nt, size_t scratch) {
     return scratch <= dfu::Shape<64, EPI>::kRingBytes;
 }
 bool fused_fits(const Plan &P) {
-    const size_t scratch = std::max<size_t>(((size_t)P.T * P.slab_rows + (size_t)P.slab_rows * 32 +
-                                             (size_t)(dfu::kThreads / 32) * P.T * 32) * 4,
-                                            (size_t)2 * dfu::kMaxSlots * 4);
+    // R1: x rows, W_g slab and per-warp partials; R2: the slabs' scores of one
+    // token; R3: top-k experts, ranks, gate weights and full softmax
+    const size_t r1 = ((size_t)P.T * P.slab_rows + (size_t)P.slab_rows * 32 +
+                       (size_t)(dfu::kThreads / 32) * P.T * 32) * 4;
+    const size_t r2 = (size_t)P.n_slabs * 32 * 4;
+    const size_t r3 = ((size_t)3 * dfu::kMaxSlots + (size_t)P.T * 32) * 4;
+    const size_t scratch = std::max(r1, std::max(r2, r3));
     return P.act == MOE_ACT_SWIGLU ? fused_fits_nt<dec::EPI_SWIGLU>(P.nt, scratch)
                                    : fused_fits_nt<dec::EPI_GELU>(P.nt, scratch);
 }
@@ -1133,9 +1219,10 @@ int stage_decode_fused(const Plan &P, const Bufs &b, const void *x, const moe_we
     p.tok_p = b.at<float>(P.fd_tokp);
     unsigned *ctr = b.at<unsigned>(P.counters);
     p.bar = ctr + 4;
+    p.bar4 = ctr + 8;
     p.tk_up = ctr + 128;
     p.tk_down = ctr + 128 + P.dec_cap;
-    p.tk_comb = ctr + 128 + 4 * P.dec_cap;
+    p.bar5 = ctr + 9;
     p.part = b.at<float>(P.dec_part);
     p.split_cap = P.dec_cap;
     p.y = y;
@@ -1222,6 +1309,14 @@ int forward_impl(const moe_config *cfg, const void *x, int64_t T, const moe_weig
         MOE_TRY(rec(1));
         MOE_TRY(stage_scan(P, b, nullptr, s));
     } else if (P.tc_router) {
+        // the SIMT router takes the dispatch into its own (cooperative) launch when it can
+        bool dispatched = false;
+        if (P.simt_router) MOE_TRY(stage_route_simt_dispatch(P, b, x, w, aux, y_zero, *dev, s, &dispatched));
+        if (dispatched) {
+            MOE_TRY(rec(1));
+            MOE_TRY(rec(2));
+            goto experts;
+        }
         MOE_TRY(stage_route_tc(P, b, x, w, logits, idx, tw, nullptr, aux, y_zero, s));
         MOE_TRY(rec(1));
     } else {
@@ -1231,6 +1326,7 @@ int forward_impl(const moe_config *cfg, const void *x, int64_t T, const moe_weig
     }
     MOE_TRY(rec(2));
     MOE_TRY(stage_permute(P, b, x, P.simt_router ? nullptr : y_zero, *dev, s));
+experts:
     MOE_TRY(rec(3));
     MOE_TRY(stage_up(P, b, w, *dev, s));
     if (P.n_shared) MOE_TRY(stage_shared_up(P, b, x, w, *dev, s));

@@ -25,9 +25,10 @@
 //       K blocks, GELU / SwiGLU epilogue -> h
 //   --- barrier 4 (h complete): only the hidden-row loads wait for it, so the
 //       down projection's weight tiles stream in while the up projection ends
-//   D   down projection + gate scale -> z (one row per slot); per 128-feature
-//       tile a ticket: the last live expert to finish that tile adds every
-//       token's kept slots in slot order into y (the combine)
+//   D   down projection + gate scale -> z (one row per slot)
+//   --- barrier 5 (z complete), epilogue warps only
+//   C   the combine, shared by all CTAs: y[t] = the kept slots' z rows of token
+//       t in slot order, with many loads in flight per thread
 // The cooperative launch keeps every CTA resident, so the barriers cannot wait
 // on a CTA that never runs; every wait is still bounded by time (status word
 // MOE_STATUS_TIMEOUT on expiry, then the CTA drains and returns).
@@ -64,9 +65,11 @@ struct Params {
     float *z;                      // [T * K, D], slot rows
     float *slab;                   // [n_slabs][T][32]
     float *tok_p;                  // [T][32] full softmax of each token
-    unsigned *bar;                 // grid barrier arrivals (zero at launch)
+    unsigned *bar;                 // arrivals of grid barriers 1-3 (zero at launch)
+    unsigned *bar4;                // arrivals of grid barrier 4 (zero at launch): a counter of its own,
+                                   // since CTAs without up-projection work arrive there before barrier 3
     unsigned *tk_up, *tk_down;     // stream-K tile tickets [split_cap] (zero at launch)
-    unsigned *tk_comb;             // [ceil(D / 128)] combine tickets (zero at launch)
+    unsigned *bar5;                // arrivals of grid barrier 5 (z complete, zero at launch)
     float *part;                   // stream-K partials [split_cap][2][BM][NT]
     int split_cap;
     void *y;                       // [T, D]
@@ -197,12 +200,19 @@ __device__ __forceinline__ void route_r1(const Params &p, uint8_t *scratch) {
     }
 }
 
-__device__ __forceinline__ void route_r2(const Params &p) {
-    const int lane = threadIdx.x & 31;
+// R2 for token t = blockIdx.x: every thread of the CTA loads the slabs' scores
+// into shared memory at once (one round trip), warp 0 adds them in slab order.
+__device__ __forceinline__ void route_r2(const Params &p, uint8_t *scratch) {
+    const int tid = threadIdx.x, lane = tid & 31;
     const int t = blockIdx.x, N = p.N, K = p.K;
+    float *sl = reinterpret_cast<float *>(scratch);   // [n_slabs][32]
+    for (int i = tid; i < p.n_slabs * 32; i += kThreads)
+        sl[i] = __ldcg(p.slab + ((size_t)(i >> 5) * p.T + t) * 32 + (i & 31));
+    __syncthreads();
+    if (tid >= 32) return;
     const bool live = lane < N;
     float s = 0.f;
-    for (int c = 0; c < p.n_slabs; ++c) s += __ldcg(p.slab + ((size_t)c * p.T + t) * 32 + lane);   // slab order
+    for (int c = 0; c < p.n_slabs; ++c) s += sl[c * 32 + lane];   // slab order
     if (live) {
         if (p.bg) s += __ldg(p.bg + lane);
         if (s != s) {
@@ -311,17 +321,22 @@ __device__ __forceinline__ void route_r3(const Params &p, const Tables &tb, uint
             const int end = tb.rowoff[e] + (tb.kept[e] + kRowAlign - 1) / kRowAlign * kRowAlign;
             for (int r = start + lane; r < end; r += 32) p.perm_slot[r] = -1;
         }
-        // statistics of the router's choice: fixed orders (tokens ascending, slots ascending)
+        // statistics of the router's choice: fixed orders (tokens ascending, slots
+        // ascending), from the gate weights and the full softmax loaded at once
         float *f_im = reinterpret_cast<float *>(s_pos);   // [32] scratch once the ranks are consumed
         float *f_pm = f_im + 32;
+        float *s_w = reinterpret_cast<float *>(s_pos + kMaxSlots);   // [T*K]
+        float *s_tp = s_w + kMaxSlots;                               // [T][32]
+        for (int i = tid; i < TK; i += kThreads) s_w[i] = __ldcg(p.topk_w + i);
+        for (int i = tid; i < p.T * 32; i += kThreads) s_tp[i] = __ldcg(p.tok_p + i);
         __syncthreads();
         if (tid < 32) {
             const int e = tid;
             float im = 0.f, pm = 0.f;
             if (e < N) {
                 for (int i = 0; i < TK; ++i)
-                    if (s_idx[i] == e) im += __ldcg(p.topk_w + i);
-                for (int t = 0; t < p.T; ++t) pm += __ldcg(p.tok_p + (size_t)t * 32 + e);
+                    if (s_idx[i] == e) im += s_w[i];
+                for (int t = 0; t < p.T; ++t) pm += s_tp[t * 32 + e];
                 pm /= (float)p.T;
             }
             f_im[e] = im;
@@ -454,7 +469,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     if ((int)blockIdx.x < p.n_slabs) route_r1<NT, EPI_UP>(p, smem);
     ok = grid_sync_all(p, 1, s_flag);
-    if (ok && (int)blockIdx.x < p.T && warp == 0) route_r2(p);
+    if (ok && (int)blockIdx.x < p.T) route_r2(p, smem);
     if (ok) ok = grid_sync_all(p, 2, s_flag);
     if (ok) {
         route_r3(p, tb, smem);
@@ -484,7 +499,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const PhaseWork &w = ph == 0 ? wu : wd;
                 const CUtensorMap *mW = ph == 0 ? &tmW1 : &tmW2;
                 const CUtensorMap *mB = ph == 0 ? &tmXp : &tmH;
-                const unsigned target = (ph == 0 ? 3u : 4u) * gridDim.x;
+                const unsigned *bar = ph == 0 ? p.bar : p.bar4;
+                const unsigned target = (ph == 0 ? 3u : 1u) * gridDim.x;
                 bool ready = false;
                 int ndef = 0;
                 int def_stage[8], def_col[8], def_row[8];
@@ -511,7 +527,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     for (int kb = pc.k0; kb < pc.k1; ++kb) {
                         if (!ready && ndef == kStages) {   // the ring holds only deferred stages: wait for the data
-                            if (!grid_wait(p.bar, target, p.timeout_ns)) {
+                            if (!grid_wait(bar, target, p.timeout_ns)) {
                                 ok = false;
                                 break;
                             }
@@ -529,7 +545,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         } else {
                             tma_load_2d(mW, &full[stage], sA + stage * S::kABytes, kb * BK, wrow);
                         }
-                        if (!ready && dec::ld_acquire_u32(p.bar) >= target) {
+                        if (!ready && dec::ld_acquire_u32(bar) >= target) {
                             ready = true;
                             flush();
                         }
@@ -549,7 +565,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 }
                 if (ok && ndef > 0) {
-                    if (grid_wait(p.bar, target, p.timeout_ns)) flush();
+                    if (grid_wait(bar, target, p.timeout_ns)) flush();
                     else ok = false;
                 }
             }
@@ -748,27 +764,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                             }
                         }
                     }
-                    // the tile's z columns are complete: the last live expert to finish this
-                    // 128-feature tile adds every token's kept slots in slot order (the combine)
-                    if (!eb.sync()) { eok = false; break; }
-                    if (et == 0) s_flag[1] = ticket_arrive(p.tk_comb + mt) == (unsigned)(*tb.nlive - 1);
-                    if (!eb.sync()) { eok = false; break; }
-                    if (s_flag[1] && d < D) {
-                        for (int t = 0; t < p.T; ++t) {
-                            float yv = 0.f;
-                            bool first = true;
-                            for (int j = 0; j < p.K; ++j) {
-                                if (tb.row[t * p.K + j] < 0) continue;   // dropped by the capacity
-                                const float v = __ldcg(p.z + (int64_t)(t * p.K + j) * D + d);
-                                yv = first ? v : yv + v;
-                                first = false;
-                            }
-                            if (p.y_bf16)
-                                static_cast<__nv_bfloat16 *>(p.y)[(int64_t)t * D + d] = __float2bfloat16_rn(yv);
-                            else
-                                static_cast<float *>(p.y)[(int64_t)t * D + d] = yv;
-                        }
-                    }
                 }
             }
             if (ph == 0 && eok) {
@@ -777,7 +772,63 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (et == 0) {
                     __threadfence();
                     fence_proxy_async_global();
-                    grid_arrive(p.bar);
+                    grid_arrive(p.bar4);
+                }
+            }
+        }
+        // ---- the combine: once every CTA's z rows are written (barrier 5), the epilogue
+        // threads of all CTAs share y: y[t, d] = z[t K, d] + ... + z[t K + K - 1, d] in slot
+        // order over the kept slots; four outputs per thread and up to eight slots each have
+        // their loads in flight together
+        if (eok && eb.sync()) {
+            if (et == 0) {
+                __threadfence();
+                grid_arrive(p.bar5);
+                s_flag[1] = grid_wait(p.bar5, gridDim.x, p.timeout_ns) ? 1 : 0;
+            }
+            if (eb.sync() && s_flag[1]) {
+                const int K = p.K;
+                const int64_t O = (int64_t)p.T * D;
+                const int64_t stride = (int64_t)gridDim.x * 128;
+                for (int64_t o0 = (int64_t)blockIdx.x * 128 + et; o0 < O; o0 += 4 * stride) {
+                    float acc[4];
+                    bool any[4];
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        acc[q] = 0.f;
+                        any[q] = false;
+                    }
+                    for (int jb = 0; jb < K; jb += 8) {
+                        float v[4][8];
+                        bool has[4][8];
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            const int64_t o = o0 + q * stride;
+                            const int64_t t = o < O ? o / D : 0;
+                            const int64_t d = o - t * D;
+#pragma unroll
+                            for (int u = 0; u < 8; ++u) {
+                                const int j = jb + u;
+                                has[q][u] = o < O && j < K && tb.row[t * K + j] >= 0;   // dropped by the capacity
+                                v[q][u] = has[q][u] ? __ldcg(p.z + (t * K + j) * D + d) : 0.f;
+                            }
+                        }
+#pragma unroll
+                        for (int q = 0; q < 4; ++q)
+#pragma unroll
+                            for (int u = 0; u < 8; ++u)
+                                if (has[q][u]) {
+                                    acc[q] = any[q] ? acc[q] + v[q][u] : v[q][u];
+                                    any[q] = true;
+                                }
+                    }
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const int64_t o = o0 + q * stride;
+                        if (o >= O) continue;
+                        if (p.y_bf16) static_cast<__nv_bfloat16 *>(p.y)[o] = __float2bfloat16_rn(acc[q]);
+                        else static_cast<float *>(p.y)[o] = acc[q];
+                    }
                 }
             }
         }

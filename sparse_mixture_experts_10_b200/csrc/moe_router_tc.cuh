@@ -68,6 +68,11 @@ struct Params {
     // SIMT router: the layer's fp32 output [T, D] to clear (each block its chunk's
     // rows) for the down projection's reductions, or nullptr
     float *y_zero;
+    // SIMT router with the dispatch (cooperative launch): the kept rows' copies,
+    // the slot -> row map, the arrivals of its grid barrier (zero at launch)
+    __nv_bfloat16 *x_perm;
+    int *slot_row;
+    unsigned *grid_bar;
     uint64_t timeout_ns;
 };
 
@@ -565,7 +570,174 @@ __device__ __forceinline__ float fma_bf16x2_acc(uint32_t x, uint32_t w, float ac
     return acc;
 }
 
-template <int NP>
+// ---------------------------------------------------------------------------
+// The dispatch inside the SIMT router (DISPATCH = true): after a grid barrier
+// (the launch is cooperative, every block resident), every block adds up the
+// chunk counts of all blocks -- per expert its total and the tokens of the
+// chunks before its own, one warp per expert -- and scatters its own chunk's
+// (token, slot) pairs into the expert segments (stable, capacity applied);
+// block 0 writes the tables and the statistics.  This replaces the last
+// block's serial table build and the separate permute launch.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned *ptr) {
+    unsigned v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(ptr) : "memory");
+    return v;
+}
+
+__device__ void simt_dispatch_chunk(const Params &p, const __nv_bfloat16 *__restrict__ x, int n_chunks, int *sm) {
+    const int N = p.N, K = p.K, T = p.T, D = p.D;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int c = blockIdx.x;
+    int *s_tot = sm, *s_base = sm + 32, *s_kept = sm + 64, *s_row = sm + 96;   // s_row [33]
+    int *s_run = sm + 136, *s_dest = sm + 176;                                 // s_dest [chunk * K]
+    for (int e = warp; e < N; e += blockDim.x / 32) {
+        int tot = 0, base = 0;
+        for (int c0 = 0; c0 < n_chunks; c0 += 32) {
+            const int cc = c0 + lane;
+            const int v = cc < n_chunks ? __ldcg(p.tile_counts + (int64_t)cc * N + e) : 0;
+            tot += v;
+            if (cc < c) base += v;
+        }
+        tot = __reduce_add_sync(0xffffffffu, tot);
+        base = __reduce_add_sync(0xffffffffu, base);
+        if (lane == 0) {
+            s_tot[e] = tot;
+            s_base[e] = base;
+        }
+    }
+    __syncthreads();
+    if (warp == 0) {
+        const int cnt = lane < N ? s_tot[lane] : 0;
+        const int kp = min(cnt, p.capacity);
+        const int pad = (kp + kRowAlign - 1) / kRowAlign * kRowAlign;
+        int ik = kp, ip = pad;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int a = __shfl_up_sync(0xffffffffu, ik, o), b = __shfl_up_sync(0xffffffffu, ip, o);
+            if (lane >= o) { ik += a; ip += b; }
+        }
+        s_kept[lane] = kp;
+        s_row[lane] = ip - pad;
+        if (lane == 31) s_row[32] = ip;
+        s_run[lane] = lane < N ? s_base[lane] : 0;
+        if (c == 0) {
+            if (lane < N) {
+                p.counts[lane] = kp;
+                p.offsets[lane] = ik - kp;
+                p.row_offsets[lane] = ip - pad;
+                const float im = (float)((double)__ldcg(p.sum_imp + lane) / kImpScale);
+                const float pm = T > 0 ? (float)((double)__ldcg(p.sum_p + lane) / kImpScale / (double)T) : 0.f;
+                if (p.aux_counts) p.aux_counts[lane] = cnt;
+                if (p.aux_importance) p.aux_importance[lane] = im;
+                if (p.aux_p_mean) p.aux_p_mean[lane] = pm;
+            }
+            const unsigned m = __ballot_sync(0xffffffffu, kp > 0);
+            if (kp > 0) p.live[__popc(m & lanemask_lt())] = lane;
+            const int routed = __reduce_add_sync(0xffffffffu, cnt);
+            if (lane == N - 1) {
+                p.offsets[N] = ik;
+                p.row_offsets[N] = ip;
+            }
+            if (lane == 0) {
+                *p.n_live = __popc(m);
+                if ((int64_t)routed != (int64_t)T * K) set_status(kStatusBounds);
+            }
+        }
+    } else if (warp == 1 && c == 0 && p.aux_scalars) {
+        // f_e = counts / (T K); switch = N sum f P; simple = N sum f^2; CV^2 = popvar / mean^2
+        const double tk = (double)T * (double)K;
+        double sw = 0.0, ss = 0.0, si = 0.0, sc = 0.0, im = 0.0, cn = 0.0;
+        if (lane < N) {
+            cn = s_tot[lane];
+            im = (double)__ldcg(p.sum_imp + lane) / kImpScale;
+            const double pm = T > 0 ? (double)__ldcg(p.sum_p + lane) / kImpScale / (double)T : 0.0;
+            const double fe = tk > 0 ? cn / tk : 0.0;
+            sw = fe * (double)(float)pm;
+            ss = fe * fe;
+            si = (double)(float)im;
+            sc = cn;
+        }
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) {
+            sw += __shfl_xor_sync(0xffffffffu, sw, o);
+            ss += __shfl_xor_sync(0xffffffffu, ss, o);
+            si += __shfl_xor_sync(0xffffffffu, si, o);
+            sc += __shfl_xor_sync(0xffffffffu, sc, o);
+        }
+        const double mi = si / N, mc = sc / N;
+        double vi = lane < N ? ((double)(float)im - mi) * ((double)(float)im - mi) : 0.0;
+        double vc = lane < N ? (cn - mc) * (cn - mc) : 0.0;
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) {
+            vi += __shfl_xor_sync(0xffffffffu, vi, o);
+            vc += __shfl_xor_sync(0xffffffffu, vc, o);
+        }
+        vi /= N;
+        vc /= N;
+        if (lane == 0) {
+            p.aux_scalars[0] = (float)(N * sw);
+            p.aux_scalars[1] = (float)(N * ss);
+            p.aux_scalars[2] = mi == 0.0 ? 0.f : (float)(vi / (mi * mi));
+            p.aux_scalars[3] = mc == 0.0 ? 0.f : (float)(vc / (mc * mc));
+        }
+    }
+    __syncthreads();
+    if (c == 0) {   // padding rows of every segment
+        for (int e = warp; e < N; e += blockDim.x / 32) {
+            const int start = s_row[e] + s_kept[e], end = s_row[e + 1];
+            for (int r = start + lane; r < end; r += 32) p.perm_slot[r] = -1;
+        }
+    }
+    // this chunk's (token, slot) pairs: stable rank inside each expert, then the copies
+    const int t_begin = c * kSimtChunk, t_end = min(T, t_begin + kSimtChunk);
+    const int n_entries = (t_end - t_begin) * K;
+    const int64_t f0 = (int64_t)t_begin * K;
+    if (warp == 0) {
+        for (int base = 0; base < n_entries; base += 32) {
+            const int f = base + lane;
+            int e = f < n_entries ? p.topk_idx[f0 + f] : -1;
+            if (f < n_entries && (e < 0 || e >= N)) {
+                set_status(kStatusBounds);
+                e = -1;
+            }
+            const unsigned peers = __match_any_sync(0xffffffffu, e);
+            const int rank = __popc(peers & lanemask_lt());
+            const int run = e >= 0 ? s_run[e] : 0;
+            __syncwarp();
+            if (e >= 0 && lane == __ffs(peers) - 1) s_run[e] = run + __popc(peers);
+            __syncwarp();
+            if (f < n_entries) {
+                const int pos = run + rank;
+                const int dest = (e >= 0 && pos < s_kept[e]) ? s_row[e] + pos : -1;
+                s_dest[f] = dest;
+                if (dest >= 0) p.perm_slot[dest] = (int)(f0 + f);
+                p.slot_row[f0 + f] = dest;
+            }
+        }
+    }
+    __syncthreads();
+    const int nvec = D / 8;
+    for (int tt = warp; tt < t_end - t_begin; tt += blockDim.x / 32) {
+        const uint4 *src = reinterpret_cast<const uint4 *>(x + (int64_t)(t_begin + tt) * D);
+        for (int v0 = lane; v0 < nvec; v0 += 128) {
+            uint4 r[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+                if (v0 + 32 * u < nvec) r[u] = __ldg(src + v0 + 32 * u);
+            for (int j = 0; j < K; ++j) {
+                const int d = s_dest[tt * K + j];
+                if (d < 0) continue;
+                uint4 *dst = reinterpret_cast<uint4 *>(p.x_perm + (int64_t)d * D);
+#pragma unroll
+                for (int u = 0; u < 4; ++u)
+                    if (v0 + 32 * u < nvec) dst[v0 + 32 * u] = r[u];
+            }
+        }
+    }
+}
+
+template <int NP, bool DISPATCH>
 __global__ void __launch_bounds__(256, NP == 8 ? 2 : 1) router_simt_kernel(const __nv_bfloat16 *__restrict__ x,
                                                                           const __nv_bfloat16 *__restrict__ Wg,
                                                                           const Params p) {
@@ -722,6 +894,35 @@ __global__ void __launch_bounds__(256, NP == 8 ? 2 : 1) router_simt_kernel(const
         p.tile_counts[(int64_t)blockIdx.x * N + tid] = cs;
         atomicAdd(p.sum_p + tid, __double2ull_rn((double)ps * kImpScale));
         atomicAdd(p.sum_imp + tid, is);
+    }
+    if (DISPATCH) {
+        // the chunk's partials are written: arrive, clear this chunk's rows of y
+        // while the others arrive, wait (bounded), then dispatch
+        __syncthreads();
+        if (tid == 0) asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(p.grid_bar) : "memory");
+        if (p.y_zero) {
+            const int64_t t0 = (int64_t)blockIdx.x * kSimtChunk;
+            const int64_t t1 = t0 + kSimtChunk < T ? t0 + kSimtChunk : (int64_t)T;
+            const int64_t n16 = (t1 - t0) * (D / 4);
+            uint4 *yb = reinterpret_cast<uint4 *>(p.y_zero + t0 * D);
+            for (int64_t i = tid; i < n16; i += blockDim.x) yb[i] = make_uint4(0u, 0u, 0u, 0u);
+        }
+        if (tid == 0) {
+            bool ok = ld_acquire_gpu(p.grid_bar) >= gridDim.x;
+            const uint64_t t0 = globaltimer_ns();
+            while (!ok) {
+#pragma unroll 1
+                for (int i = 0; i < 32 && !ok; ++i) ok = ld_acquire_gpu(p.grid_bar) >= gridDim.x;
+                if (!ok && globaltimer_ns() - t0 > p.timeout_ns) {
+                    set_status(kStatusTimeout);
+                    break;
+                }
+            }
+            *s_flag = ok ? 1 : 0;
+        }
+        __syncthreads();
+        if (*s_flag) simt_dispatch_chunk(p, x, gridDim.x, reinterpret_cast<int *>(fs));
+        return;
     }
     const bool last = last_block(p.ticket, s_flag);
     if (last)

@@ -81,14 +81,15 @@ class Layer:
         )
 
 
-def check_routing(V, ref_scores, K, inp):
+def check_routing(V, ref_scores, K, inp, C=None):
     """Logits within tolerance, top-k bit-exact on the device's logits (plus any selection bias,
-    added in fp32 as the device does), counts exact."""
+    added in fp32 as the device does), counts exact (the accepted ones under a capacity C)."""
     ph.assert_logits_close(V["logits"], ref_scores)
     sel = oracle.select_topk(ph.selection_scores(V["logits"], inp).astype(np.float64), K)
     np.testing.assert_array_equal(V["idx"], sel)
     N = V["counts"].shape[0]
-    np.testing.assert_array_equal(V["counts"], np.bincount(sel.ravel(), minlength=N))
+    counts = np.bincount(sel.ravel(), minlength=N)
+    np.testing.assert_array_equal(V["counts"], counts if C is None else np.minimum(counts, C))
 
 
 def check_dispatch(V, x, K, C=None):
@@ -126,7 +127,7 @@ def run_full(wl, inp, y_dtype=torch.float32):
     y, ws, aux = layer.forward(y_dtype=y_dtype)
     V = layer.views(ws, T)
     ref = ph.oracle_full_layer(inp, wl, wl.K, gpu_logits=V["logits"])
-    check_routing(V, ref["scores"], wl.K, inp)
+    check_routing(V, ref["scores"], wl.K, inp, ref.get("capacity"))
     ph.assert_weights_close(V["w"], ref["w"], ref["scores"])
     check_dispatch(V, inp["x"], wl.K, ref.get("capacity"))
     errs = ph.assert_y_close(y.float().cpu().numpy(), ref["y"], wl.dtype if y_dtype == torch.float32 else y_dtype)
@@ -353,7 +354,6 @@ def _full_size_sampled(name, n_rows, seed, every_expert=False):
         live = np.nonzero(V["counts"] > 0)[0]
         covered = np.unique(V["idx"][rows])
         assert np.array_equal(covered, live), "a live expert has no compared output row"
-        assert len(live) > 0.9 * wl.N
         # logits of a strided subset of 1024 rows against the oracle's fp64 scores
         strided = np.arange(0, wl.T, max(1, wl.T // 1024))[:1024]
         ph.assert_logits_close(V["logits"][strided], ph.oracle_scores(inp, wl, strided))
