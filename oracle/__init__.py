@@ -85,7 +85,9 @@ def configure(L):
     L.orc_expert_swiglu.argtypes = [i64, i64, vp, vp, vp, i32, vp, vp]
     L.orc_combine.argtypes = [i64, i64, vp, vp, vp]
     L.orc_add_shared.argtypes = [i64, vp, vp]
-    L.orc_moe_layer_rows.argtypes = [ctypes.POINTER(_Layer), i64, i64, vp, vp, vp, vp, vp, vp]
+    L.orc_moe_layer_rows.argtypes = [ctypes.POINTER(_Layer), i64, i64, vp, vp, vp, vp, vp, vp, vp]
+    L.orc_capacity_reroute.argtypes = [i64, i64, i64, vp, vp, i64, vp]
+    L.orc_selection_values.argtypes = [ctypes.POINTER(_Layer), i64, i64, vp, vp, vp]
     L.orc_gelu_grad.restype = dp
     L.orc_gelu_grad.argtypes = [dp]
     L.orc_silu_grad.restype = dp
@@ -262,7 +264,7 @@ def capacity_keep(sel, N: int, C: int) -> np.ndarray:
 
 
 def moe_layer(x, Wg, W1, W2, *, K, act, dtype_tag, bg=None, b1=None, b2=None, sel_scores=None,
-              threads=None, rows=None, bsel=None, S1=None, S2=None, sb1=None, sb2=None, keep=None):
+              threads=None, rows=None, bsel=None, S1=None, S2=None, sb1=None, sb2=None, keep=None, assign=None):
     """The whole layer on host arrays, in fp64.
 
     x [T, D]; Wg [D, N]; W1 [N, H, D] (GELU) or [N, 2H, D] (SwiGLU); W2 [N, D, H].
@@ -272,6 +274,8 @@ def moe_layer(x, Wg, W1, W2, *, K, act, dtype_tag, bg=None, b1=None, b2=None, se
     (the device's fp32 logits, plus any selection bias in fp32) while the gate
     weights use the fp64 scores.
     keep [T, K] uint8 (optional): capacity decisions (capacity_keep); dropped slots add nothing.
+    assign [T, K] int32 (optional): the expert serving each slot after a reroute
+    (capacity_reroute), -1 for none; each slot keeps its gate weight.
     rows: optional (t0, t1) range; other rows of the outputs are left as zeros.
     Returns dict(scores [T,N], sel [T,K], w [T,K], y [T,D]) in fp64 / int32.
     """
@@ -285,6 +289,7 @@ def moe_layer(x, Wg, W1, W2, *, K, act, dtype_tag, bg=None, b1=None, b2=None, se
     bgm, b1m, b2m = _c(bg, np.float32), _c(b1, np.float32), _c(b2, np.float32)
     ss = _c(sel_scores, np.float32)
     kp = _c(keep, np.uint8)
+    asg = _c(assign, np.int32)
     bselm, S1m, S2m = _c(bsel, np.float32), _mat(S1, dtype_tag), _mat(S2, dtype_tag)
     sb1m, sb2m = _c(sb1, np.float32), _c(sb2, np.float32)
     lay = _Layer(D, H, N, K, act, dtype_tag, _p(xm), _p(Wgm), _p(bgm), _p(W1m), _p(b1m), _p(W2m), _p(b2m),
@@ -302,7 +307,7 @@ def moe_layer(x, Wg, W1, W2, *, K, act, dtype_tag, bg=None, b1=None, b2=None, se
     ranges = [(a, min(a + step, t1)) for a in range(t0, t1, step)]
 
     def run(r):
-        L.orc_moe_layer_rows(ctypes.byref(lay), r[0], r[1], _p(ss), _p(kp), _p(scores), _p(sel), _p(w), _p(y))
+        L.orc_moe_layer_rows(ctypes.byref(lay), r[0], r[1], _p(ss), _p(kp), _p(asg), _p(scores), _p(sel), _p(w), _p(y))
 
     if nthr == 1 or len(ranges) == 1:
         for r in ranges:
@@ -313,17 +318,51 @@ def moe_layer(x, Wg, W1, W2, *, K, act, dtype_tag, bg=None, b1=None, b2=None, se
     return dict(scores=scores, sel=sel, w=w, y=y)
 
 
-def moe_layer_capacity(x, Wg, W1, W2, *, K, act, dtype_tag, cf, sel_scores=None, **kw):
-    """The layer with a per-expert capacity (drop): route every token, decide which
-    assignments fit (rows in order, C = capacity(cf, T, K, N) each), then evaluate."""
+def selection_values(scores, bsel=None, sel_scores=None) -> np.ndarray:
+    """The values experts are ranked on for selection, [T, N] fp64: the given fp32
+    selection scores, else the fp64 scores plus the selection-only bias."""
+    sc = np.ascontiguousarray(scores, dtype=np.float64)
+    T, N = sc.shape
+    bs, ss = _c(bsel, np.float32), _c(sel_scores, np.float32)
+    lay = _Layer(0, 0, N, 0, 0, 0, None, None, None, None, None, None, None, _p(bs), None, None, None, None)
+    v = np.zeros((T, N), dtype=np.float64)
+    lib().orc_selection_values(ctypes.byref(lay), 0, T, _p(sc), _p(ss), _p(v))
+    return v
+
+
+def capacity_reroute(v, sel, C: int) -> np.ndarray:
+    """Reroute decisions [T, K] int32: the expert serving each slot (-1: dropped)."""
+    vv = np.ascontiguousarray(v, dtype=np.float64)
+    sl = np.ascontiguousarray(sel, dtype=np.int32)
+    T, K = sl.shape
+    N = vv.shape[1]
+    assign = np.zeros((T, K), dtype=np.int32)
+    lib().orc_capacity_reroute(T, N, K, _p(vv), _p(sl), int(C), _p(assign))
+    return assign
+
+
+def moe_layer_capacity(x, Wg, W1, W2, *, K, act, dtype_tag, cf, sel_scores=None, overflow="drop", **kw):
+    """The layer with a per-expert capacity: route every token, decide which
+    assignments fit (rows in order, C = capacity(cf, T, K, N) each) and what
+    happens to the others (overflow "drop" or "reroute"), then evaluate."""
     routed = moe_layer(x, Wg, np.zeros_like(W1), np.zeros_like(W2), K=K, act=act, dtype_tag=dtype_tag,
                        sel_scores=sel_scores, **{k: v for k, v in kw.items() if k in ("bg", "bsel", "threads")})
     T = routed["sel"].shape[0]
     N = _mat(Wg, dtype_tag).shape[1]
     C = capacity(cf, T, K, N)
-    keep = capacity_keep(routed["sel"], N, C)
-    out = moe_layer(x, Wg, W1, W2, K=K, act=act, dtype_tag=dtype_tag, sel_scores=sel_scores, keep=keep, **kw)
-    out["keep"], out["capacity"] = keep, C
+    if overflow == "drop":
+        keep = capacity_keep(routed["sel"], N, C)
+        out = moe_layer(x, Wg, W1, W2, K=K, act=act, dtype_tag=dtype_tag, sel_scores=sel_scores, keep=keep, **kw)
+        out["keep"] = keep
+    elif overflow == "reroute":
+        v = selection_values(routed["scores"], kw.get("bsel"), sel_scores)
+        assign = capacity_reroute(v, routed["sel"], C)
+        out = moe_layer(x, Wg, W1, W2, K=K, act=act, dtype_tag=dtype_tag, sel_scores=sel_scores, assign=assign,
+                        **kw)
+        out["assign"], out["keep"] = assign, (assign >= 0).astype(np.uint8)
+    else:
+        raise ValueError(f"overflow must be 'drop' or 'reroute', not {overflow!r}")
+    out["capacity"] = C
     return out
 
 

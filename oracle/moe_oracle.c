@@ -282,6 +282,68 @@ void orc_capacity_keep(int64_t T, int64_t N, int64_t K, const int32_t *sel, int6
     free(load);
 }
 
+/* The values the experts are ranked on for selection: the device's fp32
+ * selection scores when given (sel_row), else the fp64 score plus the
+ * selection-only bias (if any). */
+static void orc_selection_row(int64_t N, const double *s, const float *bsel, const float *sel_row, double *v) {
+    for (int64_t e = 0; e < N; ++e)
+        v[e] = sel_row ? (double)sel_row[e] : s[e] + (bsel ? (double)bsel[e] : 0.0);
+}
+
+/* Reroute: the other overflow policy of the chapter's design notes -- an
+ * assignment that does not fit goes to the next candidate instead of being
+ * dropped.  Rows are served in order, as for the drop.  Row t first offers each
+ * of its K selected experts its slot (accepted while the expert holds fewer
+ * than C); each refused slot, in slot order, then goes to the best-ranked
+ * expert (larger selection value first, ties to the lower index) that is not
+ * already one of row t's experts and still holds fewer than C.  If no such
+ * expert is left the slot is dropped (assign -1).  The slot keeps its gate
+ * weight: the router's weights are not recomputed, as for the drop.
+ *   v [T, N]: the selection values (orc_selection_row); sel [T, K];
+ *   assign [T, K] out: the expert that serves each slot, or -1. */
+void orc_capacity_reroute(int64_t T, int64_t N, int64_t K, const double *v, const int32_t *sel, int64_t C,
+                          int32_t *assign) {
+    int64_t *load = (int64_t *)calloc((size_t)N, sizeof(int64_t));
+    uint8_t *held = (uint8_t *)malloc((size_t)N);
+    for (int64_t t = 0; t < T; ++t) {
+        const double *vt = v + t * N;
+        memset(held, 0, (size_t)N);
+        for (int64_t j = 0; j < K; ++j) held[sel[t * K + j]] = 1;
+        for (int64_t j = 0; j < K; ++j) {
+            const int32_t e = sel[t * K + j];
+            if (load[e] < C) {
+                load[e] += 1;
+                assign[t * K + j] = e;
+            } else {
+                assign[t * K + j] = -1;   /* refused: rerouted below */
+            }
+        }
+        for (int64_t j = 0; j < K; ++j) {
+            if (assign[t * K + j] >= 0) continue;
+            int64_t best = -1;
+            for (int64_t e = 0; e < N; ++e) {
+                if (held[e] || load[e] >= C) continue;
+                if (best < 0 || vt[e] > vt[best]) best = e;   /* ascending e: ties keep the lower index */
+            }
+            if (best >= 0) {
+                load[best] += 1;
+                held[best] = 1;
+                assign[t * K + j] = (int32_t)best;
+            }
+        }
+    }
+    free(load);
+    free(held);
+}
+
+/* The selection values of rows t0..t1-1 (fp64 scores plus bias, or the given
+ * fp32 selection scores), for orc_capacity_reroute. */
+void orc_selection_values(const orc_layer *L, int64_t t0, int64_t t1, const double *scores, const float *sel_scores,
+                          double *v) {
+    for (int64_t t = t0; t < t1; ++t)
+        orc_selection_row(L->N, scores + t * L->N, L->bsel, sel_scores ? sel_scores + t * L->N : NULL, v + t * L->N);
+}
+
 /* ------------------------------------------------------------------------
  * Shared expert.  "MoE(Mixture of Experts)", design notes (merits and
  * examples): the fine-grained MoE of DeepSeek-V3 adds to the many small routed
@@ -313,6 +375,8 @@ void orc_add_shared(int64_t D, const double *s, double *y) {
  *   S1/S2 (optional): the shared expert, added after the routed sum.
  *   keep [T, K] (optional): capacity decisions (orc_capacity_keep); a slot
  *       with keep 0 is not evaluated and adds nothing.
+ *   assign [T, K] (optional): the expert serving each slot after a reroute
+ *       (orc_capacity_reroute), -1 for none; the slot's gate weight is kept.
  *   scores_out [T, N]: fp64 router scores.
  *   sel_scores [T, N] (optional): if given, the expert selection is made on
  *       these scores instead of the fp64 s + bsel (used to apply the oracle's
@@ -323,8 +387,8 @@ void orc_add_shared(int64_t D, const double *s, double *y) {
  * separate threads.
  * ---------------------------------------------------------------------- */
 void orc_moe_layer_rows(const orc_layer *L, int64_t t0, int64_t t1,
-                        const float *sel_scores, const uint8_t *keep, double *scores_out,
-                        int32_t *sel_out, double *w_out, double *y_out) {
+                        const float *sel_scores, const uint8_t *keep, const int32_t *assign,
+                        double *scores_out, int32_t *sel_out, double *w_out, double *y_out) {
     int64_t D = L->D, H = L->H, N = L->N, K = L->K;
     double *x_row = (double *)malloc(sizeof(double) * (size_t)D);
     double *hid = (double *)malloc(sizeof(double) * (size_t)H);
@@ -337,19 +401,16 @@ void orc_moe_layer_rows(const orc_layer *L, int64_t t0, int64_t t1,
         double *w = w_out + t * K;
         orc_load_row(D, L->x, L->dtype, t, x_row);
         orc_router_scores(D, N, x_row, L->Wg, L->dtype, L->bg, s);
-        if (sel_scores) {
-            for (int64_t e = 0; e < N; ++e) tmp[e] = (double)sel_scores[t * N + e];
-        } else {
-            for (int64_t e = 0; e < N; ++e) tmp[e] = s[e] + (L->bsel ? (double)L->bsel[e] : 0.0);
-        }
+        orc_selection_row(N, s, L->bsel, sel_scores ? sel_scores + t * N : NULL, tmp);
         orc_select_topk(N, K, tmp, sel);
         orc_gate_weights(N, K, s, sel, w);
         for (int64_t j = 0; j < K; ++j) {
-            if (keep && !keep[t * K + j]) {
+            const int32_t e = assign ? assign[t * K + j] : sel[j];
+            if ((keep && !keep[t * K + j]) || e < 0) {
                 for (int64_t c = 0; c < D; ++c) E[j * D + c] = 0.0;   /* dropped: no contribution */
                 continue;
             }
-            orc_expert(L, sel[j], x_row, hid, E + j * D);
+            orc_expert(L, e, x_row, hid, E + j * D);
         }
         orc_combine(K, D, w, E, y_out + t * D);
         if (L->S1) {
@@ -544,7 +605,7 @@ void orc_moe_layer_backward(const orc_layer *L, int64_t T, const float *sel_scor
     int32_t *sel = (int32_t *)malloc(sizeof(int32_t) * (size_t)(T * K));
     double *w = (double *)malloc(sizeof(double) * (size_t)(T * K));
     double *y = (double *)malloc(sizeof(double) * (size_t)(T * D));
-    orc_moe_layer_rows(L, 0, T, sel_scores, NULL, scores, sel, w, y);
+    orc_moe_layer_rows(L, 0, T, sel_scores, NULL, NULL, scores, sel, w, y);
     /* batch quantities of the auxiliary losses: f_e and the importance */
     double *f = (double *)calloc((size_t)N, sizeof(double));
     double *imp = (double *)calloc((size_t)N, sizeof(double));

@@ -69,7 +69,7 @@ MUTANTS = [
     ("shared_expert_replaces_routed", "for (int64_t c = 0; c < D; ++c) y[c] = y[c] + s[c];",
      "for (int64_t c = 0; c < D; ++c) y[c] = s[c];",
      [pins.test_one_expert_with_shared_expert_is_two_dense_ffns]),
-    ("selection_bias_ignored", "tmp[e] = s[e] + (L->bsel ? (double)L->bsel[e] : 0.0);", "tmp[e] = s[e];",
+    ("selection_bias_ignored", "s[e] + (bsel ? (double)bsel[e] : 0.0);", "s[e];",
      [pins.test_selection_bias_changes_the_kept_set_not_the_weights]),
     ("selection_bias_in_weights", "        orc_gate_weights(N, K, s, sel, w);\n        for (int64_t j = 0; j < K; ++j) {",
      "        orc_gate_weights(N, K, tmp, sel, w);\n        for (int64_t j = 0; j < K; ++j) {",
@@ -77,10 +77,23 @@ MUTANTS = [
     ("capacity_floor", "return (int64_t)ceil(cf * (double)T * (double)K / (double)N);",
      "return (int64_t)floor(cf * (double)T * (double)K / (double)N);",
      [pins.test_capacity_closed_forms]),
-    ("capacity_off_by_one", "if (load[e] < C) {", "if (load[e] <= C) {",
+    ("capacity_off_by_one", "if (load[e] < C) {\n                load[e] += 1;\n                keep",
+     "if (load[e] <= C) {\n                load[e] += 1;\n                keep",
      [pins.test_capacity_keeps_the_first_C_of_each_expert_in_row_order]),
-    ("dropped_slot_still_added", "            if (keep && !keep[t * K + j]) {", "            if (0) {",
+    ("dropped_slot_still_added", "if ((keep && !keep[t * K + j]) || e < 0) {", "if (0) {",
      [pins.test_capacity_layer_is_the_masked_dense_gate]),
+    ("reroute_to_worst", "if (best < 0 || vt[e] > vt[best]) best = e;", "if (best < 0 || vt[e] < vt[best]) best = e;",
+     [pins.test_reroute_worked_examples, pins.test_reroute_equals_deferred_acceptance]),
+    ("reroute_takes_held_expert", "if (held[e] || load[e] >= C) continue;", "if (load[e] >= C) continue;",
+     [pins.test_reroute_worked_examples, pins.test_reroute_equals_deferred_acceptance]),
+    ("reroute_ignores_capacity", "if (held[e] || load[e] >= C) continue;", "if (held[e]) continue;",
+     [pins.test_reroute_worked_examples, pins.test_reroute_equals_deferred_acceptance]),
+    ("reroute_ties_to_higher_index", "if (best < 0 || vt[e] > vt[best]) best = e;",
+     "if (best < 0 || vt[e] >= vt[best]) best = e;",
+     [pins.test_reroute_worked_examples, pins.test_reroute_equals_deferred_acceptance]),
+    ("reroute_evaluates_selected_expert", "const int32_t e = assign ? assign[t * K + j] : sel[j];",
+     "const int32_t e = assign ? (assign[t * K + j] < 0 ? -1 : sel[j]) : sel[j];",
+     [pins.test_reroute_layer_against_single_expert_layers]),
     ("gelu_grad_missing_density", "+ v * exp(-0.5 * v * v) / sqrt(2.0 * 3.14159265358979323846);", ";",
      [pins.test_activation_derivatives_closed_forms, pins.test_backward_one_expert_top1_is_dense_ffn_autograd]),
     ("swiglu_grad_gate_up_swapped", "double dg = dh[n] * pre[H + n] * orc_silu_grad(pre[n]);",

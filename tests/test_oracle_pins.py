@@ -386,6 +386,120 @@ def test_large_capacity_is_the_plain_layer():
     np.testing.assert_array_equal(a["y"], b["y"])
 
 
+# --------------------------------------------------------------------------- reroute
+def test_reroute_worked_examples():
+    """Hand-worked cases of the next-candidate reroute (rows served in order, a refused slot
+    goes to the best-ranked expert the row does not hold yet that still has room)."""
+    # three rows prefer expert 0, then 1, then 2; one place each: 0, then 1, then 2
+    v = np.array([[3.0, 2.0, 1.0]] * 4)
+    sel = np.zeros((4, 1), np.int32)
+    assert oracle.capacity_reroute(v, sel, 1)[:, 0].tolist() == [0, 1, 2, -1]
+    assert oracle.capacity_reroute(v, sel, 2)[:, 0].tolist() == [0, 0, 1, 1]
+    # two slots per row: row 1 loses both first choices; its first refused slot takes the
+    # better of the two free experts (2), the second slot the next one (3)
+    v = np.array([[4.0, 3.0, 2.0, 1.0]] * 2)
+    sel = np.array([[0, 1], [0, 1]], np.int32)
+    assert oracle.capacity_reroute(v, sel, 1).tolist() == [[0, 1], [2, 3]]
+    # equal values: the lower index first, as in the selection
+    v = np.ones((2, 4))
+    assert oracle.capacity_reroute(v, sel, 1).tolist() == [[0, 1], [2, 3]]
+    # an earlier row's reroute takes the place a later row selected first
+    v = np.array([[3.0, 2.0, 1.0], [3.0, 2.0, 1.0], [1.0, 3.0, 2.0]])
+    sel = np.array([[0], [0], [1]], np.int32)
+    assert oracle.capacity_reroute(v, sel, 1)[:, 0].tolist() == [0, 1, 2]
+    assert oracle.capacity_keep(sel, 3, 1)[:, 0].tolist() == [1, 0, 1]        # the drop, for contrast
+    # a row never takes an expert twice: row 1 keeps expert 1 in slot 1, so its refused slot 0
+    # cannot go to expert 1 although it has room; expert 2 is full, so slot 0 is dropped
+    v = np.array([[3.0, 2.0, 1.0], [3.0, 2.0, 1.0]])
+    sel = np.array([[0, 1], [0, 1]], np.int32)
+    assert oracle.capacity_reroute(v, sel, np.int64(2)).tolist() == [[0, 1], [0, 1]]
+    sel1 = np.array([[0, 2], [0, 1]], np.int32)
+    assert oracle.capacity_reroute(v, sel1, 1).tolist() == [[0, 2], [-1, 1]]
+
+
+def _deferred_acceptance(v, K, C):
+    """Expert sets from deferred acceptance: every row proposes down its own ranking
+    (larger value first, ties to the lower index) until it holds K experts or has asked
+    them all; each expert keeps the C lowest-numbered rows proposing to it.  With one
+    priority order shared by all experts this reaches the serial-dictatorship outcome,
+    i.e. rows served in order each taking the K best experts still free."""
+    T, N = v.shape
+    pref = [sorted(range(N), key=lambda e: (-v[t, e], e)) for t in range(T)]
+    nxt = [0] * T
+    held = [set() for _ in range(T)]
+    accepted = [set() for _ in range(N)]
+    changed = True
+    while changed:
+        changed = False
+        for t in range(T):
+            while len(held[t]) < K and nxt[t] < N:
+                e = pref[t][nxt[t]]
+                nxt[t] += 1
+                accepted[e].add(t)
+                held[t].add(e)
+                changed = True
+                if len(accepted[e]) > C:
+                    worst = max(accepted[e])
+                    accepted[e].discard(worst)
+                    held[worst].discard(e)
+    return held
+
+
+def test_reroute_equals_deferred_acceptance():
+    """Against another algorithm: each row's set of serving experts equals the outcome of
+    deferred acceptance with the row order as the experts' common priority; slots whose
+    selected expert had room keep it, and refused slots take the new experts in rank order."""
+    rng = np.random.default_rng(89)
+    cases = 0
+    for _ in range(200):
+        T, N = int(rng.integers(1, 14)), int(rng.integers(2, 7))
+        K, C = int(rng.integers(1, min(3, N) + 1)), int(rng.integers(1, 4))
+        v = rng.integers(0, 4, size=(T, N)).astype(np.float64)       # many ties
+        sel = oracle.select_topk(v, K)
+        assign = oracle.capacity_reroute(v, sel, C)
+        sets = _deferred_acceptance(v, K, C)
+        for t in range(T):
+            got = [e for e in assign[t].tolist() if e >= 0]
+            assert len(set(got)) == len(got)
+            assert set(got) == sets[t], (t, v, sel, assign)
+            kept = [int(e) for e, a in zip(sel[t], assign[t]) if a == e]
+            new = [int(a) for e, a in zip(sel[t], assign[t]) if a != e and a >= 0]
+            order = sorted(range(N), key=lambda e: (-v[t, e], e))
+            assert new == [e for e in order if e in set(new)]           # rank order across slots
+            assert -1 not in assign[t] or len(got) == len(kept) + len(new)
+        loads = np.bincount(assign[assign >= 0], minlength=N)
+        assert (loads <= C).all()
+        cases += int((assign != sel).any())
+    assert cases > 50
+
+
+def test_reroute_layer_against_single_expert_layers():
+    """Two rows that both select expert 0 of two, one place each: the second row is served
+    by expert 1 with its gate weight (1 at K = 1), i.e. exactly the one-expert layer of
+    expert 1; the first row is the one-expert layer of expert 0.  With room for all the
+    reroute layer is the plain layer."""
+    rng = np.random.default_rng(97)
+    T, D, H, N = 2, 6, 8, 2
+    x, Wg, W1, W2, b1, b2 = _rand_layer(rng, T, D, H, N, oracle.ACT_GELU, True)
+    bg = np.array([50.0, 0.0], np.float32)                       # both rows select expert 0
+    out = oracle.moe_layer_capacity(x, Wg, W1, W2, K=1, act=oracle.ACT_GELU, dtype_tag=oracle.F32, cf=0.5,
+                                    overflow="reroute", bg=bg, b1=b1, b2=b2, threads=1)
+    assert out["capacity"] == 1 and out["assign"][:, 0].tolist() == [0, 1]
+    for t, e in ((0, 0), (1, 1)):
+        one = oracle.moe_layer(x[t:t + 1], Wg[:, e:e + 1], W1[e:e + 1], W2[e:e + 1], K=1, act=oracle.ACT_GELU,
+                               dtype_tag=oracle.F32, b1=b1[e:e + 1], b2=b2[e:e + 1], threads=1)
+        np.testing.assert_allclose(out["y"][t], one["y"][0], rtol=1e-14, atol=1e-15)
+    drop = oracle.moe_layer_capacity(x, Wg, W1, W2, K=1, act=oracle.ACT_GELU, dtype_tag=oracle.F32, cf=0.5,
+                                     bg=bg, b1=b1, b2=b2, threads=1)
+    assert (drop["y"][1] == 0).all()
+    plain = oracle.moe_layer(x, Wg, W1, W2, K=1, act=oracle.ACT_GELU, dtype_tag=oracle.F32, bg=bg, b1=b1, b2=b2,
+                             threads=1)
+    big = oracle.moe_layer_capacity(x, Wg, W1, W2, K=1, act=oracle.ACT_GELU, dtype_tag=oracle.F32, cf=4.0,
+                                    overflow="reroute", bg=bg, b1=b1, b2=b2, threads=1)
+    np.testing.assert_array_equal(big["y"], plain["y"])
+    np.testing.assert_array_equal(big["assign"], plain["sel"])
+
+
 # --------------------------------------------------------------------------- backward
 def _objective(x, Wg, W1, W2, bg, b1, b2, bsel, dy, K, act, a_s, a_i):
     """sum(y * dy) + a_s * switch + a_i * cv2_importance, from the pinned forward and statistics."""
