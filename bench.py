@@ -114,6 +114,10 @@ def parse(argv=None):
     ap.add_argument("--experts", type=int, default=0,
                     help="reduced case for profiling: override the number of experts (tokens per expert kept "
                          "when --tokens is scaled with it)")
+    ap.add_argument("--capacity-factor", type=float, default=None,
+                    help="per-expert capacity ceil(cf T K / N) (default: the workload's own)")
+    ap.add_argument("--overflow", default=None, choices=["drop", "reroute"],
+                    help="what a full expert does with a further assignment (with a capacity)")
     return ap.parse_args(argv)
 
 
@@ -125,6 +129,10 @@ def workload_from_args(args):
         kw["T"] = args.tokens
     if args.experts:
         kw["N"] = args.experts
+    if getattr(args, "capacity_factor", None) is not None:
+        kw["capacity_factor"] = args.capacity_factor
+    if getattr(args, "overflow", None) is not None:
+        kw["overflow"] = 1 if args.overflow == "reroute" else 0
     if kw:
         wl = wl.with_(name=f"{wl.name}[" + ",".join(f"{k}={v}" for k, v in kw.items()) + "]", **kw)
     return wl
@@ -189,9 +197,15 @@ def work_model(wl, T, counts=None):
 
 
 def config_dict(wl, T, world):
-    return {"workload": wl.name, "T": T, "D": wl.D, "H": wl.H, "N": wl.N, "K": wl.K,
-            "act": "swiglu" if wl.act == ACT_SWIGLU else "gelu", "global_batch": T * world,
-            "parallelism": f"dp{world}", "l2": "flushed (512 MiB write) before every step"}
+    d = {"workload": wl.name, "T": T, "D": wl.D, "H": wl.H, "N": wl.N, "K": wl.K,
+         "act": "swiglu" if wl.act == ACT_SWIGLU else "gelu", "global_batch": T * world,
+         "parallelism": f"dp{world}", "l2": "flushed (512 MiB write) before every step"}
+    if wl.n_shared:
+        d["n_shared"] = wl.n_shared
+    if wl.capacity_factor > 0:
+        d["capacity_factor"] = wl.capacity_factor
+        d["overflow"] = "reroute" if wl.overflow else "drop"
+    return d
 
 
 def gemm_peak(pk, step_ms):
@@ -559,7 +573,8 @@ def main():
 
     T = wl.T
     inp = make_inputs(wl, dev, seed=rank_seed(wl, rank))
-    cfg = moe.make_config(wl.D, wl.H, wl.N, wl.K, wl.act, moe.dtype_code(wl.dtype), wl.has_bias, wl.n_shared)
+    cfg = moe.make_config(wl.D, wl.H, wl.N, wl.K, wl.act, moe.dtype_code(wl.dtype), wl.has_bias, wl.n_shared,
+                          wl.capacity_factor, wl.overflow)
     W = moe.make_weights(inp["W_g"], inp["W1"], inp["W2"], inp["b_g"], inp["b1"], inp["b2"], inp["b_sel"],
                          inp["S1"], inp["sb1"], inp["S2"], inp["sb2"])
     ws = moe.alloc_workspace(cfg, T)

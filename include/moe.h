@@ -95,13 +95,26 @@ typedef struct {
                          (computed in double) per call; 0: no limit.
                          "MoE(Mixture of Experts)", design notes (capacity
                          factor: overflow is dropped or sent to the next
-                         candidate).  Here overflow is dropped: rows are served
-                         in token order, an assignment is accepted while its
-                         expert holds fewer than C, and a dropped assignment
-                         adds nothing to y (the kept gate weights are not
-                         renormalised).  The statistics (moe_aux) describe the
-                         router's choice before the limit. */
+                         candidate).  Rows are served in token order and an
+                         assignment is accepted while its expert holds fewer
+                         than C; what happens to the others is set by
+                         overflow.  A dropped assignment adds nothing to y (the
+                         kept gate weights are not renormalised).  The
+                         statistics (moe_aux) describe the router's choice
+                         before the limit. */
+    int32_t overflow;  /* with a capacity: MOE_OVERFLOW_DROP, or
+                         MOE_OVERFLOW_REROUTE -- each refused assignment of row
+                         t, in slot order, goes to the best-ranked expert (by
+                         the selection value, ties to the lower index) that row
+                         t does not hold yet and that still holds fewer than C,
+                         keeping its gate weight; dropped only when no such
+                         expert is left.  The reroute is sequential in t (one
+                         CTA walks the tokens) and disables the one-kernel
+                         decode path.  Ignored without a capacity. */
 } moe_config;
+
+/* moe_config.overflow */
+enum { MOE_OVERFLOW_DROP = 0, MOE_OVERFLOW_REROUTE = 1 };
 
 /* Layer parameters, all device memory.
  *  W_g [D, N] dtype      router matrix, scores = x W_g (Shazeer gate x W_g)

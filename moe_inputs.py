@@ -52,6 +52,7 @@ class Workload:
     n_shared: int = 0     # 1: a shared expert every token passes through
     sel_s: float = 0.0    # selection-only bias strength; 0 = none
     capacity_factor: float = 0.0   # per-expert capacity ceil(cf T K / N); 0 = no limit
+    overflow: int = 0     # with a capacity: 0 drop, 1 reroute to the next candidate
 
     @property
     def seed(self) -> int:

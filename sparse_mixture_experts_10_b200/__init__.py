@@ -22,6 +22,7 @@ LIB_PATH = os.path.join(_PKG, "libmoe.so")
 
 MOE_F32, MOE_BF16 = 0, 1
 MOE_ACT_GELU, MOE_ACT_SWIGLU = 0, 1
+MOE_OVERFLOW_DROP, MOE_OVERFLOW_REROUTE = 0, 1
 MOE_N_STAGES = 7
 STAGE_NAMES = ("route", "scan", "permute", "up", "down", "combine", "stats")
 
@@ -46,7 +47,8 @@ EXPORTED = ("moe_workspace_size", "moe_route", "moe_forward", "moe_forward_timed
 class moe_config(ctypes.Structure):
     _fields_ = [("DModel", ctypes.c_int32), ("DHidden", ctypes.c_int32), ("NExperts", ctypes.c_int32),
                 ("TopK", ctypes.c_int32), ("act", ctypes.c_int32), ("dtype", ctypes.c_int32),
-                ("has_bias", ctypes.c_int32), ("n_shared", ctypes.c_int32), ("capacity_factor", ctypes.c_float)]
+                ("has_bias", ctypes.c_int32), ("n_shared", ctypes.c_int32), ("capacity_factor", ctypes.c_float),
+                ("overflow", ctypes.c_int32)]
 
 
 class moe_weights(ctypes.Structure):
@@ -172,9 +174,9 @@ def dtype_code(dt: torch.dtype) -> int:
 
 
 def make_config(DModel, DHidden, NExperts, TopK, act=MOE_ACT_GELU, dtype=MOE_BF16, has_bias=False,
-                n_shared=0, capacity_factor=0.0) -> moe_config:
+                n_shared=0, capacity_factor=0.0, overflow=MOE_OVERFLOW_DROP) -> moe_config:
     return moe_config(DModel, DHidden, NExperts, TopK, act, dtype, int(bool(has_bias)), int(n_shared),
-                      float(capacity_factor))
+                      float(capacity_factor), int(overflow))
 
 
 def make_weights(W_g, W1, W2, b_g=None, b1=None, b2=None, b_sel=None, S1=None, sb1=None, S2=None,

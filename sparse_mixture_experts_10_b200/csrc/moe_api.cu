@@ -34,6 +34,7 @@ std::atomic<int64_t> g_launches{0};
 constexpr uint64_t kTimeoutNs = 1000000000ull;  // bounded waits give up after 1 s
 constexpr int kMaxDevices = 64;
 constexpr size_t kSmallRouterSmemMax = 200 * 1024;
+constexpr int64_t kRerouteSmem = 160 * 1024;   // reroute_kernel: loads + two staged batches
 constexpr int64_t kRowdotMaxT = 2048;  // below this the chunked router has too few blocks
 constexpr int64_t kDecodeMaxT = 64;    // up to this many tokens the expert GEMMs stream weights (decode path)
 constexpr int kDecodeMaxGrid = 256;    // decode GEMMs: most persistent CTAs (stream-K buffers are sized for it)
@@ -69,7 +70,9 @@ struct Plan {
     int route_splits;  // few-token router: W_g slabs per token
     int dec_cap;       // decode GEMMs: CTAs the stream-K partials and tickets are sized for
     int n_shared;      // 1: a shared expert (dense FFN over every token) is added after the routed sum
-    int capacity;      // assignments each expert accepts (rows served in order; the rest are dropped)
+    int capacity;      // assignments each expert accepts (rows served in order)
+    bool reroute;      // refused assignments go to the next candidate (reroute_kernel) instead of being dropped
+    int rr_batch;      // reroute_kernel: tokens staged per buffer
     bool fused_decode; // few tokens, N <= 32, no shared expert: the whole layer in one cooperative kernel
     bool given_routing;
     int slab_rows, n_slabs;   // fused decode: W_g rows per routing slab, slabs
@@ -77,11 +80,10 @@ struct Plan {
     // [1] statistics ticket, [2] number of live experts, [64, 128) per-token
     // tickets of the few-token router; from byte 512 the stream-K tile tickets
     // of the decode up- and down-projections and of the shared expert's two
-    // decode GEMMs (dec_cap each); then the fused decode kernel's combine
-    // tickets (one per 128 output features); then the routers' per-expert
-    // probability and gate-weight sums (u64, N each).  Words 4, 8 and 9 count
+    // decode GEMMs (dec_cap each); then the routers' per-expert probability
+    // and gate-weight sums (u64, N each).  Words 4, 8 and 9 count
     // the fused decode kernel's grid barrier arrivals, word 7 the cooperative
-    // SIMT router's.
+    // SIMT router's, word 10 is the scan's ticket after a reroute.
     size_t counters_bytes;
     size_t stat_sums;  // offset inside the counters region of the routers' fixed-point sums [2][N] (u64)
     size_t counters, logits, idx, w, counts, offsets, row_offsets, live, chunk_counts, chunk_base,
@@ -102,6 +104,7 @@ int make_plan(const moe_config *c, int64_t T, Plan *p, bool given_routing = fals
     if (c->has_bias && c->act != MOE_ACT_GELU) return MOE_ERR_UNSUPPORTED;
     if (c->n_shared != 0 && c->n_shared != 1) return MOE_ERR_INVALID_ARG;
     if (!(c->capacity_factor >= 0.0f) || c->capacity_factor > 1.0e6f) return MOE_ERR_INVALID_ARG;   // NaN too
+    if (c->overflow != MOE_OVERFLOW_DROP && c->overflow != MOE_OVERFLOW_REROUTE) return MOE_ERR_INVALID_ARG;
     const int es = c->dtype == MOE_F32 ? 4 : 2;
     const int vec = 16 / es;
     if (D % vec || H % vec) return MOE_ERR_INVALID_ARG;
@@ -120,6 +123,8 @@ int make_plan(const moe_config *c, int64_t T, Plan *p, bool given_routing = fals
     } else {
         p->capacity = INT32_MAX;
     }
+    p->reroute = c->capacity_factor > 0.0f && c->overflow == MOE_OVERFLOW_REROUTE;
+    p->rr_batch = (int)std::max<int64_t>(1, std::min<int64_t>(1024, (kRerouteSmem - N * 4 - 16) / (2 * (K + N) * 4)));
     p->np = N <= 8 ? 8 : N <= 16 ? 16 : 32;
     const bool fits = N <= 32 && (size_t)p->np * D * es + 256 <= kSmallRouterSmemMax;
     p->rowdot_router = N <= 32 && (T < kRowdotMaxT || !fits);
@@ -183,7 +188,7 @@ int make_plan(const moe_config *c, int64_t T, Plan *p, bool given_routing = fals
     p->shared_tbl = take(16);
     // fused decode: routing slabs of W_g rows (a multiple of 8 rows each, at most
     // 32 slabs) and each token's full softmax
-    p->fused_decode = p->decode && N <= dfu::kMaxN && !p->n_shared && T <= dfu::kMaxT && !given_routing;
+    p->fused_decode = p->decode && N <= dfu::kMaxN && !p->n_shared && T <= dfu::kMaxT && !given_routing && !p->reroute;
     p->slab_rows = (int)(cdiv(cdiv(D, dfu::kMaxSlabs), 8) * 8);
     p->n_slabs = (int)cdiv(D, p->slab_rows);
     p->fd_slab = take(p->fused_decode ? (size_t)p->n_slabs * T * 32 * 4 : 0);
@@ -223,6 +228,7 @@ int device_info(DeviceInfo **out) {
         if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return MOE_ERR_CUDA;
     }
     if (!d.attrs) {
+        MOE_TRY(allow_smem(reroute_kernel));
         MOE_TRY(allow_smem(tc::grouped_gemm_tc_kernel<256, tc::EPI_GELU>));
         MOE_TRY(allow_smem(tc::grouped_gemm_tc_kernel<256, tc::EPI_SWIGLU>));
         MOE_TRY(allow_smem(tc::grouped_gemm_tc_kernel<256, tc::EPI_SCATTER>));
@@ -460,7 +466,7 @@ int stage_route_tc(const Plan &P, const Bufs &b, const void *x, const moe_weight
     p.live = b.at<int>(P.live);
     p.n_live = b.at<int>(P.counters) + 2;
     p.counts_out = counts_out;
-    p.capacity = P.capacity;
+    p.capacity = P.reroute ? INT32_MAX : P.capacity;   // a reroute's tables come from the scan after it
     if (aux) {
         p.aux_counts = aux->counts;
         p.aux_importance = aux->importance;
@@ -675,11 +681,29 @@ int stage_route(const Plan &P, const Bufs &b, const void *x, const moe_weights *
     return check_launch();
 }
 
-int stage_scan(const Plan &P, const Bufs &b, int *counts_out, cudaStream_t s) {
+// The reroute ("MoE(Mixture of Experts)", design notes on the capacity
+// factor): the statistics first when no router kernel took them (they describe
+// the router's choice), then the sequential reroute over idx, then the chunk
+// histograms and the capacity scan of the rerouted assignments.
+int stage_scan(const Plan &P, const Bufs &b, int *counts_out, cudaStream_t s, int counter_word = 0);
+int stage_reroute(const Plan &P, const Bufs &b, const moe_weights *w, cudaStream_t s) {
+    const int N = P.N, K = P.K, B = P.rr_batch;
+    const size_t smem = (size_t)((N + 3) & ~3) * 4 + (size_t)2 * B * K * 4 + (size_t)2 * B * N * 4;
+    if (smem > (size_t)kRerouteSmem) return MOE_ERR_UNSUPPORTED;
+    reroute_kernel<<<1, kRerouteThreads, smem, s>>>(b.at<float>(P.logits), w->b_sel, b.at<int>(P.idx), (int)P.T, N, K,
+                                                    P.capacity, B);
+    MOE_TRY(check_launch());
+    hist_kernel<<<P.n_chunks, 256, (size_t)N * 4, s>>>(b.at<int>(P.idx), P.T * K, P.chunk_tokens * K, N, 1,
+                                                      b.at<int>(P.chunk_counts));
+    MOE_TRY(check_launch());
+    return stage_scan(P, b, nullptr, s, 10);   // word 0 may hold the router's spent ticket
+}
+
+int stage_scan(const Plan &P, const Bufs &b, int *counts_out, cudaStream_t s, int counter_word) {
     scan_kernel<<<(unsigned)cdiv(P.N, 32), 1024, 0, s>>>(
         b.at<int>(P.chunk_counts), P.n_chunks, P.N, P.T * P.K, P.capacity, b.at<int>(P.chunk_base), b.at<int>(P.counts),
-        b.at<int>(P.offsets), b.at<int>(P.row_offsets), b.at<int>(P.perm_slot), counts_out, b.at<unsigned>(P.counters),
-        b.at<int>(P.live), b.at<int>(P.counters) + 2);
+        b.at<int>(P.offsets), b.at<int>(P.row_offsets), b.at<int>(P.perm_slot), counts_out,
+        b.at<unsigned>(P.counters) + counter_word, b.at<int>(P.live), b.at<int>(P.counters) + 2);
     return check_launch();
 }
 
@@ -822,13 +846,14 @@ int stage_up(const Plan &P, const Bufs &b, const moe_weights *w, const DeviceInf
         p.tail_mode = 1;
         if (swiglu) MOE_TRY(launch_tc2<tc::EPI_SWIGLU>(ma, mb, mo, p, units, dev.pair_clusters, s));
         else MOE_TRY(launch_tc2<tc::EPI_GELU>(ma, mb, mo, p, units, dev.pair_clusters, s));
+        // the tail tiles are 128 x 256 (SwiGLU: 128 gate + 128 up rows of W1,
+        // the pair kernel's B box; GELU: one 256-row box)
         tc::Params pt = p;
         pt.tail_mode = 2;
-        pt.n_tiles = (int)cdiv(H, swiglu ? 64 : 128);
         CUtensorMap mbt = mb;
-        if (swiglu) MOE_TRY(make_map(&mbt, w->W1, (int64_t)N * 2 * H, D, 64));
-        if (swiglu) return launch_tc<128, tc::EPI_SWIGLU>(ma, mbt, mo, pt, (int64_t)N * pt.n_tiles, dev.sms, s);
-        return launch_tc<128, tc::EPI_GELU>(ma, mbt, mo, pt, (int64_t)N * pt.n_tiles, dev.sms, s);
+        if (!swiglu) MOE_TRY(make_map(&mbt, w->W1, (int64_t)N * H, D, 256));
+        if (swiglu) return launch_tc<256, tc::EPI_SWIGLU>(ma, mbt, mo, pt, (int64_t)N * pt.n_tiles, dev.sms, s);
+        return launch_tc<256, tc::EPI_GELU>(ma, mbt, mo, pt, (int64_t)N * pt.n_tiles, dev.sms, s);
     }
     simt::Params p{};
     p.A = b.at<float>(P.x_perm);
@@ -894,8 +919,9 @@ int stage_down(const Plan &P, const Bufs &b, const moe_weights *w, void *y, int 
                                             dev.pair_clusters, s));
         tc::Params pt = p;
         pt.tail_mode = 2;
-        pt.n_tiles = (int)cdiv(D, 128);
-        return launch_tc<128, tc::EPI_SCATTER>(ma, mb, mo, pt, (int64_t)N * pt.n_tiles, dev.sms, s);
+        CUtensorMap mbt;
+        MOE_TRY(make_map(&mbt, w->W2, (int64_t)N * D, H, 256));
+        return launch_tc<256, tc::EPI_SCATTER>(ma, mbt, mo, pt, (int64_t)N * pt.n_tiles, dev.sms, s);
     }
     simt::Params p{};
     p.A = b.at<float>(P.h);
@@ -1311,7 +1337,8 @@ int forward_impl(const moe_config *cfg, const void *x, int64_t T, const moe_weig
     } else if (P.tc_router) {
         // the SIMT router takes the dispatch into its own (cooperative) launch when it can
         bool dispatched = false;
-        if (P.simt_router) MOE_TRY(stage_route_simt_dispatch(P, b, x, w, aux, y_zero, *dev, s, &dispatched));
+        if (P.simt_router && !P.reroute)
+            MOE_TRY(stage_route_simt_dispatch(P, b, x, w, aux, y_zero, *dev, s, &dispatched));
         if (dispatched) {
             MOE_TRY(rec(1));
             MOE_TRY(rec(2));
@@ -1319,10 +1346,16 @@ int forward_impl(const moe_config *cfg, const void *x, int64_t T, const moe_weig
         }
         MOE_TRY(stage_route_tc(P, b, x, w, logits, idx, tw, nullptr, aux, y_zero, s));
         MOE_TRY(rec(1));
+        if (P.reroute) MOE_TRY(stage_reroute(P, b, w, s));
     } else {
         MOE_TRY(stage_route(P, b, x, w, logits, idx, tw, *dev, s));
         MOE_TRY(rec(1));
-        MOE_TRY(stage_scan(P, b, nullptr, s));
+        if (P.reroute) {
+            if (aux) MOE_TRY(stage_aux(P, b, logits, idx, tw, aux, s));   // before idx is rerouted
+            MOE_TRY(stage_reroute(P, b, w, s));
+        } else {
+            MOE_TRY(stage_scan(P, b, nullptr, s));
+        }
     }
     MOE_TRY(rec(2));
     MOE_TRY(stage_permute(P, b, x, P.simt_router ? nullptr : y_zero, *dev, s));
@@ -1336,7 +1369,7 @@ experts:
     MOE_TRY(rec(5));
     if (!combine_in_down(P, y_dtype)) MOE_TRY(stage_combine(P, b, y, y_dtype, *dev, s));
     MOE_TRY(rec(6));
-    if (aux && !P.tc_router && !P.given_routing) MOE_TRY(stage_aux(P, b, logits, idx, tw, aux, s));
+    if (aux && !P.tc_router && !P.given_routing && !P.reroute) MOE_TRY(stage_aux(P, b, logits, idx, tw, aux, s));
     MOE_TRY(rec(7));
     return MOE_OK;
 }

@@ -92,6 +92,12 @@ struct Params {
     // segment.  tail_mode 1 (pair kernel): leave each such group's last block
     // out; tail_mode 2 (1-CTA kernel): compute only those blocks, one 128-row
     // tile per group.  0: every row tile.
+    // The tail kernel is launched right behind the pair kernel and runs beside
+    // it: the pair kernel lets its dependent launch only after its own
+    // programmatic wait (so everything before it is complete and visible),
+    // the tail kernel starts without waiting, takes SMs as the pair CTAs
+    // finish, and waits for the pair kernel only before it exits (so the next
+    // kernel, which waits for the tail kernel, sees both).
     int tail_mode;
     uint64_t timeout_ns;
 };
@@ -485,7 +491,8 @@ template <int BN, int EPI>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                            const __grid_constant__ CUtensorMap tmO, const Params p) {
-    pdl_enter();
+    if (p.tail_mode == 2) pdl_launch_dependents();   // reads only what the pair kernel's wait covered
+    else pdl_enter();
     using S = Shape<BN>;
     constexpr int kStages = S::kStages;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -665,6 +672,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         tmem_dealloc(tmem_base, S::kTmemCols);
     }
+    if (p.tail_mode == 2) pdl_wait();   // complete only after the pair kernel beside it
 }
 
 // =====================================================================================
@@ -769,7 +777,8 @@ template <int EPI>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     grouped_gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                             const __grid_constant__ CUtensorMap tmO, const Params p) {
-    pdl_enter();
+    pdl_wait();                 // the dependent (a tail kernel may run beside this one) launches
+    pdl_launch_dependents();    // only once everything before this kernel is complete
     using S = Shape2;
     constexpr int BN = 256;
     constexpr int kStages = S::kStages;

@@ -381,6 +381,143 @@ __global__ void __launch_bounds__(256) hist_kernel(const int *__restrict__ idx, 
 }
 
 // ---------------------------------------------------------------------------
+// Reroute, the capacity's other overflow policy ("MoE(Mixture of Experts)",
+// design notes on the capacity factor: what overflows is dropped or passed to
+// the next candidate).  Rows are served in token order: row t offers each of
+// its K selected experts its slot, accepted while the expert holds fewer than
+// C; each refused slot, in slot order, goes to the best-ranked expert (larger
+// selection value logit + b_sel in fp32, ties to the lower index; NaN ranked as
+// -inf) that row t does not hold yet and that still holds fewer than C.  The
+// new expert is written over idx[t, j]; a slot with no such expert keeps its
+// (full) selected expert, so the capacity scan that follows drops it, and
+// every accepted slot lands within the first C of its expert.
+//
+// The order of service makes this sequential in t.  One CTA: warp 0 walks the
+// tokens with the per-expert loads in shared memory, the other 31 warps stage
+// the next batch of selections and selection values meanwhile (two buffers).
+// Warp 0 takes 32/K tokens at a time: each lane one (token, slot), its place
+// in its expert = the expert's load + the lanes before it with the same expert
+// (match.any); the tokens before the first refused slot are accepted as they
+// are, the refusing token goes through the full per-token step alone.
+// ---------------------------------------------------------------------------
+constexpr int kRerouteThreads = 1024;
+
+__device__ __forceinline__ void reroute_stage(const float *__restrict__ logits, const float *__restrict__ bsel,
+                                              const int *__restrict__ idx, int T, int N, int K, int batch, int bi,
+                                              int *sidx, float *sv, int tid0, int nthr) {
+    const int64_t t0 = (int64_t)bi * batch;
+    const int rows = (int)(T - t0 < (int64_t)batch ? T - t0 : (int64_t)batch);
+    for (int i = tid0; i < rows * K; i += nthr) {
+        int e = idx[t0 * K + i];
+        if ((unsigned)e >= (unsigned)N) {   // not an expert: counted against expert 0, flagged
+            set_status(kStatusBounds);
+            e = 0;
+        }
+        sidx[i] = e;
+    }
+    for (int i = tid0; i < rows * N; i += nthr) {
+        const int e = i % N;
+        float v = logits[t0 * N + i];
+        if (bsel) v += __ldg(bsel + e);
+        sv[i] = v != v ? -INFINITY : v;   // NaN ranked as -inf, as in the selection
+    }
+}
+
+__global__ void __launch_bounds__(kRerouteThreads, 1)
+    reroute_kernel(const float *__restrict__ logits, const float *__restrict__ bsel, int *__restrict__ idx, int T,
+                   int N, int K, int C, int batch) {
+    extern __shared__ __align__(16) unsigned char rr_smem[];
+    int *load = reinterpret_cast<int *>(rr_smem);                        // [N]
+    int *sidx = load + ((N + 3) & ~3);                                   // [2][batch * K]
+    float *sv = reinterpret_cast<float *>(sidx + 2 * batch * K);         // [2][batch * N]
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const unsigned FULL = 0xffffffffu;
+    for (int e = tid; e < N; e += kRerouteThreads) load[e] = 0;
+    const int nb = (int)((T + batch - 1) / batch);
+    reroute_stage(logits, bsel, idx, T, N, K, batch, 0, sidx, sv, tid, kRerouteThreads);
+    __syncthreads();
+    const int G = 32 / K;   // tokens per step of the fast path
+    for (int bi = 0; bi < nb; ++bi) {
+        const int cur = bi & 1;
+        int *bidx = sidx + cur * batch * K;
+        const float *bv = sv + (size_t)cur * batch * N;
+        if (warp != 0) {
+            if (bi + 1 < nb)
+                reroute_stage(logits, bsel, idx, T, N, K, batch, bi + 1, sidx + (cur ^ 1) * batch * K,
+                              sv + (size_t)(cur ^ 1) * batch * N, tid - 32, kRerouteThreads - 32);
+        } else {
+            const int64_t t0 = (int64_t)bi * batch;
+            const int rows = (int)(T - t0 < (int64_t)batch ? T - t0 : (int64_t)batch);
+            int lt = 0;
+            while (lt < rows) {
+                // fast path: G tokens, one (token, slot) per lane
+                const int g = min(G, rows - lt);
+                const bool act = lane < g * K;
+                const int tl = lane / K, j = lane - tl * K;
+                const int e = act ? bidx[(lt + tl) * K + j] : -1 - lane;   // inactive lanes: distinct keys
+                const unsigned peers = __match_any_sync(FULL, e);
+                const int pos = act ? load[e] + __popc(peers & lanemask_lt()) : 0;
+                const unsigned refused = __ballot_sync(FULL, act && pos >= C);
+                const int good = refused ? (__ffs(refused) - 1) / K : g;   // tokens accepted as they are
+                const unsigned accm = __ballot_sync(FULL, act && tl < good);
+                const unsigned pa = peers & accm;
+                if (((accm >> lane) & 1u) && (pa >> lane) == 1u) load[e] += __popc(pa);   // last lane of its expert
+                __syncwarp();
+                lt += good;
+                if (good == g) continue;
+                // the refusing token, alone: accept what fits, reroute the rest in slot order
+                const int64_t t = t0 + lt;
+                const int ej = lane < K ? bidx[lt * K + lane] : -1;
+                const bool room = lane < K && load[ej] < C;
+                if (room) load[ej] += 1;   // a token's K experts are distinct
+                __syncwarp();
+                unsigned todo = __ballot_sync(FULL, lane < K && !room);
+                uint32_t held = 0;         // bit i: expert lane + 32 i is one of the token's
+                for (int jj = 0; jj < K; ++jj) {
+                    const int h = __shfl_sync(FULL, ej, jj);
+                    if ((h & 31) == lane) held |= 1u << (h >> 5);
+                }
+                const float *vrow = bv + (size_t)lt * N;
+                while (todo) {
+                    const int js = __ffs(todo) - 1;
+                    todo &= todo - 1;
+                    float best_v = -INFINITY;
+                    int best_e = -1;
+                    for (int i = 0; lane + 32 * i < N; ++i) {
+                        const int c = lane + 32 * i;
+                        if (((held >> i) & 1u) || load[c] >= C) continue;
+                        const float v = vrow[c];
+                        if (best_e < 0 || v > best_v) {   // ascending c: ties keep the lower index
+                            best_v = v;
+                            best_e = c;
+                        }
+                    }
+#pragma unroll
+                    for (int o = 16; o; o >>= 1) {
+                        const float ov = __shfl_xor_sync(FULL, best_v, o);
+                        const int oe = __shfl_xor_sync(FULL, best_e, o);
+                        if (oe >= 0 && (best_e < 0 || ov > best_v || (ov == best_v && oe < best_e))) {
+                            best_v = ov;
+                            best_e = oe;
+                        }
+                    }
+                    if (best_e >= 0) {
+                        if (lane == 0) {
+                            load[best_e] += 1;
+                            idx[t * K + js] = best_e;
+                        }
+                        if ((best_e & 31) == lane) held |= 1u << (best_e >> 5);
+                    }
+                    __syncwarp();
+                }
+                lt += 1;
+            }
+        }
+        __syncthreads();
+    }
+}
+
+// ---------------------------------------------------------------------------
 // Expert-parallel dispatch: the (token, slot) pairs of a chunk, grouped by the
 // rank that holds their expert (bucket = expert / experts_per_rank) in stable
 // (token, slot) order, packed without padding at

@@ -81,7 +81,8 @@ def oracle_full_layer(inp, wl, K, gpu_logits=None, threads=None):
     kw = dict(K=K, act=wl.act, dtype_tag=t, bg=host(inp["b_g"]), b1=host(inp["b1"]), b2=host(inp["b2"]),
               sel_scores=sel, threads=threads, bsel=host(inp.get("b_sel")), **shared_kwargs(inp))
     if wl.capacity_factor > 0:
-        return oracle.moe_layer_capacity(*args, cf=capacity_factor(wl), **kw)
+        return oracle.moe_layer_capacity(*args, cf=capacity_factor(wl),
+                                         overflow="reroute" if wl.overflow else "drop", **kw)
     return oracle.moe_layer(*args, **kw)
 
 

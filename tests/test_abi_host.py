@@ -35,7 +35,7 @@ def test_every_declared_function_is_exported(lib):
 
 
 def test_struct_sizes_match_header_layout():
-    assert ctypes.sizeof(moe.moe_config) == 9 * 4
+    assert ctypes.sizeof(moe.moe_config) == 10 * 4
     assert ctypes.sizeof(moe.moe_weights) == 11 * 8
     assert ctypes.sizeof(moe.moe_aux) == 4 * 8
     assert ctypes.sizeof(moe.moe_workspace_layout) == 12 * 8 + 8 + 8
@@ -55,6 +55,16 @@ def test_invalid_config_rejected(lib, bad):
     assert moe.moe_workspace_size(c, 16) == 0
     rc = moe.moe_forward(c, 16, 16, moe.make_weights(16, 16, 16), 16, moe.MOE_F32, None, 256, 1 << 30, 0)
     assert rc in (moe.MOE_ERR_INVALID_ARG, moe.MOE_ERR_UNSUPPORTED)
+
+
+def test_overflow_policy_values(lib):
+    """overflow takes the two documented values only; with a capacity either sizes the workspace."""
+    for ov in (moe.MOE_OVERFLOW_DROP, moe.MOE_OVERFLOW_REROUTE):
+        c = moe.make_config(64, 256, 8, 2, moe.MOE_ACT_GELU, moe.MOE_BF16, False, capacity_factor=1.0, overflow=ov)
+        assert moe.moe_workspace_size(c, 4096) > 0
+    for ov in (-1, 2, 7):
+        c = moe.make_config(64, 256, 8, 2, moe.MOE_ACT_GELU, moe.MOE_BF16, False, capacity_factor=1.0, overflow=ov)
+        assert moe.moe_workspace_size(c, 4096) == 0
 
 
 def test_swiglu_with_bias_is_unsupported(lib):

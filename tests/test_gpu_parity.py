@@ -36,7 +36,7 @@ class Layer:
     def __init__(self, wl: Workload, inp):
         self.wl, self.inp = wl, inp
         self.cfg = moe.make_config(wl.D, wl.H, wl.N, wl.K, wl.act, moe.dtype_code(wl.dtype), wl.has_bias,
-                                   wl.n_shared, wl.capacity_factor)
+                                   wl.n_shared, wl.capacity_factor, wl.overflow)
         self.w = moe.make_weights(inp["W_g"], inp["W1"], inp["W2"], inp["b_g"], inp["b1"], inp["b2"],
                                   inp.get("b_sel"), inp.get("S1"), inp.get("sb1"), inp.get("S2"), inp.get("sb2"))
 
@@ -521,6 +521,66 @@ def test_capacity_drop(name, wl):
         assert dropped == 0
     else:
         assert dropped > 0, "the case should overflow some expert"
+
+
+REROUTE_CASES = [
+    ("fp32_small_router", Workload("rr_f32", 66, 300, 64, 256, 8, 2, ACT_GELU, torch.float32, True, 0.05,
+                                   zipf_s=1.2, random_bias=True, capacity_factor=1.0, overflow=1)),
+    ("fp32_chunked_router_k3", Workload("rr_f32c", 67, 2300, 64, 128, 16, 3, ACT_GELU, torch.float32, False, 0.05,
+                                        zipf_s=1.0, capacity_factor=0.9, overflow=1)),
+    ("bf16_simt_router_k2", Workload("rr_k2", 68, 1500, 256, 512, 6, 2, ACT_GELU, torch.bfloat16, True, 0.04,
+                                     zipf_s=1.0, random_bias=True, capacity_factor=1.0, overflow=1)),
+    ("bf16_tc_router_k8_bias", Workload("rr_tc", 69, 1200, 256, 256, 64, 8, ACT_SWIGLU, torch.bfloat16, False, 0.05,
+                                        zipf_s=1.2, sel_s=0.3, capacity_factor=0.6, overflow=1)),
+    ("bf16_shared", Workload("rr_sh", 70, 1500, 512, 1024, 8, 2, ACT_SWIGLU, torch.bfloat16, False, 0.04,
+                             zipf_s=0.9, n_shared=1, capacity_factor=0.8, overflow=1)),
+    ("decode8", WORKLOADS["decode8"].with_(zipf_s=2.0, capacity_factor=1.0, overflow=1)),
+    ("decode64_bias", WORKLOADS["decode64"].with_(zipf_s=1.0, sel_s=0.5, capacity_factor=0.5, overflow=1)),
+    ("huge_capacity", Workload("rr_big", 71, 700, 256, 256, 8, 2, ACT_SWIGLU, torch.bfloat16, False, 0.05,
+                               zipf_s=0.5, capacity_factor=8.0, overflow=1)),
+]
+
+
+@pytest.mark.parametrize("name,wl", REROUTE_CASES, ids=[c[0] for c in REROUTE_CASES])
+def test_capacity_reroute(name, wl):
+    """Per-expert capacity with the next-candidate reroute: the expert serving every slot is the
+    oracle's reroute decision on the device's selection values (bit-exact), each expert's segment
+    holds its slots in token order, dropped slots add nothing, y matches the oracle, and the
+    statistics still describe the router's own choice."""
+    inp = make_inputs(wl, "cuda")
+    layer = Layer(wl, inp)
+    T, N, K = wl.T, wl.N, wl.K
+    y, ws, aux = layer.forward()
+    V = layer.views(ws, T)
+    ref = ph.oracle_full_layer(inp, wl, K, gpu_logits=V["logits"])
+    C = ref["capacity"]
+    assert C == int(np.ceil(ph.capacity_factor(wl) * T * K / N))
+    ph.assert_logits_close(V["logits"], ref["scores"])
+    sel = oracle.select_topk(ph.selection_scores(V["logits"], inp).astype(np.float64), K)
+    assign = oracle.capacity_reroute(ph.selection_scores(V["logits"], inp).astype(np.float64), sel, C)
+    np.testing.assert_array_equal(assign, ref["assign"])
+    # idx holds the serving expert; a dropped slot keeps its (full) selected expert
+    np.testing.assert_array_equal(V["idx"], np.where(assign >= 0, assign, sel))
+    ph.assert_weights_close(V["w"], ref["w"], ref["scores"])
+    kept = assign.ravel() >= 0
+    flat = assign.ravel()
+    counts = np.bincount(flat[kept], minlength=N)
+    assert (counts <= C).all()
+    np.testing.assert_array_equal(V["counts"], counts)
+    ro = V["row_offsets"]
+    for e in range(N):
+        seg = V["perm_slot"][ro[e]:ro[e] + counts[e]]
+        np.testing.assert_array_equal(seg, np.nonzero(flat == e)[0])
+    assert np.all(V["slot_row"][~kept] == -1)
+    ph.assert_y_close(y.float().cpu().numpy(), ref["y"], wl.dtype)
+    # statistics of the router's choice, before the capacity
+    st = oracle.aux_stats(V["logits"].astype(np.float64), sel, V["w"].astype(np.float64), N)
+    np.testing.assert_array_equal(aux["counts"].cpu().numpy(), st["counts"].astype(np.int32))
+    rerouted = int(((assign != sel) & (assign >= 0)).sum())
+    if name == "huge_capacity":
+        assert rerouted == 0 and kept.all()
+    else:
+        assert rerouted > 0, "the case should reroute some slot"
 
 
 # ----------------------------------------------------------------------------- expert parallelism
