@@ -72,7 +72,8 @@ struct Plan {
     int n_shared;      // 1: a shared expert (dense FFN over every token) is added after the routed sum
     int capacity;      // assignments each expert accepts (rows served in order)
     bool reroute;      // refused assignments go to the next candidate (reroute_kernel) instead of being dropped
-    int rr_batch;      // reroute_kernel: tokens staged per buffer
+    int rr_batch;      // reroute_kernel: tokens per batch (selections staged, two buffers)
+    int rr_vbatch;     // reroute_kernel: tokens whose selection values are staged at a time
     bool fused_decode; // few tokens, N <= 32, no shared expert: the whole layer in one cooperative kernel
     bool given_routing;
     int slab_rows, n_slabs;   // fused decode: W_g rows per routing slab, slabs
@@ -124,7 +125,9 @@ int make_plan(const moe_config *c, int64_t T, Plan *p, bool given_routing = fals
         p->capacity = INT32_MAX;
     }
     p->reroute = c->capacity_factor > 0.0f && c->overflow == MOE_OVERFLOW_REROUTE;
-    p->rr_batch = (int)std::max<int64_t>(1, std::min<int64_t>(1024, (kRerouteSmem - N * 4 - 16) / (2 * (K + N) * 4)));
+    p->rr_batch = (int)std::min<int64_t>(1024, std::max<int64_t>(1, (kRerouteSmem / 4 - N * 8 - 32) / (2 * K * 4)));
+    p->rr_vbatch = (int)std::max<int64_t>(1, std::min<int64_t>(p->rr_batch,
+        (kRerouteSmem - N * 8 - 32 - (int64_t)2 * p->rr_batch * K * 4) / (N * 4)));
     p->np = N <= 8 ? 8 : N <= 16 ? 16 : 32;
     const bool fits = N <= 32 && (size_t)p->np * D * es + 256 <= kSmallRouterSmemMax;
     p->rowdot_router = N <= 32 && (T < kRowdotMaxT || !fits);
@@ -228,7 +231,12 @@ int device_info(DeviceInfo **out) {
         if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return MOE_ERR_CUDA;
     }
     if (!d.attrs) {
-        MOE_TRY(allow_smem(reroute_kernel));
+        MOE_TRY(allow_smem(reroute_kernel<1>));
+        MOE_TRY(allow_smem(reroute_kernel<2>));
+        MOE_TRY(allow_smem(reroute_kernel<4>));
+        MOE_TRY(allow_smem(reroute_kernel<8>));
+        MOE_TRY(allow_smem(reroute_kernel<16>));
+        MOE_TRY(allow_smem(reroute_kernel<32>));
         MOE_TRY(allow_smem(tc::grouped_gemm_tc_kernel<256, tc::EPI_GELU>));
         MOE_TRY(allow_smem(tc::grouped_gemm_tc_kernel<256, tc::EPI_SWIGLU>));
         MOE_TRY(allow_smem(tc::grouped_gemm_tc_kernel<256, tc::EPI_SCATTER>));
@@ -688,10 +696,20 @@ int stage_route(const Plan &P, const Bufs &b, const void *x, const moe_weights *
 int stage_scan(const Plan &P, const Bufs &b, int *counts_out, cudaStream_t s, int counter_word = 0);
 int stage_reroute(const Plan &P, const Bufs &b, const moe_weights *w, cudaStream_t s) {
     const int N = P.N, K = P.K, B = P.rr_batch;
-    const size_t smem = (size_t)((N + 3) & ~3) * 4 + (size_t)2 * B * K * 4 + (size_t)2 * B * N * 4;
+    const int VB = P.rr_vbatch;
+    const size_t smem = (size_t)2 * ((N + 3) & ~3) * 4 + (size_t)2 * B * K * 4 + (size_t)VB * N * 4;
     if (smem > (size_t)kRerouteSmem) return MOE_ERR_UNSUPPORTED;
-    reroute_kernel<<<1, kRerouteThreads, smem, s>>>(b.at<float>(P.logits), w->b_sel, b.at<int>(P.idx), (int)P.T, N, K,
-                                                    P.capacity, B);
+    const int npl = (N + 31) / 32;
+    auto go = [&](auto kernel) {
+        kernel<<<1, kRerouteThreads, smem, s>>>(b.at<float>(P.logits), w->b_sel, b.at<int>(P.idx), P.T, N, K,
+                                                P.capacity, B, VB);
+    };
+    if (npl <= 1) go(reroute_kernel<1>);
+    else if (npl <= 2) go(reroute_kernel<2>);
+    else if (npl <= 4) go(reroute_kernel<4>);
+    else if (npl <= 8) go(reroute_kernel<8>);
+    else if (npl <= 16) go(reroute_kernel<16>);
+    else go(reroute_kernel<32>);
     MOE_TRY(check_launch());
     hist_kernel<<<P.n_chunks, 256, (size_t)N * 4, s>>>(b.at<int>(P.idx), P.T * K, P.chunk_tokens * K, N, 1,
                                                       b.at<int>(P.chunk_counts));
@@ -811,6 +829,15 @@ bool narrow_tiles(const Plan &P, int64_t n_tiles_256, const DeviceInfo &dev) {
     return m_tiles_min * n_tiles_256 < (int64_t)dev.sms;
 }
 
+// Whether the experts' odd last 128-row blocks go to a 1-CTA tail kernel beside
+// the pair kernel instead of half-empty pair tiles.  The half-empty tiles cost
+// about 64 rows per expert (half the experts have an odd block count), a share
+// 64 N / (T K) of the rows; the tail kernel's tiles are less efficient (B not
+// shared by a pair) and partly run after the pair kernel, which measured slower
+// at 2.3% (6 experts x 2731 rows) and 6% (8 x 1024) and faster at 12.5%
+// (256 x 512).
+bool tail_split(const Plan &P) { return 64.0 * P.N > 0.1 * (double)(P.T * P.K); }
+
 int stage_up(const Plan &P, const Bufs &b, const moe_weights *w, const DeviceInfo &dev, cudaStream_t s) {
     if (P.decode) return stage_up_decode(P, b, w, dev, s);
     const int D = P.D, H = P.H, N = P.N;
@@ -843,6 +870,10 @@ int stage_up(const Plan &P, const Bufs &b, const moe_weights *w, const DeviceInf
         // 256-row pair tiles for each expert's pairs of 128-row blocks, then
         // 128-row tiles on one CTA for the experts' odd last blocks
         const int64_t units = (P.rows_cap / (2 * tc::BM) + N) * p.n_tiles;
+        if (!tail_split(P)) {
+            if (swiglu) return launch_tc2<tc::EPI_SWIGLU>(ma, mb, mo, p, units, dev.pair_clusters, s);
+            return launch_tc2<tc::EPI_GELU>(ma, mb, mo, p, units, dev.pair_clusters, s);
+        }
         p.tail_mode = 1;
         if (swiglu) MOE_TRY(launch_tc2<tc::EPI_SWIGLU>(ma, mb, mo, p, units, dev.pair_clusters, s));
         else MOE_TRY(launch_tc2<tc::EPI_GELU>(ma, mb, mo, p, units, dev.pair_clusters, s));
@@ -914,6 +945,9 @@ int stage_down(const Plan &P, const Bufs &b, const moe_weights *w, void *y, int 
         const int64_t upper = (P.rows_cap / tc::BM) * p.n_tiles;
         if (bn == 128) return launch_tc<128, tc::EPI_SCATTER>(ma, mb, mo, p, upper, dev.sms, s);
         // pair tiles, then the odd last blocks on one CTA (as in the up projection)
+        if (!tail_split(P))
+            return launch_tc2<tc::EPI_SCATTER>(ma, mb, mo, p, (P.rows_cap / (2 * tc::BM) + N) * p.n_tiles,
+                                               dev.pair_clusters, s);
         p.tail_mode = 1;
         MOE_TRY(launch_tc2<tc::EPI_SCATTER>(ma, mb, mo, p, (P.rows_cap / (2 * tc::BM) + N) * p.n_tiles,
                                             dev.pair_clusters, s));
@@ -1150,15 +1184,22 @@ int zero_aux(const Plan &P, moe_aux *aux, cudaStream_t s) {
 }
 
 // ---------------------------------------------------------------- fused decode
+// Routing scratch of the fused decode kernel, in its ring: R1 x rows, W_g slab
+// and per-warp partials; R2 the slabs' scores of one token; R3 top-k experts,
+// ranks, gate weights and full softmax.
+size_t fused_scratch(int T, int slab_rows, int n_slabs) {
+    const size_t r1 = ((size_t)T * slab_rows + (size_t)slab_rows * 32 + (size_t)(dfu::kThreads / 32) * T * 32) * 4;
+    const size_t r2 = (size_t)n_slabs * 32 * 4;
+    const size_t r3 = ((size_t)3 * dfu::kMaxSlots + (size_t)T * 32) * 4;
+    return std::max(r1, std::max(r2, r3));
+}
+
 template <int NT, int EPI>
 int launch_fused(const CUtensorMap &mw1, const CUtensorMap &mxp, const CUtensorMap &mw2, const CUtensorMap &mh,
                  const dfu::Params &p, int grid, cudaStream_t s) {
     using S = dfu::Shape<NT, EPI>;
-    // routing scratch (R1, R3) lives in the ring before the expert phases use it
-    const size_t scratch = std::max<size_t>(((size_t)p.T * p.slab_rows + (size_t)p.slab_rows * 32 +
-                                             (size_t)(dfu::kThreads / 32) * p.T * 32) * 4,
-                                            (size_t)2 * dfu::kMaxSlots * 4);
-    if (scratch > S::kRingBytes) return MOE_ERR_UNSUPPORTED;
+    // routing scratch (R1-R3) lives in the ring before the expert phases use it
+    if (fused_scratch(p.T, p.slab_rows, p.n_slabs) > S::kRingBytes) return MOE_ERR_UNSUPPORTED;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)grid);
     cfg.blockDim = dim3(dfu::kThreads);
@@ -1191,13 +1232,7 @@ bool fused_fits_nt(int nt, size_t scratch) {
     return scratch <= dfu::Shape<64, EPI>::kRingBytes;
 }
 bool fused_fits(const Plan &P) {
-    // R1: x rows, W_g slab and per-warp partials; R2: the slabs' scores of one
-    // token; R3: top-k experts, ranks, gate weights and full softmax
-    const size_t r1 = ((size_t)P.T * P.slab_rows + (size_t)P.slab_rows * 32 +
-                       (size_t)(dfu::kThreads / 32) * P.T * 32) * 4;
-    const size_t r2 = (size_t)P.n_slabs * 32 * 4;
-    const size_t r3 = ((size_t)3 * dfu::kMaxSlots + (size_t)P.T * 32) * 4;
-    const size_t scratch = std::max(r1, std::max(r2, r3));
+    const size_t scratch = fused_scratch((int)P.T, P.slab_rows, P.n_slabs);
     return P.act == MOE_ACT_SWIGLU ? fused_fits_nt<dec::EPI_SWIGLU>(P.nt, scratch)
                                    : fused_fits_nt<dec::EPI_GELU>(P.nt, scratch);
 }

@@ -777,8 +777,12 @@ template <int EPI>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     grouped_gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                             const __grid_constant__ CUtensorMap tmO, const Params p) {
-    pdl_wait();                 // the dependent (a tail kernel may run beside this one) launches
-    pdl_launch_dependents();    // only once everything before this kernel is complete
+    if (p.tail_mode == 1) {
+        pdl_wait();                 // the dependent (the tail kernel, run beside this one) launches
+        pdl_launch_dependents();    // only once everything before this kernel is complete
+    } else {
+        pdl_enter();
+    }
     using S = Shape2;
     constexpr int BN = 256;
     constexpr int kStages = S::kStages;

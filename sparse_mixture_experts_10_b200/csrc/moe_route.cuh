@@ -392,127 +392,200 @@ __global__ void __launch_bounds__(256) hist_kernel(const int *__restrict__ idx, 
 // (full) selected expert, so the capacity scan that follows drops it, and
 // every accepted slot lands within the first C of its expert.
 //
-// The order of service makes this sequential in t.  One CTA: warp 0 walks the
-// tokens with the per-expert loads in shared memory, the other 31 warps stage
-// the next batch of selections and selection values meanwhile (two buffers).
-// Warp 0 takes 32/K tokens at a time: each lane one (token, slot), its place
-// in its expert = the expert's load + the lanes before it with the same expert
-// (match.any); the tokens before the first refused slot are accepted as they
-// are, the refusing token goes through the full per-token step alone.
+// The order of service makes this sequential in t.  One CTA, the per-expert
+// loads in shared memory, tokens staged in batches (two buffers):
+//   * a batch in which no expert would pass C (its histogram added to the
+//     loads) is accepted whole by all threads -- the common case while the
+//     experts fill;
+//   * otherwise warp 0 walks it, vbatch tokens at a time whose selection
+//     values all threads stage first (only such batches need them): 32/K
+//     tokens per step, each lane one (token, slot), its place = the
+//     expert's load + the earlier lanes with the same expert (match.any); the
+//     tokens before the first refused slot are accepted, the refusing token
+//     takes the per-token step: its free candidates are read into registers
+//     once (NPL per lane) and each refused slot takes the best of them by a
+//     warp arg-max, in slot order.
 // ---------------------------------------------------------------------------
 constexpr int kRerouteThreads = 1024;
 
-__device__ __forceinline__ void reroute_stage(const float *__restrict__ logits, const float *__restrict__ bsel,
-                                              const int *__restrict__ idx, int T, int N, int K, int batch, int bi,
-                                              int *sidx, float *sv, int tid0, int nthr) {
-    const int64_t t0 = (int64_t)bi * batch;
-    const int rows = (int)(T - t0 < (int64_t)batch ? T - t0 : (int64_t)batch);
-    for (int i = tid0; i < rows * K; i += nthr) {
-        int e = idx[t0 * K + i];
-        if ((unsigned)e >= (unsigned)N) {   // not an expert: counted against expert 0, flagged
-            set_status(kStatusBounds);
-            e = 0;
+// The selections of tokens [t0, t0 + rows) into shared memory (eight loads in
+// flight per thread).
+__device__ __forceinline__ void reroute_stage_idx(const int *__restrict__ idx, int64_t t0, int rows, int N, int K,
+                                                  int *sidx) {
+    const int n = rows * K;
+    for (int i0 = threadIdx.x; i0 < n; i0 += 8 * kRerouteThreads) {
+        int v[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int i = i0 + u * kRerouteThreads;
+            v[u] = i < n ? idx[t0 * K + i] : 0;
         }
-        sidx[i] = e;
-    }
-    for (int i = tid0; i < rows * N; i += nthr) {
-        const int e = i % N;
-        float v = logits[t0 * N + i];
-        if (bsel) v += __ldg(bsel + e);
-        sv[i] = v != v ? -INFINITY : v;   // NaN ranked as -inf, as in the selection
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int i = i0 + u * kRerouteThreads;
+            if (i >= n) continue;
+            int e = v[u];
+            if ((unsigned)e >= (unsigned)N) {   // not an expert: counted against expert 0, flagged
+                set_status(kStatusBounds);
+                e = 0;
+            }
+            sidx[i] = e;
+        }
     }
 }
 
-__global__ void __launch_bounds__(kRerouteThreads, 1)
-    reroute_kernel(const float *__restrict__ logits, const float *__restrict__ bsel, int *__restrict__ idx, int T,
-                   int N, int K, int C, int batch) {
-    extern __shared__ __align__(16) unsigned char rr_smem[];
-    int *load = reinterpret_cast<int *>(rr_smem);                        // [N]
-    int *sidx = load + ((N + 3) & ~3);                                   // [2][batch * K]
-    float *sv = reinterpret_cast<float *>(sidx + 2 * batch * K);         // [2][batch * N]
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const unsigned FULL = 0xffffffffu;
-    for (int e = tid; e < N; e += kRerouteThreads) load[e] = 0;
-    const int nb = (int)((T + batch - 1) / batch);
-    reroute_stage(logits, bsel, idx, T, N, K, batch, 0, sidx, sv, tid, kRerouteThreads);
-    __syncthreads();
-    const int G = 32 / K;   // tokens per step of the fast path
-    for (int bi = 0; bi < nb; ++bi) {
-        const int cur = bi & 1;
-        int *bidx = sidx + cur * batch * K;
-        const float *bv = sv + (size_t)cur * batch * N;
-        if (warp != 0) {
-            if (bi + 1 < nb)
-                reroute_stage(logits, bsel, idx, T, N, K, batch, bi + 1, sidx + (cur ^ 1) * batch * K,
-                              sv + (size_t)(cur ^ 1) * batch * N, tid - 32, kRerouteThreads - 32);
-        } else {
-            const int64_t t0 = (int64_t)bi * batch;
-            const int rows = (int)(T - t0 < (int64_t)batch ? T - t0 : (int64_t)batch);
-            int lt = 0;
-            while (lt < rows) {
-                // fast path: G tokens, one (token, slot) per lane
-                const int g = min(G, rows - lt);
-                const bool act = lane < g * K;
-                const int tl = lane / K, j = lane - tl * K;
-                const int e = act ? bidx[(lt + tl) * K + j] : -1 - lane;   // inactive lanes: distinct keys
-                const unsigned peers = __match_any_sync(FULL, e);
-                const int pos = act ? load[e] + __popc(peers & lanemask_lt()) : 0;
-                const unsigned refused = __ballot_sync(FULL, act && pos >= C);
-                const int good = refused ? (__ffs(refused) - 1) / K : g;   // tokens accepted as they are
-                const unsigned accm = __ballot_sync(FULL, act && tl < good);
-                const unsigned pa = peers & accm;
-                if (((accm >> lane) & 1u) && (pa >> lane) == 1u) load[e] += __popc(pa);   // last lane of its expert
-                __syncwarp();
-                lt += good;
-                if (good == g) continue;
-                // the refusing token, alone: accept what fits, reroute the rest in slot order
-                const int64_t t = t0 + lt;
-                const int ej = lane < K ? bidx[lt * K + lane] : -1;
-                const bool room = lane < K && load[ej] < C;
-                if (room) load[ej] += 1;   // a token's K experts are distinct
-                __syncwarp();
-                unsigned todo = __ballot_sync(FULL, lane < K && !room);
-                uint32_t held = 0;         // bit i: expert lane + 32 i is one of the token's
-                for (int jj = 0; jj < K; ++jj) {
-                    const int h = __shfl_sync(FULL, ej, jj);
-                    if ((h & 31) == lane) held |= 1u << (h >> 5);
-                }
-                const float *vrow = bv + (size_t)lt * N;
-                while (todo) {
-                    const int js = __ffs(todo) - 1;
-                    todo &= todo - 1;
-                    float best_v = -INFINITY;
-                    int best_e = -1;
-                    for (int i = 0; lane + 32 * i < N; ++i) {
-                        const int c = lane + 32 * i;
-                        if (((held >> i) & 1u) || load[c] >= C) continue;
-                        const float v = vrow[c];
-                        if (best_e < 0 || v > best_v) {   // ascending c: ties keep the lower index
-                            best_v = v;
-                            best_e = c;
-                        }
-                    }
+// The selection values (logit + b_sel in fp32, NaN ranked as -inf) of tokens
+// [t0, t0 + rows) into shared memory, eight loads in flight per thread.
+__device__ __forceinline__ void reroute_stage_values(const float *__restrict__ logits, const float *__restrict__ bsel,
+                                                     int64_t t0, int rows, int N, float *sv) {
+    const int n = rows * N;
+    const float *src = logits + t0 * N;
+    for (int i0 = threadIdx.x; i0 < n; i0 += 8 * kRerouteThreads) {
+        float v[8];
 #pragma unroll
-                    for (int o = 16; o; o >>= 1) {
-                        const float ov = __shfl_xor_sync(FULL, best_v, o);
-                        const int oe = __shfl_xor_sync(FULL, best_e, o);
-                        if (oe >= 0 && (best_e < 0 || ov > best_v || (ov == best_v && oe < best_e))) {
-                            best_v = ov;
-                            best_e = oe;
-                        }
-                    }
-                    if (best_e >= 0) {
-                        if (lane == 0) {
-                            load[best_e] += 1;
-                            idx[t * K + js] = best_e;
-                        }
-                        if ((best_e & 31) == lane) held |= 1u << (best_e >> 5);
-                    }
-                    __syncwarp();
+        for (int u = 0; u < 8; ++u) {
+            const int i = i0 + u * kRerouteThreads;
+            v[u] = i < n ? src[i] : 0.f;
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int i = i0 + u * kRerouteThreads;
+            if (i >= n) continue;
+            float x = v[u];
+            if (bsel) x += __ldg(bsel + i % N);
+            sv[i] = x != x ? -INFINITY : x;
+        }
+    }
+}
+
+// Warp 0's walk over one batch (see above).
+template <int NPL>
+__device__ __forceinline__ void reroute_walk(int *load, const int *bidx, const float *bv, int *__restrict__ idx,
+                                             int64_t t0, int rows, int N, int K, int C) {
+    const int lane = threadIdx.x & 31;
+    const unsigned FULL = 0xffffffffu;
+    const int G = 32 / K;   // tokens per step of the fast path
+    int lt = 0;
+    while (lt < rows) {
+        const int g = min(G, rows - lt);
+        const bool act = lane < g * K;
+        const int tl = lane / K, j = lane - tl * K;
+        const int e = act ? bidx[(lt + tl) * K + j] : -1 - lane;   // inactive lanes: distinct keys
+        const unsigned peers = __match_any_sync(FULL, e);
+        const int pos = act ? load[e] + __popc(peers & lanemask_lt()) : 0;
+        const unsigned refused = __ballot_sync(FULL, act && pos >= C);
+        const int good = refused ? (__ffs(refused) - 1) / K : g;   // tokens accepted as they are
+        const unsigned accm = __ballot_sync(FULL, act && tl < good);
+        const unsigned pa = peers & accm;
+        if (((accm >> lane) & 1u) && (pa >> lane) == 1u) load[e] += __popc(pa);   // last lane of its expert
+        __syncwarp();
+        lt += good;
+        if (good == g) continue;
+        // the refusing token, alone: accept what fits, reroute the rest in slot order
+        const int64_t t = t0 + lt;
+        const int ej = lane < K ? bidx[lt * K + lane] : -1;
+        const bool room = lane < K && load[ej] < C;
+        if (room) load[ej] += 1;   // a token's K experts are distinct
+        __syncwarp();
+        unsigned todo = __ballot_sync(FULL, lane < K && !room);
+        uint32_t held = 0;         // bit i: expert lane + 32 i is one of the token's
+        for (int jj = 0; jj < K; ++jj) {
+            const int h = __shfl_sync(FULL, ej, jj);
+            if ((h & 31) == lane) held |= 1u << (h >> 5);
+        }
+        // this lane's free candidates, read once: value, or unavailable
+        const float *vrow = bv + (size_t)lt * N;
+        float cv[NPL];
+        bool ca[NPL];
+#pragma unroll
+        for (int i = 0; i < NPL; ++i) {
+            const int c = lane + 32 * i;
+            const bool in = c < N;
+            const int ld = in ? load[c] : C;
+            cv[i] = in ? vrow[c] : 0.f;
+            ca[i] = in && ld < C && !((held >> i) & 1u);
+        }
+        while (todo) {
+            const int js = __ffs(todo) - 1;
+            todo &= todo - 1;
+            float best_v = -INFINITY;
+            int best_e = -1;
+#pragma unroll
+            for (int i = 0; i < NPL; ++i)
+                if (ca[i] && (best_e < 0 || cv[i] > best_v)) {   // ascending experts: ties keep the lower index
+                    best_v = cv[i];
+                    best_e = lane + 32 * i;
                 }
-                lt += 1;
+#pragma unroll
+            for (int o = 16; o; o >>= 1) {
+                const float ov = __shfl_xor_sync(FULL, best_v, o);
+                const int oe = __shfl_xor_sync(FULL, best_e, o);
+                if (oe >= 0 && (best_e < 0 || ov > best_v || (ov == best_v && oe < best_e))) {
+                    best_v = ov;
+                    best_e = oe;
+                }
+            }
+            if (best_e < 0) break;   // no expert left with room: the remaining refused slots are dropped
+            if (lane == 0) {
+                load[best_e] += 1;
+                idx[t * K + js] = best_e;
+            }
+            if ((best_e & 31) == lane) {
+#pragma unroll
+                for (int i = 0; i < NPL; ++i)
+                    if ((best_e >> 5) == i) ca[i] = false;
             }
         }
+        __syncwarp();
+        lt += 1;
+    }
+}
+
+template <int NPL>
+__global__ void __launch_bounds__(kRerouteThreads, 1)
+    reroute_kernel(const float *__restrict__ logits, const float *__restrict__ bsel, int *__restrict__ idx,
+                   int64_t T, int N, int K, int C, int batch, int vbatch) {
+    extern __shared__ __align__(16) unsigned char rr_smem[];
+    const int npad = (N + 3) & ~3;
+    int *load = reinterpret_cast<int *>(rr_smem);                        // [N]
+    int *hist = load + npad;                                             // [N] the batch's histogram
+    int *sidx = hist + npad;                                             // [2][batch * K]
+    float *sv = reinterpret_cast<float *>(sidx + 2 * batch * K);         // [vbatch * N]
+    const int tid = threadIdx.x, warp = tid >> 5;
+    for (int e = tid; e < N; e += kRerouteThreads) load[e] = 0;
+    const int nb = (int)((T + batch - 1) / batch);
+    auto rows_of = [&](int bi) {
+        const int64_t t0 = (int64_t)bi * batch;
+        return (int)(T - t0 < (int64_t)batch ? T - t0 : (int64_t)batch);
+    };
+    reroute_stage_idx(idx, 0, rows_of(0), N, K, sidx);
+    __syncthreads();
+    for (int bi = 0; bi < nb; ++bi) {
+        const int cur = bi & 1;
+        const int *bidx = sidx + cur * batch * K;
+        const int64_t t0 = (int64_t)bi * batch;
+        const int rows = rows_of(bi);
+        // the whole batch at once when no expert would pass C
+        for (int e = tid; e < N; e += kRerouteThreads) hist[e] = 0;
+        __syncthreads();
+        for (int i = tid; i < rows * K; i += kRerouteThreads) atomicAdd(&hist[bidx[i]], 1);
+        __syncthreads();
+        bool over = false;
+        for (int e = tid; e < N; e += kRerouteThreads) over |= load[e] + hist[e] > C;
+        over = __syncthreads_or(over);
+        if (!over) {
+            for (int e = tid; e < N; e += kRerouteThreads) load[e] += hist[e];
+        } else {
+            // warp 0 walks the batch, vbatch tokens at a time with their values staged by all
+            for (int s0 = 0; s0 < rows; s0 += vbatch) {
+                const int vr = min(vbatch, rows - s0);
+                reroute_stage_values(logits, bsel, t0 + s0, vr, N, sv);
+                __syncthreads();
+                if (warp == 0) reroute_walk<NPL>(load, bidx + s0 * K, sv, idx, t0 + s0, vr, N, K, C);
+                __syncthreads();
+            }
+        }
+        if (bi + 1 < nb) reroute_stage_idx(idx, t0 + batch, rows_of(bi + 1), N, K, sidx + (cur ^ 1) * batch * K);
         __syncthreads();
     }
 }
