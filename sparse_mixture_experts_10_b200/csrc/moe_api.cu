@@ -1184,11 +1184,15 @@ int zero_aux(const Plan &P, moe_aux *aux, cudaStream_t s) {
 }
 
 // ---------------------------------------------------------------- fused decode
-// Routing scratch of the fused decode kernel, in its ring: R1 x rows, W_g slab
-// and per-warp partials; R2 the slabs' scores of one token; R3 top-k experts,
+// Whether the fused decode kernel is launched with programmatic serialization
+// besides the cooperative attribute (cleared if the runtime refuses the pair).
+std::atomic<bool> g_fused_pdl{true};
+
+// Routing scratch of the fused decode kernel, in its ring: R1 x rows and the
+// W_g slab; R2 the slabs' scores of one token; R3 top-k experts,
 // ranks, gate weights and full softmax.
 size_t fused_scratch(int T, int slab_rows, int n_slabs) {
-    const size_t r1 = ((size_t)T * slab_rows + (size_t)slab_rows * 32 + (size_t)(dfu::kThreads / 32) * T * 32) * 4;
+    const size_t r1 = ((size_t)T * slab_rows + (size_t)slab_rows * 32) * 4;
     const size_t r2 = (size_t)n_slabs * 32 * 4;
     const size_t r3 = ((size_t)3 * dfu::kMaxSlots + (size_t)T * 32) * 4;
     return std::max(r1, std::max(r2, r3));
@@ -1205,12 +1209,21 @@ int launch_fused(const CUtensorMap &mw1, const CUtensorMap &mxp, const CUtensorM
     cfg.blockDim = dim3(dfu::kThreads);
     cfg.dynamicSmemBytes = S::kSmem;
     cfg.stream = s;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeCooperative;   // every CTA resident: the grid barriers need it
     attr[0].val.cooperative = 1;
+    // and launched while the counters are being cleared (its pdl_enter waits for that)
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    const cudaError_t e = cudaLaunchKernelEx(&cfg, dfu::decode_layer_kernel<NT, EPI>, mw1, mxp, mw2, mh, p);
+    cfg.numAttrs = g_fused_pdl ? 2 : 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, dfu::decode_layer_kernel<NT, EPI>, mw1, mxp, mw2, mh, p);
+    if (e != cudaSuccess && cfg.numAttrs == 2) {   // the runtime refused the pair: cooperative alone
+        (void)cudaGetLastError();
+        g_fused_pdl = false;
+        cfg.numAttrs = 1;
+        e = cudaLaunchKernelEx(&cfg, dfu::decode_layer_kernel<NT, EPI>, mw1, mxp, mw2, mh, p);
+    }
     g_launches.fetch_add(1, std::memory_order_relaxed);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;

@@ -88,7 +88,7 @@ struct Shape {
     static constexpr uint32_t kTableBytes = 2 * kMaxSlots * 2 + 8 * 40 * 4;
     static constexpr int kStages0 =
         (int)((220 * 1024 - 1024 - kEpiBytes - kTableBytes - 256) / kStageBytes);
-    static constexpr int kStages = kStages0 > 8 ? 8 : kStages0;
+    static constexpr int kStages = kStages0 > 16 ? 16 : kStages0;   // as many weight tiles in flight as fit
     static constexpr uint32_t kRingBytes = kStages * kStageBytes;
     static constexpr uint32_t kTmemCols = 2 * NT < 32 ? 32 : 2 * NT;
     static constexpr size_t kSmem = 1024 + (size_t)kRingBytes + kEpiBytes + kTableBytes + (2 * kStages + 6) * 8 + 64;
@@ -150,7 +150,6 @@ __device__ __forceinline__ void route_r1(const Params &p, uint8_t *scratch) {
     if (nd <= 0) return;
     float *xs = reinterpret_cast<float *>(scratch);            // [T][R]
     float *ws = xs + (size_t)T * R;                            // [R][32]
-    float *red = ws + (size_t)R * 32;                          // [6][T][32]
     // 16-byte loads: slab rows start at multiples of 8 elements and D, N * 8 are multiples of 8
     const int xv = nd / 8;
     for (int i = tid; i < T * xv; i += kThreads) {
@@ -178,25 +177,21 @@ __device__ __forceinline__ void route_r1(const Params &p, uint8_t *scratch) {
             }
     }
     __syncthreads();
-    float acc[kMaxT];
-#pragma unroll
-    for (int t = 0; t < kMaxT; ++t) acc[t] = 0.f;
-    const float wmask = lane < N ? 1.f : 0.f;
-    for (int k = warp; k < nd; k += kThreads / 32) {
-        const float wv = wmask * ws[k * 32 + lane];
-#pragma unroll
-        for (int t = 0; t < kMaxT; ++t)
-            if (t < T) acc[t] = fmaf(xs[t * R + k], wv, acc[t]);
-    }
-#pragma unroll
-    for (int t = 0; t < kMaxT; ++t)
-        if (t < T) red[(warp * T + t) * 32 + lane] = acc[t];
-    __syncthreads();
-    for (int i = tid; i < T * 32; i += kThreads) {
-        float v = 0.f;
-#pragma unroll
-        for (int w = 0; w < kThreads / 32; ++w) v += red[w * T * 32 + i];   // warps in order
-        p.slab[(size_t)c * T * 32 + i] = v;
+    // partial scores of the slab: warp w takes tokens w, w + 6, ...; lane = expert;
+    // four running sums over the slab rows (k mod 4), added in a fixed order
+    for (int t = warp; t < T; t += kThreads / 32) {
+        const float *xr = xs + (size_t)t * R;
+        float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+        int k = 0;
+        for (; k + 4 <= nd; k += 4) {
+            a0 = fmaf(xr[k], ws[k * 32 + lane], a0);
+            a1 = fmaf(xr[k + 1], ws[(k + 1) * 32 + lane], a1);
+            a2 = fmaf(xr[k + 2], ws[(k + 2) * 32 + lane], a2);
+            a3 = fmaf(xr[k + 3], ws[(k + 3) * 32 + lane], a3);
+        }
+        for (; k < nd; ++k) a0 = fmaf(xr[k], ws[k * 32 + lane], a0);
+        const float v = (a0 + a1) + (a2 + a3);
+        p.slab[((size_t)c * T + t) * 32 + lane] = lane < N ? v : 0.f;   // lanes past N hold no expert
     }
 }
 
@@ -298,6 +293,23 @@ __device__ __forceinline__ void route_r3(const Params &p, const Tables &tb, uint
         if (keep) tb.ent[tb.koff[e] + pos] = (int16_t)i;
     }
     __syncthreads();
+    // the kept slots' token rows into x_perm, one slot per CTA at a time
+    const int nv = p.D / 8;
+    for (int i = blockIdx.x; i < TK; i += gridDim.x) {
+        const int r = tb.row[i];
+        if (r < 0) continue;
+        const uint4 *src = reinterpret_cast<const uint4 *>(p.x + (size_t)(i / p.K) * p.D);
+        uint4 *dst = reinterpret_cast<uint4 *>(p.x_perm + (size_t)r * p.D);
+        for (int v = tid; v < nv; v += kThreads) dst[v] = __ldg(src + v);
+    }
+    // x_perm written: release it to the grid (barrier 3 is waited on only by the
+    // producers, before their first token-row load); the workspace tables and the
+    // statistics follow in CTA 0, off the critical path
+    __syncthreads();
+    if (tid == 0) {
+        fence_proxy_async_global();
+        grid_arrive(p.bar);
+    }
     if (blockIdx.x == 0) {
         // the workspace tables (moe_get_workspace_layout) and the statistics
         for (int e = tid; e < N; e += kThreads) {
@@ -372,15 +384,6 @@ __device__ __forceinline__ void route_r3(const Params &p, const Tables &tb, uint
             p.aux_scalars[2] = mi == 0.0 ? 0.f : (float)(vi / (mi * mi));
             p.aux_scalars[3] = mc == 0.0 ? 0.f : (float)(vc / (mc * mc));
         }
-    }
-    // the kept slots' token rows into x_perm, one slot per CTA at a time
-    const int nv = p.D / 8;
-    for (int i = blockIdx.x; i < TK; i += gridDim.x) {
-        const int r = tb.row[i];
-        if (r < 0) continue;
-        const uint4 *src = reinterpret_cast<const uint4 *>(p.x + (size_t)(i / p.K) * p.D);
-        uint4 *dst = reinterpret_cast<uint4 *>(p.x_perm + (size_t)r * p.D);
-        for (int v = tid; v < nv; v += kThreads) dst[v] = __ldg(src + v);
     }
 }
 
@@ -472,14 +475,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (ok && (int)blockIdx.x < p.T) route_r2(p, smem);
     if (ok) ok = grid_sync_all(p, 2, s_flag);
     if (ok) {
-        route_r3(p, tb, smem);
-        // x_perm written: release it to the grid (barrier 3 is waited on only
-        // by the producer, before its first token-row load)
-        __syncthreads();
-        if (threadIdx.x == 0) {
-            fence_proxy_async_global();
-            grid_arrive(p.bar);
-        }
+        route_r3(p, tb, smem);   // arrives at barrier 3 once its x_perm rows are written
     }
     __syncthreads();
 
@@ -495,6 +491,20 @@ __global__ void __launch_bounds__(kThreads, 1)
             int stage = 0;
             uint32_t phase = 0;
             IssuedSlots iss;
+            // weight rows of a piece: the first row of its 128-row tile (SwiGLU up: gate and up halves)
+            auto a_rows = [&](int ph, const PhaseWork &w, const dec::Piece &pc, int &wrow, int &wrow2) {
+                const int g = tb.live[pc.tile / w.tpg];
+                const int mt = pc.tile % w.tpg;
+                wrow2 = 0;
+                if (ph == 0 && swiglu) {
+                    wrow = g * 2 * H + mt * (BM / 2);
+                    wrow2 = wrow + H;
+                } else if (ph == 0) {
+                    wrow = g * H + mt * BM;
+                } else {
+                    wrow = g * D + mt * BM;
+                }
+            };
             for (int ph = 0; ph < 2 && ok; ++ph) {
                 const PhaseWork &w = ph == 0 ? wu : wd;
                 const CUtensorMap *mW = ph == 0 ? &tmW1 : &tmW2;
@@ -503,7 +513,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const unsigned target = (ph == 0 ? 3u : 1u) * gridDim.x;
                 bool ready = false;
                 int ndef = 0;
-                int def_stage[8], def_col[8], def_row[8];
+                int def_stage[kStages], def_col[kStages], def_row[kStages];
                 auto flush = [&]() {
                     fence_proxy_async_global();
                     for (int q = 0; q < ndef; ++q)
@@ -513,18 +523,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int64_t u = w.u_begin; u < w.u_end && ok;) {
                     const dec::Piece pc = w.piece(u);
                     u = w.next(u, pc);
-                    const int g = tb.live[pc.tile / w.tpg];
-                    const int mt = pc.tile % w.tpg;
-                    const int trow = tb.rowoff[g];
-                    int wrow, wrow2 = 0;
-                    if (ph == 0 && swiglu) {
-                        wrow = g * 2 * H + mt * (BM / 2);
-                        wrow2 = wrow + H;
-                    } else if (ph == 0) {
-                        wrow = g * H + mt * BM;
-                    } else {
-                        wrow = g * D + mt * BM;
-                    }
+                    const int trow = tb.rowoff[tb.live[pc.tile / w.tpg]];
+                    int wrow, wrow2;
+                    a_rows(ph, w, pc, wrow, wrow2);
                     for (int kb = pc.k0; kb < pc.k1; ++kb) {
                         if (!ready && ndef == kStages) {   // the ring holds only deferred stages: wait for the data
                             if (!grid_wait(bar, target, p.timeout_ns)) {
@@ -665,24 +666,35 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (et == 0) s_flag[1] = ticket_arrive(tickets + c_first) == (unsigned)(c_last - c_first);
                     if (!eb.sync()) { eok = false; break; }
                     if (!s_flag[1]) continue;
+                    // pieces added from the last CTA's down to the first's; the loads of
+                    // GC pieces are issued together (one round trip per group)
+                    constexpr int GC = NT >= 64 ? 1 : 64 / NT;
                     float sum[NT];
-                    for (int c = c_last; c >= c_first; --c) {
-                        if (c == (int)blockIdx.x) {
+                    for (int c0 = c_last; c0 >= c_first; c0 -= GC) {
+                        float v[GC][NT];
 #pragma unroll
-                            for (int j = 0; j < NT; ++j) sum[j] = c == c_last ? acc[j] : acc[j] + sum[j];
-                        } else {
-                            const float *src =
-                                p.part + ((int64_t)(c * 2 + (w.wk.begin(c) >= ts ? 0 : 1)) * BM + L) * NT;
+                        for (int gi = 0; gi < GC; ++gi) {
+                            const int c = c0 - gi;
+                            if (c < c_first) continue;
+                            if (c == (int)blockIdx.x) {
 #pragma unroll
-                            for (int j = 0; j < NT; j += 4) {
-                                const float4 v = __ldcg(reinterpret_cast<const float4 *>(src + j));
-                                if (c == c_last) {
-                                    sum[j] = v.x; sum[j + 1] = v.y; sum[j + 2] = v.z; sum[j + 3] = v.w;
-                                } else {
-                                    sum[j] = v.x + sum[j]; sum[j + 1] = v.y + sum[j + 1];
-                                    sum[j + 2] = v.z + sum[j + 2]; sum[j + 3] = v.w + sum[j + 3];
+                                for (int j = 0; j < NT; ++j) v[gi][j] = acc[j];
+                            } else {
+                                const float *src =
+                                    p.part + ((int64_t)(c * 2 + (w.wk.begin(c) >= ts ? 0 : 1)) * BM + L) * NT;
+#pragma unroll
+                                for (int j = 0; j < NT; j += 4) {
+                                    const float4 q4 = __ldcg(reinterpret_cast<const float4 *>(src + j));
+                                    v[gi][j] = q4.x; v[gi][j + 1] = q4.y; v[gi][j + 2] = q4.z; v[gi][j + 3] = q4.w;
                                 }
                             }
+                        }
+#pragma unroll
+                        for (int gi = 0; gi < GC; ++gi) {
+                            const int c = c0 - gi;
+                            if (c < c_first) continue;
+#pragma unroll
+                            for (int j = 0; j < NT; ++j) sum[j] = c == c_last ? v[gi][j] : v[gi][j] + sum[j];
                         }
                     }
 #pragma unroll
@@ -778,8 +790,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         // ---- the combine: once every CTA's z rows are written (barrier 5), the epilogue
         // threads of all CTAs share y: y[t, d] = z[t K, d] + ... + z[t K + K - 1, d] in slot
-        // order over the kept slots; four outputs per thread and up to eight slots each have
-        // their loads in flight together
+        // order over the kept slots; two outputs per thread and four slots each have their
+        // loads in flight together
         if (eok && eb.sync()) {
             if (et == 0) {
                 __threadfence();
@@ -787,44 +799,40 @@ __global__ void __launch_bounds__(kThreads, 1)
                 s_flag[1] = grid_wait(p.bar5, gridDim.x, p.timeout_ns) ? 1 : 0;
             }
             if (eb.sync() && s_flag[1]) {
+                // compact code: this runs once per launch, so its instructions are fetched cold
                 const int K = p.K;
-                const int64_t O = (int64_t)p.T * D;
-                const int64_t stride = (int64_t)gridDim.x * 128;
-                for (int64_t o0 = (int64_t)blockIdx.x * 128 + et; o0 < O; o0 += 4 * stride) {
-                    float acc[4];
-                    bool any[4];
+                const int O = p.T * D;
+                const int stride = (int)gridDim.x * 128;
+                for (int o0 = (int)blockIdx.x * 128 + et; o0 < O; o0 += 2 * stride) {
+                    float acc[2] = {0.f, 0.f};
+                    bool any[2] = {false, false};
+                    for (int j0 = 0; j0 < K; j0 += 4) {
+                        float v[2][4];
+                        bool h[2][4];
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        acc[q] = 0.f;
-                        any[q] = false;
-                    }
-                    for (int jb = 0; jb < K; jb += 8) {
-                        float v[4][8];
-                        bool has[4][8];
+                        for (int q = 0; q < 2; ++q) {
+                            const int o = o0 + q * stride;
+                            const int t = o < O ? o / D : 0;
+                            const float *zt = p.z + (size_t)t * K * D + (o - t * D);
 #pragma unroll
-                        for (int q = 0; q < 4; ++q) {
-                            const int64_t o = o0 + q * stride;
-                            const int64_t t = o < O ? o / D : 0;
-                            const int64_t d = o - t * D;
-#pragma unroll
-                            for (int u = 0; u < 8; ++u) {
-                                const int j = jb + u;
-                                has[q][u] = o < O && j < K && tb.row[t * K + j] >= 0;   // dropped by the capacity
-                                v[q][u] = has[q][u] ? __ldcg(p.z + (t * K + j) * D + d) : 0.f;
+                            for (int u = 0; u < 4; ++u) {
+                                const int j = j0 + u;
+                                h[q][u] = o < O && j < K && tb.row[t * K + j] >= 0;   // dropped by the capacity
+                                v[q][u] = h[q][u] ? __ldcg(zt + (size_t)j * D) : 0.f;
                             }
                         }
 #pragma unroll
-                        for (int q = 0; q < 4; ++q)
+                        for (int q = 0; q < 2; ++q)
 #pragma unroll
-                            for (int u = 0; u < 8; ++u)
-                                if (has[q][u]) {
+                            for (int u = 0; u < 4; ++u)
+                                if (h[q][u]) {
                                     acc[q] = any[q] ? acc[q] + v[q][u] : v[q][u];
                                     any[q] = true;
                                 }
                     }
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        const int64_t o = o0 + q * stride;
+                    for (int q = 0; q < 2; ++q) {
+                        const int o = o0 + q * stride;
                         if (o >= O) continue;
                         if (p.y_bf16) static_cast<__nv_bfloat16 *>(p.y)[o] = __float2bfloat16_rn(acc[q]);
                         else static_cast<float *>(p.y)[o] = acc[q];
