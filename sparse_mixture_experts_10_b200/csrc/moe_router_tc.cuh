@@ -95,27 +95,33 @@ struct __align__(16) FinalScratch {
 // totals and the exclusive scan that gives each tile's first row.
 // At most 256 threads work (the scratch arrays' size); larger blocks' other
 // threads only take part in the barriers.
-__device__ void finalize_tables(const Params &p, int ntiles, FinalScratch &f, int *cnt_smem, int cap) {
+__device__ __forceinline__ void finalize_tables(const Params &p, int ntiles, FinalScratch &f, int *cnt_smem, int cap) {
     const int N = p.N, tid = threadIdx.x;
     const int nt = blockDim.x < 256 ? (int)blockDim.x : 256;
     const bool worker = tid < nt;
     const int warp = tid >> 5, lane = tid & 31;
     const bool in_smem = cnt_smem != nullptr && (int64_t)ntiles * N <= cap;
     if (in_smem) {
+        // 16-byte loads, eight in flight per thread (the matrix starts 16-byte aligned)
         const int total = ntiles * N;
-        for (int i0 = tid; worker && i0 < total; i0 += 8 * nt) {
-            int v[8];
+        const int total4 = total / 4;
+        const int4 *src4 = reinterpret_cast<const int4 *>(p.tile_counts);
+        int4 *dst4 = reinterpret_cast<int4 *>(cnt_smem);
+        for (int i0 = tid; worker && i0 < total4; i0 += 8 * nt) {
+            int4 v[8];
 #pragma unroll
-            for (int k = 0; k < 8; ++k) v[k] = i0 + k * nt < total ? __ldcg(p.tile_counts + i0 + k * nt) : 0;
+            for (int k = 0; k < 8; ++k) v[k] = i0 + k * nt < total4 ? __ldcg(src4 + i0 + k * nt) : make_int4(0, 0, 0, 0);
 #pragma unroll
             for (int k = 0; k < 8; ++k)
-                if (i0 + k * nt < total) cnt_smem[i0 + k * nt] = v[k];
+                if (i0 + k * nt < total4) dst4[i0 + k * nt] = v[k];
         }
+        for (int i = total4 * 4 + tid; worker && i < total; i += nt) cnt_smem[i] = __ldcg(p.tile_counts + i);
         __syncthreads();
     }
-    auto count_at = [&](int c, int e) -> int {
-        return in_smem ? cnt_smem[c * N + e] : __ldcg(p.tile_counts + (int64_t)c * N + e);
-    };
+    // one pointer for both cases (generic loads reach shared or global memory), so the
+    // loops below hold no per-element choice between two kinds of load
+    const int *cm = in_smem ? cnt_smem : p.tile_counts;
+    auto count_at = [&](int c, int e) -> int { return cm[(int64_t)c * N + e]; };
     int Q = nt / N;
     Q = Q < 1 ? 1 : (Q > 32 ? 32 : Q);
     const int epp = nt / Q;                       // experts per pass
@@ -267,6 +273,8 @@ struct Shape {
     static constexpr int kStages0 = (160 * 1024) / (int)kStageBytes;
     static constexpr int kStages = kStages0 > 8 ? 8 : kStages0;
     static constexpr uint32_t kTmemCols = NP <= 32 ? 32 : NP <= 64 ? 64 : NP <= 128 ? 128 : 256;
+    // the epilogue's score tile [BM][NP + 1] and 1/z per row reuse the ring
+    static_assert((size_t)BM * (NP + 1) * 4 + BM * 4 <= (size_t)kStages * kStageBytes, "score tile exceeds the ring");
     // ring + per-warp probability rows + tile counters + finalisation scratch + barriers
     static constexpr size_t kSmem = 1024 + (size_t)kStages * kStageBytes + 4 * 256 * 4 + 256 * 4 + 256 * 8 +
                                     sizeof(FinalScratch) + (2 * kStages + 2) * 8 + 64;
@@ -305,45 +313,6 @@ __device__ __forceinline__ float score(const float *bg, float acc, int e) {
     return s;
 }
 
-// Visit the N logits of this thread's token in ascending expert order, 32 (or
-// 16) TMEM columns at a time.  f(e, s) is called for e < N.
-template <int NP, typename F>
-__device__ __forceinline__ void for_each_logit(const Params &p, uint32_t tlane, F &&f) {
-#pragma unroll 1
-    for (int c = 0; c < NP; c += 32) {
-        float v[32];
-        if (NP - c >= 32) ld_cols32(tlane + c, v);
-        else ld_cols16(tlane + c, v);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-            const int e = c + i;
-            if (e < p.N && (NP - c >= 32 || i < 16)) f(e, score(p.bg, v[i], e));
-        }
-    }
-}
-
-// Keep (v, e) with its raw score r in the best-first list (tv, te, tr) of length
-// KM if it belongs there: larger selection value first, equal values in
-// ascending expert index.
-template <int KM>
-__device__ __forceinline__ void topk_insert(float (&tv)[KM], int (&te)[KM], float (&tr)[KM], float s, int e, float r) {
-    if (!(s > tv[KM - 1] || (s == tv[KM - 1] && e < te[KM - 1]))) return;
-    float cv = s, cr = r;
-    int ce = e;
-#pragma unroll
-    for (int j = 0; j < KM; ++j) {
-        const bool better = cv > tv[j] || (cv == tv[j] && ce < te[j]);
-        const float ov = tv[j], orw = tr[j];
-        const int oe = te[j];
-        tv[j] = better ? cv : ov;
-        tr[j] = better ? cr : orw;
-        te[j] = better ? ce : oe;
-        cv = better ? ov : cv;
-        cr = better ? orw : cr;
-        ce = better ? oe : ce;
-    }
-}
-
 template <int NP, int KM>
 __global__ void __launch_bounds__(kThreads, 1)
     router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
@@ -352,10 +321,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     using S = Shape<NP>;
     constexpr int kStages = S::kStages;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
-    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *smem = align_smem_1024(smem_raw);
     uint8_t *sA = smem;
     uint8_t *sB = smem + kStages * S::kABytes;
-    float *s_wp = reinterpret_cast<float *>(sB + kStages * S::kBBytes);                  // [4][256]
+    float *s_wp = reinterpret_cast<float *>(sB + kStages * S::kBBytes);                  // [256] (of [4][256])
     int *s_cnt = reinterpret_cast<int *>(s_wp + 4 * 256);                                 // [256]
     unsigned long long *s_imp = reinterpret_cast<unsigned long long *>(s_cnt + 256);      // [256]
     FinalScratch *fs = reinterpret_cast<FinalScratch *>(s_imp + 256);
@@ -443,26 +412,78 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else {
         // ------------------------------------------------------------ one token per thread
-        // warp w may only read TMEM lanes 32*(w%4)..+31, which fixes the rows it owns
+        // warp w may only read TMEM lanes 32*(w%4)..+31, which fixes the rows it owns.
+        // The scores go through a padded [BM][NP + 1] fp32 tile in the ring (free once
+        // the MMAs are complete): coalesced logits rows, conflict-free row scans for the
+        // top-k, and per-expert column sums over the tile's tokens in token order.
         const int ew = warp & 3;
         const int r = ew * 32 + lane;            // row of the tile = TMEM lane
         const int t = tile * BM + r;
         const bool live_row = t < p.T;
+        constexpr int LD = NP + 1;
+        float *S = reinterpret_cast<float *>(smem);   // [BM][LD]
+        float *inv_z_s = S + BM * LD;                  // [BM]
         const bool have = __all_sync(0xffffffffu, mbar_wait(tfull, 0, p.timeout_ns));   // warp-uniform
         tc_fence_after();
+        float smax = -INFINITY;
         if (have) {
             const uint32_t tlane = tmem_base + (static_cast<uint32_t>(ew * 32) << 16);
-            // pass 1: logits out, top-K on the selection values, the largest raw score
-            float tv[KM], tr[KM];
+            float *row = S + r * LD;
+            bool nan_seen = false;
+#pragma unroll 1
+            for (int c = 0; c < NP; c += 32) {
+                float v[32];
+                if (NP - c >= 32) ld_cols32(tlane + c, v);
+                else ld_cols16(tlane + c, v);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const int e = c + i;
+                    if (e < p.N && (NP - c >= 32 || i < 16)) {
+                        float sc = v[i] + (p.bg ? __ldg(p.bg + e) : 0.f);
+                        nan_seen |= sc != sc;
+                        sc = sc != sc ? -INFINITY : sc;   // NaN ranked as -inf (flagged below)
+                        row[e] = sc;
+                        smax = fmaxf(smax, sc);
+                    }
+                }
+            }
+            if (nan_seen) set_status(kStatusNanLogit);
+            __syncwarp();
+            // logits: this warp's 32 rows, each stored by the whole warp (coalesced)
+            for (int rr = 0; rr < 32; ++rr) {
+                const int tt = tile * BM + ew * 32 + rr;
+                if (tt >= p.T) break;
+                const float *src = S + (ew * 32 + rr) * LD;
+                for (int e = lane; e < p.N; e += 32) p.logits[(int64_t)tt * p.N + e] = src[e];
+            }
+            // top-K of the selection values, best first (larger value, then lower index):
+            // each expert as one 64-bit key, the value's order-preserving bits above the
+            // complemented index, entering the sorted key list with all positions compared
+            // at once (selects only); the raw scores are read back for the kept experts
+            unsigned long long tk[KM];
+#pragma unroll
+            for (int j = 0; j < KM; ++j) tk[j] = 0ull;   // below every real key (NaN became -inf)
+            for (int e = 0; e < p.N; ++e) {
+                const float sv = p.bsel ? row[e] + __ldg(p.bsel + e) : row[e];
+                const uint32_t u = __float_as_uint(sv);
+                const uint32_t o = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+                const unsigned long long k = ((unsigned long long)o << 32) | (uint32_t)~e;
+                bool b[KM];
+#pragma unroll
+                for (int j = 0; j < KM; ++j) b[j] = k > tk[j];
+#pragma unroll
+                for (int j = KM - 1; j >= 0; --j) {
+                    const unsigned long long nk = (j > 0 && b[j - 1]) ? tk[j - 1] : k;
+                    tk[j] = b[j] ? nk : tk[j];
+                }
+            }
+            float tr[KM];
             int te[KM];
 #pragma unroll
-            for (int j = 0; j < KM; ++j) { tv[j] = tr[j] = -INFINITY; te[j] = 0x7fffffff; }
-            float smax = -INFINITY;
-            for_each_logit<NP>(p, tlane, [&](int e, float s) {
-                if (live_row) p.logits[(int64_t)t * p.N + e] = s;
-                topk_insert<KM>(tv, te, tr, p.bsel ? s + __ldg(p.bsel + e) : s, e, s);
-                smax = fmaxf(smax, s);
-            });
+            for (int j = 0; j < KM; ++j) {
+                te[j] = (int)~(uint32_t)tk[j];
+                tr[j] = j < p.K ? row[te[j]] : -INFINITY;
+            }
             // gate weights: softmax over the K kept raw scores, shifted by their largest
             // (slot 0's without a selection bias), slot order
             float kmax = -INFINITY;
@@ -487,26 +508,31 @@ __global__ void __launch_bounds__(kThreads, 1)
                     atomicAdd(&s_imp[te[j]], (unsigned long long)__double2ull_rn((double)wj * kImpScale));
                 }
             }
-            // pass 2: normaliser of the full softmax of the raw scores
-            const float m = smax;
+            // the full softmax of the raw scores: exponentials in place, the normaliser
             float z = 0.f;
-            for_each_logit<NP>(p, tlane, [&](int e, float s) { z += expf(s - m); });
-            const float inv_z = live_row ? 1.0f / z : 0.f;
-            // pass 3: per-expert probability sums over the tile: lanes (xor tree), then warps (below)
-            for_each_logit<NP>(p, tlane, [&](int e, float s) {
-                float pe = expf(s - m) * inv_z;
-#pragma unroll
-                for (int o = 16; o >= 1; o >>= 1) pe += __shfl_xor_sync(0xffffffffu, pe, o);
-                if (lane == 0) s_wp[ew * 256 + e] = pe;
-            });
+            for (int e = 0; e < p.N; ++e) {
+                const float x = expf(row[e] - smax);
+                row[e] = x;
+                z += x;
+            }
+            inv_z_s[r] = live_row ? 1.0f / z : 0.f;
+        }
+        // per-expert probability sums over the tile's tokens, rows ascending (the four
+        // epilogue warps meet on named barrier 1)
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        if (__all_sync(0xffffffffu, have)) {
+            const int et = threadIdx.x - 64;
+            for (int e = et; e < p.N; e += 128) {
+                float ps = 0.f;
+                for (int rr = 0; rr < BM; ++rr) ps = fmaf(S[rr * LD + e], inv_z_s[rr], ps);
+                s_wp[e] = ps;
+            }
         }
     }
     tc_fence_before();
     __syncthreads();
     for (int e = threadIdx.x; e < p.N; e += blockDim.x) {
-        float ps = 0.f;
-        for (int w = 0; w < 4; ++w) ps += s_wp[w * 256 + e];
-        atomicAdd(p.sum_p + e, __double2ull_rn((double)ps * kImpScale));
+        atomicAdd(p.sum_p + e, __double2ull_rn((double)s_wp[e] * kImpScale));
         atomicAdd(p.sum_imp + e, s_imp[e]);
         p.tile_counts[(int64_t)tile * p.N + e] = s_cnt[e];
     }
@@ -963,7 +989,7 @@ __global__ void __launch_bounds__(256) router_few_kernel(const __nv_bfloat16 *__
     pdl_enter();
     __shared__ float part[8][32];
     __shared__ FinalScratch fs;
-    __shared__ int s_cnt[kFewMaxT * 32];   // the count matrix in the finalisation
+    __shared__ __align__(16) int s_cnt[kFewMaxT * 32];   // the count matrix in the finalisation (16-byte loads)
     __shared__ int s_flag;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int t = blockIdx.x, sl = blockIdx.y, S = gridDim.y, N = p.N, D = p.D;
