@@ -103,8 +103,9 @@ def parse(argv=None):
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
-    ap.add_argument("--mode", default="forward", choices=["forward", "backward"],
-                    help="backward: time the layer's backward pass (moe_backward) instead")
+    ap.add_argument("--mode", default="forward", choices=["forward", "backward", "route"],
+                    help="backward: time the layer's backward pass (moe_backward) instead; route: the "
+                         "routing stage alone (moe_route)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle sample")
     ap.add_argument("--ref-seconds", type=float, default=150.0,
@@ -542,6 +543,68 @@ def run_backward(args, wl):
     print(json.dumps(line), flush=True)
 
 
+def run_route(args, wl):
+    """Time moe_route alone (graph-captured, L2 flushed before every step) on one GPU: scores,
+    top-k, gate weights, statistics and dispatch tables, with only x and W_g allocated."""
+    import sparse_mixture_experts_10_b200 as moe
+    from sparse_mixture_experts_10_b200 import build as moe_build
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    moe_build.build()
+    moe.load_library()
+    T = wl.T
+    gen = torch.Generator(device=dev).manual_seed(wl.seed)
+    x = torch.randn(T, wl.D, device=dev, generator=gen).to(wl.dtype)
+    Wg = (torch.randn(wl.D, wl.N, device=dev, generator=gen) * wl.w_std).to(wl.dtype)
+    cfg = moe.make_config(wl.D, wl.H, wl.N, wl.K, wl.act, moe.dtype_code(wl.dtype), wl.has_bias)
+    W = moe.make_weights(Wg, None, None)
+    ws = moe.alloc_workspace(cfg, T)
+    logits = torch.empty(T, wl.N, device=dev)
+    idx = torch.empty(T, wl.K, dtype=torch.int32, device=dev)
+    tw = torch.empty(T, wl.K, device=dev)
+    counts = torch.empty(wl.N, dtype=torch.int32, device=dev)
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+
+    def step():
+        moe.check(moe.moe_route(cfg, x, T, W, logits, idx, tw, counts, ws, ws.numel()), "route")
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        step()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    sampler = ClockSampler(0)
+    sampler.start()
+    for a, b in ev:
+        flush.zero_()
+        a.record()
+        graph.replay()
+        b.record()
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    st = moe.moe_get_device_status()
+    if st != 0:
+        raise RuntimeError(f"device status {st}")
+    ms = float(np.mean([a.elapsed_time(b) for a, b in ev]))
+    es = 2 if wl.dtype == torch.bfloat16 else 4
+    # algorithmic bytes: x and W_g read, logits, top-k indices and weights written
+    nbytes = T * wl.D * es + wl.D * wl.N * es + T * wl.N * 4 + T * wl.K * 8
+    pk, pk_kind = peaks()
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    line = {"metric": METRIC + " (routing stage)", "value": T / (ms * 1e-3), "unit": "tokens/s", "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "dtype": "bf16" if wl.dtype == torch.bfloat16 else "f32", "data": "synthetic",
+            "config": config_dict(wl, T, 1) | {"mode": "route"},
+            "roofline": {"bound": "hbm", "unit": "GB/s", "achieved": gbs, "peak": float(pk["hbm_gbs"]),
+                         "peak_kind": f"{pk_kind} copy", "frac": gbs / float(pk["hbm_gbs"]),
+                         "bytes_per_step": nbytes},
+            "clocks": clocks}
+    print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse()
     wl = workload_from_args(args)
@@ -550,6 +613,9 @@ def main():
         return
     if args.mode == "backward":
         run_backward(args, wl)
+        return
+    if args.mode == "route":
+        run_route(args, wl)
         return
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
