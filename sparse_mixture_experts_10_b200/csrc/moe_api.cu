@@ -730,8 +730,9 @@ int stage_scan(const Plan &P, const Bufs &b, int *counts_out, cudaStream_t s, in
 int stage_permute(const Plan &P, const Bufs &b, const void *x, float *y_zero, const DeviceInfo &dev,
                   cudaStream_t s) {
     const size_t smem = (size_t)(2 * P.N + P.chunk_tokens * P.K) * 4;
-    // enough blocks to keep every SM copying: split each chunk's rows over several blocks
-    const int split = (int)std::max<int64_t>(1, std::min<int64_t>(8, cdiv(2 * dev.sms, P.n_chunks)));
+    // enough blocks to keep every SM copying with many rows in flight: split each
+    // chunk's rows over up to eight blocks, aiming at eight blocks per SM
+    const int split = (int)std::max<int64_t>(1, std::min<int64_t>(8, cdiv(8 * dev.sms, P.n_chunks)));
     const dim3 grid((unsigned)P.n_chunks, (unsigned)split);
     if (P.dtype == MOE_F32)
         return launch_pdl(permute_kernel<float>, grid, dim3(256), smem, s, static_cast<const float *>(x), (int)P.T, P.D,

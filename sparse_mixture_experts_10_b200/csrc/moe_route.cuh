@@ -796,15 +796,17 @@ __global__ void __launch_bounds__(256) permute_kernel(const Tin *__restrict__ x,
     const int n_tok = t_end - t_begin;
     constexpr int VEC = 16 / sizeof(Tin);
     const int nvec = D / VEC;
-    // loads that do not wait for the ranking go out first: warp 0's first 32
-    // entries and each warp's first token's first 128 slices
-    const int e_pre = warp == 0 && lane < n_entries ? topk_idx[f0 + lane] : -1;
+    // loads that do not wait for the ranking go out first: the chunk's expert
+    // indices (all threads, into s_dest, one round trip) and each warp's first
+    // token's first 128 slices
+    for (int f = tid; f < n_entries; f += blockDim.x) s_dest[f] = topk_idx[f0 + f];
     const int tt_first = blockIdx.y + gridDim.y * warp;
-    uint4 pre[4];
+    constexpr int kInFlight = 4;    // 16-byte slices per lane in flight
+    uint4 pre[kInFlight];
     if (tt_first < n_tok) {
         const uint4 *src = reinterpret_cast<const uint4 *>(x + (int64_t)(t_begin + tt_first) * D);
 #pragma unroll
-        for (int u = 0; u < 4; ++u)
+        for (int u = 0; u < kInFlight; ++u)
             if (lane + 32 * u < nvec) pre[u] = __ldg(src + lane + 32 * u);
     }
     for (int e = tid; e < N; e += blockDim.x) {
@@ -815,7 +817,7 @@ __global__ void __launch_bounds__(256) permute_kernel(const Tin *__restrict__ x,
     if (warp == 0) {
         for (int base = 0; base < n_entries; base += 32) {
             const int f = base + lane;
-            int e = f < n_entries ? (base == 0 ? e_pre : topk_idx[f0 + f]) : -1;
+            int e = f < n_entries ? s_dest[f] : -1;   // overwritten by its destination below
             if (f < n_entries && (e < 0 || e >= N)) {
                 set_status(kStatusBounds);
                 e = -1;
@@ -847,18 +849,18 @@ __global__ void __launch_bounds__(256) permute_kernel(const Tin *__restrict__ x,
     for (int tt = tt_first; tt < n_tok; tt += 8 * gridDim.y) {
         const uint4 *src = reinterpret_cast<const uint4 *>(x + (int64_t)(t_begin + tt) * D);
         const int *dest = s_dest + tt * K;
-        for (int v0 = lane; v0 < nvec; v0 += 128) {
-            uint4 r[4];
+        for (int v0 = lane; v0 < nvec; v0 += 32 * kInFlight) {
+            uint4 r[kInFlight];
             const bool prefetched = tt == tt_first && v0 == lane;
 #pragma unroll
-            for (int u = 0; u < 4; ++u)
+            for (int u = 0; u < kInFlight; ++u)
                 if (v0 + 32 * u < nvec) r[u] = prefetched ? pre[u] : __ldg(src + v0 + 32 * u);
             for (int j = 0; j < K; ++j) {
                 const int d = dest[j];
                 if (d < 0) continue;
                 uint4 *dst = reinterpret_cast<uint4 *>(x_perm + (int64_t)d * D);
 #pragma unroll
-                for (int u = 0; u < 4; ++u)
+                for (int u = 0; u < kInFlight; ++u)
                     if (v0 + 32 * u < nvec) dst[v0 + 32 * u] = r[u];
             }
         }
