@@ -209,6 +209,13 @@ def config_dict(wl, T, world):
     return d
 
 
+def fused_decode(wl, T):
+    """Whether the library runs this layer as its one-kernel decode path: bf16, at most 64
+    tokens and 32 experts, no shared expert, no reroute."""
+    return (wl.dtype == torch.bfloat16 and 0 < T <= 64 and wl.N <= 32 and not wl.n_shared and
+            not (wl.capacity_factor > 0 and wl.overflow))
+
+
 def gemm_peak(pk, step_ms):
     """(peak TFLOP/s, its name): the sustained figure for kernels inside long steps, else the burst one."""
     if step_ms > SUSTAINED_STEP_MS and "bf16_tflops_sustained" in pk:
@@ -779,9 +786,13 @@ def main():
     else:
         byt = {"route": wm["route_bytes"], "permute": wm["permute_bytes"], "combine": wm["combine_bytes"],
                "up": wm["up_weight_bytes"], "down": wm["down_weight_bytes"]}.get(names[dom], 0)
+        kname = names[dom]
+        if fused_decode(wl, T) and names[dom] == "up":
+            # the whole layer is one kernel between the "up" events: all of its bytes count
+            byt, kname = wm["decode_bytes"], "decode_layer_kernel (whole layer, one launch)"
         achieved = byt / (dom_mean_ms * 1e-3) / 1e9
         peak = float(pk["hbm_gbs"])
-        roof = {"kernel": names[dom], "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+        roof = {"kernel": kname, "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                 "frac": achieved / peak, "peak_kind": f"{pk_kind} copy",
                 "spec_peak": SPEC_PEAKS["hbm_gbs"], "frac_vs_spec": achieved / SPEC_PEAKS["hbm_gbs"]}
     roof["ms"] = dom_mean_ms
