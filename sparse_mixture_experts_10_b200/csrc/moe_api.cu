@@ -839,6 +839,19 @@ bool narrow_tiles(const Plan &P, int64_t n_tiles_256, const DeviceInfo &dev) {
 // (256 x 512).
 bool tail_split(const Plan &P) { return 64.0 * P.N > 0.1 * (double)(P.T * P.K); }
 
+// With the tail split, the SMs are divided between the two kernels from the
+// start so that both walk the experts at about the same pace (the tail tiles
+// then find their expert's weights still in L2): the tail kernel's share is
+// its expected work, about N/2 odd blocks of 128 rows at 1.3 times a pair
+// tile's cost per SM, against the pair units of the rest.
+int tail_sms(const Plan &P, const DeviceInfo &dev) {
+    const double blocks = (double)(P.T * P.K) / 128.0 + 0.5 * P.N;
+    const double tails = 0.5 * P.N, pairs = std::max(1.0, (blocks - tails) / 2.0);
+    const double share = 1.3 * tails / (2.0 * pairs + 1.3 * tails);
+    const int n = (int)(share * dev.sms + 0.5) & ~1;
+    return std::max(2, std::min(dev.sms / 2, n));
+}
+
 int stage_up(const Plan &P, const Bufs &b, const moe_weights *w, const DeviceInfo &dev, cudaStream_t s) {
     if (P.decode) return stage_up_decode(P, b, w, dev, s);
     const int D = P.D, H = P.H, N = P.N;
@@ -876,16 +889,18 @@ int stage_up(const Plan &P, const Bufs &b, const moe_weights *w, const DeviceInf
             return launch_tc2<tc::EPI_GELU>(ma, mb, mo, p, units, dev.pair_clusters, s);
         }
         p.tail_mode = 1;
-        if (swiglu) MOE_TRY(launch_tc2<tc::EPI_SWIGLU>(ma, mb, mo, p, units, dev.pair_clusters, s));
-        else MOE_TRY(launch_tc2<tc::EPI_GELU>(ma, mb, mo, p, units, dev.pair_clusters, s));
+        const int tsm = tail_sms(P, dev);
+        const int pcl = std::max(1, dev.pair_clusters - tsm / 2);
+        if (swiglu) MOE_TRY(launch_tc2<tc::EPI_SWIGLU>(ma, mb, mo, p, units, pcl, s));
+        else MOE_TRY(launch_tc2<tc::EPI_GELU>(ma, mb, mo, p, units, pcl, s));
         // the tail tiles are 128 x 256 (SwiGLU: 128 gate + 128 up rows of W1,
         // the pair kernel's B box; GELU: one 256-row box)
         tc::Params pt = p;
         pt.tail_mode = 2;
         CUtensorMap mbt = mb;
         if (!swiglu) MOE_TRY(make_map(&mbt, w->W1, (int64_t)N * H, D, 256));
-        if (swiglu) return launch_tc<256, tc::EPI_SWIGLU>(ma, mbt, mo, pt, (int64_t)N * pt.n_tiles, dev.sms, s);
-        return launch_tc<256, tc::EPI_GELU>(ma, mbt, mo, pt, (int64_t)N * pt.n_tiles, dev.sms, s);
+        if (swiglu) return launch_tc<256, tc::EPI_SWIGLU>(ma, mbt, mo, pt, (int64_t)N * pt.n_tiles, tsm, s);
+        return launch_tc<256, tc::EPI_GELU>(ma, mbt, mo, pt, (int64_t)N * pt.n_tiles, tsm, s);
     }
     simt::Params p{};
     p.A = b.at<float>(P.x_perm);
@@ -950,13 +965,14 @@ int stage_down(const Plan &P, const Bufs &b, const moe_weights *w, void *y, int 
             return launch_tc2<tc::EPI_SCATTER>(ma, mb, mo, p, (P.rows_cap / (2 * tc::BM) + N) * p.n_tiles,
                                                dev.pair_clusters, s);
         p.tail_mode = 1;
+        const int tsm = tail_sms(P, dev);
         MOE_TRY(launch_tc2<tc::EPI_SCATTER>(ma, mb, mo, p, (P.rows_cap / (2 * tc::BM) + N) * p.n_tiles,
-                                            dev.pair_clusters, s));
+                                            std::max(1, dev.pair_clusters - tsm / 2), s));
         tc::Params pt = p;
         pt.tail_mode = 2;
         CUtensorMap mbt;
         MOE_TRY(make_map(&mbt, w->W2, (int64_t)N * D, H, 256));
-        return launch_tc<256, tc::EPI_SCATTER>(ma, mbt, mo, pt, (int64_t)N * pt.n_tiles, dev.sms, s);
+        return launch_tc<256, tc::EPI_SCATTER>(ma, mbt, mo, pt, (int64_t)N * pt.n_tiles, tsm, s);
     }
     simt::Params p{};
     p.A = b.at<float>(P.h);
