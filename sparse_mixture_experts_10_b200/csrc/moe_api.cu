@@ -1206,13 +1206,17 @@ int zero_aux(const Plan &P, moe_aux *aux, cudaStream_t s) {
 std::atomic<bool> g_fused_pdl{true};
 
 // Routing scratch of the fused decode kernel, in its ring: R1 x rows and the
-// W_g slab; R2 the slabs' scores of one token; R3 top-k experts,
+// W_g slab; R2 (every token's slab sums for few tokens, after R3's arrays) the slabs' scores of one token; R3 top-k experts,
 // ranks, gate weights and full softmax.
 size_t fused_scratch(int T, int slab_rows, int n_slabs) {
     const size_t r1 = ((size_t)T * slab_rows + (size_t)slab_rows * 32) * 4;
     const size_t r2 = (size_t)n_slabs * 32 * 4;
     const size_t r3 = ((size_t)3 * dfu::kMaxSlots + (size_t)T * 32) * 4;
-    return std::max(r1, std::max(r2, r3));
+    // R2 in every CTA for few tokens: the slab sums of all tokens after R3's arrays
+    const size_t r2a = T <= dfu::kAllR2T ? ((size_t)3 * dfu::kMaxSlots + (size_t)dfu::kMaxT * 32) * 4 +
+                                               (size_t)n_slabs * T * 32 * 4
+                                         : 0;
+    return std::max(std::max(r1, r2a), std::max(r2, r3));
 }
 
 template <int NT, int EPI>

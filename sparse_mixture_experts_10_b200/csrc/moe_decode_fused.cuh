@@ -195,34 +195,35 @@ __device__ __forceinline__ void route_r1(const Params &p, uint8_t *scratch) {
     }
 }
 
-// R2 for token t = blockIdx.x: every thread of the CTA loads the slabs' scores
-// into shared memory at once (one round trip), warp 0 adds them in slab order.
-__device__ __forceinline__ void route_r2(const Params &p, uint8_t *scratch) {
-    const int tid = threadIdx.x, lane = tid & 31;
-    const int t = blockIdx.x, N = p.N, K = p.K;
-    float *sl = reinterpret_cast<float *>(scratch);   // [n_slabs][32]
-    for (int i = tid; i < p.n_slabs * 32; i += kThreads)
-        sl[i] = __ldcg(p.slab + ((size_t)(i >> 5) * p.T + t) * 32 + (i & 31));
-    __syncthreads();
-    if (tid >= 32) return;
+// R2 for token t by one warp: the slabs' scores sl[c * ld + lane] (c < n_slabs)
+// added in slab order, bias, NaN ranked as -inf, the top k (ties to the lower
+// index) on the selection values, gate weights, the full softmax.  With out the
+// results go to the workspace (logits, topk_idx, topk_w, tok_p); with s_idx the
+// selected experts also go there (shared memory, read by R3).
+__device__ __forceinline__ void r2_token(const Params &p, int t, const float *sl, int ld, bool out, int *s_idx) {
+    const int lane = threadIdx.x & 31;
+    const int N = p.N, K = p.K;
     const bool live = lane < N;
     float s = 0.f;
-    for (int c = 0; c < p.n_slabs; ++c) s += sl[c * 32 + lane];   // slab order
+    for (int c = 0; c < p.n_slabs; ++c) s += sl[c * ld + lane];   // slab order
     if (live) {
         if (p.bg) s += __ldg(p.bg + lane);
         if (s != s) {
             set_status(kStatusNanLogit);
             s = -INFINITY;
         }
-        p.logits[(size_t)t * N + lane] = s;
+        if (out) p.logits[(size_t)t * N + lane] = s;
     } else {
         s = -INFINITY;
     }
     int slot_e;
     float slot_w;
     if (segment_topk<32>(sel_value(p.bsel, s, lane, live), s, lane, !live, K, lane, lane, slot_e, slot_w)) {
-        p.topk_idx[(size_t)t * K + lane] = slot_e;
-        p.topk_w[(size_t)t * K + lane] = slot_w;
+        if (out) {
+            p.topk_idx[(size_t)t * K + lane] = slot_e;
+            p.topk_w[(size_t)t * K + lane] = slot_w;
+        }
+        if (s_idx) s_idx[t * K + lane] = slot_e;
     }
     float mx = s;
 #pragma unroll
@@ -231,17 +232,46 @@ __device__ __forceinline__ void route_r2(const Params &p, uint8_t *scratch) {
     float zs = ex;
 #pragma unroll
     for (int o = 16; o >= 1; o >>= 1) zs += __shfl_xor_sync(0xffffffffu, zs, o);
-    p.tok_p[(size_t)t * 32 + lane] = zs > 0.f ? ex / zs : 0.f;
+    if (out) p.tok_p[(size_t)t * 32 + lane] = zs > 0.f ? ex / zs : 0.f;
+}
+
+// R2 for token t = blockIdx.x: every thread of the CTA loads the slabs' scores
+// into shared memory at once (one round trip), warp 0 finishes the token.
+__device__ __forceinline__ void route_r2(const Params &p, uint8_t *scratch) {
+    const int tid = threadIdx.x;
+    const int t = blockIdx.x;
+    float *sl = reinterpret_cast<float *>(scratch);   // [n_slabs][32]
+    for (int i = tid; i < p.n_slabs * 32; i += kThreads)
+        sl[i] = __ldcg(p.slab + ((size_t)(i >> 5) * p.T + t) * 32 + (i & 31));
+    __syncthreads();
+    if (tid < 32) r2_token(p, t, sl, 32, true, nullptr);
+}
+
+// R2 for every token in every CTA (few tokens): all slabs' scores loaded at once,
+// each warp finishes tokens warp, warp + 6, ...; the selected experts land in
+// R3's index array, CTA 0 also writes the workspace.  Replaces R2 and the grid
+// barrier after it: every CTA derives the same tables from the same sums.
+constexpr int kAllR2T = 12;   // up to two tokens per warp
+__device__ __forceinline__ int r2_all_offset() { return (3 * kMaxSlots + kMaxT * 32) * 4; }
+__device__ __forceinline__ void route_r2_all(const Params &p, uint8_t *scratch) {
+    const int tid = threadIdx.x, warp = tid >> 5;
+    int *s_idx = reinterpret_cast<int *>(scratch);                          // R3's index array
+    float *sl = reinterpret_cast<float *>(scratch + r2_all_offset());       // [n_slabs][T][32]
+    const int n = p.n_slabs * p.T * 32;
+    for (int i = tid; i < n; i += kThreads) sl[i] = __ldcg(p.slab + i);
+    __syncthreads();
+    for (int t = warp; t < p.T; t += kThreads / 32) r2_token(p, t, sl + t * 32, p.T * 32, blockIdx.x == 0, s_idx);
+    __syncthreads();
 }
 
 // R3: the dispatch tables from the top-k, in every CTA.  scratch holds the
 // top-k indices and each slot's position inside its expert while they are built.
-__device__ __forceinline__ void route_r3(const Params &p, const Tables &tb, uint8_t *scratch) {
+__device__ __forceinline__ void route_r3(const Params &p, const Tables &tb, uint8_t *scratch, bool idx_ready) {
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int N = p.N, TK = p.T * p.K;
-    int *s_idx = reinterpret_cast<int *>(scratch);
+    int *s_idx = reinterpret_cast<int *>(scratch);   // filled by route_r2_all when idx_ready
     int *s_pos = s_idx + kMaxSlots;
-    for (int i = tid; i < TK; i += kThreads) {
+    for (int i = tid; !idx_ready && i < TK; i += kThreads) {
         int e = __ldcg(p.topk_idx + i);
         if (e < 0 || e >= N) {
             set_status(kStatusBounds);
@@ -472,10 +502,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     if ((int)blockIdx.x < p.n_slabs) route_r1<NT, EPI_UP>(p, smem);
     ok = grid_sync_all(p, 1, s_flag);
-    if (ok && (int)blockIdx.x < p.T) route_r2(p, smem);
-    if (ok) ok = grid_sync_all(p, 2, s_flag);
+    const bool r2_all = p.T <= kAllR2T;
+    if (r2_all) {
+        if (ok) route_r2_all(p, smem);
+    } else {
+        if (ok && (int)blockIdx.x < p.T) route_r2(p, smem);
+        if (ok) ok = grid_sync_all(p, 2, s_flag);
+    }
     if (ok) {
-        route_r3(p, tb, smem);   // arrives at barrier 3 once its x_perm rows are written
+        route_r3(p, tb, smem, r2_all);   // arrives at barrier 3 once its x_perm rows are written
     }
     __syncthreads();
 
@@ -510,7 +545,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const CUtensorMap *mW = ph == 0 ? &tmW1 : &tmW2;
                 const CUtensorMap *mB = ph == 0 ? &tmXp : &tmH;
                 const unsigned *bar = ph == 0 ? p.bar : p.bar4;
-                const unsigned target = (ph == 0 ? 3u : 1u) * gridDim.x;
+                // barrier 3 is the third arrival on p.bar (the second without barrier 2)
+                const unsigned target = (ph == 0 ? (r2_all ? 2u : 3u) : 1u) * gridDim.x;
                 bool ready = false;
                 int ndef = 0;
                 int def_stage[kStages], def_col[kStages], def_row[kStages];
