@@ -619,11 +619,18 @@ __device__ void simt_dispatch_chunk(const Params &p, const __nv_bfloat16 *__rest
     int *s_run = sm + 136, *s_dest = sm + 176;                                 // s_dest [chunk * K]
     for (int e = warp; e < N; e += blockDim.x / 32) {
         int tot = 0, base = 0;
-        for (int c0 = 0; c0 < n_chunks; c0 += 32) {
-            const int cc = c0 + lane;
-            const int v = cc < n_chunks ? __ldcg(p.tile_counts + (int64_t)cc * N + e) : 0;
-            tot += v;
-            if (cc < c) base += v;
+        for (int c0 = 0; c0 < n_chunks; c0 += 256) {   // eight chunk counts in flight per lane
+            int v[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int cc = c0 + lane + 32 * u;
+                v[u] = cc < n_chunks ? __ldcg(p.tile_counts + (int64_t)cc * N + e) : 0;
+            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                tot += v[u];
+                if (c0 + lane + 32 * u < c) base += v[u];
+            }
         }
         tot = __reduce_add_sync(0xffffffffu, tot);
         base = __reduce_add_sync(0xffffffffu, base);
@@ -719,10 +726,13 @@ __device__ void simt_dispatch_chunk(const Params &p, const __nv_bfloat16 *__rest
     const int t_begin = c * kSimtChunk, t_end = min(T, t_begin + kSimtChunk);
     const int n_entries = (t_end - t_begin) * K;
     const int64_t f0 = (int64_t)t_begin * K;
+    // the chunk's expert indices in one round trip (into s_dest, overwritten below)
+    for (int f = tid; f < n_entries; f += blockDim.x) s_dest[f] = __ldcg(p.topk_idx + f0 + f);
+    __syncthreads();
     if (warp == 0) {
         for (int base = 0; base < n_entries; base += 32) {
             const int f = base + lane;
-            int e = f < n_entries ? p.topk_idx[f0 + f] : -1;
+            int e = f < n_entries ? s_dest[f] : -1;
             if (f < n_entries && (e < 0 || e >= N)) {
                 set_status(kStatusBounds);
                 e = -1;
@@ -743,21 +753,33 @@ __device__ void simt_dispatch_chunk(const Params &p, const __nv_bfloat16 *__rest
         }
     }
     __syncthreads();
+    // the copies: a warp takes four of its tokens at a time (tt, tt + W, tt + 2W,
+    // tt + 3W for W warps), their slices' loads in flight together
     const int nvec = D / 8;
-    for (int tt = warp; tt < t_end - t_begin; tt += blockDim.x / 32) {
-        const uint4 *src = reinterpret_cast<const uint4 *>(x + (int64_t)(t_begin + tt) * D);
+    const int W = blockDim.x / 32, n_tok = t_end - t_begin;
+    for (int tt = warp; tt < n_tok; tt += 4 * W) {
         for (int v0 = lane; v0 < nvec; v0 += 128) {
-            uint4 r[4];
+            uint4 r[4][4];
 #pragma unroll
-            for (int u = 0; u < 4; ++u)
-                if (v0 + 32 * u < nvec) r[u] = __ldg(src + v0 + 32 * u);
-            for (int j = 0; j < K; ++j) {
-                const int d = s_dest[tt * K + j];
-                if (d < 0) continue;
-                uint4 *dst = reinterpret_cast<uint4 *>(p.x_perm + (int64_t)d * D);
+            for (int q = 0; q < 4; ++q) {
+                const int tq = tt + q * W;
+                const uint4 *src = reinterpret_cast<const uint4 *>(x + (int64_t)(t_begin + tq) * D);
 #pragma unroll
                 for (int u = 0; u < 4; ++u)
-                    if (v0 + 32 * u < nvec) dst[v0 + 32 * u] = r[u];
+                    if (tq < n_tok && v0 + 32 * u < nvec) r[q][u] = __ldg(src + v0 + 32 * u);
+            }
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const int tq = tt + q * W;
+                if (tq >= n_tok) break;
+                for (int j = 0; j < K; ++j) {
+                    const int d = s_dest[tq * K + j];
+                    if (d < 0) continue;
+                    uint4 *dst = reinterpret_cast<uint4 *>(p.x_perm + (int64_t)d * D);
+#pragma unroll
+                    for (int u = 0; u < 4; ++u)
+                        if (v0 + 32 * u < nvec) dst[v0 + 32 * u] = r[q][u];
+                }
             }
         }
     }
