@@ -729,7 +729,7 @@ int stage_scan(const Plan &P, const Bufs &b, int *counts_out, cudaStream_t s, in
 // down projection), else null.
 int stage_permute(const Plan &P, const Bufs &b, const void *x, float *y_zero, const DeviceInfo &dev,
                   cudaStream_t s) {
-    const size_t smem = (size_t)(2 * P.N + P.chunk_tokens * P.K) * 4;
+    const size_t smem = (size_t)(3 * P.N + 1 + P.chunk_tokens * P.K) * 4;
     // enough blocks to keep every SM copying with many rows in flight: split each
     // chunk's rows over up to eight blocks, aiming at eight blocks per SM
     const int split = (int)std::max<int64_t>(1, std::min<int64_t>(8, cdiv(8 * dev.sms, P.n_chunks)));
@@ -739,11 +739,12 @@ int stage_permute(const Plan &P, const Bufs &b, const void *x, float *y_zero, co
                           P.K, P.N, P.chunk_tokens, P.capacity, (const int *)b.at<int>(P.idx),
                           (const int *)b.at<int>(P.chunk_base),
                           (const int *)b.at<int>(P.row_offsets), b.at<int>(P.perm_slot), b.at<int>(P.slot_row),
-                          b.at<float>(P.x_perm), y_zero);
+                          b.at<float>(P.x_perm), y_zero, (const int *)nullptr);
     return launch_pdl(permute_kernel<__nv_bfloat16>, grid, dim3(256), smem, s, static_cast<const __nv_bfloat16 *>(x),
                       (int)P.T, P.D, P.K, P.N, P.chunk_tokens, P.capacity, (const int *)b.at<int>(P.idx),
                       (const int *)b.at<int>(P.chunk_base), (const int *)b.at<int>(P.row_offsets),
-                      b.at<int>(P.perm_slot), b.at<int>(P.slot_row), b.at<__nv_bfloat16>(P.x_perm), y_zero);
+                      b.at<int>(P.perm_slot), b.at<int>(P.slot_row), b.at<__nv_bfloat16>(P.x_perm), y_zero,
+                      (const int *)b.at<int>(P.counts));
 }
 
 // Expert GEMMs for few tokens (decode path): weight rows are the MMA's M

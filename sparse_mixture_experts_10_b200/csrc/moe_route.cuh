@@ -773,19 +773,25 @@ __global__ void __launch_bounds__(1024) scan_kernel(const int *__restrict__ chun
 // ---------------------------------------------------------------------------
 // Grid: (chunks, split).  Every block of a chunk ranks the chunk's entries
 // (cheap, identical results); block (c, 0) writes the index maps and block
-// (c, s) copies the entries f with f % split == s.
+// (c, s) copies the entries f with f % split == s.  With counts (the rows each
+// expert keeps), the blocks also clear the padding rows of every segment
+// (rows counts[e] .. the next 128-row boundary), spread over all blocks: the
+// grouped GEMMs compute those rows too, and zero operands draw less power on
+// the tensor cores than stale data (measured: up and down projections 2.6%
+// faster at the DeepSeek-V3 shape under the power cap).
 template <typename Tin>
 __global__ void __launch_bounds__(256) permute_kernel(const Tin *__restrict__ x, int T, int D, int K, int N,
                                                       int chunk_tokens, int capacity, const int *__restrict__ topk_idx,
                                                       const int *__restrict__ chunk_base,
                                                       const int *__restrict__ row_offsets, int *__restrict__ perm_slot,
                                                       int *__restrict__ slot_row, Tin *__restrict__ x_perm,
-                                                      float *__restrict__ y_zero) {
+                                                      float *__restrict__ y_zero, const int *__restrict__ counts) {
     pdl_enter();
     extern __shared__ int s_perm[];
     int *s_run = s_perm;            // [N] next position inside each expert's assignments
     int *s_row0 = s_perm + N;       // [N] first row of each expert's segment
-    int *s_dest = s_perm + 2 * N;   // [chunk_tokens * K]
+    int *s_pad = s_perm + 2 * N;    // [N + 1] padding rows before each expert (exclusive prefix)
+    int *s_dest = s_perm + 3 * N + 1;   // [chunk_tokens * K]
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int c = blockIdx.x;
     const bool writer = blockIdx.y == 0;
@@ -814,6 +820,22 @@ __global__ void __launch_bounds__(256) permute_kernel(const Tin *__restrict__ x,
         s_row0[e] = row_offsets[e];
     }
     __syncthreads();
+    if (counts && warp == 1) {   // padding rows per expert, exclusive prefix
+        int carry = 0;
+        for (int e0 = 0; e0 < N; e0 += 32) {
+            const int e = e0 + lane;
+            const int pad = e < N ? (e + 1 < N ? s_row0[e + 1] : row_offsets[N]) - s_row0[e] - counts[e] : 0;
+            int incl = pad;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int v = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += v;
+            }
+            if (e < N) s_pad[e] = carry + incl - pad;
+            carry += __shfl_sync(0xffffffffu, incl, 31);
+        }
+        if (lane == 0) s_pad[N] = carry;
+    }
     if (warp == 0) {
         for (int base = 0; base < n_entries; base += 32) {
             const int f = base + lane;
@@ -867,6 +889,22 @@ __global__ void __launch_bounds__(256) permute_kernel(const Tin *__restrict__ x,
         if (y_zero) {
             uint4 *yr = reinterpret_cast<uint4 *>(y_zero + (int64_t)(t_begin + tt) * D);
             for (int v = lane; v < D / 4; v += 32) yr[v] = make_uint4(0u, 0u, 0u, 0u);
+        }
+    }
+    if (counts) {
+        // padding row q (of s_pad[N]) is cleared by block q mod (blocks); its expert by
+        // binary search over the prefix
+        const int G = gridDim.x * gridDim.y, gi = blockIdx.y * gridDim.x + blockIdx.x;
+        for (int q = gi; q < s_pad[N]; q += G) {
+            int lo = 0, hi = N - 1;   // the last e with s_pad[e] <= q
+            while (lo < hi) {
+                const int mid = (lo + hi + 1) >> 1;
+                if (s_pad[mid] <= q) lo = mid;
+                else hi = mid - 1;
+            }
+            const int64_t row = (int64_t)s_row0[lo] + counts[lo] + (q - s_pad[lo]);
+            uint4 *dst = reinterpret_cast<uint4 *>(x_perm + row * D);
+            for (int v = tid; v < nvec; v += blockDim.x) dst[v] = make_uint4(0u, 0u, 0u, 0u);
         }
     }
 }
