@@ -66,12 +66,18 @@ SUSTAINED_STEP_MS = 1.0
 WHOLE_LAYER_WEIGHT_BYTES = 4 << 30
 GEMM_KERNEL_SRC = os.path.join(ROOT, "sparse_mixture_experts_10_b200", "csrc", "moe_gemm_tc.cuh")
 
-# DRAM traffic of the dominant kernel per launch, from one ncu capture
-# (dram__bytes_read.sum + dram__bytes_write.sum); keyed by workload and stage,
-# valid only while the kernel source hash is unchanged (see profiles/).
+# DRAM bytes per launch of the dominant pair GEMM (dram__bytes_read.sum + dram__bytes_write.sum) from
+# one ncu capture of the source with this hash: the GPT-2-width layer captured as is; the DeepSeek-V3
+# layer from the reduced case of 2048 tokens and 32 experts (512 rows per expert as at full size),
+# scaled by 8 (weights and token rows both grow eightfold).  The tail kernel beside the pair kernel
+# is not included.  Keyed by workload and stage; valid only while the source hash is unchanged.
 NCU_TRAFFIC = {
-    "gpt2/up": {"bytes": 108708096, "src_sha256": "7c227d73ad4b51f9796bb92c7559833d64a345edf15e8706150dde12569545b6"},
-    "gpt2/down": {"bytes": 184628992, "src_sha256": "7c227d73ad4b51f9796bb92c7559833d64a345edf15e8706150dde12569545b6"},
+    "gpt2/up": {"bytes": 54388992 + 54088704, "src_sha256": "5ff2a8acd93be22ae89939cf388d8497488fa048a891985ad4d97012dbd96b09"},
+    "gpt2/down": {"bytes": 167763456 + 12327424, "src_sha256": "5ff2a8acd93be22ae89939cf388d8497488fa048a891985ad4d97012dbd96b09"},
+    "deepseek/up": {"bytes": 8 * (2366248000 + 67960832), "src_sha256": "5ff2a8acd93be22ae89939cf388d8497488fa048a891985ad4d97012dbd96b09",
+                    "note": "scaled from the T=2048, N=32 capture"},
+    "deepseek/down": {"bytes": 8 * (1011410000 + 437825536), "src_sha256": "5ff2a8acd93be22ae89939cf388d8497488fa048a891985ad4d97012dbd96b09",
+                      "note": "scaled from the T=2048, N=32 capture"},
 }
 
 
