@@ -839,6 +839,39 @@ def test_bitwise_deterministic_runs():
         torch.cuda.empty_cache()
 
 
+CANARY_CASES = [("tiny", 300), ("gpt2", 2000), ("mixtral", 300), ("decode1", 1), ("decode8", 8),
+                ("deepseek_zipf", 1024)]
+
+
+@pytest.mark.parametrize("name,T", CANARY_CASES, ids=[f"{c[0]}_T{c[1]}" for c in CANARY_CASES])
+def test_workspace_and_output_canaries(name, T):
+    """Nothing is written outside the buffers a call is given: the workspace is embedded in a larger
+    buffer whose guard bytes (a byte pattern before and after it) must survive the layer call, and so
+    must the guard rows around y."""
+    wl = WORKLOADS[name]
+    if name.startswith("deepseek"):
+        wl = wl.with_(N=32)   # the DeepSeek-shaped layer with 32 experts (2.8 GB of weights)
+    inp = make_inputs(wl, "cuda", T=T)
+    layer = Layer(wl, inp)
+    n = moe.moe_workspace_size(layer.cfg, T)
+    guard = 1 << 16
+    big = torch.full((n + 2 * guard,), 0xA5, dtype=torch.uint8, device="cuda")
+    ws = big[guard:guard + n]
+    assert ws.data_ptr() % 256 == 0
+    yb = torch.full((T + 2, wl.D), 7.25, device="cuda")
+    y = yb[1:T + 1]
+    aux = dict(counts=torch.empty(wl.N, dtype=torch.int32, device="cuda"), importance=torch.empty(wl.N, device="cuda"),
+               p_mean=torch.empty(wl.N, device="cuda"), scalars=torch.empty(4, device="cuda"))
+    moe.check(moe.moe_forward(layer.cfg, inp["x"], T, layer.w, y, moe.MOE_F32, moe.make_aux(**aux), ws, n))
+    torch.cuda.synchronize()
+    assert moe.moe_get_device_status() == 0
+    assert bool((big[:guard] == 0xA5).all()) and bool((big[guard + n:] == 0xA5).all())
+    assert bool((yb[0] == 7.25).all()) and bool((yb[T + 1] == 7.25).all())
+    assert torch.isfinite(y).all()
+    del inp, layer, big
+    torch.cuda.empty_cache()
+
+
 def test_nan_scores_rank_last_and_flag_status():
     wl = WORKLOADS["tiny"]
     inp = make_inputs(wl, "cuda", T=64)
