@@ -82,7 +82,7 @@ NCU_TRAFFIC = {
 
 
 def rank_seed(wl, rank: int) -> int:
-    """Each rank draws its own batch (weak scaling: the per-GPU work is fixed)."""
+    """Each rank draws its own tokens (weak scaling: the per-GPU work is fixed)."""
     return wl.seed + 7919 * rank
 
 
@@ -651,7 +651,11 @@ def main():
     moe.load_library()
 
     T = wl.T
-    inp = make_inputs(wl, dev, seed=rank_seed(wl, rank))
+    # data parallelism: the weights are the same on every rank, each rank draws its own tokens
+    inp = make_inputs(wl, dev, seed=wl.seed)
+    if rank > 0:
+        gx = torch.Generator(device=dev).manual_seed(rank_seed(wl, rank))
+        inp["x"] = torch.randn(T, wl.D, device=dev, generator=gx).to(wl.dtype)
     cfg = moe.make_config(wl.D, wl.H, wl.N, wl.K, wl.act, moe.dtype_code(wl.dtype), wl.has_bias, wl.n_shared,
                           wl.capacity_factor, wl.overflow)
     W = moe.make_weights(inp["W_g"], inp["W1"], inp["W2"], inp["b_g"], inp["b1"], inp["b2"], inp["b_sel"],
