@@ -18,7 +18,8 @@ import os
 import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "libmoe.so")
+# MOE_BOUNDS_CHECK=1 selects the bounds-check build of the same library (build.py --bounds-check)
+LIB_PATH = os.path.join(_PKG, "libmoe_debug.so" if os.environ.get("MOE_BOUNDS_CHECK") == "1" else "libmoe.so")
 
 MOE_F32, MOE_BF16 = 0, 1
 MOE_ACT_GELU, MOE_ACT_SWIGLU = 0, 1

@@ -950,6 +950,7 @@ int stage_down(const Plan &P, const Bufs &b, const moe_weights *w, void *y, int 
         p.bias = bias;
         p.perm_slot = b.at<int>(P.perm_slot);
         p.gate_w = b.at<float>(P.w);
+        p.slot_limit = P.T * P.K;
         p.timeout_ns = kTimeoutNs;
         CUtensorMap mo = ma;   // unused unless z is written by rows
         if (combine_in_down(P, y_dtype)) {   // y was cleared by the router or the permute kernel
@@ -1156,11 +1157,12 @@ int stage_combine(const Plan &P, const Bufs &b, void *y, int y_dtype, const Devi
     const int *slot_row = b.at<int>(P.slot_row);
     const int z_by_row = P.dtype == MOE_BF16 && !P.decode ? 1 : 0;
     const float *shared = P.n_shared ? b.at<float>(P.s_out) : nullptr;
+    const int64_t z_rows = z_by_row ? (int64_t)P.rows_cap : P.T * P.K;
     if (y_dtype == MOE_F32)
-        return launch_pdl(combine_kernel<float>, dim3(grid), dim3(256), 0, s, (const float *)b.at<float>(P.z), P.T, P.D,
-                          P.K, slot_row, z_by_row, shared, static_cast<float *>(y));
-    return launch_pdl(combine_kernel<__nv_bfloat16>, dim3(grid), dim3(256), 0, s, (const float *)b.at<float>(P.z), P.T,
-                      P.D, P.K, slot_row, z_by_row, shared, static_cast<__nv_bfloat16 *>(y));
+        return launch_pdl(combine_kernel<float>, dim3(grid), dim3(256), 0, s, (const float *)b.at<float>(P.z), z_rows,
+                          P.T, P.D, P.K, slot_row, z_by_row, shared, static_cast<float *>(y));
+    return launch_pdl(combine_kernel<__nv_bfloat16>, dim3(grid), dim3(256), 0, s, (const float *)b.at<float>(P.z),
+                      z_rows, P.T, P.D, P.K, slot_row, z_by_row, shared, static_cast<__nv_bfloat16 *>(y));
 }
 
 int stage_aux(const Plan &P, const Bufs &b, const float *logits, const int *idx, const float *tw, moe_aux *aux,
@@ -1692,9 +1694,9 @@ int moe_ep_combine(const moe_config *cfg, const float *z_back, int64_t T, const 
     const int64_t nq = T * (P.D / 4);
     const int grid = (int)std::min<int64_t>(cdiv(nq, 256), (int64_t)dev->sms * 8);
     if (y_dtype == MOE_F32)
-        return launch_pdl(combine_kernel<float>, dim3(grid), dim3(256), 0, s, z_back, T, P.D, P.K, (const int *)send_pos,
-                          1, (const float *)nullptr, static_cast<float *>(y));
-    return launch_pdl(combine_kernel<__nv_bfloat16>, dim3(grid), dim3(256), 0, s, z_back, T, P.D, P.K,
+        return launch_pdl(combine_kernel<float>, dim3(grid), dim3(256), 0, s, z_back, T * P.K, T, P.D, P.K,
+                          (const int *)send_pos, 1, (const float *)nullptr, static_cast<float *>(y));
+    return launch_pdl(combine_kernel<__nv_bfloat16>, dim3(grid), dim3(256), 0, s, z_back, T * P.K, T, P.D, P.K,
                       (const int *)send_pos, 1, (const float *)nullptr, static_cast<__nv_bfloat16 *>(y));
 }
 
@@ -1885,7 +1887,7 @@ int moe_backward(const moe_config *cfg, const void *x, int64_t T, const moe_weig
     else MOE_TRY(backward_gemms<__nv_bfloat16>(B, b, x, w, gr, 1, s));
     // dx[t] = sum_j dx_perm[row of (t, j)] in slot order + W_g ds[t]
     const int grid_c = (int)std::min<int64_t>(cdiv(T * (D / 4), 256), (int64_t)dev->sms * 8);
-    combine_kernel<float><<<grid_c, 256, 0, s>>>(b.at<float>(B.dxp), T, D, K, b.at<int>(P.slot_row), 1,
+    combine_kernel<float><<<grid_c, 256, 0, s>>>(b.at<float>(B.dxp), (int64_t)P.rows_cap, T, D, K, b.at<int>(P.slot_row), 1,
                                                  b.at<float>(B.dxr), gr->dx);
     MOE_TRY(check_launch());
     // bias gradients: column sums over each expert's rows (row order), over the tokens for b_g

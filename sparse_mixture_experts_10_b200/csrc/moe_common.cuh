@@ -22,6 +22,22 @@ constexpr int kStatusNanLogit = 4;
 
 __device__ __forceinline__ void set_status(int bits) { atomicOr(&g_status, bits); }
 
+// Bounds-check build (compiled with -DMOE_DEBUG_BOUNDS): MOE_BOUNDS(cond)
+// evaluates cond, and where it is false sets the bounds bit of the status
+// word and yields false, so that the caller skips the access instead of
+// faulting.  In the normal build it is the constant true and cond is never
+// evaluated.
+#ifdef MOE_DEBUG_BOUNDS
+constexpr bool kDebugBounds = true;
+#else
+constexpr bool kDebugBounds = false;
+#endif
+__device__ __forceinline__ bool bounds_ok(bool ok) {
+    if (!ok) set_status(kStatusBounds);
+    return ok;
+}
+#define MOE_BOUNDS(cond) (!::moe::kDebugBounds || ::moe::bounds_ok(cond))
+
 __device__ __forceinline__ uint64_t globaltimer_ns() {
     uint64_t t;
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));

@@ -100,6 +100,7 @@ struct Params {
     // kernel, which waits for the tail kernel, sees both).
     int tail_mode;
     uint64_t timeout_ns;
+    int64_t slot_limit;       // EPI_SCATTER: entries of gate_w (checked in the bounds-check build when > 0)
 };
 
 __device__ __forceinline__ void red_add_v4(float *ptr, float a, float b, float c, float d) {
@@ -143,6 +144,14 @@ struct Shape2 {
 struct TileCoord {
     int g, row0, nt;
 };
+
+// Bounds-check build: a group table's segments start on 128-row blocks and
+// do not decrease.
+__device__ __forceinline__ bool group_table_ok(const int *s_rowoff, int G) {
+    bool ok = s_rowoff[0] >= 0 && s_rowoff[0] % BM == 0;
+    for (int g = 0; g < G; ++g) ok = ok && s_rowoff[g + 1] >= s_rowoff[g] && s_rowoff[g + 1] % BM == 0;
+    return ok;
+}
 
 // Tile i of 128-row tiles: group, first row and column tile.
 __device__ __forceinline__ TileCoord decode_tile(int i, const int *s_rowoff, int G, int n_tiles, int dense_mtiles) {
@@ -333,6 +342,7 @@ __device__ __forceinline__ RowGate load_row_gate(const Params &p, int row, int r
     if (EPI == EPI_SCATTER && row < row_limit) {
         if (p.perm_slot) {
             r.slot = p.perm_slot[row];
+            if (r.slot >= 0 && !MOE_BOUNDS(p.slot_limit <= 0 || r.slot < p.slot_limit)) r.slot = -1;
             if (r.slot >= 0) r.gw = p.gate_w[r.slot];
         } else {   // dense rows (shared expert): row r is token r, weight 1
             r.slot = row;
@@ -555,7 +565,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int dense_mtiles = (p.dense_rows + BM - 1) / BM;
     const int m_tiles = rowoff ? s_rowoff[G] / BM : dense_mtiles;
     const bool tails = rowoff && p.tail_mode == 2;
-    const int total = tails ? s_tcum[G] * p.n_tiles : m_tiles * p.n_tiles;
+    // a table that fails the bounds-check build's test: no tiles at all
+    const bool tbl_ok = !rowoff || MOE_BOUNDS(group_table_ok(s_rowoff, G));
+    const int total = !tbl_ok ? 0 : tails ? s_tcum[G] * p.n_tiles : m_tiles * p.n_tiles;
     auto tile_of = [&](int i) {
         return tails ? decode_tail_tile(i, s_rowoff, s_tcum, G, p.n_tiles)
                      : decode_tile(i, rowoff, G, p.n_tiles, dense_mtiles);
@@ -847,7 +859,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const int *rowoff = p.row_offsets ? s_rowoff : nullptr;
     const int dense_units = (p.dense_rows + 2 * BM - 1) / (2 * BM);
     const int units = rowoff ? s_units[G] : dense_units;
-    const int total = units * p.n_tiles;
+    const bool tbl_ok = !rowoff || MOE_BOUNDS(group_table_ok(s_rowoff, G));
+    const int total = tbl_ok ? units * p.n_tiles : 0;
 
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer (both CTAs)

@@ -854,7 +854,10 @@ __global__ void __launch_bounds__(256) permute_kernel(const Tin *__restrict__ x,
             if (f < n_entries) {
                 // the assignment's position among its expert's: accepted below the capacity
                 const int pos = base_row + rank;
-                const int dest = (e >= 0 && pos < capacity) ? s_row0[e] + pos : -1;
+                int dest = (e >= 0 && pos < capacity) ? s_row0[e] + pos : -1;
+                // bounds-check build: the row lies inside its expert's padded segment
+                if (dest >= 0 && !MOE_BOUNDS(pos >= 0 && dest < (e + 1 < N ? s_row0[e + 1] : row_offsets[N])))
+                    dest = -1;
                 s_dest[f] = dest;
                 if (writer) {
                     if (dest >= 0) perm_slot[dest] = (int)(f0 + f);
@@ -903,6 +906,7 @@ __global__ void __launch_bounds__(256) permute_kernel(const Tin *__restrict__ x,
                 else hi = mid - 1;
             }
             const int64_t row = (int64_t)s_row0[lo] + counts[lo] + (q - s_pad[lo]);
+            if (!MOE_BOUNDS(counts[lo] >= 0 && row < row_offsets[N])) continue;
             uint4 *dst = reinterpret_cast<uint4 *>(x_perm + row * D);
             for (int v = tid; v < nvec; v += blockDim.x) dst[v] = make_uint4(0u, 0u, 0u, 0u);
         }
@@ -933,10 +937,11 @@ __global__ void __launch_bounds__(256) zero_kernel(uint4 *__restrict__ p, int64_
 // ---------------------------------------------------------------------------
 // slot_row: the permuted row of each slot, -1 for a slot dropped by the
 // capacity limit (it adds nothing); z_by_row: z rows are permuted rows (bf16
-// prefill) rather than slots.
+// prefill) rather than slots; z_rows: the rows z holds (checked in the
+// bounds-check build).
 template <typename Tout>
-__global__ void __launch_bounds__(256) combine_kernel(const float *__restrict__ z, int64_t T, int D, int K,
-                                                      const int *__restrict__ slot_row, int z_by_row,
+__global__ void __launch_bounds__(256) combine_kernel(const float *__restrict__ z, int64_t z_rows, int64_t T, int D,
+                                                      int K, const int *__restrict__ slot_row, int z_by_row,
                                                       const float *__restrict__ shared, Tout *__restrict__ y) {
     pdl_enter();
     const int64_t nq = T * (D / 4);
@@ -950,6 +955,7 @@ __global__ void __launch_bounds__(256) combine_kernel(const float *__restrict__ 
             const int rr = __ldg(slot_row + t * K + j);
             if (rr < 0) continue;
             const int64_t r = z_by_row ? (int64_t)rr : t * K + j;
+            if (!MOE_BOUNDS(r < z_rows)) continue;
             const float4 v = *reinterpret_cast<const float4 *>(z + r * D + d);
             if (first) {
                 acc = v;

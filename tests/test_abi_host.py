@@ -34,6 +34,16 @@ def test_every_declared_function_is_exported(lib):
     assert sorted(moe.EXPORTED) == names
 
 
+def test_bounds_check_build_exports_the_same_functions():
+    """The bounds-check build (-DMOE_DEBUG_BOUNDS, loaded under MOE_BOUNDS_CHECK=1) is the same
+    library with index checks compiled in: it builds for sm_100a and exports every declared function."""
+    path = moe_build.build(bounds_check=True)
+    assert path.endswith("libmoe_debug.so") and path != moe_build.LIB
+    dbg = ctypes.CDLL(path)
+    for n in header_functions():
+        assert hasattr(dbg, n), n
+
+
 def test_struct_sizes_match_header_layout():
     assert ctypes.sizeof(moe.moe_config) == 10 * 4
     assert ctypes.sizeof(moe.moe_weights) == 11 * 8
