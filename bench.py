@@ -222,12 +222,6 @@ def fused_decode(wl, T):
             not (wl.capacity_factor > 0 and wl.overflow))
 
 
-def row_stream_decode(wl, T):
-    """Whether the one-kernel decode path streams whole weight rows (at most 4 tokens and 8
-    (token, slot) pairs) rather than running tensor-core tiles."""
-    return fused_decode(wl, T) and T <= 4 and T * wl.K <= 8
-
-
 def gemm_peak(pk, step_ms):
     """(peak TFLOP/s, its name): the sustained figure for kernels inside long steps, else the burst one."""
     if step_ms > SUSTAINED_STEP_MS and "bf16_tflops_sustained" in pk:
@@ -805,9 +799,7 @@ def main():
         kname = names[dom]
         if fused_decode(wl, T) and names[dom] == "up":
             # the whole layer is one kernel between the "up" events: all of its bytes count
-            byt = wm["decode_bytes"]
-            kname = ("decode_stream_kernel" if row_stream_decode(wl, T) else "decode_layer_kernel") + \
-                " (whole layer, one launch)"
+            byt, kname = wm["decode_bytes"], "decode_layer_kernel (whole layer, one launch)"
         achieved = byt / (dom_mean_ms * 1e-3) / 1e9
         peak = float(pk["hbm_gbs"])
         roof = {"kernel": kname, "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",

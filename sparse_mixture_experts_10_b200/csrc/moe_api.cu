@@ -15,7 +15,6 @@
 #include "moe_backward.cuh"
 #include "moe_common.cuh"
 #include "moe_decode_fused.cuh"
-#include "moe_decode_stream.cuh"
 #include "moe_gemm_simt.cuh"
 #include "moe_gemm_decode.cuh"
 #include "moe_gemm_tc.cuh"
@@ -264,8 +263,6 @@ int device_info(DeviceInfo **out) {
         MOE_FUSED_ATTR(32);
         MOE_FUSED_ATTR(64);
 #undef MOE_FUSED_ATTR
-        MOE_TRY(allow_smem(dst::decode_stream_kernel<dec::EPI_SWIGLU>));
-        MOE_TRY(allow_smem(dst::decode_stream_kernel<dec::EPI_GELU>));
         MOE_TRY(allow_smem(rtc::router_simt_kernel<8, false>));
         MOE_TRY(allow_smem(rtc::router_simt_kernel<16, false>));
         MOE_TRY(allow_smem(rtc::router_simt_kernel<32, false>));
@@ -1277,11 +1274,17 @@ bool fused_fits(const Plan &P) {
                                    : fused_fits_nt<dec::EPI_GELU>(P.nt, scratch);
 }
 
-// Arguments of the fused decode kernels (moe_decode_fused.cuh, moe_decode_stream.cuh).
-dfu::Params fused_params(const Plan &P, const Bufs &b, const void *x, const moe_weights *w, void *y, int y_dtype,
-                         moe_aux *aux) {
+// The whole layer for few tokens in one cooperative kernel (moe_decode_fused.cuh).
+int stage_decode_fused(const Plan &P, const Bufs &b, const void *x, const moe_weights *w, void *y, int y_dtype,
+                       moe_aux *aux, const DeviceInfo &dev, cudaStream_t s) {
     const int D = P.D, H = P.H, N = P.N;
     const bool swiglu = P.act == MOE_ACT_SWIGLU;
+    const int grid = dev.sms;
+    CUtensorMap mw1, mxp, mw2, mh;
+    MOE_TRY(make_map(&mw1, w->W1, (int64_t)N * (swiglu ? 2 * H : H), D, swiglu ? 64 : 128));
+    MOE_TRY(make_map(&mxp, b.ws + P.x_perm, P.rows_cap, D, P.nt));
+    MOE_TRY(make_map(&mw2, w->W2, (int64_t)N * D, H, 128));
+    MOE_TRY(make_map(&mh, b.ws + P.h, P.rows_cap, H, P.nt));
     dfu::Params p{};
     p.T = (int)P.T;
     p.D = D;
@@ -1329,70 +1332,8 @@ dfu::Params fused_params(const Plan &P, const Bufs &b, const void *x, const moe_
         p.aux_scalars = aux->scalars;
     }
     p.timeout_ns = kTimeoutNs;
-    p.W1 = w->W1;
-    p.W2 = w->W2;
-    return p;
-}
-
-// The whole layer for few tokens in one cooperative kernel (moe_decode_fused.cuh).
-int stage_decode_fused(const Plan &P, const Bufs &b, const void *x, const moe_weights *w, void *y, int y_dtype,
-                       moe_aux *aux, const DeviceInfo &dev, cudaStream_t s) {
-    const int D = P.D, H = P.H, N = P.N;
-    const bool swiglu = P.act == MOE_ACT_SWIGLU;
-    const int grid = dev.sms;
-    CUtensorMap mw1, mxp, mw2, mh;
-    MOE_TRY(make_map(&mw1, w->W1, (int64_t)N * (swiglu ? 2 * H : H), D, swiglu ? 64 : 128));
-    MOE_TRY(make_map(&mxp, b.ws + P.x_perm, P.rows_cap, D, P.nt));
-    MOE_TRY(make_map(&mw2, w->W2, (int64_t)N * D, H, 128));
-    MOE_TRY(make_map(&mh, b.ws + P.h, P.rows_cap, H, P.nt));
-    const dfu::Params p = fused_params(P, b, x, w, y, y_dtype, aux);
     if (swiglu) return launch_fused_nt<dec::EPI_SWIGLU>(P.nt, mw1, mxp, mw2, mh, p, grid, s);
     return launch_fused_nt<dec::EPI_GELU>(P.nt, mw1, mxp, mw2, mh, p, grid, s);
-}
-
-// Shared-memory plan of the row-streaming decode kernel (moe_decode_stream.cuh),
-// or false when the layer does not suit it: more tokens or slots than its
-// shared-memory x and h rows hold, or rows too long for an 8-stage ring.
-bool stream_plan(const Plan &P, dst::Smem *sm) {
-    if (P.T > dst::kMaxT || P.T * P.K > dst::kMaxSlots) return false;
-    const uint32_t sb = (uint32_t)(cdiv((int64_t)std::max(P.D, P.H) * 2, 128) * 128);
-    const int64_t xh = std::max<int64_t>(P.T * P.D * 2, P.T * P.K * P.H * 2);
-    *sm = dst::Smem{sb, 0, (uint32_t)(cdiv(xh, 128) * 128)};
-    const size_t fixed = sm->total(), limit = 227 * 1024;
-    if (fixed + 8 * (size_t)sb > limit) return false;
-    sm->stages = (uint32_t)std::min<size_t>(dst::kMaxStages, (limit - fixed) / sb);
-    // the routing scratch (R1-R3) lives in the ring before the stream uses it
-    return fused_scratch((int)P.T, P.slab_rows, P.n_slabs) <= sm->ring_bytes();
-}
-
-// The whole layer for one or two tokens as one stream of whole weight rows.
-int stage_decode_stream(const Plan &P, const Bufs &b, const void *x, const moe_weights *w, void *y, int y_dtype,
-                        moe_aux *aux, const dst::Smem &sm, const DeviceInfo &dev, cudaStream_t s) {
-    const dfu::Params p = fused_params(P, b, x, w, y, y_dtype, aux);
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)dev.sms);
-    cfg.blockDim = dim3(dst::kThreads);
-    cfg.dynamicSmemBytes = sm.total();
-    cfg.stream = s;
-    cudaLaunchAttribute attr[2];
-    attr[0].id = cudaLaunchAttributeCooperative;   // every CTA resident: the grid barriers need it
-    attr[0].val.cooperative = 1;
-    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[1].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = g_fused_pdl ? 2 : 1;
-    auto kern = P.act == MOE_ACT_SWIGLU ? dst::decode_stream_kernel<dec::EPI_SWIGLU>
-                                        : dst::decode_stream_kernel<dec::EPI_GELU>;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, kern, p, sm);
-    if (e != cudaSuccess && cfg.numAttrs == 2) {   // the runtime refused the pair: cooperative alone
-        (void)cudaGetLastError();
-        g_fused_pdl = false;
-        cfg.numAttrs = 1;
-        e = cudaLaunchKernelEx(&cfg, kern, p, sm);
-    }
-    g_launches.fetch_add(1, std::memory_order_relaxed);
-    if (e != cudaSuccess) return MOE_ERR_CUDA;
-    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
 int check_weights(const Plan &P, const moe_weights *w, bool need_experts) {
@@ -1451,9 +1392,7 @@ int forward_impl(const moe_config *cfg, const void *x, int64_t T, const moe_weig
     if (P.fused_decode && dev->sms >= (int)P.T && dev->sms >= P.n_slabs && dev->sms <= P.dec_cap &&
         aligned16(w->W_g) && fused_fits(P)) {
         for (int i = 1; i <= 3; ++i) MOE_TRY(rec(i));
-        dst::Smem sm;
-        if (stream_plan(P, &sm)) MOE_TRY(stage_decode_stream(P, b, x, w, y, y_dtype, aux, sm, *dev, s));
-        else MOE_TRY(stage_decode_fused(P, b, x, w, y, y_dtype, aux, *dev, s));
+        MOE_TRY(stage_decode_fused(P, b, x, w, y, y_dtype, aux, *dev, s));
         for (int i = 4; i <= MOE_N_STAGES; ++i) MOE_TRY(rec(i));
         return MOE_OK;
     }

@@ -77,7 +77,6 @@ struct Params {
     int *aux_counts;
     float *aux_importance, *aux_p_mean, *aux_scalars;
     uint64_t timeout_ns;
-    const void *W1, *W2;           // expert weights (the row-streaming kernel, moe_decode_stream.cuh)
 };
 
 template <int NT, int EPI_UP>
@@ -141,8 +140,6 @@ struct Tables {
     int *nlive;     // [1]
 };
 
-// (The routing phases run with any block size that is a multiple of 32: the
-// row-streaming kernel of moe_decode_stream.cuh uses them too.)
 // ------------------------------------------------------------------ routing phases
 template <int NT, int EPI_UP>
 __device__ __forceinline__ void route_r1(const Params &p, uint8_t *scratch) {
@@ -155,7 +152,7 @@ __device__ __forceinline__ void route_r1(const Params &p, uint8_t *scratch) {
     float *ws = xs + (size_t)T * R;                            // [R][32]
     // 16-byte loads: slab rows start at multiples of 8 elements and D, N * 8 are multiples of 8
     const int xv = nd / 8;
-    for (int i = tid; i < T * xv; i += (int)blockDim.x) {
+    for (int i = tid; i < T * xv; i += kThreads) {
         const int t = i / xv, v = i - t * xv;
         const uint4 q = __ldg(reinterpret_cast<const uint4 *>(p.x + (size_t)t * D + d0) + v);
         float f[8];
@@ -164,7 +161,7 @@ __device__ __forceinline__ void route_r1(const Params &p, uint8_t *scratch) {
         for (int k = 0; k < 8; ++k) xs[t * R + v * 8 + k] = f[k];
     }
     const int wtot = nd * N;   // W_g slab is contiguous: rows d0.., N experts each
-    for (int i = tid * 8; i < wtot; i += (int)blockDim.x * 8) {
+    for (int i = tid * 8; i < wtot; i += kThreads * 8) {
         float f[8];
         if (i + 8 <= wtot && ((d0 * N) % 8) == 0) {
             Vec16<__nv_bfloat16>::unpack(__ldg(reinterpret_cast<const uint4 *>(p.Wg + (size_t)d0 * N + i)), f);
@@ -182,7 +179,7 @@ __device__ __forceinline__ void route_r1(const Params &p, uint8_t *scratch) {
     __syncthreads();
     // partial scores of the slab: warp w takes tokens w, w + 6, ...; lane = expert;
     // four running sums over the slab rows (k mod 4), added in a fixed order
-    for (int t = warp; t < T; t += (int)(blockDim.x >> 5)) {
+    for (int t = warp; t < T; t += kThreads / 32) {
         const float *xr = xs + (size_t)t * R;
         float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
         int k = 0;
@@ -244,7 +241,7 @@ __device__ __forceinline__ void route_r2(const Params &p, uint8_t *scratch) {
     const int tid = threadIdx.x;
     const int t = blockIdx.x;
     float *sl = reinterpret_cast<float *>(scratch);   // [n_slabs][32]
-    for (int i = tid; i < p.n_slabs * 32; i += (int)blockDim.x)
+    for (int i = tid; i < p.n_slabs * 32; i += kThreads)
         sl[i] = __ldcg(p.slab + ((size_t)(i >> 5) * p.T + t) * 32 + (i & 31));
     __syncthreads();
     if (tid < 32) r2_token(p, t, sl, 32, true, nullptr);
@@ -261,9 +258,9 @@ __device__ __forceinline__ void route_r2_all(const Params &p, uint8_t *scratch) 
     int *s_idx = reinterpret_cast<int *>(scratch);                          // R3's index array
     float *sl = reinterpret_cast<float *>(scratch + r2_all_offset());       // [n_slabs][T][32]
     const int n = p.n_slabs * p.T * 32;
-    for (int i = tid; i < n; i += (int)blockDim.x) sl[i] = __ldcg(p.slab + i);
+    for (int i = tid; i < n; i += kThreads) sl[i] = __ldcg(p.slab + i);
     __syncthreads();
-    for (int t = warp; t < p.T; t += (int)(blockDim.x >> 5)) r2_token(p, t, sl + t * 32, p.T * 32, blockIdx.x == 0, s_idx);
+    for (int t = warp; t < p.T; t += kThreads / 32) r2_token(p, t, sl + t * 32, p.T * 32, blockIdx.x == 0, s_idx);
     __syncthreads();
 }
 
@@ -274,7 +271,7 @@ __device__ __forceinline__ void route_r3(const Params &p, const Tables &tb, uint
     const int N = p.N, TK = p.T * p.K;
     int *s_idx = reinterpret_cast<int *>(scratch);   // filled by route_r2_all when idx_ready
     int *s_pos = s_idx + kMaxSlots;
-    for (int i = tid; !idx_ready && i < TK; i += (int)blockDim.x) {
+    for (int i = tid; !idx_ready && i < TK; i += kThreads) {
         int e = __ldcg(p.topk_idx + i);
         if (e < 0 || e >= N) {
             set_status(kStatusBounds);
@@ -319,7 +316,7 @@ __device__ __forceinline__ void route_r3(const Params &p, const Tables &tb, uint
         if (lane == 0) *tb.nlive = __popc(m);
     }
     __syncthreads();
-    for (int i = tid; i < TK; i += (int)blockDim.x) {
+    for (int i = tid; i < TK; i += kThreads) {
         const int e = s_idx[i], pos = s_pos[i];
         const bool keep = e >= 0 && pos < tb.kept[e];
         tb.row[i] = (int16_t)(keep ? tb.rowoff[e] + pos : -1);
@@ -333,7 +330,7 @@ __device__ __forceinline__ void route_r3(const Params &p, const Tables &tb, uint
         if (r < 0) continue;
         const uint4 *src = reinterpret_cast<const uint4 *>(p.x + (size_t)(i / p.K) * p.D);
         uint4 *dst = reinterpret_cast<uint4 *>(p.x_perm + (size_t)r * p.D);
-        for (int v = tid; v < nv; v += (int)blockDim.x) dst[v] = __ldg(src + v);
+        for (int v = tid; v < nv; v += kThreads) dst[v] = __ldg(src + v);
     }
     // x_perm written: release it to the grid (barrier 3 is waited on only by the
     // producers, before their first token-row load); the workspace tables and the
@@ -345,7 +342,7 @@ __device__ __forceinline__ void route_r3(const Params &p, const Tables &tb, uint
     }
     if (blockIdx.x == 0) {
         // the workspace tables (moe_get_workspace_layout) and the statistics
-        for (int e = tid; e < N; e += (int)blockDim.x) {
+        for (int e = tid; e < N; e += kThreads) {
             p.counts[e] = tb.kept[e];
             p.offsets[e] = tb.koff[e];
             p.row_offsets[e] = tb.rowoff[e];
@@ -355,13 +352,13 @@ __device__ __forceinline__ void route_r3(const Params &p, const Tables &tb, uint
             p.row_offsets[N] = tb.rowoff[N - 1] + (tb.kept[N - 1] + kRowAlign - 1) / kRowAlign * kRowAlign;
             *p.n_live = *tb.nlive;
         }
-        for (int i = tid; i < *tb.nlive; i += (int)blockDim.x) p.live[i] = tb.live[i];
-        for (int i = tid; i < TK; i += (int)blockDim.x) {
+        for (int i = tid; i < *tb.nlive; i += kThreads) p.live[i] = tb.live[i];
+        for (int i = tid; i < TK; i += kThreads) {
             const int r = tb.row[i];
             p.slot_row[i] = r;
             if (r >= 0) p.perm_slot[r] = i;
         }
-        for (int e = warp; e < N; e += (int)(blockDim.x >> 5)) {
+        for (int e = warp; e < N; e += kThreads / 32) {
             const int start = tb.rowoff[e] + tb.kept[e];
             const int end = tb.rowoff[e] + (tb.kept[e] + kRowAlign - 1) / kRowAlign * kRowAlign;
             for (int r = start + lane; r < end; r += 32) p.perm_slot[r] = -1;
@@ -372,8 +369,8 @@ __device__ __forceinline__ void route_r3(const Params &p, const Tables &tb, uint
         float *f_pm = f_im + 32;
         float *s_w = reinterpret_cast<float *>(s_pos + kMaxSlots);   // [T*K]
         float *s_tp = s_w + kMaxSlots;                               // [T][32]
-        for (int i = tid; i < TK; i += (int)blockDim.x) s_w[i] = __ldcg(p.topk_w + i);
-        for (int i = tid; i < p.T * 32; i += (int)blockDim.x) s_tp[i] = __ldcg(p.tok_p + i);
+        for (int i = tid; i < TK; i += kThreads) s_w[i] = __ldcg(p.topk_w + i);
+        for (int i = tid; i < p.T * 32; i += kThreads) s_tp[i] = __ldcg(p.tok_p + i);
         __syncthreads();
         if (tid < 32) {
             const int e = tid;
