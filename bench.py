@@ -222,6 +222,27 @@ def fused_decode(wl, T):
             not (wl.capacity_factor > 0 and wl.overflow))
 
 
+def stream_floor_ms(nbytes, flush, dev, reps=10):
+    """Median time of one plain read of nbytes from HBM (torch.sum over a bf16 tensor of that
+    size, fp32 accumulation; L2 flushed before each run, CUDA events around the launch): what a
+    single pass over that many bytes takes on this GPU, launch, ramp and tail included.  Context
+    for a layer that must read the same bytes once (the decode path), not a bound it is held to."""
+    t = torch.ones(max(nbytes // 2, 1), dtype=torch.bfloat16, device=dev)
+    out = torch.empty((), dtype=torch.float32, device=dev)
+    ms = []
+    for i in range(reps + 3):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        torch.sum(t, dim=0, dtype=torch.float32, out=out)
+        b.record()
+        torch.cuda.synchronize()
+        if i >= 3:
+            ms.append(a.elapsed_time(b))
+    del t
+    return float(np.median(ms))
+
+
 def gemm_peak(pk, step_ms):
     """(peak TFLOP/s, its name): the sustained figure for kernels inside long steps, else the burst one."""
     if step_ms > SUSTAINED_STEP_MS and "bf16_tflops_sustained" in pk:
@@ -838,6 +859,12 @@ def main():
         gbs = wm["decode_bytes"] / (ms_per_step * 1e-3) / 1e9
         layer.update({"decode_bytes": wm["decode_bytes"], "GB/s": gbs, "frac_vs_spec": gbs / SPEC_PEAKS["hbm_gbs"],
                       "frac_of_measured": gbs / float(pk["hbm_gbs"]), "live_experts": wm["live_experts"]})
+        # a plain read of the same bytes, timed the same way: the rate one pass of this size reaches
+        fl_ms = stream_floor_ms(int(wm["decode_bytes"]), flush, dev)
+        roof["stream_floor"] = {"ms": fl_ms, "GB/s": wm["decode_bytes"] / (fl_ms * 1e-3) / 1e9,
+                                "frac_of_copy": wm["decode_bytes"] / (fl_ms * 1e-3) / 1e9 / float(pk["hbm_gbs"]),
+                                "how": "torch.sum over a bf16 tensor of the layer's bytes, L2 flushed, median of 10"}
+        roof["frac_of_stream_floor"] = fl_ms / dom_mean_ms
 
     line = {"metric": METRIC, "value": tokens_per_s, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",

@@ -405,6 +405,29 @@ def test_decode_layer_is_one_kernel(name, wl):
     check_aux(aux, V, wl.N, wl.K)
 
 
+@pytest.mark.parametrize("name,wl", [
+    ("gpt-oss T=2", WORKLOADS["decode1"].with_(T=2)),
+    ("gpt-oss T=2 skewed, capacity drop", WORKLOADS["decode1"].with_(T=2, zipf_s=2.0, capacity_factor=0.5)),
+    ("GELU + biases, T=4 K=2", Workload("small_gelu", 72, 4, 1024, 1024, 6, 2, ACT_GELU, torch.bfloat16, True,
+                                        0.03, random_bias=True, zipf_s=0.3)),
+    ("ragged D/H, T=2 K=3, selection bias", Workload("small_rag", 73, 2, 1000, 712, 12, 3, ACT_SWIGLU,
+                                                     torch.bfloat16, False, 0.04, zipf_s=0.5, sel_s=0.5)),
+    ("one token, K=8 of 32", Workload("small_k8", 74, 1, 512, 384, 32, 8, ACT_SWIGLU, torch.bfloat16, False, 0.05)),
+], ids=lambda v: v if isinstance(v, str) else "")
+def test_decode_few_tokens(name, wl):
+    """One to four tokens: the one-kernel decode path (two launches per layer call, counter clear
+    included) with routing bit-exact, y within the bf16 tolerance and the statistics, for dropped
+    slots, ragged D / H, a selection bias and K = 8."""
+    inp = make_inputs(wl, "cuda")
+    layer = Layer(wl, inp)
+    layer.forward(with_aux=False)
+    n0 = moe.moe_launch_count()
+    layer.forward(with_aux=False)
+    assert moe.moe_launch_count() - n0 == 2
+    run_layer, y, ws, aux, V, ref, errs = run_full(wl, inp)
+    check_aux(aux, V, wl.N, wl.K)
+
+
 @pytest.mark.parametrize("N,K,T", [(12, 3, 300), (32, 4, 300), (6, 2, 1), (20, 4, 40), (32, 8, 64), (33, 2, 50)])
 def test_bf16_router_paths(N, K, T):
     """bf16 routers: the SIMT router with 16 and 32 padded experts (T > 64), the few-token
