@@ -176,15 +176,21 @@ def simt_router_clears_y(wl, T) -> bool:
     return fused_combine(wl, T) and wl.N <= 32
 
 
-def work_model(wl, T, counts=None):
-    """Algorithmic work per layer call (routed rows only, no padding), per stage."""
+def work_model(wl, T, counts=None, kept=None):
+    """Algorithmic work per layer call (routed rows only, no padding), per stage.  With a
+    per-expert capacity, kept holds each expert's accepted (token, slot) pairs: only those rows
+    are copied, multiplied and combined (a dropped pair costs no expert work)."""
     D, H, N, K = wl.D, wl.H, wl.N, wl.K
     b = 4 if wl.dtype == torch.float32 else 2
     c_up = 4 if wl.act == ACT_SWIGLU else 2
-    up_flops = T * K * c_up * D * H
-    down_flops = T * K * 2 * D * H
+    rows = int(np.asarray(kept).sum()) if kept is not None else T * K
+    if kept is not None:
+        live = int((np.asarray(kept) > 0).sum())
+    else:
+        live = int((np.asarray(counts) > 0).sum()) if counts is not None else min(N, T * K)
+    up_flops = rows * c_up * D * H
+    down_flops = rows * 2 * D * H
     router_flops = T * 2 * D * N
-    live = int((np.asarray(counts) > 0).sum()) if counts is not None else min(N, T * K)
     up_rows = 2 * H if wl.act == ACT_SWIGLU else H
     y_clear = T * D * 4 if fused_combine(wl, T) else 0
     by_router = simt_router_clears_y(wl, T)
@@ -194,8 +200,8 @@ def work_model(wl, T, counts=None):
         # x, W_g, logits, top-k indices and weights (+ the clear of y when the router does it)
         route_bytes=T * D * b + D * N * b + T * N * 4 + T * K * 8 + (y_clear if by_router else 0),
         # x read once, its K copies written, the slot maps (+ the clear of y otherwise)
-        permute_bytes=T * D * b + T * K * D * b + T * K * 8 + (0 if by_router else y_clear),
-        combine_bytes=0 if fused_combine(wl, T) else T * K * D * 4 + T * D * 4,
+        permute_bytes=T * D * b + rows * D * b + T * K * 8 + (0 if by_router else y_clear),
+        combine_bytes=0 if fused_combine(wl, T) else rows * D * 4 + T * D * 4,
         up_weight_bytes=live * up_rows * D * b, down_weight_bytes=live * D * H * b,
         live_experts=live,
         # whole-layer bytes a memory-bound (decode) step must move: the live experts' weights, x, y, W_g
@@ -707,7 +713,11 @@ def main():
     st = moe.moe_get_device_status()
     if st != 0:
         raise RuntimeError(f"device status {st} after warm-up")
-    counts = aux_t["counts"].cpu().numpy()
+    counts = aux_t["counts"].cpu().numpy()   # the router's choice, before any capacity
+    kept = None
+    if wl.capacity_factor > 0:   # the accepted pairs per expert, from the workspace tables
+        Lw = moe.moe_get_workspace_layout(cfg, T)
+        kept = ws[Lw.counts:Lw.counts + 4 * wl.N].view(torch.int32).cpu().numpy()
 
     def capture(stage_events):
         g = torch.cuda.CUDAGraph()
@@ -803,7 +813,7 @@ def main():
     aux_global = gstats.report() if gstats is not None else None
 
     # ---- roofline of the dominant kernel (its duration from the timed steps)
-    wm = work_model(wl, T, counts)
+    wm = work_model(wl, T, counts, kept)
     pk, pk_kind = peaks()
     decode = wl.name.startswith("decode")
     if names[dom] in ("up", "down") and not decode:

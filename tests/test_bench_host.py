@@ -137,3 +137,22 @@ def test_reduced_profiling_case_keeps_the_shape_per_expert():
     assert wl.T * wl.K // wl.N == full.T * full.K // full.N      # 512 assignments per expert either way
     assert wl.name.startswith("deepseek[")
     assert bench.workload_from_args(bench.parse([])) == WORKLOADS["deepseek"]
+
+
+def test_capacity_counts_only_the_kept_pairs():
+    """With a per-expert capacity the dropped (token, slot) pairs cost no expert work: FLOPs,
+    copies and combine reads follow the accepted pairs, the slot maps all T*K pairs."""
+    wl = WORKLOADS["deepseek_zipf"].with_(capacity_factor=1.0)
+    T, D, H, N, K = wl.T, wl.D, wl.H, wl.N, wl.K
+    kept = np.zeros(N, dtype=np.int64)
+    kept[:40] = 512                       # 40 experts full at C = T*K/N, the rest dropped
+    rows = 40 * 512
+    m = bench.work_model(wl, T, np.full(N, T * K // N), kept)
+    assert m["up_flops"] == 4 * rows * D * H
+    assert m["down_flops"] == 2 * rows * D * H
+    assert m["flops"] == 2 * T * D * N + 6 * rows * D * H
+    assert m["permute_bytes"] == T * D * 2 + rows * D * 2 + T * K * 8
+    assert m["combine_bytes"] == rows * D * 4 + T * D * 4
+    assert m["live_experts"] == 40
+    # without a capacity every routed pair is work
+    assert bench.work_model(wl, T)["up_flops"] == 4 * T * K * D * H
