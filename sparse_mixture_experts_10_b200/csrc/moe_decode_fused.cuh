@@ -264,9 +264,95 @@ __device__ __forceinline__ void route_r2_all(const Params &p, uint8_t *scratch) 
     __syncthreads();
 }
 
+// CTA 0 after R3: the workspace tables (moe_get_workspace_layout) and the
+// statistics of the router's choice, by threads tid < nth of the CTA that sync()
+// brings together; s_idx holds the T*K selected experts, stat has room for
+// 64 + T*K + 32*T floats.
+template <class Sync>
+__device__ __forceinline__ void r3_publish(const Params &p, const Tables &tb, const int *s_idx, float *stat, int tid,
+                                           int nth, Sync sync) {
+    const int warp = tid >> 5, lane = tid & 31;
+    const int N = p.N, TK = p.T * p.K;
+    // the workspace tables (moe_get_workspace_layout) and the statistics
+    for (int e = tid; e < N; e += nth) {
+        p.counts[e] = tb.kept[e];
+        p.offsets[e] = tb.koff[e];
+        p.row_offsets[e] = tb.rowoff[e];
+    }
+    if (tid == 0) {
+        p.offsets[N] = tb.koff[N - 1] + tb.kept[N - 1];
+        p.row_offsets[N] = tb.rowoff[N - 1] + (tb.kept[N - 1] + kRowAlign - 1) / kRowAlign * kRowAlign;
+        *p.n_live = *tb.nlive;
+    }
+    for (int i = tid; i < *tb.nlive; i += nth) p.live[i] = tb.live[i];
+    for (int i = tid; i < TK; i += nth) {
+        const int r = tb.row[i];
+        p.slot_row[i] = r;
+        if (r >= 0) p.perm_slot[r] = i;
+    }
+    for (int e = warp; e < N; e += (nth >> 5)) {
+        const int start = tb.rowoff[e] + tb.kept[e];
+        const int end = tb.rowoff[e] + (tb.kept[e] + kRowAlign - 1) / kRowAlign * kRowAlign;
+        for (int r = start + lane; r < end; r += 32) p.perm_slot[r] = -1;
+    }
+    // statistics of the router's choice: fixed orders (tokens ascending, slots
+    // ascending), from the gate weights and the full softmax loaded at once
+    float *f_im = stat, *f_pm = stat + 32;   // [32] each
+    float *s_w = stat + 64;                  // [T*K]
+    float *s_tp = s_w + TK;                  // [T][32]
+    for (int i = tid; i < TK; i += nth) s_w[i] = __ldcg(p.topk_w + i);
+    for (int i = tid; i < p.T * 32; i += nth) s_tp[i] = __ldcg(p.tok_p + i);
+    sync();
+    if (tid < 32) {
+        const int e = tid;
+        float im = 0.f, pm = 0.f;
+        if (e < N) {
+            for (int i = 0; i < TK; ++i)
+                if (s_idx[i] == e) im += s_w[i];
+            for (int t = 0; t < p.T; ++t) pm += s_tp[t * 32 + e];
+            pm /= (float)p.T;
+        }
+        f_im[e] = im;
+        f_pm[e] = pm;
+        if (e < N) {
+            if (p.aux_counts) p.aux_counts[e] = tb.cnt[e];
+            if (p.aux_importance) p.aux_importance[e] = im;
+            if (p.aux_p_mean) p.aux_p_mean[e] = pm;
+        }
+    }
+    sync();
+    if (tid == 0 && p.aux_scalars) {
+        const double tk = (double)p.T * (double)p.K;
+        double sw = 0.0, ss = 0.0, mi = 0.0, mc = 0.0;
+        for (int e = 0; e < N; ++e) {
+            const double f = tb.cnt[e] / tk;
+            sw += f * f_pm[e];
+            ss += f * f;
+            mi += f_im[e];
+            mc += tb.cnt[e];
+        }
+        mi /= N;
+        mc /= N;
+        double vi = 0.0, vc = 0.0;
+        for (int e = 0; e < N; ++e) {
+            vi += (f_im[e] - mi) * (f_im[e] - mi);
+            vc += (tb.cnt[e] - mc) * (tb.cnt[e] - mc);
+        }
+        vi /= N;
+        vc /= N;
+        p.aux_scalars[0] = (float)(N * sw);
+        p.aux_scalars[1] = (float)(N * ss);
+        p.aux_scalars[2] = mi == 0.0 ? 0.f : (float)(vi / (mi * mi));
+        p.aux_scalars[3] = mc == 0.0 ? 0.f : (float)(vc / (mc * mc));
+    }
+}
+
 // R3: the dispatch tables from the top-k, in every CTA.  scratch holds the
 // top-k indices and each slot's position inside its expert while they are built.
-__device__ __forceinline__ void route_r3(const Params &p, const Tables &tb, uint8_t *scratch, bool idx_ready) {
+// With publish false, CTA 0 leaves the workspace tables and the statistics to
+// the caller (r3_publish).
+__device__ __forceinline__ void route_r3(const Params &p, const Tables &tb, uint8_t *scratch, bool idx_ready,
+                                         bool publish = true) {
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int N = p.N, TK = p.T * p.K;
     int *s_idx = reinterpret_cast<int *>(scratch);   // filled by route_r2_all when idx_ready
@@ -340,81 +426,8 @@ __device__ __forceinline__ void route_r3(const Params &p, const Tables &tb, uint
         fence_proxy_async_global();
         grid_arrive(p.bar);
     }
-    if (blockIdx.x == 0) {
-        // the workspace tables (moe_get_workspace_layout) and the statistics
-        for (int e = tid; e < N; e += kThreads) {
-            p.counts[e] = tb.kept[e];
-            p.offsets[e] = tb.koff[e];
-            p.row_offsets[e] = tb.rowoff[e];
-        }
-        if (tid == 0) {
-            p.offsets[N] = tb.koff[N - 1] + tb.kept[N - 1];
-            p.row_offsets[N] = tb.rowoff[N - 1] + (tb.kept[N - 1] + kRowAlign - 1) / kRowAlign * kRowAlign;
-            *p.n_live = *tb.nlive;
-        }
-        for (int i = tid; i < *tb.nlive; i += kThreads) p.live[i] = tb.live[i];
-        for (int i = tid; i < TK; i += kThreads) {
-            const int r = tb.row[i];
-            p.slot_row[i] = r;
-            if (r >= 0) p.perm_slot[r] = i;
-        }
-        for (int e = warp; e < N; e += kThreads / 32) {
-            const int start = tb.rowoff[e] + tb.kept[e];
-            const int end = tb.rowoff[e] + (tb.kept[e] + kRowAlign - 1) / kRowAlign * kRowAlign;
-            for (int r = start + lane; r < end; r += 32) p.perm_slot[r] = -1;
-        }
-        // statistics of the router's choice: fixed orders (tokens ascending, slots
-        // ascending), from the gate weights and the full softmax loaded at once
-        float *f_im = reinterpret_cast<float *>(s_pos);   // [32] scratch once the ranks are consumed
-        float *f_pm = f_im + 32;
-        float *s_w = reinterpret_cast<float *>(s_pos + kMaxSlots);   // [T*K]
-        float *s_tp = s_w + kMaxSlots;                               // [T][32]
-        for (int i = tid; i < TK; i += kThreads) s_w[i] = __ldcg(p.topk_w + i);
-        for (int i = tid; i < p.T * 32; i += kThreads) s_tp[i] = __ldcg(p.tok_p + i);
-        __syncthreads();
-        if (tid < 32) {
-            const int e = tid;
-            float im = 0.f, pm = 0.f;
-            if (e < N) {
-                for (int i = 0; i < TK; ++i)
-                    if (s_idx[i] == e) im += s_w[i];
-                for (int t = 0; t < p.T; ++t) pm += s_tp[t * 32 + e];
-                pm /= (float)p.T;
-            }
-            f_im[e] = im;
-            f_pm[e] = pm;
-            if (e < N) {
-                if (p.aux_counts) p.aux_counts[e] = tb.cnt[e];
-                if (p.aux_importance) p.aux_importance[e] = im;
-                if (p.aux_p_mean) p.aux_p_mean[e] = pm;
-            }
-        }
-        __syncthreads();
-        if (tid == 0 && p.aux_scalars) {
-            const double tk = (double)p.T * (double)p.K;
-            double sw = 0.0, ss = 0.0, mi = 0.0, mc = 0.0;
-            for (int e = 0; e < N; ++e) {
-                const double f = tb.cnt[e] / tk;
-                sw += f * f_pm[e];
-                ss += f * f;
-                mi += f_im[e];
-                mc += tb.cnt[e];
-            }
-            mi /= N;
-            mc /= N;
-            double vi = 0.0, vc = 0.0;
-            for (int e = 0; e < N; ++e) {
-                vi += (f_im[e] - mi) * (f_im[e] - mi);
-                vc += (tb.cnt[e] - mc) * (tb.cnt[e] - mc);
-            }
-            vi /= N;
-            vc /= N;
-            p.aux_scalars[0] = (float)(N * sw);
-            p.aux_scalars[1] = (float)(N * ss);
-            p.aux_scalars[2] = mi == 0.0 ? 0.f : (float)(vi / (mi * mi));
-            p.aux_scalars[3] = mc == 0.0 ? 0.f : (float)(vc / (mc * mc));
-        }
-    }
+    if (publish && blockIdx.x == 0)
+        r3_publish(p, tb, s_idx, reinterpret_cast<float *>(s_pos), tid, kThreads, [] { __syncthreads(); });
 }
 
 // ------------------------------------------------------------------ the expert phases
@@ -509,8 +522,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (ok && (int)blockIdx.x < p.T) route_r2(p, smem);
         if (ok) ok = grid_sync_all(p, 2, s_flag);
     }
+    // CTA 0's workspace tables and statistics: done by its epilogue warps while
+    // they wait for their first accumulator (so that CTA 0's weight stream
+    // starts with everyone else's) when the selection and the scratch fit the
+    // epilogue staging area, which is idle until then
+    const int TK = p.T * p.K;
+    const bool defer = (size_t)(2 * TK + 64 + 32 * p.T) * 4 <= S::kEpiBytes;
     if (ok) {
-        route_r3(p, tb, smem, r2_all);   // arrives at barrier 3 once its x_perm rows are written
+        route_r3(p, tb, smem, r2_all, !defer);   // arrives at barrier 3 once its x_perm rows are written
+        if (defer && blockIdx.x == 0)
+            for (int i = threadIdx.x; i < TK; i += kThreads) reinterpret_cast<int *>(sE)[i] = reinterpret_cast<const int *>(smem)[i];
     }
     __syncthreads();
 
@@ -659,6 +680,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int q = warp & 3;
         const int L = q * 32 + lane;        // TMEM lane = weight row within the tile
         const int et = threadIdx.x - 64;    // 0..127
+        if (defer && blockIdx.x == 0) {
+            auto epi_sync = [] { asm volatile("bar.sync 1, 128;" ::: "memory"); };
+            r3_publish(p, tb, reinterpret_cast<const int *>(sE), reinterpret_cast<float *>(sE) + TK, et, 128, epi_sync);
+            epi_sync();   // sE is the staging area again from here on
+        }
         dec::EpiBarrier eb{epib, 0u, p.timeout_ns};
         int local = 0;
         bool eok = true;
