@@ -347,12 +347,34 @@ __device__ __forceinline__ void r3_publish(const Params &p, const Tables &tb, co
     }
 }
 
+// The kept slots' token rows into x_perm, one slot per CTA at a time, by threads
+// tid < nth that sync() brings together; then the CTA releases x_perm to the grid
+// (barrier 3 is waited on only by the producers, before their first token-row
+// load).
+template <class Sync>
+__device__ __forceinline__ void r3_copy_rows(const Params &p, const Tables &tb, int tid, int nth, Sync sync) {
+    const int nv = p.D / 8, TK = p.T * p.K;
+    for (int i = blockIdx.x; i < TK; i += gridDim.x) {
+        const int r = tb.row[i];
+        if (r < 0) continue;
+        const uint4 *src = reinterpret_cast<const uint4 *>(p.x + (size_t)(i / p.K) * p.D);
+        uint4 *dst = reinterpret_cast<uint4 *>(p.x_perm + (size_t)r * p.D);
+        for (int v = tid; v < nv; v += nth) dst[v] = __ldg(src + v);
+    }
+    sync();
+    if (tid == 0) {
+        fence_proxy_async_global();
+        grid_arrive(p.bar);
+    }
+}
+
 // R3: the dispatch tables from the top-k, in every CTA.  scratch holds the
 // top-k indices and each slot's position inside its expert while they are built.
 // With publish false, CTA 0 leaves the workspace tables and the statistics to
-// the caller (r3_publish).
+// the caller (r3_publish); with copy_rows false, the x_perm copies and the
+// arrival at barrier 3 are left to the caller too (r3_copy_rows).
 __device__ __forceinline__ void route_r3(const Params &p, const Tables &tb, uint8_t *scratch, bool idx_ready,
-                                         bool publish = true) {
+                                         bool publish = true, bool copy_rows = true) {
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int N = p.N, TK = p.T * p.K;
     int *s_idx = reinterpret_cast<int *>(scratch);   // filled by route_r2_all when idx_ready
@@ -409,23 +431,7 @@ __device__ __forceinline__ void route_r3(const Params &p, const Tables &tb, uint
         if (keep) tb.ent[tb.koff[e] + pos] = (int16_t)i;
     }
     __syncthreads();
-    // the kept slots' token rows into x_perm, one slot per CTA at a time
-    const int nv = p.D / 8;
-    for (int i = blockIdx.x; i < TK; i += gridDim.x) {
-        const int r = tb.row[i];
-        if (r < 0) continue;
-        const uint4 *src = reinterpret_cast<const uint4 *>(p.x + (size_t)(i / p.K) * p.D);
-        uint4 *dst = reinterpret_cast<uint4 *>(p.x_perm + (size_t)r * p.D);
-        for (int v = tid; v < nv; v += kThreads) dst[v] = __ldg(src + v);
-    }
-    // x_perm written: release it to the grid (barrier 3 is waited on only by the
-    // producers, before their first token-row load); the workspace tables and the
-    // statistics follow in CTA 0, off the critical path
-    __syncthreads();
-    if (tid == 0) {
-        fence_proxy_async_global();
-        grid_arrive(p.bar);
-    }
+    if (copy_rows) r3_copy_rows(p, tb, tid, kThreads, [] { __syncthreads(); });
     if (publish && blockIdx.x == 0)
         r3_publish(p, tb, s_idx, reinterpret_cast<float *>(s_pos), tid, kThreads, [] { __syncthreads(); });
 }
@@ -528,8 +534,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     // epilogue staging area, which is idle until then
     const int TK = p.T * p.K;
     const bool defer = (size_t)(2 * TK + 64 + 32 * p.T) * 4 <= S::kEpiBytes;
+    // with at most 8 rows to copy, the x_perm copies (CTAs 0 .. TK - 1) and the
+    // arrival at barrier 3 go to the epilogue warps too, so that no producer
+    // starts late (decode1 0.4 to 1.4 us faster on two boxes); with more rows
+    // the copies take longer in 128 threads and barrier 3 comes later (decode8
+    // 1.5 us slower), so they stay here
+    const bool defer_copy = TK <= 8;
     if (ok) {
-        route_r3(p, tb, smem, r2_all, !defer);   // arrives at barrier 3 once its x_perm rows are written
+        route_r3(p, tb, smem, r2_all, !defer, !defer_copy);
         if (defer && blockIdx.x == 0)
             for (int i = threadIdx.x; i < TK; i += kThreads) reinterpret_cast<int *>(sE)[i] = reinterpret_cast<const int *>(smem)[i];
     }
@@ -680,8 +692,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int q = warp & 3;
         const int L = q * 32 + lane;        // TMEM lane = weight row within the tile
         const int et = threadIdx.x - 64;    // 0..127
+        // the x_perm copies and the arrival at barrier 3, then (CTA 0) the tables and
+        // the statistics, while the producer already streams weight tiles
+        auto epi_sync = [] { asm volatile("bar.sync 1, 128;" ::: "memory"); };
+        if (defer_copy) r3_copy_rows(p, tb, et, 128, epi_sync);
         if (defer && blockIdx.x == 0) {
-            auto epi_sync = [] { asm volatile("bar.sync 1, 128;" ::: "memory"); };
             r3_publish(p, tb, reinterpret_cast<const int *>(sE), reinterpret_cast<float *>(sE) + TK, et, 128, epi_sync);
             epi_sync();   // sE is the staging area again from here on
         }
