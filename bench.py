@@ -72,11 +72,11 @@ GEMM_KERNEL_SRC = os.path.join(ROOT, "sparse_mixture_experts_10_b200", "csrc", "
 # scaled by 8 (weights and token rows both grow eightfold).  The tail kernel beside the pair kernel
 # is not included.  Keyed by workload and stage; valid only while the source hash is unchanged.
 NCU_TRAFFIC = {
-    "gpt2/up": {"bytes": 54388992 + 54088704, "src_sha256": "5ff2a8acd93be22ae89939cf388d8497488fa048a891985ad4d97012dbd96b09"},
-    "gpt2/down": {"bytes": 167763456 + 12327424, "src_sha256": "5ff2a8acd93be22ae89939cf388d8497488fa048a891985ad4d97012dbd96b09"},
-    "deepseek/up": {"bytes": 8 * (2366248000 + 67960832), "src_sha256": "5ff2a8acd93be22ae89939cf388d8497488fa048a891985ad4d97012dbd96b09",
+    "gpt2/up": {"bytes": 54389760 + 53961216, "src_sha256": "410a9cd9ccbbf5b3802a66ad2371756e66bd410e05e0ccfb4cedcff2781a330b"},
+    "gpt2/down": {"bytes": 166587136 + 10543360, "src_sha256": "410a9cd9ccbbf5b3802a66ad2371756e66bd410e05e0ccfb4cedcff2781a330b"},
+    "deepseek/up": {"bytes": 8 * (2115678000 + 66724608), "src_sha256": "410a9cd9ccbbf5b3802a66ad2371756e66bd410e05e0ccfb4cedcff2781a330b",
                     "note": "scaled from the T=2048, N=32 capture"},
-    "deepseek/down": {"bytes": 8 * (1011410000 + 437825536), "src_sha256": "5ff2a8acd93be22ae89939cf388d8497488fa048a891985ad4d97012dbd96b09",
+    "deepseek/down": {"bytes": 8 * (1008105000 + 440681728), "src_sha256": "410a9cd9ccbbf5b3802a66ad2371756e66bd410e05e0ccfb4cedcff2781a330b",
                       "note": "scaled from the T=2048, N=32 capture"},
 }
 
