@@ -201,6 +201,8 @@ def work_model(wl, T, counts=None, kept=None):
         route_bytes=T * D * b + D * N * b + T * N * 4 + T * K * 8 + (y_clear if by_router else 0),
         # x read once, its K copies written, the slot maps (+ the clear of y otherwise)
         permute_bytes=T * D * b + rows * D * b + T * K * 8 + (0 if by_router else y_clear),
+        # the part of them that is written: x_perm (+ the clear of y when the permute does it)
+        permute_write_bytes=rows * D * b + (0 if by_router else y_clear),
         combine_bytes=0 if fused_combine(wl, T) else rows * D * 4 + T * D * 4,
         up_weight_bytes=live * up_rows * D * b, down_weight_bytes=live * D * H * b,
         live_experts=live,
@@ -241,6 +243,26 @@ def stream_floor_ms(nbytes, flush, dev, reps=10):
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record()
         torch.sum(t, dim=0, dtype=torch.float32, out=out)
+        b.record()
+        torch.cuda.synchronize()
+        if i >= 3:
+            ms.append(a.elapsed_time(b))
+    del t
+    return float(np.median(ms))
+
+
+def write_floor_ms(nbytes, flush, dev, reps=8):
+    """Median time of one plain write of nbytes to HBM (torch zero_ of a bf16 tensor that size;
+    L2 flushed before each run, CUDA events around the launch).  On these B200s a write stream
+    reaches well under the copy rate (which counts reads and writes), so it is the reference for a
+    stage whose bytes are mostly written (the permute)."""
+    t = torch.empty(max(nbytes // 2, 1), dtype=torch.bfloat16, device=dev)
+    ms = []
+    for i in range(reps + 3):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        t.zero_()
         b.record()
         torch.cuda.synchronize()
         if i >= 3:
@@ -848,6 +870,14 @@ def main():
             d["GB/s"] = wm["route_bytes"] / (mean_stage[s] * 1e-3) / 1e9
         elif nm == "permute":
             d["GB/s"] = wm["permute_bytes"] / (mean_stage[s] * 1e-3) / 1e9
+            wb = int(wm["permute_write_bytes"])
+            if not decode and wb >= (64 << 20) and mean_stage[s] > 0.02:
+                # a plain write of the bytes the permute writes, timed the same way
+                wf = write_floor_ms(wb, flush, dev)
+                d["write_floor"] = {"ms": wf, "GB/s": wb / (wf * 1e-3) / 1e9, "bytes": wb,
+                                    "how": "torch zero_ of a bf16 tensor of the permute's written bytes, L2 flushed, "
+                                           "median of 8"}
+                d["frac_of_write_floor"] = wf / mean_stage[s]
         elif nm == "combine":
             d["GB/s"] = wm["combine_bytes"] / (mean_stage[s] * 1e-3) / 1e9
         elif nm in ("up", "down"):

@@ -156,3 +156,14 @@ def test_capacity_counts_only_the_kept_pairs():
     assert m["live_experts"] == 40
     # without a capacity every routed pair is work
     assert bench.work_model(wl, T)["up_flops"] == 4 * T * K * D * H
+
+
+def test_permute_write_bytes_are_the_copies_and_any_clear_of_y():
+    wl = WORKLOADS["deepseek"]   # K = 8: the permute writes the copies, nobody clears y
+    T, D, K = wl.T, wl.D, wl.K
+    m = bench.work_model(wl, T)
+    assert m["permute_write_bytes"] == T * K * D * 2
+    assert m["permute_bytes"] - m["permute_write_bytes"] == T * D * 2 + T * K * 8
+    wl = WORKLOADS["mixtral"]    # K = 2, N <= 32: the SIMT router clears y, not the permute
+    m = bench.work_model(wl, wl.T)
+    assert m["permute_write_bytes"] == wl.T * wl.K * wl.D * 2
